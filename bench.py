@@ -1,0 +1,421 @@
+#!/usr/bin/env python
+"""Benchmark: CSA + HCA decode over an MXFP4 KV cache at 512K-1M context on B200.
+
+One step = one decode token for every request of the batch through one CSA layer
+and one HCA layer (the CSA/HCA alternation), i.e. every row of the hot path:
+  a1+a2  csa_compress_quantize: the 4 newest tokens -> one CSA block (MXFP4 + e4m3 key),
+         the 128 newest tokens -> one HCA block
+  a3+a4  csa_index_topk over every visible CSA block (k = 1024)
+  a5+a6+a8 csa_decode_attend: selected blocks + 128-token bf16 window, one joint softmax
+  a7     hca_decode_attend: every HCA block + the window
+Workload (default, per GPU): 32 requests, context lengths uniform in [512K, 1M]
+tokens (multiples of 128), D = 512 shared latent, 64 query heads, indexer 4 x 128
+with e4m3 keys, k = 1024, W = 128. Synthetic data (seeded torch RNG on the GPU).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0). With N > 1 every rank runs its own independent
+batch (weak scaling, no data-path collective); time = max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+B, D, H, M_CSA, M_HCA, W = 32, 512, 64, 4, 128, 128
+H_I, D_I, TOPK = 4, 128, 1024
+CTX_MIN, CTX_MAX = 524288, 1048576
+CAP_CSA, CAP_HCA = CTX_MAX // M_CSA, CTX_MAX // M_HCA
+OUR_KERNELS_PER_STEP = 12  # compress 2x(pool, commit); index: schedule, scan, select x2; attend 2x(schedule, main)
+SEED = 0x5EED0C5A
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+# ----------------------------------------------------------------------------- workload
+def context_lengths(rank: int) -> np.ndarray:
+    from fp4_kv_cache_csa_b200 import datagen
+
+    g = datagen.generator(1000 + rank)
+    return (g.integers(CTX_MIN // 128, CTX_MAX // 128, size=B, endpoint=True) * 128).astype(np.int64)
+
+
+class Workload:
+    """Device-resident caches and per-step inputs for one rank."""
+
+    def __init__(self, rank: int, device):
+        import torch
+
+        import fp4_kv_cache_csa_b200 as csa
+
+        self.T = context_lengths(rank)
+        n_csa = self.T // M_CSA           # blocks after this step's append
+        n_hca = self.T // M_HCA
+        self.n_csa, self.n_hca = n_csa, n_hca
+        gen = torch.Generator(device=device)
+        gen.manual_seed(SEED + rank)
+        self.csa = csa.Cache.allocate(B, CAP_CSA, D, M_CSA, D_I, csa.CSA_IDX_E4M3, device)
+        self.hca = csa.Cache.allocate(B, CAP_HCA, D, M_HCA, 0, csa.CSA_IDX_BF16, device)
+        for cache, n in ((self.csa, n_csa), (self.hca, n_hca)):
+            for b in range(B):
+                nb = int(n[b])
+                cache.fp4[b, :nb].random_(0, 256, generator=gen)
+                cache.scale[b, :nb].random_(123, 127, generator=gen)
+                if cache.idx_key is not None:
+                    k = torch.randn(nb, D_I, device=device, generator=gen) * 0.5
+                    cache.idx_key[b, :nb] = k.to(torch.float8_e4m3fn).view(torch.uint8)
+        self.base_csa = torch.tensor(n_csa - 1, dtype=torch.int32, device=device)
+        self.base_hca = torch.tensor(n_hca - 1, dtype=torch.int32, device=device)
+        bf = torch.bfloat16
+        self.kv4 = torch.randn(B * M_CSA, D, device=device, generator=gen).to(bf)
+        self.idx4 = torch.randn(B * M_CSA, D_I, device=device, generator=gen).to(bf)
+        self.kv128 = torch.randn(B * M_HCA, D, device=device, generator=gen).to(bf)
+        self.gate_w = (torch.randn(D, device=device, generator=gen) * 0.02).float()
+        self.offs4 = torch.arange(0, B * M_CSA + 1, M_CSA, dtype=torch.int32, device=device)
+        self.offs128 = torch.arange(0, B * M_HCA + 1, M_HCA, dtype=torch.int32, device=device)
+        self.q_csa = torch.randn(B, H, D, device=device, generator=gen).to(bf)
+        self.q_hca = torch.randn(B, H, D, device=device, generator=gen).to(bf)
+        self.q_idx = torch.randn(B, H_I, D_I, device=device, generator=gen).to(bf)
+        self.w = (torch.randn(B, H_I, device=device, generator=gen) / math.sqrt(H_I)).float()
+        self.q_offsets = torch.arange(B + 1, dtype=torch.int32, device=device)
+        self.q_pos = torch.tensor(self.T - 1, dtype=torch.int32, device=device)
+        self.win = torch.randn(B * W, D, device=device, generator=gen).to(bf)
+        self.win_start = torch.arange(0, B * W, W, dtype=torch.int64, device=device)
+        self.win_len = torch.full((B,), W, dtype=torch.int32, device=device)
+        self.sel = torch.empty(B, TOPK, dtype=torch.int32, device=device)
+        self.out_csa = torch.empty(B, H, D, dtype=torch.float32, device=device)
+        self.out_hca = torch.empty(B, H, D, dtype=torch.float32, device=device)
+        self.lse = torch.empty(B, H, dtype=torch.float32, device=device)
+        self.ws_idx = torch.empty(csa.csa_index_topk_workspace(self.csa, B, TOPK), dtype=torch.uint8, device=device)
+        nws = max(csa.csa_attend_workspace(self.csa, B, H), csa.csa_attend_workspace(self.hca, B, H))
+        self.ws_att = torch.empty(nws, dtype=torch.uint8, device=device)
+        self.scale = D ** -0.5
+
+    # the three stages of one step; every launch is one of libcsa's kernels or a memset
+    def stage_compress(self):
+        import fp4_kv_cache_csa_b200 as csa
+
+        self.csa.n_blocks.copy_(self.base_csa)
+        self.hca.n_blocks.copy_(self.base_hca)
+        csa.csa_compress_quantize(self.csa, self.kv4, self.idx4, self.gate_w, self.offs4)
+        csa.csa_compress_quantize(self.hca, self.kv128, None, self.gate_w, self.offs128)
+
+    def stage_index(self):
+        import fp4_kv_cache_csa_b200 as csa
+
+        csa.csa_index_topk(self.csa, self.q_idx, self.w, self.q_offsets, self.q_pos, TOPK, sel_idx=self.sel,
+                           workspace=self.ws_idx)
+
+    def stage_attend(self):
+        import fp4_kv_cache_csa_b200 as csa
+
+        csa.csa_decode_attend(self.csa, self.q_csa, self.q_offsets, self.sel, self.win, self.win_start, self.win_len,
+                              max_win=W, softmax_scale=self.scale, out=self.out_csa, lse=self.lse,
+                              workspace=self.ws_att)
+        csa.hca_decode_attend(self.hca, self.q_hca, self.q_offsets, self.q_pos, self.win, self.win_start,
+                              self.win_len, max_win=W, softmax_scale=self.scale, out=self.out_hca,
+                              workspace=self.ws_att)
+
+    # algorithmic HBM bytes: what the method must move at least once per step
+    def bytes_index(self) -> float:
+        keys = float(np.sum(self.n_csa)) * D_I
+        return keys + B * (H_I * D_I * 2 + H_I * 4 + TOPK * 4)
+
+    def bytes_step(self) -> float:
+        entry = D // 2 + D // 32
+        sel = float(np.sum(np.minimum(self.n_csa, TOPK))) * entry
+        hca = float(np.sum(self.n_hca)) * entry
+        win = 2.0 * B * W * D * 2
+        q = 2.0 * B * H * D * 2
+        out = 2.0 * B * H * D * 4
+        comp = B * (M_CSA * (D + D_I) * 2 + entry + D_I) + B * (M_HCA * D * 2 + entry)
+        return self.bytes_index() + sel + hca + win + q + out + comp
+
+    def step_inputs(self):
+        """Per-step inputs a caller streams in (new tokens, queries) and the outputs it reads back."""
+        ins = [self.kv4, self.idx4, self.kv128, self.q_csa, self.q_hca, self.q_idx, self.w]
+        outs = [self.out_csa, self.out_hca]
+        return ins, outs
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    def __init__(self, index: int):
+        self.index, self.samples, self.proc = index, [], None
+
+    def start(self):
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.samples.append(parts)
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, max_mhz_default=1965.0):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        mx = [float(s[2]) for s in self.samples if s[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for s in self.samples for k in range(4) if s[5 + k].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else max_mhz_default,
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- oracle baseline
+def cpu_baseline(n_requests: int = 2):
+    """The oracle (plain C, double precision, OpenMP over independent units) doing the step's work for a
+    bounded sample of requests: compress of the new CSA and HCA blocks, indexer + top-k over the full
+    visible key cache, CSA attention, HCA attention. Returns (tokens/s, cores, sample description)."""
+    import oracle
+    from fp4_kv_cache_csa_b200 import datagen
+
+    T = context_lengths(0)[:n_requests]
+    total = 0.0
+    for r in range(n_requests):
+        n_csa, n_hca = int(T[r] // M_CSA), int(T[r] // M_HCA)
+        keys = datagen.to_e4m3_bytes(datagen.normal_f32((1, n_csa, D_I), 2000 + r, 1, std=0.5))
+        fp4, sc = datagen.random_cache_bytes(n_csa, D, 2000 + r, 2)
+        hfp4, hsc = datagen.random_cache_bytes(n_hca, D, 2000 + r, 3)
+        kv4 = datagen.normal_bf16((M_CSA, D), 2000 + r, 4)
+        idx4 = datagen.normal_bf16((M_CSA, D_I), 2000 + r, 5)
+        kv128 = datagen.normal_bf16((M_HCA, D), 2000 + r, 6)
+        wg = datagen.normal_f32((D,), 2000 + r, 7, std=0.02)
+        q = datagen.normal_bf16((1, H, D), 2000 + r, 8)
+        q_idx = datagen.normal_bf16((1, H_I, D_I), 2000 + r, 9)
+        w = datagen.normal_f32((1, H_I), 2000 + r, 10, std=0.5)
+        win = datagen.normal_bf16((W, D), 2000 + r, 11)
+        fp4 = fp4.reshape(1, n_csa, D // 2)
+        sc = sc.reshape(1, n_csa, D // 32)
+        hfp4 = hfp4.reshape(1, n_hca, D // 2)
+        hsc = hsc.reshape(1, n_hca, D // 32)
+        qo, qp = np.array([0, 1], np.int32), np.array([T[r] - 1], np.int32)
+        ws, wl = np.array([0], np.int64), np.array([W], np.int32)
+        t0 = time.perf_counter()
+        oracle.compress(kv4, idx4, wg, np.array([0, M_CSA], np.int32), np.array([n_csa - 1], np.int32), m=M_CSA,
+                        cap=n_csa, idx_dtype=1, fp4=fp4, scale=sc, idx_key=keys)
+        oracle.compress(kv128, None, wg, np.array([0, M_HCA], np.int32), np.array([n_hca - 1], np.int32), m=M_HCA,
+                        cap=n_hca, fp4=hfp4, scale=hsc)
+        sel, _, _ = oracle.index_topk(keys, np.array([n_csa], np.int32), qo, qp, q_idx, w, m=M_CSA, k=TOPK,
+                                      idx_dtype=1)
+        oracle.csa_attend(fp4, sc, qo, q, sel, win, ws, wl, D ** -0.5)
+        oracle.hca_attend(hfp4, hsc, np.array([n_hca], np.int32), qo, qp, q, win, ws, wl, D ** -0.5, m=M_HCA)
+        total += time.perf_counter() - t0
+    return n_requests / total, oracle.num_threads(), \
+        f"{n_requests} of the {B} requests of one step (contexts {', '.join(str(int(t)) for t in T)} tokens)"
+
+
+# ----------------------------------------------------------------------------- main
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d.get("hbm_gbs", 6650.0)), "measured"
+    return 6650.0, "fallback"
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    n_req = 2
+    # one "step" of the oracle = the step's work for n_req requests
+    times = []
+    for _ in range(args.warmup + args.steps):
+        v, cores, sample = cpu_baseline(n_req)
+        times.append(n_req / v)
+    t = statistics.mean(times[args.warmup:])
+    value = n_req / t
+    line = {"impl": "reference", "metric": "CSA decode tokens/s and achieved HBM TB/s at 1M ctx (MXFP4 KV), vs roofline",
+            "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded)",
+            "config": {"workload": "csa_hca_decode_b32_ctx512k-1m", "global_batch": B, "seq_len": CTX_MAX,
+                       "parallelism": "replicas", "l2": "inputs larger than L2 (full key cache streamed)"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    import fp4_kv_cache_csa_b200 as csa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
+    csa.load_library()
+
+    wl = Workload(rank, device)
+    torch.cuda.synchronize()
+    stream = torch.cuda.Stream(device)
+    graphs = []
+    with torch.cuda.stream(stream):
+        for fn in (wl.stage_compress, wl.stage_index, wl.stage_attend):  # eager pass before capture
+            fn()
+        stream.synchronize()
+        for fn in (wl.stage_compress, wl.stage_index, wl.stage_attend):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                fn()
+            graphs.append(g)
+    torch.cuda.synchronize()
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=device)  # > 126 MB L2
+
+    def replay_step(evs=None):
+        for s, g in enumerate(graphs):
+            if evs is not None:
+                evs[s].record(stream)
+            g.replay()
+        if evs is not None:
+            evs[3].record(stream)
+
+    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local)
+    clocks.start()
+    with torch.cuda.stream(stream):
+        for _ in range(max(args.warmup, 3)):
+            flush.zero_()
+            replay_step()
+    stream.synchronize()
+    status = csa.csa_read_device_status(wl.csa, stream) | csa.csa_read_device_status(wl.hca, stream)
+
+    # ---- device-resident timed region
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    with torch.cuda.stream(stream):
+        for k in range(args.steps):
+            flush.zero_()  # outside the events: every step starts with a cold L2
+            replay_step(ev[k])
+    stream.synchronize()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks.stop()
+    st_ms = np.array([[ev[k][s].elapsed_time(ev[k][s + 1]) for s in range(3)] for k in range(args.steps)])
+    step_ms = st_ms.sum(axis=1)
+    ms = float(step_ms.mean())
+
+    # ---- end-to-end: pinned host inputs in, results out, every step
+    ins, outs = wl.step_inputs()
+    h_ins = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t.cpu()) for t in ins]
+    h_outs = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+    h2d = sum(t.numel() * t.element_size() for t in h_ins)
+    d2h = sum(t.numel() * t.element_size() for t in h_outs)
+    e2e_n = max(3, min(args.steps, 50))
+    e0 = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_n)]
+    e1 = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_n)]
+    with torch.cuda.stream(stream):
+        for k in range(e2e_n):
+            flush.zero_()
+            e0[k].record(stream)
+            for d_, h_ in zip(ins, h_ins):
+                d_.copy_(h_, non_blocking=True)
+            replay_step()
+            for h_, d_ in zip(h_outs, outs):
+                h_.copy_(d_, non_blocking=True)
+            e1[k].record(stream)
+    stream.synchronize()
+    e2e_ms = float(np.mean([e0[k].elapsed_time(e1[k]) for k in range(e2e_n)]))
+
+    if world > 1:
+        t = torch.tensor([ms, e2e_ms, float(st_ms[:, 1].mean())], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, e2e_ms, idx_ms = (float(x) for x in t.tolist())
+    else:
+        idx_ms = float(st_ms[:, 1].mean())
+    tokens = B * world
+    value = tokens / (ms * 1e-3)
+    peak, peak_kind = measured_peaks()
+    achieved = wl.bytes_index() / (idx_ms * 1e-3) / 1e9  # GB/s of the indexer stage
+    hbm_tbs = wl.bytes_step() / (ms * 1e-3) / 1e12
+
+    line = {
+        "metric": "CSA decode tokens/s and achieved HBM TB/s at 1M ctx (MXFP4 KV), vs roofline",
+        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp32-acc/fp16-mma",
+        "data": "synthetic (seeded torch RNG on device)",
+        "config": {"workload": "csa_hca_decode_b32_ctx512k-1m", "global_batch": tokens, "seq_len": CTX_MAX,
+                   "parallelism": f"replicas x{world}", "per_gpu_batch": B, "topk": TOPK, "heads": H, "dim": D,
+                   "l2": "flushed between steps (512 MB write) and inputs larger than L2"},
+        "hbm_tbs": hbm_tbs,
+        "stage_ms": {"compress": float(st_ms[:, 0].mean()), "index_topk": float(st_ms[:, 1].mean()),
+                     "attend_csa_hca": float(st_ms[:, 2].mean())},
+        "roofline": {"bound": "hbm", "kernel": "csa_index_topk (scan + select)", "achieved": achieved, "peak": peak,
+                     "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind, "traffic": None},
+        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": OUR_KERNELS_PER_STEP * args.steps,
+        "clocks": clocks.summary(),
+        "device_status": status,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, cores, sample = cpu_baseline()
+        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample}
+    if world > 1:
+        dist.barrier()
+    del graphs
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

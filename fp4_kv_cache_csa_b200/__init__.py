@@ -1,0 +1,250 @@
+"""Python binding of libcsa: CSA / HCA / window attention over an MXFP4 KV cache on B200.
+
+Argument marshalling only. Every step of the method runs in the CUDA kernels of
+libcsa.so (built in-tree by ``python -m fp4_kv_cache_csa_b200.build``); PyTorch
+is used for device memory and streams. Importing this module does not load the
+library; the first call does, and raises ``CsaError`` if it is missing -- there
+is no CPU fallback.
+
+The function names mirror the C ABI in include/csa.h:
+    csa_compress_quantize, csa_index_topk, csa_decode_attend, hca_decode_attend,
+    csa_read_device_status (+ the workspace-size queries).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcsa.so")
+
+CSA_IDX_BF16 = 0
+CSA_IDX_E4M3 = 1
+
+CSA_DEV_TOKEN_COUNT = 0x1
+CSA_DEV_CAPACITY = 0x2
+CSA_DEV_BAD_INDEX = 0x4
+CSA_DEV_BAD_WINDOW = 0x8
+CSA_DEV_TIMEOUT = 0x10
+
+EXPORTED = (
+    "csa_status_string", "csa_version", "csa_compress_quantize", "csa_index_topk_workspace", "csa_index_topk",
+    "csa_attend_workspace", "csa_decode_attend", "hca_decode_attend", "csa_read_device_status",
+)
+
+
+class CsaError(RuntimeError):
+    pass
+
+
+class _CCache(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32), ("dim", ctypes.c_int32), ("block", ctypes.c_int32), ("capacity", ctypes.c_int32),
+        ("fp4", ctypes.c_void_p), ("scale", ctypes.c_void_p), ("idx_key", ctypes.c_void_p),
+        ("idx_dim", ctypes.c_int32), ("idx_dtype", ctypes.c_int32),
+        ("n_blocks", ctypes.c_void_p), ("status", ctypes.c_void_p),
+    ]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libcsa.so and declare the C signatures. Raises CsaError if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise CsaError(f"libcsa.so not found at {path}: build it with `python -m fp4_kv_cache_csa_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, I, S = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+    CP = ctypes.POINTER(_CCache)
+    lib.csa_status_string.argtypes = [I]
+    lib.csa_status_string.restype = ctypes.c_char_p
+    lib.csa_version.argtypes = []
+    lib.csa_version.restype = I
+    lib.csa_compress_quantize.argtypes = [CP, P, P, P, P, I, P]
+    lib.csa_compress_quantize.restype = I
+    lib.csa_index_topk_workspace.argtypes = [CP, I, I]
+    lib.csa_index_topk_workspace.restype = S
+    lib.csa_index_topk.argtypes = [CP, P, P, I, I, P, P, I, P, P, S, P]
+    lib.csa_index_topk.restype = I
+    lib.csa_attend_workspace.argtypes = [CP, I, I]
+    lib.csa_attend_workspace.restype = S
+    lib.csa_decode_attend.argtypes = [CP, P, I, I, P, P, I, P, P, P, I, ctypes.c_float, P, P, P, S, P]
+    lib.csa_decode_attend.restype = I
+    lib.hca_decode_attend.argtypes = [CP, P, I, I, P, P, P, P, P, I, ctypes.c_float, P, P, P, S, P]
+    lib.hca_decode_attend.restype = I
+    lib.csa_read_device_status.argtypes = [CP, P, ctypes.POINTER(I)]
+    lib.csa_read_device_status.restype = I
+    _lib = lib
+    return lib
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        msg = load_library().csa_status_string(status).decode()
+        raise CsaError(f"{what}: {msg} (status {status})")
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream):
+    import torch
+
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+@dataclass
+class Cache:
+    """One compressed cache (one layer): device tensors owned by the caller (see include/csa.h).
+
+    fp4 [B, cap, D/2] uint8, scale [B, cap, D/32] uint8, idx_key [B, cap, dI] bf16 / uint8 (e4m3) or None,
+    n_blocks [B] int32, status [1] int32 or None.
+    """
+    fp4: object
+    scale: object
+    n_blocks: object
+    block: int
+    idx_key: object = None
+    idx_dtype: int = CSA_IDX_BF16
+    status: object = None
+
+    @property
+    def batch(self) -> int:
+        return self.fp4.shape[0]
+
+    @property
+    def capacity(self) -> int:
+        return self.fp4.shape[1]
+
+    @property
+    def dim(self) -> int:
+        return self.fp4.shape[2] * 2
+
+    @property
+    def idx_dim(self) -> int:
+        return 0 if self.idx_key is None else self.idx_key.shape[2]
+
+    def c_struct(self) -> _CCache:
+        return _CCache(self.batch, self.dim, self.block, self.capacity, _ptr(self.fp4), _ptr(self.scale),
+                       _ptr(self.idx_key), self.idx_dim, self.idx_dtype, _ptr(self.n_blocks), _ptr(self.status))
+
+    @staticmethod
+    def allocate(batch: int, capacity: int, dim: int, block: int, idx_dim: int = 0, idx_dtype: int = CSA_IDX_BF16,
+                 device="cuda"):
+        """Zero-filled cache tensors on `device` (torch allocation; the library allocates nothing)."""
+        import torch
+
+        idx = None
+        if idx_dim:
+            dt = torch.bfloat16 if idx_dtype == CSA_IDX_BF16 else torch.uint8
+            idx = torch.zeros(batch, capacity, idx_dim, dtype=dt, device=device)
+        return Cache(fp4=torch.zeros(batch, capacity, dim // 2, dtype=torch.uint8, device=device),
+                     scale=torch.zeros(batch, capacity, dim // 32, dtype=torch.uint8, device=device),
+                     n_blocks=torch.zeros(batch, dtype=torch.int32, device=device), block=block,
+                     idx_key=idx, idx_dtype=idx_dtype, status=torch.zeros(1, dtype=torch.int32, device=device))
+
+
+def csa_version() -> int:
+    return load_library().csa_version()
+
+
+def csa_compress_quantize(cache: Cache, kv_tok, idx_tok, gate_w, tok_offsets, stream=None):
+    """Rows a1+a2: pool every m new tokens of each request into one block and store it (MXFP4 + indexer key)."""
+    lib = load_library()
+    c = cache.c_struct()
+    _check(lib.csa_compress_quantize(ctypes.byref(c), _ptr(kv_tok), _ptr(idx_tok), _ptr(gate_w), _ptr(tok_offsets),
+                                     int(kv_tok.shape[0]), _stream(stream)), "csa_compress_quantize")
+
+
+def csa_index_topk_workspace(cache: Cache, n_queries: int, topk: int) -> int:
+    return int(load_library().csa_index_topk_workspace(ctypes.byref(cache.c_struct()), n_queries, topk))
+
+
+def csa_attend_workspace(cache: Cache, n_queries: int, heads: int) -> int:
+    return int(load_library().csa_attend_workspace(ctypes.byref(cache.c_struct()), n_queries, heads))
+
+
+def _workspace(nbytes: int, workspace, device):
+    import torch
+
+    if workspace is not None:
+        return workspace
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def csa_index_topk(cache: Cache, q_idx, w, q_offsets, q_pos, topk: int, sel_idx=None, workspace=None, stream=None):
+    """Rows a3+a4: indexer scores of every visible block and the top-k blocks per query (ascending, -1 padded)."""
+    import torch
+
+    lib = load_library()
+    n_queries, idx_heads = int(q_idx.shape[0]), int(q_idx.shape[1])
+    if sel_idx is None:
+        sel_idx = torch.empty(n_queries, topk, dtype=torch.int32, device=q_idx.device)
+    need = csa_index_topk_workspace(cache, n_queries, topk)
+    workspace = _workspace(need, workspace, q_idx.device)
+    c = cache.c_struct()
+    _check(lib.csa_index_topk(ctypes.byref(c), _ptr(q_idx), _ptr(w), n_queries, idx_heads, _ptr(q_offsets),
+                              _ptr(q_pos), topk, _ptr(sel_idx), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "csa_index_topk")
+    return sel_idx
+
+
+def csa_decode_attend(cache: Cache, q, q_offsets, sel_idx, win_kv=None, win_start=None, win_len=None,
+                      max_win: int = 128, softmax_scale: Optional[float] = None, out=None, lse=None,
+                      workspace=None, stream=None):
+    """Rows a5+a6+a8: joint softmax attention over the selected compressed entries and the window."""
+    import torch
+
+    lib = load_library()
+    n_queries, heads, D = (int(x) for x in q.shape)
+    if softmax_scale is None:
+        softmax_scale = D ** -0.5
+    if out is None:
+        out = torch.empty(n_queries, heads, D, dtype=torch.float32, device=q.device)
+    need = csa_attend_workspace(cache, n_queries, heads)
+    workspace = _workspace(need, workspace, q.device)
+    c = cache.c_struct()
+    _check(lib.csa_decode_attend(ctypes.byref(c), _ptr(q), n_queries, heads, _ptr(q_offsets), _ptr(sel_idx),
+                                 int(sel_idx.shape[1]), _ptr(win_kv), _ptr(win_start), _ptr(win_len), max_win,
+                                 float(softmax_scale), _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
+                                 _stream(stream)), "csa_decode_attend")
+    return out
+
+
+def hca_decode_attend(cache: Cache, q, q_offsets, q_pos, win_kv=None, win_start=None, win_len=None,
+                      max_win: int = 128, softmax_scale: Optional[float] = None, out=None, lse=None,
+                      workspace=None, stream=None):
+    """Row a7 (+a8): dense attention over every visible compressed entry and the window."""
+    import torch
+
+    lib = load_library()
+    n_queries, heads, D = (int(x) for x in q.shape)
+    if softmax_scale is None:
+        softmax_scale = D ** -0.5
+    if out is None:
+        out = torch.empty(n_queries, heads, D, dtype=torch.float32, device=q.device)
+    need = csa_attend_workspace(cache, n_queries, heads)
+    workspace = _workspace(need, workspace, q.device)
+    c = cache.c_struct()
+    _check(lib.hca_decode_attend(ctypes.byref(c), _ptr(q), n_queries, heads, _ptr(q_offsets), _ptr(q_pos),
+                                 _ptr(win_kv), _ptr(win_start), _ptr(win_len), max_win, float(softmax_scale),
+                                 _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "hca_decode_attend")
+    return out
+
+
+def csa_read_device_status(cache: Cache, stream=None) -> int:
+    """Synchronize, return and clear the device status bits (CSA_DEV_*)."""
+    lib = load_library()
+    v = ctypes.c_int32(0)
+    c = cache.c_struct()
+    _check(lib.csa_read_device_status(ctypes.byref(c), _stream(stream), ctypes.byref(v)), "csa_read_device_status")
+    return int(v.value)

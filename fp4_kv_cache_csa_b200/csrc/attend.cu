@@ -1,0 +1,859 @@
+// attend.cu -- rows a5 + a6 + a7 + a8: dequantize the attended MXFP4 entries
+// right before attention, one joint softmax over compressed entries and the
+// uncompressed window, split over CTAs with a log-sum-exp merge.
+//
+// Sources: "Frontier Architecture Decoding Notes (4): DeepSeek V4", section 1
+// (CSA attends the top-k compressed entries, HCA every entry of a 128x
+// compressed cache, plus the latest 128 tokens uncompressed);
+// DeepSeek-V4.1-Flash podcast transcript, cue 16 (MXFP4 main KV, dequantized
+// right before attention). All heads share one latent vector per entry that is
+// both key and value (cue 8: a shared latent), so the heads x D by D x entries
+// products are dense contractions and run on the tcgen05 tensor cores.
+//
+// Design (one CTA per SM, 128 threads, thread j <-> entry j of a 128-entry tile):
+//   * Work = the flat list of 128-entry tiles of all queries (compressed tiles
+//     first, then window tiles), cut into equal contiguous ranges, one per CTA.
+//     A CTA whose range covers a whole query writes the output directly;
+//     otherwise it writes an unnormalized partial and the last CTA to finish
+//     that query (atomic counter, no waiting) merges the partials.
+//   * Operands are fp16 in shared memory. Entry j is stored as
+//     E'_j = e_j * 2^-R_j with R_j the largest E8M0 exponent of the row (or the
+//     exponent of max|x| for a window row): every E2M1 x 2^X value is exact in
+//     fp16 within 2^24 of the row's largest group. The query is stored as
+//     q * 2^-sQ (exact for bf16 values within 2^31 of max|q|).
+//   * S^T = E' Q'^T: M = 128 entries (TMEM lanes), N = 64 heads (columns).
+//   * Softmax in the log2 domain, thread j holding the 64 head logits of its
+//     entry: u = log2(e) * scale * <q,e_j> + R_j. Each head h keeps a reference
+//     rho_h, raised (and the TMEM accumulator rescaled) only when a tile's
+//     max exceeds it by more than 8; P'_{j,h} = 2^(u - rho_h) <= 256 is stored
+//     in fp16 (11-bit significand), folding the row factor 2^R_j back in.
+//   * O^T += E'^T P': M = 128 latent channels per d-tile, N = 64 heads, K = 16
+//     entries per MMA; O^T lives in TMEM for the whole segment.
+//   * out = O / l and lse = ln 2 * (rho + log2 l), l = sum_j 2^(lambda_j - rho).
+// Compressed tiles are loaded into registers one tile ahead (prefetch while
+// the tensor core works); window tiles (bf16) are copied with cp.async into
+// the operand buffer and converted in place.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp4.h>
+
+#include "common.cuh"
+
+namespace csa {
+
+namespace {
+
+constexpr int kTile = 128;
+constexpr int kHeads = 64;
+constexpr int kThreads = 128;
+constexpr long long kWaitCycles = 2000000000LL;  // bounded mbarrier wait (~1 s)
+
+template <int D>
+struct Cfg {
+    static constexpr int KCH = D / 64;                    // 128-byte k-chunks per row
+    static constexpr int DT = D / 128;                    // O^T d-tiles
+    static constexpr int GPR = D / 32;                    // MXFP4 groups per row
+    static constexpr int CODE_V = D / 32;                 // 16-byte code loads per row (D/2 bytes)
+    static constexpr int E_BYTES = kTile * D * 2;
+    static constexpr int Q_BYTES = kHeads * D * 2;
+    static constexpr int P_BYTES = kTile * kHeads * 2;
+    static constexpr int KREG = kTile * 128;              // bytes per k-chunk region of E'
+    static constexpr int QREG = kHeads * 128;             // bytes per k-chunk region of Q'
+    static constexpr int TMEM_USED = kHeads + DT * kHeads;
+    static constexpr int TMEM_COLS = TMEM_USED <= 128 ? 128 : TMEM_USED <= 256 ? 256 : 512;
+    static constexpr int MISC_BYTES = 4096;
+    static constexpr int SMEM = 1024 + E_BYTES + Q_BYTES + P_BYTES + MISC_BYTES;
+};
+
+// ---------------------------------------------------------------- PTX helpers
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+    // tcgen05 shared-memory matrix descriptor: start >> 4, LBO >> 4, SBO >> 4,
+    // version 1 (bits 46-47), 128-byte swizzle (layout type 2, bits 61-63).
+    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor, kind::f16: D f32 (bits 4-5 = 1), A/B f16 (0),
+// A/B major (bits 15/16), N >> 3 (bits 17-22), M >> 4 (bits 24-28).
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool a_mn, bool b_mn) {
+    return (1u << 4) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
+           ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n"
+        :
+        : "r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t mbar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ void mbar_init(uint32_t mbar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(mbar), "r"(count) : "memory");
+}
+
+// Wait for the phase with this parity to complete; gives up after kWaitCycles.
+__device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity) {
+    const long long t0 = clock64();
+    while (true) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}\n"
+            : "=r"(done)
+            : "r"(mbar), "r"(parity)
+            : "memory");
+        if (done) return true;
+        if (clock64() - t0 > kWaitCycles) return false;
+    }
+}
+
+#define CSA_LD16(base, r)                                                                                    \
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];" \
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), \
+                   "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),       \
+                   "=r"(r[15])                                                                              \
+                 : "r"(base))
+#define CSA_ST16(base, r)                                                                                     \
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" \
+                 ::"r"(base), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), \
+                   "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])     \
+                 : "memory")
+
+// 64 consecutive 32-bit TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
+    uint32_t r[16];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        CSA_LD16(taddr + 16 * q, r);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) v[16 * q + k] = __uint_as_float(r[k]);
+    }
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_st64(uint32_t taddr, const float (&v)[64]) {
+    uint32_t r[16];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+#pragma unroll
+        for (int k = 0; k < 16; ++k) r[k] = __float_as_uint(v[16 * q + k]);
+        CSA_ST16(taddr + 16 * q, r);
+    }
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+// Butterfly transpose-reduction: 64 values per lane -> lane L ends with the
+// reduction over all 32 lanes of entries 2L and 2L+1 (in v[0], v[1]).
+template <bool MAX>
+__device__ __forceinline__ void transpose_reduce64(float (&v)[64]) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int half = 32, o = 16; o >= 1; half >>= 1, o >>= 1) {
+        const bool hi = (lane & o) != 0;
+#pragma unroll
+        for (int k = 0; k < half; ++k) {
+            const float send = hi ? v[k] : v[k + half];
+            const float keep = hi ? v[k + half] : v[k];
+            const float got = __shfl_xor_sync(0xffffffffu, send, o);
+            v[k] = MAX ? fmaxf(keep, got) : keep + got;
+        }
+    }
+}
+
+// ---------------------------------------------------------------- arguments
+struct AttArgs {
+    const uint8_t *fp4, *scale;      // cache planes
+    const int32_t *n_blocks;
+    const __nv_bfloat16 *q;          // [Nq][H][D]
+    const int32_t *sel_idx;          // CSA: [Nq][topk]; HCA: null
+    const __nv_bfloat16 *win_kv;     // [rows][D] or null
+    const int64_t *win_start;
+    float *out, *lse;
+    int32_t *status;
+    // schedule (workspace)
+    const int32_t *req, *nent, *ctiles, *wlen;
+    const long long *tprefix;        // [Nq+1]
+    uint32_t *counters;              // [Nq]
+    float *part_o, *part_rho, *part_l;  // [2G][64][D], [2G][64], [2G][64]
+    int Nq, H, cap, topk;
+    float scale_log2;                // softmax_scale * log2(e)
+};
+
+// Per-row prefetch of one compressed entry (codes + E8M0 bytes).
+template <int D>
+struct RowRegs {
+    uint4 code[Cfg<D>::CODE_V];
+    uint4 sc;
+    int valid;
+};
+
+struct TileRef {
+    int i;      // query (-1: none)
+    int lt;     // local tile index within the query
+    int win;    // 1: window tile
+};
+
+__device__ __forceinline__ TileRef locate(const AttArgs &a, long long t) {
+    int lo = 0, hi = a.Nq - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (a.tprefix[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    TileRef r;
+    r.i = lo;
+    r.lt = (int)(t - a.tprefix[lo]);
+    r.win = r.lt >= a.ctiles[lo];
+    return r;
+}
+
+// Issue the loads of this thread's row of a compressed tile.
+template <int D>
+__device__ __forceinline__ void prefetch_row(const AttArgs &a, const TileRef &tr, RowRegs<D> &rr) {
+    rr.valid = 0;
+    const int j = threadIdx.x;
+    const int slot = tr.lt * kTile + j;
+    const int i = tr.i;
+    const int b = a.req[i];
+    int blk = -1;
+    if (slot < a.nent[i]) {
+        if (a.sel_idx) {
+            blk = a.sel_idx[(size_t)i * a.topk + slot];
+            if (blk >= a.n_blocks[b] || blk >= a.cap) {
+                flag(a.status, CSA_DEV_BAD_INDEX);
+                blk = -1;
+            }
+        } else {
+            blk = slot;
+        }
+    }
+    if (blk >= 0) {
+        const size_t row = (size_t)b * a.cap + blk;
+        const uint4 *src = reinterpret_cast<const uint4 *>(a.fp4 + row * (D / 2));
+#pragma unroll
+        for (int v = 0; v < Cfg<D>::CODE_V; ++v) rr.code[v] = __ldg(src + v);
+        if constexpr (D / 32 >= 16) {
+            rr.sc = __ldg(reinterpret_cast<const uint4 *>(a.scale + row * (D / 32)));
+        } else {
+            rr.sc = make_uint4(__ldg(reinterpret_cast<const uint32_t *>(a.scale + row * (D / 32))), 0, 0, 0);
+        }
+        rr.valid = 1;
+    }
+}
+
+// Byte k of the row's scale bytes.
+template <int D>
+__device__ __forceinline__ int scale_byte(const RowRegs<D> &rr, int k) {
+    const uint32_t w = k < 4 ? rr.sc.x : k < 8 ? rr.sc.y : k < 12 ? rr.sc.z : rr.sc.w;
+    return (int)((w >> (8 * (k & 3))) & 0xFF);
+}
+
+// Swizzled byte offset of 16-byte chunk kc (channels 8kc..8kc+7) of row j of E'.
+template <int D>
+__device__ __forceinline__ uint32_t e_chunk_off(int j, int kc) {
+    return (uint32_t)((kc >> 3) * Cfg<D>::KREG + (j >> 3) * 1024 + (j & 7) * 128 + (((kc & 7) ^ (j & 7)) << 4));
+}
+
+// Dequantize this thread's prefetched row into E' (fp16, scaled by 2^-R_j).
+// Returns R_j (the row's largest E8M0 exponent); invalid rows are zero.
+template <int D>
+__device__ __forceinline__ int dequant_row(const RowRegs<D> &rr, uint8_t *E) {
+    const int j = threadIdx.x;
+    if (!rr.valid) {
+#pragma unroll 4
+        for (int kc = 0; kc < D / 8; ++kc) *reinterpret_cast<uint4 *>(E + e_chunk_off<D>(j, kc)) = make_uint4(0, 0, 0, 0);
+        return 0;
+    }
+    int rmax = 0;
+#pragma unroll
+    for (int g = 0; g < Cfg<D>::GPR; ++g) rmax = max(rmax, scale_byte<D>(rr, g));
+#pragma unroll
+    for (int g = 0; g < Cfg<D>::GPR; ++g) {
+        const int k = scale_byte<D>(rr, g) - rmax;  // <= 0
+        // 2^k in fp16: normal for k >= -14, subnormal down to -24, else 0
+        const uint16_t hb = k >= -14 ? (uint16_t)((k + 15) << 10) : k >= -24 ? (uint16_t)(1u << (k + 24)) : 0;
+        __half2 s2 = __halves2half2(__ushort_as_half(hb), __ushort_as_half(hb));
+        const uint32_t *w = reinterpret_cast<const uint32_t *>(&rr.code[g]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {  // 4 bytes -> 8 channels -> one 16-byte chunk
+            uint32_t outw[4];
+#pragma unroll
+            for (int bb = 0; bb < 4; ++bb) {
+                __half2_raw hr = __nv_cvt_fp4x2_to_halfraw2((__nv_fp4x2_storage_t)((w[c] >> (8 * bb)) & 0xFF), __NV_E2M1);
+                __half2 h = __hmul2(*reinterpret_cast<__half2 *>(&hr), s2);
+                outw[bb] = *reinterpret_cast<uint32_t *>(&h);
+            }
+            *reinterpret_cast<uint4 *>(E + e_chunk_off<D>(j, 4 * g + c)) = make_uint4(outw[0], outw[1], outw[2], outw[3]);
+        }
+    }
+    return rmax - 127;
+}
+
+// Window tile: cp.async the bf16 rows into E' and convert them in place to
+// fp16 scaled by 2^-R_j, R_j = exponent of the row's max |x|.
+template <int D>
+__device__ __forceinline__ int load_window_row(const AttArgs &a, const TileRef &tr, uint8_t *E, uint32_t E_s, bool &valid) {
+    const int j = threadIdx.x;
+    const int r = (tr.lt - a.ctiles[tr.i]) * kTile + j;
+    valid = r < a.wlen[tr.i];
+    if (!valid) {
+        for (int kc = 0; kc < D / 8; ++kc) *reinterpret_cast<uint4 *>(E + e_chunk_off<D>(j, kc)) = make_uint4(0, 0, 0, 0);
+        return 0;
+    }
+    const __nv_bfloat16 *src = a.win_kv + ((size_t)a.win_start[tr.i] + r) * D;
+#pragma unroll 8
+    for (int kc = 0; kc < D / 8; ++kc) cp_async16(E_s + e_chunk_off<D>(j, kc), src + 8 * kc);
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_all;" ::: "memory");
+    float mx = 0.f;
+    for (int kc = 0; kc < D / 8; ++kc) {
+        uint4 u = *reinterpret_cast<const uint4 *>(E + e_chunk_off<D>(j, kc));
+        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            float2 f = __bfloat1622float2(h[k]);
+            mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
+        }
+    }
+    const int R = mx > 0.f ? (int)((__float_as_uint(mx) >> 23) & 0xFF) - 127 : 0;
+    const float inv = ldexpf(1.0f, -R);
+    for (int kc = 0; kc < D / 8; ++kc) {
+        uint4 u = *reinterpret_cast<const uint4 *>(E + e_chunk_off<D>(j, kc));
+        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+        uint32_t o[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            float2 f = __bfloat1622float2(h[k]);
+            __half2 hh = __floats2half2_rn(f.x * inv, f.y * inv);
+            o[k] = *reinterpret_cast<uint32_t *>(&hh);
+        }
+        *reinterpret_cast<uint4 *>(E + e_chunk_off<D>(j, kc)) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    return R;
+}
+
+// Q' = q * 2^-sQ in fp16, K-major with 128-byte swizzle, heads >= H zero.
+// Returns sQ.
+template <int D>
+__device__ int load_query(const AttArgs &a, int i, uint8_t *Q, float *red) {
+    const int tid = threadIdx.x;
+    const __nv_bfloat16 *qi = a.q + (size_t)i * a.H * D;
+    const int nchunks = a.H * (D / 8);
+    float mx = 0.f;
+    for (int c = tid; c < nchunks; c += kThreads) {
+        uint4 u = __ldg(reinterpret_cast<const uint4 *>(qi) + c);
+        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            float2 f = __bfloat1622float2(h[k]);
+            mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
+        }
+    }
+    mx = warp_max(mx);
+    if ((tid & 31) == 0) red[tid >> 5] = mx;
+    __syncthreads();
+    mx = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    __syncthreads();
+    const int sQ = mx > 0.f ? (int)((__float_as_uint(mx) >> 23) & 0xFF) - 127 - 14 : 0;
+    const float inv = ldexpf(1.0f, -sQ);
+    // chunk (h, kc): consecutive threads take consecutive heads, so the
+    // swizzled 16-byte stores of a warp spread over all eight bank groups
+    for (int c = tid; c < kHeads * (D / 8); c += kThreads) {
+        const int h = c % kHeads;
+        const int kc = c / kHeads;
+        uint32_t o[4] = {0u, 0u, 0u, 0u};
+        if (h < a.H) {
+            uint4 u = __ldg(reinterpret_cast<const uint4 *>(qi + (size_t)h * D) + kc);
+            const __nv_bfloat162 *hh = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                float2 f = __bfloat1622float2(hh[k]);
+                __half2 x = __floats2half2_rn(f.x * inv, f.y * inv);
+                o[k] = *reinterpret_cast<uint32_t *>(&x);
+            }
+        }
+        const uint32_t off = (uint32_t)((kc >> 3) * Cfg<D>::QREG + (h >> 3) * 1024 + (h & 7) * 128 + (((kc & 7) ^ (h & 7)) << 4));
+        *reinterpret_cast<uint4 *>(Q + off) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    return sQ;
+}
+
+// ---------------------------------------------------------------- schedule
+__global__ void attend_schedule_kernel(const int32_t *q_offsets, const int32_t *q_pos, const int32_t *n_blocks,
+                                       const int32_t *win_len, int batch, int Nq, int m, int cap, int topk, int max_win,
+                                       int H, int D, int32_t *req, int32_t *nent, int32_t *ctiles, int32_t *wlen,
+                                       long long *tprefix, float *out, float *lse, int32_t *status) {
+    __shared__ long long red[32];
+    __shared__ long long round_total;
+    long long carry = 0;
+    for (int base = 0; base < Nq; base += blockDim.x) {
+        const int i = base + threadIdx.x;
+        long long tiles = 0;
+        if (i < Nq) {
+            const int b = request_of(q_offsets, batch, i);
+            int ne = 0;
+            if (b >= 0) ne = (q_pos ? min(visible_blocks(q_pos[i], m, n_blocks[b]), cap) : topk);
+            int wl = win_len ? win_len[i] : 0;
+            if (wl < 0 || wl > max_win) {
+                flag(status, CSA_DEV_BAD_WINDOW);
+                wl = min(max(wl, 0), max_win);
+            }
+            if (b < 0) wl = 0;
+            const int ct = (ne + kTile - 1) / kTile;
+            req[i] = b < 0 ? 0 : b;
+            nent[i] = ne;
+            ctiles[i] = ct;
+            wlen[i] = wl;
+            tiles = ct + (wl + kTile - 1) / kTile;
+        }
+        const long long incl = block_inclusive_scan<long long>(tiles, red);
+        if (i < Nq) tprefix[i + 1] = carry + incl;
+        if (i == 0) tprefix[0] = 0;
+        if (threadIdx.x == blockDim.x - 1) round_total = incl;
+        __syncthreads();
+        carry += round_total;
+        __syncthreads();
+    }
+    // queries with no entry at all: out = 0, lse = -inf
+    __syncthreads();
+    for (int i = 0; i < Nq; ++i) {
+        if (tprefix[i + 1] != tprefix[i]) continue;
+        for (int k = threadIdx.x; k < H * D; k += blockDim.x) out[(size_t)i * H * D + k] = 0.f;
+        if (lse)
+            for (int k = threadIdx.x; k < H; k += blockDim.x) lse[(size_t)i * H + k] = -INFINITY;
+    }
+}
+
+// ---------------------------------------------------------------- main kernel
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
+    using C = Cfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *E = smem;
+    uint8_t *Q = E + C::E_BYTES;
+    uint8_t *P = Q + C::Q_BYTES;
+    uint8_t *misc = P + C::P_BYTES;
+    uint64_t *mbar = reinterpret_cast<uint64_t *>(misc);            // [0] S done, [1] PV done
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + 16);
+    int *flags = reinterpret_cast<int *>(misc + 32);                // [0] rescale, [1] last, [2] abort
+    float *rho = reinterpret_cast<float *>(misc + 64);              // [64]
+    float *alpha = rho + 64;                                        // [64]
+    float *wred = alpha + 64;                                       // [4][64]
+    float *red = wred + 4 * 64;                                     // [32]
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const long long T = a.tprefix[a.Nq];
+    const int G = gridDim.x, c = blockIdx.x;
+    const long long t_begin = T * c / G, t_end = T * (c + 1) / G;
+    if (t_begin >= t_end) return;
+
+    const uint32_t E_s = smem_u32(E), Q_s = smem_u32(Q), P_s = smem_u32(P);
+    const uint32_t mbar_s = smem_u32(&mbar[0]), mbar_pv = smem_u32(&mbar[1]);
+    if (tid == 0) {
+        mbar_init(mbar_s, 1);
+        mbar_init(mbar_pv, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        flags[2] = 0;
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(C::TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tmem_s = tmem;                 // S^T: columns [0, 64)
+    const uint32_t tmem_o = tmem + kHeads;        // O^T d-tile dt: columns 64 + 64 dt
+    const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+    uint32_t ph_s = 0, ph_pv = 0;
+    bool pv_pending = false;
+
+    constexpr uint32_t IDESC_S = idesc_f16(kTile, kHeads, false, false);
+    constexpr uint32_t IDESC_PV = idesc_f16(kTile, kHeads, true, true);
+
+    RowRegs<D> rr;
+    TileRef cur = locate(a, t_begin);
+    if (!cur.win) prefetch_row<D>(a, cur, rr);
+
+    long long t = t_begin;
+    bool aborted = false;
+    while (t < t_end && !aborted) {
+        // ---------------- segment = the tiles of query cur.i inside [t, t_end)
+        const int i = cur.i;
+        const long long seg_begin = t;
+        const long long seg_end = min(t_end, a.tprefix[i + 1]);
+        const bool whole = (seg_begin == a.tprefix[i]) && (seg_end == a.tprefix[i + 1]);
+        // the previous segment's PV must finish before Q' and O^T are reused
+        if (pv_pending) {
+            const bool ok = mbar_wait(mbar_pv, ph_pv);
+            ph_pv ^= 1;
+            pv_pending = false;
+            if (__syncthreads_or(!ok)) { aborted = true; break; }
+        }
+        const int sQ = load_query<D>(a, i, Q, red);
+        float l_part[2] = {0.f, 0.f};  // per-warp partial row sums of heads 2*lane, 2*lane+1
+        bool first = true;
+
+        for (; t < seg_end; ++t) {
+            // ---- operand E' for this tile ----
+            if (pv_pending) {
+                const bool ok = mbar_wait(mbar_pv, ph_pv);
+                ph_pv ^= 1;
+                pv_pending = false;
+                if (__syncthreads_or(!ok)) { aborted = true; break; }
+            }
+            int Rj;
+            bool valid;
+            if (cur.win) {
+                Rj = load_window_row<D>(a, cur, E, E_s, valid);
+            } else {
+                valid = rr.valid;
+                Rj = dequant_row<D>(rr, E);
+            }
+            // next tile (possibly of the next query): start its loads now
+            TileRef nxt;
+            nxt.i = -1;
+            if (t + 1 < t_end) {
+                nxt = locate(a, t + 1);
+                if (!nxt.win) prefetch_row<D>(a, nxt, rr);
+            }
+            fence_async_smem();
+            tc_fence_before();
+            __syncthreads();
+
+            // ---- S^T = E' Q'^T ----
+            if (tid == 0) {
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t koff = (uint32_t)((kk & 3) * 32);
+                    const uint64_t da = desc_sw128(E_s + (kk >> 2) * C::KREG + koff, 16, 1024);
+                    const uint64_t db = desc_sw128(Q_s + (kk >> 2) * C::QREG + koff, 16, 1024);
+                    mma_f16(tmem_s, da, db, IDESC_S, kk > 0);
+                }
+                mma_commit(mbar_s);
+            }
+            {
+                const bool ok = mbar_wait(mbar_s, ph_s);
+                ph_s ^= 1;
+                if (__syncthreads_or(!ok)) { aborted = true; break; }
+            }
+            tc_fence_after();
+            float u[64];
+            tmem_ld64(tmem_s + lane_off, u);
+            // u = log2(e) * scale * <q, e_j> + R_j, or -inf for an empty row
+            {
+                const float cj = ldexpf(a.scale_log2, Rj + sQ);
+#pragma unroll
+                for (int h = 0; h < 64; ++h) u[h] = valid ? fmaf(u[h], cj, (float)Rj) : -INFINITY;
+            }
+            // ---- per-head tile max -> reference update ----
+            {
+                float m[64];
+#pragma unroll
+                for (int h = 0; h < 64; ++h) m[h] = u[h];
+                transpose_reduce64<true>(m);
+                wred[warp * 64 + 2 * lane] = m[0];
+                wred[warp * 64 + 2 * lane + 1] = m[1];
+            }
+            __syncthreads();
+            if (tid < 64) {
+                const float M = fmaxf(fmaxf(wred[tid], wred[64 + tid]), fmaxf(wred[128 + tid], wred[192 + tid]));
+                float al = 1.f;
+                if (first) {
+                    rho[tid] = (M == -INFINITY) ? 0.f : M;
+                } else if (M > rho[tid] + 8.f) {
+                    al = exp2f(rho[tid] - M);
+                    rho[tid] = M;
+                }
+                alpha[tid] = al;
+                if (al != 1.f) flags[0] = 1;
+            }
+            __syncthreads();
+            if (flags[0]) {  // rescale O^T columns and the row sums (PV of the previous tile is complete)
+                tc_fence_after();
+#pragma unroll 1
+                for (int dt = 0; dt < C::DT; ++dt) {
+                    float o[64];
+                    tmem_ld64(tmem_o + 64 * dt + lane_off, o);
+#pragma unroll
+                    for (int h = 0; h < 64; ++h) o[h] *= alpha[h];
+                    tmem_st64(tmem_o + 64 * dt + lane_off, o);
+                }
+                l_part[0] *= alpha[2 * lane];
+                l_part[1] *= alpha[2 * lane + 1];
+            }
+            // ---- P' = 2^(u - rho) (fp16) and row sums ----
+            {
+                const float rj_inv = ldexpf(1.0f, -Rj);
+                uint32_t pk[32];
+                float ls[64];
+#pragma unroll
+                for (int h = 0; h < 64; h += 2) {
+                    const float p0 = exp2f(u[h] - rho[h]);
+                    const float p1 = exp2f(u[h + 1] - rho[h + 1]);
+                    __half2 hh = __floats2half2_rn(p0, p1);
+                    pk[h / 2] = *reinterpret_cast<uint32_t *>(&hh);
+                    ls[h] = p0 * rj_inv;
+                    ls[h + 1] = p1 * rj_inv;
+                }
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc) {
+                    const uint32_t off = (uint32_t)((tid >> 3) * 1024 + (tid & 7) * 128 + ((cc ^ (tid & 7)) << 4));
+                    *reinterpret_cast<uint4 *>(P + off) = make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
+                }
+                transpose_reduce64<false>(ls);
+                l_part[0] += ls[0];
+                l_part[1] += ls[1];
+            }
+            fence_async_smem();
+            tc_fence_before();
+            __syncthreads();
+            if (tid == 0) {
+                flags[0] = 0;
+                tc_fence_after();
+#pragma unroll
+                for (int dt = 0; dt < C::DT; ++dt) {
+#pragma unroll
+                    for (int kj = 0; kj < kTile / 16; ++kj) {
+                        const uint64_t da = desc_sw128(E_s + (2 * dt) * C::KREG + kj * 2048, C::KREG, 1024);
+                        const uint64_t db = desc_sw128(P_s + kj * 2048, 8192, 1024);
+                        mma_f16(tmem_o + 64 * dt, da, db, IDESC_PV, (first && kj == 0) ? 0u : 1u);
+                    }
+                }
+                mma_commit(mbar_pv);
+            }
+            pv_pending = true;
+            first = false;
+            if (nxt.i >= 0) cur = nxt;
+        }
+        if (aborted) break;
+
+        // ---------------- segment epilogue
+        {
+            const bool ok = mbar_wait(mbar_pv, ph_pv);
+            ph_pv ^= 1;
+            pv_pending = false;
+            if (__syncthreads_or(!ok)) { aborted = true; break; }
+        }
+        tc_fence_after();
+        wred[warp * 64 + 2 * lane] = l_part[0];
+        wred[warp * 64 + 2 * lane + 1] = l_part[1];
+        __syncthreads();
+        if (tid < 64) {
+            const float l = wred[tid] + wred[64 + tid] + wred[128 + tid] + wred[192 + tid];
+            alpha[tid] = l;  // l_h
+        }
+        __syncthreads();
+        const int b_slot = 2 * c + ((seg_begin == T * c / G) ? 0 : 1);
+        if (whole) {
+            for (int dt = 0; dt < C::DT; ++dt) {
+                float o[64];
+                tmem_ld64(tmem_o + 64 * dt + lane_off, o);
+                const int d = 128 * dt + 32 * warp + lane;
+#pragma unroll
+                for (int h = 0; h < 64; ++h) {
+                    if (h < a.H) {
+                        const float l = alpha[h];
+                        a.out[((size_t)i * a.H + h) * D + d] = l > 0.f ? o[h] / l : 0.f;
+                    }
+                }
+            }
+            if (a.lse && tid < a.H) {
+                const float l = alpha[tid];
+                a.lse[(size_t)i * a.H + tid] = l > 0.f ? (rho[tid] + log2f(l)) * 0.69314718055994531f : -INFINITY;
+            }
+        } else {
+            float *po = a.part_o + (size_t)b_slot * kHeads * D;
+            for (int dt = 0; dt < C::DT; ++dt) {
+                float o[64];
+                tmem_ld64(tmem_o + 64 * dt + lane_off, o);
+                const int d = 128 * dt + 32 * warp + lane;
+#pragma unroll
+                for (int h = 0; h < 64; ++h)
+                    if (h < a.H) po[(size_t)h * D + d] = o[h];
+            }
+            if (tid < 64) {
+                a.part_rho[(size_t)b_slot * kHeads + tid] = rho[tid];
+                a.part_l[(size_t)b_slot * kHeads + tid] = alpha[tid];
+            }
+            __threadfence();
+            __syncthreads();
+            if (tid == 0) {
+                // completion is counted in tiles: the CTA that brings the count to
+                // the query's tile total is the last one and merges
+                const long long Ti = a.tprefix[i], Ti1 = a.tprefix[i + 1];
+                const uint32_t seg_tiles = (uint32_t)(seg_end - seg_begin);
+                const uint32_t prev = atomicAdd(a.counters + i, seg_tiles);
+                flags[1] = (prev + seg_tiles == (uint32_t)(Ti1 - Ti)) ? 1 : 0;
+                if (flags[1]) {
+                    // partial slots of every CTA whose (non-empty) range meets [Ti, Ti1)
+                    int *slots = reinterpret_cast<int *>(wred);
+                    int np = 0;
+                    const int c_first = (int)(((Ti + 1) * G - 1) / T);
+                    const int c_last = (int)((Ti1 * G - 1) / T);
+                    for (int cc = c_first; cc <= c_last && np < 4 * 64; ++cc) {
+                        const long long rb = T * cc / G, re = T * (cc + 1) / G;
+                        if (rb >= re) continue;
+                        slots[np++] = 2 * cc + (rb >= Ti ? 0 : 1);
+                    }
+                    flags[3] = np;
+                }
+            }
+            __syncthreads();
+            if (flags[1]) {  // last CTA of this query: merge every partial
+                __threadfence();
+                const int np = flags[3];
+                const int *slots = reinterpret_cast<const int *>(wred);
+                float *wts = reinterpret_cast<float *>(E);  // E' is free now: [np][64] weights
+                if (tid < 64) {
+                    float rmax = -INFINITY;
+                    for (int p = 0; p < np; ++p)
+                        rmax = fmaxf(rmax, __ldcg(a.part_rho + (size_t)slots[p] * kHeads + tid));
+                    float lsum = 0.f;
+                    for (int p = 0; p < np; ++p) {
+                        const float wgt = exp2f(__ldcg(a.part_rho + (size_t)slots[p] * kHeads + tid) - rmax);
+                        wts[p * 64 + tid] = wgt;
+                        lsum += wgt * __ldcg(a.part_l + (size_t)slots[p] * kHeads + tid);
+                    }
+                    rho[tid] = rmax;
+                    alpha[tid] = lsum;
+                }
+                __syncthreads();
+                for (int k = tid; k < a.H * D; k += kThreads) {
+                    const int h = k / D;
+                    float acc = 0.f;
+                    for (int p = 0; p < np; ++p)
+                        acc += wts[p * 64 + h] * __ldcg(a.part_o + (size_t)slots[p] * kHeads * D + k);
+                    const float l = alpha[h];
+                    a.out[(size_t)i * a.H * D + k] = l > 0.f ? acc / l : 0.f;
+                }
+                if (a.lse && tid < a.H) {
+                    const float l = alpha[tid];
+                    a.lse[(size_t)i * a.H + tid] = l > 0.f ? (rho[tid] + log2f(l)) * 0.69314718055994531f : -INFINITY;
+                }
+            }
+        }
+        __syncthreads();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    }
+
+    if (aborted) {
+        if (tid == 0) flag(a.status, CSA_DEV_TIMEOUT);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TMEM_COLS) : "memory");
+}
+
+}  // namespace
+
+size_t attend_workspace_bytes(int Nq, int D, int num_ctas) {
+    size_t off = 0;
+    auto take = [&](size_t bytes) { off = (off + bytes + 255) & ~size_t(255); };
+    take(4 * (size_t)Nq);            // req
+    take(4 * (size_t)Nq);            // nent
+    take(4 * (size_t)Nq);            // ctiles
+    take(4 * (size_t)Nq);            // wlen
+    take(8 * (size_t)(Nq + 1));      // tprefix
+    take(4 * (size_t)Nq);            // counters
+    take(4 * (size_t)2 * num_ctas * kHeads * D);  // part_o
+    take(4 * (size_t)2 * num_ctas * kHeads);      // part_rho
+    take(4 * (size_t)2 * num_ctas * kHeads);      // part_l
+    return off;
+}
+
+cudaError_t launch_attend(const csa_cache &c, const void *q, int Nq, int H, const int32_t *q_offsets,
+                          const int32_t *q_pos, const int32_t *sel_idx, int topk, const void *win_kv,
+                          const int64_t *win_start, const int32_t *win_len, int max_win, float softmax_scale,
+                          float *out, float *lse, void *workspace, int num_ctas, cudaStream_t s) {
+    const int D = c.dim;
+    char *base = static_cast<char *>(workspace);
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        char *p = base + off;
+        off = (off + bytes + 255) & ~size_t(255);
+        return p;
+    };
+    AttArgs a;
+    int32_t *req = reinterpret_cast<int32_t *>(take(4 * (size_t)Nq));
+    int32_t *nent = reinterpret_cast<int32_t *>(take(4 * (size_t)Nq));
+    int32_t *ctiles = reinterpret_cast<int32_t *>(take(4 * (size_t)Nq));
+    int32_t *wlen = reinterpret_cast<int32_t *>(take(4 * (size_t)Nq));
+    long long *tprefix = reinterpret_cast<long long *>(take(8 * (size_t)(Nq + 1)));
+    uint32_t *counters = reinterpret_cast<uint32_t *>(take(4 * (size_t)Nq));
+    a.part_o = reinterpret_cast<float *>(take(4 * (size_t)2 * num_ctas * kHeads * D));
+    a.part_rho = reinterpret_cast<float *>(take(4 * (size_t)2 * num_ctas * kHeads));
+    a.part_l = reinterpret_cast<float *>(take(4 * (size_t)2 * num_ctas * kHeads));
+    a.fp4 = c.fp4;
+    a.scale = c.scale;
+    a.n_blocks = c.n_blocks;
+    a.q = static_cast<const __nv_bfloat16 *>(q);
+    a.sel_idx = sel_idx;
+    a.win_kv = static_cast<const __nv_bfloat16 *>(win_kv);
+    a.win_start = win_start;
+    a.out = out;
+    a.lse = lse;
+    a.status = c.status;
+    a.req = req;
+    a.nent = nent;
+    a.ctiles = ctiles;
+    a.wlen = wlen;
+    a.tprefix = tprefix;
+    a.counters = counters;
+    a.Nq = Nq;
+    a.H = H;
+    a.cap = c.capacity;
+    a.topk = topk;
+    a.scale_log2 = softmax_scale * 1.4426950408889634f;
+
+    cudaError_t err = cudaMemsetAsync(counters, 0, 4 * (size_t)Nq, s);
+    if (err != cudaSuccess) return err;
+    attend_schedule_kernel<<<1, 1024, 0, s>>>(q_offsets, sel_idx ? nullptr : q_pos, c.n_blocks,
+                                              win_kv ? win_len : nullptr, c.batch, Nq, c.block, c.capacity, topk, max_win, H, D,
+                                              req, nent, ctiles, wlen, tprefix, out, lse, c.status);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    if (D == 512) {
+        const int smem = Cfg<512>::SMEM;
+        if ((err = cudaFuncSetAttribute(attend_kernel<512>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
+            return err;
+        attend_kernel<512><<<num_ctas, kThreads, smem, s>>>(a);
+    } else if (D == 128) {
+        const int smem = Cfg<128>::SMEM;
+        if ((err = cudaFuncSetAttribute(attend_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
+            return err;
+        attend_kernel<128><<<num_ctas, kThreads, smem, s>>>(a);
+    } else {
+        return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace csa

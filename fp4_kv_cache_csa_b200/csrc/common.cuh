@@ -1,0 +1,84 @@
+// common.cuh -- small device helpers shared by the libcsa kernels (sm_100a).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/csa.h"
+
+namespace csa {
+
+constexpr int kWarp = 32;
+
+__device__ __forceinline__ void flag(int32_t *status, int32_t bits) {
+    if (status) atomicOr(status, bits);
+}
+
+// Order-preserving map from float32 to uint32: a larger score gives a larger
+// key. -0 is folded into +0 first, so the two compare equal.
+__device__ __forceinline__ uint32_t ordered_key(float s) {
+    uint32_t u = __float_as_uint(s);
+    if (u == 0x80000000u) u = 0u;
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+// Index of the request that owns query i: the b with q_offsets[b] <= i < q_offsets[b+1]
+// (binary search; -1 when i is outside [q_offsets[0], q_offsets[batch])).
+__device__ __forceinline__ int request_of(const int32_t *q_offsets, int batch, int i) {
+    if (i < q_offsets[0] || i >= q_offsets[batch]) return -1;
+    int lo = 0, hi = batch - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (q_offsets[mid] <= i) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+// Blocks visible to a query at absolute position pos: causal at block
+// granularity and no more than the filled blocks.
+__device__ __forceinline__ int visible_blocks(int pos, int m, int filled) {
+    long long v = ((long long)pos + 1) / m;
+    if (v > filled) v = filled;
+    if (v < 0) v = 0;
+    return (int)v;
+}
+
+// Inclusive prefix sum over the threads of a block (blockDim.x multiple of 32).
+template <typename T>
+__device__ T block_inclusive_scan(T v, T *smem /* >= 32 entries */) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        T y = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += y;
+    }
+    if (lane == 31) smem[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        T s = lane < nw ? smem[lane] : T(0);
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            T y = __shfl_up_sync(0xffffffffu, s, o);
+            if (lane >= o) s += y;
+        }
+        if (lane < nw) smem[lane] = s;
+    }
+    __syncthreads();
+    if (warp > 0) v += smem[warp - 1];
+    __syncthreads();
+    return v;
+}
+
+}  // namespace csa

@@ -1,0 +1,268 @@
+// compress.cu -- rows a1 + a2: softmax-gated m-token pooling and MXFP4
+// quantization of the pooled entry, plus the pooled indexer key.
+//
+// Source: "Frontier Architecture Decoding Notes (4): DeepSeek V4", section 1
+// (KV of every 4 tokens compressed into one entry for CSA, up to 128 for HCA);
+// DeepSeek-V4.1-Flash podcast transcript, cue 16 (main KV stored as MXFP4,
+// E2M1 elements). Pooling form, gate and E8M0/32 scale: the library's stated
+// readings (see include/csa.h).
+//
+// One warp builds one block. Lane l owns E = D/32 consecutive channels
+// [l*E, l*E+E) and EI = dI/32 consecutive indexer channels, so every token row
+// is read as one coalesced warp-wide load. The gate softmax is computed online
+// (running max and rescaled sums) in a single pass over the m tokens. The
+// kernel is HBM-bound: it reads m*(D+dI)*2 bytes and writes D/2 + D/32 + key
+// bytes per block.
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+#include "common.cuh"
+
+namespace csa {
+
+namespace {
+
+constexpr int kWarpsPerCta = 4;
+
+// E2M1 code of a scaled value s (|s| < 8), round to nearest with ties to the
+// even code, saturating at 6; the sign bit is kept even when the magnitude
+// rounds to zero. Thresholds are the midpoints between neighbouring
+// magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6; "<=" sends a tie to the lower (even)
+// code, "<" sends it to the upper (even) code.
+__device__ __forceinline__ uint32_t e2m1_code(float s) {
+    uint32_t sign = (__float_as_uint(s) >> 28) & 8u;
+    float a = fabsf(s);
+    uint32_t c = a <= 0.25f ? 0u : a < 0.75f ? 1u : a <= 1.25f ? 2u : a < 1.75f ? 3u
+               : a <= 2.5f ? 4u : a < 3.5f ? 5u : a <= 5.0f ? 6u : 7u;
+    return sign | c;
+}
+
+template <int N>
+__device__ __forceinline__ void load_bf16(const __nv_bfloat16 *p, float (&x)[N]) {
+    static_assert(N % 2 == 0, "even channel count per lane");
+    if constexpr (N % 8 == 0) {
+#pragma unroll
+        for (int v = 0; v < N / 8; ++v) {
+            uint4 u = __ldg(reinterpret_cast<const uint4 *>(p) + v);
+            const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                float2 f = __bfloat1622float2(h[k]);
+                x[8 * v + 2 * k] = f.x;
+                x[8 * v + 2 * k + 1] = f.y;
+            }
+        }
+    } else if constexpr (N % 4 == 0) {
+#pragma unroll
+        for (int v = 0; v < N / 4; ++v) {
+            uint2 u = __ldg(reinterpret_cast<const uint2 *>(p) + v);
+            const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                float2 f = __bfloat1622float2(h[k]);
+                x[4 * v + 2 * k] = f.x;
+                x[4 * v + 2 * k + 1] = f.y;
+            }
+        }
+    } else {
+#pragma unroll
+        for (int v = 0; v < N / 2; ++v) {
+            float2 f = __bfloat1622float2(__ldg(reinterpret_cast<const __nv_bfloat162 *>(p) + v));
+            x[2 * v] = f.x;
+            x[2 * v + 1] = f.y;
+        }
+    }
+}
+
+struct CompressArgs {
+    const __nv_bfloat16 *kv_tok;   // [n_tokens][D]
+    const __nv_bfloat16 *idx_tok;  // [n_tokens][dI] or null
+    const float *gate_w;           // [D]
+    const int32_t *tok_offsets;    // [B+1]
+    const int32_t *n_blocks;       // [B]
+    uint8_t *fp4;                  // [B][cap][D/2]
+    uint8_t *scale;                // [B][cap][D/32]
+    uint8_t *idx_key;              // [B][cap][dI * esize] or null
+    int32_t *status;
+    int m, cap, D, dI;
+    int idx_e4m3;
+};
+
+// E channels per lane (D = 32*E), EI indexer channels per lane (0 = no indexer keys).
+template <int E, int EI>
+__global__ void __launch_bounds__(kWarpsPerCta * kWarp)
+pool_quantize_kernel(CompressArgs a) {
+    const int lane = threadIdx.x & 31;
+    const int b = blockIdx.y;
+    const int jb = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
+    const int t_begin = a.tok_offsets[b];
+    const int count = a.tok_offsets[b + 1] - t_begin;
+    const int base = a.n_blocks[b];
+    if (count < 0 || count % a.m != 0) {
+        if (jb == 0 && lane == 0) flag(a.status, CSA_DEV_TOKEN_COUNT);
+        return;
+    }
+    const int nb = count / a.m;
+    if ((long long)base + nb > a.cap) {
+        if (jb == 0 && lane == 0) flag(a.status, CSA_DEV_CAPACITY);
+        return;
+    }
+    if (jb >= nb) return;
+
+    float wg[E];
+#pragma unroll
+    for (int k = 0; k < E; ++k) wg[k] = __ldg(a.gate_w + lane * E + k);
+
+    // Online softmax over the block's tokens: mu = running max logit,
+    // den = sum exp(g - mu), acc = sum exp(g - mu) * x.
+    float acc[E], acck[EI > 0 ? EI : 1];
+    float mu = -INFINITY, den = 0.f;
+#pragma unroll
+    for (int k = 0; k < E; ++k) acc[k] = 0.f;
+#pragma unroll
+    for (int k = 0; k < (EI > 0 ? EI : 1); ++k) acck[k] = 0.f;
+
+    const long long tok0 = (long long)t_begin + (long long)jb * a.m;
+    for (int t = 0; t < a.m; ++t) {
+        float x[E];
+        load_bf16<E>(a.kv_tok + (tok0 + t) * a.D + lane * E, x);
+        float part = 0.f;
+#pragma unroll
+        for (int k = 0; k < E; ++k) part = fmaf(x[k], wg[k], part);
+        const float g = warp_sum(part);
+        float xk[EI > 0 ? EI : 2];
+        if constexpr (EI > 0) load_bf16<EI>(a.idx_tok + (tok0 + t) * a.dI + lane * EI, xk);
+        if (g > mu) {  // new maximum: rescale what has been accumulated
+            const float r = (mu == -INFINITY) ? 0.f : expf(mu - g);
+            den *= r;
+#pragma unroll
+            for (int k = 0; k < E; ++k) acc[k] *= r;
+            if constexpr (EI > 0) {
+#pragma unroll
+                for (int k = 0; k < EI; ++k) acck[k] *= r;
+            }
+            mu = g;
+        }
+        const float p = expf(g - mu);
+        den += p;
+#pragma unroll
+        for (int k = 0; k < E; ++k) acc[k] = fmaf(p, x[k], acc[k]);
+        if constexpr (EI > 0) {
+#pragma unroll
+            for (int k = 0; k < EI; ++k) acck[k] = fmaf(p, xk[k], acck[k]);
+        }
+    }
+
+    const size_t row = (size_t)b * a.cap + base + jb;
+    // ---- main entry -> MXFP4 ----
+    float e[E];
+    float amax = 0.f;
+#pragma unroll
+    for (int k = 0; k < E; ++k) {
+        e[k] = acc[k] / den;
+        amax = fmaxf(amax, fabsf(e[k]));
+    }
+    // a 32-element group spans 32/E lanes
+#pragma unroll
+    for (int o = 1; o < 32 / E; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    // X = floor(log2 amax) - 2 from the exponent field, clamped to >= -127
+    // (zero and subnormal amax land on the clamp); byte = X + 127.
+    const int expbits = (int)((__float_as_uint(amax) >> 23) & 0xFF);
+    const int sbyte = max(expbits - 2, 0);
+    const float inv = __uint_as_float((uint32_t)(254 - sbyte) << 23);  // 2^-X, X = sbyte-127
+    uint32_t packed[E / 2 > 0 ? E / 2 : 1];
+#pragma unroll
+    for (int k = 0; k < E; k += 2)
+        packed[k / 2] = e2m1_code(e[k] * inv) | (e2m1_code(e[k + 1] * inv) << 4);
+    uint8_t *dst = a.fp4 + row * (a.D / 2) + lane * (E / 2);
+    if constexpr (E == 16) {
+        uint2 w;
+        w.x = packed[0] | (packed[1] << 8) | (packed[2] << 16) | (packed[3] << 24);
+        w.y = packed[4] | (packed[5] << 8) | (packed[6] << 16) | (packed[7] << 24);
+        *reinterpret_cast<uint2 *>(dst) = w;
+    } else if constexpr (E == 8) {
+        *reinterpret_cast<uint32_t *>(dst) = packed[0] | (packed[1] << 8) | (packed[2] << 16) | (packed[3] << 24);
+    } else if constexpr (E == 4) {
+        *reinterpret_cast<uint16_t *>(dst) = (uint16_t)(packed[0] | (packed[1] << 8));
+    } else {
+        dst[0] = (uint8_t)packed[0];
+    }
+    if (lane % (32 / E) == 0) a.scale[row * (a.D / 32) + lane / (32 / E)] = (uint8_t)sbyte;
+
+    // ---- pooled indexer key -> bf16 or e4m3 ----
+    if constexpr (EI > 0) {
+        if (a.idx_e4m3) {
+            uint8_t *kd = a.idx_key + row * a.dI + lane * EI;
+#pragma unroll
+            for (int k = 0; k < EI; ++k)
+                kd[k] = (uint8_t)__nv_cvt_float_to_fp8(acck[k] / den, __NV_SATFINITE, __NV_E4M3);
+        } else {
+            __nv_bfloat16 *kd = reinterpret_cast<__nv_bfloat16 *>(a.idx_key + row * a.dI * 2) + lane * EI;
+#pragma unroll
+            for (int k = 0; k < EI; ++k) kd[k] = __float2bfloat16_rn(acck[k] / den);
+        }
+    }
+}
+
+// Advance n_blocks after the pooling kernel has read the old values; applies
+// the same checks, so a rejected request is left untouched.
+__global__ void commit_kernel(const int32_t *tok_offsets, int32_t *n_blocks, int batch, int m, int cap) {
+    for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < batch; b += gridDim.x * blockDim.x) {
+        const int count = tok_offsets[b + 1] - tok_offsets[b];
+        if (count < 0 || count % m != 0) continue;
+        if ((long long)n_blocks[b] + count / m > cap) continue;
+        n_blocks[b] += count / m;
+    }
+}
+
+template <int E>
+cudaError_t launch_e(const CompressArgs &a, dim3 grid, cudaStream_t s) {
+    const dim3 block(kWarpsPerCta * kWarp);
+    switch (a.idx_key ? a.dI / 32 : 0) {
+        case 0: pool_quantize_kernel<E, 0><<<grid, block, 0, s>>>(a); break;
+        case 2: pool_quantize_kernel<E, 2><<<grid, block, 0, s>>>(a); break;
+        case 4: pool_quantize_kernel<E, 4><<<grid, block, 0, s>>>(a); break;
+        case 8: pool_quantize_kernel<E, 8><<<grid, block, 0, s>>>(a); break;
+        default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+// Host launcher; arguments already validated by the C-ABI layer.
+cudaError_t launch_compress(const csa_cache &c, const void *kv_tok, const void *idx_tok, const float *gate_w,
+                            const int32_t *tok_offsets, int32_t n_tokens, cudaStream_t s) {
+    CompressArgs a;
+    a.kv_tok = static_cast<const __nv_bfloat16 *>(kv_tok);
+    a.idx_tok = static_cast<const __nv_bfloat16 *>(idx_tok);
+    a.gate_w = gate_w;
+    a.tok_offsets = tok_offsets;
+    a.n_blocks = c.n_blocks;
+    a.fp4 = c.fp4;
+    a.scale = c.scale;
+    a.idx_key = static_cast<uint8_t *>(c.idx_key);
+    a.status = c.status;
+    a.m = c.block;
+    a.cap = c.capacity;
+    a.D = c.dim;
+    a.dI = c.idx_key ? c.idx_dim : 0;
+    a.idx_e4m3 = c.idx_dtype == CSA_IDX_E4M3;
+    const int max_blocks = (n_tokens + c.block - 1) / c.block;
+    if (max_blocks > 0) {
+        dim3 grid((max_blocks + kWarpsPerCta - 1) / kWarpsPerCta, c.batch);
+        cudaError_t err;
+        switch (c.dim / 32) {
+            case 2: err = launch_e<2>(a, grid, s); break;
+            case 4: err = launch_e<4>(a, grid, s); break;
+            case 8: err = launch_e<8>(a, grid, s); break;
+            case 16: err = launch_e<16>(a, grid, s); break;
+            default: return cudaErrorInvalidValue;
+        }
+        if (err != cudaSuccess) return err;
+    }
+    commit_kernel<<<(c.batch + 255) / 256, 256, 0, s>>>(tok_offsets, c.n_blocks, c.batch, c.block, c.capacity);
+    return cudaGetLastError();
+}
+
+}  // namespace csa

@@ -1,0 +1,620 @@
+// indexer.cu -- rows a3 + a4: indexer scoring of every visible compressed
+// block and per-query top-k block selection.
+//
+// Source: DeepSeek-V4.1-Flash podcast transcript, cue 12 (an indexer query
+// scores the indexer keys projected from the main KV; the top-k selection is
+// attended); "Frontier Architecture Decoding Notes (4): DeepSeek V4",
+// section 1 ("top-k over blocks"). Score form and tie rule: the library's
+// stated readings, s_j = sum_h w_h * ReLU(q_h . k_j), ties to the lower j.
+//
+// Kernels, in launch order (one stream):
+//   schedule_kernel   per query: owning request, visible block count n_vis,
+//                     prefix over queries of ceil(n_vis/16) key groups.
+//   scan_kernel       streams every visible key exactly once (the dominant HBM
+//                     traffic at long context). The flat list of 16-key groups
+//                     is cut into equal contiguous ranges, one per CTA, so
+//                     ragged contexts stay balanced. Each warp turns 16 keys x
+//                     d_I into tensor-core A fragments straight from its
+//                     coalesced 128-bit loads (no shared-memory staging) and
+//                     multiplies them by the query's H_I x d_I indexer matrix
+//                     (mma.sync m16n8k16, fp32 accumulation; heads padded to 8).
+//                     The per-key contraction is tiny (H_I = 4 outputs), so the
+//                     tensor core only relieves the FP32 pipe: the kernel stays
+//                     bound by HBM. It writes the fp32 score of every key and a
+//                     4096-bin histogram of the top 12 bits of each score's
+//                     order-preserving key.
+//   select_pass_kernel  many CTAs per query: from the histogram, the bin b*
+//                     holding the k-th largest score; marks every key above b*
+//                     in a per-query bitmap and appends the keys inside b* to a
+//                     candidate list, with a histogram of their next 12 bits.
+//   select_final_kernel one CTA per query: radix refinement among the
+//                     candidates (remaining score bits, then the block index
+//                     for exact ties, lower index first), then the bitmap is
+//                     compacted into ascending block indices padded with -1.
+// Every float comparison is on the score's order-preserving uint32 key
+// (-0 folded into +0), so selection is exact for the scores computed here.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
+#include "common.cuh"
+
+namespace csa {
+
+namespace {
+
+constexpr int kBins = 4096;        // histogram bins per level (12 bits)
+constexpr int kScanThreads = 256;  // 8 warps
+constexpr int kSelThreads = 1024;
+constexpr int kPassSlices = 16;    // CTAs per query in select_pass_kernel
+
+// ---------------------------------------------------------------- workspace
+struct IndexWs {
+    int32_t *req;        // [Nq]
+    int32_t *n_vis;      // [Nq]
+    long long *gprefix;  // [Nq+1]
+    // zeroed region starts here
+    uint32_t *hist1;     // [Nq][4096]
+    uint32_t *hist2;     // [Nq][4096]
+    uint32_t *bitmap;    // [Nq][words]
+    uint32_t *ncand;     // [Nq]
+    // end of zeroed region
+    uint32_t *cand_key;  // [Nq][ccap]
+    int32_t *cand_idx;   // [Nq][ccap]
+    float *scores;       // [Nq][cap]
+    size_t zero_bytes;
+    int words, ccap;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+size_t carve(void *base, int Nq, int cap, IndexWs *w) {
+    const int words = (cap + 31) / 32;
+    const int ccap = 32768;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        size_t o = off;
+        off = align256(off + bytes);
+        return o;
+    };
+    size_t o_req = take(sizeof(int32_t) * Nq);
+    size_t o_nvis = take(sizeof(int32_t) * Nq);
+    size_t o_gp = take(sizeof(long long) * (Nq + 1));
+    size_t z0 = off;
+    size_t o_h1 = take(sizeof(uint32_t) * kBins * (size_t)Nq);
+    size_t o_h2 = take(sizeof(uint32_t) * kBins * (size_t)Nq);
+    size_t o_bm = take(sizeof(uint32_t) * (size_t)words * Nq);
+    size_t o_nc = take(sizeof(uint32_t) * Nq);
+    size_t z1 = off;
+    size_t o_ck = take(sizeof(uint32_t) * (size_t)ccap * Nq);
+    size_t o_ci = take(sizeof(int32_t) * (size_t)ccap * Nq);
+    size_t o_sc = take(sizeof(float) * (size_t)cap * Nq);
+    if (w) {
+        char *b = static_cast<char *>(base);
+        w->req = reinterpret_cast<int32_t *>(b + o_req);
+        w->n_vis = reinterpret_cast<int32_t *>(b + o_nvis);
+        w->gprefix = reinterpret_cast<long long *>(b + o_gp);
+        w->hist1 = reinterpret_cast<uint32_t *>(b + o_h1);
+        w->hist2 = reinterpret_cast<uint32_t *>(b + o_h2);
+        w->bitmap = reinterpret_cast<uint32_t *>(b + o_bm);
+        w->ncand = reinterpret_cast<uint32_t *>(b + o_nc);
+        w->cand_key = reinterpret_cast<uint32_t *>(b + o_ck);
+        w->cand_idx = reinterpret_cast<int32_t *>(b + o_ci);
+        w->scores = reinterpret_cast<float *>(b + o_sc);
+        w->zero_bytes = z1 - z0;
+        w->words = words;
+        w->ccap = ccap;
+    }
+    return off;
+}
+
+// ---------------------------------------------------------------- schedule
+__global__ void schedule_kernel(const int32_t *q_offsets, const int32_t *q_pos, const int32_t *n_blocks,
+                                int batch, int Nq, int m, int cap, int32_t *req, int32_t *n_vis, long long *gprefix) {
+    __shared__ long long red[32];
+    __shared__ long long round_total;
+    long long carry = 0;
+    for (int base = 0; base < Nq; base += blockDim.x) {
+        const int i = base + threadIdx.x;
+        long long groups = 0;
+        if (i < Nq) {
+            const int b = request_of(q_offsets, batch, i);
+            const int n = (b < 0) ? 0 : min(visible_blocks(q_pos[i], m, n_blocks[b]), cap);
+            req[i] = b;
+            n_vis[i] = n;
+            groups = (n + 15) / 16;
+        }
+        const long long incl = block_inclusive_scan<long long>(groups, red);
+        if (i < Nq) gprefix[i + 1] = carry + incl;
+        if (i == 0) gprefix[0] = 0;
+        // total of this round, from the last thread
+        if (threadIdx.x == blockDim.x - 1) round_total = incl;
+        __syncthreads();
+        carry += round_total;
+        __syncthreads();
+    }
+}
+
+// ---------------------------------------------------------------- scan
+__device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Two E4M3 bytes (low byte first) -> packed f16x2 (exact: E4M3 is a subset of f16).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_bytes) {
+    __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two_bytes & 0xFFFFu), __NV_E4M3);
+    return (uint32_t)h.x | ((uint32_t)h.y << 16);
+}
+
+struct ScanArgs {
+    const uint8_t *keys;          // [B][cap][dI*esize]
+    const __nv_bfloat16 *q_idx;   // [Nq][H_I][dI]
+    const float *w;               // [Nq][H_I]
+    const int32_t *req, *n_vis;
+    const long long *gprefix;
+    float *scores;                // [Nq][cap]
+    uint32_t *hist1;              // [Nq][4096]
+    int Nq, H_I, cap;
+};
+
+// Dimension permutation. The dot product sums over all d_I channels, so the
+// channels may be fed to the MMA in any order as long as keys and query use
+// the same one. Thread t of a quad owns the contiguous channels
+// [t*EPT, (t+1)*EPT) of its key rows (EPT = d_I/4) and uses channels
+// t*EPT + 4s + {0,1} as MMA k-columns 2t,2t+1 and t*EPT + 4s + {2,3} as
+// columns 2t+8,2t+9 of k-step s. The query's B fragment uses the identical
+// map, so each thread reads one contiguous stretch of every row.
+template <bool E4M3, int KS>
+struct ScanCfg {
+    static constexpr int EPT = 4 * KS;                   // channels per thread per row
+    static constexpr int ROW_BYTES_T = EPT * (E4M3 ? 1 : 2);
+    static constexpr int NV = ROW_BYTES_T / 16;          // uint4 loads per thread per row
+    static constexpr int KEY_BYTES = 4 * ROW_BYTES_T;    // bytes per key row
+    static constexpr int U = (16 / (2 * NV)) > 0 ? 16 / (2 * NV) : 1;  // groups in flight per warp
+};
+
+template <bool E4M3, int KS>
+__global__ void __launch_bounds__(kScanThreads, 2) scan_kernel(ScanArgs a) {
+    using C = ScanCfg<E4M3, KS>;
+    __shared__ uint32_t hist[kBins];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    const long long NG = a.gprefix[a.Nq];
+    long long gb = NG * blockIdx.x / gridDim.x;
+    const long long ge = NG * (blockIdx.x + 1) / gridDim.x;
+
+    while (gb < ge) {
+        // query that owns group gb
+        int lo = 0, hi = a.Nq - 1;
+        while (lo < hi) {
+            int mid = (lo + hi + 1) >> 1;
+            if (a.gprefix[mid] <= gb) lo = mid; else hi = mid - 1;
+        }
+        const int i = lo;
+        const long long seg_end = min(ge, a.gprefix[i + 1]);
+        const int b = a.req[i];
+        const int n = a.n_vis[i];
+
+        // ---- query fragments: B[k][n=head] with the dimension permutation ----
+        uint32_t bq[KS][2];
+        float w_lo = 0.f, w_hi = 0.f;  // weights of heads 2t and 2t+1 (scaled, see below)
+        {
+            float qv[C::EPT];
+            const bool live = g < a.H_I;
+#pragma unroll
+            for (int k = 0; k < C::EPT; ++k) qv[k] = 0.f;
+            if (live) {
+                const __nv_bfloat16 *qp = a.q_idx + ((size_t)i * a.H_I + g) * (C::EPT * 4) + t * C::EPT;
+#pragma unroll
+                for (int v = 0; v < C::EPT / 8; ++v) {
+                    uint4 u = __ldg(reinterpret_cast<const uint4 *>(qp) + v);
+                    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        float2 f = __bfloat1622float2(h[k]);
+                        qv[8 * v + 2 * k] = f.x;
+                        qv[8 * v + 2 * k + 1] = f.y;
+                    }
+                }
+            }
+            int kexp = 0;  // power-of-two scale of this head's query (fp16 path only)
+            if constexpr (E4M3) {
+                // fp16 operands: scale head h's query by 2^k_h so its largest
+                // magnitude lands in [2^14, 2^15); every bf16 value within 2^31
+                // of it converts exactly. ReLU(2^k x) = 2^k ReLU(x), so the
+                // head weight carries 2^-k_h and the score is unchanged.
+                float mx = 0.f;
+#pragma unroll
+                for (int k = 0; k < C::EPT; ++k) mx = fmaxf(mx, fabsf(qv[k]));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                const int e = (int)((__float_as_uint(mx) >> 23) & 0xFF) - 127;
+                kexp = (mx > 0.f) ? min(14 - e, 126) : 0;
+                const float sc = ldexpf(1.0f, kexp);
+#pragma unroll
+                for (int s = 0; s < KS; ++s) {
+                    __half2 h0 = __floats2half2_rn(qv[4 * s] * sc, qv[4 * s + 1] * sc);
+                    __half2 h1 = __floats2half2_rn(qv[4 * s + 2] * sc, qv[4 * s + 3] * sc);
+                    bq[s][0] = *reinterpret_cast<uint32_t *>(&h0);
+                    bq[s][1] = *reinterpret_cast<uint32_t *>(&h1);
+                }
+            } else {
+#pragma unroll
+                for (int s = 0; s < KS; ++s) {
+                    __nv_bfloat162 h0 = __floats2bfloat162_rn(qv[4 * s], qv[4 * s + 1]);
+                    __nv_bfloat162 h1 = __floats2bfloat162_rn(qv[4 * s + 2], qv[4 * s + 3]);
+                    bq[s][0] = *reinterpret_cast<uint32_t *>(&h0);
+                    bq[s][1] = *reinterpret_cast<uint32_t *>(&h1);
+                }
+            }
+            const int h0 = 2 * t, h1 = 2 * t + 1;
+            const int k0 = __shfl_sync(0xffffffffu, kexp, (4 * h0) & 31);
+            const int k1 = __shfl_sync(0xffffffffu, kexp, (4 * h1) & 31);
+            if (h0 < a.H_I) w_lo = ldexpf(a.w[(size_t)i * a.H_I + h0], -k0);
+            if (h1 < a.H_I) w_hi = ldexpf(a.w[(size_t)i * a.H_I + h1], -k1);
+        }
+
+        for (int k = threadIdx.x; k < kBins; k += kScanThreads) hist[k] = 0;
+        __syncthreads();
+
+        const uint8_t *kbase = a.keys + (size_t)b * a.cap * C::KEY_BYTES;
+        float *srow = a.scores + (size_t)i * a.cap;
+        const long long lg0 = gb - a.gprefix[i];   // local group index of gb
+        const long long nloc = seg_end - gb;        // groups of this query in this CTA
+
+        for (long long u0 = warp; u0 < nloc; u0 += 8LL * C::U) {
+            uint4 raw[C::U][2][C::NV];
+#pragma unroll
+            for (int uu = 0; uu < C::U; ++uu) {
+                const long long lg = lg0 + u0 + 8LL * uu;
+                const bool gv = (u0 + 8LL * uu) < nloc;
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    const long long r = 16 * lg + g + 8 * half;
+                    const bool ok = gv && r < n;
+                    const uint4 *src = reinterpret_cast<const uint4 *>(kbase + r * C::KEY_BYTES + t * C::ROW_BYTES_T);
+#pragma unroll
+                    for (int v = 0; v < C::NV; ++v) raw[uu][half][v] = ok ? __ldg(src + v) : make_uint4(0, 0, 0, 0);
+                }
+            }
+#pragma unroll
+            for (int uu = 0; uu < C::U; ++uu) {
+                const long long lg = lg0 + u0 + 8LL * uu;
+                const bool gv = (u0 + 8LL * uu) < nloc;
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                const uint32_t *w0 = reinterpret_cast<const uint32_t *>(raw[uu][0]);
+                const uint32_t *w1 = reinterpret_cast<const uint32_t *>(raw[uu][1]);
+#pragma unroll
+                for (int s = 0; s < KS; ++s) {
+                    uint32_t af[4];
+                    if constexpr (E4M3) {
+                        af[0] = e4m3x2_to_f16x2(w0[s]);          // row g,   cols 2t,2t+1
+                        af[1] = e4m3x2_to_f16x2(w1[s]);          // row g+8, cols 2t,2t+1
+                        af[2] = e4m3x2_to_f16x2(w0[s] >> 16);    // row g,   cols 2t+8,2t+9
+                        af[3] = e4m3x2_to_f16x2(w1[s] >> 16);    // row g+8, cols 2t+8,2t+9
+                        mma_f16(acc, af, bq[s][0], bq[s][1]);
+                    } else {
+                        af[0] = w0[2 * s];
+                        af[1] = w1[2 * s];
+                        af[2] = w0[2 * s + 1];
+                        af[3] = w1[2 * s + 1];
+                        mma_bf16(acc, af, bq[s][0], bq[s][1]);
+                    }
+                }
+                // acc[0..1]: row g, heads 2t,2t+1; acc[2..3]: row g+8
+                float p0 = w_lo * fmaxf(acc[0], 0.f) + w_hi * fmaxf(acc[1], 0.f);
+                float p1 = w_lo * fmaxf(acc[2], 0.f) + w_hi * fmaxf(acc[3], 0.f);
+                p0 += __shfl_xor_sync(0xffffffffu, p0, 1);
+                p1 += __shfl_xor_sync(0xffffffffu, p1, 1);
+                p0 += __shfl_xor_sync(0xffffffffu, p0, 2);
+                p1 += __shfl_xor_sync(0xffffffffu, p1, 2);
+                if (gv && t < 2) {
+                    const long long r = 16 * lg + g + 8 * t;
+                    const float sc = t == 0 ? p0 : p1;
+                    if (r < n) {
+                        srow[r] = sc;
+                        atomicAdd(&hist[ordered_key(sc) >> 20], 1u);
+                    }
+                }
+            }
+        }
+        __syncthreads();
+        uint32_t *gh = a.hist1 + (size_t)i * kBins;
+        const volatile uint32_t *vh = hist;
+        for (int k = threadIdx.x; k < kBins; k += kScanThreads) {
+            const uint32_t c = vh[k];
+            if (c) atomicAdd(gh + k, c);
+        }
+        __syncthreads();
+        gb = seg_end;
+    }
+}
+
+// ---------------------------------------------------------------- select
+struct SelArgs {
+    const int32_t *n_vis;
+    const float *scores;
+    uint32_t *hist1, *hist2, *bitmap, *ncand, *cand_key;
+    int32_t *cand_idx;
+    int32_t *sel_idx;
+    int Nq, cap, topk, words, ccap;
+};
+
+struct BinPick {
+    int bin;          // chosen digit
+    uint32_t above;   // elements with a larger digit
+    uint32_t at;      // elements with this digit
+};
+
+// Largest digit d such that count(digit >= d) >= need, in a histogram of
+// nbins (<= 4096) bins held in shared memory. All threads get the result.
+__device__ BinPick pick_bin(const uint32_t *h, int nbins, uint32_t need, uint32_t *scan_smem, BinPick *out) {
+    const int per = (nbins + blockDim.x - 1) / blockDim.x;
+    // thread t owns bins [base, base+per) counted from the top
+    const int rt = threadIdx.x;  // rank from the top
+    const int top = nbins - 1 - rt * per;
+    uint32_t mine = 0;
+    for (int k = 0; k < per; ++k)
+        if (top - k >= 0) mine += h[top - k];
+    const uint32_t incl = block_inclusive_scan<uint32_t>(mine, scan_smem);
+    const uint32_t excl = incl - mine;
+    if (excl < need && incl >= need) {
+        uint32_t run = excl;
+        for (int k = 0; k < per; ++k) {
+            const int d = top - k;
+            if (d < 0) break;
+            if (run + h[d] >= need) {
+                out->bin = d;
+                out->above = run;
+                out->at = h[d];
+                break;
+            }
+            run += h[d];
+        }
+    }
+    __syncthreads();
+    BinPick r = *out;
+    __syncthreads();
+    return r;
+}
+
+__device__ __forceinline__ void mark(uint32_t *bm, int j) { atomicOr(bm + (j >> 5), 1u << (j & 31)); }
+
+__global__ void __launch_bounds__(kSelThreads) select_pass_kernel(SelArgs a) {
+    __shared__ uint32_t h[kBins];
+    __shared__ uint32_t h2[kBins];
+    __shared__ uint32_t scan_smem[32];
+    __shared__ BinPick pick;
+    const int i = blockIdx.y;
+    const int n = a.n_vis[i];
+    const int K = min(a.topk, n);
+    if (K == n) return;  // everything visible is selected; the final kernel handles it
+    for (int k = threadIdx.x; k < kBins; k += blockDim.x) {
+        h[k] = a.hist1[(size_t)i * kBins + k];
+        h2[k] = 0;
+    }
+    __syncthreads();
+    const BinPick p = pick_bin(h, kBins, (uint32_t)K, scan_smem, &pick);
+    const bool take_all_at = (p.above + p.at == (uint32_t)K);
+    uint32_t *bm = a.bitmap + (size_t)i * a.words;
+    const float *s = a.scores + (size_t)i * a.cap;
+    // slice of the row handled by this CTA
+    const int per = (n + gridDim.x - 1) / gridDim.x;
+    const int j0 = blockIdx.x * per, j1 = min(n, j0 + per);
+    for (int j = j0 + threadIdx.x; j < j1; j += blockDim.x) {
+        const uint32_t key = ordered_key(s[j]);
+        const int d = (int)(key >> 20);
+        if (d > p.bin || (d == p.bin && take_all_at)) {
+            mark(bm, j);
+        } else if (d == p.bin) {
+            atomicAdd(&h2[(key >> 8) & 0xFFF], 1u);
+            const uint32_t pos = atomicAdd(a.ncand + i, 1u);
+            if (pos < (uint32_t)a.ccap) {
+                a.cand_key[(size_t)i * a.ccap + pos] = key;
+                a.cand_idx[(size_t)i * a.ccap + pos] = j;
+            }
+        }
+    }
+    __syncthreads();
+    if (!take_all_at) {
+        const volatile uint32_t *vh2 = h2;
+        for (int k = threadIdx.x; k < kBins; k += blockDim.x) {
+            const uint32_t c = vh2[k];
+            if (c) atomicAdd(a.hist2 + (size_t)i * kBins + k, c);
+        }
+    }
+}
+
+// Digits of the refinement levels after the first (key bits 31..20):
+//   level 1: key bits 19..8   level 2: key bits 7..0
+//   level 3: 4095 - block index bits 19..8   level 4: 255 - block index bits 7..0
+// (the block-index digits are reversed so that "largest digit first" takes the
+// lower index first). The prefix of a level is the digits of all earlier ones.
+__device__ __forceinline__ int level_digit(int level, uint32_t key, int j) {
+    switch (level) {
+        case 1: return (int)((key >> 8) & 0xFFF);
+        case 2: return (int)(key & 0xFF);
+        case 3: return 4095 - ((j >> 8) & 0xFFF);
+        default: return 255 - (j & 0xFF);
+    }
+}
+__device__ __forceinline__ int level_bins(int level) { return (level == 1 || level == 3) ? 4096 : 256; }
+
+__global__ void __launch_bounds__(kSelThreads) select_final_kernel(SelArgs a) {
+    extern __shared__ uint32_t dyn[];
+    uint32_t *bm = dyn;                  // [words]
+    __shared__ uint32_t h[kBins];
+    __shared__ uint32_t hn[kBins];
+    __shared__ uint32_t scan_smem[32];
+    __shared__ BinPick pick;
+    __shared__ int prefix_digit[5];
+    const int i = blockIdx.x;
+    const int n = a.n_vis[i];
+    const int K = min(a.topk, n);
+    int32_t *out = a.sel_idx + (size_t)i * a.topk;
+    const int words = (n + 31) / 32;
+
+    if (K == n) {  // select every visible block
+        for (int r = threadIdx.x; r < a.topk; r += blockDim.x) out[r] = r < n ? r : -1;
+        return;
+    }
+    const uint32_t *gbm = a.bitmap + (size_t)i * a.words;
+    for (int w = threadIdx.x; w < words; w += blockDim.x) bm[w] = gbm[w];
+    for (int k = threadIdx.x; k < kBins; k += blockDim.x) h[k] = a.hist1[(size_t)i * kBins + k];
+    __syncthreads();
+    const BinPick p1 = pick_bin(h, kBins, (uint32_t)K, scan_smem, &pick);
+    uint32_t need = (uint32_t)K - p1.above;
+    if (p1.above + p1.at != (uint32_t)K) {
+        // refine inside bin p1.bin
+        const uint32_t nc = a.ncand[i];
+        const bool in_list = nc <= (uint32_t)a.ccap;
+        const uint32_t *ck = a.cand_key + (size_t)i * a.ccap;
+        const int32_t *cj = a.cand_idx + (size_t)i * a.ccap;
+        const float *s = a.scores + (size_t)i * a.cap;
+        for (int k = threadIdx.x; k < kBins; k += blockDim.x) h[k] = a.hist2[(size_t)i * kBins + k];
+        if (threadIdx.x == 0) prefix_digit[0] = p1.bin;
+        __syncthreads();
+        for (int level = 1; level <= 4; ++level) {
+            const int nb = level_bins(level);
+            const BinPick p = pick_bin(h, nb, need, scan_smem, &pick);
+            if (threadIdx.x == 0) prefix_digit[level] = p.bin;
+            const bool done = (p.above + p.at == need);
+            for (int k = threadIdx.x; k < kBins; k += blockDim.x) hn[k] = 0;
+            __syncthreads();
+            // one pass over the elements that share all earlier digits
+            auto visit = [&](uint32_t key, int j) {
+                if ((int)(key >> 20) != prefix_digit[0]) return;
+                for (int l = 1; l < level; ++l)
+                    if (level_digit(l, key, j) != prefix_digit[l]) return;
+                const int d = level_digit(level, key, j);
+                if (d > p.bin || (d == p.bin && done)) mark(bm, j);
+                else if (d == p.bin && level < 4) atomicAdd(&hn[level_digit(level + 1, key, j)], 1u);
+            };
+            if (in_list) {
+                for (uint32_t c = threadIdx.x; c < nc; c += blockDim.x) visit(ck[c], cj[c]);
+            } else {
+                for (int j = threadIdx.x; j < n; j += blockDim.x) visit(ordered_key(s[j]), j);
+            }
+            __syncthreads();
+            if (done) break;
+            need -= p.above;
+            const volatile uint32_t *vhn = hn;
+            for (int k = threadIdx.x; k < kBins; k += blockDim.x) h[k] = vhn[k];
+            __syncthreads();
+        }
+    }
+    __syncthreads();
+    // ---- compaction: bitmap -> ascending block indices ----
+    // Rounds of blockDim.x words; each word is read once (through a volatile
+    // view, after the barrier that ends the marking) and that single value
+    // gives both the thread's count and the indices it writes.
+    __shared__ uint32_t round_total;
+    const volatile uint32_t *vbm = bm;
+    uint32_t base = 0;
+    for (int wr = 0; wr < words; wr += blockDim.x) {
+        const int w = wr + threadIdx.x;
+        uint32_t bits = 0;
+        if (w < words) {
+            bits = vbm[w];
+            if (w == words - 1 && (n & 31)) bits &= (1u << (n & 31)) - 1u;
+        }
+        const uint32_t cnt = __popc(bits);
+        const uint32_t incl = block_inclusive_scan<uint32_t>(cnt, scan_smem);
+        uint32_t pos = base + incl - cnt;
+        while (bits) {
+            const int bit = __ffs(bits) - 1;
+            bits &= bits - 1;
+            if (pos < (uint32_t)a.topk) out[pos] = w * 32 + bit;
+            ++pos;
+        }
+        if (threadIdx.x == blockDim.x - 1) round_total = incl;
+        __syncthreads();
+        base += round_total;
+        __syncthreads();
+    }
+    // total selected = K by construction; pad the rest
+    for (int r = K + threadIdx.x; r < a.topk; r += blockDim.x) out[r] = -1;
+}
+
+template <bool E4M3, int KS>
+cudaError_t launch_scan(const ScanArgs &sa, int grid, cudaStream_t s) {
+    scan_kernel<E4M3, KS><<<grid, kScanThreads, 0, s>>>(sa);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t index_topk_workspace_bytes(int Nq, int cap) { return carve(nullptr, Nq, cap, nullptr); }
+
+int index_select_smem_bytes(int cap) { return ((cap + 31) / 32) * 4; }
+
+cudaError_t launch_index_topk(const csa_cache &c, const void *q_idx, const float *w, int Nq, int H_I,
+                              const int32_t *q_offsets, const int32_t *q_pos, int topk, int32_t *sel_idx,
+                              void *workspace, int num_sms, cudaStream_t s) {
+    IndexWs ws;
+    carve(workspace, Nq, c.capacity, &ws);
+    cudaError_t err = cudaMemsetAsync(ws.hist1, 0, ws.zero_bytes, s);
+    if (err != cudaSuccess) return err;
+    schedule_kernel<<<1, 1024, 0, s>>>(q_offsets, q_pos, c.n_blocks, c.batch, Nq, c.block, c.capacity, ws.req, ws.n_vis,
+                                       ws.gprefix);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+
+    ScanArgs sa;
+    sa.keys = static_cast<const uint8_t *>(c.idx_key);
+    sa.q_idx = static_cast<const __nv_bfloat16 *>(q_idx);
+    sa.w = w;
+    sa.req = ws.req;
+    sa.n_vis = ws.n_vis;
+    sa.gprefix = ws.gprefix;
+    sa.scores = ws.scores;
+    sa.hist1 = ws.hist1;
+    sa.Nq = Nq;
+    sa.H_I = H_I;
+    sa.cap = c.capacity;
+    const int grid = num_sms * 2;
+    const bool e4 = c.idx_dtype == CSA_IDX_E4M3;
+    switch (c.idx_dim / 16) {
+        case 4: err = e4 ? launch_scan<true, 4>(sa, grid, s) : launch_scan<false, 4>(sa, grid, s); break;
+        case 8: err = e4 ? launch_scan<true, 8>(sa, grid, s) : launch_scan<false, 8>(sa, grid, s); break;
+        case 16: err = e4 ? launch_scan<true, 16>(sa, grid, s) : launch_scan<false, 16>(sa, grid, s); break;
+        default: return cudaErrorInvalidValue;
+    }
+    if (err != cudaSuccess) return err;
+
+    SelArgs sel;
+    sel.n_vis = ws.n_vis;
+    sel.scores = ws.scores;
+    sel.hist1 = ws.hist1;
+    sel.hist2 = ws.hist2;
+    sel.bitmap = ws.bitmap;
+    sel.ncand = ws.ncand;
+    sel.cand_key = ws.cand_key;
+    sel.cand_idx = ws.cand_idx;
+    sel.sel_idx = sel_idx;
+    sel.Nq = Nq;
+    sel.cap = c.capacity;
+    sel.topk = topk;
+    sel.words = ws.words;
+    sel.ccap = ws.ccap;
+    select_pass_kernel<<<dim3(kPassSlices, Nq), kSelThreads, 0, s>>>(sel);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    const int smem = index_select_smem_bytes(c.capacity);
+    if (smem > 48 * 1024) {
+        err = cudaFuncSetAttribute(select_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (err != cudaSuccess) return err;
+    }
+    select_final_kernel<<<Nq, kSelThreads, smem, s>>>(sel);
+    return cudaGetLastError();
+}
+
+}  // namespace csa

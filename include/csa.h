@@ -1,0 +1,200 @@
+/*
+ * csa.h -- C ABI of libcsa: compressed sparse attention (CSA), heavily
+ * compressed attention (HCA) and the uncompressed sliding window over a KV cache
+ * stored as MXFP4, for NVIDIA B200 (sm_100a).
+ *
+ * What the calls compute (page title and section):
+ *   "Frontier Architecture Decoding Notes (4): DeepSeek V4", section 1:
+ *     CSA compresses the KV of every 4 tokens into one entry and attends to the
+ *     top-k entries chosen per query; HCA compresses up to 128x and attends to
+ *     every entry; the most recent 128 tokens are attended uncompressed.
+ *   DeepSeek-V4.1-Flash podcast transcript, cue 12: indexer keys come from the
+ *     main KV; an indexer query scores them and the top-k are attended.
+ *   Same transcript, cue 16: the main KV is stored as MXFP4 (E2M1 elements
+ *     with a shared block scale) and dequantized right before attention.
+ * Readings where the pages are silent (the library's documented assumptions):
+ *   pooling is a softmax-gated weighted sum of the m tokens with one scalar
+ *   gate logit per token, g_t = <kv_t, w_g>; indexer score
+ *   s_j = sum_h w_h * ReLU(<q_idx_h, k_j>); top-k ties go to the lower block
+ *   index; one joint softmax covers the selected entries and the window;
+ *   MXFP4 = E2M1 elements with one E8M0 scale per 32 elements (OCP MX v1.0).
+ *
+ * Conventions for every call:
+ *   - Pointers inside csa_cache and every tensor argument are DEVICE pointers,
+ *     owned by the caller. The library allocates no memory and keeps no state;
+ *     scratch space is the caller's `workspace`.
+ *   - Every call checks its arguments on the host first. On an argument error
+ *     it returns the error code and launches nothing.
+ *   - Otherwise it enqueues its kernels on `stream` and returns CSA_OK without
+ *     synchronizing; a launch failure returns CSA_ERR_CUDA.
+ *   - Conditions only the device can see (a token count that is not a
+ *     multiple of m, a cache overflow, an out-of-range selected index or
+ *     window) set bits in cache->status (CSA_DEV_* below) when that pointer is
+ *     not NULL; the offending item is skipped, never trapped. Read the word
+ *     with csa_read_device_status() after the work has completed.
+ *   - bf16 means IEEE binary32 truncated to its upper 16 bits; e4m3 is OCP FP8
+ *     E4M3 ("fn": no infinities, max 448).
+ *   - All tensors are dense and row-major; every pointer must be 16-byte aligned.
+ */
+#ifndef CSA_H
+#define CSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *csa_stream_t; /* same type as cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+    CSA_OK = 0,
+    CSA_ERR_NULL = 1,        /* a required pointer is NULL                      */
+    CSA_ERR_SHAPE = 2,       /* a size is out of range or inconsistent          */
+    CSA_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned                */
+    CSA_ERR_UNSUPPORTED = 4, /* valid request this build does not implement     */
+    CSA_ERR_WORKSPACE = 5,   /* workspace NULL or smaller than required         */
+    CSA_ERR_CUDA = 6         /* a CUDA runtime call or kernel launch failed     */
+} csa_status;
+
+typedef enum { CSA_IDX_BF16 = 0, CSA_IDX_E4M3 = 1 } csa_idx_dtype;
+
+/* Bits OR-ed into *cache->status by the kernels. */
+#define CSA_DEV_TOKEN_COUNT 0x1  /* a request's new-token count is not a multiple of m: request skipped */
+#define CSA_DEV_CAPACITY    0x2  /* appending would exceed capacity: request skipped                  */
+#define CSA_DEV_BAD_INDEX   0x4  /* a selected block index >= the visible count: entry skipped          */
+#define CSA_DEV_BAD_WINDOW  0x8  /* win_len outside [0, max_win]: clamped                              */
+#define CSA_DEV_TIMEOUT     0x10 /* a bounded wait inside a kernel ran out: that tile's result is invalid */
+
+/*
+ * One compressed cache (one layer). Per request b and block j:
+ *   fp4     [batch][capacity][dim/2]   two E2M1 codes per byte, element 2i in the
+ *                                      low nibble, element 2i+1 in the high nibble
+ *   scale   [batch][capacity][dim/32]  E8M0 bytes, value 2^(byte-127)
+ *   idx_key [batch][capacity][idx_dim] bf16 or e4m3 pooled indexer keys; NULL for
+ *                                      a cache that is only attended densely (HCA)
+ *   n_blocks [batch]                   filled blocks per request; advanced by
+ *                                      csa_compress_quantize
+ *   status                             one int32 of CSA_DEV_* bits, or NULL
+ * An element's value is E2M1(code) * 2^(scale - 127).
+ */
+typedef struct {
+    int32_t batch;     /* requests, >= 1                                  */
+    int32_t dim;       /* D (K = V latent width); 128 or 512 for attention; multiple of 32 for compression */
+    int32_t block;     /* m, tokens pooled per entry, 1..128              */
+    int32_t capacity;  /* blocks per request, >= 1                        */
+    uint8_t *fp4;
+    uint8_t *scale;
+    void *idx_key;
+    int32_t idx_dim;   /* d_I, multiple of 16, <= 256 (0 when idx_key is NULL) */
+    int32_t idx_dtype; /* csa_idx_dtype                                   */
+    int32_t *n_blocks;
+    int32_t *status;
+} csa_cache;
+
+/* Human-readable name of a csa_status value. Never NULL. */
+const char *csa_status_string(int32_t status);
+
+/* Library ABI version (major * 100 + minor). */
+int32_t csa_version(void);
+
+/*
+ * Rows a1 + a2: gated block pooling and MXFP4 quantization.
+ * For each request b the new tokens are rows tok_offsets[b] .. tok_offsets[b+1]-1
+ * of kv_tok / idx_tok. Every m consecutive tokens become one block, appended at
+ * block n_blocks[b], n_blocks[b]+1, ...; n_blocks[b] is then advanced.
+ *   gate logit   g_t = sum_d kv_t[d] * gate_w[d]            (float32)
+ *   weights      a = softmax over the block's m logits
+ *   main entry   e[d] = sum_t a_t kv_t[d], stored as MXFP4:
+ *                per 32 elements X = floor(log2(max|e|)) - 2 clamped to [-127,127]
+ *                (X = -127 for an all-zero group), code = E2M1 round-to-nearest-even
+ *                of e * 2^-X saturated to +-6, sign kept (a negative value that
+ *                rounds to zero is code 0x8)
+ *   indexer key  k[c] = sum_t a_t idx_t[c], stored as bf16 (RNE) or e4m3 (RNE,
+ *                saturated to +-448) per cache->idx_dtype
+ * Arguments:
+ *   kv_tok      bf16 [n_tokens][dim]
+ *   idx_tok     bf16 [n_tokens][idx_dim]; required iff cache->idx_key != NULL
+ *   gate_w      float32 [dim]
+ *   tok_offsets int32 [batch+1] device, non-decreasing, tok_offsets[batch] <= n_tokens
+ *   n_tokens    rows of kv_tok (host value; bounds the launch)
+ * Device checks: a count that is not a multiple of m sets CSA_DEV_TOKEN_COUNT,
+ * an append beyond capacity sets CSA_DEV_CAPACITY; that request is left untouched.
+ */
+csa_status csa_compress_quantize(const csa_cache *cache, const void *kv_tok, const void *idx_tok,
+                                 const float *gate_w, const int32_t *tok_offsets, int32_t n_tokens,
+                                 csa_stream_t stream);
+
+/* Bytes of workspace csa_index_topk needs for these sizes (0 on bad sizes). */
+size_t csa_index_topk_workspace(const csa_cache *cache, int32_t n_queries, int32_t topk);
+
+/*
+ * Rows a3 + a4: indexer scoring and top-k block selection.
+ * Query i belongs to the request b with q_offsets[b] <= i < q_offsets[b+1] and
+ * sits at absolute token position q_pos[i]. It sees the blocks
+ * j < n_vis = min(floor((q_pos[i]+1)/m), n_blocks[b]) (causal at block granularity).
+ *   s_j = sum_{h < idx_heads} w[i][h] * max(0, sum_c q_idx[i][h][c] * key_j[c])
+ * sel_idx[i] receives the min(topk, n_vis) blocks with the largest s_j (float32
+ * comparison, -0 counted as +0, ties to the lower j) in ascending block order,
+ * padded with -1.
+ * Arguments:
+ *   q_idx     bf16 [n_queries][idx_heads][idx_dim]
+ *   w         float32 [n_queries][idx_heads]
+ *   q_offsets int32 [batch+1] device; q_pos int32 [n_queries] device
+ *   sel_idx   int32 [n_queries][topk] device, written
+ *   idx_heads 1..8; topk 1..4096
+ *   workspace >= csa_index_topk_workspace(cache, n_queries, topk) bytes, 256-byte aligned
+ */
+csa_status csa_index_topk(const csa_cache *cache, const void *q_idx, const float *w, int32_t n_queries,
+                          int32_t idx_heads, const int32_t *q_offsets, const int32_t *q_pos, int32_t topk,
+                          int32_t *sel_idx, void *workspace, size_t workspace_bytes, csa_stream_t stream);
+
+/* Bytes of workspace csa_decode_attend / hca_decode_attend need (0 on bad sizes). */
+size_t csa_attend_workspace(const csa_cache *cache, int32_t n_queries, int32_t heads);
+
+/*
+ * Rows a5 + a6 + a8: CSA joint attention.
+ * For query i and head h the entries are the dequantized blocks sel_idx[i][0..topk)
+ * of request b (negative indices are padding and ignored) followed by the window
+ * rows win_kv[win_start[i] + t], 0 <= t < win_len[i]. With
+ * logit = softmax_scale * <q[i][h], x>:
+ *   out[i][h] = sum_x softmax(logit)_x * x,   lse[i][h] = ln sum_x exp(logit_x).
+ * An empty entry set gives out = 0 and lse = -inf.
+ * Arguments:
+ *   q          bf16 [n_queries][heads][dim]   (heads == 64 or 16 with dim 512 or 128, see DESIGN)
+ *   sel_idx    int32 [n_queries][topk] device; entries must be < n_blocks[b]
+ *              (larger ones set CSA_DEV_BAD_INDEX and are skipped)
+ *   win_kv     bf16 [rows][dim]; win_start int64 [n_queries]; win_len int32 [n_queries]
+ *              (all three may be NULL together: no window); max_win bounds win_len
+ *   out        float32 [n_queries][heads][dim]; lse float32 [n_queries][heads] or NULL
+ *   workspace  >= csa_attend_workspace(cache, n_queries, heads) bytes, 256-byte aligned
+ */
+csa_status csa_decode_attend(const csa_cache *cache, const void *q, int32_t n_queries, int32_t heads,
+                             const int32_t *q_offsets, const int32_t *sel_idx, int32_t topk,
+                             const void *win_kv, const int64_t *win_start, const int32_t *win_len,
+                             int32_t max_win, float softmax_scale, float *out, float *lse,
+                             void *workspace, size_t workspace_bytes, csa_stream_t stream);
+
+/*
+ * Row a7 (+ a8): HCA dense attention. As csa_decode_attend, but the compressed
+ * entries of query i are every visible block j < min(floor((q_pos[i]+1)/m),
+ * n_blocks[b]) of the cache, in order; no indexer, no selection.
+ */
+csa_status hca_decode_attend(const csa_cache *cache, const void *q, int32_t n_queries, int32_t heads,
+                             const int32_t *q_offsets, const int32_t *q_pos,
+                             const void *win_kv, const int64_t *win_start, const int32_t *win_len,
+                             int32_t max_win, float softmax_scale, float *out, float *lse,
+                             void *workspace, size_t workspace_bytes, csa_stream_t stream);
+
+/*
+ * Waits for `stream`, then copies *cache->status to *out_flags and clears the
+ * device word. The only call that synchronizes. Returns CSA_ERR_NULL when
+ * cache->status is NULL.
+ */
+csa_status csa_read_device_status(const csa_cache *cache, csa_stream_t stream, int32_t *out_flags);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CSA_H */

@@ -62,7 +62,7 @@ def _load():
         lib.orc_e4m3_encode.restype = ctypes.c_uint8
         lib.orc_mxfp4_quantize_group.argtypes = [P, P, P]
         lib.orc_mxfp4_quantize_group.restype = None
-        lib.orc_compress.argtypes = [I, I, I, I, I, I, P, P, P, P, P, P, P, P, P]
+        lib.orc_compress.argtypes = [I, I, I, I, I, I, P, P, P, P, P, P, P, P, P, P]
         lib.orc_compress.restype = I
         lib.orc_index_scores.argtypes = [I, I, I, I, I, I, I, P, P, P, P, P, P, P, P]
         lib.orc_index_scores.restype = None
@@ -172,12 +172,14 @@ def compress(kv_tok, idx_tok, w_g, tok_offsets, n_blocks, *, m, cap, idx_dtype=I
     if idx_tok is not None and idx_key is None:
         idx_key = np.zeros((B, cap, kb), np.uint8)
     pooled = np.zeros((B, cap, D), np.float32) if return_pooled else None
+    pooled_idx = np.zeros((B, cap, dI), np.float32) if (return_pooled and idx_tok is not None) else None
     st = _load().orc_compress(B, D, dI, m, idx_dtype, cap, _ptr(kv_tok), _ptr(idx_tok), _ptr(w_g),
                               _ptr(tok_offsets), _ptr(n_blocks), _ptr(fp4), _ptr(scale),
-                              _ptr(idx_key) if idx_tok is not None else None, _ptr(pooled))
+                              _ptr(idx_key) if idx_tok is not None else None, _ptr(pooled), _ptr(pooled_idx))
     out = dict(fp4=fp4, scale=scale, idx_key=idx_key, n_blocks=n_blocks, status=st)
     if return_pooled:
         out["pooled"] = pooled
+        out["pooled_idx"] = pooled_idx
     return out
 
 

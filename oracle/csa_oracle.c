@@ -143,7 +143,8 @@ static size_t idx_key_bytes(int idx_dtype, int dI) { return (size_t)dI * (idx_dt
 int orc_compress(int B, int D, int dI, int m, int idx_dtype, int cap,
                  const uint16_t *kv_tok, const uint16_t *idx_tok, const float *w_g,
                  const int32_t *tok_offsets, int32_t *n_blocks,
-                 uint8_t *fp4, uint8_t *scale, uint8_t *idx_key, float *pooled_out) {
+                 uint8_t *fp4, uint8_t *scale, uint8_t *idx_key, float *pooled_out,
+                 float *pooled_idx_out) {
     int status = 0;
     for (int b = 0; b < B; ++b) {
         int count = tok_offsets[b + 1] - tok_offsets[b];
@@ -195,6 +196,7 @@ int orc_compress(int B, int D, int dI, int m, int idx_dtype, int cap,
                     double acc = 0.0;
                     for (int t = 0; t < m; ++t) acc += alpha[t] * orc_bf16_decode(idx_tok[(t0 + t) * dI + c]);
                     float kf = (float)acc;
+                    if (pooled_idx_out) pooled_idx_out[row * dI + c] = kf;
                     if (idx_dtype == 0) {
                         uint16_t bits = orc_bf16_encode(kf);
                         memcpy(dst + 2 * c, &bits, 2);

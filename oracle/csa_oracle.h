@@ -55,14 +55,15 @@ void     orc_mxfp4_quantize_group(const float *v, uint8_t *codes, uint8_t *scale
  *   fp4   [B][cap][D/2]  two codes per byte, element 2i in the low nibble
  *   scale [B][cap][D/32] E8M0 bytes
  *   idx_key [B][cap][dI] bf16 (idx_dtype 0) or e4m3 (idx_dtype 1)
- * Optional pooled_out [B][cap][D] float receives the float32 pooled value
- * before quantization (NULL to skip).
+ * Optional pooled_out [B][cap][D] float and pooled_idx_out [B][cap][dI] float
+ * receive the float32 pooled values before quantization (NULL to skip).
  * Returns 0, or -1 when a request's token count is not a multiple of m or
  * would overflow the capacity (nothing is written for that request). */
 int orc_compress(int B, int D, int dI, int m, int idx_dtype, int cap,
                  const uint16_t *kv_tok, const uint16_t *idx_tok, const float *w_g,
                  const int32_t *tok_offsets, int32_t *n_blocks,
-                 uint8_t *fp4, uint8_t *scale, uint8_t *idx_key, float *pooled_out);
+                 uint8_t *fp4, uint8_t *scale, uint8_t *idx_key, float *pooled_out,
+                 float *pooled_idx_out);
 
 /* ---- a3: indexer scores ---------------------------------------------- */
 /* Query i belongs to request req(i) given by q_offsets [B+1]. Visible blocks:

@@ -1,0 +1,169 @@
+"""Comparison rules between the CUDA path and the oracle (shared by the GPU tests).
+
+Bytes and indices are compared exactly. The only allowed differences are the
+near-ties where both sides legitimately round differently because the GPU
+accumulates in float32 in another order than the oracle's double precision:
+
+* MXFP4 element code: the oracle's scaled value v * 2^-X lies within
+  1e-5 relative (floor 4e-6) of an E2M1 rounding midpoint, or within the GPU's
+  float32 pooling error bound tol (in value units, 2^-14 times the largest
+  |token| pooled into that element: the pooled value is a weighted sum whose
+  rounding error scales with its terms, not with the result); the GPU code
+  must then be one of the two neighbouring codes.
+* MXFP4 scale byte: the oracle's float32 group amax lies within 1e-5 relative of
+  a power of two; the GPU group must then be a correct quantization of the
+  oracle's pooled values with the GPU's scale (same near-midpoint rule).
+* BF16 / E4M3 indexer keys: the oracle's float32 value lies within 1e-5 relative
+  of a rounding midpoint of the format; the GPU byte must be a neighbour.
+* top-k: where the oracle's k-th and (k+1)-th scores differ by less than 1e-5
+  relative, the GPU's set only has to be a valid top-k of the oracle's scores
+  within that tolerance (attention is then checked on the GPU's own set).
+Such exceptions must stay rare (the tests bound their count).
+
+Attention outputs: per (query, head) row, max_d |gpu - ref| / max_d |ref| <= 2e-3.
+"""
+import math
+
+import numpy as np
+
+import oracle
+
+REL = 1e-5
+E2M1_MID = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+ATT_TOL = 2e-3
+POOL_TOL = 2.0 ** -14
+
+
+def pooling_tolerance(tok_bits, offsets, n_blocks_before, m, cap):
+    """[B, cap, C] bound on the GPU's pooled-value error: POOL_TOL * max |token| over each block's tokens."""
+    x = np.abs((np.asarray(tok_bits, np.uint32) << 16).view(np.float32))
+    B = len(offsets) - 1
+    out = np.zeros((B, cap, x.shape[1]), np.float32)
+    for b in range(B):
+        t0, t1 = int(offsets[b]), int(offsets[b + 1])
+        nb = (t1 - t0) // m
+        if nb:
+            blk = x[t0:t0 + nb * m].reshape(nb, m, -1).max(axis=1)
+            out[b, n_blocks_before[b]:n_blocks_before[b] + nb] = POOL_TOL * blk
+    return out
+
+
+def unpack_codes(fp4):
+    fp4 = np.asarray(fp4, np.uint8)
+    return np.stack([fp4 & 0xF, fp4 >> 4], axis=-1).reshape(*fp4.shape[:-1], fp4.shape[-1] * 2)
+
+
+def near_e2m1_midpoint(s, tol_scaled=0.0):
+    a = np.abs(s)
+    d = np.min(np.abs(a[..., None] - E2M1_MID), axis=-1)
+    nearest_mid = E2M1_MID[np.argmin(np.abs(a[..., None] - E2M1_MID), axis=-1)]
+    return d <= np.maximum(np.maximum(REL * nearest_mid, 4e-6), tol_scaled)
+
+
+def e2m1_neighbours(c1, c2):
+    c1 = c1.astype(np.int32)
+    c2 = c2.astype(np.int32)
+    same_sign = (c1 & 8) == (c2 & 8)
+    both_zero = ((c1 & 7) == 0) & ((c2 & 7) == 0)
+    return (same_sign & (np.abs((c1 & 7) - (c2 & 7)) <= 1)) | both_zero | \
+        (((c1 & 7) <= 1) & ((c2 & 7) <= 1))
+
+
+def check_mxfp4(gpu_fp4, gpu_scale, orc_fp4, orc_scale, pooled, strict=False, max_frac=1e-3, tol=None):
+    """Compare MXFP4 planes [n, D/2], [n, D/32] against the oracle's bytes and float32 pooled values [n, D].
+    tol: optional [n, D] absolute error bound of the GPU's pooled values."""
+    gpu_fp4, gpu_scale = np.asarray(gpu_fp4), np.asarray(gpu_scale)
+    if strict:
+        assert np.array_equal(gpu_scale, orc_scale), "scale bytes differ (strict)"
+        assert np.array_equal(gpu_fp4, orc_fp4), "codes differ (strict)"
+        return 0
+    n, D = pooled.shape
+    gc, oc = unpack_codes(gpu_fp4), unpack_codes(orc_fp4)
+    exceptions = 0
+    bad_scale = np.argwhere(gpu_scale != orc_scale)
+    pooled64 = pooled.astype(np.float64)
+    for r, g in bad_scale:
+        grp = pooled[r, 32 * g:32 * g + 32]
+        amax = float(np.max(np.abs(grp)))
+        assert amax > 0
+        frac = math.log2(amax) - math.floor(math.log2(amax))
+        lo_p, hi_p = 2.0 ** math.floor(math.log2(amax)), 2.0 ** math.ceil(math.log2(amax))
+        gtol = 0.0 if tol is None else float(np.max(tol[r, 32 * g:32 * g + 32]))
+        near_pow2 = min(abs(amax - lo_p), abs(amax - hi_p)) <= max(REL * amax, gtol)
+        assert near_pow2, f"scale byte differs at row {r} group {g} (amax {amax}, frac {frac})"
+        X = int(gpu_scale[r, g]) - 127
+        s = np.ldexp(pooled64[r, 32 * g:32 * g + 32], -X)
+        ts = 0.0 if tol is None else np.ldexp(tol[r, 32 * g:32 * g + 32].astype(np.float64), -X)
+        want = np.array([oracle.e2m1_encode(float(v)) for v in np.clip(s, -1e9, 1e9)])
+        got = gc[r, 32 * g:32 * g + 32]
+        ok = (got == want) | (near_e2m1_midpoint(s, ts) & e2m1_neighbours(got, want))
+        assert ok.all(), f"group ({r},{g}) with the GPU scale is not a valid quantization"
+        oc[r, 32 * g:32 * g + 32] = got
+        exceptions += 1
+    diff = np.argwhere(gc != oc)
+    if len(diff):
+        X = (orc_scale.astype(np.int64) - 127).repeat(32, axis=-1)
+        s = np.ldexp(pooled64, -X)
+        rr, dd = diff[:, 0], diff[:, 1]
+        ts = 0.0 if tol is None else np.ldexp(tol.astype(np.float64), -X)[rr, dd]
+        ok = near_e2m1_midpoint(s[rr, dd], ts) & e2m1_neighbours(gc[rr, dd], oc[rr, dd])
+        assert ok.all(), f"{(~ok).sum()} codes differ away from a rounding midpoint, e.g. {diff[~ok][:5]}"
+        exceptions += len(diff)
+    assert exceptions <= max(4, max_frac * gc.size), f"too many near-tie exceptions: {exceptions}"
+    return exceptions
+
+
+def check_keys(gpu_keys, orc_keys, pooled_keys, dtype, max_frac=1e-3, tol=None):
+    """Indexer keys: bf16 (uint16 view) or e4m3 (uint8) against the oracle's, near-ties allowed
+    (within 1e-5 relative of a rounding midpoint, or within tol: the GPU's pooling error bound)."""
+    gpu_keys, orc_keys = np.asarray(gpu_keys), np.asarray(orc_keys)
+    diff = np.argwhere(gpu_keys != orc_keys)
+    if not len(diff):
+        return 0
+    vals = pooled_keys[tuple(diff.T)].astype(np.float64)
+    tols = np.zeros(len(vals)) if tol is None else tol[tuple(diff.T)].astype(np.float64)
+    for v, g, o, tv in zip(vals, gpu_keys[tuple(diff.T)], orc_keys[tuple(diff.T)], tols):
+        if dtype == "bf16":
+            dec = lambda b: oracle.bf16_decode(int(b))
+        else:
+            dec = lambda b: oracle.e4m3_decode(int(b))
+        a, b = dec(g), dec(o)
+        mid = 0.5 * (a + b)
+        assert abs(v - mid) <= max(REL * max(abs(mid), 1e-30), tv), \
+            f"key byte differs away from a midpoint: v={v} gpu={a} orc={b}"
+    assert len(diff) <= max(4, max_frac * gpu_keys.size)
+    return len(diff)
+
+
+def check_topk(gpu_sel, orc_sel, scores, n_vis, k):
+    """Exact match per query unless the oracle's k-th/(k+1)-th scores are a near-tie; then the GPU set
+    must be a valid top-k of the oracle scores within the tolerance. Returns the near-tie query ids."""
+    gpu_sel, orc_sel = np.asarray(gpu_sel), np.asarray(orc_sel)
+    near = []
+    for i in range(gpu_sel.shape[0]):
+        if np.array_equal(gpu_sel[i], orc_sel[i]):
+            continue
+        n = int(n_vis[i])
+        K = min(k, n)
+        s = scores[i, :n].astype(np.float64)
+        order = np.lexsort((np.arange(n), -s))
+        kth, nxt = s[order[K - 1]], s[order[K]] if K < n else -np.inf
+        tol = REL * max(abs(kth), 1e-30)
+        assert abs(kth - nxt) < tol, f"query {i}: top-k differs without a near-tie ({kth} vs {nxt})"
+        g = gpu_sel[i]
+        assert np.all(g[K:] == -1) and np.all(np.diff(g[:K]) > 0) and g[0] >= 0 and g[K - 1] < n
+        chosen = np.zeros(n, bool)
+        chosen[g[:K]] = True
+        assert s[chosen].min() >= kth - tol and (not (~chosen).any() or s[~chosen].max() <= kth + tol)
+        near.append(i)
+    return near
+
+
+def attention_row_error(gpu_out, ref_out):
+    """max over rows of max_d |gpu - ref| / max_d |ref| (rows with ref == 0 compare absolutely)."""
+    g = np.asarray(gpu_out, np.float64)
+    r = np.asarray(ref_out, np.float64)
+    num = np.max(np.abs(g - r), axis=-1)
+    den = np.max(np.abs(r), axis=-1)
+    err = np.where(den > 0, num / np.where(den > 0, den, 1), num)
+    return float(err.max()), err

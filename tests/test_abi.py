@@ -1,0 +1,126 @@
+"""C-ABI boundary checks that need no GPU: the library loads, exports every
+function include/csa.h declares, and rejects bad arguments on the host with the
+documented status codes (nothing is launched, so no device is touched)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import fp4_kv_cache_csa_b200 as csa
+from fp4_kv_cache_csa_b200 import build as csa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+OK, ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_UNSUPPORTED, ERR_WORKSPACE = 0, 1, 2, 3, 4, 5
+
+
+@pytest.fixture(scope="module")
+def lib():
+    csa_build.build()
+    return csa.load_library()
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "csa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*([a-z_0-9]+)\s*\(", text, flags=re.M)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = header_functions()
+    assert set(names) == set(csa.EXPORTED), names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert lib.csa_version() == 100
+    assert lib.csa_status_string(0) == b"ok"
+    assert lib.csa_status_string(99) == b"unknown status"
+
+
+def fake_cache(**kw):
+    # host addresses that are never dereferenced (every call below fails validation first)
+    d = dict(batch=2, dim=512, block=4, capacity=1024, fp4=0x10000, scale=0x20000, idx_key=0x30000,
+             idx_dim=128, idx_dtype=1, n_blocks=0x40000, status=0)
+    d.update(kw)
+    c = csa._CCache(d["batch"], d["dim"], d["block"], d["capacity"], d["fp4"], d["scale"], d["idx_key"],
+                    d["idx_dim"], d["idx_dtype"], d["n_blocks"], d["status"] or None)
+    return c
+
+
+def compress(lib, c, kv=0x50000, idx=0x60000, gate=0x70000, offs=0x80000, n=16):
+    return lib.csa_compress_quantize(ctypes.byref(c) if c is not None else None, kv, idx, gate, offs, n, None)
+
+
+def test_compress_validation(lib):
+    assert compress(lib, None) == ERR_NULL
+    assert compress(lib, fake_cache(fp4=0)) == ERR_NULL
+    assert compress(lib, fake_cache(), kv=0) == ERR_NULL
+    assert compress(lib, fake_cache(), idx=0) == ERR_NULL            # cache has keys, no key tokens
+    assert compress(lib, fake_cache(idx_key=0), idx=0x60000) == ERR_NULL
+    assert compress(lib, fake_cache(block=0)) == ERR_SHAPE
+    assert compress(lib, fake_cache(block=129)) == ERR_SHAPE
+    assert compress(lib, fake_cache(dim=100)) == ERR_SHAPE
+    assert compress(lib, fake_cache(dim=1024)) == ERR_UNSUPPORTED
+    assert compress(lib, fake_cache(idx_dim=96)) == ERR_UNSUPPORTED
+    assert compress(lib, fake_cache(capacity=(1 << 20) + 1)) == ERR_UNSUPPORTED
+    assert compress(lib, fake_cache(fp4=0x10008)) == ERR_ALIGN
+    assert compress(lib, fake_cache(), kv=0x50008) == ERR_ALIGN
+    assert compress(lib, fake_cache(), n=-1) == ERR_SHAPE
+
+
+def test_index_topk_validation(lib):
+    c = fake_cache()
+    ws = lib.csa_index_topk_workspace(ctypes.byref(c), 32, 1024)
+    assert ws > 32 * 1024 * 4  # at least the score rows
+    assert lib.csa_index_topk_workspace(ctypes.byref(c), 0, 1024) == 0
+
+    def call(cache=c, q=0x90000, w=0xA0000, nq=32, hi=4, offs=0xB0000, pos=0xC0000, k=1024, sel=0xD0000,
+             wsp=0x1000000, wsb=None):
+        return lib.csa_index_topk(ctypes.byref(cache), q, w, nq, hi, offs, pos, k, sel, wsp,
+                                  ws if wsb is None else wsb, None)
+
+    assert call(cache=fake_cache(idx_key=0)) == ERR_NULL
+    assert call(q=0) == ERR_NULL
+    assert call(nq=0) == ERR_SHAPE
+    assert call(k=0) == ERR_SHAPE
+    assert call(hi=9) == ERR_UNSUPPORTED
+    assert call(k=5000) == ERR_UNSUPPORTED
+    assert call(q=0x90008) == ERR_ALIGN
+    assert call(wsp=0) == ERR_WORKSPACE
+    assert call(wsb=ws - 1) == ERR_WORKSPACE
+    assert call(wsp=0x1000010) == ERR_ALIGN
+
+
+def test_attend_validation(lib):
+    c = fake_cache()
+
+    def call(cache=c, q=0x90000, nq=4, heads=64, offs=0xB0000, sel=0xD0000, k=64, win=0xE0000, ws_=0xF0000,
+             wl=0xF1000, maxw=128, out=0x1000000, lse=0):
+        return lib.csa_decode_attend(ctypes.byref(cache), q, nq, heads, offs, sel, k, win, ws_, wl, maxw, 0.1, out,
+                                     lse or None, 0x2000000, 1 << 30, None)
+
+    assert call(q=0) == ERR_NULL
+    assert call(out=0) == ERR_NULL
+    assert call(win=0) == ERR_NULL          # window pointers are all-or-none
+    assert call(nq=0) == ERR_SHAPE
+    assert call(maxw=-1) == ERR_SHAPE
+    assert call(heads=65) == ERR_UNSUPPORTED
+    assert call(cache=fake_cache(dim=256)) == ERR_UNSUPPORTED
+    assert call(q=0x90008) == ERR_ALIGN
+    assert lib.hca_decode_attend(ctypes.byref(c), 0x90000, 4, 64, 0xB0000, None, None, None, None, 128, 0.1,
+                                 0x1000000, None, 0x2000000, 1 << 30, None) != OK
+
+
+def test_read_status_needs_status_word(lib):
+    v = ctypes.c_int32(0)
+    assert lib.csa_read_device_status(ctypes.byref(fake_cache()), None, ctypes.byref(v)) == ERR_NULL
+
+
+def test_missing_library_raises():
+    saved = csa._lib
+    try:
+        csa._lib = None
+        with pytest.raises(csa.CsaError):
+            csa.load_library("/nonexistent/libcsa.so")
+    finally:
+        csa._lib = saved
