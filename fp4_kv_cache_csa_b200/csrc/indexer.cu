@@ -608,11 +608,11 @@ cudaError_t launch_index_topk(const csa_cache &c, const void *q_idx, const float
     sel.ccap = ws.ccap;
     select_pass_kernel<<<dim3(kPassSlices, Nq), kSelThreads, 0, s>>>(sel);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    // the bitmap (dynamic) comes on top of ~33 KB of static shared memory:
+    // opt in to the dynamic size every time (cheap, and valid during capture)
     const int smem = index_select_smem_bytes(c.capacity);
-    if (smem > 48 * 1024) {
-        err = cudaFuncSetAttribute(select_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (err != cudaSuccess) return err;
-    }
+    err = cudaFuncSetAttribute(select_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err != cudaSuccess) return err;
     select_final_kernel<<<Nq, kSelThreads, smem, s>>>(sel);
     return cudaGetLastError();
 }

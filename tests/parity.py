@@ -10,6 +10,9 @@ accumulates in float32 in another order than the oracle's double precision:
   |token| pooled into that element: the pooled value is a weighted sum whose
   rounding error scales with its terms, not with the result); the GPU code
   must then be one of the two neighbouring codes.
+* The sign of a zero code (0x0 / 0x8) follows the sign of a value that rounds to
+  zero magnitude; it may differ where the oracle's value is within that same
+  bound of 0.
 * MXFP4 scale byte: the oracle's float32 group amax lies within 1e-5 relative of
   a power of two; the GPU group must then be a correct quantization of the
   oracle's pooled values with the GPU's scale (same near-midpoint rule).
@@ -54,10 +57,14 @@ def unpack_codes(fp4):
 
 
 def near_e2m1_midpoint(s, tol_scaled=0.0):
+    """Within tolerance of an E2M1 rounding midpoint, or of 0 (where the sign bit of a value that
+    rounds to zero magnitude is decided: codes 0x0 and 0x8)."""
     a = np.abs(s)
     d = np.min(np.abs(a[..., None] - E2M1_MID), axis=-1)
     nearest_mid = E2M1_MID[np.argmin(np.abs(a[..., None] - E2M1_MID), axis=-1)]
-    return d <= np.maximum(np.maximum(REL * nearest_mid, 4e-6), tol_scaled)
+    near_mid = d <= np.maximum(np.maximum(REL * nearest_mid, 4e-6), tol_scaled)
+    near_zero = a <= np.maximum(4e-6, tol_scaled)
+    return near_mid | near_zero
 
 
 def e2m1_neighbours(c1, c2):

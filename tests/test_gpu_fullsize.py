@@ -1,0 +1,138 @@
+"""Parity at the full workload sizes, in the launch configuration the benchmark times.
+
+The GPU runs the whole batch; the oracle recomputes sampled queries one by one.
+  * csa_b32_1m: 32 requests, 131072..262144 blocks each (512K..1M tokens, m = 4),
+    e4m3 indexer keys, k = 1024, D = 512, 64 heads, 128-token window.
+  * hca_b64_1m: 64 requests x 8192 blocks (1M tokens, m = 128), dense.
+  * csa_b8_64k: 8 requests x 65536 tokens from raw tokens through every kernel
+    (per-channel LogNormal(0, 0.5) activations), checked stage by stage.
+Cache contents for the first two are seeded bytes (the kernels' inputs), not
+outputs of the compression kernel."""
+import numpy as np
+import pytest
+
+import oracle
+from fp4_kv_cache_csa_b200 import datagen
+from gpu_util import dev, host, make_cache
+import parity
+
+pytestmark = pytest.mark.gpu
+
+
+def test_csa_b32_1m_sampled():
+    import torch
+
+    import fp4_kv_cache_csa_b200 as csa
+
+    wl = datagen.WORKLOADS["csa_b32_1m"]
+    B, D, H, dI, k, W = wl.batch, wl.dim, wl.heads, wl.idx_dim, wl.topk, wl.window
+    n = (datagen.context_lengths(wl, 500) // wl.block).astype(np.int64)
+    cap = int(n.max())
+    sample = [0, 17, int(np.argmax(n))]
+    fp4_d = torch.empty(B, cap, D // 2, dtype=torch.uint8, device="cuda")
+    sc_d = torch.empty(B, cap, D // 32, dtype=torch.uint8, device="cuda")
+    key_d = torch.empty(B, cap, dI, dtype=torch.uint8, device="cuda")
+    host_rows = {}
+    for b in range(B):
+        f, s = datagen.random_cache_bytes(cap, D, 501, b)
+        kx = datagen.to_e4m3_bytes(datagen.normal_f32((cap, dI), 502, b, std=0.5))
+        fp4_d[b].copy_(torch.from_numpy(f))
+        sc_d[b].copy_(torch.from_numpy(s))
+        key_d[b].copy_(torch.from_numpy(kx))
+        if b in sample:
+            host_rows[b] = (f, s, kx)
+    cache = csa.Cache(fp4=fp4_d, scale=sc_d, n_blocks=dev(n.astype(np.int32)), block=wl.block, idx_key=key_d,
+                      idx_dtype=csa.CSA_IDX_E4M3, status=torch.zeros(1, dtype=torch.int32, device="cuda"))
+    q = datagen.normal_bf16((B, H, D), 503, 1)
+    q_idx = datagen.normal_bf16((B, wl.idx_heads, dI), 503, 2)
+    w = datagen.normal_f32((B, wl.idx_heads), 503, 3, std=0.5)
+    win = datagen.normal_bf16((B * W, D), 503, 4)
+    qo = np.arange(B + 1, dtype=np.int32)
+    qp = (n * wl.block - 1).astype(np.int32)
+    ws_, wl_ = (np.arange(B) * W).astype(np.int64), np.full(B, W, np.int32)
+    sel = host(csa.csa_index_topk(cache, dev(q_idx), dev(w), dev(qo), dev(qp), k))
+    out = host(csa.csa_decode_attend(cache, dev(q), dev(qo), dev(sel), dev(win), dev(ws_), dev(wl_)))
+    assert csa.csa_read_device_status(cache) == 0
+    for b in sample:
+        f, s, kx = host_rows[b]
+        one = np.array([0, 1], np.int32)
+        sel_ref, scores, n_vis = oracle.index_topk(kx[None], n[b:b + 1].astype(np.int32), one, qp[b:b + 1],
+                                                   q_idx[b:b + 1], w[b:b + 1], m=wl.block, k=k, idx_dtype=1)
+        near = parity.check_topk(sel[b:b + 1], sel_ref, scores, n_vis, k)
+        use = sel[b:b + 1] if near else sel_ref  # near-tie: attention on the GPU's own selection
+        ref, _ = oracle.csa_attend(f[None], s[None], one, q[b:b + 1], use, win[b * W:(b + 1) * W],
+                                   np.array([0], np.int64), np.array([W], np.int32), D ** -0.5)
+        err, _ = parity.attention_row_error(out[b:b + 1], ref)
+        assert err <= parity.ATT_TOL, (b, err)
+
+
+def test_hca_b64_1m_sampled():
+    import torch
+
+    import fp4_kv_cache_csa_b200 as csa
+
+    wl = datagen.WORKLOADS["hca_b64_1m"]
+    B, D, H, W = wl.batch, wl.dim, wl.heads, wl.window
+    cap = wl.ctx_max // wl.block
+    f, s = datagen.random_cache_bytes(B * cap, D, 510, 0, scale_lo=119, scale_hi=122)
+    f, s = f.reshape(B, cap, D // 2), s.reshape(B, cap, D // 32)
+    cache = make_cache(f, s, np.full(B, cap, np.int32), wl.block)
+    q = datagen.normal_bf16((B, H, D), 511, 1)
+    win = datagen.normal_bf16((B * W, D), 511, 2)
+    qo = np.arange(B + 1, dtype=np.int32)
+    qp = np.full(B, wl.ctx_max - 1, np.int32)
+    ws_, wl_ = (np.arange(B) * W).astype(np.int64), np.full(B, W, np.int32)
+    out = host(csa.hca_decode_attend(cache, dev(q), dev(qo), dev(qp), dev(win), dev(ws_), dev(wl_)))
+    assert csa.csa_read_device_status(cache) == 0
+    one = np.array([0, 1], np.int32)
+    for b in (0, 31, 63):
+        ref, _ = oracle.hca_attend(f[b:b + 1], s[b:b + 1], np.array([cap], np.int32), one, qp[b:b + 1], q[b:b + 1],
+                                   win[b * W:(b + 1) * W], np.array([0], np.int64), np.array([W], np.int32),
+                                   D ** -0.5, m=wl.block)
+        err, _ = parity.attention_row_error(out[b:b + 1], ref)
+        assert err <= parity.ATT_TOL, (b, err)
+
+
+def test_csa_b8_64k_from_tokens():
+    import torch
+
+    import fp4_kv_cache_csa_b200 as csa
+
+    wl = datagen.WORKLOADS["csa_b8_64k"]
+    B, D, H, dI, m, k, W, T = wl.batch, wl.dim, wl.heads, wl.idx_dim, wl.block, wl.topk, wl.window, wl.ctx_max
+    cap = T // m
+    kv = datagen.normal_bf16((B * T, D), 520, 1, channel_lognormal=wl.channel_lognormal)
+    it = datagen.normal_bf16((B * T, dI), 520, 2, channel_lognormal=wl.channel_lognormal)
+    wg = datagen.normal_f32((D,), 520, 3, std=0.02)
+    offs = (np.arange(B + 1) * T).astype(np.int32)
+    ref = oracle.compress(kv, it, wg, offs, np.zeros(B, np.int32), m=m, cap=cap, return_pooled=True)
+    # stage 1: pooling + quantization of all 8 x 16384 blocks
+    cache = csa.Cache.allocate(B, cap, D, m, dI, csa.CSA_IDX_BF16)
+    csa.csa_compress_quantize(cache, dev(kv), dev(it), dev(wg), dev(offs))
+    assert csa.csa_read_device_status(cache) == 0
+    tol = parity.pooling_tolerance(kv, offs, np.zeros(B, np.int64), m, cap)
+    parity.check_mxfp4(host(cache.fp4).reshape(B * cap, -1), host(cache.scale).reshape(B * cap, -1),
+                       ref["fp4"].reshape(B * cap, -1), ref["scale"].reshape(B * cap, -1),
+                       ref["pooled"].reshape(B * cap, D), tol=tol.reshape(B * cap, D))
+    parity.check_keys(host(cache.idx_key).view(np.uint16), ref["idx_key"].view(np.uint16).reshape(B, cap, dI),
+                      ref["pooled_idx"], "bf16", tol=parity.pooling_tolerance(it, offs, np.zeros(B, np.int64), m, cap))
+    # stage 2: indexer + top-k on the oracle's cache
+    ocache = make_cache(ref["fp4"], ref["scale"], ref["n_blocks"], m, ref["idx_key"].view(np.uint16), 0)
+    q = datagen.normal_bf16((B, H, D), 521, 1, channel_lognormal=wl.channel_lognormal)
+    q_idx = datagen.normal_bf16((B, wl.idx_heads, dI), 521, 2, channel_lognormal=wl.channel_lognormal)
+    w = datagen.normal_f32((B, wl.idx_heads), 521, 3, std=0.5)
+    qo = np.arange(B + 1, dtype=np.int32)
+    qp = np.full(B, T - 1, np.int32)
+    sel_ref, scores, n_vis = oracle.index_topk(ref["idx_key"], ref["n_blocks"], qo, qp, q_idx, w, m=m, k=k)
+    sel = host(csa.csa_index_topk(ocache, dev(q_idx), dev(w), dev(qo), dev(qp), k))
+    near = parity.check_topk(sel, sel_ref, scores, n_vis, k)
+    # stage 3: joint attention over the selection (the GPU's where the oracle has a near-tie) + window
+    use = sel_ref.copy()
+    use[near] = sel[near]
+    win = np.concatenate([kv[b * T + T - W:b * T + T] for b in range(B)])
+    ws_, wl_ = (np.arange(B) * W).astype(np.int64), np.full(B, W, np.int32)
+    out = host(csa.csa_decode_attend(ocache, dev(q), dev(qo), dev(use), dev(win), dev(ws_), dev(wl_)))
+    want, _ = oracle.csa_attend(ref["fp4"], ref["scale"], qo, q, use, win, ws_, wl_, D ** -0.5)
+    err, _ = parity.attention_row_error(out, want)
+    assert err <= parity.ATT_TOL, err
+    assert csa.csa_read_device_status(ocache) == 0
