@@ -32,6 +32,7 @@ CSA_DEV_TIMEOUT = 0x10
 EXPORTED = (
     "csa_status_string", "csa_version", "csa_compress_quantize", "csa_index_topk_workspace", "csa_index_topk",
     "csa_attend_workspace", "csa_decode_attend", "hca_decode_attend", "csa_read_device_status",
+    "csa_index_topk_noalloc",
 )
 
 
@@ -71,6 +72,8 @@ def load_library(path: str = LIB_PATH):
     lib.csa_index_topk_workspace.restype = S
     lib.csa_index_topk.argtypes = [CP, P, P, I, I, P, P, I, P, P, S, P]
     lib.csa_index_topk.restype = I
+    lib.csa_index_topk_noalloc.argtypes = [CP, P, P, I, I, P, P, I, P, P]
+    lib.csa_index_topk_noalloc.restype = I
     lib.csa_attend_workspace.argtypes = [CP, I, I]
     lib.csa_attend_workspace.restype = S
     lib.csa_decode_attend.argtypes = [CP, P, I, I, P, P, I, P, P, P, I, ctypes.c_float, P, P, P, S, P]
@@ -166,6 +169,17 @@ def csa_compress_quantize(cache: Cache, kv_tok, idx_tok, gate_w, tok_offsets, st
 
 def csa_index_topk_workspace(cache: Cache, n_queries: int, topk: int) -> int:
     return int(load_library().csa_index_topk_workspace(ctypes.byref(cache.c_struct()), n_queries, topk))
+
+
+def csa_index_topk_noalloc(cache: Cache, q_idx, w, q_offsets, q_pos, topk: int, sel_idx, stream=None):
+    """csa_index_topk with the library's fixed 32 MiB device scratch instead of a workspace, for
+    callers that cannot allocate device memory (see include/csa.h). sel_idx must be passed in."""
+    lib = load_library()
+    c = cache.c_struct()
+    _check(lib.csa_index_topk_noalloc(ctypes.byref(c), _ptr(q_idx), _ptr(w), int(q_idx.shape[0]),
+                                      int(q_idx.shape[1]), _ptr(q_offsets), _ptr(q_pos), topk, _ptr(sel_idx),
+                                      _stream(stream)), "csa_index_topk_noalloc")
+    return sel_idx
 
 
 def csa_attend_workspace(cache: Cache, n_queries: int, heads: int) -> int:

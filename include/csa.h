@@ -22,7 +22,8 @@
  * Conventions for every call:
  *   - Pointers inside csa_cache and every tensor argument are DEVICE pointers,
  *     owned by the caller. The library allocates no memory and keeps no state;
- *     scratch space is the caller's `workspace`.
+ *     scratch space is the caller's `workspace` (csa_index_topk_noalloc alone
+ *     uses a fixed scratch array the library holds instead).
  *   - Every call checks its arguments on the host first. On an argument error
  *     it returns the error code and launches nothing.
  *   - Otherwise it enqueues its kernels on `stream` and returns CSA_OK without
@@ -149,6 +150,31 @@ size_t csa_index_topk_workspace(const csa_cache *cache, int32_t n_queries, int32
 csa_status csa_index_topk(const csa_cache *cache, const void *q_idx, const float *w, int32_t n_queries,
                           int32_t idx_heads, const int32_t *q_offsets, const int32_t *q_pos, int32_t topk,
                           int32_t *sel_idx, void *workspace, size_t workspace_bytes, csa_stream_t stream);
+
+/*
+ * csa_index_topk without a caller workspace. The method has no counterpart to
+ * this call: it exists for callers that cannot allocate device memory -- a
+ * plugin or embedded runtime whose host framework owns every allocation, a
+ * deployment with a fixed memory budget, or code that cannot afford the
+ * device-wide synchronization an allocation may bring. The caller still
+ * passes all inputs and outputs exactly as for csa_index_topk (same meaning,
+ * same results); only the scratch space is the library's.
+ *   - The scratch is one fixed 32 MiB array in device memory, held on every
+ *     GPU that loads the library until the process exits. Sizes whose
+ *     csa_index_topk_workspace() exceeds 32 MiB are rejected with
+ *     CSA_ERR_WORKSPACE before anything is launched.
+ *   - The first call on each device looks up that array's device address
+ *     (once, with the device current). Make that first call before any
+ *     stream capture on the device.
+ *   - Every call uses the same array; each call clears what must start at
+ *     zero, so leftovers from the previous call do not matter. Calls that
+ *     overlap on the GPU (other streams, or another host thread) race on the
+ *     array: serialize them.
+ *   - Nothing here calls cudaMalloc, cudaFree or any allocating routine.
+ */
+csa_status csa_index_topk_noalloc(const csa_cache *cache, const void *q_idx, const float *w, int32_t n_queries,
+                                  int32_t idx_heads, const int32_t *q_offsets, const int32_t *q_pos, int32_t topk,
+                                  int32_t *sel_idx, csa_stream_t stream);
 
 /* Bytes of workspace csa_decode_attend / hca_decode_attend need (0 on bad sizes). */
 size_t csa_attend_workspace(const csa_cache *cache, int32_t n_queries, int32_t heads);

@@ -1,0 +1,59 @@
+"""csa_index_topk_noalloc: the indexer + top-k call for callers that cannot
+allocate device memory (a host framework that owns every allocation, a fixed
+memory budget, or code that cannot afford an allocation's synchronization).
+Its scratch is a fixed 32 MiB array inside the library instead of a caller
+workspace, so its results must equal csa_index_topk's exactly; and since every
+call reuses that array, two calls in a row (with different inputs) must each
+still match. This file is collected last on purpose."""
+import ctypes
+
+import numpy as np
+import pytest
+
+import fp4_kv_cache_csa_b200 as csa
+from fp4_kv_cache_csa_b200 import build as csa_build
+from fp4_kv_cache_csa_b200 import datagen
+
+ERR_WORKSPACE = 5
+
+
+def _inputs(seed, lengths, dI, idx_dtype, k):
+    import torch
+
+    from gpu_util import dev, make_cache
+
+    B = len(lengths)
+    cap = max(lengths) + 3
+    x = datagen.normal_f32((B, cap, dI), seed, 1, std=0.5)
+    keys = datagen.to_bf16_bits(x) if idx_dtype == 0 else datagen.to_e4m3_bytes(x)
+    cache = make_cache(np.zeros((B, cap, 64), np.uint8), np.zeros((B, cap, 4), np.uint8), lengths, 4, keys,
+                       idx_dtype)
+    q_idx = dev(datagen.normal_bf16((B, 4, dI), seed, 2))
+    w = dev(datagen.normal_f32((B, 4), seed, 3, std=0.5))
+    qo = dev(np.arange(B + 1, dtype=np.int32))
+    qp = dev((np.asarray(lengths) * 4 - 1).astype(np.int32))
+    return cache, q_idx, w, qo, qp, torch
+
+
+@pytest.mark.gpu
+def test_noalloc_matches_the_workspace_call_twice_in_a_row():
+    cases = [(71, [5000, 16384, 700, 12001], 128, 1, 512),   # e4m3 keys, ragged
+             (72, [9000, 300, 16000], 64, 0, 1024)]           # bf16 keys, another shape
+    for seed, lengths, dI, dt, k in cases:  # two consecutive calls on the shared scratch
+        cache, q_idx, w, qo, qp, torch = _inputs(seed, lengths, dI, dt, k)
+        want = csa.csa_index_topk(cache, q_idx, w, qo, qp, k)
+        got = torch.full_like(want, -7)
+        csa.csa_index_topk_noalloc(cache, q_idx, w, qo, qp, k, got)
+        torch.cuda.synchronize()
+        assert torch.equal(got, want), seed
+        assert csa.csa_read_device_status(cache) == 0
+
+
+def test_noalloc_rejects_sizes_beyond_its_scratch():
+    # checked on the host before any device work: 32 queries x 262144 blocks needs > 32 MiB
+    csa_build.build()
+    lib = csa.load_library()
+    c = csa._CCache(32, 512, 4, 262144, 0x10000, 0x20000, 0x30000, 128, 1, 0x40000, None)
+    assert lib.csa_index_topk_workspace(ctypes.byref(c), 32, 1024) > (32 << 20)
+    st = lib.csa_index_topk_noalloc(ctypes.byref(c), 0x90000, 0xA0000, 32, 4, 0xB0000, 0xC0000, 1024, 0xD0000, None)
+    assert st == ERR_WORKSPACE
