@@ -38,8 +38,13 @@ B, D, H, M_CSA, M_HCA, W = 32, 512, 64, 4, 128, 128
 H_I, D_I, TOPK = 4, 128, 1024
 CTX_MIN, CTX_MAX = 524288, 1048576
 CAP_CSA, CAP_HCA = CTX_MAX // M_CSA, CTX_MAX // M_HCA
-OUR_KERNELS_PER_STEP = 12  # compress 2x(pool, commit); index: schedule, scan, select x2; attend 2x(schedule, main)
+OUR_KERNELS_PER_STEP = 14  # compress 2x(pool, commit); index: schedule, scan, select x2; attend 2x(schedule, main, merge)
 SEED = 0x5EED0C5A
+
+
+def set_batch(n: int):
+    global B
+    B = int(n)
 
 
 def log(*a):
@@ -51,7 +56,7 @@ def context_lengths(rank: int) -> np.ndarray:
     from fp4_kv_cache_csa_b200 import datagen
 
     g = datagen.generator(1000 + rank)
-    return (g.integers(CTX_MIN // 128, CTX_MAX // 128, size=B, endpoint=True) * 128).astype(np.int64)
+    return (g.integers(CTX_MIN // 128, CTX_MAX // 128, size=32, endpoint=True) * 128).astype(np.int64)[:B]
 
 
 class Workload:
@@ -280,7 +285,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=B, help="requests per GPU (default 32; smaller only for profiling)")
     args = ap.parse_args()
+    set_batch(args.batch)
     if args.impl == "reference":
         return run_reference(args)
 

@@ -14,8 +14,8 @@
 //   * Work = the flat list of 128-entry tiles of all queries (compressed tiles
 //     first, then window tiles), cut into equal contiguous ranges, one per CTA.
 //     A CTA whose range covers a whole query writes the output directly;
-//     otherwise it writes an unnormalized partial and the last CTA to finish
-//     that query (atomic counter, no waiting) merges the partials.
+//     otherwise it writes an unnormalized partial, and attend_merge_kernel
+//     (one CTA per query and 8-head slice) combines the partials.
 //   * Operands are fp16 in shared memory. Entry j is stored as
 //     E'_j = e_j * 2^-R_j with R_j the largest E8M0 exponent of the row (or the
 //     exponent of max|x| for a window row): every E2M1 x 2^X value is exact in
@@ -50,7 +50,6 @@ constexpr long long kWaitCycles = 2000000000LL;  // bounded mbarrier wait (~1 s)
 
 template <int D>
 struct Cfg {
-    static constexpr int KCH = D / 64;                    // 128-byte k-chunks per row
     static constexpr int DT = D / 128;                    // O^T d-tiles
     static constexpr int GPR = D / 32;                    // MXFP4 groups per row
     static constexpr int CODE_V = D / 32;                 // 16-byte code loads per row (D/2 bytes)
@@ -194,7 +193,6 @@ struct AttArgs {
     // schedule (workspace)
     const int32_t *req, *nent, *ctiles, *wlen;
     const long long *tprefix;        // [Nq+1]
-    uint32_t *counters;              // [Nq]
     float *part_o, *part_rho, *part_l;  // [2G][64][D], [2G][64], [2G][64]
     int Nq, H, cap, topk;
     float scale_log2;                // softmax_scale * log2(e)
@@ -359,6 +357,7 @@ __device__ int load_query(const AttArgs &a, int i, uint8_t *Q, float *red) {
     const __nv_bfloat16 *qi = a.q + (size_t)i * a.H * D;
     const int nchunks = a.H * (D / 8);
     float mx = 0.f;
+#pragma unroll 8
     for (int c = tid; c < nchunks; c += kThreads) {
         uint4 u = __ldg(reinterpret_cast<const uint4 *>(qi) + c);
         const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
@@ -377,6 +376,7 @@ __device__ int load_query(const AttArgs &a, int i, uint8_t *Q, float *red) {
     const float inv = ldexpf(1.0f, -sQ);
     // chunk (h, kc): consecutive threads take consecutive heads, so the
     // swizzled 16-byte stores of a warp spread over all eight bank groups
+#pragma unroll 8
     for (int c = tid; c < kHeads * (D / 8); c += kThreads) {
         const int h = c % kHeads;
         const int kc = c / kHeads;
@@ -440,6 +440,73 @@ __global__ void attend_schedule_kernel(const int32_t *q_offsets, const int32_t *
         for (int k = threadIdx.x; k < H * D; k += blockDim.x) out[(size_t)i * H * D + k] = 0.f;
         if (lse)
             for (int k = threadIdx.x; k < H; k += blockDim.x) lse[(size_t)i * H + k] = -INFINITY;
+    }
+}
+
+// ---------------------------------------------------------------- split merge
+// Row a8: a query whose tiles were spread over several CTAs has one partial
+// (unnormalized O, reference rho, row sum l) per CTA; combine them with the
+// log-sum-exp rule. One CTA per (query, 8-head slice); queries that a single
+// CTA covered were written directly by attend_kernel and are skipped.
+constexpr int kMergeHeads = 8;
+
+__global__ void __launch_bounds__(256) attend_merge_kernel(const long long *tprefix, int Nq, int H, int D, int G,
+                                                           const float *part_o, const float *part_rho,
+                                                           const float *part_l, float *out, float *lse) {
+    __shared__ int slots[256];
+    __shared__ float wts[256 * kMergeHeads];
+    __shared__ float inv_l[kMergeHeads];
+    __shared__ int np_s;
+    const int i = blockIdx.x;
+    const int h0 = blockIdx.y * kMergeHeads;
+    if (h0 >= H) return;
+    const long long T = tprefix[Nq], Ti = tprefix[i], Ti1 = tprefix[i + 1];
+    if (Ti1 == Ti) return;  // no entry at all: written by the schedule kernel
+    const int c_first = (int)(((Ti + 1) * G - 1) / T);
+    const int c_last = (int)((Ti1 * G - 1) / T);
+    if (c_first == c_last) return;  // one CTA covered the query and wrote it
+    if (threadIdx.x == 0) {
+        int np = 0;
+        for (int cc = c_first; cc <= c_last && np < 256; ++cc) {
+            const long long rb = T * cc / G, re = T * (cc + 1) / G;
+            if (rb >= re) continue;  // CTA with an empty range
+            slots[np++] = 2 * cc + (rb >= Ti ? 0 : 1);
+        }
+        np_s = np;
+    }
+    __syncthreads();
+    const int np = np_s;
+    const int nh = min(kMergeHeads, H - h0);
+    if (threadIdx.x < nh) {
+        const int h = h0 + threadIdx.x;
+        float rmax = -INFINITY;
+        for (int p = 0; p < np; ++p) rmax = fmaxf(rmax, part_rho[(size_t)slots[p] * kHeads + h]);
+        float l = 0.f;
+        for (int p = 0; p < np; ++p) {
+            const float wgt = exp2f(part_rho[(size_t)slots[p] * kHeads + h] - rmax);
+            wts[p * kMergeHeads + threadIdx.x] = wgt;
+            l += wgt * part_l[(size_t)slots[p] * kHeads + h];
+        }
+        inv_l[threadIdx.x] = l > 0.f ? 1.f / l : 0.f;
+        if (lse) lse[(size_t)i * H + h] = l > 0.f ? (rmax + log2f(l)) * 0.69314718055994531f : -INFINITY;
+    }
+    __syncthreads();
+    // float4 over the latent dimension; independent loads across partials
+    const int per_head = D / 4;
+    for (int v = threadIdx.x; v < nh * per_head; v += blockDim.x) {
+        const int hh = v / per_head, d4 = v % per_head;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int p = 0; p < np; ++p) {
+            const float4 o = __ldcg(reinterpret_cast<const float4 *>(part_o + ((size_t)slots[p] * kHeads + h0 + hh) * D) + d4);
+            const float wgt = wts[p * kMergeHeads + hh];
+            acc.x = fmaf(wgt, o.x, acc.x);
+            acc.y = fmaf(wgt, o.y, acc.y);
+            acc.z = fmaf(wgt, o.z, acc.z);
+            acc.w = fmaf(wgt, o.w, acc.w);
+        }
+        const float il = inv_l[hh];
+        reinterpret_cast<float4 *>(out + ((size_t)i * H + h0 + hh) * D)[d4] =
+            make_float4(acc.x * il, acc.y * il, acc.z * il, acc.w * il);
     }
 }
 
@@ -562,22 +629,20 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
                 if (__syncthreads_or(!ok)) { aborted = true; break; }
             }
             tc_fence_after();
-            float u[64];
-            tmem_ld64(tmem_s + lane_off, u);
-            // u = log2(e) * scale * <q, e_j> + R_j, or -inf for an empty row
-            {
-                const float cj = ldexpf(a.scale_log2, Rj + sQ);
-#pragma unroll
-                for (int h = 0; h < 64; ++h) u[h] = valid ? fmaf(u[h], cj, (float)Rj) : -INFINITY;
-            }
+            // u = log2(e) * scale * <q, e_j> + R_j, or -inf for an empty row.
+            // S^T stays in TMEM and is read twice (max, then P'), so no second
+            // 64-value copy has to live in registers.
+            const float cj = ldexpf(a.scale_log2, Rj + sQ);
+            const float rjf = (float)Rj;
             // ---- per-head tile max -> reference update ----
             {
-                float m[64];
+                float u[64];
+                tmem_ld64(tmem_s + lane_off, u);
 #pragma unroll
-                for (int h = 0; h < 64; ++h) m[h] = u[h];
-                transpose_reduce64<true>(m);
-                wred[warp * 64 + 2 * lane] = m[0];
-                wred[warp * 64 + 2 * lane + 1] = m[1];
+                for (int h = 0; h < 64; ++h) u[h] = valid ? fmaf(u[h], cj, rjf) : -INFINITY;
+                transpose_reduce64<true>(u);  // in place: lane L keeps heads 2L, 2L+1
+                wred[warp * 64 + 2 * lane] = u[0];
+                wred[warp * 64 + 2 * lane + 1] = u[1];
             }
             __syncthreads();
             if (tid < 64) {
@@ -606,28 +671,30 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
                 l_part[0] *= alpha[2 * lane];
                 l_part[1] *= alpha[2 * lane + 1];
             }
-            // ---- P' = 2^(u - rho) (fp16) and row sums ----
+            // ---- P' = 2^(u - rho) (fp16, 8 heads per 16-byte store) and row sums ----
             {
+                float u[64];
+                tmem_ld64(tmem_s + lane_off, u);
                 const float rj_inv = ldexpf(1.0f, -Rj);
-                uint32_t pk[32];
-                float ls[64];
-#pragma unroll
-                for (int h = 0; h < 64; h += 2) {
-                    const float p0 = exp2f(u[h] - rho[h]);
-                    const float p1 = exp2f(u[h + 1] - rho[h + 1]);
-                    __half2 hh = __floats2half2_rn(p0, p1);
-                    pk[h / 2] = *reinterpret_cast<uint32_t *>(&hh);
-                    ls[h] = p0 * rj_inv;
-                    ls[h + 1] = p1 * rj_inv;
-                }
 #pragma unroll
                 for (int cc = 0; cc < 8; ++cc) {
+                    uint32_t pk[4];
+#pragma unroll
+                    for (int q2 = 0; q2 < 4; ++q2) {
+                        const int h = 8 * cc + 2 * q2;
+                        const float p0 = valid ? exp2f(fmaf(u[h], cj, rjf) - rho[h]) : 0.f;
+                        const float p1 = valid ? exp2f(fmaf(u[h + 1], cj, rjf) - rho[h + 1]) : 0.f;
+                        __half2 hh = __floats2half2_rn(p0, p1);
+                        pk[q2] = *reinterpret_cast<uint32_t *>(&hh);
+                        u[h] = p0 * rj_inv;      // row-sum term, in place
+                        u[h + 1] = p1 * rj_inv;
+                    }
                     const uint32_t off = (uint32_t)((tid >> 3) * 1024 + (tid & 7) * 128 + ((cc ^ (tid & 7)) << 4));
-                    *reinterpret_cast<uint4 *>(P + off) = make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
+                    *reinterpret_cast<uint4 *>(P + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 }
-                transpose_reduce64<false>(ls);
-                l_part[0] += ls[0];
-                l_part[1] += ls[1];
+                transpose_reduce64<false>(u);
+                l_part[0] += u[0];
+                l_part[1] += u[1];
             }
             fence_async_smem();
             tc_fence_before();
@@ -700,62 +767,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
                 a.part_rho[(size_t)b_slot * kHeads + tid] = rho[tid];
                 a.part_l[(size_t)b_slot * kHeads + tid] = alpha[tid];
             }
-            __threadfence();
-            __syncthreads();
-            if (tid == 0) {
-                // completion is counted in tiles: the CTA that brings the count to
-                // the query's tile total is the last one and merges
-                const long long Ti = a.tprefix[i], Ti1 = a.tprefix[i + 1];
-                const uint32_t seg_tiles = (uint32_t)(seg_end - seg_begin);
-                const uint32_t prev = atomicAdd(a.counters + i, seg_tiles);
-                flags[1] = (prev + seg_tiles == (uint32_t)(Ti1 - Ti)) ? 1 : 0;
-                if (flags[1]) {
-                    // partial slots of every CTA whose (non-empty) range meets [Ti, Ti1)
-                    int *slots = reinterpret_cast<int *>(wred);
-                    int np = 0;
-                    const int c_first = (int)(((Ti + 1) * G - 1) / T);
-                    const int c_last = (int)((Ti1 * G - 1) / T);
-                    for (int cc = c_first; cc <= c_last && np < 4 * 64; ++cc) {
-                        const long long rb = T * cc / G, re = T * (cc + 1) / G;
-                        if (rb >= re) continue;
-                        slots[np++] = 2 * cc + (rb >= Ti ? 0 : 1);
-                    }
-                    flags[3] = np;
-                }
-            }
-            __syncthreads();
-            if (flags[1]) {  // last CTA of this query: merge every partial
-                __threadfence();
-                const int np = flags[3];
-                const int *slots = reinterpret_cast<const int *>(wred);
-                float *wts = reinterpret_cast<float *>(E);  // E' is free now: [np][64] weights
-                if (tid < 64) {
-                    float rmax = -INFINITY;
-                    for (int p = 0; p < np; ++p)
-                        rmax = fmaxf(rmax, __ldcg(a.part_rho + (size_t)slots[p] * kHeads + tid));
-                    float lsum = 0.f;
-                    for (int p = 0; p < np; ++p) {
-                        const float wgt = exp2f(__ldcg(a.part_rho + (size_t)slots[p] * kHeads + tid) - rmax);
-                        wts[p * 64 + tid] = wgt;
-                        lsum += wgt * __ldcg(a.part_l + (size_t)slots[p] * kHeads + tid);
-                    }
-                    rho[tid] = rmax;
-                    alpha[tid] = lsum;
-                }
-                __syncthreads();
-                for (int k = tid; k < a.H * D; k += kThreads) {
-                    const int h = k / D;
-                    float acc = 0.f;
-                    for (int p = 0; p < np; ++p)
-                        acc += wts[p * 64 + h] * __ldcg(a.part_o + (size_t)slots[p] * kHeads * D + k);
-                    const float l = alpha[h];
-                    a.out[(size_t)i * a.H * D + k] = l > 0.f ? acc / l : 0.f;
-                }
-                if (a.lse && tid < a.H) {
-                    const float l = alpha[tid];
-                    a.lse[(size_t)i * a.H + tid] = l > 0.f ? (rho[tid] + log2f(l)) * 0.69314718055994531f : -INFINITY;
-                }
-            }
         }
         __syncthreads();
         tc_fence_before();
@@ -783,7 +794,6 @@ size_t attend_workspace_bytes(int Nq, int D, int num_ctas) {
     take(4 * (size_t)Nq);            // ctiles
     take(4 * (size_t)Nq);            // wlen
     take(8 * (size_t)(Nq + 1));      // tprefix
-    take(4 * (size_t)Nq);            // counters
     take(4 * (size_t)2 * num_ctas * kHeads * D);  // part_o
     take(4 * (size_t)2 * num_ctas * kHeads);      // part_rho
     take(4 * (size_t)2 * num_ctas * kHeads);      // part_l
@@ -808,7 +818,6 @@ cudaError_t launch_attend(const csa_cache &c, const void *q, int Nq, int H, cons
     int32_t *ctiles = reinterpret_cast<int32_t *>(take(4 * (size_t)Nq));
     int32_t *wlen = reinterpret_cast<int32_t *>(take(4 * (size_t)Nq));
     long long *tprefix = reinterpret_cast<long long *>(take(8 * (size_t)(Nq + 1)));
-    uint32_t *counters = reinterpret_cast<uint32_t *>(take(4 * (size_t)Nq));
     a.part_o = reinterpret_cast<float *>(take(4 * (size_t)2 * num_ctas * kHeads * D));
     a.part_rho = reinterpret_cast<float *>(take(4 * (size_t)2 * num_ctas * kHeads));
     a.part_l = reinterpret_cast<float *>(take(4 * (size_t)2 * num_ctas * kHeads));
@@ -827,15 +836,13 @@ cudaError_t launch_attend(const csa_cache &c, const void *q, int Nq, int H, cons
     a.ctiles = ctiles;
     a.wlen = wlen;
     a.tprefix = tprefix;
-    a.counters = counters;
     a.Nq = Nq;
     a.H = H;
     a.cap = c.capacity;
     a.topk = topk;
     a.scale_log2 = softmax_scale * 1.4426950408889634f;
 
-    cudaError_t err = cudaMemsetAsync(counters, 0, 4 * (size_t)Nq, s);
-    if (err != cudaSuccess) return err;
+    cudaError_t err;
     attend_schedule_kernel<<<1, 1024, 0, s>>>(q_offsets, sel_idx ? nullptr : q_pos, c.n_blocks,
                                               win_kv ? win_len : nullptr, c.batch, Nq, c.block, c.capacity, topk, max_win, H, D,
                                               req, nent, ctiles, wlen, tprefix, out, lse, c.status);
@@ -853,6 +860,9 @@ cudaError_t launch_attend(const csa_cache &c, const void *q, int Nq, int H, cons
     } else {
         return cudaErrorInvalidValue;
     }
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    attend_merge_kernel<<<dim3(Nq, (H + kMergeHeads - 1) / kMergeHeads), 256, 0, s>>>(
+        tprefix, Nq, H, D, num_ctas, a.part_o, a.part_rho, a.part_l, out, lse);
     return cudaGetLastError();
 }
 

@@ -7,9 +7,10 @@
 // E2M1 elements). Pooling form, gate and E8M0/32 scale: the library's stated
 // readings (see include/csa.h).
 //
-// One warp builds one block. Lane l owns E = D/32 consecutive channels
-// [l*E, l*E+E) and EI = dI/32 consecutive indexer channels, so every token row
-// is read as one coalesced warp-wide load. The gate softmax is computed online
+// One warp builds one block (eight warps share a block when m >= 32). Lane l
+// owns E = D/32 consecutive channels [l*E, l*E+E) and EI = dI/32 consecutive
+// indexer channels, so every token row is read as one coalesced warp-wide load;
+// four tokens are loaded per step. The gate softmax is computed online
 // (running max and rescaled sums) in a single pass over the m tokens. The
 // kernel is HBM-bound: it reads m*(D+dI)*2 bytes and writes D/2 + D/32 + key
 // bytes per block.
@@ -88,23 +89,30 @@ struct CompressArgs {
     int idx_e4m3;
 };
 
-// E channels per lane (D = 32*E), EI indexer channels per lane (0 = no indexer keys).
-template <int E, int EI>
-__global__ void __launch_bounds__(kWarpsPerCta * kWarp)
+// E channels per lane (D = 32*E), EI indexer channels per lane (0 = no
+// indexer keys), WPB warps per block: WPB = 1 puts four independent blocks in
+// a CTA; WPB = 8 splits one block's tokens over eight warps (large m), whose
+// online-softmax states are then combined through shared memory.
+template <int E, int EI, int WPB>
+__global__ void __launch_bounds__(WPB == 1 ? kWarpsPerCta * kWarp : WPB * kWarp)
 pool_quantize_kernel(CompressArgs a) {
+    constexpr int EK = EI > 0 ? EI : 2;
+    constexpr int kChunk = 4;  // tokens in flight per warp step
     const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
     const int b = blockIdx.y;
-    const int jb = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
+    const int jb = WPB == 1 ? blockIdx.x * kWarpsPerCta + warp : blockIdx.x;
+    const int wib = WPB == 1 ? 0 : warp;  // warp index inside the block's team
     const int t_begin = a.tok_offsets[b];
     const int count = a.tok_offsets[b + 1] - t_begin;
     const int base = a.n_blocks[b];
     if (count < 0 || count % a.m != 0) {
-        if (jb == 0 && lane == 0) flag(a.status, CSA_DEV_TOKEN_COUNT);
+        if (jb == 0 && threadIdx.x == 0) flag(a.status, CSA_DEV_TOKEN_COUNT);
         return;
     }
     const int nb = count / a.m;
     if ((long long)base + nb > a.cap) {
-        if (jb == 0 && lane == 0) flag(a.status, CSA_DEV_CAPACITY);
+        if (jb == 0 && threadIdx.x == 0) flag(a.status, CSA_DEV_CAPACITY);
         return;
     }
     if (jb >= nb) return;
@@ -113,43 +121,91 @@ pool_quantize_kernel(CompressArgs a) {
 #pragma unroll
     for (int k = 0; k < E; ++k) wg[k] = __ldg(a.gate_w + lane * E + k);
 
-    // Online softmax over the block's tokens: mu = running max logit,
+    // Online softmax over this warp's tokens: mu = running max logit,
     // den = sum exp(g - mu), acc = sum exp(g - mu) * x.
-    float acc[E], acck[EI > 0 ? EI : 1];
+    float acc[E], acck[EK];
     float mu = -INFINITY, den = 0.f;
 #pragma unroll
     for (int k = 0; k < E; ++k) acc[k] = 0.f;
 #pragma unroll
-    for (int k = 0; k < (EI > 0 ? EI : 1); ++k) acck[k] = 0.f;
+    for (int k = 0; k < EK; ++k) acck[k] = 0.f;
 
     const long long tok0 = (long long)t_begin + (long long)jb * a.m;
-    for (int t = 0; t < a.m; ++t) {
-        float x[E];
-        load_bf16<E>(a.kv_tok + (tok0 + t) * a.D + lane * E, x);
-        float part = 0.f;
+    for (int c0 = wib * kChunk; c0 < a.m; c0 += WPB * kChunk) {
+        float x[kChunk][E], xk[kChunk][EK], g[kChunk];
 #pragma unroll
-        for (int k = 0; k < E; ++k) part = fmaf(x[k], wg[k], part);
-        const float g = warp_sum(part);
-        float xk[EI > 0 ? EI : 2];
-        if constexpr (EI > 0) load_bf16<EI>(a.idx_tok + (tok0 + t) * a.dI + lane * EI, xk);
-        if (g > mu) {  // new maximum: rescale what has been accumulated
-            const float r = (mu == -INFINITY) ? 0.f : expf(mu - g);
+        for (int u = 0; u < kChunk; ++u) {
+            if (c0 + u < a.m) {
+                load_bf16<E>(a.kv_tok + (tok0 + c0 + u) * a.D + lane * E, x[u]);
+                if constexpr (EI > 0) load_bf16<EI>(a.idx_tok + (tok0 + c0 + u) * a.dI + lane * EI, xk[u]);
+            }
+        }
+        float cmax = -INFINITY;
+#pragma unroll
+        for (int u = 0; u < kChunk; ++u) {
+            if (c0 + u < a.m) {
+                float part = 0.f;
+#pragma unroll
+                for (int k = 0; k < E; ++k) part = fmaf(x[u][k], wg[k], part);
+                g[u] = warp_sum(part);
+                cmax = fmaxf(cmax, g[u]);
+            }
+        }
+        if (cmax > mu) {  // new maximum: rescale what has been accumulated
+            const float r = (mu == -INFINITY) ? 0.f : expf(mu - cmax);
             den *= r;
 #pragma unroll
             for (int k = 0; k < E; ++k) acc[k] *= r;
-            if constexpr (EI > 0) {
 #pragma unroll
-                for (int k = 0; k < EI; ++k) acck[k] *= r;
-            }
-            mu = g;
+            for (int k = 0; k < EK; ++k) acck[k] *= r;
+            mu = cmax;
         }
-        const float p = expf(g - mu);
-        den += p;
 #pragma unroll
-        for (int k = 0; k < E; ++k) acc[k] = fmaf(p, x[k], acc[k]);
-        if constexpr (EI > 0) {
+        for (int u = 0; u < kChunk; ++u) {
+            if (c0 + u < a.m) {
+                const float p = expf(g[u] - mu);
+                den += p;
 #pragma unroll
-            for (int k = 0; k < EI; ++k) acck[k] = fmaf(p, xk[k], acck[k]);
+                for (int k = 0; k < E; ++k) acc[k] = fmaf(p, x[u][k], acc[k]);
+                if constexpr (EI > 0) {
+#pragma unroll
+                    for (int k = 0; k < EI; ++k) acck[k] = fmaf(p, xk[u][k], acck[k]);
+                }
+            }
+        }
+    }
+
+    if constexpr (WPB > 1) {
+        // combine the warps' partial softmax states; warp 0 finishes the block
+        __shared__ float s_mu[WPB], s_den[WPB];
+        __shared__ float s_acc[WPB][32 * E];
+        __shared__ float s_acck[WPB][32 * EK];
+        if (lane == 0) {
+            s_mu[warp] = mu;
+            s_den[warp] = den;
+        }
+#pragma unroll
+        for (int k = 0; k < E; ++k) s_acc[warp][lane * E + k] = acc[k];
+#pragma unroll
+        for (int k = 0; k < EK; ++k) s_acck[warp][lane * EK + k] = acck[k];
+        __syncthreads();
+        if (warp != 0) return;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < WPB; ++w) M = fmaxf(M, s_mu[w]);
+        den = 0.f;
+#pragma unroll
+        for (int k = 0; k < E; ++k) acc[k] = 0.f;
+#pragma unroll
+        for (int k = 0; k < EK; ++k) acck[k] = 0.f;
+#pragma unroll
+        for (int w = 0; w < WPB; ++w) {
+            const float f = (s_mu[w] == -INFINITY) ? 0.f : expf(s_mu[w] - M);
+            den = fmaf(s_den[w], f, den);
+#pragma unroll
+            for (int k = 0; k < E; ++k) acc[k] = fmaf(s_acc[w][lane * E + k], f, acc[k]);
+#pragma unroll
+            for (int k = 0; k < EK; ++k) acck[k] = fmaf(s_acck[w][lane * EK + k], f, acck[k]);
         }
     }
 
@@ -215,17 +271,24 @@ __global__ void commit_kernel(const int32_t *tok_offsets, int32_t *n_blocks, int
     }
 }
 
-template <int E>
-cudaError_t launch_e(const CompressArgs &a, dim3 grid, cudaStream_t s) {
-    const dim3 block(kWarpsPerCta * kWarp);
+template <int E, int WPB>
+cudaError_t launch_ew(const CompressArgs &a, dim3 grid, cudaStream_t s) {
+    const dim3 block(WPB == 1 ? kWarpsPerCta * kWarp : WPB * kWarp);
     switch (a.idx_key ? a.dI / 32 : 0) {
-        case 0: pool_quantize_kernel<E, 0><<<grid, block, 0, s>>>(a); break;
-        case 2: pool_quantize_kernel<E, 2><<<grid, block, 0, s>>>(a); break;
-        case 4: pool_quantize_kernel<E, 4><<<grid, block, 0, s>>>(a); break;
-        case 8: pool_quantize_kernel<E, 8><<<grid, block, 0, s>>>(a); break;
+        case 0: pool_quantize_kernel<E, 0, WPB><<<grid, block, 0, s>>>(a); break;
+        case 2: pool_quantize_kernel<E, 2, WPB><<<grid, block, 0, s>>>(a); break;
+        case 4: pool_quantize_kernel<E, 4, WPB><<<grid, block, 0, s>>>(a); break;
+        case 8: pool_quantize_kernel<E, 8, WPB><<<grid, block, 0, s>>>(a); break;
         default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();
+}
+
+// m >= 32: eight warps per block; otherwise four blocks per CTA, one warp each
+template <int E>
+cudaError_t launch_e(const CompressArgs &a, int max_blocks, int batch, cudaStream_t s) {
+    if (a.m >= 32) return launch_ew<E, 8>(a, dim3(max_blocks, batch), s);
+    return launch_ew<E, 1>(a, dim3((max_blocks + kWarpsPerCta - 1) / kWarpsPerCta, batch), s);
 }
 
 }  // namespace
@@ -250,13 +313,12 @@ cudaError_t launch_compress(const csa_cache &c, const void *kv_tok, const void *
     a.idx_e4m3 = c.idx_dtype == CSA_IDX_E4M3;
     const int max_blocks = (n_tokens + c.block - 1) / c.block;
     if (max_blocks > 0) {
-        dim3 grid((max_blocks + kWarpsPerCta - 1) / kWarpsPerCta, c.batch);
         cudaError_t err;
         switch (c.dim / 32) {
-            case 2: err = launch_e<2>(a, grid, s); break;
-            case 4: err = launch_e<4>(a, grid, s); break;
-            case 8: err = launch_e<8>(a, grid, s); break;
-            case 16: err = launch_e<16>(a, grid, s); break;
+            case 2: err = launch_e<2>(a, max_blocks, c.batch, s); break;
+            case 4: err = launch_e<4>(a, max_blocks, c.batch, s); break;
+            case 8: err = launch_e<8>(a, max_blocks, c.batch, s); break;
+            case 16: err = launch_e<16>(a, max_blocks, c.batch, s); break;
             default: return cudaErrorInvalidValue;
         }
         if (err != cudaSuccess) return err;

@@ -22,7 +22,7 @@ cudaError_t launch_attend(const csa_cache &c, const void *q, int Nq, int H, cons
 
 namespace {
 
-constexpr int kMaxCapacity = 1 << 20;  // block indices are resolved on 20 bits by the top-k select
+constexpr int kMaxCapacity = 1 << 19;  // the top-k select keeps two bitmaps of this many bits in shared memory
 constexpr int kMaxTopk = 4096;
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }

@@ -23,14 +23,22 @@
 //                     bound by HBM. It writes the fp32 score of every key and a
 //                     4096-bin histogram of the top 12 bits of each score's
 //                     order-preserving key.
-//   select_pass_kernel  many CTAs per query: from the histogram, the bin b*
-//                     holding the k-th largest score; marks every key above b*
-//                     in a per-query bitmap and appends the keys inside b* to a
-//                     candidate list, with a histogram of their next 12 bits.
-//   select_final_kernel one CTA per query: radix refinement among the
-//                     candidates (remaining score bits, then the block index
-//                     for exact ties, lower index first), then the bitmap is
-//                     compacted into ascending block indices padded with -1.
+//                     The CTA that completes a query's scan (a group counter,
+//                     no waiting) finds from the histogram the bin b* holding
+//                     the k-th largest key.
+//   select_pass_kernel  a wide grid over every score row: 128 scores per warp
+//                     step (float4 loads); keys above b* become bitmap words
+//                     (built with warp shuffles, stored plainly: each word has
+//                     one writer); keys inside b* are appended to a short
+//                     per-query candidate list (warp-aggregated atomics).
+//   select_final_kernel one CTA per query: exact selection among the b*
+//                     members in shared memory -- radix levels on the remaining
+//                     12 + 8 key bits while keys still differ, then, for members
+//                     tied on the whole key, the lowest block indices in index
+//                     order from a second bitmap -- and the bitmap is compacted
+//                     with warp scans into ascending block indices padded with
+//                     -1. If a query's candidate list overflowed, the selection
+//                     reads its full score row instead.
 // Every float comparison is on the score's order-preserving uint32 key
 // (-0 folded into +0), so selection is exact for the scores computed here.
 #include <cuda_bf16.h>
@@ -46,16 +54,19 @@ namespace {
 constexpr int kBins = 4096;        // histogram bins per level (12 bits)
 constexpr int kScanThreads = 256;  // 8 warps
 constexpr int kSelThreads = 1024;
-constexpr int kPassSlices = 16;    // CTAs per query in select_pass_kernel
+constexpr int kPassThreads = 256;
+constexpr int kCandCap = 32768;    // candidate slots per query (members of the threshold bin)
 
 // ---------------------------------------------------------------- workspace
 struct IndexWs {
     int32_t *req;        // [Nq]
     int32_t *n_vis;      // [Nq]
     long long *gprefix;  // [Nq+1]
+    int32_t *thresh;     // [Nq][3]: keys with a bin above thresh[0] are selected, thresh[1] of them;
+                         //          keys in bin thresh[2] (-1: none) are refined
     // zeroed region starts here
+    uint32_t *done;      // [Nq] key groups scanned so far
     uint32_t *hist1;     // [Nq][4096]
-    uint32_t *hist2;     // [Nq][4096]
     uint32_t *bitmap;    // [Nq][words]
     uint32_t *ncand;     // [Nq]
     // end of zeroed region
@@ -70,7 +81,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 size_t carve(void *base, int Nq, int cap, IndexWs *w) {
     const int words = (cap + 31) / 32;
-    const int ccap = 32768;
+    const int ccap = kCandCap;
     size_t off = 0;
     auto take = [&](size_t bytes) {
         size_t o = off;
@@ -80,9 +91,10 @@ size_t carve(void *base, int Nq, int cap, IndexWs *w) {
     size_t o_req = take(sizeof(int32_t) * Nq);
     size_t o_nvis = take(sizeof(int32_t) * Nq);
     size_t o_gp = take(sizeof(long long) * (Nq + 1));
+    size_t o_th = take(sizeof(int32_t) * 3 * (size_t)Nq);
     size_t z0 = off;
+    size_t o_dn = take(sizeof(uint32_t) * Nq);
     size_t o_h1 = take(sizeof(uint32_t) * kBins * (size_t)Nq);
-    size_t o_h2 = take(sizeof(uint32_t) * kBins * (size_t)Nq);
     size_t o_bm = take(sizeof(uint32_t) * (size_t)words * Nq);
     size_t o_nc = take(sizeof(uint32_t) * Nq);
     size_t z1 = off;
@@ -94,8 +106,9 @@ size_t carve(void *base, int Nq, int cap, IndexWs *w) {
         w->req = reinterpret_cast<int32_t *>(b + o_req);
         w->n_vis = reinterpret_cast<int32_t *>(b + o_nvis);
         w->gprefix = reinterpret_cast<long long *>(b + o_gp);
+        w->thresh = reinterpret_cast<int32_t *>(b + o_th);
+        w->done = reinterpret_cast<uint32_t *>(b + o_dn);
         w->hist1 = reinterpret_cast<uint32_t *>(b + o_h1);
-        w->hist2 = reinterpret_cast<uint32_t *>(b + o_h2);
         w->bitmap = reinterpret_cast<uint32_t *>(b + o_bm);
         w->ncand = reinterpret_cast<uint32_t *>(b + o_nc);
         w->cand_key = reinterpret_cast<uint32_t *>(b + o_ck);
@@ -110,7 +123,8 @@ size_t carve(void *base, int Nq, int cap, IndexWs *w) {
 
 // ---------------------------------------------------------------- schedule
 __global__ void schedule_kernel(const int32_t *q_offsets, const int32_t *q_pos, const int32_t *n_blocks,
-                                int batch, int Nq, int m, int cap, int32_t *req, int32_t *n_vis, long long *gprefix) {
+                                int batch, int Nq, int m, int cap, int topk, int32_t *req, int32_t *n_vis,
+                                long long *gprefix, int32_t *thresh) {
     __shared__ long long red[32];
     __shared__ long long round_total;
     long long carry = 0;
@@ -123,6 +137,11 @@ __global__ void schedule_kernel(const int32_t *q_offsets, const int32_t *q_pos, 
             req[i] = b;
             n_vis[i] = n;
             groups = (n + 15) / 16;
+            if (topk >= n) {  // every visible block is selected; no threshold needed
+                thresh[3 * i] = -1;
+                thresh[3 * i + 1] = n;
+                thresh[3 * i + 2] = -1;
+            }
         }
         const long long incl = block_inclusive_scan<long long>(groups, red);
         if (i < Nq) gprefix[i + 1] = carry + incl;
@@ -133,6 +152,44 @@ __global__ void schedule_kernel(const int32_t *q_offsets, const int32_t *q_pos, 
         carry += round_total;
         __syncthreads();
     }
+}
+
+// ---------------------------------------------------------------- radix helper
+struct BinPick {
+    int bin;          // chosen digit
+    uint32_t above;   // elements with a larger digit
+    uint32_t at;      // elements with this digit
+};
+
+// Largest digit d such that count(digit >= d) >= need, in a histogram of
+// nbins (<= 4096) bins held in shared memory. All threads get the result.
+__device__ BinPick pick_bin(const uint32_t *h, int nbins, uint32_t need, uint32_t *scan_smem, BinPick *out) {
+    const int per = (nbins + blockDim.x - 1) / blockDim.x;
+    const int top = nbins - 1 - (int)threadIdx.x * per;  // this thread: bins [top-per+1, top]
+    const volatile uint32_t *vh = h;
+    uint32_t mine = 0;
+    for (int k = 0; k < per; ++k)
+        if (top - k >= 0) mine += vh[top - k];
+    const uint32_t incl = block_inclusive_scan<uint32_t>(mine, scan_smem);
+    const uint32_t excl = incl - mine;
+    if (excl < need && incl >= need) {
+        uint32_t run = excl;
+        for (int k = 0; k < per; ++k) {
+            const int d = top - k;
+            if (d < 0) break;
+            if (run + vh[d] >= need) {
+                out->bin = d;
+                out->above = run;
+                out->at = vh[d];
+                break;
+            }
+            run += vh[d];
+        }
+    }
+    __syncthreads();
+    BinPick r = *out;
+    __syncthreads();
+    return r;
 }
 
 // ---------------------------------------------------------------- scan
@@ -164,7 +221,9 @@ struct ScanArgs {
     const long long *gprefix;
     float *scores;                // [Nq][cap]
     uint32_t *hist1;              // [Nq][4096]
-    int Nq, H_I, cap;
+    uint32_t *done;               // [Nq]
+    int32_t *thresh;              // [Nq][3]
+    int Nq, H_I, cap, topk;
 };
 
 // Dimension permutation. The dot product sums over all d_I channels, so the
@@ -187,6 +246,9 @@ template <bool E4M3, int KS>
 __global__ void __launch_bounds__(kScanThreads, 2) scan_kernel(ScanArgs a) {
     using C = ScanCfg<E4M3, KS>;
     __shared__ uint32_t hist[kBins];
+    __shared__ uint32_t scan_smem[32];
+    __shared__ BinPick pick;
+    __shared__ int last_flag;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
     const long long NG = a.gprefix[a.Nq];
@@ -335,6 +397,28 @@ __global__ void __launch_bounds__(kScanThreads, 2) scan_kernel(ScanArgs a) {
             const uint32_t c = vh[k];
             if (c) atomicAdd(gh + k, c);
         }
+        // the CTA that completes a query's scan finds its k-th key bin (no waiting:
+        // groups are counted, and only the one that brings the count to the total acts)
+        __threadfence();
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            const uint32_t total = (uint32_t)(a.gprefix[i + 1] - a.gprefix[i]);
+            const uint32_t mine = (uint32_t)nloc;
+            last_flag = (atomicAdd(a.done + i, mine) + mine == total) && (a.topk < n);
+        }
+        __syncthreads();
+        if (last_flag) {
+            __threadfence();
+            for (int k = threadIdx.x; k < kBins; k += kScanThreads) hist[k] = __ldcg(gh + k);
+            __syncthreads();
+            const BinPick p = pick_bin(hist, kBins, (uint32_t)a.topk, scan_smem, &pick);
+            if (threadIdx.x == 0) {
+                const bool all_at = p.above + p.at == (uint32_t)a.topk;  // the whole bin is selected
+                a.thresh[3 * i] = all_at ? p.bin - 1 : p.bin;            // bins above this are selected
+                a.thresh[3 * i + 1] = (int)p.above;
+                a.thresh[3 * i + 2] = all_at ? -1 : p.bin;                // bin refined by the final kernel
+            }
+        }
         __syncthreads();
         gb = seg_end;
     }
@@ -344,206 +428,303 @@ __global__ void __launch_bounds__(kScanThreads, 2) scan_kernel(ScanArgs a) {
 struct SelArgs {
     const int32_t *n_vis;
     const float *scores;
-    uint32_t *hist1, *hist2, *bitmap, *ncand, *cand_key;
+    const uint32_t *hist1;
+    int32_t *thresh;
+    uint32_t *bitmap, *ncand, *cand_key;
     int32_t *cand_idx;
     int32_t *sel_idx;
     int Nq, cap, topk, words, ccap;
+    int smem_cands;  // candidates that fit in shared memory after the bitmap
 };
 
-struct BinPick {
-    int bin;          // chosen digit
-    uint32_t above;   // elements with a larger digit
-    uint32_t at;      // elements with this digit
-};
-
-// Largest digit d such that count(digit >= d) >= need, in a histogram of
-// nbins (<= 4096) bins held in shared memory. All threads get the result.
-__device__ BinPick pick_bin(const uint32_t *h, int nbins, uint32_t need, uint32_t *scan_smem, BinPick *out) {
-    const int per = (nbins + blockDim.x - 1) / blockDim.x;
-    // thread t owns bins [base, base+per) counted from the top
-    const int rt = threadIdx.x;  // rank from the top
-    const int top = nbins - 1 - rt * per;
-    uint32_t mine = 0;
-    for (int k = 0; k < per; ++k)
-        if (top - k >= 0) mine += h[top - k];
-    const uint32_t incl = block_inclusive_scan<uint32_t>(mine, scan_smem);
-    const uint32_t excl = incl - mine;
-    if (excl < need && incl >= need) {
-        uint32_t run = excl;
-        for (int k = 0; k < per; ++k) {
-            const int d = top - k;
-            if (d < 0) break;
-            if (run + h[d] >= need) {
-                out->bin = d;
-                out->above = run;
-                out->at = h[d];
-                break;
-            }
-            run += h[d];
-        }
-    }
-    __syncthreads();
-    BinPick r = *out;
-    __syncthreads();
-    return r;
-}
-
-__device__ __forceinline__ void mark(uint32_t *bm, int j) { atomicOr(bm + (j >> 5), 1u << (j & 31)); }
-
-__global__ void __launch_bounds__(kSelThreads) select_pass_kernel(SelArgs a) {
-    __shared__ uint32_t h[kBins];
-    __shared__ uint32_t h2[kBins];
-    __shared__ uint32_t scan_smem[32];
-    __shared__ BinPick pick;
+// Keys above the threshold bin -> bitmap; keys in it -> candidate list.
+// Grid: (chunks of 128 x kPassThreads/32 scores, Nq).
+__global__ void __launch_bounds__(kPassThreads) select_pass_kernel(SelArgs a) {
     const int i = blockIdx.y;
     const int n = a.n_vis[i];
-    const int K = min(a.topk, n);
-    if (K == n) return;  // everything visible is selected; the final kernel handles it
-    for (int k = threadIdx.x; k < kBins; k += blockDim.x) {
-        h[k] = a.hist1[(size_t)i * kBins + k];
-        h2[k] = 0;
-    }
-    __syncthreads();
-    const BinPick p = pick_bin(h, kBins, (uint32_t)K, scan_smem, &pick);
-    const bool take_all_at = (p.above + p.at == (uint32_t)K);
-    uint32_t *bm = a.bitmap + (size_t)i * a.words;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int above_bin = a.thresh[3 * i];      // select keys whose bin is > above_bin
+    const int cand_bin = a.thresh[3 * i + 2];   // refine keys whose bin == cand_bin
+    if (above_bin < 0 && cand_bin < 0) return;  // everything selected: the final kernel writes it
     const float *s = a.scores + (size_t)i * a.cap;
-    // slice of the row handled by this CTA
-    const int per = (n + gridDim.x - 1) / gridDim.x;
-    const int j0 = blockIdx.x * per, j1 = min(n, j0 + per);
-    for (int j = j0 + threadIdx.x; j < j1; j += blockDim.x) {
-        const uint32_t key = ordered_key(s[j]);
-        const int d = (int)(key >> 20);
-        if (d > p.bin || (d == p.bin && take_all_at)) {
-            mark(bm, j);
-        } else if (d == p.bin) {
-            atomicAdd(&h2[(key >> 8) & 0xFFF], 1u);
-            const uint32_t pos = atomicAdd(a.ncand + i, 1u);
-            if (pos < (uint32_t)a.ccap) {
-                a.cand_key[(size_t)i * a.ccap + pos] = key;
-                a.cand_idx[(size_t)i * a.ccap + pos] = j;
-            }
+    uint32_t *bm = a.bitmap + (size_t)i * a.words;
+    const int warps_total = gridDim.x * (kPassThreads / 32);
+    for (int base = (blockIdx.x * (kPassThreads / 32) + warp) * 128; base < n; base += warps_total * 128) {
+        // lane l holds scores [base + 4l, base + 4l + 4)
+        const int j0 = base + 4 * lane;
+        float v[4];
+        if (j0 + 3 < n && ((((size_t)i * a.cap + j0) & 3) == 0)) {
+            const float4 f = __ldcg(reinterpret_cast<const float4 *>(s + j0));
+            v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+        } else {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) v[u] = (j0 + u < n) ? __ldcg(s + j0 + u) : -INFINITY;
         }
-    }
-    __syncthreads();
-    if (!take_all_at) {
-        const volatile uint32_t *vh2 = h2;
-        for (int k = threadIdx.x; k < kBins; k += blockDim.x) {
-            const uint32_t c = vh2[k];
-            if (c) atomicAdd(a.hist2 + (size_t)i * kBins + k, c);
+        uint32_t nib = 0, cmask = 0;
+        uint32_t key[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            key[u] = ordered_key(v[u]);
+            const int d = (int)(key[u] >> 20);
+            const bool ok = j0 + u < n;
+            if (ok && d > above_bin) nib |= 1u << u;
+            if (ok && d == cand_bin) cmask |= 1u << u;
+        }
+        // word w of this 128-score chunk = nibbles of lanes 8w .. 8w+7
+        uint32_t word = nib << (4 * (lane & 7));
+        word |= __shfl_xor_sync(0xffffffffu, word, 1);
+        word |= __shfl_xor_sync(0xffffffffu, word, 2);
+        word |= __shfl_xor_sync(0xffffffffu, word, 4);
+        if ((lane & 7) == 0 && base + 32 * (lane >> 3) < n) bm[(base >> 5) + (lane >> 3)] = word;
+        // candidates: warp-aggregated append
+        const uint32_t cnt = __popc(cmask);
+        uint32_t incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        const uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
+        if (total) {
+            uint32_t at = 0;
+            if (lane == 31) at = atomicAdd(a.ncand + i, total);
+            at = __shfl_sync(0xffffffffu, at, 31);
+            uint32_t pos = at + incl - cnt;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                if (cmask & (1u << u)) {
+                    if (pos < (uint32_t)a.ccap) {
+                        a.cand_key[(size_t)i * a.ccap + pos] = key[u];
+                        a.cand_idx[(size_t)i * a.ccap + pos] = j0 + u;
+                    }
+                    ++pos;
+                }
+            }
         }
     }
 }
 
-// Digits of the refinement levels after the first (key bits 31..20):
-//   level 1: key bits 19..8   level 2: key bits 7..0
-//   level 3: 4095 - block index bits 19..8   level 4: 255 - block index bits 7..0
-// (the block-index digits are reversed so that "largest digit first" takes the
-// lower index first). The prefix of a level is the digits of all earlier ones.
-__device__ __forceinline__ int level_digit(int level, uint32_t key, int j) {
-    switch (level) {
-        case 1: return (int)((key >> 8) & 0xFFF);
-        case 2: return (int)(key & 0xFF);
-        case 3: return 4095 - ((j >> 8) & 0xFFF);
-        default: return 255 - (j & 0xFF);
-    }
+// Warp-scan compaction helpers over a shared bitmap of `words` words, split
+// into one contiguous run of words per warp.
+struct WordRun {
+    int begin, end;
+};
+__device__ __forceinline__ WordRun warp_run(int words) {
+    const int nwarps = blockDim.x >> 5, warp = threadIdx.x >> 5;
+    const int wpw = (words + nwarps - 1) / nwarps;
+    const int b = min(words, warp * wpw);
+    return {b, min(words, b + wpw)};
 }
-__device__ __forceinline__ int level_bins(int level) { return (level == 1 || level == 3) ? 4096 : 256; }
+
+// Number of set bits of every warp's run, as exclusive prefix sums in warp_base[]
+// (and the total in *total). Bits at or beyond n are ignored.
+__device__ void run_prefix(const volatile uint32_t *bits, int words, int n, uint32_t *warp_base, uint32_t *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    const WordRun r = warp_run(words);
+    uint32_t cnt = 0;
+    for (int w = r.begin + lane; w < r.end; w += 32) {
+        uint32_t b = bits[w];
+        if (w == words - 1 && (n & 31)) b &= (1u << (n & 31)) - 1u;
+        cnt += __popc(b);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+    if (lane == 0) warp_base[warp] = cnt;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t run = 0;
+        for (int w = 0; w < nwarps; ++w) {
+            const uint32_t c = warp_base[w];
+            warp_base[w] = run;
+            run += c;
+        }
+        *total = run;
+    }
+    __syncthreads();
+}
+
+// Exact selection among the members of the threshold bin, then ascending output.
+//   * score levels: key bits 19..8, then 7..0 (12- and 8-bit radix histograms),
+//     run only while the remaining members do not all share one key;
+//   * members that tie on the full key: the `need` lowest block indices, taken
+//     in index order from a second bitmap (prefix counts by warp scans).
+__device__ __forceinline__ int key_digit(int level, uint32_t key) {
+    return level == 1 ? (int)((key >> 8) & 0xFFF) : (int)(key & 0xFF);
+}
 
 __global__ void __launch_bounds__(kSelThreads) select_final_kernel(SelArgs a) {
     extern __shared__ uint32_t dyn[];
-    uint32_t *bm = dyn;                  // [words]
+    uint32_t *bm = dyn;                                                // [words] selected blocks
+    uint32_t *tie = dyn + a.words;                                     // [words] members tied on the key
+    uint32_t *sck = dyn + 2 * a.words;                                 // [smem_cands] candidate keys
+    int32_t *scj = reinterpret_cast<int32_t *>(sck + a.smem_cands);   // [smem_cands] candidate indices
     __shared__ uint32_t h[kBins];
-    __shared__ uint32_t hn[kBins];
     __shared__ uint32_t scan_smem[32];
     __shared__ BinPick pick;
-    __shared__ int prefix_digit[5];
+    __shared__ uint32_t warp_base[32], total_s, kmin_s, kmax_s;
+    __shared__ int prefix_digit[3];
     const int i = blockIdx.x;
     const int n = a.n_vis[i];
     const int K = min(a.topk, n);
     int32_t *out = a.sel_idx + (size_t)i * a.topk;
-    const int words = (n + 31) / 32;
-
     if (K == n) {  // select every visible block
         for (int r = threadIdx.x; r < a.topk; r += blockDim.x) out[r] = r < n ? r : -1;
         return;
     }
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int words = (n + 31) / 32;
     const uint32_t *gbm = a.bitmap + (size_t)i * a.words;
-    for (int w = threadIdx.x; w < words; w += blockDim.x) bm[w] = gbm[w];
-    for (int k = threadIdx.x; k < kBins; k += blockDim.x) h[k] = a.hist1[(size_t)i * kBins + k];
+    for (int w = threadIdx.x; w < words; w += blockDim.x) {
+        bm[w] = __ldcg(gbm + w);
+        tie[w] = 0u;
+    }
+    if (threadIdx.x == 0) {
+        kmin_s = 0xFFFFFFFFu;
+        kmax_s = 0u;
+    }
+    const int cand_bin = a.thresh[3 * i + 2];
     __syncthreads();
-    const BinPick p1 = pick_bin(h, kBins, (uint32_t)K, scan_smem, &pick);
-    uint32_t need = (uint32_t)K - p1.above;
-    if (p1.above + p1.at != (uint32_t)K) {
-        // refine inside bin p1.bin
+    if (cand_bin >= 0) {
+        uint32_t need = (uint32_t)(K - a.thresh[3 * i + 1]);
         const uint32_t nc = a.ncand[i];
         const bool in_list = nc <= (uint32_t)a.ccap;
+        const bool in_smem = in_list && nc <= (uint32_t)a.smem_cands;
         const uint32_t *ck = a.cand_key + (size_t)i * a.ccap;
         const int32_t *cj = a.cand_idx + (size_t)i * a.ccap;
         const float *s = a.scores + (size_t)i * a.cap;
-        for (int k = threadIdx.x; k < kBins; k += blockDim.x) h[k] = a.hist2[(size_t)i * kBins + k];
-        if (threadIdx.x == 0) prefix_digit[0] = p1.bin;
-        __syncthreads();
-        for (int level = 1; level <= 4; ++level) {
-            const int nb = level_bins(level);
-            const BinPick p = pick_bin(h, nb, need, scan_smem, &pick);
-            if (threadIdx.x == 0) prefix_digit[level] = p.bin;
-            const bool done = (p.above + p.at == need);
-            for (int k = threadIdx.x; k < kBins; k += blockDim.x) hn[k] = 0;
-            __syncthreads();
-            // one pass over the elements that share all earlier digits
-            auto visit = [&](uint32_t key, int j) {
-                if ((int)(key >> 20) != prefix_digit[0]) return;
-                for (int l = 1; l < level; ++l)
-                    if (level_digit(l, key, j) != prefix_digit[l]) return;
-                const int d = level_digit(level, key, j);
-                if (d > p.bin || (d == p.bin && done)) mark(bm, j);
-                else if (d == p.bin && level < 4) atomicAdd(&hn[level_digit(level + 1, key, j)], 1u);
-            };
-            if (in_list) {
-                for (uint32_t c = threadIdx.x; c < nc; c += blockDim.x) visit(ck[c], cj[c]);
+        // every member of the threshold bin: f(key, j)
+        auto for_each = [&](auto &&f) {
+            if (in_smem) {
+                for (uint32_t c = threadIdx.x; c < nc; c += blockDim.x) f(sck[c], scj[c]);
+            } else if (in_list) {
+                for (uint32_t c = threadIdx.x; c < nc; c += blockDim.x) f(__ldcg(ck + c), __ldcg(cj + c));
             } else {
-                for (int j = threadIdx.x; j < n; j += blockDim.x) visit(ordered_key(s[j]), j);
+                for (int j = threadIdx.x; j < n; j += blockDim.x) {
+                    const uint32_t key = ordered_key(__ldcg(s + j));
+                    if ((int)(key >> 20) == cand_bin) f(key, j);
+                }
             }
+        };
+        // load (into shared memory when it fits) and the key range
+        uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+        if (in_smem) {
+#pragma unroll 4
+            for (uint32_t c = threadIdx.x; c < nc; c += blockDim.x) {
+                const uint32_t key = __ldcg(ck + c);
+                sck[c] = key;
+                scj[c] = __ldcg(cj + c);
+                lo = min(lo, key);
+                hi = max(hi, key);
+            }
+        } else {
+            for_each([&](uint32_t key, int) { lo = min(lo, key); hi = max(hi, key); });
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+            hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+        }
+        if (lane == 0) {
+            atomicMin(&kmin_s, lo);
+            atomicMax(&kmax_s, hi);
+        }
+        if (threadIdx.x == 0) prefix_digit[0] = cand_bin;
+        __syncthreads();
+        bool done = false;
+        // ---- score levels while the members' keys still differ
+        const bool all_tied = kmin_s == kmax_s;
+        for (int level = 1; level <= 2 && !all_tied && !done; ++level) {
+            for (int k = threadIdx.x; k < kBins; k += blockDim.x) h[k] = 0u;
             __syncthreads();
-            if (done) break;
+            for_each([&](uint32_t key, int j) {
+                if (level == 2 && key_digit(1, key) != prefix_digit[1]) return;
+                atomicAdd(&h[key_digit(level, key)], 1u);
+            });
+            __syncthreads();
+            const BinPick p = pick_bin(h, level == 1 ? 4096 : 256, need, scan_smem, &pick);
+            if (threadIdx.x == 0) prefix_digit[level] = p.bin;
+            done = (p.above + p.at == need);
+            __syncthreads();
+            for_each([&](uint32_t key, int j) {
+                if (level == 2 && key_digit(1, key) != prefix_digit[1]) return;
+                const int d = key_digit(level, key);
+                if (d > p.bin || (d == p.bin && done)) atomicOr(&bm[j >> 5], 1u << (j & 31));
+            });
+            __syncthreads();
             need -= p.above;
-            const volatile uint32_t *vhn = hn;
-            for (int k = threadIdx.x; k < kBins; k += blockDim.x) h[k] = vhn[k];
+        }
+        // ---- members tied on the full key: the `need` lowest block indices
+        if (!done) {
+            const int levels = all_tied ? 0 : 2;  // key digits fixed so far (beyond the bin)
+            for_each([&](uint32_t key, int j) {
+                for (int l = 1; l <= levels; ++l)
+                    if (key_digit(l, key) != prefix_digit[l]) return;
+                atomicOr(&tie[j >> 5], 1u << (j & 31));
+            });
             __syncthreads();
+            const volatile uint32_t *vtie = tie;
+            run_prefix(vtie, words, n, warp_base, &total_s);
+            // keep the first `need` tied members (in index order) and add them to bm
+            const WordRun r = warp_run(words);
+            uint32_t base = warp_base[warp];
+            for (int wc = r.begin; wc < r.end; wc += 32) {
+                const int w = wc + lane;
+                uint32_t b = w < r.end ? vtie[w] : 0u;
+                if (w == words - 1 && (n & 31)) b &= (1u << (n & 31)) - 1u;
+                const uint32_t c = __popc(b);
+                uint32_t incl = c;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += y;
+                }
+                const uint32_t first = base + incl - c;  // tied members before this word
+                if (first < need && b) {
+                    uint32_t keep = b;
+                    if (first + c > need) {  // keep only the lowest (need - first) bits
+                        uint32_t left = need - first;
+                        keep = 0u;
+                        while (left--) {
+                            const uint32_t lowbit = b & (~b + 1u);
+                            keep |= lowbit;
+                            b ^= lowbit;
+                        }
+                    }
+                    atomicOr(&bm[w], keep);
+                }
+                base += __shfl_sync(0xffffffffu, incl, 31);
+            }
         }
     }
     __syncthreads();
-    // ---- compaction: bitmap -> ascending block indices ----
-    // Rounds of blockDim.x words; each word is read once (through a volatile
-    // view, after the barrier that ends the marking) and that single value
-    // gives both the thread's count and the indices it writes.
-    __shared__ uint32_t round_total;
+
+    // ---- compaction: bitmap -> ascending block indices (warp scans) ----
     const volatile uint32_t *vbm = bm;
-    uint32_t base = 0;
-    for (int wr = 0; wr < words; wr += blockDim.x) {
-        const int w = wr + threadIdx.x;
-        uint32_t bits = 0;
-        if (w < words) {
-            bits = vbm[w];
-            if (w == words - 1 && (n & 31)) bits &= (1u << (n & 31)) - 1u;
+    run_prefix(vbm, words, n, warp_base, &total_s);
+    const WordRun r = warp_run(words);
+    uint32_t base = warp_base[warp];
+    for (int wc = r.begin; wc < r.end; wc += 32) {
+        const int w = wc + lane;
+        uint32_t bits = w < r.end ? vbm[w] : 0u;
+        if (w == words - 1 && (n & 31)) bits &= (1u << (n & 31)) - 1u;
+        const uint32_t c = __popc(bits);
+        uint32_t incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
         }
-        const uint32_t cnt = __popc(bits);
-        const uint32_t incl = block_inclusive_scan<uint32_t>(cnt, scan_smem);
-        uint32_t pos = base + incl - cnt;
+        uint32_t pos = base + incl - c;
         while (bits) {
             const int bit = __ffs(bits) - 1;
             bits &= bits - 1;
             if (pos < (uint32_t)a.topk) out[pos] = w * 32 + bit;
             ++pos;
         }
-        if (threadIdx.x == blockDim.x - 1) round_total = incl;
-        __syncthreads();
-        base += round_total;
-        __syncthreads();
+        base += __shfl_sync(0xffffffffu, incl, 31);
     }
-    // total selected = K by construction; pad the rest
-    for (int r = K + threadIdx.x; r < a.topk; r += blockDim.x) out[r] = -1;
+    // exactly K are selected; pad the rest
+    for (int r2 = K + threadIdx.x; r2 < a.topk; r2 += blockDim.x) out[r2] = -1;
 }
 
 template <bool E4M3, int KS>
@@ -556,17 +737,15 @@ cudaError_t launch_scan(const ScanArgs &sa, int grid, cudaStream_t s) {
 
 size_t index_topk_workspace_bytes(int Nq, int cap) { return carve(nullptr, Nq, cap, nullptr); }
 
-int index_select_smem_bytes(int cap) { return ((cap + 31) / 32) * 4; }
-
 cudaError_t launch_index_topk(const csa_cache &c, const void *q_idx, const float *w, int Nq, int H_I,
                               const int32_t *q_offsets, const int32_t *q_pos, int topk, int32_t *sel_idx,
                               void *workspace, int num_sms, cudaStream_t s) {
     IndexWs ws;
     carve(workspace, Nq, c.capacity, &ws);
-    cudaError_t err = cudaMemsetAsync(ws.hist1, 0, ws.zero_bytes, s);
+    cudaError_t err = cudaMemsetAsync(ws.done, 0, ws.zero_bytes, s);  // counters, histograms, bitmaps
     if (err != cudaSuccess) return err;
-    schedule_kernel<<<1, 1024, 0, s>>>(q_offsets, q_pos, c.n_blocks, c.batch, Nq, c.block, c.capacity, ws.req, ws.n_vis,
-                                       ws.gprefix);
+    schedule_kernel<<<1, 1024, 0, s>>>(q_offsets, q_pos, c.n_blocks, c.batch, Nq, c.block, c.capacity, topk,
+                                       ws.req, ws.n_vis, ws.gprefix, ws.thresh);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
 
     ScanArgs sa;
@@ -578,9 +757,12 @@ cudaError_t launch_index_topk(const csa_cache &c, const void *q_idx, const float
     sa.gprefix = ws.gprefix;
     sa.scores = ws.scores;
     sa.hist1 = ws.hist1;
+    sa.done = ws.done;
+    sa.thresh = ws.thresh;
     sa.Nq = Nq;
     sa.H_I = H_I;
     sa.cap = c.capacity;
+    sa.topk = topk;
     const int grid = num_sms * 2;
     const bool e4 = c.idx_dtype == CSA_IDX_E4M3;
     switch (c.idx_dim / 16) {
@@ -595,7 +777,7 @@ cudaError_t launch_index_topk(const csa_cache &c, const void *q_idx, const float
     sel.n_vis = ws.n_vis;
     sel.scores = ws.scores;
     sel.hist1 = ws.hist1;
-    sel.hist2 = ws.hist2;
+    sel.thresh = ws.thresh;
     sel.bitmap = ws.bitmap;
     sel.ncand = ws.ncand;
     sel.cand_key = ws.cand_key;
@@ -606,11 +788,21 @@ cudaError_t launch_index_topk(const csa_cache &c, const void *q_idx, const float
     sel.topk = topk;
     sel.words = ws.words;
     sel.ccap = ws.ccap;
-    select_pass_kernel<<<dim3(kPassSlices, Nq), kSelThreads, 0, s>>>(sel);
+    // enough warps to cover the rows with a few 128-score steps each
+    const int chunks_per_cta = 128 * (kPassThreads / 32);
+    int gx = (c.capacity + chunks_per_cta - 1) / chunks_per_cta;
+    const int want = (16 * num_sms + Nq - 1) / Nq;
+    if (gx > want) gx = want;
+    if (gx < 1) gx = 1;
+    select_pass_kernel<<<dim3(gx, Nq), kPassThreads, 0, s>>>(sel);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    // the bitmap (dynamic) comes on top of ~33 KB of static shared memory:
-    // opt in to the dynamic size every time (cheap, and valid during capture)
-    const int smem = index_select_smem_bytes(c.capacity);
+    // dynamic shared memory: the bitmap, then as many candidates as fit next to
+    // the ~33 KB of static shared memory (opt in every time: cheap, valid in capture)
+    const int kDynMax = 200 * 1024;
+    sel.smem_cands = (kDynMax - 8 * ws.words) / 8;
+    if (sel.smem_cands < 0) sel.smem_cands = 0;
+    if (sel.smem_cands > ws.ccap) sel.smem_cands = ws.ccap;
+    const int smem = 8 * ws.words + 8 * sel.smem_cands;
     err = cudaFuncSetAttribute(select_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
     select_final_kernel<<<Nq, kSelThreads, smem, s>>>(sel);

@@ -84,7 +84,7 @@ typedef struct {
     int32_t batch;     /* requests, >= 1                                  */
     int32_t dim;       /* D (K = V latent width); 128 or 512 for attention; multiple of 32 for compression */
     int32_t block;     /* m, tokens pooled per entry, 1..128              */
-    int32_t capacity;  /* blocks per request, >= 1                        */
+    int32_t capacity;  /* blocks per request, 1 .. 2^19                   */
     uint8_t *fp4;
     uint8_t *scale;
     void *idx_key;

@@ -62,7 +62,7 @@ def test_compress_validation(lib):
     assert compress(lib, fake_cache(dim=100)) == ERR_SHAPE
     assert compress(lib, fake_cache(dim=1024)) == ERR_UNSUPPORTED
     assert compress(lib, fake_cache(idx_dim=96)) == ERR_UNSUPPORTED
-    assert compress(lib, fake_cache(capacity=(1 << 20) + 1)) == ERR_UNSUPPORTED
+    assert compress(lib, fake_cache(capacity=(1 << 19) + 1)) == ERR_UNSUPPORTED
     assert compress(lib, fake_cache(fp4=0x10008)) == ERR_ALIGN
     assert compress(lib, fake_cache(), kv=0x50008) == ERR_ALIGN
     assert compress(lib, fake_cache(), n=-1) == ERR_SHAPE
