@@ -193,6 +193,7 @@ struct AttArgs {
     // schedule (workspace)
     const int32_t *req, *nent, *ctiles, *wlen;
     const long long *tprefix;        // [Nq+1]
+    const int32_t *sq;               // [Nq] query scale exponents
     float *part_o, *part_rho, *part_l;  // [2G][64][D], [2G][64], [2G][64]
     int Nq, H, cap, topk;
     float scale_log2;                // softmax_scale * log2(e)
@@ -206,47 +207,76 @@ struct RowRegs {
     int valid;
 };
 
+// Everything the tile loop needs about one tile, gathered ahead of time so
+// that no dependent global load sits on the per-tile critical path.
 struct TileRef {
-    int i;      // query (-1: none)
-    int lt;     // local tile index within the query
-    int win;    // 1: window tile
+    int i;             // query
+    int lt;            // local tile index within the query
+    int win;           // 1: window tile
+    int b;             // request of the query
+    int nent;          // compressed entry slots of the query
+    int ctiles;        // compressed tiles of the query
+    int wlen;          // window rows of the query
+    int nblk;          // filled blocks of request b (bound of a selected index)
+    long long t0, t1;  // the query's tiles [t0, t1) in the flat tile list
 };
 
+__device__ __forceinline__ TileRef query_ref(const AttArgs &a, int i, long long t) {
+    TileRef r;
+    r.i = i;
+    r.t0 = a.tprefix[i];
+    r.t1 = a.tprefix[i + 1];
+    r.lt = (int)(t - r.t0);
+    r.b = a.req[i];
+    r.nent = a.nent[i];
+    r.ctiles = a.ctiles[i];
+    r.wlen = a.wlen[i];
+    r.nblk = a.n_blocks[r.b];
+    r.win = r.lt >= r.ctiles;
+    return r;
+}
+
+// The tile holding flat index t (binary search; once per CTA).
 __device__ __forceinline__ TileRef locate(const AttArgs &a, long long t) {
     int lo = 0, hi = a.Nq - 1;
     while (lo < hi) {
         int mid = (lo + hi + 1) >> 1;
         if (a.tprefix[mid] <= t) lo = mid; else hi = mid - 1;
     }
-    TileRef r;
-    r.i = lo;
-    r.lt = (int)(t - a.tprefix[lo]);
-    r.win = r.lt >= a.ctiles[lo];
-    return r;
+    return query_ref(a, lo, t);
+}
+
+// The tile after r (t_next = its flat index): the same query, or the next one with tiles.
+__device__ __forceinline__ TileRef advance(const AttArgs &a, const TileRef &r, long long t_next) {
+    if (t_next < r.t1) {
+        TileRef n = r;
+        n.lt += 1;
+        n.win = n.lt >= n.ctiles;
+        return n;
+    }
+    int i = r.i + 1;
+    while (i < a.Nq - 1 && a.tprefix[i + 1] == a.tprefix[i]) ++i;  // skip queries without tiles
+    return query_ref(a, i, t_next);
+}
+
+// This thread's row of a compressed tile: the raw selected index (CSA) or the
+// slot itself (HCA); -1 for padding rows. Checked against the bound at use.
+__device__ __forceinline__ int row_block_raw(const AttArgs &a, const TileRef &tr) {
+    const int slot = tr.lt * kTile + (int)threadIdx.x;
+    if (tr.win || slot >= tr.nent) return -1;
+    return a.sel_idx ? a.sel_idx[(size_t)tr.i * a.topk + slot] : slot;
 }
 
 // Issue the loads of this thread's row of a compressed tile.
 template <int D>
-__device__ __forceinline__ void prefetch_row(const AttArgs &a, const TileRef &tr, RowRegs<D> &rr) {
+__device__ __forceinline__ void prefetch_row(const AttArgs &a, const TileRef &tr, int blk, RowRegs<D> &rr) {
     rr.valid = 0;
-    const int j = threadIdx.x;
-    const int slot = tr.lt * kTile + j;
-    const int i = tr.i;
-    const int b = a.req[i];
-    int blk = -1;
-    if (slot < a.nent[i]) {
-        if (a.sel_idx) {
-            blk = a.sel_idx[(size_t)i * a.topk + slot];
-            if (blk >= a.n_blocks[b] || blk >= a.cap) {
-                flag(a.status, CSA_DEV_BAD_INDEX);
-                blk = -1;
-            }
-        } else {
-            blk = slot;
-        }
+    if (blk >= 0 && (blk >= tr.nblk || blk >= a.cap)) {
+        flag(a.status, CSA_DEV_BAD_INDEX);
+        blk = -1;
     }
     if (blk >= 0) {
-        const size_t row = (size_t)b * a.cap + blk;
+        const size_t row = (size_t)tr.b * a.cap + blk;
         const uint4 *src = reinterpret_cast<const uint4 *>(a.fp4 + row * (D / 2));
 #pragma unroll
         for (int v = 0; v < Cfg<D>::CODE_V; ++v) rr.code[v] = __ldg(src + v);
@@ -312,8 +342,8 @@ __device__ __forceinline__ int dequant_row(const RowRegs<D> &rr, uint8_t *E) {
 template <int D>
 __device__ __forceinline__ int load_window_row(const AttArgs &a, const TileRef &tr, uint8_t *E, uint32_t E_s, bool &valid) {
     const int j = threadIdx.x;
-    const int r = (tr.lt - a.ctiles[tr.i]) * kTile + j;
-    valid = r < a.wlen[tr.i];
+    const int r = (tr.lt - tr.ctiles) * kTile + j;
+    valid = r < tr.wlen;
     if (!valid) {
         for (int kc = 0; kc < D / 8; ++kc) *reinterpret_cast<uint4 *>(E + e_chunk_off<D>(j, kc)) = make_uint4(0, 0, 0, 0);
         return 0;
@@ -350,29 +380,12 @@ __device__ __forceinline__ int load_window_row(const AttArgs &a, const TileRef &
 }
 
 // Q' = q * 2^-sQ in fp16, K-major with 128-byte swizzle, heads >= H zero.
-// Returns sQ.
+// sQ (from the schedule kernel) puts max|q| in [2^14, 2^15), so every bf16
+// value within 2^31 of the maximum converts exactly.
 template <int D>
-__device__ int load_query(const AttArgs &a, int i, uint8_t *Q, float *red) {
+__device__ void load_query(const AttArgs &a, int i, int sQ, uint8_t *Q) {
     const int tid = threadIdx.x;
     const __nv_bfloat16 *qi = a.q + (size_t)i * a.H * D;
-    const int nchunks = a.H * (D / 8);
-    float mx = 0.f;
-#pragma unroll 8
-    for (int c = tid; c < nchunks; c += kThreads) {
-        uint4 u = __ldg(reinterpret_cast<const uint4 *>(qi) + c);
-        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            float2 f = __bfloat1622float2(h[k]);
-            mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
-        }
-    }
-    mx = warp_max(mx);
-    if ((tid & 31) == 0) red[tid >> 5] = mx;
-    __syncthreads();
-    mx = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-    __syncthreads();
-    const int sQ = mx > 0.f ? (int)((__float_as_uint(mx) >> 23) & 0xFF) - 127 - 14 : 0;
     const float inv = ldexpf(1.0f, -sQ);
     // chunk (h, kc): consecutive threads take consecutive heads, so the
     // swizzled 16-byte stores of a warp spread over all eight bank groups
@@ -394,32 +407,77 @@ __device__ int load_query(const AttArgs &a, int i, uint8_t *Q, float *red) {
         const uint32_t off = (uint32_t)((kc >> 3) * Cfg<D>::QREG + (h >> 3) * 1024 + (h & 7) * 128 + (((kc & 7) ^ (h & 7)) << 4));
         *reinterpret_cast<uint4 *>(Q + off) = make_uint4(o[0], o[1], o[2], o[3]);
     }
-    return sQ;
 }
 
 // ---------------------------------------------------------------- schedule
-__global__ void attend_schedule_kernel(const int32_t *q_offsets, const int32_t *q_pos, const int32_t *n_blocks,
-                                       const int32_t *win_len, int batch, int Nq, int m, int cap, int topk, int max_win,
-                                       int H, int D, int32_t *req, int32_t *nent, int32_t *ctiles, int32_t *wlen,
-                                       long long *tprefix, float *out, float *lse, int32_t *status) {
+// One CTA per query. Every CTA: its query's scale exponent sq[i] (from
+// max|q|) and, when the query has no entry at all, out = 0 and lse = -inf.
+// CTA 0 also writes the per-query tile counts and their prefix.
+__device__ __forceinline__ void query_tiles(const int32_t *q_offsets, const int32_t *q_pos, const int32_t *n_blocks,
+                                            const int32_t *win_len, int batch, int m, int cap, int topk, int max_win,
+                                            int i, int32_t *status, int &b_out, int &ne, int &ct, int &wl) {
+    const int b = request_of(q_offsets, batch, i);
+    ne = 0;
+    if (b >= 0) ne = (q_pos ? min(visible_blocks(q_pos[i], m, n_blocks[b]), cap) : topk);
+    wl = win_len ? win_len[i] : 0;
+    if (wl < 0 || wl > max_win) {
+        if (status) atomicOr(status, CSA_DEV_BAD_WINDOW);
+        wl = min(max(wl, 0), max_win);
+    }
+    if (b < 0) wl = 0;
+    ct = (ne + kTile - 1) / kTile;
+    b_out = b < 0 ? 0 : b;
+}
+
+__global__ void __launch_bounds__(256) attend_schedule_kernel(
+    const int32_t *q_offsets, const int32_t *q_pos, const int32_t *n_blocks, const int32_t *win_len, int batch,
+    int Nq, int m, int cap, int topk, int max_win, const __nv_bfloat16 *q, int H, int D, int32_t *req, int32_t *nent,
+    int32_t *ctiles, int32_t *wlen, long long *tprefix, int32_t *sq, float *out, float *lse, int32_t *status) {
     __shared__ long long red[32];
     __shared__ long long round_total;
+    __shared__ float fred[8];
+    const int qi = blockIdx.x;
+    // ---- this CTA's query: scale exponent and the empty case
+    {
+        const __nv_bfloat16 *qp = q + (size_t)qi * H * D;
+        const int nchunks = H * D / 8;
+        float mx = 0.f;
+#pragma unroll 4
+        for (int c = threadIdx.x; c < nchunks; c += blockDim.x) {
+            uint4 u = __ldg(reinterpret_cast<const uint4 *>(qp) + c);
+            const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                float2 f = __bfloat1622float2(h2[k]);
+                mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
+            }
+        }
+        mx = warp_max(mx);
+        if ((threadIdx.x & 31) == 0) fred[threadIdx.x >> 5] = mx;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            float m8 = 0.f;
+            for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m8 = fmaxf(m8, fred[w]);
+            sq[qi] = m8 > 0.f ? (int)((__float_as_uint(m8) >> 23) & 0xFF) - 127 - 14 : 0;
+        }
+        int b, ne, ct, wl;
+        query_tiles(q_offsets, q_pos, n_blocks, win_len, batch, m, cap, topk, max_win, qi, nullptr, b, ne, ct, wl);
+        if (ct + (wl + kTile - 1) / kTile == 0) {
+            for (int k = threadIdx.x; k < H * D; k += blockDim.x) out[(size_t)qi * H * D + k] = 0.f;
+            if (lse)
+                for (int k = threadIdx.x; k < H; k += blockDim.x) lse[(size_t)qi * H + k] = -INFINITY;
+        }
+    }
+    if (blockIdx.x != 0) return;
+    // ---- CTA 0: tile counts and prefix over all queries
     long long carry = 0;
     for (int base = 0; base < Nq; base += blockDim.x) {
         const int i = base + threadIdx.x;
         long long tiles = 0;
         if (i < Nq) {
-            const int b = request_of(q_offsets, batch, i);
-            int ne = 0;
-            if (b >= 0) ne = (q_pos ? min(visible_blocks(q_pos[i], m, n_blocks[b]), cap) : topk);
-            int wl = win_len ? win_len[i] : 0;
-            if (wl < 0 || wl > max_win) {
-                flag(status, CSA_DEV_BAD_WINDOW);
-                wl = min(max(wl, 0), max_win);
-            }
-            if (b < 0) wl = 0;
-            const int ct = (ne + kTile - 1) / kTile;
-            req[i] = b < 0 ? 0 : b;
+            int b, ne, ct, wl;
+            query_tiles(q_offsets, q_pos, n_blocks, win_len, batch, m, cap, topk, max_win, i, status, b, ne, ct, wl);
+            req[i] = b;
             nent[i] = ne;
             ctiles[i] = ct;
             wlen[i] = wl;
@@ -432,14 +490,6 @@ __global__ void attend_schedule_kernel(const int32_t *q_offsets, const int32_t *
         __syncthreads();
         carry += round_total;
         __syncthreads();
-    }
-    // queries with no entry at all: out = 0, lse = -inf
-    __syncthreads();
-    for (int i = 0; i < Nq; ++i) {
-        if (tprefix[i + 1] != tprefix[i]) continue;
-        for (int k = threadIdx.x; k < H * D; k += blockDim.x) out[(size_t)i * H * D + k] = 0.f;
-        if (lse)
-            for (int k = threadIdx.x; k < H; k += blockDim.x) lse[(size_t)i * H + k] = -INFINITY;
     }
 }
 
@@ -526,7 +576,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
     float *rho = reinterpret_cast<float *>(misc + 64);              // [64]
     float *alpha = rho + 64;                                        // [64]
     float *wred = alpha + 64;                                       // [4][64]
-    float *red = wred + 4 * 64;                                     // [32]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const long long T = a.tprefix[a.Nq];
@@ -563,7 +612,14 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
 
     RowRegs<D> rr;
     TileRef cur = locate(a, t_begin);
-    if (!cur.win) prefetch_row<D>(a, cur, rr);
+    prefetch_row<D>(a, cur, row_block_raw(a, cur), rr);
+    // the next tile and this thread's selected index in it (one tile ahead of its row loads)
+    TileRef nxt = cur;
+    int blk_nxt = -1;
+    if (t_begin + 1 < t_end) {
+        nxt = advance(a, cur, t_begin + 1);
+        blk_nxt = row_block_raw(a, nxt);
+    }
 
     long long t = t_begin;
     bool aborted = false;
@@ -571,8 +627,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
         // ---------------- segment = the tiles of query cur.i inside [t, t_end)
         const int i = cur.i;
         const long long seg_begin = t;
-        const long long seg_end = min(t_end, a.tprefix[i + 1]);
-        const bool whole = (seg_begin == a.tprefix[i]) && (seg_end == a.tprefix[i + 1]);
+        const long long seg_end = min(t_end, cur.t1);
+        const bool whole = (seg_begin == cur.t0) && (seg_end == cur.t1);
         // the previous segment's PV must finish before Q' and O^T are reused
         if (pv_pending) {
             const bool ok = mbar_wait(mbar_pv, ph_pv);
@@ -580,7 +636,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
             pv_pending = false;
             if (__syncthreads_or(!ok)) { aborted = true; break; }
         }
-        const int sQ = load_query<D>(a, i, Q, red);
+        const int sQ = a.sq[i];
+        load_query<D>(a, i, sQ, Q);
         float l_part[2] = {0.f, 0.f};  // per-warp partial row sums of heads 2*lane, 2*lane+1
         bool first = true;
 
@@ -600,12 +657,16 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
                 valid = rr.valid;
                 Rj = dequant_row<D>(rr, E);
             }
-            // next tile (possibly of the next query): start its loads now
-            TileRef nxt;
-            nxt.i = -1;
+            // next tile (possibly of the next query): start its row loads now,
+            // and the selected index of the tile after it
+            TileRef nxt2 = nxt;
+            int blk_nxt2 = -1;
             if (t + 1 < t_end) {
-                nxt = locate(a, t + 1);
-                if (!nxt.win) prefetch_row<D>(a, nxt, rr);
+                prefetch_row<D>(a, nxt, blk_nxt, rr);
+                if (t + 2 < t_end) {
+                    nxt2 = advance(a, nxt, t + 2);
+                    blk_nxt2 = row_block_raw(a, nxt2);
+                }
             }
             fence_async_smem();
             tc_fence_before();
@@ -715,7 +776,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
             }
             pv_pending = true;
             first = false;
-            if (nxt.i >= 0) cur = nxt;
+            if (t + 1 < t_end) {
+                cur = nxt;
+                nxt = nxt2;
+                blk_nxt = blk_nxt2;
+            }
         }
         if (aborted) break;
 
@@ -794,6 +859,7 @@ size_t attend_workspace_bytes(int Nq, int D, int num_ctas) {
     take(4 * (size_t)Nq);            // ctiles
     take(4 * (size_t)Nq);            // wlen
     take(8 * (size_t)(Nq + 1));      // tprefix
+    take(4 * (size_t)Nq);            // sq
     take(4 * (size_t)2 * num_ctas * kHeads * D);  // part_o
     take(4 * (size_t)2 * num_ctas * kHeads);      // part_rho
     take(4 * (size_t)2 * num_ctas * kHeads);      // part_l
@@ -818,6 +884,7 @@ cudaError_t launch_attend(const csa_cache &c, const void *q, int Nq, int H, cons
     int32_t *ctiles = reinterpret_cast<int32_t *>(take(4 * (size_t)Nq));
     int32_t *wlen = reinterpret_cast<int32_t *>(take(4 * (size_t)Nq));
     long long *tprefix = reinterpret_cast<long long *>(take(8 * (size_t)(Nq + 1)));
+    int32_t *sq = reinterpret_cast<int32_t *>(take(4 * (size_t)Nq));
     a.part_o = reinterpret_cast<float *>(take(4 * (size_t)2 * num_ctas * kHeads * D));
     a.part_rho = reinterpret_cast<float *>(take(4 * (size_t)2 * num_ctas * kHeads));
     a.part_l = reinterpret_cast<float *>(take(4 * (size_t)2 * num_ctas * kHeads));
@@ -836,6 +903,7 @@ cudaError_t launch_attend(const csa_cache &c, const void *q, int Nq, int H, cons
     a.ctiles = ctiles;
     a.wlen = wlen;
     a.tprefix = tprefix;
+    a.sq = sq;
     a.Nq = Nq;
     a.H = H;
     a.cap = c.capacity;
@@ -843,9 +911,10 @@ cudaError_t launch_attend(const csa_cache &c, const void *q, int Nq, int H, cons
     a.scale_log2 = softmax_scale * 1.4426950408889634f;
 
     cudaError_t err;
-    attend_schedule_kernel<<<1, 1024, 0, s>>>(q_offsets, sel_idx ? nullptr : q_pos, c.n_blocks,
-                                              win_kv ? win_len : nullptr, c.batch, Nq, c.block, c.capacity, topk, max_win, H, D,
-                                              req, nent, ctiles, wlen, tprefix, out, lse, c.status);
+    attend_schedule_kernel<<<Nq, 256, 0, s>>>(q_offsets, sel_idx ? nullptr : q_pos, c.n_blocks,
+                                               win_kv ? win_len : nullptr, c.batch, Nq, c.block, c.capacity, topk,
+                                               max_win, static_cast<const __nv_bfloat16 *>(q), H, D, req, nent, ctiles,
+                                               wlen, tprefix, sq, out, lse, c.status);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     if (D == 512) {
         const int smem = Cfg<512>::SMEM;
