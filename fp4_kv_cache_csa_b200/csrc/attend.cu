@@ -10,7 +10,8 @@
 // both key and value (cue 8: a shared latent), so the heads x D by D x entries
 // products are dense contractions and run on the tcgen05 tensor cores.
 //
-// Design (one CTA per SM, 128 threads, thread j <-> entry j of a 128-entry tile):
+// Design (one CTA per SM, 256 threads; entry j of a 128-entry tile belongs to
+// threads j and j + 128, which take one half of its D channels each):
 //   * Work = the flat list of 128-entry tiles of all queries (compressed tiles
 //     first, then window tiles), cut into equal contiguous ranges, one per CTA.
 //     A CTA whose range covers a whole query writes the output directly;
@@ -22,16 +23,21 @@
 //     fp16 within 2^24 of the row's largest group. The query is stored as
 //     q * 2^-sQ (exact for bf16 values within 2^31 of max|q|).
 //   * S^T = E' Q'^T: M = 128 entries (TMEM lanes), N = 64 heads (columns).
-//   * Softmax in the log2 domain, thread j holding the 64 head logits of its
-//     entry: u = log2(e) * scale * <q,e_j> + R_j. Each head h keeps a reference
-//     rho_h, raised (and the TMEM accumulator rescaled) only when a tile's
-//     max exceeds it by more than 8; P'_{j,h} = 2^(u - rho_h) <= 256 is stored
-//     in fp16 (11-bit significand), folding the row factor 2^R_j back in.
+//   * Softmax in the log2 domain, thread (j, half) holding 32 head logits of
+//     entry j: u = log2(e) * scale * <q,e_j> + R_j. Each head h keeps a
+//     reference rho_h, set from the first tile's maximum and raised (with the
+//     TMEM accumulator rescaled) only when some logit exceeds it by more than
+//     8, so the per-head maximum over entries (a cross-thread reduction) is
+//     taken only then; P'_{j,h} = 2^(u - rho_h) <= 256 is stored in fp16,
+//     folding the row factor 2^R_j back in. The row sums stay per thread and
+//     are reduced once per segment.
 //   * O^T += E'^T P': M = 128 latent channels per d-tile, N = 64 heads, K = 16
-//     entries per MMA; O^T lives in TMEM for the whole segment.
+//     entries per MMA; O^T lives in TMEM for the whole segment. The PV MMAs of
+//     the low and high channel halves complete on separate barriers, so each
+//     half of the next tile is dequantized as soon as its channels are free.
 //   * out = O / l and lse = ln 2 * (rho + log2 l), l = sum_j 2^(lambda_j - rho).
-// Compressed tiles are loaded into registers one tile ahead (prefetch while
-// the tensor core works); window tiles (bf16) are copied with cp.async into
+// Compressed rows are loaded into registers one tile ahead (their selected
+// indices two tiles ahead); window tiles (bf16) are copied with cp.async into
 // the operand buffer and converted in place.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -45,7 +51,7 @@ namespace {
 
 constexpr int kTile = 128;
 constexpr int kHeads = 64;
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;
 constexpr long long kWaitCycles = 2000000000LL;  // bounded mbarrier wait (~1 s)
 
 template <int D>
@@ -53,6 +59,7 @@ struct Cfg {
     static constexpr int DT = D / 128;                    // O^T d-tiles
     static constexpr int GPR = D / 32;                    // MXFP4 groups per row
     static constexpr int CODE_V = D / 32;                 // 16-byte code loads per row (D/2 bytes)
+    static constexpr int HALF_V = CODE_V / 2;             // ... per half row
     static constexpr int E_BYTES = kTile * D * 2;
     static constexpr int Q_BYTES = kHeads * D * 2;
     static constexpr int P_BYTES = kTile * kHeads * 2;
@@ -135,11 +142,11 @@ __device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity) {
                    "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])     \
                  : "memory")
 
-// 64 consecutive 32-bit TMEM columns of this thread's lane.
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
+// 32 consecutive 32-bit TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     uint32_t r[16];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < 2; ++q) {
         CSA_LD16(taddr + 16 * q, r);
 #pragma unroll
         for (int k = 0; k < 16; ++k) v[16 * q + k] = __uint_as_float(r[k]);
@@ -147,10 +154,10 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-__device__ __forceinline__ void tmem_st64(uint32_t taddr, const float (&v)[64]) {
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
     uint32_t r[16];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < 2; ++q) {
 #pragma unroll
         for (int k = 0; k < 16; ++k) r[k] = __float_as_uint(v[16 * q + k]);
         CSA_ST16(taddr + 16 * q, r);
@@ -158,26 +165,26 @@ __device__ __forceinline__ void tmem_st64(uint32_t taddr, const float (&v)[64]) 
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-
-// Butterfly transpose-reduction: 64 values per lane -> lane L ends with the
-// reduction over all 32 lanes of entries 2L and 2L+1 (in v[0], v[1]).
+// Butterfly transpose-reduction: 32 values per lane -> lane L ends with the
+// reduction over all 32 lanes of value L (in v[0]).
 template <bool MAX>
-__device__ __forceinline__ void transpose_reduce64(float (&v)[64]) {
+__device__ __forceinline__ void transpose_reduce32(float (&v)[32]) {
     const int lane = threadIdx.x & 31;
 #pragma unroll
-    for (int half = 32, o = 16; o >= 1; half >>= 1, o >>= 1) {
-        const bool hi = (lane & o) != 0;
+    for (int half = 16; half >= 1; half >>= 1) {
+        const bool hi = (lane & half) != 0;
 #pragma unroll
         for (int k = 0; k < half; ++k) {
             const float send = hi ? v[k] : v[k + half];
             const float keep = hi ? v[k + half] : v[k];
-            const float got = __shfl_xor_sync(0xffffffffu, send, o);
+            const float got = __shfl_xor_sync(0xffffffffu, send, half);
             v[k] = MAX ? fmaxf(keep, got) : keep + got;
         }
     }
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
 
 // ---------------------------------------------------------------- arguments
@@ -199,10 +206,11 @@ struct AttArgs {
     float scale_log2;                // softmax_scale * log2(e)
 };
 
-// Per-row prefetch of one compressed entry (codes + E8M0 bytes).
+// Prefetch of this thread's half of one compressed entry: its codes and all
+// of the row's E8M0 bytes (R_j is the maximum over the whole row).
 template <int D>
 struct RowRegs {
-    uint4 code[Cfg<D>::CODE_V];
+    uint4 code[Cfg<D>::HALF_V];
     uint4 sc;
     int valid;
 };
@@ -262,7 +270,7 @@ __device__ __forceinline__ TileRef advance(const AttArgs &a, const TileRef &r, l
 // This thread's row of a compressed tile: the raw selected index (CSA) or the
 // slot itself (HCA); -1 for padding rows. Checked against the bound at use.
 __device__ __forceinline__ int row_block_raw(const AttArgs &a, const TileRef &tr) {
-    const int slot = tr.lt * kTile + (int)threadIdx.x;
+    const int slot = tr.lt * kTile + (int)(threadIdx.x & (kTile - 1));
     if (tr.win || slot >= tr.nent) return -1;
     return a.sel_idx ? a.sel_idx[(size_t)tr.i * a.topk + slot] : slot;
 }
@@ -277,9 +285,9 @@ __device__ __forceinline__ void prefetch_row(const AttArgs &a, const TileRef &tr
     }
     if (blk >= 0) {
         const size_t row = (size_t)tr.b * a.cap + blk;
-        const uint4 *src = reinterpret_cast<const uint4 *>(a.fp4 + row * (D / 2));
+        const uint4 *src = reinterpret_cast<const uint4 *>(a.fp4 + row * (D / 2)) + (threadIdx.x >> 7) * Cfg<D>::HALF_V;
 #pragma unroll
-        for (int v = 0; v < Cfg<D>::CODE_V; ++v) rr.code[v] = __ldg(src + v);
+        for (int v = 0; v < Cfg<D>::HALF_V; ++v) rr.code[v] = __ldg(src + v);
         if constexpr (D / 32 >= 16) {
             rr.sc = __ldg(reinterpret_cast<const uint4 *>(a.scale + row * (D / 32)));
         } else {
@@ -302,26 +310,29 @@ __device__ __forceinline__ uint32_t e_chunk_off(int j, int kc) {
     return (uint32_t)((kc >> 3) * Cfg<D>::KREG + (j >> 3) * 1024 + (j & 7) * 128 + (((kc & 7) ^ (j & 7)) << 4));
 }
 
-// Dequantize this thread's prefetched row into E' (fp16, scaled by 2^-R_j).
-// Returns R_j (the row's largest E8M0 exponent); invalid rows are zero.
+// Dequantize this thread's half of its prefetched row into E' (fp16, scaled
+// by 2^-R_j). Returns R_j (the row's largest E8M0 exponent); invalid rows are zero.
 template <int D>
 __device__ __forceinline__ int dequant_row(const RowRegs<D> &rr, uint8_t *E) {
-    const int j = threadIdx.x;
+    const int j = threadIdx.x & (kTile - 1);
+    const int g0 = (threadIdx.x >> 7) * (Cfg<D>::GPR / 2);  // first group of this half
     if (!rr.valid) {
 #pragma unroll 4
-        for (int kc = 0; kc < D / 8; ++kc) *reinterpret_cast<uint4 *>(E + e_chunk_off<D>(j, kc)) = make_uint4(0, 0, 0, 0);
+        for (int kc = 4 * g0; kc < 4 * g0 + D / 16; ++kc)
+            *reinterpret_cast<uint4 *>(E + e_chunk_off<D>(j, kc)) = make_uint4(0, 0, 0, 0);
         return 0;
     }
     int rmax = 0;
 #pragma unroll
     for (int g = 0; g < Cfg<D>::GPR; ++g) rmax = max(rmax, scale_byte<D>(rr, g));
 #pragma unroll
-    for (int g = 0; g < Cfg<D>::GPR; ++g) {
+    for (int gl = 0; gl < Cfg<D>::GPR / 2; ++gl) {
+        const int g = g0 + gl;
         const int k = scale_byte<D>(rr, g) - rmax;  // <= 0
         // 2^k in fp16: normal for k >= -14, subnormal down to -24, else 0
         const uint16_t hb = k >= -14 ? (uint16_t)((k + 15) << 10) : k >= -24 ? (uint16_t)(1u << (k + 24)) : 0;
         __half2 s2 = __halves2half2(__ushort_as_half(hb), __ushort_as_half(hb));
-        const uint32_t *w = reinterpret_cast<const uint32_t *>(&rr.code[g]);
+        const uint32_t *w = reinterpret_cast<const uint32_t *>(&rr.code[gl]);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {  // 4 bytes -> 8 channels -> one 16-byte chunk
             uint32_t outw[4];
@@ -337,34 +348,43 @@ __device__ __forceinline__ int dequant_row(const RowRegs<D> &rr, uint8_t *E) {
     return rmax - 127;
 }
 
-// Window tile: cp.async the bf16 rows into E' and convert them in place to
-// fp16 scaled by 2^-R_j, R_j = exponent of the row's max |x|.
+// Window tile: cp.async this thread's half of the bf16 row into E' and convert
+// it in place to fp16 scaled by 2^-R_j, R_j = exponent of the row's max |x|
+// (the two halves exchange their maxima through xmax[256]). Called by all
+// threads of the CTA together.
 template <int D>
-__device__ __forceinline__ int load_window_row(const AttArgs &a, const TileRef &tr, uint8_t *E, uint32_t E_s, bool &valid) {
-    const int j = threadIdx.x;
+__device__ __forceinline__ int load_window_row(const AttArgs &a, const TileRef &tr, uint8_t *E, uint32_t E_s,
+                                               float *xmax, bool &valid) {
+    const int j = threadIdx.x & (kTile - 1);
+    const int kc0 = (threadIdx.x >> 7) * (D / 16);
     const int r = (tr.lt - tr.ctiles) * kTile + j;
     valid = r < tr.wlen;
-    if (!valid) {
-        for (int kc = 0; kc < D / 8; ++kc) *reinterpret_cast<uint4 *>(E + e_chunk_off<D>(j, kc)) = make_uint4(0, 0, 0, 0);
-        return 0;
-    }
-    const __nv_bfloat16 *src = a.win_kv + ((size_t)a.win_start[tr.i] + r) * D;
-#pragma unroll 8
-    for (int kc = 0; kc < D / 8; ++kc) cp_async16(E_s + e_chunk_off<D>(j, kc), src + 8 * kc);
-    asm volatile("cp.async.commit_group;\n\tcp.async.wait_all;" ::: "memory");
     float mx = 0.f;
-    for (int kc = 0; kc < D / 8; ++kc) {
-        uint4 u = *reinterpret_cast<const uint4 *>(E + e_chunk_off<D>(j, kc));
-        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+    if (!valid) {
+        for (int kc = kc0; kc < kc0 + D / 16; ++kc)
+            *reinterpret_cast<uint4 *>(E + e_chunk_off<D>(j, kc)) = make_uint4(0, 0, 0, 0);
+    } else {
+        const __nv_bfloat16 *src = a.win_kv + ((size_t)a.win_start[tr.i] + r) * D;
+#pragma unroll 8
+        for (int kc = kc0; kc < kc0 + D / 16; ++kc) cp_async16(E_s + e_chunk_off<D>(j, kc), src + 8 * kc);
+        asm volatile("cp.async.commit_group;\n\tcp.async.wait_all;" ::: "memory");
+        for (int kc = kc0; kc < kc0 + D / 16; ++kc) {
+            uint4 u = *reinterpret_cast<const uint4 *>(E + e_chunk_off<D>(j, kc));
+            const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            float2 f = __bfloat1622float2(h[k]);
-            mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
+            for (int k = 0; k < 4; ++k) {
+                float2 f = __bfloat1622float2(h[k]);
+                mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
+            }
         }
     }
+    xmax[threadIdx.x] = mx;
+    __syncthreads();
+    mx = fmaxf(xmax[j], xmax[j + kTile]);
+    if (!valid) return 0;
     const int R = mx > 0.f ? (int)((__float_as_uint(mx) >> 23) & 0xFF) - 127 : 0;
     const float inv = ldexpf(1.0f, -R);
-    for (int kc = 0; kc < D / 8; ++kc) {
+    for (int kc = kc0; kc < kc0 + D / 16; ++kc) {
         uint4 u = *reinterpret_cast<const uint4 *>(E + e_chunk_off<D>(j, kc));
         const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
         uint32_t o[4];
@@ -533,7 +553,8 @@ __global__ void __launch_bounds__(256) attend_merge_kernel(const long long *tpre
         for (int p = 0; p < np; ++p) rmax = fmaxf(rmax, part_rho[(size_t)slots[p] * kHeads + h]);
         float l = 0.f;
         for (int p = 0; p < np; ++p) {
-            const float wgt = exp2f(part_rho[(size_t)slots[p] * kHeads + h] - rmax);
+            // rho = -inf: no entry of this head in that partial (or in any, if rmax is -inf)
+            const float wgt = rmax == -INFINITY ? 0.f : exp2f(part_rho[(size_t)slots[p] * kHeads + h] - rmax);
             wts[p * kMergeHeads + threadIdx.x] = wgt;
             l += wgt * part_l[(size_t)slots[p] * kHeads + h];
         }
@@ -570,26 +591,31 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
     uint8_t *Q = E + C::E_BYTES;
     uint8_t *P = Q + C::Q_BYTES;
     uint8_t *misc = P + C::P_BYTES;
-    uint64_t *mbar = reinterpret_cast<uint64_t *>(misc);            // [0] S done, [1] PV done
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + 16);
-    int *flags = reinterpret_cast<int *>(misc + 32);                // [0] rescale, [1] last, [2] abort
+    uint64_t *mbar = reinterpret_cast<uint64_t *>(misc);            // [0] S done, [1] PV low half, [2] PV high half
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + 32);
+    int *flags = reinterpret_cast<int *>(misc + 48);                // [0] rescale, [1] abort
     float *rho = reinterpret_cast<float *>(misc + 64);              // [64]
     float *alpha = rho + 64;                                        // [64]
     float *wred = alpha + 64;                                       // [4][64]
+    float *xmax = wred + 4 * 64;                                    // [256]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int hf = tid >> 7;               // channel half (dequant) = head half (softmax)
     const long long T = a.tprefix[a.Nq];
     const int G = gridDim.x, c = blockIdx.x;
     const long long t_begin = T * c / G, t_end = T * (c + 1) / G;
     if (t_begin >= t_end) return;
 
     const uint32_t E_s = smem_u32(E), Q_s = smem_u32(Q), P_s = smem_u32(P);
-    const uint32_t mbar_s = smem_u32(&mbar[0]), mbar_pv = smem_u32(&mbar[1]);
+    const uint32_t mbar_s = smem_u32(&mbar[0]), mbar_lo = smem_u32(&mbar[1]), mbar_hi = smem_u32(&mbar[2]);
+    const uint32_t mbar_own = hf ? mbar_hi : mbar_lo;
     if (tid == 0) {
         mbar_init(mbar_s, 1);
-        mbar_init(mbar_pv, 1);
+        mbar_init(mbar_lo, 1);
+        mbar_init(mbar_hi, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        flags[2] = 0;
+        flags[0] = 0;
+        flags[1] = 0;
     }
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
@@ -601,10 +627,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tmem_s = tmem;                 // S^T: columns [0, 64)
-    const uint32_t tmem_o = tmem + kHeads;        // O^T d-tile dt: columns 64 + 64 dt
-    const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
-    uint32_t ph_s = 0, ph_pv = 0;
+    // TMEM lanes: warp w reaches lanes 32 (w % 4) .. + 31; its thread takes
+    // the 32 columns of head half hf of S^T (cols 0..63) and of every O^T d-tile
+    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+    const uint32_t tmem_s = tmem + lane_off + 32 * hf;               // S^T, this thread's 32 heads
+    const uint32_t tmem_o = tmem + lane_off + kHeads + 32 * hf;      // O^T d-tile dt at + 64 dt
+    uint32_t ph_s = 0;
+    uint32_t n_pv = 0;          // PV groups committed so far (each completes both halves' barriers once)
     bool pv_pending = false;
 
     constexpr uint32_t IDESC_S = idesc_f16(kTile, kHeads, false, false);
@@ -631,28 +660,28 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
         const bool whole = (seg_begin == cur.t0) && (seg_end == cur.t1);
         // the previous segment's PV must finish before Q' and O^T are reused
         if (pv_pending) {
-            const bool ok = mbar_wait(mbar_pv, ph_pv);
-            ph_pv ^= 1;
+            const bool ok = mbar_wait(mbar_lo, (n_pv - 1) & 1) && mbar_wait(mbar_hi, (n_pv - 1) & 1);
             pv_pending = false;
             if (__syncthreads_or(!ok)) { aborted = true; break; }
         }
         const int sQ = a.sq[i];
         load_query<D>(a, i, sQ, Q);
-        float l_part[2] = {0.f, 0.f};  // per-warp partial row sums of heads 2*lane, 2*lane+1
+        float lsum[32];         // row sums of this thread's 32 heads over its entries
+#pragma unroll
+        for (int k = 0; k < 32; ++k) lsum[k] = 0.f;
         bool first = true;
 
         for (; t < seg_end; ++t) {
-            // ---- operand E' for this tile ----
+            // ---- operand E' for this tile (each half waits for its own channels) ----
+            bool ok = true;
             if (pv_pending) {
-                const bool ok = mbar_wait(mbar_pv, ph_pv);
-                ph_pv ^= 1;
+                ok = mbar_wait(mbar_own, (n_pv - 1) & 1);
                 pv_pending = false;
-                if (__syncthreads_or(!ok)) { aborted = true; break; }
             }
             int Rj;
             bool valid;
             if (cur.win) {
-                Rj = load_window_row<D>(a, cur, E, E_s, valid);
+                Rj = load_window_row<D>(a, cur, E, E_s, xmax, valid);
             } else {
                 valid = rr.valid;
                 Rj = dequant_row<D>(rr, E);
@@ -670,7 +699,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
             }
             fence_async_smem();
             tc_fence_before();
-            __syncthreads();
+            if (__syncthreads_or(!ok)) { aborted = true; break; }
 
             // ---- S^T = E' Q'^T ----
             if (tid == 0) {
@@ -680,82 +709,93 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
                     const uint32_t koff = (uint32_t)((kk & 3) * 32);
                     const uint64_t da = desc_sw128(E_s + (kk >> 2) * C::KREG + koff, 16, 1024);
                     const uint64_t db = desc_sw128(Q_s + (kk >> 2) * C::QREG + koff, 16, 1024);
-                    mma_f16(tmem_s, da, db, IDESC_S, kk > 0);
+                    mma_f16(tmem, da, db, IDESC_S, kk > 0);
                 }
                 mma_commit(mbar_s);
             }
-            {
-                const bool ok = mbar_wait(mbar_s, ph_s);
-                ph_s ^= 1;
-                if (__syncthreads_or(!ok)) { aborted = true; break; }
-            }
+            if (!mbar_wait(mbar_s, ph_s)) flags[1] = 1;
+            ph_s ^= 1;
             tc_fence_after();
-            // u = log2(e) * scale * <q, e_j> + R_j, or -inf for an empty row.
-            // S^T stays in TMEM and is read twice (max, then P'), so no second
-            // 64-value copy has to live in registers.
+            // u = log2(e) * scale * <q, e_j> + R_j, or -inf for an empty row
             const float cj = ldexpf(a.scale_log2, Rj + sQ);
             const float rjf = (float)Rj;
-            // ---- per-head tile max -> reference update ----
-            {
-                float u[64];
-                tmem_ld64(tmem_s + lane_off, u);
+            float u[32];
+            tmem_ld32(tmem_s, u);
 #pragma unroll
-                for (int h = 0; h < 64; ++h) u[h] = valid ? fmaf(u[h], cj, rjf) : -INFINITY;
-                transpose_reduce64<true>(u);  // in place: lane L keeps heads 2L, 2L+1
-                wred[warp * 64 + 2 * lane] = u[0];
-                wred[warp * 64 + 2 * lane + 1] = u[1];
+            for (int k = 0; k < 32; ++k) u[k] = valid ? fmaf(u[k], cj, rjf) : -INFINITY;
+            float rh[32];
+#pragma unroll
+            for (int k = 0; k < 32; k += 4) {
+                const float4 r4 = *reinterpret_cast<const float4 *>(rho + 32 * hf + k);
+                rh[k] = r4.x; rh[k + 1] = r4.y; rh[k + 2] = r4.z; rh[k + 3] = r4.w;
             }
-            __syncthreads();
-            if (tid < 64) {
-                const float M = fmaxf(fmaxf(wred[tid], wred[64 + tid]), fmaxf(wred[128 + tid], wred[192 + tid]));
-                float al = 1.f;
-                if (first) {
-                    rho[tid] = (M == -INFINITY) ? 0.f : M;
-                } else if (M > rho[tid] + 8.f) {
-                    al = exp2f(rho[tid] - M);
-                    rho[tid] = M;
+            float over = -INFINITY;  // largest u - rho of this thread (rho stale on the first tile)
+#pragma unroll
+            for (int k = 0; k < 32; ++k) over = fmaxf(over, u[k] - rh[k]);
+            const bool need = __syncthreads_or(first || over > 8.f);
+            if (flags[1]) { aborted = true; break; }
+            if (need) {
+                // ---- per-head tile maximum -> reference update (first tile, or a logit > rho + 8)
+                {
+                    float m[32];
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) m[k] = u[k];
+                    transpose_reduce32<true>(m);  // lane L: head 32 hf + L over this warp's 32 entries
+                    wred[(warp & 3) * 64 + 32 * hf + lane] = m[0];
                 }
-                alpha[tid] = al;
-                if (al != 1.f) flags[0] = 1;
-            }
-            __syncthreads();
-            if (flags[0]) {  // rescale O^T columns and the row sums (PV of the previous tile is complete)
-                tc_fence_after();
+                __syncthreads();
+                if (tid < 64) {
+                    const float M = fmaxf(fmaxf(wred[tid], wred[64 + tid]), fmaxf(wred[128 + tid], wred[192 + tid]));
+                    float al = 1.f;
+                    if (first) {
+                        rho[tid] = M;  // may be -inf: no entry for this head yet
+                    } else if (M > rho[tid] + 8.f) {
+                        al = rho[tid] == -INFINITY ? 0.f : exp2f(rho[tid] - M);
+                        rho[tid] = M;
+                    }
+                    alpha[tid] = al;
+                    if (al != 1.f) flags[0] = 1;
+                }
+                __syncthreads();
+                if (flags[0]) {  // rescale O^T columns and row sums (PV of the previous tile is complete)
 #pragma unroll 1
-                for (int dt = 0; dt < C::DT; ++dt) {
-                    float o[64];
-                    tmem_ld64(tmem_o + 64 * dt + lane_off, o);
+                    for (int dt = 0; dt < C::DT; ++dt) {
+                        float o[32];
+                        tmem_ld32(tmem_o + 64 * dt, o);
 #pragma unroll
-                    for (int h = 0; h < 64; ++h) o[h] *= alpha[h];
-                    tmem_st64(tmem_o + 64 * dt + lane_off, o);
+                        for (int k = 0; k < 32; ++k) o[k] *= alpha[32 * hf + k];
+                        tmem_st32(tmem_o + 64 * dt, o);
+                    }
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) lsum[k] *= alpha[32 * hf + k];
                 }
-                l_part[0] *= alpha[2 * lane];
-                l_part[1] *= alpha[2 * lane + 1];
+#pragma unroll
+                for (int k = 0; k < 32; k += 4) {
+                    const float4 r4 = *reinterpret_cast<const float4 *>(rho + 32 * hf + k);
+                    rh[k] = r4.x; rh[k + 1] = r4.y; rh[k + 2] = r4.z; rh[k + 3] = r4.w;
+                }
             }
             // ---- P' = 2^(u - rho) (fp16, 8 heads per 16-byte store) and row sums ----
             {
-                float u[64];
-                tmem_ld64(tmem_s + lane_off, u);
+                const int j = tid & (kTile - 1);
                 const float rj_inv = ldexpf(1.0f, -Rj);
 #pragma unroll
-                for (int cc = 0; cc < 8; ++cc) {
+                for (int cc = 0; cc < 4; ++cc) {
                     uint32_t pk[4];
 #pragma unroll
                     for (int q2 = 0; q2 < 4; ++q2) {
-                        const int h = 8 * cc + 2 * q2;
-                        const float p0 = valid ? exp2f(fmaf(u[h], cj, rjf) - rho[h]) : 0.f;
-                        const float p1 = valid ? exp2f(fmaf(u[h + 1], cj, rjf) - rho[h + 1]) : 0.f;
+                        const int k = 8 * cc + 2 * q2;
+                        const float p0 = valid ? exp2f(u[k] - rh[k]) : 0.f;
+                        const float p1 = valid ? exp2f(u[k + 1] - rh[k + 1]) : 0.f;
                         __half2 hh = __floats2half2_rn(p0, p1);
                         pk[q2] = *reinterpret_cast<uint32_t *>(&hh);
-                        u[h] = p0 * rj_inv;      // row-sum term, in place
-                        u[h + 1] = p1 * rj_inv;
+                        lsum[k] = fmaf(p0, rj_inv, lsum[k]);
+                        lsum[k + 1] = fmaf(p1, rj_inv, lsum[k + 1]);
                     }
-                    const uint32_t off = (uint32_t)((tid >> 3) * 1024 + (tid & 7) * 128 + ((cc ^ (tid & 7)) << 4));
+                    const int chunk = 4 * hf + cc;
+                    const uint32_t off = (uint32_t)((j >> 3) * 1024 + (j & 7) * 128 + ((chunk ^ (j & 7)) << 4));
                     *reinterpret_cast<uint4 *>(P + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 }
-                transpose_reduce64<false>(u);
-                l_part[0] += u[0];
-                l_part[1] += u[1];
             }
             fence_async_smem();
             tc_fence_before();
@@ -769,11 +809,14 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
                     for (int kj = 0; kj < kTile / 16; ++kj) {
                         const uint64_t da = desc_sw128(E_s + (2 * dt) * C::KREG + kj * 2048, C::KREG, 1024);
                         const uint64_t db = desc_sw128(P_s + kj * 2048, 8192, 1024);
-                        mma_f16(tmem_o + 64 * dt, da, db, IDESC_PV, (first && kj == 0) ? 0u : 1u);
+                        mma_f16(tmem + kHeads + 64 * dt, da, db, IDESC_PV, (first && kj == 0) ? 0u : 1u);
                     }
+                    if (dt == C::DT / 2 - 1) mma_commit(mbar_lo);  // channels of the low half done
                 }
-                mma_commit(mbar_pv);
+                if (C::DT == 1) mma_commit(mbar_lo);
+                mma_commit(mbar_hi);
             }
+            ++n_pv;
             pv_pending = true;
             first = false;
             if (t + 1 < t_end) {
@@ -786,14 +829,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
 
         // ---------------- segment epilogue
         {
-            const bool ok = mbar_wait(mbar_pv, ph_pv);
-            ph_pv ^= 1;
+            const bool ok = mbar_wait(mbar_lo, (n_pv - 1) & 1) && mbar_wait(mbar_hi, (n_pv - 1) & 1);
             pv_pending = false;
             if (__syncthreads_or(!ok)) { aborted = true; break; }
         }
         tc_fence_after();
-        wred[warp * 64 + 2 * lane] = l_part[0];
-        wred[warp * 64 + 2 * lane + 1] = l_part[1];
+        transpose_reduce32<false>(lsum);  // lane L: head 32 hf + L over this warp's entries
+        wred[(warp & 3) * 64 + 32 * hf + lane] = lsum[0];
         __syncthreads();
         if (tid < 64) {
             const float l = wred[tid] + wred[64 + tid] + wred[128 + tid] + wred[192 + tid];
@@ -801,39 +843,33 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
         }
         __syncthreads();
         const int b_slot = 2 * c + ((seg_begin == T * c / G) ? 0 : 1);
-        if (whole) {
-            for (int dt = 0; dt < C::DT; ++dt) {
-                float o[64];
-                tmem_ld64(tmem_o + 64 * dt + lane_off, o);
-                const int d = 128 * dt + 32 * warp + lane;
+        float *dst = whole ? a.out + (size_t)i * a.H * D : a.part_o + (size_t)b_slot * kHeads * D;
+        for (int dt = 0; dt < C::DT; ++dt) {
+            float o[32];
+            tmem_ld32(tmem_o + 64 * dt, o);
+            const int d = 128 * dt + 32 * (warp & 3) + lane;
 #pragma unroll
-                for (int h = 0; h < 64; ++h) {
-                    if (h < a.H) {
+            for (int k = 0; k < 32; ++k) {
+                const int h = 32 * hf + k;
+                if (h < a.H) {
+                    float v = o[k];
+                    if (whole) {
                         const float l = alpha[h];
-                        a.out[((size_t)i * a.H + h) * D + d] = l > 0.f ? o[h] / l : 0.f;
+                        v = l > 0.f ? v / l : 0.f;
                     }
+                    dst[(size_t)h * D + d] = v;
                 }
             }
+        }
+        if (whole) {
             if (a.lse && tid < a.H) {
                 const float l = alpha[tid];
                 a.lse[(size_t)i * a.H + tid] = l > 0.f ? (rho[tid] + log2f(l)) * 0.69314718055994531f : -INFINITY;
             }
-        } else {
-            float *po = a.part_o + (size_t)b_slot * kHeads * D;
-            for (int dt = 0; dt < C::DT; ++dt) {
-                float o[64];
-                tmem_ld64(tmem_o + 64 * dt + lane_off, o);
-                const int d = 128 * dt + 32 * warp + lane;
-#pragma unroll
-                for (int h = 0; h < 64; ++h)
-                    if (h < a.H) po[(size_t)h * D + d] = o[h];
-            }
-            if (tid < 64) {
-                a.part_rho[(size_t)b_slot * kHeads + tid] = rho[tid];
-                a.part_l[(size_t)b_slot * kHeads + tid] = alpha[tid];
-            }
+        } else if (tid < 64) {
+            a.part_rho[(size_t)b_slot * kHeads + tid] = rho[tid];
+            a.part_l[(size_t)b_slot * kHeads + tid] = alpha[tid];
         }
-        __syncthreads();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
