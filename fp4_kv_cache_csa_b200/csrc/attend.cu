@@ -130,6 +130,23 @@ __device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity) {
     }
 }
 
+__device__ __forceinline__ void mbar_expect_tx(uint32_t mbar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mbar), "r"(bytes) : "memory");
+}
+
+// Bulk copy (no tensor map, no multicast) of `bytes` from global memory to this
+// CTA's shared memory, completing on mbar's transaction count.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t mbar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(mbar)
+                 : "memory");
+}
+
+// Programmatic dependent launch: wait for the preceding grid's results / let
+// the next grid start its prologue.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 #define CSA_LD16(base, r)                                                                                    \
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];" \
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), \
@@ -188,19 +205,26 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
 }
 
 // ---------------------------------------------------------------- arguments
+// Per-query schedule record (written by the schedule kernel's CTA 0).
+struct QInfo {
+    int4 a;        // request, entry slots, compressed tiles, window rows
+    int4 b;        // filled blocks of the request, 0, 0, 0
+    longlong2 t;   // the query's tiles [t0, t1) in the flat tile list
+};
+
 struct AttArgs {
     const uint8_t *fp4, *scale;      // cache planes
-    const int32_t *n_blocks;
-    const __nv_bfloat16 *q;          // [Nq][H][D]
     const int32_t *sel_idx;          // CSA: [Nq][topk]; HCA: null
     const __nv_bfloat16 *win_kv;     // [rows][D] or null
     const int64_t *win_start;
     float *out, *lse;
     int32_t *status;
     // schedule (workspace)
-    const int32_t *req, *nent, *ctiles, *wlen;
+    const QInfo *qinfo;              // [Nq]
     const long long *tprefix;        // [Nq+1]
+    const int32_t *cta_q;            // [G] first query of each CTA's range
     const int32_t *sq;               // [Nq] query scale exponents
+    const uint8_t *qimg;             // [Nq][Q_BYTES] Q' images
     float *part_o, *part_rho, *part_l;  // [2G][64][D], [2G][64], [2G][64]
     int Nq, H, cap, topk;
     float scale_log2;                // softmax_scale * log2(e)
@@ -230,28 +254,22 @@ struct TileRef {
 };
 
 __device__ __forceinline__ TileRef query_ref(const AttArgs &a, int i, long long t) {
+    const QInfo *qi = a.qinfo + i;
+    const int4 x = qi->a;
+    const int4 y = qi->b;
+    const longlong2 z = qi->t;
     TileRef r;
     r.i = i;
-    r.t0 = a.tprefix[i];
-    r.t1 = a.tprefix[i + 1];
+    r.b = x.x;
+    r.nent = x.y;
+    r.ctiles = x.z;
+    r.wlen = x.w;
+    r.nblk = y.x;
+    r.t0 = z.x;
+    r.t1 = z.y;
     r.lt = (int)(t - r.t0);
-    r.b = a.req[i];
-    r.nent = a.nent[i];
-    r.ctiles = a.ctiles[i];
-    r.wlen = a.wlen[i];
-    r.nblk = a.n_blocks[r.b];
     r.win = r.lt >= r.ctiles;
     return r;
-}
-
-// The tile holding flat index t (binary search; once per CTA).
-__device__ __forceinline__ TileRef locate(const AttArgs &a, long long t) {
-    int lo = 0, hi = a.Nq - 1;
-    while (lo < hi) {
-        int mid = (lo + hi + 1) >> 1;
-        if (a.tprefix[mid] <= t) lo = mid; else hi = mid - 1;
-    }
-    return query_ref(a, lo, t);
 }
 
 // The tile after r (t_next = its flat index): the same query, or the next one with tiles.
@@ -399,40 +417,12 @@ __device__ __forceinline__ int load_window_row(const AttArgs &a, const TileRef &
     return R;
 }
 
-// Q' = q * 2^-sQ in fp16, K-major with 128-byte swizzle, heads >= H zero.
-// sQ (from the schedule kernel) puts max|q| in [2^14, 2^15), so every bf16
-// value within 2^31 of the maximum converts exactly.
-template <int D>
-__device__ void load_query(const AttArgs &a, int i, int sQ, uint8_t *Q) {
-    const int tid = threadIdx.x;
-    const __nv_bfloat16 *qi = a.q + (size_t)i * a.H * D;
-    const float inv = ldexpf(1.0f, -sQ);
-    // chunk (h, kc): consecutive threads take consecutive heads, so the
-    // swizzled 16-byte stores of a warp spread over all eight bank groups
-#pragma unroll 8
-    for (int c = tid; c < kHeads * (D / 8); c += kThreads) {
-        const int h = c % kHeads;
-        const int kc = c / kHeads;
-        uint32_t o[4] = {0u, 0u, 0u, 0u};
-        if (h < a.H) {
-            uint4 u = __ldg(reinterpret_cast<const uint4 *>(qi + (size_t)h * D) + kc);
-            const __nv_bfloat162 *hh = reinterpret_cast<const __nv_bfloat162 *>(&u);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                float2 f = __bfloat1622float2(hh[k]);
-                __half2 x = __floats2half2_rn(f.x * inv, f.y * inv);
-                o[k] = *reinterpret_cast<uint32_t *>(&x);
-            }
-        }
-        const uint32_t off = (uint32_t)((kc >> 3) * Cfg<D>::QREG + (h >> 3) * 1024 + (h & 7) * 128 + (((kc & 7) ^ (h & 7)) << 4));
-        *reinterpret_cast<uint4 *>(Q + off) = make_uint4(o[0], o[1], o[2], o[3]);
-    }
-}
-
 // ---------------------------------------------------------------- schedule
 // One CTA per query. Every CTA: its query's scale exponent sq[i] (from
-// max|q|) and, when the query has no entry at all, out = 0 and lse = -inf.
-// CTA 0 also writes the per-query tile counts and their prefix.
+// max|q|), the Q' image (q * 2^-sq in fp16, in the swizzled K-major layout
+// the MMA reads, heads >= H zero) and, when the query has no entry at all,
+// out = 0 and lse = -inf. CTA 0 also writes the per-query records, the tile
+// prefix and the first query of every attention CTA's range.
 __device__ __forceinline__ void query_tiles(const int32_t *q_offsets, const int32_t *q_pos, const int32_t *n_blocks,
                                             const int32_t *win_len, int batch, int m, int cap, int topk, int max_win,
                                             int i, int32_t *status, int &b_out, int &ne, int &ct, int &wl) {
@@ -449,15 +439,18 @@ __device__ __forceinline__ void query_tiles(const int32_t *q_offsets, const int3
     b_out = b < 0 ? 0 : b;
 }
 
+template <int D>
 __global__ void __launch_bounds__(256) attend_schedule_kernel(
     const int32_t *q_offsets, const int32_t *q_pos, const int32_t *n_blocks, const int32_t *win_len, int batch,
-    int Nq, int m, int cap, int topk, int max_win, const __nv_bfloat16 *q, int H, int D, int32_t *req, int32_t *nent,
-    int32_t *ctiles, int32_t *wlen, long long *tprefix, int32_t *sq, float *out, float *lse, int32_t *status) {
+    int Nq, int m, int cap, int topk, int max_win, const __nv_bfloat16 *q, int H, int G, QInfo *qinfo,
+    long long *tprefix, int32_t *cta_q, int32_t *sq, uint8_t *qimg, float *out, float *lse, int32_t *status) {
     __shared__ long long red[32];
     __shared__ long long round_total;
     __shared__ float fred[8];
+    __shared__ int sq_s;
+    grid_dep_launch();  // the attention kernel may start its prologue; it waits for this grid's results
     const int qi = blockIdx.x;
-    // ---- this CTA's query: scale exponent and the empty case
+    // ---- this CTA's query: scale exponent, Q' image and the empty case
     {
         const __nv_bfloat16 *qp = q + (size_t)qi * H * D;
         const int nchunks = H * D / 8;
@@ -478,7 +471,31 @@ __global__ void __launch_bounds__(256) attend_schedule_kernel(
         if (threadIdx.x == 0) {
             float m8 = 0.f;
             for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m8 = fmaxf(m8, fred[w]);
-            sq[qi] = m8 > 0.f ? (int)((__float_as_uint(m8) >> 23) & 0xFF) - 127 - 14 : 0;
+            // 2^-sq puts max|q| in [2^14, 2^15): every bf16 value within 2^31 of it is exact in fp16
+            sq_s = m8 > 0.f ? (int)((__float_as_uint(m8) >> 23) & 0xFF) - 127 - 14 : 0;
+            sq[qi] = sq_s;
+        }
+        __syncthreads();
+        const float inv = ldexpf(1.0f, -sq_s);
+        uint8_t *img = qimg + (size_t)qi * Cfg<D>::Q_BYTES;
+        // chunk (h, kc): 8 channels of head h
+        for (int c = threadIdx.x; c < kHeads * (D / 8); c += blockDim.x) {
+            const int h = c / (D / 8);
+            const int kc = c % (D / 8);
+            uint32_t o[4] = {0u, 0u, 0u, 0u};
+            if (h < H) {
+                uint4 u = __ldg(reinterpret_cast<const uint4 *>(qp + (size_t)h * D) + kc);
+                const __nv_bfloat162 *hh = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    float2 f = __bfloat1622float2(hh[k]);
+                    __half2 x = __floats2half2_rn(f.x * inv, f.y * inv);
+                    o[k] = *reinterpret_cast<uint32_t *>(&x);
+                }
+            }
+            const size_t off =
+                (size_t)(kc >> 3) * Cfg<D>::QREG + (h >> 3) * 1024 + (h & 7) * 128 + (((kc & 7) ^ (h & 7)) << 4);
+            *reinterpret_cast<uint4 *>(img + off) = make_uint4(o[0], o[1], o[2], o[3]);
         }
         int b, ne, ct, wl;
         query_tiles(q_offsets, q_pos, n_blocks, win_len, batch, m, cap, topk, max_win, qi, nullptr, b, ne, ct, wl);
@@ -489,27 +506,44 @@ __global__ void __launch_bounds__(256) attend_schedule_kernel(
         }
     }
     if (blockIdx.x != 0) return;
-    // ---- CTA 0: tile counts and prefix over all queries
+    // ---- CTA 0: per-query records, tile prefix, first query of every CTA range
     long long carry = 0;
     for (int base = 0; base < Nq; base += blockDim.x) {
         const int i = base + threadIdx.x;
         long long tiles = 0;
+        int b = 0, ne = 0, ct = 0, wl = 0;
         if (i < Nq) {
-            int b, ne, ct, wl;
             query_tiles(q_offsets, q_pos, n_blocks, win_len, batch, m, cap, topk, max_win, i, status, b, ne, ct, wl);
-            req[i] = b;
-            nent[i] = ne;
-            ctiles[i] = ct;
-            wlen[i] = wl;
             tiles = ct + (wl + kTile - 1) / kTile;
         }
         const long long incl = block_inclusive_scan<long long>(tiles, red);
-        if (i < Nq) tprefix[i + 1] = carry + incl;
+        if (i < Nq) {
+            const long long t0 = carry + incl - tiles;
+            tprefix[i + 1] = t0 + tiles;
+            QInfo r;
+            r.a = make_int4(b, ne, ct, wl);
+            r.b = make_int4(n_blocks[b], 0, 0, 0);
+            r.t = make_longlong2(t0, t0 + tiles);
+            qinfo[i] = r;
+        }
         if (i == 0) tprefix[0] = 0;
         if (threadIdx.x == blockDim.x - 1) round_total = incl;
         __syncthreads();
         carry += round_total;
         __syncthreads();
+    }
+    __threadfence_block();
+    __syncthreads();
+    // first query of CTA c: the last i with tprefix[i] <= t_begin(c)
+    const long long T = carry;
+    for (int c = threadIdx.x; c < G; c += blockDim.x) {
+        const long long tb = T * c / G;
+        int lo = 0, hi = Nq - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (tprefix[mid] <= tb) lo = mid; else hi = mid - 1;
+        }
+        cta_q[c] = lo;
     }
 }
 
@@ -527,6 +561,7 @@ __global__ void __launch_bounds__(256) attend_merge_kernel(const long long *tpre
     __shared__ float wts[256 * kMergeHeads];
     __shared__ float inv_l[kMergeHeads];
     __shared__ int np_s;
+    grid_dep_wait();
     const int i = blockIdx.x;
     const int h0 = blockIdx.y * kMergeHeads;
     if (h0 >= H) return;
@@ -591,7 +626,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
     uint8_t *Q = E + C::E_BYTES;
     uint8_t *P = Q + C::Q_BYTES;
     uint8_t *misc = P + C::P_BYTES;
-    uint64_t *mbar = reinterpret_cast<uint64_t *>(misc);            // [0] S done, [1] PV low half, [2] PV high half
+    uint64_t *mbar = reinterpret_cast<uint64_t *>(misc);            // [0] S done, [1] PV low half, [2] PV high half, [3] Q' loaded
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + 32);
     int *flags = reinterpret_cast<int *>(misc + 48);                // [0] rescale, [1] abort
     float *rho = reinterpret_cast<float *>(misc + 64);              // [64]
@@ -601,6 +636,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int hf = tid >> 7;               // channel half (dequant) = head half (softmax)
+    grid_dep_wait();                       // the schedule kernel's records (programmatic launch)
     const long long T = a.tprefix[a.Nq];
     const int G = gridDim.x, c = blockIdx.x;
     const long long t_begin = T * c / G, t_end = T * (c + 1) / G;
@@ -608,11 +644,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
 
     const uint32_t E_s = smem_u32(E), Q_s = smem_u32(Q), P_s = smem_u32(P);
     const uint32_t mbar_s = smem_u32(&mbar[0]), mbar_lo = smem_u32(&mbar[1]), mbar_hi = smem_u32(&mbar[2]);
+    const uint32_t mbar_q = smem_u32(&mbar[3]);
     const uint32_t mbar_own = hf ? mbar_hi : mbar_lo;
     if (tid == 0) {
         mbar_init(mbar_s, 1);
         mbar_init(mbar_lo, 1);
         mbar_init(mbar_hi, 1);
+        mbar_init(mbar_q, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         flags[0] = 0;
         flags[1] = 0;
@@ -640,7 +678,14 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
     constexpr uint32_t IDESC_PV = idesc_f16(kTile, kHeads, true, true);
 
     RowRegs<D> rr;
-    TileRef cur = locate(a, t_begin);
+    TileRef cur = query_ref(a, a.cta_q[c], t_begin);
+    // the first query's Q' image: one bulk copy (the schedule kernel wrote it)
+    if (tid == 0) {
+        mbar_expect_tx(mbar_q, C::Q_BYTES);
+        bulk_g2s(Q_s, a.qimg + (size_t)cur.i * C::Q_BYTES, C::Q_BYTES, mbar_q);
+    }
+    uint32_t n_q = 0;           // Q' copies waited for
+    uint32_t n_q_issued = 1;    // ... and issued
     prefetch_row<D>(a, cur, row_block_raw(a, cur), rr);
     // the next tile and this thread's selected index in it (one tile ahead of its row loads)
     TileRef nxt = cur;
@@ -665,7 +710,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
             if (__syncthreads_or(!ok)) { aborted = true; break; }
         }
         const int sQ = a.sq[i];
-        load_query<D>(a, i, sQ, Q);
+        // Q' of this query (issued at kernel start or in the previous segment's epilogue)
+        if (__syncthreads_or(!mbar_wait(mbar_q, n_q & 1))) { aborted = true; break; }
+        ++n_q;
         float lsum[32];         // row sums of this thread's 32 heads over its entries
 #pragma unroll
         for (int k = 0; k < 32; ++k) lsum[k] = 0.f;
@@ -834,6 +881,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
             if (__syncthreads_or(!ok)) { aborted = true; break; }
         }
         tc_fence_after();
+        if (t < t_end && tid == 0) {  // the next segment's Q' (this segment's S MMAs are complete)
+            mbar_expect_tx(mbar_q, C::Q_BYTES);
+            bulk_g2s(Q_s, a.qimg + (size_t)cur.i * C::Q_BYTES, C::Q_BYTES, mbar_q);
+        }
+        if (t < t_end) ++n_q_issued;
         transpose_reduce32<false>(lsum);  // lane L: head 32 hf + L over this warp's entries
         wred[(warp & 3) * 64 + 32 * hf + lane] = lsum[0];
         __syncthreads();
@@ -877,6 +929,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
 
     if (aborted) {
         if (tid == 0) flag(a.status, CSA_DEV_TIMEOUT);
+        if (n_q_issued > n_q) mbar_wait(mbar_q, n_q & 1);  // no copy may land after the CTA exits
     }
     tc_fence_before();
     __syncthreads();
@@ -885,20 +938,49 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TMEM_COLS) : "memory");
 }
 
+template <int D>
+cudaError_t launch_main(const AttArgs &a, int num_ctas, cudaStream_t s) {
+    cudaError_t err;
+    const int smem = Cfg<D>::SMEM;
+    if ((err = cudaFuncSetAttribute(attend_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
+        return err;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(num_ctas);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, attend_kernel<D>, a);
+}
+
+template <int D>
+cudaError_t launch_schedule(const csa_cache &c, const AttArgs &a, const int32_t *q_offsets, const int32_t *q_pos,
+                            const int32_t *win_len, int topk, int max_win, const void *q, int num_ctas, QInfo *qinfo,
+                            long long *tprefix, int32_t *cta_q, int32_t *sq, uint8_t *qimg, cudaStream_t s) {
+    attend_schedule_kernel<D><<<a.Nq, 256, 0, s>>>(q_offsets, q_pos, c.n_blocks, win_len, c.batch, a.Nq, c.block,
+                                                   c.capacity, topk, max_win, static_cast<const __nv_bfloat16 *>(q),
+                                                   a.H, num_ctas, qinfo, tprefix, cta_q, sq, qimg, a.out, a.lse,
+                                                   c.status);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 size_t attend_workspace_bytes(int Nq, int D, int num_ctas) {
     size_t off = 0;
     auto take = [&](size_t bytes) { off = (off + bytes + 255) & ~size_t(255); };
-    take(4 * (size_t)Nq);            // req
-    take(4 * (size_t)Nq);            // nent
-    take(4 * (size_t)Nq);            // ctiles
-    take(4 * (size_t)Nq);            // wlen
-    take(8 * (size_t)(Nq + 1));      // tprefix
-    take(4 * (size_t)Nq);            // sq
-    take(4 * (size_t)2 * num_ctas * kHeads * D);  // part_o
-    take(4 * (size_t)2 * num_ctas * kHeads);      // part_rho
-    take(4 * (size_t)2 * num_ctas * kHeads);      // part_l
+    take(sizeof(QInfo) * (size_t)Nq);                 // qinfo
+    take(8 * (size_t)(Nq + 1));                       // tprefix
+    take(4 * (size_t)num_ctas);                       // cta_q
+    take(4 * (size_t)Nq);                             // sq
+    take((size_t)Nq * kHeads * D * 2);                // qimg
+    take(4 * (size_t)2 * num_ctas * kHeads * D);      // part_o
+    take(4 * (size_t)2 * num_ctas * kHeads);          // part_rho
+    take(4 * (size_t)2 * num_ctas * kHeads);          // part_l
     return off;
 }
 
@@ -915,31 +997,27 @@ cudaError_t launch_attend(const csa_cache &c, const void *q, int Nq, int H, cons
         return p;
     };
     AttArgs a;
-    int32_t *req = reinterpret_cast<int32_t *>(take(4 * (size_t)Nq));
-    int32_t *nent = reinterpret_cast<int32_t *>(take(4 * (size_t)Nq));
-    int32_t *ctiles = reinterpret_cast<int32_t *>(take(4 * (size_t)Nq));
-    int32_t *wlen = reinterpret_cast<int32_t *>(take(4 * (size_t)Nq));
+    QInfo *qinfo = reinterpret_cast<QInfo *>(take(sizeof(QInfo) * (size_t)Nq));
     long long *tprefix = reinterpret_cast<long long *>(take(8 * (size_t)(Nq + 1)));
+    int32_t *cta_q = reinterpret_cast<int32_t *>(take(4 * (size_t)num_ctas));
     int32_t *sq = reinterpret_cast<int32_t *>(take(4 * (size_t)Nq));
+    uint8_t *qimg = reinterpret_cast<uint8_t *>(take((size_t)Nq * kHeads * D * 2));
     a.part_o = reinterpret_cast<float *>(take(4 * (size_t)2 * num_ctas * kHeads * D));
     a.part_rho = reinterpret_cast<float *>(take(4 * (size_t)2 * num_ctas * kHeads));
     a.part_l = reinterpret_cast<float *>(take(4 * (size_t)2 * num_ctas * kHeads));
     a.fp4 = c.fp4;
     a.scale = c.scale;
-    a.n_blocks = c.n_blocks;
-    a.q = static_cast<const __nv_bfloat16 *>(q);
     a.sel_idx = sel_idx;
     a.win_kv = static_cast<const __nv_bfloat16 *>(win_kv);
     a.win_start = win_start;
     a.out = out;
     a.lse = lse;
     a.status = c.status;
-    a.req = req;
-    a.nent = nent;
-    a.ctiles = ctiles;
-    a.wlen = wlen;
+    a.qinfo = qinfo;
     a.tprefix = tprefix;
+    a.cta_q = cta_q;
     a.sq = sq;
+    a.qimg = qimg;
     a.Nq = Nq;
     a.H = H;
     a.cap = c.capacity;
@@ -947,28 +1025,33 @@ cudaError_t launch_attend(const csa_cache &c, const void *q, int Nq, int H, cons
     a.scale_log2 = softmax_scale * 1.4426950408889634f;
 
     cudaError_t err;
-    attend_schedule_kernel<<<Nq, 256, 0, s>>>(q_offsets, sel_idx ? nullptr : q_pos, c.n_blocks,
-                                               win_kv ? win_len : nullptr, c.batch, Nq, c.block, c.capacity, topk,
-                                               max_win, static_cast<const __nv_bfloat16 *>(q), H, D, req, nent, ctiles,
-                                               wlen, tprefix, sq, out, lse, c.status);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    const int32_t *qp = sel_idx ? nullptr : q_pos;
+    const int32_t *wl = win_kv ? win_len : nullptr;
     if (D == 512) {
-        const int smem = Cfg<512>::SMEM;
-        if ((err = cudaFuncSetAttribute(attend_kernel<512>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
+        if ((err = launch_schedule<512>(c, a, q_offsets, qp, wl, topk, max_win, q, num_ctas, qinfo, tprefix, cta_q, sq,
+                                        qimg, s)) != cudaSuccess)
             return err;
-        attend_kernel<512><<<num_ctas, kThreads, smem, s>>>(a);
+        if ((err = launch_main<512>(a, num_ctas, s)) != cudaSuccess) return err;
     } else if (D == 128) {
-        const int smem = Cfg<128>::SMEM;
-        if ((err = cudaFuncSetAttribute(attend_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
+        if ((err = launch_schedule<128>(c, a, q_offsets, qp, wl, topk, max_win, q, num_ctas, qinfo, tprefix, cta_q, sq,
+                                        qimg, s)) != cudaSuccess)
             return err;
-        attend_kernel<128><<<num_ctas, kThreads, smem, s>>>(a);
+        if ((err = launch_main<128>(a, num_ctas, s)) != cudaSuccess) return err;
     } else {
         return cudaErrorInvalidValue;
     }
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    attend_merge_kernel<<<dim3(Nq, (H + kMergeHeads - 1) / kMergeHeads), 256, 0, s>>>(
-        tprefix, Nq, H, D, num_ctas, a.part_o, a.part_rho, a.part_l, out, lse);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(Nq, (H + kMergeHeads - 1) / kMergeHeads);
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, attend_merge_kernel, (const long long *)tprefix, Nq, H, D, num_ctas,
+                              (const float *)a.part_o, (const float *)a.part_rho, (const float *)a.part_l, out, lse);
 }
 
 }  // namespace csa
