@@ -10,6 +10,29 @@ namespace csa {
 
 constexpr int kWarp = 32;
 
+// Programmatic dependent launch: a kernel launched with launch_pdl() may start
+// while the previous kernel on the stream finishes; grid_dep_wait() blocks until
+// that kernel has completed and its writes are visible, grid_dep_launch() lets
+// the next kernel begin its launch early.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Launch kern<<<grid, block, smem, s>>>(args...) with programmatic stream serialization.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 __device__ __forceinline__ void flag(int32_t *status, int32_t bits) {
     if (status) atomicOr(status, bits);
 }

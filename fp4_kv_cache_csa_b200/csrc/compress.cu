@@ -38,40 +38,41 @@ __device__ __forceinline__ uint32_t e2m1_code(float s) {
     return sign | c;
 }
 
+// N consecutive bf16 values as N/2 raw 32-bit words (widest loads that fit).
 template <int N>
-__device__ __forceinline__ void load_bf16(const __nv_bfloat16 *p, float (&x)[N]) {
+__device__ __forceinline__ void load_raw(const __nv_bfloat16 *p, uint32_t (&w)[N / 2]) {
     static_assert(N % 2 == 0, "even channel count per lane");
     if constexpr (N % 8 == 0) {
 #pragma unroll
         for (int v = 0; v < N / 8; ++v) {
-            uint4 u = __ldg(reinterpret_cast<const uint4 *>(p) + v);
-            const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                float2 f = __bfloat1622float2(h[k]);
-                x[8 * v + 2 * k] = f.x;
-                x[8 * v + 2 * k + 1] = f.y;
-            }
+            const uint4 u = __ldg(reinterpret_cast<const uint4 *>(p) + v);
+            w[4 * v] = u.x;
+            w[4 * v + 1] = u.y;
+            w[4 * v + 2] = u.z;
+            w[4 * v + 3] = u.w;
         }
     } else if constexpr (N % 4 == 0) {
 #pragma unroll
         for (int v = 0; v < N / 4; ++v) {
-            uint2 u = __ldg(reinterpret_cast<const uint2 *>(p) + v);
-            const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
-#pragma unroll
-            for (int k = 0; k < 2; ++k) {
-                float2 f = __bfloat1622float2(h[k]);
-                x[4 * v + 2 * k] = f.x;
-                x[4 * v + 2 * k + 1] = f.y;
-            }
+            const uint2 u = __ldg(reinterpret_cast<const uint2 *>(p) + v);
+            w[2 * v] = u.x;
+            w[2 * v + 1] = u.y;
         }
     } else {
 #pragma unroll
-        for (int v = 0; v < N / 2; ++v) {
-            float2 f = __bfloat1622float2(__ldg(reinterpret_cast<const __nv_bfloat162 *>(p) + v));
-            x[2 * v] = f.x;
-            x[2 * v + 1] = f.y;
-        }
+        for (int v = 0; v < N / 2; ++v) w[v] = __ldg(reinterpret_cast<const uint32_t *>(p) + v);
+    }
+}
+
+template <int N>
+__device__ __forceinline__ void unpack_bf16(const uint32_t (&w)[N / 2], float (&x)[N]) {
+#pragma unroll
+    for (int v = 0; v < N / 2; ++v) {
+        __nv_bfloat162 h;
+        *reinterpret_cast<uint32_t *>(&h) = w[v];
+        const float2 f = __bfloat1622float2(h);
+        x[2 * v] = f.x;
+        x[2 * v + 1] = f.y;
     }
 }
 
@@ -91,13 +92,19 @@ struct CompressArgs {
 
 // E channels per lane (D = 32*E), EI indexer channels per lane (0 = no
 // indexer keys), WPB warps per block: WPB = 1 puts four independent blocks in
-// a CTA; WPB = 8 splits one block's tokens over eight warps (large m), whose
-// online-softmax states are then combined through shared memory.
+// a CTA; WPB > 1 splits one block's tokens over WPB warps (large m), whose
+// online-softmax states are then combined through shared memory. Each warp
+// loads kChunk tokens at a time.
 template <int E, int EI, int WPB>
 __global__ void __launch_bounds__(WPB == 1 ? kWarpsPerCta * kWarp : WPB * kWarp)
 pool_quantize_kernel(CompressArgs a) {
     constexpr int EK = EI > 0 ? EI : 2;
-    constexpr int kChunk = 4;  // tokens in flight per warp step
+    // tokens in flight per warp step (fewer where 16 warps would run out of registers)
+    constexpr int kChunk = WPB == 1 ? 4 : (WPB == 16 && E + EK >= 20) ? 4 : 8;
+    // inputs may come from the previous kernel on the stream: wait for it, then
+    // let the next kernel (the commit) begin launching
+    grid_dep_wait();
+    grid_dep_launch();
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int b = blockIdx.y;
@@ -105,17 +112,10 @@ pool_quantize_kernel(CompressArgs a) {
     const int wib = WPB == 1 ? 0 : warp;  // warp index inside the block's team
     const int t_begin = a.tok_offsets[b];
     const int count = a.tok_offsets[b + 1] - t_begin;
-    const int base = a.n_blocks[b];
-    if (count < 0 || count % a.m != 0) {
-        if (jb == 0 && threadIdx.x == 0) flag(a.status, CSA_DEV_TOKEN_COUNT);
-        return;
-    }
-    const int nb = count / a.m;
-    if ((long long)base + nb > a.cap) {
-        if (jb == 0 && threadIdx.x == 0) flag(a.status, CSA_DEV_CAPACITY);
-        return;
-    }
-    if (jb >= nb) return;
+    const bool count_ok = count >= 0 && count % a.m == 0;
+    const int nb = count_ok ? count / a.m : 0;
+    const bool active = jb < nb;  // CTA-uniform when WPB > 1
+    const int base = a.n_blocks[b];  // checked after the token loads are in flight
 
     float wg[E];
 #pragma unroll
@@ -131,49 +131,56 @@ pool_quantize_kernel(CompressArgs a) {
     for (int k = 0; k < EK; ++k) acck[k] = 0.f;
 
     const long long tok0 = (long long)t_begin + (long long)jb * a.m;
-    for (int c0 = wib * kChunk; c0 < a.m; c0 += WPB * kChunk) {
-        float x[kChunk][E], xk[kChunk][EK], g[kChunk];
+    for (int c0 = wib * kChunk; active && c0 < a.m; c0 += WPB * kChunk) {
+        uint32_t xr[kChunk][E / 2], kr[kChunk][EK / 2];
 #pragma unroll
         for (int u = 0; u < kChunk; ++u) {
             if (c0 + u < a.m) {
-                load_bf16<E>(a.kv_tok + (tok0 + c0 + u) * a.D + lane * E, x[u]);
-                if constexpr (EI > 0) load_bf16<EI>(a.idx_tok + (tok0 + c0 + u) * a.dI + lane * EI, xk[u]);
+                load_raw<E>(a.kv_tok + (tok0 + c0 + u) * a.D + lane * E, xr[u]);
+                if constexpr (EI > 0) load_raw<EI>(a.idx_tok + (tok0 + c0 + u) * a.dI + lane * EI, kr[u]);
             }
         }
-        float cmax = -INFINITY;
 #pragma unroll
         for (int u = 0; u < kChunk; ++u) {
             if (c0 + u < a.m) {
+                float x[E];
+                unpack_bf16<E>(xr[u], x);
                 float part = 0.f;
 #pragma unroll
-                for (int k = 0; k < E; ++k) part = fmaf(x[u][k], wg[k], part);
-                g[u] = warp_sum(part);
-                cmax = fmaxf(cmax, g[u]);
-            }
-        }
-        if (cmax > mu) {  // new maximum: rescale what has been accumulated
-            const float r = (mu == -INFINITY) ? 0.f : expf(mu - cmax);
-            den *= r;
+                for (int k = 0; k < E; ++k) part = fmaf(x[k], wg[k], part);
+                const float g = warp_sum(part);
+                if (g > mu) {  // new maximum: rescale what has been accumulated
+                    const float r = (mu == -INFINITY) ? 0.f : expf(mu - g);
+                    den *= r;
 #pragma unroll
-            for (int k = 0; k < E; ++k) acc[k] *= r;
+                    for (int k = 0; k < E; ++k) acc[k] *= r;
 #pragma unroll
-            for (int k = 0; k < EK; ++k) acck[k] *= r;
-            mu = cmax;
-        }
-#pragma unroll
-        for (int u = 0; u < kChunk; ++u) {
-            if (c0 + u < a.m) {
-                const float p = expf(g[u] - mu);
+                    for (int k = 0; k < EK; ++k) acck[k] *= r;
+                    mu = g;
+                }
+                const float p = expf(g - mu);
                 den += p;
 #pragma unroll
-                for (int k = 0; k < E; ++k) acc[k] = fmaf(p, x[u][k], acc[k]);
+                for (int k = 0; k < E; ++k) acc[k] = fmaf(p, x[k], acc[k]);
                 if constexpr (EI > 0) {
+                    float xk[EI];
+                    unpack_bf16<EI>(kr[u], xk);
 #pragma unroll
-                    for (int k = 0; k < EI; ++k) acck[k] = fmaf(p, xk[u][k], acck[k]);
+                    for (int k = 0; k < EI; ++k) acck[k] = fmaf(p, xk[k], acck[k]);
                 }
             }
         }
     }
+
+    if (!count_ok) {
+        if (jb == 0 && threadIdx.x == 0) flag(a.status, CSA_DEV_TOKEN_COUNT);
+        return;
+    }
+    if ((long long)base + nb > a.cap) {
+        if (jb == 0 && threadIdx.x == 0) flag(a.status, CSA_DEV_CAPACITY);
+        return;
+    }
+    if (!active) return;
 
     if constexpr (WPB > 1) {
         // combine the warps' partial softmax states; warp 0 finishes the block
@@ -263,6 +270,7 @@ pool_quantize_kernel(CompressArgs a) {
 // Advance n_blocks after the pooling kernel has read the old values; applies
 // the same checks, so a rejected request is left untouched.
 __global__ void commit_kernel(const int32_t *tok_offsets, int32_t *n_blocks, int batch, int m, int cap) {
+    grid_dep_wait();
     for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < batch; b += gridDim.x * blockDim.x) {
         const int count = tok_offsets[b + 1] - tok_offsets[b];
         if (count < 0 || count % m != 0) continue;
@@ -271,23 +279,35 @@ __global__ void commit_kernel(const int32_t *tok_offsets, int32_t *n_blocks, int
     }
 }
 
-template <int E, int WPB>
-cudaError_t launch_ew(const CompressArgs &a, dim3 grid, cudaStream_t s) {
-    const dim3 block(WPB == 1 ? kWarpsPerCta * kWarp : WPB * kWarp);
-    switch (a.idx_key ? a.dI / 32 : 0) {
-        case 0: pool_quantize_kernel<E, 0, WPB><<<grid, block, 0, s>>>(a); break;
-        case 2: pool_quantize_kernel<E, 2, WPB><<<grid, block, 0, s>>>(a); break;
-        case 4: pool_quantize_kernel<E, 4, WPB><<<grid, block, 0, s>>>(a); break;
-        case 8: pool_quantize_kernel<E, 8, WPB><<<grid, block, 0, s>>>(a); break;
-        default: return cudaErrorInvalidValue;
-    }
-    return cudaGetLastError();
+// Warps of a block team: 16, or 8 when the team's combine buffers would not
+// fit the 48 KB of static shared memory.
+template <int E, int EI>
+constexpr int team_warps() {
+    return (E + (EI > 0 ? EI : 2)) * kWarp * 4 * 16 <= 40 * 1024 ? 16 : 8;
 }
 
-// m >= 32: eight warps per block; otherwise four blocks per CTA, one warp each
+template <int E, int EI, int WPB>
+cudaError_t launch_one(const CompressArgs &a, dim3 grid, cudaStream_t s) {
+    constexpr int W = WPB == 1 ? 1 : team_warps<E, EI>();
+    const dim3 block(W == 1 ? kWarpsPerCta * kWarp : W * kWarp);
+    return launch_pdl(pool_quantize_kernel<E, EI, W>, grid, block, 0, s, a);
+}
+
+template <int E, int WPB>
+cudaError_t launch_ew(const CompressArgs &a, dim3 grid, cudaStream_t s) {
+    switch (a.idx_key ? a.dI / 32 : 0) {
+        case 0: return launch_one<E, 0, WPB>(a, grid, s);
+        case 2: return launch_one<E, 2, WPB>(a, grid, s);
+        case 4: return launch_one<E, 4, WPB>(a, grid, s);
+        case 8: return launch_one<E, 8, WPB>(a, grid, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+// m >= 32: a team of warps per block; otherwise four blocks per CTA, one warp each
 template <int E>
 cudaError_t launch_e(const CompressArgs &a, int max_blocks, int batch, cudaStream_t s) {
-    if (a.m >= 32) return launch_ew<E, 8>(a, dim3(max_blocks, batch), s);
+    if (a.m >= 32) return launch_ew<E, 2>(a, dim3(max_blocks, batch), s);
     return launch_ew<E, 1>(a, dim3((max_blocks + kWarpsPerCta - 1) / kWarpsPerCta, batch), s);
 }
 
@@ -323,8 +343,8 @@ cudaError_t launch_compress(const csa_cache &c, const void *kv_tok, const void *
         }
         if (err != cudaSuccess) return err;
     }
-    commit_kernel<<<(c.batch + 255) / 256, 256, 0, s>>>(tok_offsets, c.n_blocks, c.batch, c.block, c.capacity);
-    return cudaGetLastError();
+    return launch_pdl(commit_kernel, dim3((c.batch + 255) / 256), dim3(256), 0, s, tok_offsets, c.n_blocks, c.batch,
+                      c.block, c.capacity);
 }
 
 }  // namespace csa

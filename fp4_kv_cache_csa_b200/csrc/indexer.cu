@@ -127,6 +127,8 @@ __global__ void schedule_kernel(const int32_t *q_offsets, const int32_t *q_pos, 
                                 long long *gprefix, int32_t *thresh) {
     __shared__ long long red[32];
     __shared__ long long round_total;
+    grid_dep_wait();
+    grid_dep_launch();
     long long carry = 0;
     for (int base = 0; base < Nq; base += blockDim.x) {
         const int i = base + threadIdx.x;
@@ -245,6 +247,8 @@ struct ScanCfg {
 template <bool E4M3, int KS>
 __global__ void __launch_bounds__(kScanThreads, 2) scan_kernel(ScanArgs a) {
     using C = ScanCfg<E4M3, KS>;
+    grid_dep_wait();    // the schedule kernel's ranges (programmatic launch)
+    grid_dep_launch();
     __shared__ uint32_t hist[kBins];
     __shared__ uint32_t scan_smem[32];
     __shared__ BinPick pick;
@@ -440,6 +444,8 @@ struct SelArgs {
 // Keys above the threshold bin -> bitmap; keys in it -> candidate list.
 // Grid: (chunks of 128 x kPassThreads/32 scores, Nq).
 __global__ void __launch_bounds__(kPassThreads) select_pass_kernel(SelArgs a) {
+    grid_dep_wait();
+    grid_dep_launch();
     const int i = blockIdx.y;
     const int n = a.n_vis[i];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -554,6 +560,7 @@ __device__ __forceinline__ int key_digit(int level, uint32_t key) {
 
 __global__ void __launch_bounds__(kSelThreads) select_final_kernel(SelArgs a) {
     extern __shared__ uint32_t dyn[];
+    grid_dep_wait();
     uint32_t *bm = dyn;                                                // [words] selected blocks
     uint32_t *tie = dyn + a.words;                                     // [words] members tied on the key
     uint32_t *sck = dyn + 2 * a.words;                                 // [smem_cands] candidate keys
@@ -729,8 +736,7 @@ __global__ void __launch_bounds__(kSelThreads) select_final_kernel(SelArgs a) {
 
 template <bool E4M3, int KS>
 cudaError_t launch_scan(const ScanArgs &sa, int grid, cudaStream_t s) {
-    scan_kernel<E4M3, KS><<<grid, kScanThreads, 0, s>>>(sa);
-    return cudaGetLastError();
+    return launch_pdl(scan_kernel<E4M3, KS>, dim3(grid), dim3(kScanThreads), 0, s, sa);
 }
 
 }  // namespace
@@ -744,9 +750,9 @@ cudaError_t launch_index_topk(const csa_cache &c, const void *q_idx, const float
     carve(workspace, Nq, c.capacity, &ws);
     cudaError_t err = cudaMemsetAsync(ws.done, 0, ws.zero_bytes, s);  // counters, histograms, bitmaps
     if (err != cudaSuccess) return err;
-    schedule_kernel<<<1, 1024, 0, s>>>(q_offsets, q_pos, c.n_blocks, c.batch, Nq, c.block, c.capacity, topk,
-                                       ws.req, ws.n_vis, ws.gprefix, ws.thresh);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    err = launch_pdl(schedule_kernel, dim3(1), dim3(1024), 0, s, q_offsets, q_pos, c.n_blocks, c.batch, Nq, c.block,
+                     c.capacity, topk, ws.req, ws.n_vis, ws.gprefix, ws.thresh);
+    if (err != cudaSuccess) return err;
 
     ScanArgs sa;
     sa.keys = static_cast<const uint8_t *>(c.idx_key);
@@ -794,8 +800,7 @@ cudaError_t launch_index_topk(const csa_cache &c, const void *q_idx, const float
     const int want = (16 * num_sms + Nq - 1) / Nq;
     if (gx > want) gx = want;
     if (gx < 1) gx = 1;
-    select_pass_kernel<<<dim3(gx, Nq), kPassThreads, 0, s>>>(sel);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    if ((err = launch_pdl(select_pass_kernel, dim3(gx, Nq), dim3(kPassThreads), 0, s, sel)) != cudaSuccess) return err;
     // dynamic shared memory: the bitmap, then as many candidates as fit next to
     // the ~33 KB of static shared memory (opt in every time: cheap, valid in capture)
     const int kDynMax = 200 * 1024;
@@ -805,8 +810,7 @@ cudaError_t launch_index_topk(const csa_cache &c, const void *q_idx, const float
     const int smem = 8 * ws.words + 8 * sel.smem_cands;
     err = cudaFuncSetAttribute(select_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
-    select_final_kernel<<<Nq, kSelThreads, smem, s>>>(sel);
-    return cudaGetLastError();
+    return launch_pdl(select_final_kernel, dim3(Nq), dim3(kSelThreads), (size_t)smem, s, sel);
 }
 
 }  // namespace csa
