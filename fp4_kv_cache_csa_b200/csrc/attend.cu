@@ -414,7 +414,7 @@ __device__ __forceinline__ int load_window_row(const AttArgs &a, const TileRef &
 }
 
 // ---------------------------------------------------------------- schedule
-// One CTA per query. Every CTA: its query's scale exponent sq[i] (from
+// One CTA of 1024 threads per query. Every CTA: its query's scale exponent sq[i] (from
 // max|q|), the Q' image (q * 2^-sq in fp16, in the swizzled K-major layout
 // the MMA reads, heads >= H zero) and, when the query has no entry at all,
 // out = 0 and lse = -inf. CTA 0 also writes the per-query records, the tile
@@ -436,25 +436,29 @@ __device__ __forceinline__ void query_tiles(const int32_t *q_offsets, const int3
 }
 
 template <int D>
-__global__ void __launch_bounds__(256) attend_schedule_kernel(
+__global__ void __launch_bounds__(1024) attend_schedule_kernel(
     const int32_t *q_offsets, const int32_t *q_pos, const int32_t *n_blocks, const int32_t *win_len, int batch,
     int Nq, int m, int cap, int topk, int max_win, const __nv_bfloat16 *q, int H, int G, QInfo *qinfo,
     long long *tprefix, int32_t *cta_q, int32_t *sq, uint8_t *qimg, float *out, float *lse, int32_t *status) {
     __shared__ long long red[32];
     __shared__ long long round_total;
-    __shared__ float fred[8];
+    __shared__ float fred[32];
     __shared__ int sq_s;
     grid_dep_launch();  // the attention kernel may start its prologue; it waits for this grid's results
     const int qi = blockIdx.x;
     // ---- this CTA's query: scale exponent, Q' image and the empty case
     {
+        // the query is read once: chunk c = 8 channels (h = c / (D/8), kc = c % (D/8)), kept in registers
+        constexpr int kPer = (kHeads * (D / 8) + 1023) / 1024;
         const __nv_bfloat16 *qp = q + (size_t)qi * H * D;
         const int nchunks = H * D / 8;
+        uint4 u[kPer];
         float mx = 0.f;
-#pragma unroll 4
-        for (int c = threadIdx.x; c < nchunks; c += blockDim.x) {
-            uint4 u = __ldg(reinterpret_cast<const uint4 *>(qp) + c);
-            const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+            const int c = threadIdx.x + j * 1024;
+            u[j] = c < nchunks ? __ldg(reinterpret_cast<const uint4 *>(qp) + c) : make_uint4(0, 0, 0, 0);
+            const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&u[j]);
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 float2 f = __bfloat1622float2(h2[k]);
@@ -474,20 +478,19 @@ __global__ void __launch_bounds__(256) attend_schedule_kernel(
         __syncthreads();
         const float inv = ldexpf(1.0f, -sq_s);
         uint8_t *img = qimg + (size_t)qi * Cfg<D>::Q_BYTES;
-        // chunk (h, kc): 8 channels of head h
-        for (int c = threadIdx.x; c < kHeads * (D / 8); c += blockDim.x) {
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+            const int c = threadIdx.x + j * 1024;
+            if (c >= kHeads * (D / 8)) break;
             const int h = c / (D / 8);
             const int kc = c % (D / 8);
-            uint32_t o[4] = {0u, 0u, 0u, 0u};
-            if (h < H) {
-                uint4 u = __ldg(reinterpret_cast<const uint4 *>(qp + (size_t)h * D) + kc);
-                const __nv_bfloat162 *hh = reinterpret_cast<const __nv_bfloat162 *>(&u);
+            uint32_t o[4];
+            const __nv_bfloat162 *hh = reinterpret_cast<const __nv_bfloat162 *>(&u[j]);  // zero for h >= H
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    float2 f = __bfloat1622float2(hh[k]);
-                    __half2 x = __floats2half2_rn(f.x * inv, f.y * inv);
-                    o[k] = *reinterpret_cast<uint32_t *>(&x);
-                }
+            for (int k = 0; k < 4; ++k) {
+                float2 f = __bfloat1622float2(hh[k]);
+                __half2 x = __floats2half2_rn(f.x * inv, f.y * inv);
+                o[k] = *reinterpret_cast<uint32_t *>(&x);
             }
             const size_t off =
                 (size_t)(kc >> 3) * Cfg<D>::QREG + (h >> 3) * 1024 + (h & 7) * 128 + (((kc & 7) ^ (h & 7)) << 4);
@@ -546,7 +549,7 @@ __global__ void __launch_bounds__(256) attend_schedule_kernel(
 // ---------------------------------------------------------------- split merge
 // Row a8: a query whose tiles were spread over several CTAs has one partial
 // (unnormalized O, reference rho, row sum l) per CTA; combine them with the
-// log-sum-exp rule. One CTA per (query, 8-head slice); queries that a single
+// log-sum-exp rule. One CTA per (query, 8-head slice, 128 channels); queries that a single
 // CTA covered were written directly by attend_kernel and are skipped.
 constexpr int kMergeHeads = 8;
 
@@ -590,16 +593,32 @@ __global__ void __launch_bounds__(256) attend_merge_kernel(const long long *tpre
             l += wgt * part_l[(size_t)slots[p] * kHeads + h];
         }
         inv_l[threadIdx.x] = l > 0.f ? 1.f / l : 0.f;
-        if (lse) lse[(size_t)i * H + h] = l > 0.f ? (rmax + log2f(l)) * 0.69314718055994531f : -INFINITY;
+        if (lse && blockIdx.z == 0) lse[(size_t)i * H + h] = l > 0.f ? (rmax + log2f(l)) * 0.69314718055994531f : -INFINITY;
     }
     __syncthreads();
-    // float4 over the latent dimension; independent loads across partials
-    const int per_head = D / 4;
-    for (int v = threadIdx.x; v < nh * per_head; v += blockDim.x) {
-        const int hh = v / per_head, d4 = v % per_head;
+    // one float4 of one head per thread: this CTA's 8 heads x 128 channels (blockIdx.z);
+    // four partials in flight at a time
+    const int hh = threadIdx.x >> 5, d4 = blockIdx.z * 32 + (threadIdx.x & 31);
+    if (hh < nh && d4 < D / 4) {
+        const float4 *src = reinterpret_cast<const float4 *>(part_o + (size_t)(h0 + hh) * D) + d4;
+        const size_t slot_stride = (size_t)kHeads * D / 4;  // float4s per partial
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int p = 0; p < np; ++p) {
-            const float4 o = __ldcg(reinterpret_cast<const float4 *>(part_o + ((size_t)slots[p] * kHeads + h0 + hh) * D) + d4);
+        int p = 0;
+        for (; p + 4 <= np; p += 4) {
+            float4 o[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) o[k] = __ldcg(src + (size_t)slots[p + k] * slot_stride);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float wgt = wts[(p + k) * kMergeHeads + hh];
+                acc.x = fmaf(wgt, o[k].x, acc.x);
+                acc.y = fmaf(wgt, o[k].y, acc.y);
+                acc.z = fmaf(wgt, o[k].z, acc.z);
+                acc.w = fmaf(wgt, o[k].w, acc.w);
+            }
+        }
+        for (; p < np; ++p) {
+            const float4 o = __ldcg(src + (size_t)slots[p] * slot_stride);
             const float wgt = wts[p * kMergeHeads + hh];
             acc.x = fmaf(wgt, o.x, acc.x);
             acc.y = fmaf(wgt, o.y, acc.y);
@@ -957,7 +976,7 @@ template <int D>
 cudaError_t launch_schedule(const csa_cache &c, const AttArgs &a, const int32_t *q_offsets, const int32_t *q_pos,
                             const int32_t *win_len, int topk, int max_win, const void *q, int num_ctas, QInfo *qinfo,
                             long long *tprefix, int32_t *cta_q, int32_t *sq, uint8_t *qimg, cudaStream_t s) {
-    attend_schedule_kernel<D><<<a.Nq, 256, 0, s>>>(q_offsets, q_pos, c.n_blocks, win_len, c.batch, a.Nq, c.block,
+    attend_schedule_kernel<D><<<a.Nq, 1024, 0, s>>>(q_offsets, q_pos, c.n_blocks, win_len, c.batch, a.Nq, c.block,
                                                    c.capacity, topk, max_win, static_cast<const __nv_bfloat16 *>(q),
                                                    a.H, num_ctas, qinfo, tprefix, cta_q, sq, qimg, a.out, a.lse,
                                                    c.status);
@@ -1037,7 +1056,7 @@ cudaError_t launch_attend(const csa_cache &c, const void *q, int Nq, int H, cons
         return cudaErrorInvalidValue;
     }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(Nq, (H + kMergeHeads - 1) / kMergeHeads);
+    cfg.gridDim = dim3(Nq, (H + kMergeHeads - 1) / kMergeHeads, D / 128);
     cfg.blockDim = dim3(256);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = s;
