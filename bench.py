@@ -358,27 +358,67 @@ def main():
     step_ms = st_ms.sum(axis=1)
     ms = float(step_ms.mean())
 
-    # ---- end-to-end: pinned host inputs in, results out, every step
+    # ---- end-to-end: pinned host inputs in, results out, every step. Two buffer
+    # sets (each with its own graphs): step k+1's inputs are copied in and step
+    # k-1's results copied out (own streams) while step k computes.
+    import copy
+
     ins, outs = wl.step_inputs()
-    h_ins = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t.cpu()) for t in ins]
-    h_outs = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
-    h2d = sum(t.numel() * t.element_size() for t in h_ins)
-    d2h = sum(t.numel() * t.element_size() for t in h_outs)
-    e2e_n = max(3, min(args.steps, 50))
-    e0 = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_n)]
-    e1 = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_n)]
+    wl2 = copy.copy(wl)
+    for name in ("kv4", "idx4", "kv128", "q_csa", "q_hca", "q_idx", "w", "out_csa", "out_hca"):
+        setattr(wl2, name, torch.empty_like(getattr(wl, name)))
+    ins2, outs2 = wl2.step_inputs()
+    graphs2 = []
     with torch.cuda.stream(stream):
-        for k in range(e2e_n):
-            flush.zero_()
-            e0[k].record(stream)
-            for d_, h_ in zip(ins, h_ins):
-                d_.copy_(h_, non_blocking=True)
-            replay_step()
-            for h_, d_ in zip(h_outs, outs):
-                h_.copy_(d_, non_blocking=True)
-            e1[k].record(stream)
+        for fn in (wl2.stage_compress, wl2.stage_index, wl2.stage_attend):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                fn()
+            graphs2.append(g)
+        for g in graphs2:  # first replay outside the timed loop
+            g.replay()
+    torch.cuda.synchronize()
+    sets = [(ins, outs, graphs), (ins2, outs2, graphs2)]
+    h_ins = [[torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t.cpu()) for t in ins] for _ in range(2)]
+    h_outs = [[torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs] for _ in range(2)]
+    h2d = sum(t.numel() * t.element_size() for t in h_ins[0])
+    d2h = sum(t.numel() * t.element_size() for t in h_outs[0])
+    e2e_n = max(4, min(args.steps, 50))
+    up, down = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    ready = [torch.cuda.Event() for _ in range(2)]
+    computed = [torch.cuda.Event() for _ in range(2)]
+    drained = [torch.cuda.Event() for _ in range(2)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     stream.synchronize()
-    e2e_ms = float(np.mean([e0[k].elapsed_time(e1[k]) for k in range(e2e_n)]))
+    t_start.record(stream)
+    up.wait_event(t_start)
+    down.wait_event(t_start)
+    for k in range(e2e_n):
+        b = k % 2
+        d_ins, d_outs, gs = sets[b]
+        if k >= 2:
+            up.wait_event(computed[b])  # step k-2 has finished reading this set's inputs
+        with torch.cuda.stream(up):
+            for d_, h_ in zip(d_ins, h_ins[b]):
+                d_.copy_(h_, non_blocking=True)
+        ready[b].record(up)
+        stream.wait_event(ready[b])
+        if k >= 2:
+            stream.wait_event(drained[b])  # step k-2's results are out of this set's outputs
+        with torch.cuda.stream(stream):
+            for g in gs:
+                g.replay()
+        computed[b].record(stream)
+        down.wait_event(computed[b])
+        with torch.cuda.stream(down):
+            for h_, d_ in zip(h_outs[b], d_outs):
+                h_.copy_(d_, non_blocking=True)
+        drained[b].record(down)
+    stream.wait_stream(down)
+    t_end.record(stream)
+    stream.synchronize()
+    e2e_ms = t_start.elapsed_time(t_end) / e2e_n
+    del graphs2
 
     if world > 1:
         t = torch.tensor([ms, e2e_ms, float(st_ms[:, 1].mean())], dtype=torch.float64, device=device)
@@ -406,7 +446,8 @@ def main():
         "roofline": {"bound": "hbm", "kernel": "csa_index_topk (scan + select)", "achieved": achieved, "peak": peak,
                      "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind, "traffic": None},
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_n,
+                "overlap": "step k+1 inputs in and step k-1 results out while step k computes"},
         "gpu_launches": OUR_KERNELS_PER_STEP * args.steps,
         "clocks": clocks.summary(),
         "device_status": status,

@@ -454,99 +454,98 @@ __global__ void __launch_bounds__(kPassThreads) select_pass_kernel(SelArgs a) {
     if (above_bin < 0 && cand_bin < 0) return;  // everything selected: the final kernel writes it
     const float *s = a.scores + (size_t)i * a.cap;
     uint32_t *bm = a.bitmap + (size_t)i * a.words;
+    // each warp takes kPassChunks consecutive 128-score chunks per step, all loads first
+    constexpr int kPassChunks = 4;
     const int warps_total = gridDim.x * (kPassThreads / 32);
-    for (int base = (blockIdx.x * (kPassThreads / 32) + warp) * 128; base < n; base += warps_total * 128) {
-        // lane l holds scores [base + 4l, base + 4l + 4)
-        const int j0 = base + 4 * lane;
-        float v[4];
-        if (j0 + 3 < n && ((((size_t)i * a.cap + j0) & 3) == 0)) {
-            const float4 f = __ldcg(reinterpret_cast<const float4 *>(s + j0));
-            v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
-        } else {
+    for (int base0 = (blockIdx.x * (kPassThreads / 32) + warp) * 128 * kPassChunks; base0 < n;
+         base0 += warps_total * 128 * kPassChunks) {
+        float vv[kPassChunks][4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) v[u] = (j0 + u < n) ? __ldcg(s + j0 + u) : -INFINITY;
-        }
-        uint32_t nib = 0, cmask = 0;
-        uint32_t key[4];
+        for (int ch = 0; ch < kPassChunks; ++ch) {
+            const int j0 = base0 + 128 * ch + 4 * lane;
+            if (j0 + 3 < n && ((((size_t)i * a.cap + j0) & 3) == 0)) {
+                const float4 f = __ldcg(reinterpret_cast<const float4 *>(s + j0));
+                vv[ch][0] = f.x; vv[ch][1] = f.y; vv[ch][2] = f.z; vv[ch][3] = f.w;
+            } else {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            key[u] = ordered_key(v[u]);
-            const int d = (int)(key[u] >> 20);
-            const bool ok = j0 + u < n;
-            if (ok && d > above_bin) nib |= 1u << u;
-            if (ok && d == cand_bin) cmask |= 1u << u;
+                for (int u = 0; u < 4; ++u) vv[ch][u] = (j0 + u < n) ? __ldcg(s + j0 + u) : -INFINITY;
+            }
         }
-        // word w of this 128-score chunk = nibbles of lanes 8w .. 8w+7
-        uint32_t word = nib << (4 * (lane & 7));
-        word |= __shfl_xor_sync(0xffffffffu, word, 1);
-        word |= __shfl_xor_sync(0xffffffffu, word, 2);
-        word |= __shfl_xor_sync(0xffffffffu, word, 4);
-        if ((lane & 7) == 0 && base + 32 * (lane >> 3) < n) bm[(base >> 5) + (lane >> 3)] = word;
-        // candidates: warp-aggregated append
-        const uint32_t cnt = __popc(cmask);
-        uint32_t incl = cnt;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += y;
-        }
-        const uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
-        if (total) {
-            uint32_t at = 0;
-            if (lane == 31) at = atomicAdd(a.ncand + i, total);
-            at = __shfl_sync(0xffffffffu, at, 31);
-            uint32_t pos = at + incl - cnt;
+        for (int ch = 0; ch < kPassChunks; ++ch) {
+            const int base = base0 + 128 * ch;
+            if (base >= n) break;
+            // lane l holds scores [base + 4l, base + 4l + 4)
+            const int j0 = base + 4 * lane;
+            const float *v = vv[ch];
+            uint32_t nib = 0, cmask = 0;
+            uint32_t key[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                if (cmask & (1u << u)) {
-                    if (pos < (uint32_t)a.ccap) {
-                        a.cand_key[(size_t)i * a.ccap + pos] = key[u];
-                        a.cand_idx[(size_t)i * a.ccap + pos] = j0 + u;
+                key[u] = ordered_key(v[u]);
+                const int d = (int)(key[u] >> 20);
+                const bool ok = j0 + u < n;
+                if (ok && d > above_bin) nib |= 1u << u;
+                if (ok && d == cand_bin) cmask |= 1u << u;
+            }
+            // word w of this 128-score chunk = nibbles of lanes 8w .. 8w+7
+            uint32_t word = nib << (4 * (lane & 7));
+            word |= __shfl_xor_sync(0xffffffffu, word, 1);
+            word |= __shfl_xor_sync(0xffffffffu, word, 2);
+            word |= __shfl_xor_sync(0xffffffffu, word, 4);
+            if ((lane & 7) == 0 && base + 32 * (lane >> 3) < n) bm[(base >> 5) + (lane >> 3)] = word;
+            // candidates: warp-aggregated append
+            const uint32_t cnt = __popc(cmask);
+            uint32_t incl = cnt;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            const uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
+            if (total) {
+                uint32_t at = 0;
+                if (lane == 31) at = atomicAdd(a.ncand + i, total);
+                at = __shfl_sync(0xffffffffu, at, 31);
+                uint32_t pos = at + incl - cnt;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    if (cmask & (1u << u)) {
+                        if (pos < (uint32_t)a.ccap) {
+                            a.cand_key[(size_t)i * a.ccap + pos] = key[u];
+                            a.cand_idx[(size_t)i * a.ccap + pos] = j0 + u;
+                        }
+                        ++pos;
                     }
-                    ++pos;
                 }
             }
         }
     }
 }
 
-// Warp-scan compaction helpers over a shared bitmap of `words` words, split
-// into one contiguous run of words per warp.
-struct WordRun {
-    int begin, end;
-};
-__device__ __forceinline__ WordRun warp_run(int words) {
-    const int nwarps = blockDim.x >> 5, warp = threadIdx.x >> 5;
-    const int wpw = (words + nwarps - 1) / nwarps;
-    const int b = min(words, warp * wpw);
-    return {b, min(words, b + wpw)};
+// Compaction over a shared bitmap of `words` words (bits at or beyond n
+// ignored), split into one contiguous segment of wpt words per thread.
+constexpr int kMaxSegWords = 16;  // (2^19 blocks / 32 bits per word) / 1024 threads
+
+__device__ __forceinline__ uint32_t seg_word(const volatile uint32_t *bits, int w, int words, int n) {
+    uint32_t b = bits[w];
+    if (w == words - 1 && (n & 31)) b &= (1u << (n & 31)) - 1u;
+    return b;
 }
 
-// Number of set bits of every warp's run, as exclusive prefix sums in warp_base[]
-// (and the total in *total). Bits at or beyond n are ignored.
-__device__ void run_prefix(const volatile uint32_t *bits, int words, int n, uint32_t *warp_base, uint32_t *total) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-    const WordRun r = warp_run(words);
-    uint32_t cnt = 0;
-    for (int w = r.begin + lane; w < r.end; w += 32) {
-        uint32_t b = bits[w];
-        if (w == words - 1 && (n & 31)) b &= (1u << (n & 31)) - 1u;
-        cnt += __popc(b);
+// Set bits before this thread's segment (exclusive block prefix); *total gets the sum.
+__device__ uint32_t seg_prefix(const volatile uint32_t *bits, int words, int n, int wpt, uint32_t *scan_smem,
+                               uint32_t *total) {
+    const int w0 = threadIdx.x * wpt;
+    uint32_t c = 0;
+    for (int k = 0; k < wpt; ++k) {
+        const int w = w0 + k;
+        if (w < words) c += __popc(seg_word(bits, w, words, n));
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-    if (lane == 0) warp_base[warp] = cnt;
+    const uint32_t incl = block_inclusive_scan<uint32_t>(c, scan_smem);
+    if (threadIdx.x == blockDim.x - 1) *total = incl;
     __syncthreads();
-    if (threadIdx.x == 0) {
-        uint32_t run = 0;
-        for (int w = 0; w < nwarps; ++w) {
-            const uint32_t c = warp_base[w];
-            warp_base[w] = run;
-            run += c;
-        }
-        *total = run;
-    }
-    __syncthreads();
+    return incl - c;
 }
 
 // Exact selection among the members of the threshold bin, then ascending output.
@@ -568,7 +567,7 @@ __global__ void __launch_bounds__(kSelThreads) select_final_kernel(SelArgs a) {
     __shared__ uint32_t h[kBins];
     __shared__ uint32_t scan_smem[32];
     __shared__ BinPick pick;
-    __shared__ uint32_t warp_base[32], total_s, kmin_s, kmax_s;
+    __shared__ uint32_t total_s, kmin_s, kmax_s;
     __shared__ int prefix_digit[3];
     const int i = blockIdx.x;
     const int n = a.n_vis[i];
@@ -578,12 +577,26 @@ __global__ void __launch_bounds__(kSelThreads) select_final_kernel(SelArgs a) {
         for (int r = threadIdx.x; r < a.topk; r += blockDim.x) out[r] = r < n ? r : -1;
         return;
     }
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
     const int words = (n + 31) / 32;
     const uint32_t *gbm = a.bitmap + (size_t)i * a.words;
-    for (int w = threadIdx.x; w < words; w += blockDim.x) {
-        bm[w] = __ldcg(gbm + w);
-        tie[w] = 0u;
+    const int wpt = (words + kSelThreads - 1) / kSelThreads;  // <= kMaxSegWords
+    const int w0 = threadIdx.x * wpt;
+    {   // coalesced: word tid + k * blockDim, all loads in flight at once
+        uint32_t v[kMaxSegWords];
+#pragma unroll
+        for (int k = 0; k < kMaxSegWords; ++k) {
+            const int w = threadIdx.x + k * kSelThreads;
+            if (w < words) v[k] = __ldcg(gbm + w);
+        }
+#pragma unroll
+        for (int k = 0; k < kMaxSegWords; ++k) {
+            const int w = threadIdx.x + k * kSelThreads;
+            if (w < words) {
+                bm[w] = v[k];
+                tie[w] = 0u;
+            }
+        }
     }
     if (threadIdx.x == 0) {
         kmin_s = 0xFFFFFFFFu;
@@ -670,23 +683,14 @@ __global__ void __launch_bounds__(kSelThreads) select_final_kernel(SelArgs a) {
             });
             __syncthreads();
             const volatile uint32_t *vtie = tie;
-            run_prefix(vtie, words, n, warp_base, &total_s);
             // keep the first `need` tied members (in index order) and add them to bm
-            const WordRun r = warp_run(words);
-            uint32_t base = warp_base[warp];
-            for (int wc = r.begin; wc < r.end; wc += 32) {
-                const int w = wc + lane;
-                uint32_t b = w < r.end ? vtie[w] : 0u;
-                if (w == words - 1 && (n & 31)) b &= (1u << (n & 31)) - 1u;
+            uint32_t first = seg_prefix(vtie, words, n, wpt, scan_smem, &total_s);  // tied members before
+            for (int k = 0; k < wpt; ++k) {
+                const int w = w0 + k;
+                if (w >= words || first >= need) break;
+                uint32_t b = seg_word(vtie, w, words, n);
                 const uint32_t c = __popc(b);
-                uint32_t incl = c;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-                    if (lane >= o) incl += y;
-                }
-                const uint32_t first = base + incl - c;  // tied members before this word
-                if (first < need && b) {
+                if (b) {
                     uint32_t keep = b;
                     if (first + c > need) {  // keep only the lowest (need - first) bits
                         uint32_t left = need - first;
@@ -699,36 +703,25 @@ __global__ void __launch_bounds__(kSelThreads) select_final_kernel(SelArgs a) {
                     }
                     atomicOr(&bm[w], keep);
                 }
-                base += __shfl_sync(0xffffffffu, incl, 31);
+                first += c;
             }
         }
     }
     __syncthreads();
 
-    // ---- compaction: bitmap -> ascending block indices (warp scans) ----
+    // ---- compaction: bitmap -> ascending block indices (one word segment per thread) ----
     const volatile uint32_t *vbm = bm;
-    run_prefix(vbm, words, n, warp_base, &total_s);
-    const WordRun r = warp_run(words);
-    uint32_t base = warp_base[warp];
-    for (int wc = r.begin; wc < r.end; wc += 32) {
-        const int w = wc + lane;
-        uint32_t bits = w < r.end ? vbm[w] : 0u;
-        if (w == words - 1 && (n & 31)) bits &= (1u << (n & 31)) - 1u;
-        const uint32_t c = __popc(bits);
-        uint32_t incl = c;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += y;
-        }
-        uint32_t pos = base + incl - c;
+    uint32_t pos = seg_prefix(vbm, words, n, wpt, scan_smem, &total_s);
+    for (int k = 0; k < wpt; ++k) {
+        const int w = w0 + k;
+        if (w >= words) break;
+        uint32_t bits = seg_word(vbm, w, words, n);
         while (bits) {
             const int bit = __ffs(bits) - 1;
             bits &= bits - 1;
             if (pos < (uint32_t)a.topk) out[pos] = w * 32 + bit;
             ++pos;
         }
-        base += __shfl_sync(0xffffffffu, incl, 31);
     }
     // exactly K are selected; pad the rest
     for (int r2 = K + threadIdx.x; r2 < a.topk; r2 += blockDim.x) out[r2] = -1;
