@@ -110,7 +110,10 @@ class Workload:
         self.ws_att = torch.empty(nws, dtype=torch.uint8, device=device)
         self.scale = D ** -0.5
 
-    # the three stages of one step; every launch is one of libcsa's kernels or a memset
+    def stages(self):
+        return (self.stage_compress, self.stage_index, self.stage_attend_csa, self.stage_attend_hca)
+
+    # the stages of one step; every launch is one of libcsa's kernels, a memset or the n_blocks reset copy
     def stage_compress(self):
         import fp4_kv_cache_csa_b200 as csa
 
@@ -125,12 +128,16 @@ class Workload:
         csa.csa_index_topk(self.csa, self.q_idx, self.w, self.q_offsets, self.q_pos, TOPK, sel_idx=self.sel,
                            workspace=self.ws_idx)
 
-    def stage_attend(self):
+    def stage_attend_csa(self):
         import fp4_kv_cache_csa_b200 as csa
 
         csa.csa_decode_attend(self.csa, self.q_csa, self.q_offsets, self.sel, self.win, self.win_start, self.win_len,
                               max_win=W, softmax_scale=self.scale, out=self.out_csa, lse=self.lse,
                               workspace=self.ws_att)
+
+    def stage_attend_hca(self):
+        import fp4_kv_cache_csa_b200 as csa
+
         csa.hca_decode_attend(self.hca, self.q_hca, self.q_offsets, self.q_pos, self.win, self.win_start,
                               self.win_len, max_win=W, softmax_scale=self.scale, out=self.out_hca,
                               workspace=self.ws_att)
@@ -139,6 +146,12 @@ class Workload:
     def bytes_index(self) -> float:
         keys = float(np.sum(self.n_csa)) * D_I
         return keys + B * (H_I * D_I * 2 + H_I * 4 + TOPK * 4)
+
+    def bytes_csa_layer(self) -> float:
+        """The CSA layer's read/write set at decode: indexer keys, the selected entries, window, q, out."""
+        entry = D // 2 + D // 32
+        sel = float(np.sum(np.minimum(self.n_csa, TOPK))) * entry
+        return self.bytes_index() + sel + B * (W * D * 2 + H * D * 2 + H * D * 4)
 
     def bytes_step(self) -> float:
         entry = D // 2 + D // 32
@@ -312,10 +325,10 @@ def main():
     stream = torch.cuda.Stream(device)
     graphs = []
     with torch.cuda.stream(stream):
-        for fn in (wl.stage_compress, wl.stage_index, wl.stage_attend):  # eager pass before capture
+        for fn in wl.stages():  # eager pass before capture
             fn()
         stream.synchronize()
-        for fn in (wl.stage_compress, wl.stage_index, wl.stage_attend):
+        for fn in wl.stages():
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
                 fn()
@@ -329,7 +342,7 @@ def main():
                 evs[s].record(stream)
             g.replay()
         if evs is not None:
-            evs[3].record(stream)
+            evs[len(graphs)].record(stream)
 
     clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local)
     clocks.start()
@@ -344,7 +357,7 @@ def main():
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(graphs) + 1)] for _ in range(args.steps)]
     with torch.cuda.stream(stream):
         for k in range(args.steps):
             flush.zero_()  # outside the events: every step starts with a cold L2
@@ -354,7 +367,7 @@ def main():
     if world > 1:
         dist.barrier()
     clocks.stop()
-    st_ms = np.array([[ev[k][s].elapsed_time(ev[k][s + 1]) for s in range(3)] for k in range(args.steps)])
+    st_ms = np.array([[ev[k][s].elapsed_time(ev[k][s + 1]) for s in range(len(graphs))] for k in range(args.steps)])
     step_ms = st_ms.sum(axis=1)
     ms = float(step_ms.mean())
 
@@ -366,11 +379,11 @@ def main():
     ins, outs = wl.step_inputs()
     wl2 = copy.copy(wl)
     for name in ("kv4", "idx4", "kv128", "q_csa", "q_hca", "q_idx", "w", "out_csa", "out_hca"):
-        setattr(wl2, name, torch.empty_like(getattr(wl, name)))
+        setattr(wl2, name, getattr(wl, name).clone())
     ins2, outs2 = wl2.step_inputs()
     graphs2 = []
     with torch.cuda.stream(stream):
-        for fn in (wl2.stage_compress, wl2.stage_index, wl2.stage_attend):
+        for fn in wl2.stages():
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
                 fn()
@@ -421,11 +434,13 @@ def main():
     del graphs2
 
     if world > 1:
-        t = torch.tensor([ms, e2e_ms, float(st_ms[:, 1].mean())], dtype=torch.float64, device=device)
+        t = torch.tensor([ms, e2e_ms, float(st_ms[:, 1].mean()), float((st_ms[:, 1] + st_ms[:, 2]).mean())],
+                         dtype=torch.float64, device=device)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, e2e_ms, idx_ms = (float(x) for x in t.tolist())
+        ms, e2e_ms, idx_ms, csa_ms = (float(x) for x in t.tolist())
     else:
         idx_ms = float(st_ms[:, 1].mean())
+        csa_ms = float((st_ms[:, 1] + st_ms[:, 2]).mean())
     tokens = B * world
     value = tokens / (ms * 1e-3)
     peak, peak_kind = measured_peaks()
@@ -442,7 +457,12 @@ def main():
                    "l2": "flushed between steps (512 MB write) and inputs larger than L2"},
         "hbm_tbs": hbm_tbs,
         "stage_ms": {"compress": float(st_ms[:, 0].mean()), "index_topk": float(st_ms[:, 1].mean()),
-                     "attend_csa_hca": float(st_ms[:, 2].mean())},
+                     "attend_csa": float(st_ms[:, 2].mean()), "attend_hca": float(st_ms[:, 3].mean())},
+        # one CSA layer at decode (indexer + top-k + CSA attention) against its own HBM roofline
+        "csa_layer": {"ms": csa_ms, "tokens_per_s": tokens / (csa_ms * 1e-3),
+                      "algorithmic_bytes": wl.bytes_csa_layer(),
+                      "achieved_gbs": wl.bytes_csa_layer() / (csa_ms * 1e-3) / 1e9,
+                      "frac_of_hbm_peak": wl.bytes_csa_layer() / (csa_ms * 1e-3) / 1e9 / peak},
         "roofline": {"bound": "hbm", "kernel": "csa_index_topk (scan + select)", "achieved": achieved, "peak": peak,
                      "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind, "traffic": None},
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
