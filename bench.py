@@ -143,6 +143,9 @@ class Workload:
                               workspace=self.ws_att)
 
     # algorithmic HBM bytes: what the method must move at least once per step
+    def key_bytes(self) -> float:
+        return float(np.sum(self.n_csa)) * D_I
+
     def bytes_index(self) -> float:
         keys = float(np.sum(self.n_csa)) * D_I
         return keys + B * (H_I * D_I * 2 + H_I * 4 + TOPK * 4)
@@ -265,6 +268,25 @@ def measured_peaks():
             d = json.load(f)
         return float(d.get("hbm_gbs", 6650.0)), "measured"
     return 6650.0, "fallback"
+
+
+# DRAM traffic of one indexer call (schedule + scan + both select kernels) from one ncu
+# capture at 8 requests (profiles/dram_traffic_csa_hca_decode_b8.md): read + write bytes
+# and the key bytes of that call; scaled to this run by key bytes. Valid only for the
+# indexer source it was taken on (hash below); otherwise reported as null.
+INDEX_TRAFFIC_CAPTURE = {"bytes": 217.5e6 + 3.484e6, "key_bytes": 210.427904e6, "source_hash": "899bd5063ae638e6"}
+
+
+def index_traffic(key_bytes: float):
+    import hashlib
+
+    h = hashlib.sha256()
+    for f in ("indexer.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "fp4_kv_cache_csa_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    if h.hexdigest()[:16] != INDEX_TRAFFIC_CAPTURE["source_hash"]:
+        return None
+    return INDEX_TRAFFIC_CAPTURE["bytes"] * key_bytes / INDEX_TRAFFIC_CAPTURE["key_bytes"] / 1e9  # GB per call
 
 
 def run_reference(args):
@@ -464,7 +486,8 @@ def main():
                       "achieved_gbs": wl.bytes_csa_layer() / (csa_ms * 1e-3) / 1e9,
                       "frac_of_hbm_peak": wl.bytes_csa_layer() / (csa_ms * 1e-3) / 1e9 / peak},
         "roofline": {"bound": "hbm", "kernel": "csa_index_topk (scan + select)", "achieved": achieved, "peak": peak,
-                     "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind, "traffic": None},
+                     "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind,
+                     "traffic": index_traffic(wl.key_bytes()), "traffic_unit": "GB per call (ncu, scaled by keys)"},
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_n,
                 "overlap": "step k+1 inputs in and step k-1 results out while step k computes"},
