@@ -82,13 +82,13 @@ typedef enum { CSA_IDX_BF16 = 0, CSA_IDX_E4M3 = 1 } csa_idx_dtype;
  */
 typedef struct {
     int32_t batch;     /* requests, >= 1                                  */
-    int32_t dim;       /* D (K = V latent width); 128 or 512 for attention; multiple of 32 for compression */
+    int32_t dim;       /* D (K = V latent width): 64, 128, 256 or 512 for compression, 128 or 512 for attention */
     int32_t block;     /* m, tokens pooled per entry, 1..128              */
     int32_t capacity;  /* blocks per request, 1 .. 2^19                   */
     uint8_t *fp4;
     uint8_t *scale;
     void *idx_key;
-    int32_t idx_dim;   /* d_I, multiple of 16, <= 256 (0 when idx_key is NULL) */
+    int32_t idx_dim;   /* d_I: 64, 128 or 256 (0 when idx_key is NULL)     */
     int32_t idx_dtype; /* csa_idx_dtype                                   */
     int32_t *n_blocks;
     int32_t *status;
@@ -188,13 +188,15 @@ size_t csa_attend_workspace(const csa_cache *cache, int32_t n_queries, int32_t h
  *   out[i][h] = sum_x softmax(logit)_x * x,   lse[i][h] = ln sum_x exp(logit_x).
  * An empty entry set gives out = 0 and lse = -inf.
  * Arguments:
- *   q          bf16 [n_queries][heads][dim]   (heads == 64 or 16 with dim 512 or 128, see DESIGN)
+ *   q          bf16 [n_queries][heads][dim]   heads 1..64, dim 128 or 512
  *   sel_idx    int32 [n_queries][topk] device; entries must be < n_blocks[b]
  *              (larger ones set CSA_DEV_BAD_INDEX and are skipped)
  *   win_kv     bf16 [rows][dim]; win_start int64 [n_queries]; win_len int32 [n_queries]
  *              (all three may be NULL together: no window); max_win bounds win_len
  *   out        float32 [n_queries][heads][dim]; lse float32 [n_queries][heads] or NULL
- *   workspace  >= csa_attend_workspace(cache, n_queries, heads) bytes, 256-byte aligned
+ *   workspace  >= csa_attend_workspace(cache, n_queries, heads) bytes, 256-byte aligned;
+ *              it holds an fp16 copy of every query (n_queries * 64 * dim * 2 bytes)
+ *              and two partial outputs per SM
  */
 csa_status csa_decode_attend(const csa_cache *cache, const void *q, int32_t n_queries, int32_t heads,
                              const int32_t *q_offsets, const int32_t *sel_idx, int32_t topk,
