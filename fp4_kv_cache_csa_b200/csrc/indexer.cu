@@ -9,11 +9,13 @@
 //
 // Kernels, in launch order (one stream):
 //   schedule_kernel   per query: owning request, visible block count n_vis,
-//                     prefix over queries of ceil(n_vis/16) key groups.
+//                     prefix over queries of ceil(n_vis/16) key groups plus a
+//                     start cost (kSegCost units) per query.
 //   scan_kernel       streams every visible key exactly once (the dominant HBM
-//                     traffic at long context). The flat list of 16-key groups
-//                     is cut into equal contiguous ranges, one per CTA, so
-//                     ragged contexts stay balanced. Each warp turns 16 keys x
+//                     traffic at long context). One 16-warp CTA per SM. The
+//                     flat list of 16-key groups (plus a fixed start cost per
+//                     query) is cut into equal contiguous ranges, one per CTA,
+//                     so ragged contexts stay balanced. Each warp turns 16 keys x
 //                     d_I into tensor-core A fragments straight from its
 //                     coalesced 128-bit loads (no shared-memory staging) and
 //                     multiplies them by the query's H_I x d_I indexer matrix
@@ -52,7 +54,13 @@ namespace csa {
 namespace {
 
 constexpr int kBins = 4096;        // histogram bins per level (12 bits)
-constexpr int kScanThreads = 256;  // 8 warps
+constexpr int kScanThreads = 512;  // 16 warps, one CTA per SM
+constexpr int kScanWarps = kScanThreads / 32;
+// Work units charged for starting a query in a scan range (query fragments,
+// histogram clear and flush, completion count): about as long as scanning this
+// many 16-key groups. The flat split counts them, so ranges that cross a query
+// boundary get fewer keys.
+constexpr int kSegCost = 96;
 constexpr int kSelThreads = 1024;
 constexpr int kPassThreads = 256;
 constexpr int kCandCap = 32768;    // candidate slots per query (members of the threshold bin)
@@ -139,6 +147,7 @@ __global__ void schedule_kernel(const int32_t *q_offsets, const int32_t *q_pos, 
             req[i] = b;
             n_vis[i] = n;
             groups = (n + 15) / 16;
+            if (groups > 0) groups += kSegCost;  // units: the start cost, then one per 16-key group
             if (topk >= n) {  // every visible block is selected; no threshold needed
                 thresh[3 * i] = -1;
                 thresh[3 * i + 1] = n;
@@ -245,7 +254,7 @@ struct ScanCfg {
 };
 
 template <bool E4M3, int KS>
-__global__ void __launch_bounds__(kScanThreads, 2) scan_kernel(ScanArgs a) {
+__global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a) {
     using C = ScanCfg<E4M3, KS>;
     grid_dep_wait();    // the schedule kernel's ranges (programmatic launch)
     grid_dep_launch();
@@ -270,6 +279,14 @@ __global__ void __launch_bounds__(kScanThreads, 2) scan_kernel(ScanArgs a) {
         const long long seg_end = min(ge, a.gprefix[i + 1]);
         const int b = a.req[i];
         const int n = a.n_vis[i];
+        // units [gb, seg_end) of query i: the first kSegCost units are its start cost
+        const long long ngroups = (n + 15) / 16;
+        const long long lg0 = max(gb - a.gprefix[i] - kSegCost, 0LL);   // local group index
+        const long long nloc = seg_end - a.gprefix[i] - kSegCost - lg0;  // groups of this query here
+        if (nloc <= 0) {  // the range holds only start-cost units of this query
+            gb = seg_end;
+            continue;
+        }
 
         // ---- query fragments: B[k][n=head] with the dimension permutation ----
         uint32_t bq[KS][2];
@@ -335,15 +352,13 @@ __global__ void __launch_bounds__(kScanThreads, 2) scan_kernel(ScanArgs a) {
 
         const uint8_t *kbase = a.keys + (size_t)b * a.cap * C::KEY_BYTES;
         float *srow = a.scores + (size_t)i * a.cap;
-        const long long lg0 = gb - a.gprefix[i];   // local group index of gb
-        const long long nloc = seg_end - gb;        // groups of this query in this CTA
 
-        for (long long u0 = warp; u0 < nloc; u0 += 8LL * C::U) {
+        for (long long u0 = warp; u0 < nloc; u0 += (long long)kScanWarps * C::U) {
             uint4 raw[C::U][2][C::NV];
 #pragma unroll
             for (int uu = 0; uu < C::U; ++uu) {
-                const long long lg = lg0 + u0 + 8LL * uu;
-                const bool gv = (u0 + 8LL * uu) < nloc;
+                const long long lg = lg0 + u0 + (long long)kScanWarps * uu;
+                const bool gv = (u0 + (long long)kScanWarps * uu) < nloc;
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     const long long r = 16 * lg + g + 8 * half;
@@ -355,8 +370,8 @@ __global__ void __launch_bounds__(kScanThreads, 2) scan_kernel(ScanArgs a) {
             }
 #pragma unroll
             for (int uu = 0; uu < C::U; ++uu) {
-                const long long lg = lg0 + u0 + 8LL * uu;
-                const bool gv = (u0 + 8LL * uu) < nloc;
+                const long long lg = lg0 + u0 + (long long)kScanWarps * uu;
+                const bool gv = (u0 + (long long)kScanWarps * uu) < nloc;
                 float acc[4] = {0.f, 0.f, 0.f, 0.f};
                 const uint32_t *w0 = reinterpret_cast<const uint32_t *>(raw[uu][0]);
                 const uint32_t *w1 = reinterpret_cast<const uint32_t *>(raw[uu][1]);
@@ -406,7 +421,7 @@ __global__ void __launch_bounds__(kScanThreads, 2) scan_kernel(ScanArgs a) {
         __threadfence();
         __syncthreads();
         if (threadIdx.x == 0) {
-            const uint32_t total = (uint32_t)(a.gprefix[i + 1] - a.gprefix[i]);
+            const uint32_t total = (uint32_t)ngroups;
             const uint32_t mine = (uint32_t)nloc;
             last_flag = (atomicAdd(a.done + i, mine) + mine == total) && (a.topk < n);
         }
@@ -762,7 +777,7 @@ cudaError_t launch_index_topk(const csa_cache &c, const void *q_idx, const float
     sa.H_I = H_I;
     sa.cap = c.capacity;
     sa.topk = topk;
-    const int grid = num_sms * 2;
+    const int grid = num_sms;
     const bool e4 = c.idx_dtype == CSA_IDX_E4M3;
     switch (c.idx_dim / 16) {
         case 4: err = e4 ? launch_scan<true, 4>(sa, grid, s) : launch_scan<false, 4>(sa, grid, s); break;
