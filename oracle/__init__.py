@@ -27,6 +27,14 @@ _lib = None
 IDX_BF16 = 0
 IDX_E4M3 = 1
 
+# scale formats of the FP4 cache: E8M0 per 32 elements (OCP MXFP4), E4M3 per 16
+SCALE_E8M0_32 = 0
+SCALE_E4M3_16 = 1
+
+
+def group_size(scale_fmt: int) -> int:
+    return 32 if scale_fmt == SCALE_E8M0_32 else 16
+
 
 def build(force: bool = False) -> str:
     """Compile csa_oracle.c into _liboracle.so (gcc, OpenMP, no fast-math, no FMA contraction)."""
@@ -62,15 +70,17 @@ def _load():
         lib.orc_e4m3_encode.restype = ctypes.c_uint8
         lib.orc_mxfp4_quantize_group.argtypes = [P, P, P]
         lib.orc_mxfp4_quantize_group.restype = None
-        lib.orc_compress.argtypes = [I, I, I, I, I, I, P, P, P, P, P, P, P, P, P, P]
+        lib.orc_e4m3x16_quantize_group.argtypes = [P, P, P]
+        lib.orc_e4m3x16_quantize_group.restype = None
+        lib.orc_compress.argtypes = [I, I, I, I, I, I, I, P, P, P, P, P, P, P, P, P, P]
         lib.orc_compress.restype = I
         lib.orc_index_scores.argtypes = [I, I, I, I, I, I, I, P, P, P, P, P, P, P, P]
         lib.orc_index_scores.restype = None
         lib.orc_topk.argtypes = [I, I, I, P, P, P]
         lib.orc_topk.restype = None
-        lib.orc_csa_attend.argtypes = [I, I, I, I, I, I, P, P, P, P, P, P, P, P, D, P, P]
+        lib.orc_csa_attend.argtypes = [I, I, I, I, I, I, P, P, I, P, P, P, P, P, P, D, P, P]
         lib.orc_csa_attend.restype = None
-        lib.orc_hca_attend.argtypes = [I, I, I, I, I, I, P, P, P, P, P, P, P, P, P, D, P, P]
+        lib.orc_hca_attend.argtypes = [I, I, I, I, I, I, P, P, I, P, P, P, P, P, P, P, D, P, P]
         lib.orc_hca_attend.restype = None
         lib.orc_num_threads.argtypes = []
         lib.orc_num_threads.restype = I
@@ -129,6 +139,35 @@ def mxfp4_quantize_group(v):
     return codes, int(sb[0])
 
 
+def e4m3x16_quantize_group(v):
+    """16 float32 values -> (codes[16] one per byte, E4M3 scale byte)."""
+    v = _c(v, np.float32)
+    assert v.shape == (16,)
+    codes = np.zeros(16, np.uint8)
+    sb = np.zeros(1, np.uint8)
+    _load().orc_e4m3x16_quantize_group(_ptr(v), _ptr(codes), _ptr(sb))
+    return codes, int(sb[0])
+
+
+def e4m3x16_dequantize(fp4_rows, scale_rows):
+    """Dequantize [..., D/2] packed codes + [..., D/16] E4M3 scale bytes to float64 [..., D]:
+    value = E2M1(code) * E4M3(scale byte of its 16-element group)."""
+    fp4_rows = np.asarray(fp4_rows, np.uint8)
+    scale_rows = np.asarray(scale_rows, np.uint8)
+    codes = np.stack([fp4_rows & 0xF, fp4_rows >> 4], axis=-1).reshape(*fp4_rows.shape[:-1], fp4_rows.shape[-1] * 2)
+    table = np.array([e2m1_decode(c) for c in range(16)], np.float64)
+    stable = np.array([e4m3_decode(c) for c in range(256)], np.float64)
+    s = np.repeat(stable[scale_rows], 16, axis=-1)
+    assert s.shape[-1] == codes.shape[-1]
+    return table[codes] * s
+
+
+def fp4_dequantize(fp4_rows, scale_rows, scale_fmt=SCALE_E8M0_32):
+    if scale_fmt == SCALE_E8M0_32:
+        return mxfp4_dequantize(fp4_rows, scale_rows)
+    return e4m3x16_dequantize(fp4_rows, scale_rows)
+
+
 def mxfp4_dequantize(fp4_rows, scale_rows):
     """Dequantize [..., D/2] packed codes + [..., D/32] scale bytes to float64 [..., D].
 
@@ -151,8 +190,8 @@ def mxfp4_dequantize(fp4_rows, scale_rows):
 # ---- the method ------------------------------------------------------------
 
 def compress(kv_tok, idx_tok, w_g, tok_offsets, n_blocks, *, m, cap, idx_dtype=IDX_BF16,
-             fp4=None, scale=None, idx_key=None, return_pooled=False):
-    """Gated m-token pooling + MXFP4 quantization (rows a1, a2).
+             scale_fmt=SCALE_E8M0_32, fp4=None, scale=None, idx_key=None, return_pooled=False):
+    """Gated m-token pooling + FP4 quantization (rows a1, a2), scales per scale_fmt.
 
     kv_tok [T, D] uint16 (bf16 bits), idx_tok [T, dI] uint16 or None, w_g [D] float32,
     tok_offsets [B+1] int32, n_blocks [B] int32 (copied, returned updated).
@@ -168,12 +207,13 @@ def compress(kv_tok, idx_tok, w_g, tok_offsets, n_blocks, *, m, cap, idx_dtype=I
     w_g = _c(w_g, np.float32)
     kb = dI * (2 if idx_dtype == IDX_BF16 else 1)
     fp4 = np.zeros((B, cap, D // 2), np.uint8) if fp4 is None else fp4
-    scale = np.zeros((B, cap, D // 32), np.uint8) if scale is None else scale
+    scale = np.zeros((B, cap, D // group_size(scale_fmt)), np.uint8) if scale is None else scale
+    assert scale.shape == (B, cap, D // group_size(scale_fmt))
     if idx_tok is not None and idx_key is None:
         idx_key = np.zeros((B, cap, kb), np.uint8)
     pooled = np.zeros((B, cap, D), np.float32) if return_pooled else None
     pooled_idx = np.zeros((B, cap, dI), np.float32) if (return_pooled and idx_tok is not None) else None
-    st = _load().orc_compress(B, D, dI, m, idx_dtype, cap, _ptr(kv_tok), _ptr(idx_tok), _ptr(w_g),
+    st = _load().orc_compress(B, D, dI, m, idx_dtype, scale_fmt, cap, _ptr(kv_tok), _ptr(idx_tok), _ptr(w_g),
                               _ptr(tok_offsets), _ptr(n_blocks), _ptr(fp4), _ptr(scale),
                               _ptr(idx_key) if idx_tok is not None else None, _ptr(pooled), _ptr(pooled_idx))
     out = dict(fp4=fp4, scale=scale, idx_key=idx_key, n_blocks=n_blocks, status=st)
@@ -212,7 +252,8 @@ def index_topk(idx_key, n_blocks, q_offsets, q_pos, q_idx, w, *, m, k, idx_dtype
     return topk(scores, n_vis, k), scores, n_vis
 
 
-def csa_attend(fp4, scale, q_offsets, q, sel_idx, win_kv, win_start, win_len, softmax_scale):
+def csa_attend(fp4, scale, q_offsets, q, sel_idx, win_kv, win_start, win_len, softmax_scale, *,
+               scale_fmt=SCALE_E8M0_32):
     """Joint softmax attention over the selected compressed entries + window (rows a5, a6).
     Returns (out [Nq, H, D] float64, lse [Nq, H] float64)."""
     fp4 = _c(fp4, np.uint8)
@@ -226,13 +267,15 @@ def csa_attend(fp4, scale, q_offsets, q, sel_idx, win_kv, win_start, win_len, so
     out = np.empty((Nq, H, D), np.float64)
     lse = np.empty((Nq, H), np.float64)
     win_kv = _c(win_kv if win_kv is not None else np.zeros((1, D), np.uint16), np.uint16)
-    _load().orc_csa_attend(B, Nq, H, D, cap, k, _ptr(fp4), _ptr(scale), _ptr(_c(q_offsets, np.int32)),
+    assert scale.shape == (B, cap, D // group_size(scale_fmt))
+    _load().orc_csa_attend(B, Nq, H, D, cap, k, _ptr(fp4), _ptr(scale), scale_fmt, _ptr(_c(q_offsets, np.int32)),
                            _ptr(q), _ptr(sel_idx), _ptr(win_kv), _ptr(_c(win_start, np.int64)),
                            _ptr(_c(win_len, np.int32)), float(softmax_scale), _ptr(out), _ptr(lse))
     return out, lse
 
 
-def hca_attend(fp4, scale, n_blocks, q_offsets, q_pos, q, win_kv, win_start, win_len, softmax_scale, *, m):
+def hca_attend(fp4, scale, n_blocks, q_offsets, q_pos, q, win_kv, win_start, win_len, softmax_scale, *, m,
+               scale_fmt=SCALE_E8M0_32):
     """Dense attention over every visible compressed entry + window (row a7)."""
     fp4 = _c(fp4, np.uint8)
     scale = _c(scale, np.uint8)
@@ -243,7 +286,8 @@ def hca_attend(fp4, scale, n_blocks, q_offsets, q_pos, q, win_kv, win_start, win
     out = np.empty((Nq, H, D), np.float64)
     lse = np.empty((Nq, H), np.float64)
     win_kv = _c(win_kv if win_kv is not None else np.zeros((1, D), np.uint16), np.uint16)
-    _load().orc_hca_attend(B, Nq, H, D, m, cap, _ptr(fp4), _ptr(scale), _ptr(_c(n_blocks, np.int32)),
+    assert scale.shape == (B, cap, D // group_size(scale_fmt))
+    _load().orc_hca_attend(B, Nq, H, D, m, cap, _ptr(fp4), _ptr(scale), scale_fmt, _ptr(_c(n_blocks, np.int32)),
                            _ptr(_c(q_offsets, np.int32)), _ptr(_c(q_pos, np.int32)), _ptr(q),
                            _ptr(win_kv), _ptr(_c(win_start, np.int64)), _ptr(_c(win_len, np.int32)),
                            float(softmax_scale), _ptr(out), _ptr(lse))

@@ -119,11 +119,41 @@ void orc_mxfp4_quantize_group(const float *v, uint8_t *codes, uint8_t *scale_byt
     for (int i = 0; i < 32; ++i) codes[i] = orc_e2m1_encode(ldexp((double)v[i], -X));
 }
 
-static double mxfp4_element(const uint8_t *fp4_row, const uint8_t *scale_row, int d) {
+/* One 16-element group of the E4M3-scaled variant (DeepSeek-V4.1-Flash podcast
+ * transcript, cue 16: E2M1 elements, one E4M3 scale per sixteen channels, no
+ * second-level global scale). The scale is the E4M3 rounding (nearest, ties to
+ * even, saturating at 448) of amax / 6, so that the largest magnitude maps near
+ * E2M1's largest value 6; each element is the E2M1 rounding of v / scale. A
+ * scale that rounds to zero gives zero-magnitude codes that keep each
+ * element's sign. Both quotients are taken in double; the rounding decision is
+ * the one on the exact quotient (a rounded quotient of two floats never lands
+ * on an E2M1 or E4M3 midpoint unless the exact one does), so it also matches a
+ * correctly rounded float32 quotient or an exact threshold comparison. */
+void orc_e4m3x16_quantize_group(const float *v, uint8_t *codes, uint8_t *scale_byte) {
+    double amax = 0.0;
+    for (int i = 0; i < 16; ++i) amax = fmax(amax, fabs((double)v[i]));
+    uint8_t sb = orc_e4m3_encode(amax / 6.0);
+    double s = orc_e4m3_decode(sb);
+    *scale_byte = sb;
+    for (int i = 0; i < 16; ++i) {
+        if (s == 0.0)
+            codes[i] = signbit(v[i]) ? 0x8 : 0x0;
+        else
+            codes[i] = orc_e2m1_encode((double)v[i] / s);
+    }
+}
+
+/* Elements per scale byte: 32 for E8M0 scales (scale_fmt 0), 16 for E4M3 (1). */
+static int group_size(int scale_fmt) { return scale_fmt == 0 ? 32 : 16; }
+
+/* Element d of a stored row: E2M1(code) * 2^(byte - 127) (E8M0 scale) or
+ * E2M1(code) * E4M3(byte) (E4M3 scale). */
+static double fp4_element(const uint8_t *fp4_row, const uint8_t *scale_row, int d, int scale_fmt) {
     uint8_t byte = fp4_row[d / 2];
     uint8_t code = (d % 2 == 0) ? (byte & 0xF) : (byte >> 4);
-    int X = (int)scale_row[d / 32] - 127;
-    return ldexp(orc_e2m1_decode(code), X);
+    uint8_t sb = scale_row[d / group_size(scale_fmt)];
+    if (scale_fmt == 0) return ldexp(orc_e2m1_decode(code), (int)sb - 127);
+    return orc_e2m1_decode(code) * orc_e4m3_decode(sb);
 }
 
 static double idx_key_element(const uint8_t *key_row, int idx_dtype, int c) {
@@ -140,7 +170,7 @@ static size_t idx_key_bytes(int idx_dtype, int dI) { return (size_t)dI * (idx_dt
 /* ======================================================================
  * a1 + a2: gated block pooling, then quantization of the pooled block
  * ====================================================================== */
-int orc_compress(int B, int D, int dI, int m, int idx_dtype, int cap,
+int orc_compress(int B, int D, int dI, int m, int idx_dtype, int scale_fmt, int cap,
                  const uint16_t *kv_tok, const uint16_t *idx_tok, const float *w_g,
                  const int32_t *tok_offsets, int32_t *n_blocks,
                  uint8_t *fp4, uint8_t *scale, uint8_t *idx_key, float *pooled_out,
@@ -181,13 +211,17 @@ int orc_compress(int B, int D, int dI, int m, int idx_dtype, int cap,
             }
             size_t row = (size_t)b * cap + j;
             if (pooled_out) memcpy(pooled_out + row * D, e, sizeof(float) * D);
-            /* MXFP4: one E8M0 scale per 32 elements, two codes per byte */
-            for (int grp = 0; grp < D / 32; ++grp) {
+            /* FP4: one scale byte per group (E8M0 per 32 or E4M3 per 16), two codes per byte */
+            int gs = group_size(scale_fmt);
+            for (int grp = 0; grp < D / gs; ++grp) {
                 uint8_t codes[32], sb;
-                orc_mxfp4_quantize_group(e + 32 * grp, codes, &sb);
-                scale[row * (D / 32) + grp] = sb;
-                for (int i = 0; i < 16; ++i)
-                    fp4[row * (D / 2) + 16 * grp + i] = (uint8_t)(codes[2 * i] | (codes[2 * i + 1] << 4));
+                if (scale_fmt == 0)
+                    orc_mxfp4_quantize_group(e + gs * grp, codes, &sb);
+                else
+                    orc_e4m3x16_quantize_group(e + gs * grp, codes, &sb);
+                scale[row * (D / gs) + grp] = sb;
+                for (int i = 0; i < gs / 2; ++i)
+                    fp4[row * (D / 2) + (gs / 2) * grp + i] = (uint8_t)(codes[2 * i] | (codes[2 * i + 1] << 4));
             }
             /* pooled indexer key with the same gate, stored as bf16 or e4m3 */
             if (idx_key) {
@@ -326,15 +360,15 @@ static double attend_rows(const double *qh, const double *x, int n, int D, doubl
 
 /* Gather the entry rows of query i: compressed blocks (dequantized) then window rows. */
 static int gather_entries(int D, int cap, int b, const int32_t *blocks, int nblk,
-                          const uint8_t *fp4, const uint8_t *scale,
+                          const uint8_t *fp4, const uint8_t *scale, int scale_fmt,
                           const uint16_t *win_kv, int64_t wstart, int wlen, double *x) {
     int n = 0;
     for (int r = 0; r < nblk; ++r) {
         int j = blocks[r];
         if (j < 0) continue;
         const uint8_t *frow = fp4 + ((size_t)b * cap + j) * (D / 2);
-        const uint8_t *srow = scale + ((size_t)b * cap + j) * (D / 32);
-        for (int d = 0; d < D; ++d) x[(size_t)n * D + d] = mxfp4_element(frow, srow, d);
+        const uint8_t *srow = scale + ((size_t)b * cap + j) * (D / group_size(scale_fmt));
+        for (int d = 0; d < D; ++d) x[(size_t)n * D + d] = fp4_element(frow, srow, d, scale_fmt);
         ++n;
     }
     for (int t = 0; t < wlen; ++t) {
@@ -356,7 +390,7 @@ static void attend_query(int i, int H, int D, int n, const double *x, const uint
 }
 
 void orc_csa_attend(int B, int Nq, int H, int D, int cap, int k,
-                    const uint8_t *fp4, const uint8_t *scale,
+                    const uint8_t *fp4, const uint8_t *scale, int scale_fmt,
                     const int32_t *q_offsets, const uint16_t *q, const int32_t *sel_idx,
                     const uint16_t *win_kv, const int64_t *win_start, const int32_t *win_len,
                     double softmax_scale, double *out, double *lse) {
@@ -365,7 +399,7 @@ void orc_csa_attend(int B, int Nq, int H, int D, int cap, int k,
         int b = request_of(q_offsets, B, i);
         int wlen = win_len ? win_len[i] : 0;
         double *x = malloc(sizeof(double) * (size_t)(k + wlen + 1) * D);
-        int n = gather_entries(D, cap, b, sel_idx + (size_t)i * k, b < 0 ? 0 : k, fp4, scale,
+        int n = gather_entries(D, cap, b, sel_idx + (size_t)i * k, b < 0 ? 0 : k, fp4, scale, scale_fmt,
                                win_kv, win_start ? win_start[i] : 0, wlen, x);
         attend_query(i, H, D, n, x, q, softmax_scale, out, lse);
         free(x);
@@ -373,7 +407,7 @@ void orc_csa_attend(int B, int Nq, int H, int D, int cap, int k,
 }
 
 void orc_hca_attend(int B, int Nq, int H, int D, int m, int cap,
-                    const uint8_t *fp4, const uint8_t *scale, const int32_t *n_blocks,
+                    const uint8_t *fp4, const uint8_t *scale, int scale_fmt, const int32_t *n_blocks,
                     const int32_t *q_offsets, const int32_t *q_pos, const uint16_t *q,
                     const uint16_t *win_kv, const int64_t *win_start, const int32_t *win_len,
                     double softmax_scale, double *out, double *lse) {
@@ -386,7 +420,7 @@ void orc_hca_attend(int B, int Nq, int H, int D, int m, int cap,
         int32_t *all = malloc(sizeof(int32_t) * (n_vis > 0 ? n_vis : 1));
         for (int j = 0; j < n_vis; ++j) all[j] = j;
         double *x = malloc(sizeof(double) * (size_t)(n_vis + wlen + 1) * D);
-        int n = gather_entries(D, cap, b, all, n_vis, fp4, scale, win_kv, win_start ? win_start[i] : 0, wlen, x);
+        int n = gather_entries(D, cap, b, all, n_vis, fp4, scale, scale_fmt, win_kv, win_start ? win_start[i] : 0, wlen, x);
         attend_query(i, H, D, n, x, q, softmax_scale, out, lse);
         free(x);
         free(all);

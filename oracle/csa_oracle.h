@@ -19,6 +19,8 @@
  *   repository's design notes: softmax-gated pooling with a per-token scalar
  *   gate, score = sum_h w_h * ReLU(q_h . k), ties to the lower block index,
  *   one joint softmax over selected entries plus window, E8M0 scale per 32.
+ *   The page's own scale format (one E4M3 scale per 16 elements, cue 16) is
+ *   the second supported format.
  *
  * Precision: every floating-point step is carried out in double. Where a float
  * result decides an integer (an MXFP4 code or scale, an E4M3/BF16 byte pattern,
@@ -45,21 +47,26 @@ uint8_t  orc_e4m3_encode(double x);           /* RNE, saturate at +-448       */
 /* One 32-element MXFP4 group: codes[i] holds the E2M1 code of v[i] (one per
  * byte, not packed); *scale_byte is the E8M0 byte (exponent + 127). */
 void     orc_mxfp4_quantize_group(const float *v, uint8_t *codes, uint8_t *scale_byte);
+/* One 16-element group of the E4M3-scaled variant: *scale_byte is the E4M3
+ * byte of amax/6 (RNE, saturating); codes[i] the E2M1 code of v[i] / scale. */
+void     orc_e4m3x16_quantize_group(const float *v, uint8_t *codes, uint8_t *scale_byte);
 
 /* ---- a1+a2: gated block pooling + quantization ------------------------ */
 /* For each request b, tokens [tok_offsets[b], tok_offsets[b+1]) are pooled
  * m at a time into blocks appended at n_blocks[b] (n_blocks is updated).
  * kv_tok:  [T_total][D] bf16, idx_tok: [T_total][dI] bf16 (may be NULL when
  * idx_key is NULL), w_g: [D] float.
+ * scale_fmt selects the scale format: 0 = one E8M0 byte per 32 elements
+ * (OCP MXFP4), 1 = one E4M3 byte per 16 elements.
  * Output planes (per request stride = cap blocks):
  *   fp4   [B][cap][D/2]  two codes per byte, element 2i in the low nibble
- *   scale [B][cap][D/32] E8M0 bytes
+ *   scale [B][cap][D/32] E8M0 bytes, or [B][cap][D/16] E4M3 bytes
  *   idx_key [B][cap][dI] bf16 (idx_dtype 0) or e4m3 (idx_dtype 1)
  * Optional pooled_out [B][cap][D] float and pooled_idx_out [B][cap][dI] float
  * receive the float32 pooled values before quantization (NULL to skip).
  * Returns 0, or -1 when a request's token count is not a multiple of m or
  * would overflow the capacity (nothing is written for that request). */
-int orc_compress(int B, int D, int dI, int m, int idx_dtype, int cap,
+int orc_compress(int B, int D, int dI, int m, int idx_dtype, int scale_fmt, int cap,
                  const uint16_t *kv_tok, const uint16_t *idx_tok, const float *w_g,
                  const int32_t *tok_offsets, int32_t *n_blocks,
                  uint8_t *fp4, uint8_t *scale, uint8_t *idx_key, float *pooled_out,
@@ -90,10 +97,11 @@ void orc_topk(int Nq, int cap, int k, const float *scores, const int32_t *n_vis,
  * win_kv[win_start[i] + t], t < win_len[i]. Logits are
  * softmax_scale * <q[i][h], x>; out[i][h] = sum softmax * x and
  * lse[i][h] = natural log of sum exp(logit). An empty entry set gives out = 0
- * and lse = -INFINITY. q: [Nq][H][D] bf16; out: [Nq][H][D] double;
+ * and lse = -INFINITY. The cache planes are read in the scale format
+ * scale_fmt (as for orc_compress). q: [Nq][H][D] bf16; out: [Nq][H][D] double;
  * lse: [Nq][H] double (may be NULL). */
 void orc_csa_attend(int B, int Nq, int H, int D, int cap, int k,
-                    const uint8_t *fp4, const uint8_t *scale,
+                    const uint8_t *fp4, const uint8_t *scale, int scale_fmt,
                     const int32_t *q_offsets, const uint16_t *q, const int32_t *sel_idx,
                     const uint16_t *win_kv, const int64_t *win_start, const int32_t *win_len,
                     double softmax_scale, double *out, double *lse);
@@ -102,7 +110,7 @@ void orc_csa_attend(int B, int Nq, int H, int D, int cap, int k,
 /* As orc_csa_attend, but the compressed entries are all visible blocks
  * j < min(floor((q_pos[i]+1)/m), n_blocks[req]) in order. */
 void orc_hca_attend(int B, int Nq, int H, int D, int m, int cap,
-                    const uint8_t *fp4, const uint8_t *scale, const int32_t *n_blocks,
+                    const uint8_t *fp4, const uint8_t *scale, int scale_fmt, const int32_t *n_blocks,
                     const int32_t *q_offsets, const int32_t *q_pos, const uint16_t *q,
                     const uint16_t *win_kv, const int64_t *win_start, const int32_t *win_len,
                     double softmax_scale, double *out, double *lse);

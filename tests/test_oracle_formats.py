@@ -155,3 +155,109 @@ def test_bf16_encode_matches_torch():
     assert np.array_equal(got, ref)
     for bits in g.integers(0, 0x7F80, 2000):
         assert oracle.bf16_decode(int(bits)) == float(np.array([int(bits) << 16], np.uint32).view(np.float32)[0])
+
+
+# ---------------------------------------------------------------- E4M3 scale per 16 elements
+
+def _read_groups(name):
+    rows = []
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            v, sb, codes = line.split("|")
+            rows.append((np.array([float(x) for x in v.split()], np.float32), int(sb, 0),
+                         np.array([int(c, 0) for c in codes.split()], np.uint8)))
+    return rows
+
+
+def test_e4m3x16_scale_golden():
+    for amax, byte in _read_golden("e4m3x16_scale.txt"):
+        for pos in (0, 9, 15):
+            v = np.zeros(16, np.float32)
+            v[pos] = np.float32(amax)
+            _, sb = oracle.e4m3x16_quantize_group(v)
+            assert sb == byte, amax
+            v[pos] = -np.float32(amax)  # the sign of the largest element does not matter
+            assert oracle.e4m3x16_quantize_group(v)[1] == byte, amax
+
+
+def test_e4m3x16_group_golden():
+    for v, sb, codes in _read_groups("e4m3x16_groups.txt"):
+        got, gsb = oracle.e4m3x16_quantize_group(v)
+        assert gsb == sb, v
+        assert np.array_equal(got, codes), v
+
+
+def test_e4m3x16_roundtrip_every_scale_and_code():
+    # a group of exactly representable values E2M1(c) * s whose largest magnitude is
+    # 6 s comes back with scale s and the same codes, for every positive finite s
+    for sb in range(1, 0x7F):
+        s = e4m3_by_bits(sb)
+        codes = np.arange(16, dtype=np.uint8)
+        v = np.array([e2m1_by_bits(int(c)) * s for c in codes], np.float64)
+        assert np.all(v.astype(np.float32).astype(np.float64) == v)
+        got, gsb = oracle.e4m3x16_quantize_group(v.astype(np.float32))
+        assert gsb == sb
+        assert np.array_equal(got, codes), sb  # includes -0 -> 0x8 and +-6 -> 0x7 / 0xF
+
+
+def test_e4m3x16_brute_force_nearest():
+    # scale: the nearest E4M3 value to amax / 6 among all 127 finite magnitudes
+    # (ties to the even code, saturation at 448); codes: the nearest E2M1 value
+    # to v / s, again by brute force over the 8 magnitudes
+    mags = np.array([e4m3_by_bits(c) for c in range(0x7F)])
+    e2 = np.array([e2m1_by_bits(c) for c in range(8)])
+    g = np.random.default_rng(5)
+    for trial in range(400):
+        v = (g.standard_normal(16) * 10.0 ** g.uniform(-4, 3.6)).astype(np.float32)
+        codes, sb = oracle.e4m3x16_quantize_group(v)
+        r = float(np.max(np.abs(v.astype(np.float64)))) / 6.0
+        d = np.abs(mags - r)
+        best = np.flatnonzero(d == d.min())
+        want = best[0] if len(best) == 1 else [c for c in best if c % 2 == 0][0]
+        if r > 448.0:
+            want = 0x7E
+        assert sb == want
+        s = mags[sb]
+        for x, c in zip(v.astype(np.float64), codes):
+            if s == 0.0:
+                assert (c & 7) == 0
+                continue
+            qd = np.abs(e2 - abs(x) / s)
+            cand = np.flatnonzero(qd == qd.min())
+            mag = cand[0] if len(cand) == 1 else [k for k in cand if k % 2 == 0][0]
+            assert (c & 7) == mag
+            assert (c >> 3) == (1 if np.signbit(x) else 0)
+
+
+def test_e4m3x16_error_bound():
+    # every element within half an E2M1 step of v at scale s, or saturated at 6 s;
+    # the scale within half an E4M3 step of amax / 6 (relative 2^-4 for normal s)
+    g = np.random.default_rng(6)
+    for trial in range(300):
+        v = (g.standard_normal(16) * 10.0 ** g.uniform(-1, 2.5)).astype(np.float32)
+        codes, sb = oracle.e4m3x16_quantize_group(v)
+        s = e4m3_by_bits(sb)
+        amax = float(np.max(np.abs(v.astype(np.float64))))
+        assert abs(s - amax / 6.0) <= (amax / 6.0) * 2.0 ** -4 * (1 + 1e-12)
+        deq = np.array([e2m1_by_bits(int(c)) * s for c in codes])
+        for x, y in zip(v.astype(np.float64), deq):
+            q = abs(x) / s
+            if q > 6.0:
+                assert abs(y) == 6.0 * s and np.sign(y) == np.sign(x)
+                continue
+            half_step = 0.25 if q <= 2.0 else 0.5 if q <= 4.0 else 1.0
+            assert abs(y - x) <= half_step * s * (1 + 1e-12)
+
+
+def test_e4m3x16_dequantize_matches_definition():
+    g = np.random.default_rng(7)
+    fp4 = g.integers(0, 256, size=(3, 32), dtype=np.uint8)
+    sc = g.integers(0, 0x7F, size=(3, 4), dtype=np.uint8)
+    deq = oracle.fp4_dequantize(fp4, sc, oracle.SCALE_E4M3_16)
+    for r in range(3):
+        for d in range(64):
+            code = (fp4[r, d // 2] >> (4 * (d % 2))) & 0xF
+            assert deq[r, d] == e2m1_by_bits(int(code)) * e4m3_by_bits(int(sc[r, d // 16]))

@@ -319,3 +319,67 @@ def test_csa_brute_force_subset_then_textbook():
     x = np.concatenate([rows[list(best)].astype(np.float64), bf16_val(bf16(win_rows))])
     ref, _ = _textbook(bf16_val(q[0]), x, 0.2)
     np.testing.assert_allclose(out[0], ref, rtol=1e-10, atol=1e-12)
+
+
+# ---------------------------------------------------------------- E4M3 scale per 16 elements
+
+def lossless_tokens_e4m3x16(n, D, seed):
+    """Tokens whose every 16-group is exactly E2M1 x s with amax = 6 s for an E4M3
+    scale s, so the E4M3-per-16 format stores them without loss."""
+    g = np.random.default_rng(seed)
+    mags = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6])
+    vals = g.choice(mags, size=(n, D // 16, 16)) * g.choice([-1.0, 1.0], size=(n, D // 16, 16))
+    vals[:, :, 3] = np.where(vals[:, :, 3] < 0, -6.0, 6.0)
+    s_codes = g.integers(0x20, 0x48, size=(n, D // 16))  # E4M3 scales 2^-3 .. 2^2 * 1.875
+    s = np.array([[oracle.e4m3_decode(int(c)) for c in row] for row in s_codes])
+    return (vals * s[:, :, None]).reshape(n, D).astype(np.float32)
+
+
+def test_pool_m1_quantizes_the_token_e4m3x16():
+    g = np.random.default_rng(40)
+    kv = g.standard_normal((32, 128)).astype(np.float32)
+    r = oracle.compress(bf16(kv), None, np.zeros(128, np.float32), np.array([0, 32], np.int32),
+                        np.zeros(1, np.int32), m=1, cap=32, scale_fmt=oracle.SCALE_E4M3_16, return_pooled=True)
+    tok = bf16_val(bf16(kv))
+    assert r["scale"].shape == (1, 32, 8)
+    for j in range(32):
+        for grp in range(8):
+            codes, sb = oracle.e4m3x16_quantize_group(tok[j, 16 * grp:16 * grp + 16].astype(np.float32))
+            assert r["scale"][0, j, grp] == sb
+            assert np.array_equal(r["fp4"][0, j, 8 * grp:8 * grp + 8], codes[0::2] | (codes[1::2] << 4))
+
+
+def test_e4m3x16_lossless_dense_is_textbook_attention():
+    n, D, H = 24, 128, 4
+    rows = lossless_tokens_e4m3x16(n, D, 41)
+    r = oracle.compress(bf16(rows), None, np.zeros(D, np.float32), np.array([0, n], np.int32),
+                        np.zeros(1, np.int32), m=1, cap=n, scale_fmt=oracle.SCALE_E4M3_16)
+    assert np.array_equal(oracle.fp4_dequantize(r["fp4"][0], r["scale"][0], oracle.SCALE_E4M3_16),
+                          rows.astype(np.float64))
+    g = np.random.default_rng(42)
+    q = bf16(g.standard_normal((1, H, D)))
+    sel = np.arange(n, dtype=np.int32)[None]
+    out, lse = oracle.csa_attend(r["fp4"], r["scale"], np.array([0, 1], np.int32), q, sel, None, None, None,
+                                 1 / math.sqrt(D), scale_fmt=oracle.SCALE_E4M3_16)
+    ref, ref_lse = _textbook(bf16_val(q[0]), rows.astype(np.float64), 1 / math.sqrt(D))
+    np.testing.assert_allclose(out[0], ref, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(lse[0], ref_lse, rtol=1e-12)
+    hout, hlse = oracle.hca_attend(r["fp4"], r["scale"], r["n_blocks"], np.array([0, 1], np.int32),
+                                   np.array([n - 1], np.int32), q, None, None, None, 1 / math.sqrt(D), m=1,
+                                   scale_fmt=oracle.SCALE_E4M3_16)
+    np.testing.assert_allclose(hout, out, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(hlse, lse, rtol=1e-12)
+
+
+def test_e4m3x16_is_finer_than_e8m0x32_on_gaussian_blocks():
+    # the per-16 E4M3 scale tracks each group's magnitude more closely than a
+    # power-of-two per-32 scale: its mean squared error is lower on N(0,1) rows
+    g = np.random.default_rng(43)
+    kv = g.standard_normal((256, 128)).astype(np.float32)
+    tok = bf16_val(bf16(kv))
+    err = {}
+    for fmt in (oracle.SCALE_E8M0_32, oracle.SCALE_E4M3_16):
+        r = oracle.compress(bf16(kv), None, np.zeros(128, np.float32), np.array([0, 256], np.int32),
+                            np.zeros(1, np.int32), m=1, cap=256, scale_fmt=fmt)
+        err[fmt] = np.mean((oracle.fp4_dequantize(r["fp4"][0], r["scale"][0], fmt) - tok) ** 2)
+    assert err[oracle.SCALE_E4M3_16] < err[oracle.SCALE_E8M0_32]
