@@ -23,6 +23,9 @@ LIB_PATH = os.path.join(_HERE, "libcsa.so")
 CSA_IDX_BF16 = 0
 CSA_IDX_E4M3 = 1
 
+CSA_SCALE_E8M0_32 = 0  # one E8M0 scale byte per 32 elements (OCP MXFP4)
+CSA_SCALE_E4M3_16 = 1  # one E4M3 scale byte per 16 elements
+
 CSA_DEV_TOKEN_COUNT = 0x1
 CSA_DEV_CAPACITY = 0x2
 CSA_DEV_BAD_INDEX = 0x4
@@ -45,7 +48,7 @@ class _CCache(ctypes.Structure):
         ("batch", ctypes.c_int32), ("dim", ctypes.c_int32), ("block", ctypes.c_int32), ("capacity", ctypes.c_int32),
         ("fp4", ctypes.c_void_p), ("scale", ctypes.c_void_p), ("idx_key", ctypes.c_void_p),
         ("idx_dim", ctypes.c_int32), ("idx_dtype", ctypes.c_int32),
-        ("n_blocks", ctypes.c_void_p), ("status", ctypes.c_void_p),
+        ("n_blocks", ctypes.c_void_p), ("status", ctypes.c_void_p), ("scale_fmt", ctypes.c_int32),
     ]
 
 
@@ -108,8 +111,8 @@ def _stream(stream):
 class Cache:
     """One compressed cache (one layer): device tensors owned by the caller (see include/csa.h).
 
-    fp4 [B, cap, D/2] uint8, scale [B, cap, D/32] uint8, idx_key [B, cap, dI] bf16 / uint8 (e4m3) or None,
-    n_blocks [B] int32, status [1] int32 or None.
+    fp4 [B, cap, D/2] uint8, scale [B, cap, D/32] uint8 (E8M0) or [B, cap, D/16] uint8 (E4M3),
+    idx_key [B, cap, dI] bf16 / uint8 (e4m3) or None, n_blocks [B] int32, status [1] int32 or None.
     """
     fp4: object
     scale: object
@@ -118,6 +121,7 @@ class Cache:
     idx_key: object = None
     idx_dtype: int = CSA_IDX_BF16
     status: object = None
+    scale_fmt: int = CSA_SCALE_E8M0_32
 
     @property
     def batch(self) -> int:
@@ -137,11 +141,12 @@ class Cache:
 
     def c_struct(self) -> _CCache:
         return _CCache(self.batch, self.dim, self.block, self.capacity, _ptr(self.fp4), _ptr(self.scale),
-                       _ptr(self.idx_key), self.idx_dim, self.idx_dtype, _ptr(self.n_blocks), _ptr(self.status))
+                       _ptr(self.idx_key), self.idx_dim, self.idx_dtype, _ptr(self.n_blocks), _ptr(self.status),
+                       self.scale_fmt)
 
     @staticmethod
     def allocate(batch: int, capacity: int, dim: int, block: int, idx_dim: int = 0, idx_dtype: int = CSA_IDX_BF16,
-                 device="cuda"):
+                 device="cuda", scale_fmt: int = CSA_SCALE_E8M0_32):
         """Zero-filled cache tensors on `device` (torch allocation; the library allocates nothing)."""
         import torch
 
@@ -150,9 +155,11 @@ class Cache:
             dt = torch.bfloat16 if idx_dtype == CSA_IDX_BF16 else torch.uint8
             idx = torch.zeros(batch, capacity, idx_dim, dtype=dt, device=device)
         return Cache(fp4=torch.zeros(batch, capacity, dim // 2, dtype=torch.uint8, device=device),
-                     scale=torch.zeros(batch, capacity, dim // 32, dtype=torch.uint8, device=device),
+                     scale=torch.zeros(batch, capacity, dim // (32 if scale_fmt == CSA_SCALE_E8M0_32 else 16),
+                                       dtype=torch.uint8, device=device),
                      n_blocks=torch.zeros(batch, dtype=torch.int32, device=device), block=block,
-                     idx_key=idx, idx_dtype=idx_dtype, status=torch.zeros(1, dtype=torch.int32, device=device))
+                     idx_key=idx, idx_dtype=idx_dtype, status=torch.zeros(1, dtype=torch.int32, device=device),
+                     scale_fmt=scale_fmt)
 
 
 def csa_version() -> int:
@@ -160,7 +167,7 @@ def csa_version() -> int:
 
 
 def csa_compress_quantize(cache: Cache, kv_tok, idx_tok, gate_w, tok_offsets, stream=None):
-    """Rows a1+a2: pool every m new tokens of each request into one block and store it (MXFP4 + indexer key)."""
+    """Rows a1+a2: pool every m new tokens of each request into one block and store it (FP4 + indexer key)."""
     lib = load_library()
     c = cache.c_struct()
     _check(lib.csa_compress_quantize(ctypes.byref(c), _ptr(kv_tok), _ptr(idx_tok), _ptr(gate_w), _ptr(tok_offsets),

@@ -20,7 +20,9 @@
 //   * Operands are fp16 in shared memory. Entry j is stored as
 //     E'_j = e_j * 2^-R_j with R_j the largest E8M0 exponent of the row (or the
 //     exponent of max|x| for a window row): every E2M1 x 2^X value is exact in
-//     fp16 within 2^24 of the row's largest group. The query is stored as
+//     fp16 within 2^24 of the row's largest group. With one E4M3 scale per 16
+//     elements (the cache's other format) every E2M1 x E4M3 value is exact
+//     in fp16 as it stands, so E'_j = e_j and R_j = 0. The query is stored as
 //     q * 2^-sQ (exact for bf16 values within 2^31 of max|q|).
 //   * S^T = E' Q'^T: M = 128 entries (TMEM lanes), N = 64 heads (columns).
 //   * Softmax in the log2 domain, thread (j, half) holding 32 head logits of
@@ -42,6 +44,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp4.h>
+#include <cuda_fp8.h>
 
 #include "common.cuh"
 
@@ -226,8 +229,13 @@ struct AttArgs {
     float scale_log2;                // softmax_scale * log2(e)
 };
 
-// Prefetch of this thread's half of one compressed entry: its codes and all
-// of the row's E8M0 bytes (R_j is the maximum over the whole row).
+// Scale formats of the cache (template argument SF of the kernel).
+constexpr int kScaleE8M0x32 = 0;  // one E8M0 byte per 32 elements
+constexpr int kScaleE4M3x16 = 1;  // one E4M3 byte per 16 elements
+
+// Prefetch of this thread's half of one compressed entry: its codes and the
+// scale bytes it needs -- for E8M0 scales all D/32 bytes of the row (R_j is
+// the maximum over the whole row), for E4M3 scales the D/32 bytes of its half.
 template <int D>
 struct RowRegs {
     uint4 code[Cfg<D>::HALF_V];
@@ -290,7 +298,7 @@ __device__ __forceinline__ int row_block_raw(const AttArgs &a, const TileRef &tr
 }
 
 // Issue the loads of this thread's row of a compressed tile.
-template <int D>
+template <int D, int SF>
 __device__ __forceinline__ void prefetch_row(const AttArgs &a, const TileRef &tr, int blk, RowRegs<D> &rr) {
     rr.valid = 0;
     if (blk >= 0 && (blk >= tr.nblk || blk >= a.cap)) {
@@ -302,10 +310,13 @@ __device__ __forceinline__ void prefetch_row(const AttArgs &a, const TileRef &tr
         const uint4 *src = reinterpret_cast<const uint4 *>(a.fp4 + row * (D / 2)) + (threadIdx.x >> 7) * Cfg<D>::HALF_V;
 #pragma unroll
         for (int v = 0; v < Cfg<D>::HALF_V; ++v) rr.code[v] = __ldg(src + v);
+        // D/32 scale bytes either way: the whole row (E8M0) or this half (E4M3, D/16 per row)
+        const uint8_t *sp = SF == kScaleE4M3x16 ? a.scale + row * (D / 16) + (threadIdx.x >> 7) * (D / 32)
+                                                : a.scale + row * (D / 32);
         if constexpr (D / 32 >= 16) {
-            rr.sc = __ldg(reinterpret_cast<const uint4 *>(a.scale + row * (D / 32)));
+            rr.sc = __ldg(reinterpret_cast<const uint4 *>(sp));
         } else {
-            rr.sc = make_uint4(__ldg(reinterpret_cast<const uint32_t *>(a.scale + row * (D / 32))), 0, 0, 0);
+            rr.sc = make_uint4(__ldg(reinterpret_cast<const uint32_t *>(sp)), 0, 0, 0);
         }
         rr.valid = 1;
     }
@@ -324,42 +335,77 @@ __device__ __forceinline__ uint32_t e_chunk_off(int j, int kc) {
     return (uint32_t)((kc >> 3) * Cfg<D>::KREG + (j >> 3) * 1024 + (j & 7) * 128 + (((kc & 7) ^ (j & 7)) << 4));
 }
 
-// Dequantize this thread's half of its prefetched row into E' (fp16, scaled
-// by 2^-R_j). Returns R_j (the row's largest E8M0 exponent); invalid rows are zero.
-template <int D>
+// Dequantize this thread's half of its prefetched row into E' (fp16).
+// E8M0 scales: E'_j = e_j * 2^-R_j, returns R_j (the row's largest E8M0
+// exponent). E4M3 scales: every E2M1 x E4M3 product is exact in fp16 (at most
+// 6 significant bits, magnitudes 2^-10 .. 2688), so E' = e and R_j = 0.
+// Invalid rows are zero.
+template <int D, int SF>
 __device__ __forceinline__ int dequant_row(const RowRegs<D> &rr, uint8_t *E) {
     const int j = threadIdx.x & (kTile - 1);
-    const int g0 = (threadIdx.x >> 7) * (Cfg<D>::GPR / 2);  // first group of this half
+    const int g0 = (threadIdx.x >> 7) * (Cfg<D>::GPR / 2);  // first 32-element group of this half
     if (!rr.valid) {
 #pragma unroll 4
         for (int kc = 4 * g0; kc < 4 * g0 + D / 16; ++kc)
             *reinterpret_cast<uint4 *>(E + e_chunk_off<D>(j, kc)) = make_uint4(0, 0, 0, 0);
         return 0;
     }
-    int rmax = 0;
+    if constexpr (SF == kScaleE4M3x16) {
 #pragma unroll
-    for (int g = 0; g < Cfg<D>::GPR; ++g) rmax = max(rmax, scale_byte<D>(rr, g));
+        for (int gl = 0; gl < Cfg<D>::GPR / 2; ++gl) {
+            const int g = g0 + gl;
+            const uint32_t *w = reinterpret_cast<const uint32_t *>(&rr.code[gl]);
+            // code bytes 0..7 of this uint4 are 16-element group 2 gl of the half, 8..15 group 2 gl + 1
+            __half2 s2[2];
 #pragma unroll
-    for (int gl = 0; gl < Cfg<D>::GPR / 2; ++gl) {
-        const int g = g0 + gl;
-        const int k = scale_byte<D>(rr, g) - rmax;  // <= 0
-        // 2^k in fp16: normal for k >= -14, subnormal down to -24, else 0
-        const uint16_t hb = k >= -14 ? (uint16_t)((k + 15) << 10) : k >= -24 ? (uint16_t)(1u << (k + 24)) : 0;
-        __half2 s2 = __halves2half2(__ushort_as_half(hb), __ushort_as_half(hb));
-        const uint32_t *w = reinterpret_cast<const uint32_t *>(&rr.code[gl]);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {  // 4 bytes -> 8 channels -> one 16-byte chunk
-            uint32_t outw[4];
-#pragma unroll
-            for (int bb = 0; bb < 4; ++bb) {
-                __half2_raw hr = __nv_cvt_fp4x2_to_halfraw2((__nv_fp4x2_storage_t)((w[c] >> (8 * bb)) & 0xFF), __NV_E2M1);
-                __half2 h = __hmul2(*reinterpret_cast<__half2 *>(&hr), s2);
-                outw[bb] = *reinterpret_cast<uint32_t *>(&h);
+            for (int h = 0; h < 2; ++h) {
+                const __half_raw hr = __nv_cvt_fp8_to_halfraw(
+                    (__nv_fp8_storage_t)scale_byte<D>(rr, 2 * gl + h), __NV_E4M3);
+                s2[h] = __halves2half2(__half(hr), __half(hr));
             }
-            *reinterpret_cast<uint4 *>(E + e_chunk_off<D>(j, 4 * g + c)) = make_uint4(outw[0], outw[1], outw[2], outw[3]);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t outw[4];
+#pragma unroll
+                for (int bb = 0; bb < 4; ++bb) {
+                    __half2_raw hr =
+                        __nv_cvt_fp4x2_to_halfraw2((__nv_fp4x2_storage_t)((w[c] >> (8 * bb)) & 0xFF), __NV_E2M1);
+                    __half2 h = __hmul2(*reinterpret_cast<__half2 *>(&hr), s2[c >> 1]);
+                    outw[bb] = *reinterpret_cast<uint32_t *>(&h);
+                }
+                *reinterpret_cast<uint4 *>(E + e_chunk_off<D>(j, 4 * g + c)) =
+                    make_uint4(outw[0], outw[1], outw[2], outw[3]);
+            }
         }
+        return 0;
+    } else {
+        int rmax = 0;
+#pragma unroll
+        for (int g = 0; g < Cfg<D>::GPR; ++g) rmax = max(rmax, scale_byte<D>(rr, g));
+#pragma unroll
+        for (int gl = 0; gl < Cfg<D>::GPR / 2; ++gl) {
+            const int g = g0 + gl;
+            const int k = scale_byte<D>(rr, g) - rmax;  // <= 0
+            // 2^k in fp16: normal for k >= -14, subnormal down to -24, else 0
+            const uint16_t hb = k >= -14 ? (uint16_t)((k + 15) << 10) : k >= -24 ? (uint16_t)(1u << (k + 24)) : 0;
+            __half2 s2 = __halves2half2(__ushort_as_half(hb), __ushort_as_half(hb));
+            const uint32_t *w = reinterpret_cast<const uint32_t *>(&rr.code[gl]);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {  // 4 bytes -> 8 channels -> one 16-byte chunk
+                uint32_t outw[4];
+#pragma unroll
+                for (int bb = 0; bb < 4; ++bb) {
+                    __half2_raw hr =
+                        __nv_cvt_fp4x2_to_halfraw2((__nv_fp4x2_storage_t)((w[c] >> (8 * bb)) & 0xFF), __NV_E2M1);
+                    __half2 h = __hmul2(*reinterpret_cast<__half2 *>(&hr), s2);
+                    outw[bb] = *reinterpret_cast<uint32_t *>(&h);
+                }
+                *reinterpret_cast<uint4 *>(E + e_chunk_off<D>(j, 4 * g + c)) =
+                    make_uint4(outw[0], outw[1], outw[2], outw[3]);
+            }
+        }
+        return rmax - 127;
     }
-    return rmax - 127;
 }
 
 // Window tile: cp.async this thread's half of the bf16 row into E' and convert
@@ -632,7 +678,7 @@ __global__ void __launch_bounds__(256) attend_merge_kernel(const long long *tpre
 }
 
 // ---------------------------------------------------------------- main kernel
-template <int D>
+template <int D, int SF>
 __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
     using C = Cfg<D>;
     extern __shared__ uint8_t smem_raw[];
@@ -701,7 +747,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
     }
     uint32_t n_q = 0;           // Q' copies waited for
     uint32_t n_q_issued = 1;    // ... and issued
-    prefetch_row<D>(a, cur, row_block_raw(a, cur), rr);
+    prefetch_row<D, SF>(a, cur, row_block_raw(a, cur), rr);
     // the next tile and this thread's selected index in it (one tile ahead of its row loads)
     TileRef nxt = cur;
     int blk_nxt = -1;
@@ -746,14 +792,14 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
                 Rj = load_window_row<D>(a, cur, E, E_s, xmax, valid);
             } else {
                 valid = rr.valid;
-                Rj = dequant_row<D>(rr, E);
+                Rj = dequant_row<D, SF>(rr, E);
             }
             // next tile (possibly of the next query): start its row loads now,
             // and the selected index of the tile after it
             TileRef nxt2 = nxt;
             int blk_nxt2 = -1;
             if (t + 1 < t_end) {
-                prefetch_row<D>(a, nxt, blk_nxt, rr);
+                prefetch_row<D, SF>(a, nxt, blk_nxt, rr);
                 if (t + 2 < t_end) {
                     nxt2 = advance(a, nxt, t + 2);
                     blk_nxt2 = row_block_raw(a, nxt2);
@@ -953,11 +999,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TMEM_COLS) : "memory");
 }
 
-template <int D>
+template <int D, int SF>
 cudaError_t launch_main(const AttArgs &a, int num_ctas, cudaStream_t s) {
     cudaError_t err;
     const int smem = Cfg<D>::SMEM;
-    if ((err = cudaFuncSetAttribute(attend_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
+    if ((err = cudaFuncSetAttribute(attend_kernel<D, SF>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
+        cudaSuccess)
         return err;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(num_ctas);
@@ -969,7 +1016,7 @@ cudaError_t launch_main(const AttArgs &a, int num_ctas, cudaStream_t s) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, attend_kernel<D>, a);
+    return cudaLaunchKernelEx(&cfg, attend_kernel<D, SF>, a);
 }
 
 template <int D>
@@ -1046,12 +1093,16 @@ cudaError_t launch_attend(const csa_cache &c, const void *q, int Nq, int H, cons
         if ((err = launch_schedule<512>(c, a, q_offsets, qp, wl, topk, max_win, q, num_ctas, qinfo, tprefix, cta_q, sq,
                                         qimg, s)) != cudaSuccess)
             return err;
-        if ((err = launch_main<512>(a, num_ctas, s)) != cudaSuccess) return err;
+        err = c.scale_fmt == CSA_SCALE_E4M3_16 ? launch_main<512, kScaleE4M3x16>(a, num_ctas, s)
+                                                : launch_main<512, kScaleE8M0x32>(a, num_ctas, s);
+        if (err != cudaSuccess) return err;
     } else if (D == 128) {
         if ((err = launch_schedule<128>(c, a, q_offsets, qp, wl, topk, max_win, q, num_ctas, qinfo, tprefix, cta_q, sq,
                                         qimg, s)) != cudaSuccess)
             return err;
-        if ((err = launch_main<128>(a, num_ctas, s)) != cudaSuccess) return err;
+        err = c.scale_fmt == CSA_SCALE_E4M3_16 ? launch_main<128, kScaleE4M3x16>(a, num_ctas, s)
+                                                : launch_main<128, kScaleE8M0x32>(a, num_ctas, s);
+        if (err != cudaSuccess) return err;
     } else {
         return cudaErrorInvalidValue;
     }

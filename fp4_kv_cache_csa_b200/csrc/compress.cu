@@ -4,8 +4,9 @@
 // Source: "Frontier Architecture Decoding Notes (4): DeepSeek V4", section 1
 // (KV of every 4 tokens compressed into one entry for CSA, up to 128 for HCA);
 // DeepSeek-V4.1-Flash podcast transcript, cue 16 (main KV stored as MXFP4,
-// E2M1 elements). Pooling form, gate and E8M0/32 scale: the library's stated
-// readings (see include/csa.h).
+// E2M1 elements with one E4M3 scale per sixteen channels). Pooling form, gate
+// and the E8M0/32 scale (the default format): the library's stated readings
+// (see include/csa.h).
 //
 // One warp builds one block (eight warps share a block when m >= 32). Lane l
 // owns E = D/32 consecutive channels [l*E, l*E+E) and EI = dI/32 consecutive
@@ -15,6 +16,7 @@
 // kernel is HBM-bound: it reads m*(D+dI)*2 bytes and writes D/2 + D/32 + key
 // bytes per block.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_fp8.h>
 
 #include "common.cuh"
@@ -24,6 +26,20 @@ namespace csa {
 namespace {
 
 constexpr int kWarpsPerCta = 4;
+
+// E2M1 code of v / s for a group scale s > 0 (E4M3 scales), from the rounding
+// midpoints scaled by s: th[k] = mid_k * s is exact in float32 (a midpoint has
+// at most 3 significant bits, an E4M3 value 4), so comparing |v| with th[k]
+// takes the decision on the exact quotient, with no division. Same tie rule
+// and saturation as e2m1_code. s = 0 is passed as +inf: every code is a zero
+// magnitude with the element's sign.
+__device__ __forceinline__ uint32_t e2m1_code_th(float v, const float (&th)[7]) {
+    uint32_t sign = (__float_as_uint(v) >> 28) & 8u;
+    float a = fabsf(v);
+    uint32_t c = a <= th[0] ? 0u : a < th[1] ? 1u : a <= th[2] ? 2u : a < th[3] ? 3u
+               : a <= th[4] ? 4u : a < th[5] ? 5u : a <= th[6] ? 6u : 7u;
+    return sign | c;
+}
 
 // E2M1 code of a scaled value s (|s| < 8), round to nearest with ties to the
 // even code, saturating at 6; the sign bit is kept even when the magnitude
@@ -83,11 +99,12 @@ struct CompressArgs {
     const int32_t *tok_offsets;    // [B+1]
     const int32_t *n_blocks;       // [B]
     uint8_t *fp4;                  // [B][cap][D/2]
-    uint8_t *scale;                // [B][cap][D/32]
+    uint8_t *scale;                // [B][cap][D/32] (E8M0) or [B][cap][D/16] (E4M3)
     uint8_t *idx_key;              // [B][cap][dI * esize] or null
     int32_t *status;
     int m, cap, D, dI;
     int idx_e4m3;
+    int scale_e4m3;                // 1: one E4M3 scale per 16 elements, 0: one E8M0 scale per 32
 };
 
 // E channels per lane (D = 32*E), EI indexer channels per lane (0 = no
@@ -217,7 +234,8 @@ pool_quantize_kernel(CompressArgs a) {
     }
 
     const size_t row = (size_t)b * a.cap + base + jb;
-    // ---- main entry -> MXFP4 ----
+    // ---- main entry -> FP4 codes + one scale byte per group ----
+    static_assert(E <= 16, "a lane's channels lie inside one 16-element group");
     float e[E];
     float amax = 0.f;
 #pragma unroll
@@ -225,18 +243,32 @@ pool_quantize_kernel(CompressArgs a) {
         e[k] = acc[k] / den;
         amax = fmaxf(amax, fabsf(e[k]));
     }
-    // a 32-element group spans 32/E lanes
-#pragma unroll
-    for (int o = 1; o < 32 / E; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    // X = floor(log2 amax) - 2 from the exponent field, clamped to >= -127
-    // (zero and subnormal amax land on the clamp); byte = X + 127.
-    const int expbits = (int)((__float_as_uint(amax) >> 23) & 0xFF);
-    const int sbyte = max(expbits - 2, 0);
-    const float inv = __uint_as_float((uint32_t)(254 - sbyte) << 23);  // 2^-X, X = sbyte-127
     uint32_t packed[E / 2 > 0 ? E / 2 : 1];
+    if (a.scale_e4m3) {
+        // a 16-element group spans 16/E lanes; s = E4M3(amax / 6), RNE, saturating
 #pragma unroll
-    for (int k = 0; k < E; k += 2)
-        packed[k / 2] = e2m1_code(e[k] * inv) | (e2m1_code(e[k + 1] * inv) << 4);
+        for (int o = 1; o < 16 / E; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        const __nv_fp8_storage_t sb = __nv_cvt_float_to_fp8(__fdiv_rn(amax, 6.0f), __NV_SATFINITE, __NV_E4M3);
+        const float sv = __half2float(__half(__nv_cvt_fp8_to_halfraw(sb, __NV_E4M3)));
+        const float sc = sv > 0.f ? sv : INFINITY;
+        const float th[7] = {0.25f * sc, 0.75f * sc, 1.25f * sc, 1.75f * sc, 2.5f * sc, 3.5f * sc, 5.0f * sc};
+#pragma unroll
+        for (int k = 0; k < E; k += 2) packed[k / 2] = e2m1_code_th(e[k], th) | (e2m1_code_th(e[k + 1], th) << 4);
+        if (lane % (16 / E) == 0) a.scale[row * (a.D / 16) + lane / (16 / E)] = (uint8_t)sb;
+    } else {
+        // a 32-element group spans 32/E lanes
+#pragma unroll
+        for (int o = 1; o < 32 / E; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        // X = floor(log2 amax) - 2 from the exponent field, clamped to >= -127
+        // (zero and subnormal amax land on the clamp); byte = X + 127.
+        const int expbits = (int)((__float_as_uint(amax) >> 23) & 0xFF);
+        const int sbyte = max(expbits - 2, 0);
+        const float inv = __uint_as_float((uint32_t)(254 - sbyte) << 23);  // 2^-X, X = sbyte-127
+#pragma unroll
+        for (int k = 0; k < E; k += 2)
+            packed[k / 2] = e2m1_code(e[k] * inv) | (e2m1_code(e[k + 1] * inv) << 4);
+        if (lane % (32 / E) == 0) a.scale[row * (a.D / 32) + lane / (32 / E)] = (uint8_t)sbyte;
+    }
     uint8_t *dst = a.fp4 + row * (a.D / 2) + lane * (E / 2);
     if constexpr (E == 16) {
         uint2 w;
@@ -250,7 +282,6 @@ pool_quantize_kernel(CompressArgs a) {
     } else {
         dst[0] = (uint8_t)packed[0];
     }
-    if (lane % (32 / E) == 0) a.scale[row * (a.D / 32) + lane / (32 / E)] = (uint8_t)sbyte;
 
     // ---- pooled indexer key -> bf16 or e4m3 ----
     if constexpr (EI > 0) {
@@ -331,6 +362,7 @@ cudaError_t launch_compress(const csa_cache &c, const void *kv_tok, const void *
     a.D = c.dim;
     a.dI = c.idx_key ? c.idx_dim : 0;
     a.idx_e4m3 = c.idx_dtype == CSA_IDX_E4M3;
+    a.scale_e4m3 = c.scale_fmt == CSA_SCALE_E4M3_16;
     const int max_blocks = (n_tokens + c.block - 1) / c.block;
     if (max_blocks > 0) {
         cudaError_t err;

@@ -40,7 +40,8 @@ csa_status check_cache(const csa_cache *c) {
     if (c->batch < 1 || c->capacity < 1 || c->block < 1 || c->block > 128) return CSA_ERR_SHAPE;
     if (c->dim < 64 || c->dim % 32 != 0) return CSA_ERR_SHAPE;
     if (c->capacity > kMaxCapacity) return CSA_ERR_UNSUPPORTED;
-    if (!aligned(c->fp4, 16) || !aligned(c->scale, 4) || !aligned(c->n_blocks, 4)) return CSA_ERR_ALIGN;
+    if (c->scale_fmt != CSA_SCALE_E8M0_32 && c->scale_fmt != CSA_SCALE_E4M3_16) return CSA_ERR_SHAPE;
+    if (!aligned(c->fp4, 16) || !aligned(c->scale, 16) || !aligned(c->n_blocks, 4)) return CSA_ERR_ALIGN;
     if (c->status && !aligned(c->status, 4)) return CSA_ERR_ALIGN;
     if (c->idx_key) {
         if (c->idx_dtype != CSA_IDX_BF16 && c->idx_dtype != CSA_IDX_E4M3) return CSA_ERR_SHAPE;
@@ -69,7 +70,7 @@ const char *csa_status_string(int32_t status) {
     }
 }
 
-int32_t csa_version(void) { return 100; }
+int32_t csa_version(void) { return 101; }
 
 csa_status csa_compress_quantize(const csa_cache *cache, const void *kv_tok, const void *idx_tok, const float *gate_w,
                                  const int32_t *tok_offsets, int32_t n_tokens, csa_stream_t stream) {

@@ -107,6 +107,17 @@ def random_cache_bytes(n_rows: int, dim: int, *ids: int, scale_lo: int = 123, sc
     return fp4, sc
 
 
+def random_cache_bytes_e4m3x16(n_rows: int, dim: int, *ids: int, scale_lo: int = 0x1C, scale_hi: int = 0x2C):
+    """Raw FP4 cache rows with one E4M3 scale byte per 16 elements, drawn as
+    bytes: uniform code bytes and scale bytes uniform in [scale_lo, scale_hi]
+    (0x1C .. 0x2C spans the scales a pooled N(0,1) group lands in). Returns
+    (fp4 [n, dim/2] u8, scale [n, dim/16] u8)."""
+    g = generator(*ids)
+    fp4 = g.integers(0, 256, size=(n_rows, dim // 2), dtype=np.uint8)
+    sc = g.integers(scale_lo, scale_hi, size=(n_rows, dim // 16), endpoint=True, dtype=np.uint8)
+    return fp4, sc
+
+
 def decode_inputs(wl: Workload, n_queries_per_req: int = 1, *, seed_base: int = 100):
     """Per-query decode tensors: q [Nq, H, D] bf16, q_idx [Nq, H_I, d_I] bf16,
     w [Nq, H_I] f32 (N(0,1)/sqrt(H_I))."""

@@ -17,7 +17,9 @@
  *   gate logit per token, g_t = <kv_t, w_g>; indexer score
  *   s_j = sum_h w_h * ReLU(<q_idx_h, k_j>); top-k ties go to the lower block
  *   index; one joint softmax covers the selected entries and the window;
- *   MXFP4 = E2M1 elements with one E8M0 scale per 32 elements (OCP MX v1.0).
+ *   MXFP4 = E2M1 elements with one E8M0 scale per 32 elements (OCP MX v1.0);
+ *   a cache may instead hold one E4M3 scale per 16 elements (cue 16's own
+ *   wording), selected by csa_cache.scale_fmt.
  *
  * Conventions for every call:
  *   - Pointers inside csa_cache and every tensor argument are DEVICE pointers,
@@ -61,6 +63,14 @@ typedef enum {
 
 typedef enum { CSA_IDX_BF16 = 0, CSA_IDX_E4M3 = 1 } csa_idx_dtype;
 
+/* Scale format of the FP4 main KV (E2M1 elements in both):
+ *   CSA_SCALE_E8M0_32  one E8M0 byte per 32 elements, value 2^(byte - 127)
+ *                      (OCP MX v1.0 MXFP4);
+ *   CSA_SCALE_E4M3_16  one E4M3 byte per 16 elements, no second-level scale
+ *                      (the format the DeepSeek-V4.1-Flash podcast transcript
+ *                      names in cue 16). */
+typedef enum { CSA_SCALE_E8M0_32 = 0, CSA_SCALE_E4M3_16 = 1 } csa_scale_fmt;
+
 /* Bits OR-ed into *cache->status by the kernels. */
 #define CSA_DEV_TOKEN_COUNT 0x1  /* a request's new-token count is not a multiple of m: request skipped */
 #define CSA_DEV_CAPACITY    0x2  /* appending would exceed capacity: request skipped                  */
@@ -72,13 +82,17 @@ typedef enum { CSA_IDX_BF16 = 0, CSA_IDX_E4M3 = 1 } csa_idx_dtype;
  * One compressed cache (one layer). Per request b and block j:
  *   fp4     [batch][capacity][dim/2]   two E2M1 codes per byte, element 2i in the
  *                                      low nibble, element 2i+1 in the high nibble
- *   scale   [batch][capacity][dim/32]  E8M0 bytes, value 2^(byte-127)
+ *   scale   [batch][capacity][dim/32]  E8M0 bytes, value 2^(byte-127)  (CSA_SCALE_E8M0_32)
+ *           [batch][capacity][dim/16]  E4M3 bytes                      (CSA_SCALE_E4M3_16)
  *   idx_key [batch][capacity][idx_dim] bf16 or e4m3 pooled indexer keys; NULL for
  *                                      a cache that is only attended densely (HCA)
  *   n_blocks [batch]                   filled blocks per request; advanced by
  *                                      csa_compress_quantize
  *   status                             one int32 of CSA_DEV_* bits, or NULL
- * An element's value is E2M1(code) * 2^(scale - 127).
+ * An element's value is E2M1(code) * 2^(scale - 127) for E8M0 scales and
+ * E2M1(code) * E4M3(scale) for E4M3 scales (the scale byte of its group).
+ * scale_fmt was added after status, so the offsets of the other fields are
+ * those of ABI version 100.
  */
 typedef struct {
     int32_t batch;     /* requests, >= 1                                  */
@@ -92,12 +106,13 @@ typedef struct {
     int32_t idx_dtype; /* csa_idx_dtype                                   */
     int32_t *n_blocks;
     int32_t *status;
+    int32_t scale_fmt; /* csa_scale_fmt                                  */
 } csa_cache;
 
 /* Human-readable name of a csa_status value. Never NULL. */
 const char *csa_status_string(int32_t status);
 
-/* Library ABI version (major * 100 + minor). */
+/* Library ABI version (major * 100 + minor). 101 added csa_cache.scale_fmt. */
 int32_t csa_version(void);
 
 /*
@@ -107,11 +122,15 @@ int32_t csa_version(void);
  * block n_blocks[b], n_blocks[b]+1, ...; n_blocks[b] is then advanced.
  *   gate logit   g_t = sum_d kv_t[d] * gate_w[d]            (float32)
  *   weights      a = softmax over the block's m logits
- *   main entry   e[d] = sum_t a_t kv_t[d], stored as MXFP4:
- *                per 32 elements X = floor(log2(max|e|)) - 2 clamped to [-127,127]
- *                (X = -127 for an all-zero group), code = E2M1 round-to-nearest-even
- *                of e * 2^-X saturated to +-6, sign kept (a negative value that
- *                rounds to zero is code 0x8)
+ *   main entry   e[d] = sum_t a_t kv_t[d], stored as FP4 in the cache's scale format:
+ *                E8M0/32: per 32 elements X = floor(log2(max|e|)) - 2 clamped to
+ *                [-127,127] (X = -127 for an all-zero group), code = E2M1
+ *                round-to-nearest-even of e * 2^-X saturated to +-6;
+ *                E4M3/16: per 16 elements s = E4M3 round-to-nearest-even of
+ *                max|e| / 6 saturated to 448, code = E2M1 round-to-nearest-even
+ *                of e / s saturated to +-6 (zero magnitude when s = 0);
+ *                in both the sign is kept (a negative value that rounds to
+ *                zero is code 0x8)
  *   indexer key  k[c] = sum_t a_t idx_t[c], stored as bf16 (RNE) or e4m3 (RNE,
  *                saturated to +-448) per cache->idx_dtype
  * Arguments:

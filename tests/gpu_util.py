@@ -21,7 +21,7 @@ def host(t):
     return t.cpu().numpy()
 
 
-def make_cache(fp4, scale, n_blocks, block, idx_key=None, idx_dtype=0):
+def make_cache(fp4, scale, n_blocks, block, idx_key=None, idx_dtype=0, scale_fmt=0):
     """Device cache from numpy planes (idx_key as raw bytes [B, cap, key_bytes])."""
     import torch
 
@@ -33,4 +33,5 @@ def make_cache(fp4, scale, n_blocks, block, idx_key=None, idx_dtype=0):
         if idx_dtype == 0:
             ik = ik.view(torch.bfloat16)
     return csa.Cache(fp4=dev(fp4), scale=dev(scale), n_blocks=dev(np.asarray(n_blocks, np.int32)), block=block,
-                     idx_key=ik, idx_dtype=idx_dtype, status=torch.zeros(1, dtype=torch.int32, device="cuda"))
+                     idx_key=ik, idx_dtype=idx_dtype, status=torch.zeros(1, dtype=torch.int32, device="cuda"),
+                     scale_fmt=scale_fmt)

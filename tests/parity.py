@@ -14,8 +14,11 @@ accumulates in float32 in another order than the oracle's double precision:
   zero magnitude; it may differ where the oracle's value is within that same
   bound of 0.
 * MXFP4 scale byte: the oracle's float32 group amax lies within 1e-5 relative of
-  a power of two; the GPU group must then be a correct quantization of the
-  oracle's pooled values with the GPU's scale (same near-midpoint rule).
+  a power of two (E8M0 per 32), or amax / 6 lies within 1e-5 relative of the
+  midpoint of the two E4M3 scales (E4M3 per 16); the GPU group must then be a
+  correct quantization of the oracle's pooled values with the GPU's scale
+  (same near-midpoint rule).
+* E4M3-per-16 codes: as for MXFP4, with the scaled value v / s.
 * BF16 / E4M3 indexer keys: the oracle's float32 value lies within 1e-5 relative
   of a rounding midpoint of the format; the GPU byte must be a neighbour.
 * top-k: where the oracle's k-th and (k+1)-th scores differ by less than 1e-5
@@ -76,44 +79,69 @@ def e2m1_neighbours(c1, c2):
         (((c1 & 7) <= 1) & ((c2 & 7) <= 1))
 
 
-def check_mxfp4(gpu_fp4, gpu_scale, orc_fp4, orc_scale, pooled, strict=False, max_frac=1e-3, tol=None):
-    """Compare MXFP4 planes [n, D/2], [n, D/32] against the oracle's bytes and float32 pooled values [n, D].
-    tol: optional [n, D] absolute error bound of the GPU's pooled values."""
+def _scale_values(scale_bytes, scale_fmt):
+    """Decoded scale of every group: 2^(byte-127) (E8M0) or the E4M3 value."""
+    b = np.asarray(scale_bytes).astype(np.int64)
+    if scale_fmt == oracle.SCALE_E8M0_32:
+        return np.ldexp(1.0, b - 127)
+    table = np.array([oracle.e4m3_decode(c) for c in range(256)], np.float64)
+    return table[b]
+
+
+def _scale_near_tie(amax, gpu_byte, orc_byte, scale_fmt, gtol):
+    """Whether a differing scale byte is a near-tie of the scale rule on the oracle's group amax."""
+    if scale_fmt == oracle.SCALE_E8M0_32:
+        lo_p, hi_p = 2.0 ** math.floor(math.log2(amax)), 2.0 ** math.ceil(math.log2(amax))
+        return min(abs(amax - lo_p), abs(amax - hi_p)) <= max(REL * amax, gtol)
+    # E4M3 of amax / 6: two neighbouring scale codes, the ratio near their midpoint
+    if abs(int(gpu_byte) - int(orc_byte)) != 1 or max(int(gpu_byte), int(orc_byte)) > 0x7E:
+        return False
+    mid = 0.5 * (oracle.e4m3_decode(int(gpu_byte)) + oracle.e4m3_decode(int(orc_byte)))
+    return abs(amax / 6.0 - mid) <= max(REL * mid, gtol / 6.0)
+
+
+def check_mxfp4(gpu_fp4, gpu_scale, orc_fp4, orc_scale, pooled, strict=False, max_frac=1e-3, tol=None,
+                scale_fmt=oracle.SCALE_E8M0_32):
+    """Compare FP4 planes [n, D/2], [n, D/G] (G = 32 for E8M0 scales, 16 for E4M3) against the
+    oracle's bytes and float32 pooled values [n, D]. tol: optional [n, D] absolute error bound of
+    the GPU's pooled values."""
     gpu_fp4, gpu_scale = np.asarray(gpu_fp4), np.asarray(gpu_scale)
     if strict:
         assert np.array_equal(gpu_scale, orc_scale), "scale bytes differ (strict)"
         assert np.array_equal(gpu_fp4, orc_fp4), "codes differ (strict)"
         return 0
+    G = oracle.group_size(scale_fmt)
     n, D = pooled.shape
     gc, oc = unpack_codes(gpu_fp4), unpack_codes(orc_fp4)
     exceptions = 0
     bad_scale = np.argwhere(gpu_scale != orc_scale)
     pooled64 = pooled.astype(np.float64)
     for r, g in bad_scale:
-        grp = pooled[r, 32 * g:32 * g + 32]
+        grp = pooled[r, G * g:G * g + G]
         amax = float(np.max(np.abs(grp)))
         assert amax > 0
-        frac = math.log2(amax) - math.floor(math.log2(amax))
-        lo_p, hi_p = 2.0 ** math.floor(math.log2(amax)), 2.0 ** math.ceil(math.log2(amax))
-        gtol = 0.0 if tol is None else float(np.max(tol[r, 32 * g:32 * g + 32]))
-        near_pow2 = min(abs(amax - lo_p), abs(amax - hi_p)) <= max(REL * amax, gtol)
-        assert near_pow2, f"scale byte differs at row {r} group {g} (amax {amax}, frac {frac})"
-        X = int(gpu_scale[r, g]) - 127
-        s = np.ldexp(pooled64[r, 32 * g:32 * g + 32], -X)
-        ts = 0.0 if tol is None else np.ldexp(tol[r, 32 * g:32 * g + 32].astype(np.float64), -X)
+        gtol = 0.0 if tol is None else float(np.max(tol[r, G * g:G * g + G]))
+        assert _scale_near_tie(amax, gpu_scale[r, g], orc_scale[r, g], scale_fmt, gtol), \
+            f"scale byte differs at row {r} group {g} (amax {amax})"
+        sv = float(_scale_values(gpu_scale[r, g], scale_fmt))
+        assert sv > 0
+        s = pooled64[r, G * g:G * g + G] / sv
+        ts = 0.0 if tol is None else tol[r, G * g:G * g + G].astype(np.float64) / sv
         want = np.array([oracle.e2m1_encode(float(v)) for v in np.clip(s, -1e9, 1e9)])
-        got = gc[r, 32 * g:32 * g + 32]
+        got = gc[r, G * g:G * g + G]
         ok = (got == want) | (near_e2m1_midpoint(s, ts) & e2m1_neighbours(got, want))
         assert ok.all(), f"group ({r},{g}) with the GPU scale is not a valid quantization"
-        oc[r, 32 * g:32 * g + 32] = got
+        oc[r, G * g:G * g + G] = got
         exceptions += 1
     diff = np.argwhere(gc != oc)
     if len(diff):
-        X = (orc_scale.astype(np.int64) - 127).repeat(32, axis=-1)
-        s = np.ldexp(pooled64, -X)
+        sv = _scale_values(orc_scale, scale_fmt).repeat(G, axis=-1)
         rr, dd = diff[:, 0], diff[:, 1]
-        ts = 0.0 if tol is None else np.ldexp(tol.astype(np.float64), -X)[rr, dd]
-        ok = near_e2m1_midpoint(s[rr, dd], ts) & e2m1_neighbours(gc[rr, dd], oc[rr, dd])
+        svd = sv[rr, dd]
+        # a zero scale stores every element as a zero magnitude: only the sign can differ
+        s = np.where(svd > 0, pooled64[rr, dd] / np.where(svd > 0, svd, 1.0), 0.0)
+        ts = 0.0 if tol is None else tol[rr, dd].astype(np.float64) / np.where(svd > 0, svd, 1.0)
+        ok = near_e2m1_midpoint(s, ts) & e2m1_neighbours(gc[rr, dd], oc[rr, dd])
         assert ok.all(), f"{(~ok).sum()} codes differ away from a rounding midpoint, e.g. {diff[~ok][:5]}"
         exceptions += len(diff)
     assert exceptions <= max(4, max_frac * gc.size), f"too many near-tie exceptions: {exceptions}"

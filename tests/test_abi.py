@@ -32,7 +32,7 @@ def test_every_declared_symbol_is_exported(lib):
     assert set(names) == set(csa.EXPORTED), names
     for n in names:
         assert hasattr(lib, n), n
-    assert lib.csa_version() == 100
+    assert lib.csa_version() == 101
     assert lib.csa_status_string(0) == b"ok"
     assert lib.csa_status_string(99) == b"unknown status"
 
@@ -40,10 +40,10 @@ def test_every_declared_symbol_is_exported(lib):
 def fake_cache(**kw):
     # host addresses that are never dereferenced (every call below fails validation first)
     d = dict(batch=2, dim=512, block=4, capacity=1024, fp4=0x10000, scale=0x20000, idx_key=0x30000,
-             idx_dim=128, idx_dtype=1, n_blocks=0x40000, status=0)
+             idx_dim=128, idx_dtype=1, n_blocks=0x40000, status=0, scale_fmt=0)
     d.update(kw)
     c = csa._CCache(d["batch"], d["dim"], d["block"], d["capacity"], d["fp4"], d["scale"], d["idx_key"],
-                    d["idx_dim"], d["idx_dtype"], d["n_blocks"], d["status"] or None)
+                    d["idx_dim"], d["idx_dtype"], d["n_blocks"], d["status"] or None, d["scale_fmt"])
     return c
 
 
@@ -64,6 +64,9 @@ def test_compress_validation(lib):
     assert compress(lib, fake_cache(idx_dim=96)) == ERR_UNSUPPORTED
     assert compress(lib, fake_cache(capacity=(1 << 19) + 1)) == ERR_UNSUPPORTED
     assert compress(lib, fake_cache(fp4=0x10008)) == ERR_ALIGN
+    assert compress(lib, fake_cache(scale=0x20004)) == ERR_ALIGN
+    assert compress(lib, fake_cache(scale_fmt=2)) == ERR_SHAPE
+    assert compress(lib, fake_cache(scale_fmt=-1)) == ERR_SHAPE
     assert compress(lib, fake_cache(), kv=0x50008) == ERR_ALIGN
     assert compress(lib, fake_cache(), n=-1) == ERR_SHAPE
 
@@ -124,3 +127,18 @@ def test_missing_library_raises():
             csa.load_library("/nonexistent/libcsa.so")
     finally:
         csa._lib = saved
+
+
+def test_cache_struct_layout_matches_the_header(tmp_path):
+    # the ctypes mirror of csa_cache has the C compiler's field offsets and size
+    src = tmp_path / "layout.c"
+    fields = [f[0] for f in csa._CCache._fields_]
+    body = "".join(f'printf("%zu\\n", offsetof(csa_cache, {f}));' for f in fields)
+    src.write_text('#include <stddef.h>\n#include <stdio.h>\n#include "csa.h"\n'
+                   f'int main(void) {{ {body} printf("%zu\\n", sizeof(csa_cache)); return 0; }}\n')
+    exe = tmp_path / "layout"
+    import subprocess
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    got = [int(x) for x in subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()]
+    want = [getattr(csa._CCache, f).offset for f in fields] + [ctypes.sizeof(csa._CCache)]
+    assert got == want

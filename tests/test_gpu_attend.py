@@ -1,7 +1,7 @@
 """GPU parity of csa_decode_attend / hca_decode_attend (rows a5-a8) against the oracle.
 
-Cache bytes are seeded inputs (uniform E2M1 code bytes, E8M0 scale bytes in the
-range pooled N(0,1) blocks land in); queries and window rows are N(0,1) bf16.
+Cache bytes are seeded inputs (uniform E2M1 code bytes, E8M0 or E4M3 scale bytes
+in the range pooled N(0,1) blocks land in); queries and window rows are N(0,1) bf16.
 Tolerance: per (query, head) row, max_d |gpu - oracle| / max_d |oracle| <= 2e-3;
 lse within 1e-3 + 1e-4 |lse|."""
 import numpy as np
@@ -20,6 +20,11 @@ def cache_bytes(B, cap, D, seed, lo=123, hi=126):
     return fp4.reshape(B, cap, D // 2), sc.reshape(B, cap, D // 32)
 
 
+def cache_bytes_e4m3x16(B, cap, D, seed, lo=0x1C, hi=0x2C):
+    fp4, sc = datagen.random_cache_bytes_e4m3x16(B * cap, D, seed, 44, scale_lo=lo, scale_hi=hi)
+    return fp4.reshape(B, cap, D // 2), sc.reshape(B, cap, D // 16)
+
+
 def window(Nq, W, D, seed, wlen=None):
     win = datagen.normal_bf16((Nq * W, D), seed, 41)
     ws = (np.arange(Nq) * W).astype(np.int64)
@@ -36,7 +41,7 @@ def check(out, lse, ref, ref_lse, H):
     return err
 
 
-def run_csa(fp4, sc, n_blocks, q_offsets, sel, H, D, win=None, ws=None, wl=None, seed=50, max_win=128):
+def run_csa(fp4, sc, n_blocks, q_offsets, sel, H, D, win=None, ws=None, wl=None, seed=50, max_win=128, scale_fmt=0):
     import torch
 
     import fp4_kv_cache_csa_b200 as csa
@@ -44,8 +49,8 @@ def run_csa(fp4, sc, n_blocks, q_offsets, sel, H, D, win=None, ws=None, wl=None,
     Nq = int(q_offsets[-1])
     q = datagen.normal_bf16((Nq, H, D), seed, 42)
     scale = 1.0 / np.sqrt(D)
-    ref, ref_lse = oracle.csa_attend(fp4, sc, q_offsets, q, sel, win, ws, wl, scale)
-    cache = make_cache(fp4, sc, n_blocks, 4)
+    ref, ref_lse = oracle.csa_attend(fp4, sc, q_offsets, q, sel, win, ws, wl, scale, scale_fmt=scale_fmt)
+    cache = make_cache(fp4, sc, n_blocks, 4, scale_fmt=scale_fmt)
     lse = torch.empty(Nq, H, dtype=torch.float32, device="cuda")
     out = csa.csa_decode_attend(cache, dev(q), dev(np.asarray(q_offsets, np.int32)), dev(sel),
                                 None if win is None else dev(win), None if ws is None else dev(ws),
@@ -131,7 +136,7 @@ def test_scale_spread_rows():
 
 # ---------------------------------------------------------------- HCA
 
-def run_hca(fp4, sc, n_blocks, q_offsets, q_pos, H, D, m, win=None, ws=None, wl=None, seed=60):
+def run_hca(fp4, sc, n_blocks, q_offsets, q_pos, H, D, m, win=None, ws=None, wl=None, seed=60, scale_fmt=0):
     import torch
 
     import fp4_kv_cache_csa_b200 as csa
@@ -139,8 +144,9 @@ def run_hca(fp4, sc, n_blocks, q_offsets, q_pos, H, D, m, win=None, ws=None, wl=
     Nq = int(q_offsets[-1])
     q = datagen.normal_bf16((Nq, H, D), seed, 43)
     scale = 1.0 / np.sqrt(D)
-    ref, ref_lse = oracle.hca_attend(fp4, sc, n_blocks, q_offsets, q_pos, q, win, ws, wl, scale, m=m)
-    cache = make_cache(fp4, sc, n_blocks, m)
+    ref, ref_lse = oracle.hca_attend(fp4, sc, n_blocks, q_offsets, q_pos, q, win, ws, wl, scale, m=m,
+                                     scale_fmt=scale_fmt)
+    cache = make_cache(fp4, sc, n_blocks, m, scale_fmt=scale_fmt)
     lse = torch.empty(Nq, H, dtype=torch.float32, device="cuda")
     out = csa.hca_decode_attend(cache, dev(q), dev(np.asarray(q_offsets, np.int32)), dev(np.asarray(q_pos, np.int32)),
                                 None if win is None else dev(win), None if ws is None else dev(ws),
@@ -178,3 +184,42 @@ def test_csa_with_all_blocks_equals_hca():
     b = host(csa.hca_decode_attend(cache, q, dev(np.array([0, 1], np.int32)), dev(np.array([2559], np.int32)),
                                    dev(win), dev(ws), dev(wl)))
     assert parity.attention_row_error(a, b)[0] <= 1e-5
+
+
+# ---------------------------------------------------------------- E4M3 scale per 16 elements
+
+E4 = oracle.SCALE_E4M3_16
+
+
+def test_e4m3x16_csa_d512_h64():
+    fp4, sc = cache_bytes_e4m3x16(2, 16384, 512, 70)
+    sel = random_sel([16384, 9000], 1024, 2, 71, pad_from=[1024, 333])
+    win, ws, wl = window(2, 128, 512, 72, wlen=[128, 41])
+    err, st = run_csa(fp4, sc, [16384, 9000], np.array([0, 1, 2], np.int32), sel, 64, 512, win, ws, wl,
+                      scale_fmt=E4)
+    assert st == 0
+
+
+def test_e4m3x16_csa_d128_h16_split():
+    # 2048 selected entries per query: each query spans several CTAs and is merged
+    fp4, sc = cache_bytes_e4m3x16(1, 4096, 128, 73)
+    sel = random_sel([4096, 4096, 4096], 2048, 3, 74)
+    win, ws, wl = window(3, 128, 128, 75)
+    err, st = run_csa(fp4, sc, [4096], np.array([0, 3], np.int32), sel, 16, 128, win, ws, wl, scale_fmt=E4)
+    assert st == 0
+
+
+def test_e4m3x16_full_scale_range_is_exact_in_fp16():
+    # scale bytes over every positive finite E4M3 value (2^-9 .. 448, subnormals included):
+    # every E2M1 x E4M3 product is exact in fp16, with no per-row normalisation
+    fp4, sc = cache_bytes_e4m3x16(1, 2048, 512, 76, lo=0x01, hi=0x7E)
+    sel = random_sel([2048], 512, 1, 77)
+    win, ws, wl = window(1, 128, 512, 78)
+    run_csa(fp4, sc, [2048], np.array([0, 1], np.int32), sel, 64, 512, win, ws, wl, scale_fmt=E4)
+
+
+def test_e4m3x16_hca_dense():
+    fp4, sc = cache_bytes_e4m3x16(2, 8192, 512, 79)
+    win, ws, wl = window(2, 128, 512, 80)
+    run_hca(fp4, sc, [8192, 5000], np.array([0, 1, 2], np.int32), np.array([1048575, 700000], np.int32), 64, 512,
+            128, win, ws, wl, scale_fmt=E4)
