@@ -42,9 +42,26 @@ OUR_KERNELS_PER_STEP = 14  # compress 2x(pool, commit); index: schedule, scan, s
 SEED = 0x5EED0C5A
 
 
+SCALE_FMT = 0  # 0: one E8M0 scale per 32 elements (MXFP4, the headline format); 1: one E4M3 scale per 16
+SCALE_FMT_NAMES = {"e8m0x32": 0, "e4m3x16": 1}
+
+
 def set_batch(n: int):
     global B
     B = int(n)
+
+
+def set_scale_fmt(name: str):
+    global SCALE_FMT
+    SCALE_FMT = SCALE_FMT_NAMES[name]
+
+
+def scale_group() -> int:
+    return 32 if SCALE_FMT == 0 else 16
+
+
+def scale_fmt_name() -> str:
+    return {v: k for k, v in SCALE_FMT_NAMES.items()}[SCALE_FMT]
 
 
 def log(*a):
@@ -73,13 +90,15 @@ class Workload:
         self.n_csa, self.n_hca = n_csa, n_hca
         gen = torch.Generator(device=device)
         gen.manual_seed(SEED + rank)
-        self.csa = csa.Cache.allocate(B, CAP_CSA, D, M_CSA, D_I, csa.CSA_IDX_E4M3, device)
-        self.hca = csa.Cache.allocate(B, CAP_HCA, D, M_HCA, 0, csa.CSA_IDX_BF16, device)
+        self.csa = csa.Cache.allocate(B, CAP_CSA, D, M_CSA, D_I, csa.CSA_IDX_E4M3, device, scale_fmt=SCALE_FMT)
+        self.hca = csa.Cache.allocate(B, CAP_HCA, D, M_HCA, 0, csa.CSA_IDX_BF16, device, scale_fmt=SCALE_FMT)
+        # scale bytes in the range pooled N(0,1) groups land in: E8M0 123..126, E4M3 0x1C..0x2C
+        s_lo, s_hi = (123, 127) if SCALE_FMT == 0 else (0x1C, 0x2D)
         for cache, n in ((self.csa, n_csa), (self.hca, n_hca)):
             for b in range(B):
                 nb = int(n[b])
                 cache.fp4[b, :nb].random_(0, 256, generator=gen)
-                cache.scale[b, :nb].random_(123, 127, generator=gen)
+                cache.scale[b, :nb].random_(s_lo, s_hi, generator=gen)
                 if cache.idx_key is not None:
                     k = torch.randn(nb, D_I, device=device, generator=gen) * 0.5
                     cache.idx_key[b, :nb] = k.to(torch.float8_e4m3fn).view(torch.uint8)
@@ -152,12 +171,12 @@ class Workload:
 
     def bytes_csa_layer(self) -> float:
         """The CSA layer's read/write set at decode: indexer keys, the selected entries, window, q, out."""
-        entry = D // 2 + D // 32
+        entry = D // 2 + D // scale_group()
         sel = float(np.sum(np.minimum(self.n_csa, TOPK))) * entry
         return self.bytes_index() + sel + B * (W * D * 2 + H * D * 2 + H * D * 4)
 
     def bytes_step(self) -> float:
-        entry = D // 2 + D // 32
+        entry = D // 2 + D // scale_group()
         sel = float(np.sum(np.minimum(self.n_csa, TOPK))) * entry
         hca = float(np.sum(self.n_hca)) * entry
         win = 2.0 * B * W * D * 2
@@ -230,8 +249,9 @@ def cpu_baseline(n_requests: int = 2):
     for r in range(n_requests):
         n_csa, n_hca = int(T[r] // M_CSA), int(T[r] // M_HCA)
         keys = datagen.to_e4m3_bytes(datagen.normal_f32((1, n_csa, D_I), 2000 + r, 1, std=0.5))
-        fp4, sc = datagen.random_cache_bytes(n_csa, D, 2000 + r, 2)
-        hfp4, hsc = datagen.random_cache_bytes(n_hca, D, 2000 + r, 3)
+        gen_cache = datagen.random_cache_bytes if SCALE_FMT == 0 else datagen.random_cache_bytes_e4m3x16
+        fp4, sc = gen_cache(n_csa, D, 2000 + r, 2)
+        hfp4, hsc = gen_cache(n_hca, D, 2000 + r, 3)
         kv4 = datagen.normal_bf16((M_CSA, D), 2000 + r, 4)
         idx4 = datagen.normal_bf16((M_CSA, D_I), 2000 + r, 5)
         kv128 = datagen.normal_bf16((M_HCA, D), 2000 + r, 6)
@@ -241,20 +261,21 @@ def cpu_baseline(n_requests: int = 2):
         w = datagen.normal_f32((1, H_I), 2000 + r, 10, std=0.5)
         win = datagen.normal_bf16((W, D), 2000 + r, 11)
         fp4 = fp4.reshape(1, n_csa, D // 2)
-        sc = sc.reshape(1, n_csa, D // 32)
+        sc = sc.reshape(1, n_csa, D // scale_group())
         hfp4 = hfp4.reshape(1, n_hca, D // 2)
-        hsc = hsc.reshape(1, n_hca, D // 32)
+        hsc = hsc.reshape(1, n_hca, D // scale_group())
         qo, qp = np.array([0, 1], np.int32), np.array([T[r] - 1], np.int32)
         ws, wl = np.array([0], np.int64), np.array([W], np.int32)
         t0 = time.perf_counter()
         oracle.compress(kv4, idx4, wg, np.array([0, M_CSA], np.int32), np.array([n_csa - 1], np.int32), m=M_CSA,
-                        cap=n_csa, idx_dtype=1, fp4=fp4, scale=sc, idx_key=keys)
+                        cap=n_csa, idx_dtype=1, scale_fmt=SCALE_FMT, fp4=fp4, scale=sc, idx_key=keys)
         oracle.compress(kv128, None, wg, np.array([0, M_HCA], np.int32), np.array([n_hca - 1], np.int32), m=M_HCA,
-                        cap=n_hca, fp4=hfp4, scale=hsc)
+                        cap=n_hca, scale_fmt=SCALE_FMT, fp4=hfp4, scale=hsc)
         sel, _, _ = oracle.index_topk(keys, np.array([n_csa], np.int32), qo, qp, q_idx, w, m=M_CSA, k=TOPK,
                                       idx_dtype=1)
-        oracle.csa_attend(fp4, sc, qo, q, sel, win, ws, wl, D ** -0.5)
-        oracle.hca_attend(hfp4, hsc, np.array([n_hca], np.int32), qo, qp, q, win, ws, wl, D ** -0.5, m=M_HCA)
+        oracle.csa_attend(fp4, sc, qo, q, sel, win, ws, wl, D ** -0.5, scale_fmt=SCALE_FMT)
+        oracle.hca_attend(hfp4, hsc, np.array([n_hca], np.int32), qo, qp, q, win, ws, wl, D ** -0.5, m=M_HCA,
+                          scale_fmt=SCALE_FMT)
         total += time.perf_counter() - t0
     return n_requests / total, oracle.num_threads(), \
         f"{n_requests} of the {B} requests of one step (contexts {', '.join(str(int(t)) for t in T)} tokens)"
@@ -306,7 +327,8 @@ def run_reference(args):
             "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded)",
             "config": {"workload": "csa_hca_decode_b32_ctx512k-1m", "global_batch": B, "seq_len": CTX_MAX,
-                       "parallelism": "replicas", "l2": "inputs larger than L2 (full key cache streamed)"},
+                       "parallelism": "replicas", "scale_fmt": scale_fmt_name(),
+                       "l2": "inputs larger than L2 (full key cache streamed)"},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -321,8 +343,11 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=B, help="requests per GPU (default 32; smaller only for profiling)")
+    ap.add_argument("--scale-fmt", default="e8m0x32", choices=sorted(SCALE_FMT_NAMES),
+                    help="FP4 scale format of both caches (default: E8M0 per 32 elements, MXFP4)")
     args = ap.parse_args()
     set_batch(args.batch)
+    set_scale_fmt(args.scale_fmt)
     if args.impl == "reference":
         return run_reference(args)
 
@@ -476,6 +501,7 @@ def main():
         "data": "synthetic (seeded torch RNG on device)",
         "config": {"workload": "csa_hca_decode_b32_ctx512k-1m", "global_batch": tokens, "seq_len": CTX_MAX,
                    "parallelism": f"replicas x{world}", "per_gpu_batch": B, "topk": TOPK, "heads": H, "dim": D,
+                   "scale_fmt": scale_fmt_name(),
                    "l2": "flushed between steps (512 MB write) and inputs larger than L2"},
         "hbm_tbs": hbm_tbs,
         "stage_ms": {"compress": float(st_ms[:, 0].mean()), "index_topk": float(st_ms[:, 1].mean()),

@@ -5,7 +5,8 @@ The GPU runs the whole batch; the oracle recomputes sampled queries one by one.
     e4m3 indexer keys, k = 1024, D = 512, 64 heads, 128-token window.
   * hca_b64_1m: 64 requests x 8192 blocks (1M tokens, m = 128), dense.
   * csa_b8_64k: 8 requests x 65536 tokens from raw tokens through every kernel
-    (per-channel LogNormal(0, 0.5) activations), checked stage by stage.
+    (per-channel LogNormal(0, 0.5) activations), checked stage by stage, in both
+    scale formats (E8M0 per 32, E4M3 per 16).
 Cache contents for the first two are seeded bytes (the kernels' inputs), not
 outputs of the compression kernel."""
 import numpy as np
@@ -93,7 +94,8 @@ def test_hca_b64_1m_sampled():
         assert err <= parity.ATT_TOL, (b, err)
 
 
-def test_csa_b8_64k_from_tokens():
+@pytest.mark.parametrize("scale_fmt", [oracle.SCALE_E8M0_32, oracle.SCALE_E4M3_16])
+def test_csa_b8_64k_from_tokens(scale_fmt):
     import torch
 
     import fp4_kv_cache_csa_b200 as csa
@@ -105,19 +107,21 @@ def test_csa_b8_64k_from_tokens():
     it = datagen.normal_bf16((B * T, dI), 520, 2, channel_lognormal=wl.channel_lognormal)
     wg = datagen.normal_f32((D,), 520, 3, std=0.02)
     offs = (np.arange(B + 1) * T).astype(np.int32)
-    ref = oracle.compress(kv, it, wg, offs, np.zeros(B, np.int32), m=m, cap=cap, return_pooled=True)
+    ref = oracle.compress(kv, it, wg, offs, np.zeros(B, np.int32), m=m, cap=cap, scale_fmt=scale_fmt,
+                          return_pooled=True)
     # stage 1: pooling + quantization of all 8 x 16384 blocks
-    cache = csa.Cache.allocate(B, cap, D, m, dI, csa.CSA_IDX_BF16)
+    cache = csa.Cache.allocate(B, cap, D, m, dI, csa.CSA_IDX_BF16, scale_fmt=scale_fmt)
     csa.csa_compress_quantize(cache, dev(kv), dev(it), dev(wg), dev(offs))
     assert csa.csa_read_device_status(cache) == 0
     tol = parity.pooling_tolerance(kv, offs, np.zeros(B, np.int64), m, cap)
     parity.check_mxfp4(host(cache.fp4).reshape(B * cap, -1), host(cache.scale).reshape(B * cap, -1),
                        ref["fp4"].reshape(B * cap, -1), ref["scale"].reshape(B * cap, -1),
-                       ref["pooled"].reshape(B * cap, D), tol=tol.reshape(B * cap, D))
+                       ref["pooled"].reshape(B * cap, D), tol=tol.reshape(B * cap, D), scale_fmt=scale_fmt)
     parity.check_keys(host(cache.idx_key).view(np.uint16), ref["idx_key"].view(np.uint16).reshape(B, cap, dI),
                       ref["pooled_idx"], "bf16", tol=parity.pooling_tolerance(it, offs, np.zeros(B, np.int64), m, cap))
     # stage 2: indexer + top-k on the oracle's cache
-    ocache = make_cache(ref["fp4"], ref["scale"], ref["n_blocks"], m, ref["idx_key"].view(np.uint16), 0)
+    ocache = make_cache(ref["fp4"], ref["scale"], ref["n_blocks"], m, ref["idx_key"].view(np.uint16), 0,
+                        scale_fmt=scale_fmt)
     q = datagen.normal_bf16((B, H, D), 521, 1, channel_lognormal=wl.channel_lognormal)
     q_idx = datagen.normal_bf16((B, wl.idx_heads, dI), 521, 2, channel_lognormal=wl.channel_lognormal)
     w = datagen.normal_f32((B, wl.idx_heads), 521, 3, std=0.5)
@@ -132,7 +136,7 @@ def test_csa_b8_64k_from_tokens():
     win = np.concatenate([kv[b * T + T - W:b * T + T] for b in range(B)])
     ws_, wl_ = (np.arange(B) * W).astype(np.int64), np.full(B, W, np.int32)
     out = host(csa.csa_decode_attend(ocache, dev(q), dev(qo), dev(use), dev(win), dev(ws_), dev(wl_)))
-    want, _ = oracle.csa_attend(ref["fp4"], ref["scale"], qo, q, use, win, ws_, wl_, D ** -0.5)
+    want, _ = oracle.csa_attend(ref["fp4"], ref["scale"], qo, q, use, win, ws_, wl_, D ** -0.5, scale_fmt=scale_fmt)
     err, _ = parity.attention_row_error(out, want)
     assert err <= parity.ATT_TOL, err
     assert csa.csa_read_device_status(ocache) == 0
