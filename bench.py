@@ -194,46 +194,99 @@ class Workload:
 
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
-    def __init__(self, index: int):
-        self.index, self.samples, self.proc = index, [], None
+    """SM clock and clock-event reasons of this rank's GPU, read (never set) through NVML every
+    few milliseconds on a host thread, so that even a short timed region has samples; falls back
+    to `nvidia-smi --query-gpu ... -lms 100` where NVML cannot be loaded. The timed region is
+    marked with mark_start() / mark_end() (host time after a device synchronize) and the summary
+    uses the samples inside it."""
+
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4))
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.device_index, self.period = device_index, period_s
+        self.samples = []  # (t, sm_mhz, max_mhz, reasons bitmask)
+        self.t0 = self.t1 = None
+        self._stop = threading.Event()
+        self.source = None
+
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(self.device_index)
+        try:
+            return pynvml, pynvml.nvmlDeviceGetHandleByUUID(f"GPU-{props.uuid}")
+        except Exception:
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
 
     def start(self):
-        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
-            return
-        self.thread = threading.Thread(target=self._read, daemon=True)
+            nv, h = self._nvml_handle()
+            reasons_fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+            mx = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+
+            def loop():
+                while not self._stop.is_set():
+                    try:
+                        self.samples.append((time.perf_counter(), float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
+                                             mx, int(reasons_fn(h))))
+                    except Exception:
+                        pass
+                    time.sleep(self.period)
+
+            self.source = "nvml"
+        except Exception:
+            q = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+            try:
+                proc = subprocess.Popen(["nvidia-smi", f"--id={self.device_index}", f"--query-gpu={q}",
+                                         "--format=csv,noheader,nounits", "-lms", "100"],
+                                        stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            except OSError:
+                return
+            self.proc = proc
+
+            def loop():
+                for line in proc.stdout:
+                    p = [x.strip() for x in line.split(",")]
+                    if len(p) >= 6 and p[0].replace(".", "").isdigit():
+                        bits = sum(b for (_, b), v in zip(self.REASONS, p[2:6]) if v.lower().startswith("active"))
+                        mx = float(p[1]) if p[1].replace(".", "").isdigit() else 1965.0
+                        self.samples.append((time.perf_counter(), float(p[0]), mx, bits))
+
+            self.source = "nvidia-smi"
+        self.thread = threading.Thread(target=loop, daemon=True)
         self.thread.start()
 
-    def _read(self):
-        for line in self.proc.stdout:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) >= 9:
-                self.samples.append(parts)
+    def mark_start(self):
+        self.t0 = time.perf_counter()
+
+    def mark_end(self):
+        self.t1 = time.perf_counter()
 
     def stop(self):
-        if self.proc:
+        self._stop.set()
+        if getattr(self, "proc", None):
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
+        if getattr(self, "thread", None):
+            self.thread.join(timeout=5)
 
-    def summary(self, max_mhz_default=1965.0):
-        if not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        sm = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
-        mx = [float(s[2]) for s in self.samples if s[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[k] for s in self.samples for k in range(4) if s[5 + k].lower().startswith("active")})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else max_mhz_default,
-                "reasons": reasons, "samples": len(self.samples)}
+    def summary(self):
+        inside = [x for x in self.samples if self.t0 is not None and self.t0 <= x[0] <= self.t1]
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "source": self.source}
+        reasons = sorted({name for x in inside for name, bit in self.REASONS if x[3] & bit})
+        return {"sm_mhz": statistics.median(x[1] for x in inside), "sm_max_mhz": max(x[2] for x in inside),
+                "reasons": reasons, "samples": len(inside), "source": self.source,
+                "window_ms": (self.t1 - self.t0) * 1e3}
 
 
 # ----------------------------------------------------------------------------- oracle baseline
@@ -391,7 +444,7 @@ def main():
         if evs is not None:
             evs[len(graphs)].record(stream)
 
-    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local)
+    clocks = ClockSampler(torch.cuda.current_device())
     clocks.start()
     with torch.cuda.stream(stream):
         for _ in range(max(args.warmup, 3)):
@@ -404,6 +457,7 @@ def main():
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    clocks.mark_start()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(graphs) + 1)] for _ in range(args.steps)]
     with torch.cuda.stream(stream):
         for k in range(args.steps):
@@ -411,6 +465,7 @@ def main():
             replay_step(ev[k])
     stream.synchronize()
     torch.cuda.synchronize()
+    clocks.mark_end()
     if world > 1:
         dist.barrier()
     clocks.stop()
@@ -445,6 +500,20 @@ def main():
     d2h = sum(t.numel() * t.element_size() for t in h_outs[0])
     e2e_n = max(4, min(args.steps, 50))
     up, down = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    # the host link alone: one step's input copies, then one step's output copies (best of 5)
+    link_ms = []
+    for src, dst, st_ in ((h_ins[0], ins, up), (outs, h_outs[0], down)):
+        best = float("inf")
+        for _ in range(5):
+            a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a_.record(st_)
+            with torch.cuda.stream(st_):
+                for s_, d_ in zip(src, dst):
+                    d_.copy_(s_, non_blocking=True)
+            b_.record(st_)
+            b_.synchronize()
+            best = min(best, a_.elapsed_time(b_))
+        link_ms.append(best)
     ready = [torch.cuda.Event() for _ in range(2)]
     computed = [torch.cuda.Event() for _ in range(2)]
     drained = [torch.cuda.Event() for _ in range(2)]
@@ -516,7 +585,8 @@ def main():
                      "traffic": index_traffic(wl.key_bytes()), "traffic_unit": "GB per call (ncu, scaled by keys)"},
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_n,
-                "overlap": "step k+1 inputs in and step k-1 results out while step k computes"},
+                "overlap": "step k+1 inputs in and step k-1 results out while step k computes",
+                "link_h2d_gbs": h2d / (link_ms[0] * 1e-3) / 1e9, "link_d2h_gbs": d2h / (link_ms[1] * 1e-3) / 1e9},
         "gpu_launches": OUR_KERNELS_PER_STEP * args.steps,
         "clocks": clocks.summary(),
         "device_status": status,

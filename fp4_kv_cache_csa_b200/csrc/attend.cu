@@ -133,6 +133,10 @@ __device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity) {
     }
 }
 
+__device__ __forceinline__ void mbar_arrive(uint32_t mbar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(mbar) : "memory");
+}
+
 __device__ __forceinline__ void mbar_expect_tx(uint32_t mbar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mbar), "r"(bytes) : "memory");
 }
@@ -145,6 +149,17 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
                  : "memory");
 }
 
+// Bulk copy of `bytes` from this CTA's shared memory to global memory (one
+// bulk-async group per call); bulk_wait_read() returns once every issued
+// group has finished reading shared memory, bulk_wait_all() once it has
+// also written global memory.
+__device__ __forceinline__ void bulk_s2g(void *dst, uint32_t src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;\n\t"
+                 "cp.async.bulk.commit_group;" ::"l"(dst), "r"(src), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 #define CSA_LD16(base, r)                                                                                    \
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];" \
@@ -335,24 +350,29 @@ __device__ __forceinline__ uint32_t e_chunk_off(int j, int kc) {
     return (uint32_t)((kc >> 3) * Cfg<D>::KREG + (j >> 3) * 1024 + (j & 7) * 128 + (((kc & 7) ^ (j & 7)) << 4));
 }
 
-// Dequantize this thread's half of its prefetched row into E' (fp16).
-// E8M0 scales: E'_j = e_j * 2^-R_j, returns R_j (the row's largest E8M0
-// exponent). E4M3 scales: every E2M1 x E4M3 product is exact in fp16 (at most
-// 6 significant bits, magnitudes 2^-10 .. 2688), so E' = e and R_j = 0.
+// Dequantize one quarter of this thread's prefetched row into E' (fp16): the
+// first (part 0) or second (part 1) half of its channel half. Part 0 of all
+// threads covers channels [0, D/4) and [D/2, 3D/4) -- the "low" channel set,
+// which the S and PV products of a tile consume first; part 1 the rest.
+// E8M0 scales: E'_j = e_j * 2^-R_j, and part 0 returns R_j (the row's largest
+// E8M0 exponent). E4M3 scales: every E2M1 x E4M3 product is exact in fp16 (at
+// most 6 significant bits, magnitudes 2^-10 .. 2688), so E' = e and R_j = 0.
 // Invalid rows are zero.
 template <int D, int SF>
-__device__ __forceinline__ int dequant_row(const RowRegs<D> &rr, uint8_t *E) {
+__device__ __forceinline__ int dequant_part(const RowRegs<D> &rr, uint8_t *E, int part) {
+    constexpr int GQ = Cfg<D>::GPR / 4;                     // 32-element groups per quarter row
     const int j = threadIdx.x & (kTile - 1);
     const int g0 = (threadIdx.x >> 7) * (Cfg<D>::GPR / 2);  // first 32-element group of this half
     if (!rr.valid) {
-#pragma unroll 4
-        for (int kc = 4 * g0; kc < 4 * g0 + D / 16; ++kc)
+#pragma unroll
+        for (int kc = 4 * (g0 + part * GQ); kc < 4 * (g0 + part * GQ + GQ); ++kc)
             *reinterpret_cast<uint4 *>(E + e_chunk_off<D>(j, kc)) = make_uint4(0, 0, 0, 0);
         return 0;
     }
     if constexpr (SF == kScaleE4M3x16) {
 #pragma unroll
-        for (int gl = 0; gl < Cfg<D>::GPR / 2; ++gl) {
+        for (int gq = 0; gq < GQ; ++gq) {
+            const int gl = part * GQ + gq;
             const int g = g0 + gl;
             const uint32_t *w = reinterpret_cast<const uint32_t *>(&rr.code[gl]);
             // code bytes 0..7 of this uint4 are 16-element group 2 gl of the half, 8..15 group 2 gl + 1
@@ -383,7 +403,8 @@ __device__ __forceinline__ int dequant_row(const RowRegs<D> &rr, uint8_t *E) {
 #pragma unroll
         for (int g = 0; g < Cfg<D>::GPR; ++g) rmax = max(rmax, scale_byte<D>(rr, g));
 #pragma unroll
-        for (int gl = 0; gl < Cfg<D>::GPR / 2; ++gl) {
+        for (int gq = 0; gq < GQ; ++gq) {
+            const int gl = part * GQ + gq;
             const int g = g0 + gl;
             const int k = scale_byte<D>(rr, g) - rmax;  // <= 0
             // 2^k in fp16: normal for k >= -14, subnormal down to -24, else 0
@@ -406,6 +427,16 @@ __device__ __forceinline__ int dequant_row(const RowRegs<D> &rr, uint8_t *E) {
         }
         return rmax - 127;
     }
+}
+
+// Whether K-chunk kk (channels 16 kk .. 16 kk + 15) / O^T d-tile dt lies in the low channel set.
+template <int D>
+__host__ __device__ constexpr bool low_chunk(int kk) {
+    return ((16 * kk) % (D / 2)) < D / 4;
+}
+template <int D>
+__host__ __device__ constexpr bool low_dtile(int dt) {
+    return D == 128 || ((128 * dt) % (D / 2)) < D / 4;
 }
 
 // Window tile: cp.async this thread's half of the bf16 row into E' and convert
@@ -687,10 +718,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
     uint8_t *Q = E + C::E_BYTES;
     uint8_t *P = Q + C::Q_BYTES;
     uint8_t *misc = P + C::P_BYTES;
-    uint64_t *mbar = reinterpret_cast<uint64_t *>(misc);            // [0] S done, [1] PV low half, [2] PV high half, [3] Q' loaded
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + 32);
-    int *flags = reinterpret_cast<int *>(misc + 48);                // [0] rescale, [1] abort
-    float *rho = reinterpret_cast<float *>(misc + 64);              // [64]
+    // [0] S done, [1] PV of the low channel set done, [2] PV all done, [3] Q' loaded,
+    // [4] / [5] low / high channel set of E' written (256 arrivals each)
+    uint64_t *mbar = reinterpret_cast<uint64_t *>(misc);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + 64);
+    int *flags = reinterpret_cast<int *>(misc + 80);                // [0] rescale, [1] abort
+    float *rho = reinterpret_cast<float *>(misc + 128);             // [64]
     float *alpha = rho + 64;                                        // [64]
     float *wred = alpha + 64;                                       // [4][64]
     float *xmax = wred + 4 * 64;                                    // [256]
@@ -706,12 +739,14 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
     const uint32_t E_s = smem_u32(E), Q_s = smem_u32(Q), P_s = smem_u32(P);
     const uint32_t mbar_s = smem_u32(&mbar[0]), mbar_lo = smem_u32(&mbar[1]), mbar_hi = smem_u32(&mbar[2]);
     const uint32_t mbar_q = smem_u32(&mbar[3]);
-    const uint32_t mbar_own = hf ? mbar_hi : mbar_lo;
+    const uint32_t mbar_elo = smem_u32(&mbar[4]), mbar_ehi = smem_u32(&mbar[5]);
     if (tid == 0) {
         mbar_init(mbar_s, 1);
         mbar_init(mbar_lo, 1);
         mbar_init(mbar_hi, 1);
         mbar_init(mbar_q, 1);
+        mbar_init(mbar_elo, kThreads);
+        mbar_init(mbar_ehi, kThreads);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         flags[0] = 0;
         flags[1] = 0;
@@ -731,7 +766,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     const uint32_t tmem_s = tmem + lane_off + 32 * hf;               // S^T, this thread's 32 heads
     const uint32_t tmem_o = tmem + lane_off + kHeads + 32 * hf;      // O^T d-tile dt at + 64 dt
-    uint32_t ph_s = 0;
+    uint32_t ph_s = 0, ph_e = 0;
     uint32_t n_pv = 0;          // PV groups committed so far (each completes both halves' barriers once)
     bool pv_pending = false;
 
@@ -771,6 +806,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
             if (__syncthreads_or(!ok)) { aborted = true; break; }
         }
         const int sQ = a.sq[i];
+        // the previous segment's output copy has read the E' buffer
+        if (tid == 0 && seg_begin != t_begin) bulk_wait_read();
         // Q' of this query (issued at kernel start or in the previous segment's epilogue)
         if (__syncthreads_or(!mbar_wait(mbar_q, n_q & 1))) { aborted = true; break; }
         ++n_q;
@@ -780,20 +817,43 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
         bool first = true;
 
         for (; t < seg_end; ++t) {
-            // ---- operand E' for this tile (each half waits for its own channels) ----
+            // ---- operand E' for this tile, low channel set first: its S MMAs run
+            // while the high set is converted. Each set waits for the previous
+            // tile's PV MMAs that read those channels.
             bool ok = true;
-            if (pv_pending) {
-                ok = mbar_wait(mbar_own, (n_pv - 1) & 1);
-                pv_pending = false;
-            }
             int Rj;
             bool valid;
+            if (pv_pending) ok = mbar_wait(mbar_lo, (n_pv - 1) & 1);
             if (cur.win) {
+                if (pv_pending) ok = mbar_wait(mbar_hi, (n_pv - 1) & 1) && ok;
                 Rj = load_window_row<D>(a, cur, E, E_s, xmax, valid);
             } else {
                 valid = rr.valid;
-                Rj = dequant_row<D, SF>(rr, E);
+                Rj = dequant_part<D, SF>(rr, E, 0);
             }
+            fence_async_smem();
+            tc_fence_before();
+            mbar_arrive(mbar_elo);
+            if (warp == 0) {  // S^T = E' Q'^T over the low channel set
+                ok = mbar_wait(mbar_elo, ph_e) && ok;
+                tc_fence_after();
+                if (lane == 0 && ok) {
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        if (!low_chunk<D>(kk)) continue;
+                        const uint32_t koff = (uint32_t)((kk & 3) * 32);
+                        const uint64_t da = desc_sw128(E_s + (kk >> 2) * C::KREG + koff, 16, 1024);
+                        const uint64_t db = desc_sw128(Q_s + (kk >> 2) * C::QREG + koff, 16, 1024);
+                        mma_f16(tmem, da, db, IDESC_S, kk > 0);
+                    }
+                }
+                __syncwarp();
+            }
+            if (!cur.win) {
+                if (pv_pending) ok = mbar_wait(mbar_hi, (n_pv - 1) & 1) && ok;
+                dequant_part<D, SF>(rr, E, 1);
+            }
+            pv_pending = false;
             // next tile (possibly of the next query): start its row loads now,
             // and the selected index of the tile after it
             TileRef nxt2 = nxt;
@@ -807,20 +867,27 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
             }
             fence_async_smem();
             tc_fence_before();
-            if (__syncthreads_or(!ok)) { aborted = true; break; }
-
-            // ---- S^T = E' Q'^T ----
-            if (tid == 0) {
+            mbar_arrive(mbar_ehi);
+            if (warp == 0) {  // ... and the high set
+                ok = mbar_wait(mbar_ehi, ph_e) && ok;
                 tc_fence_after();
+                if (lane == 0 && ok) {
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t koff = (uint32_t)((kk & 3) * 32);
-                    const uint64_t da = desc_sw128(E_s + (kk >> 2) * C::KREG + koff, 16, 1024);
-                    const uint64_t db = desc_sw128(Q_s + (kk >> 2) * C::QREG + koff, 16, 1024);
-                    mma_f16(tmem, da, db, IDESC_S, kk > 0);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        if (low_chunk<D>(kk)) continue;
+                        const uint32_t koff = (uint32_t)((kk & 3) * 32);
+                        const uint64_t da = desc_sw128(E_s + (kk >> 2) * C::KREG + koff, 16, 1024);
+                        const uint64_t db = desc_sw128(Q_s + (kk >> 2) * C::QREG + koff, 16, 1024);
+                        mma_f16(tmem, da, db, IDESC_S, 1u);
+                    }
+                    mma_commit(mbar_s);
                 }
-                mma_commit(mbar_s);
+                __syncwarp();
             }
+            ph_e ^= 1;
+            // a failed wait anywhere leaves S uncommitted: every thread's S wait then runs
+            // out and the vote below aborts the CTA
+            if (!ok) flags[1] = 1;
             if (!mbar_wait(mbar_s, ph_s)) flags[1] = 1;
             ph_s ^= 1;
             tc_fence_after();
@@ -912,17 +979,19 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
                 flags[0] = 0;
                 tc_fence_after();
 #pragma unroll
-                for (int dt = 0; dt < C::DT; ++dt) {
+                for (int pass = 0; pass < 2; ++pass) {  // low channel set, then the high one
 #pragma unroll
-                    for (int kj = 0; kj < kTile / 16; ++kj) {
-                        const uint64_t da = desc_sw128(E_s + (2 * dt) * C::KREG + kj * 2048, C::KREG, 1024);
-                        const uint64_t db = desc_sw128(P_s + kj * 2048, 8192, 1024);
-                        mma_f16(tmem + kHeads + 64 * dt, da, db, IDESC_PV, (first && kj == 0) ? 0u : 1u);
+                    for (int dt = 0; dt < C::DT; ++dt) {
+                        if (low_dtile<D>(dt) != (pass == 0)) continue;
+#pragma unroll
+                        for (int kj = 0; kj < kTile / 16; ++kj) {
+                            const uint64_t da = desc_sw128(E_s + (2 * dt) * C::KREG + kj * 2048, C::KREG, 1024);
+                            const uint64_t db = desc_sw128(P_s + kj * 2048, 8192, 1024);
+                            mma_f16(tmem + kHeads + 64 * dt, da, db, IDESC_PV, (first && kj == 0) ? 0u : 1u);
+                        }
                     }
-                    if (dt == C::DT / 2 - 1) mma_commit(mbar_lo);  // channels of the low half done
+                    mma_commit(pass == 0 ? mbar_lo : mbar_hi);
                 }
-                if (C::DT == 1) mma_commit(mbar_lo);
-                mma_commit(mbar_hi);
             }
             ++n_pv;
             pv_pending = true;
@@ -957,6 +1026,14 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
         __syncthreads();
         const int b_slot = 2 * c + ((seg_begin == T * c / G) ? 0 : 1);
         float *dst = whole ? a.out + (size_t)i * a.H * D : a.part_o + (size_t)b_slot * kHeads * D;
+        // O^T (or O / l for a whole query) -> the E' buffer as [head][channel] fp32
+        // (64 x D x 4 bytes = the buffer's size), then one bulk copy of the H used rows
+        if (whole && tid < 64) {
+            const float l = alpha[tid];
+            xmax[tid] = l > 0.f ? 1.0f / l : 0.f;
+        }
+        __syncthreads();
+        float *ostage = reinterpret_cast<float *>(E);
         for (int dt = 0; dt < C::DT; ++dt) {
             float o[32];
             tmem_ld32(tmem_o + 64 * dt, o);
@@ -964,16 +1041,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
 #pragma unroll
             for (int k = 0; k < 32; ++k) {
                 const int h = 32 * hf + k;
-                if (h < a.H) {
-                    float v = o[k];
-                    if (whole) {
-                        const float l = alpha[h];
-                        v = l > 0.f ? v / l : 0.f;
-                    }
-                    dst[(size_t)h * D + d] = v;
-                }
+                ostage[h * D + d] = whole ? o[k] * xmax[h] : o[k];
             }
         }
+        fence_async_smem();
+        __syncthreads();
+        if (tid == 0) bulk_s2g(dst, E_s, (uint32_t)(a.H * D * 4));
         if (whole) {
             if (a.lse && tid < a.H) {
                 const float l = alpha[tid];
@@ -992,6 +1065,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
         if (tid == 0) flag(a.status, CSA_DEV_TIMEOUT);
         if (n_q_issued > n_q) mbar_wait(mbar_q, n_q & 1);  // no copy may land after the CTA exits
     }
+    if (tid == 0) bulk_wait_all();  // output copies complete before the CTA's shared memory goes away
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
