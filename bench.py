@@ -195,82 +195,95 @@ class Workload:
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
     """SM clock and clock-event reasons of this rank's GPU, read (never set) through NVML every
-    few milliseconds on a host thread, so that even a short timed region has samples; falls back
-    to `nvidia-smi --query-gpu ... -lms 100` where NVML cannot be loaded. The timed region is
-    marked with mark_start() / mark_end() (host time after a device synchronize) and the summary
-    uses the samples inside it."""
+    2 ms by a separate sampler process (a thread of this process would wait for the
+    interpreter lock while the timed loop runs), so that even a short timed region has samples;
+    falls back to `nvidia-smi --query-gpu ... -lms 100`. The timed region is marked with
+    mark_start() / mark_end() (CLOCK_MONOTONIC after a device synchronize) and the summary uses
+    the samples inside it."""
 
     REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
                ("sw_power_cap", 0x4))
+    SCRIPT = r"""
+import sys, time
+import pynvml
+pynvml.nvmlInit()
+uuid, pci, period = sys.argv[1], sys.argv[2], float(sys.argv[3])
+try:
+    h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+except Exception:
+    h = pynvml.nvmlDeviceGetHandleByPciBusId(pci)
+reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+    pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+print("ready", flush=True)
+while True:
+    t = time.monotonic()
+    print(t, pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM), mx, int(reasons(h)), flush=True)
+    time.sleep(period)
+"""
 
-    def __init__(self, device_index: int, period_s: float = 0.005):
+    def __init__(self, device_index: int, period_s: float = 0.002):
         self.device_index, self.period = device_index, period_s
         self.samples = []  # (t, sm_mhz, max_mhz, reasons bitmask)
         self.t0 = self.t1 = None
-        self._stop = threading.Event()
+        self.proc = None
         self.source = None
 
-    def _nvml_handle(self):
-        import pynvml
+    def start(self):
         import torch
 
-        pynvml.nvmlInit()
         props = torch.cuda.get_device_properties(self.device_index)
+        uuid = f"GPU-{props.uuid}"
+        pci = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
         try:
-            return pynvml, pynvml.nvmlDeviceGetHandleByUUID(f"GPU-{props.uuid}")
-        except Exception:
-            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
-            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
-
-    def start(self):
-        try:
-            nv, h = self._nvml_handle()
-            reasons_fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
-                nv.nvmlDeviceGetCurrentClocksThrottleReasons
-            mx = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
-
-            def loop():
-                while not self._stop.is_set():
-                    try:
-                        self.samples.append((time.perf_counter(), float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
-                                             mx, int(reasons_fn(h))))
-                    except Exception:
-                        pass
-                    time.sleep(self.period)
-
+            self.proc = subprocess.Popen([sys.executable, "-c", self.SCRIPT, uuid, pci, str(self.period)],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            first = self.proc.stdout.readline()
+            if not first.startswith("ready"):
+                raise OSError("nvml sampler did not start")
             self.source = "nvml"
-        except Exception:
+
+            def parse(line):
+                p = line.split()
+                if len(p) == 4:
+                    self.samples.append((float(p[0]), float(p[1]), float(p[2]), int(p[3])))
+        except OSError:
+            if self.proc:
+                self.proc.kill()
             q = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
             try:
-                proc = subprocess.Popen(["nvidia-smi", f"--id={self.device_index}", f"--query-gpu={q}",
-                                         "--format=csv,noheader,nounits", "-lms", "100"],
-                                        stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                self.proc = subprocess.Popen(["nvidia-smi", f"--id={pci}", f"--query-gpu={q}",
+                                              "--format=csv,noheader,nounits", "-lms", "100"],
+                                             stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             except OSError:
+                self.proc = None
                 return
-            self.proc = proc
-
-            def loop():
-                for line in proc.stdout:
-                    p = [x.strip() for x in line.split(",")]
-                    if len(p) >= 6 and p[0].replace(".", "").isdigit():
-                        bits = sum(b for (_, b), v in zip(self.REASONS, p[2:6]) if v.lower().startswith("active"))
-                        mx = float(p[1]) if p[1].replace(".", "").isdigit() else 1965.0
-                        self.samples.append((time.perf_counter(), float(p[0]), mx, bits))
-
             self.source = "nvidia-smi"
+
+            def parse(line):
+                p = [x.strip() for x in line.split(",")]
+                if len(p) >= 6 and p[0].replace(".", "").isdigit():
+                    bits = sum(b for (_, b), v in zip(self.REASONS, p[2:6]) if v.lower().startswith("active"))
+                    mx = float(p[1]) if p[1].replace(".", "").isdigit() else 1965.0
+                    self.samples.append((time.monotonic(), float(p[0]), mx, bits))
+
+        def loop():
+            for line in self.proc.stdout:
+                parse(line)
+
         self.thread = threading.Thread(target=loop, daemon=True)
         self.thread.start()
 
     def mark_start(self):
-        self.t0 = time.perf_counter()
+        self.t0 = time.monotonic()
 
     def mark_end(self):
-        self.t1 = time.perf_counter()
+        self.t1 = time.monotonic()
 
     def stop(self):
-        self._stop.set()
-        if getattr(self, "proc", None):
+        if self.proc:
+            time.sleep(3 * self.period)  # the sampler's reading of the region's end
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)

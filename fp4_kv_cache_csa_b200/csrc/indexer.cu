@@ -218,6 +218,29 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// L2 eviction policies: the key stream is read once and should leave the L2
+// first; the score rows are read again by the selection kernels and should stay.
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint4 ld_stream(const uint4 *p, uint64_t pol) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p), "l"(pol));
+    return v;
+}
+__device__ __forceinline__ void st_keep(float *p, float v, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(p), "f"(v), "l"(pol) : "memory");
+}
+
 // Two E4M3 bytes (low byte first) -> packed f16x2 (exact: E4M3 is a subset of f16).
 __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_bytes) {
     __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two_bytes & 0xFFFFu), __NV_E4M3);
@@ -264,6 +287,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a) {
     __shared__ int last_flag;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
+    const uint64_t pol_stream = policy_evict_first(), pol_keep = policy_evict_last();
     const long long NG = a.gprefix[a.Nq];
     long long gb = NG * blockIdx.x / gridDim.x;
     const long long ge = NG * (blockIdx.x + 1) / gridDim.x;
@@ -365,7 +389,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a) {
                     const bool ok = gv && r < n;
                     const uint4 *src = reinterpret_cast<const uint4 *>(kbase + r * C::KEY_BYTES + t * C::ROW_BYTES_T);
 #pragma unroll
-                    for (int v = 0; v < C::NV; ++v) raw[uu][half][v] = ok ? __ldg(src + v) : make_uint4(0, 0, 0, 0);
+                    for (int v = 0; v < C::NV; ++v) raw[uu][half][v] = ok ? ld_stream(src + v, pol_stream) : make_uint4(0, 0, 0, 0);
                 }
             }
 #pragma unroll
@@ -403,7 +427,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a) {
                     const long long r = 16 * lg + g + 8 * t;
                     const float sc = t == 0 ? p0 : p1;
                     if (r < n) {
-                        srow[r] = sc;
+                        st_keep(srow + r, sc, pol_keep);
                         atomicAdd(&hist[ordered_key(sc) >> 20], 1u);
                     }
                 }
