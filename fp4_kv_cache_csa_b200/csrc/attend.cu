@@ -491,11 +491,12 @@ __device__ __forceinline__ int load_window_row(const AttArgs &a, const TileRef &
 }
 
 // ---------------------------------------------------------------- schedule
-// One CTA of 1024 threads per query. Every CTA: its query's scale exponent sq[i] (from
+// One CTA of 1024 threads per query: its query's scale exponent sq[i] (from
 // max|q|), the Q' image (q * 2^-sq in fp16, in the swizzled K-major layout
 // the MMA reads, heads >= H zero) and, when the query has no entry at all,
-// out = 0 and lse = -inf. CTA 0 also writes the per-query records, the tile
-// prefix and the first query of every attention CTA's range.
+// out = 0 and lse = -inf. One more CTA, in parallel with those, writes the
+// per-query records, the tile prefix and the first query of every attention
+// CTA's range.
 __device__ __forceinline__ void query_tiles(const int32_t *q_offsets, const int32_t *q_pos, const int32_t *n_blocks,
                                             const int32_t *win_len, int batch, int m, int cap, int topk, int max_win,
                                             int i, int32_t *status, int &b_out, int &ne, int &ct, int &wl) {
@@ -523,8 +524,8 @@ __global__ void __launch_bounds__(1024) attend_schedule_kernel(
     __shared__ int sq_s;
     grid_dep_launch();  // the attention kernel may start its prologue; it waits for this grid's results
     const int qi = blockIdx.x;
-    // ---- this CTA's query: scale exponent, Q' image and the empty case
-    {
+    // ---- CTAs 0 .. Nq-1: one query each: scale exponent, Q' image and the empty case
+    if (qi < Nq) {
         // the query is read once: chunk c = 8 channels (h = c / (D/8), kc = c % (D/8)), kept in registers
         constexpr int kPer = (kHeads * (D / 8) + 1023) / 1024;
         const __nv_bfloat16 *qp = q + (size_t)qi * H * D;
@@ -581,8 +582,9 @@ __global__ void __launch_bounds__(1024) attend_schedule_kernel(
                 for (int k = threadIdx.x; k < H; k += blockDim.x) lse[(size_t)qi * H + k] = -INFINITY;
         }
     }
-    if (blockIdx.x != 0) return;
-    // ---- CTA 0: per-query records, tile prefix, first query of every CTA range
+    if (qi != Nq) return;
+    // ---- CTA Nq (in parallel with the others): per-query records, tile prefix,
+    // first query of every CTA range
     long long carry = 0;
     for (int base = 0; base < Nq; base += blockDim.x) {
         const int i = base + threadIdx.x;
@@ -1097,7 +1099,7 @@ template <int D>
 cudaError_t launch_schedule(const csa_cache &c, const AttArgs &a, const int32_t *q_offsets, const int32_t *q_pos,
                             const int32_t *win_len, int topk, int max_win, const void *q, int num_ctas, QInfo *qinfo,
                             long long *tprefix, int32_t *cta_q, int32_t *sq, uint8_t *qimg, cudaStream_t s) {
-    attend_schedule_kernel<D><<<a.Nq, 1024, 0, s>>>(q_offsets, q_pos, c.n_blocks, win_len, c.batch, a.Nq, c.block,
+    attend_schedule_kernel<D><<<a.Nq + 1, 1024, 0, s>>>(q_offsets, q_pos, c.n_blocks, win_len, c.batch, a.Nq, c.block,
                                                    c.capacity, topk, max_win, static_cast<const __nv_bfloat16 *>(q),
                                                    a.H, num_ctas, qinfo, tprefix, cta_q, sq, qimg, a.out, a.lse,
                                                    c.status);
