@@ -200,18 +200,19 @@ pool_quantize_kernel(CompressArgs a) {
     if (!active) return;
 
     if constexpr (WPB > 1) {
-        // combine the warps' partial softmax states; warp 0 finishes the block
+        // combine the warps' partial softmax states; warp 0 finishes the block.
+        // Channel k of lane l sits at [k][l]: consecutive lanes hit consecutive banks.
         __shared__ float s_mu[WPB], s_den[WPB];
-        __shared__ float s_acc[WPB][32 * E];
-        __shared__ float s_acck[WPB][32 * EK];
+        __shared__ float s_acc[WPB][E][32];
+        __shared__ float s_acck[WPB][EK][32];
         if (lane == 0) {
             s_mu[warp] = mu;
             s_den[warp] = den;
         }
 #pragma unroll
-        for (int k = 0; k < E; ++k) s_acc[warp][lane * E + k] = acc[k];
+        for (int k = 0; k < E; ++k) s_acc[warp][k][lane] = acc[k];
 #pragma unroll
-        for (int k = 0; k < EK; ++k) s_acck[warp][lane * EK + k] = acck[k];
+        for (int k = 0; k < EK; ++k) s_acck[warp][k][lane] = acck[k];
         __syncthreads();
         if (warp != 0) return;
         float M = -INFINITY;
@@ -227,9 +228,9 @@ pool_quantize_kernel(CompressArgs a) {
             const float f = (s_mu[w] == -INFINITY) ? 0.f : expf(s_mu[w] - M);
             den = fmaf(s_den[w], f, den);
 #pragma unroll
-            for (int k = 0; k < E; ++k) acc[k] = fmaf(s_acc[w][lane * E + k], f, acc[k]);
+            for (int k = 0; k < E; ++k) acc[k] = fmaf(s_acc[w][k][lane], f, acc[k]);
 #pragma unroll
-            for (int k = 0; k < EK; ++k) acck[k] = fmaf(s_acck[w][lane * EK + k], f, acck[k]);
+            for (int k = 0; k < EK; ++k) acck[k] = fmaf(s_acck[w][k][lane], f, acck[k]);
         }
     }
 
