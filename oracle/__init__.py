@@ -78,6 +78,10 @@ def _load():
         lib.orc_index_scores.restype = None
         lib.orc_topk.argtypes = [I, I, I, P, P, P]
         lib.orc_topk.restype = None
+        lib.orc_index_pool.argtypes = [I, I, I, I, P, P, P]
+        lib.orc_index_pool.restype = None
+        lib.orc_reindex_topk.argtypes = [I, I, I, I, I, P, P, P, P]
+        lib.orc_reindex_topk.restype = None
         lib.orc_csa_attend.argtypes = [I, I, I, I, I, I, P, P, I, P, P, P, P, P, P, D, P, P]
         lib.orc_csa_attend.restype = None
         lib.orc_hca_attend.argtypes = [I, I, I, I, I, I, P, P, I, P, P, P, P, P, P, P, D, P, P]
@@ -244,6 +248,26 @@ def topk(scores, n_vis, k):
     Nq, cap = scores.shape
     sel = np.empty((Nq, k), np.int32)
     _load().orc_topk(Nq, cap, k, _ptr(scores), _ptr(_c(n_vis, np.int32)), _ptr(sel))
+    return sel
+
+
+def index_pool(scores, n_vis, *, G, P):
+    """Hierarchical indexer pool: the P best blocks of G entries by block-max score (ascending, -1 padded)."""
+    scores = _c(scores, np.float32)
+    Nq, cap = scores.shape
+    pool = np.empty((Nq, P), np.int32)
+    _load().orc_index_pool(Nq, cap, G, P, _ptr(scores), _ptr(_c(n_vis, np.int32)), _ptr(pool))
+    return pool
+
+
+def reindex_topk(scores, n_vis, pool, *, G, k):
+    """Reindex-mode top-k restricted to the pool's entries (ascending, -1 padded)."""
+    scores = _c(scores, np.float32)
+    Nq, cap = scores.shape
+    pool = _c(pool, np.int32)
+    P = pool.shape[1]
+    sel = np.empty((Nq, k), np.int32)
+    _load().orc_reindex_topk(Nq, cap, G, P, k, _ptr(scores), _ptr(_c(n_vis, np.int32)), _ptr(pool), _ptr(sel))
     return sel
 
 

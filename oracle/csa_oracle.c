@@ -332,6 +332,67 @@ void orc_topk(int Nq, int cap, int k, const float *scores, const int32_t *n_vis,
 }
 
 /* ======================================================================
+ * Hierarchical indexer (DeepSeek-V4.1-Flash podcast transcript, cue 14) and
+ * CSA2 Reindex mode (cue 12)
+ * ====================================================================== */
+
+/* First stage, run with the Full-mode layer's scores: group the visible
+ * entries into blocks of G consecutive entries (block b holds entries
+ * [G b, G b + G) below n_vis), score each block by the largest score of its
+ * entries, and keep the P blocks with the largest block score, ties to the
+ * lower block index; pool_blk[i] lists them ascending, padded with -1. */
+void orc_index_pool(int Nq, int cap, int G, int P, const float *scores, const int32_t *n_vis, int32_t *pool_blk) {
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int i = 0; i < Nq; ++i) {
+        int n = n_vis[i];
+        int nb = (n + G - 1) / G;
+        scored_t *list = malloc(sizeof(scored_t) * (nb > 0 ? nb : 1));
+        for (int b = 0; b < nb; ++b) {
+            float best = -INFINITY;
+            for (int j = G * b; j < G * b + G && j < n; ++j) best = fmaxf(best, scores[(size_t)i * cap + j]);
+            list[b].s = best;
+            list[b].j = b;
+        }
+        qsort(list, nb, sizeof(scored_t), by_score_then_index);
+        int take = nb < P ? nb : P;
+        int32_t *row = pool_blk + (size_t)i * P;
+        for (int r = 0; r < take; ++r) row[r] = list[r].j;
+        qsort(row, take, sizeof(int32_t), ascending_int);
+        for (int r = take; r < P; ++r) row[r] = -1;
+        free(list);
+    }
+}
+
+/* Reindex-mode selection: the layer's own scores, restricted to the visible
+ * entries of query i's pool blocks; the min(k, |pool entries|) largest, ties
+ * to the lower entry index, ascending, padded with -1. */
+void orc_reindex_topk(int Nq, int cap, int G, int P, int k, const float *scores, const int32_t *n_vis,
+                      const int32_t *pool_blk, int32_t *sel_idx) {
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int i = 0; i < Nq; ++i) {
+        int n = n_vis[i];
+        scored_t *list = malloc(sizeof(scored_t) * ((size_t)G * P + 1));
+        int cnt = 0;
+        for (int r = 0; r < P; ++r) {
+            int b = pool_blk[(size_t)i * P + r];
+            if (b < 0) continue;
+            for (int j = G * b; j < G * b + G && j < n; ++j) {
+                list[cnt].s = scores[(size_t)i * cap + j];
+                list[cnt].j = j;
+                ++cnt;
+            }
+        }
+        qsort(list, cnt, sizeof(scored_t), by_score_then_index);
+        int take = cnt < k ? cnt : k;
+        int32_t *row = sel_idx + (size_t)i * k;
+        for (int r = 0; r < take; ++r) row[r] = list[r].j;
+        qsort(row, take, sizeof(int32_t), ascending_int);
+        for (int r = take; r < k; ++r) row[r] = -1;
+        free(list);
+    }
+}
+
+/* ======================================================================
  * a5 + a6 (+ a7): one joint softmax over compressed entries and window rows
  * ====================================================================== */
 

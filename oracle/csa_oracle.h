@@ -91,6 +91,17 @@ void orc_index_scores(int B, int Nq, int H_I, int dI, int idx_dtype, int m, int 
 void orc_topk(int Nq, int cap, int k, const float *scores, const int32_t *n_vis,
               int32_t *sel_idx);
 
+/* ---- hierarchical indexer pool and CSA2 Reindex selection -------------- */
+/* Pool (Full-mode layer): blocks of G consecutive visible entries scored by
+ * their largest score; the P best blocks (ties to the lower block index),
+ * ascending, -1 padded, into pool_blk [Nq][P]. */
+void orc_index_pool(int Nq, int cap, int G, int P, const float *scores, const int32_t *n_vis, int32_t *pool_blk);
+/* Reindex: top-k (ties to the lower entry index) among the visible entries of
+ * the pool blocks only, ascending, -1 padded, into sel_idx [Nq][k]. scores are
+ * the Reindex layer's own scores (row stride cap). */
+void orc_reindex_topk(int Nq, int cap, int G, int P, int k, const float *scores, const int32_t *n_vis,
+                      const int32_t *pool_blk, int32_t *sel_idx);
+
 /* ---- a5+a6: CSA joint attention --------------------------------------- */
 /* For query i and head h, the entries are the dequantized cache blocks listed
  * in sel_idx[i][0..k) (negative entries ignored) followed by the window rows

@@ -383,3 +383,77 @@ def test_e4m3x16_is_finer_than_e8m0x32_on_gaussian_blocks():
                             np.zeros(1, np.int32), m=1, cap=256, scale_fmt=fmt)
         err[fmt] = np.mean((oracle.fp4_dequantize(r["fp4"][0], r["scale"][0], fmt) - tok) ** 2)
     assert err[oracle.SCALE_E4M3_16] < err[oracle.SCALE_E8M0_32]
+
+
+# ---------------------------------------------------------------- hierarchical pool and Reindex
+
+def _read_pool_golden():
+    rows = []
+    with open(os.path.join(GOLDEN, "pool_reindex_tiny.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            parts = [p.split() for p in line.split("|")]
+            rows.append((int(parts[0][0]), np.array(parts[1], np.float32), np.array(parts[2], np.float32),
+                         [int(x) for x in parts[3]], [int(x) for x in parts[4]], [int(x) for x in parts[5]]))
+    return rows
+
+
+def test_pool_and_reindex_golden():
+    for n, full, re, pool_want, k3, k5 in _read_pool_golden():
+        pool = oracle.index_pool(full[None], [n], G=4, P=2)
+        assert list(pool[0]) == pool_want
+        assert list(oracle.reindex_topk(re[None], [n], pool, G=4, k=3)[0]) == k3
+        assert list(oracle.reindex_topk(re[None], [n], pool, G=4, k=5)[0]) == k5
+
+
+def test_pool_brute_force_subsets():
+    # the kept set maximises the sum of block maxima, ties broken towards lower block ids
+    g = np.random.default_rng(50)
+    for trial in range(60):
+        n = int(g.integers(1, 30))
+        G = int(g.choice([1, 2, 3, 4, 8]))
+        P = int(g.integers(1, 6))
+        sc = (g.integers(-3, 4, size=32)).astype(np.float32)  # many ties
+        pool = oracle.index_pool(sc[None], [n], G=G, P=P)[0]
+        nb = (n + G - 1) // G
+        bmax = [max(sc[G * b:min(G * b + G, n)]) for b in range(nb)]
+        take = min(P, nb)
+        best = max(itertools.combinations(range(nb), take),
+                   key=lambda s: (sum(bmax[b] for b in s), tuple(-b for b in s)))
+        assert list(pool[:take]) == list(best)
+        assert all(x == -1 for x in pool[take:])
+
+
+def test_reindex_brute_force_subsets():
+    g = np.random.default_rng(51)
+    for trial in range(60):
+        n, G, P = int(g.integers(1, 24)), int(g.choice([2, 4])), int(g.integers(1, 5))
+        k = int(g.integers(1, 6))
+        full = g.integers(-3, 4, size=24).astype(np.float32)
+        re = g.integers(-3, 4, size=24).astype(np.float32)
+        pool = oracle.index_pool(full[None], [n], G=G, P=P)
+        sel = oracle.reindex_topk(re[None], [n], pool, G=G, k=k)[0]
+        cand = sorted(j for b in pool[0] if b >= 0 for j in range(G * b, min(G * b + G, n)))
+        take = min(k, len(cand))
+        best = max(itertools.combinations(cand, take), key=lambda s: (sum(re[j] for j in s), tuple(-j for j in s)))
+        assert list(sel[:take]) == list(best)
+        assert all(x == -1 for x in sel[take:])
+
+
+def test_reindex_with_the_whole_context_pooled_is_the_full_topk():
+    # when the pool covers every visible entry, Reindex is the plain top-k of its scores
+    g = np.random.default_rng(52)
+    sc = g.standard_normal((3, 200)).astype(np.float32)
+    n_vis = np.array([200, 137, 9], np.int32)
+    pool = oracle.index_pool(g.standard_normal((3, 200)).astype(np.float32), n_vis, G=8, P=25)
+    for k in (1, 16, 64):
+        assert np.array_equal(oracle.reindex_topk(sc, n_vis, pool, G=8, k=k), oracle.topk(sc, n_vis, k))
+
+
+def test_pool_with_single_entry_blocks_is_the_topk():
+    g = np.random.default_rng(53)
+    sc = np.round(g.standard_normal((4, 100)) * 3).astype(np.float32)
+    n_vis = np.array([100, 50, 7, 0], np.int32)
+    assert np.array_equal(oracle.index_pool(sc, n_vis, G=1, P=10), oracle.topk(sc, n_vis, 10))
