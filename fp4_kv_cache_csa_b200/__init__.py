@@ -35,7 +35,8 @@ CSA_DEV_TIMEOUT = 0x10
 EXPORTED = (
     "csa_status_string", "csa_version", "csa_compress_quantize", "csa_index_topk_workspace", "csa_index_topk",
     "csa_attend_workspace", "csa_decode_attend", "hca_decode_attend", "csa_read_device_status",
-    "csa_index_topk_noalloc",
+    "csa_index_topk_noalloc", "csa_index_pool_workspace", "csa_index_topk_pool", "csa_index_reindex_workspace",
+    "csa_index_topk_reindex",
 )
 
 
@@ -77,6 +78,14 @@ def load_library(path: str = LIB_PATH):
     lib.csa_index_topk.restype = I
     lib.csa_index_topk_noalloc.argtypes = [CP, P, P, I, I, P, P, I, P, P]
     lib.csa_index_topk_noalloc.restype = I
+    lib.csa_index_pool_workspace.argtypes = [CP, I, I, I, I]
+    lib.csa_index_pool_workspace.restype = S
+    lib.csa_index_topk_pool.argtypes = [CP, P, P, I, I, P, P, I, P, I, I, P, P, S, P]
+    lib.csa_index_topk_pool.restype = I
+    lib.csa_index_reindex_workspace.argtypes = [CP, I, I, I]
+    lib.csa_index_reindex_workspace.restype = S
+    lib.csa_index_topk_reindex.argtypes = [CP, P, P, I, I, P, P, I, P, I, I, P, P, S, P]
+    lib.csa_index_topk_reindex.restype = I
     lib.csa_attend_workspace.argtypes = [CP, I, I]
     lib.csa_attend_workspace.restype = S
     lib.csa_decode_attend.argtypes = [CP, P, I, I, P, P, I, P, P, P, I, ctypes.c_float, P, P, P, S, P]
@@ -215,6 +224,47 @@ def csa_index_topk(cache: Cache, q_idx, w, q_offsets, q_pos, topk: int, sel_idx=
     _check(lib.csa_index_topk(ctypes.byref(c), _ptr(q_idx), _ptr(w), n_queries, idx_heads, _ptr(q_offsets),
                               _ptr(q_pos), topk, _ptr(sel_idx), _ptr(workspace), workspace.numel(), _stream(stream)),
            "csa_index_topk")
+    return sel_idx
+
+
+def csa_index_topk_pool(cache: Cache, q_idx, w, q_offsets, q_pos, topk: int, pool_group: int = 8,
+                        pool_blocks: int = 2000, sel_idx=None, pool_blk=None, workspace=None, stream=None):
+    """A Full-mode layer's indexer: its top-k (as csa_index_topk) and the candidate pool of the
+    hierarchical indexer (the pool_blocks best groups of pool_group blocks by their best score)."""
+    import torch
+
+    lib = load_library()
+    n_queries, idx_heads = int(q_idx.shape[0]), int(q_idx.shape[1])
+    if sel_idx is None:
+        sel_idx = torch.empty(n_queries, topk, dtype=torch.int32, device=q_idx.device)
+    if pool_blk is None:
+        pool_blk = torch.empty(n_queries, pool_blocks, dtype=torch.int32, device=q_idx.device)
+    need = int(lib.csa_index_pool_workspace(ctypes.byref(cache.c_struct()), n_queries, topk, pool_group,
+                                            pool_blocks))
+    workspace = _workspace(need, workspace, q_idx.device)
+    c = cache.c_struct()
+    _check(lib.csa_index_topk_pool(ctypes.byref(c), _ptr(q_idx), _ptr(w), n_queries, idx_heads, _ptr(q_offsets),
+                                   _ptr(q_pos), topk, _ptr(sel_idx), pool_group, pool_blocks, _ptr(pool_blk),
+                                   _ptr(workspace), workspace.numel(), _stream(stream)), "csa_index_topk_pool")
+    return sel_idx, pool_blk
+
+
+def csa_index_topk_reindex(cache: Cache, q_idx, w, q_offsets, q_pos, topk: int, pool_blk, pool_group: int = 8,
+                           sel_idx=None, workspace=None, stream=None):
+    """A Reindex-mode layer's indexer: its own query scored only against the pool's blocks."""
+    import torch
+
+    lib = load_library()
+    n_queries, idx_heads = int(q_idx.shape[0]), int(q_idx.shape[1])
+    pool_blocks = int(pool_blk.shape[1])
+    if sel_idx is None:
+        sel_idx = torch.empty(n_queries, topk, dtype=torch.int32, device=q_idx.device)
+    need = int(lib.csa_index_reindex_workspace(ctypes.byref(cache.c_struct()), n_queries, pool_group, pool_blocks))
+    workspace = _workspace(need, workspace, q_idx.device)
+    c = cache.c_struct()
+    _check(lib.csa_index_topk_reindex(ctypes.byref(c), _ptr(q_idx), _ptr(w), n_queries, idx_heads, _ptr(q_offsets),
+                                      _ptr(q_pos), topk, _ptr(sel_idx), pool_group, pool_blocks, _ptr(pool_blk),
+                                      _ptr(workspace), workspace.numel(), _stream(stream)), "csa_index_topk_reindex")
     return sel_idx
 
 

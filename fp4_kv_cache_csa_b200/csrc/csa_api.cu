@@ -13,6 +13,16 @@ size_t index_topk_workspace_bytes(int Nq, int cap);
 cudaError_t launch_index_topk(const csa_cache &c, const void *q_idx, const float *w, int Nq, int H_I,
                               const int32_t *q_offsets, const int32_t *q_pos, int topk, int32_t *sel_idx,
                               void *workspace, int num_sms, cudaStream_t s);
+size_t index_pool_workspace_bytes(int Nq, int cap, int G, int P);
+cudaError_t launch_index_topk_pool(const csa_cache &c, const void *q_idx, const float *w, int Nq, int H_I,
+                                   const int32_t *q_offsets, const int32_t *q_pos, int topk, int32_t *sel_idx,
+                                   int pool_shift, int P, int32_t *pool_blk, void *workspace, int num_sms,
+                                   cudaStream_t s);
+size_t index_reindex_workspace_bytes(int Nq, int G, int P);
+cudaError_t launch_index_topk_reindex(const csa_cache &c, const void *q_idx, const float *w, int Nq, int H_I,
+                                      const int32_t *q_offsets, const int32_t *q_pos, int topk, int32_t *sel_idx,
+                                      int pool_shift, int P, const int32_t *pool_blk, void *workspace, int num_sms,
+                                      cudaStream_t s);
 size_t attend_workspace_bytes(int Nq, int D, int num_ctas);
 cudaError_t launch_attend(const csa_cache &c, const void *q, int Nq, int H, const int32_t *q_offsets,
                           const int32_t *q_pos, const int32_t *sel_idx, int topk, const void *win_kv,
@@ -70,7 +80,7 @@ const char *csa_status_string(int32_t status) {
     }
 }
 
-int32_t csa_version(void) { return 101; }
+int32_t csa_version(void) { return 102; }
 
 csa_status csa_compress_quantize(const csa_cache *cache, const void *kv_tok, const void *idx_tok, const float *gate_w,
                                  const int32_t *tok_offsets, int32_t n_tokens, csa_stream_t stream) {
@@ -109,6 +119,88 @@ csa_status csa_index_topk(const csa_cache *cache, const void *q_idx, const float
     if (sms <= 0) return CSA_ERR_CUDA;
     return from_cuda(csa::launch_index_topk(*cache, q_idx, w, n_queries, idx_heads, q_offsets, q_pos, topk, sel_idx,
                                             workspace, sms, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+// log2 of a pool block size (1, 2, 4, ... 32 entries), or -1
+static int pool_shift_of(int32_t g) {
+    for (int k = 0; k <= 5; ++k)
+        if (g == (1 << k)) return k;
+    return -1;
+}
+
+// Checks shared by the pool and Reindex calls.
+static csa_status check_index(const csa_cache *cache, const void *q_idx, const float *w, int32_t n_queries,
+                              int32_t idx_heads, const int32_t *q_offsets, const int32_t *q_pos, int32_t topk,
+                              const int32_t *sel_idx) {
+    csa_status st = check_cache(cache);
+    if (st != CSA_OK) return st;
+    if (!cache->idx_key || !q_idx || !w || !q_offsets || !q_pos || !sel_idx) return CSA_ERR_NULL;
+    if (n_queries < 1 || idx_heads < 1 || topk < 1) return CSA_ERR_SHAPE;
+    if (idx_heads > 8 || topk > kMaxTopk) return CSA_ERR_UNSUPPORTED;
+    if (!aligned(q_idx, 16) || !aligned(w, 4) || !aligned(q_offsets, 4) || !aligned(q_pos, 4) ||
+        !aligned(sel_idx, 4))
+        return CSA_ERR_ALIGN;
+    return CSA_OK;
+}
+
+static bool pool_sizes_ok(int32_t pool_group, int32_t pool_blocks) {
+    return pool_shift_of(pool_group) >= 0 && pool_blocks >= 1 && pool_blocks <= kMaxTopk &&
+           (long long)pool_group * pool_blocks <= kMaxCapacity;
+}
+
+size_t csa_index_pool_workspace(const csa_cache *cache, int32_t n_queries, int32_t topk, int32_t pool_group,
+                                int32_t pool_blocks) {
+    if (!cache || n_queries < 1 || topk < 1 || cache->capacity < 1 || cache->capacity > kMaxCapacity ||
+        !pool_sizes_ok(pool_group, pool_blocks))
+        return 0;
+    return csa::index_pool_workspace_bytes(n_queries, cache->capacity, pool_group, pool_blocks);
+}
+
+csa_status csa_index_topk_pool(const csa_cache *cache, const void *q_idx, const float *w, int32_t n_queries,
+                               int32_t idx_heads, const int32_t *q_offsets, const int32_t *q_pos, int32_t topk,
+                               int32_t *sel_idx, int32_t pool_group, int32_t pool_blocks, int32_t *pool_blk,
+                               void *workspace, size_t workspace_bytes, csa_stream_t stream) {
+    csa_status st = check_index(cache, q_idx, w, n_queries, idx_heads, q_offsets, q_pos, topk, sel_idx);
+    if (st != CSA_OK) return st;
+    if (!pool_blk) return CSA_ERR_NULL;
+    if (pool_shift_of(pool_group) < 0 || pool_blocks < 1) return CSA_ERR_SHAPE;
+    if (!pool_sizes_ok(pool_group, pool_blocks)) return CSA_ERR_UNSUPPORTED;
+    if (!aligned(pool_blk, 4)) return CSA_ERR_ALIGN;
+    const size_t need = csa_index_pool_workspace(cache, n_queries, topk, pool_group, pool_blocks);
+    if (!workspace || workspace_bytes < need) return CSA_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return CSA_ERR_ALIGN;
+    const int sms = num_sms();
+    if (sms <= 0) return CSA_ERR_CUDA;
+    return from_cuda(csa::launch_index_topk_pool(*cache, q_idx, w, n_queries, idx_heads, q_offsets, q_pos, topk,
+                                                 sel_idx, pool_shift_of(pool_group), pool_blocks, pool_blk, workspace,
+                                                 sms, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t csa_index_reindex_workspace(const csa_cache *cache, int32_t n_queries, int32_t pool_group,
+                                   int32_t pool_blocks) {
+    if (!cache || n_queries < 1 || !pool_sizes_ok(pool_group, pool_blocks)) return 0;
+    return csa::index_reindex_workspace_bytes(n_queries, pool_group, pool_blocks);
+}
+
+csa_status csa_index_topk_reindex(const csa_cache *cache, const void *q_idx, const float *w, int32_t n_queries,
+                                  int32_t idx_heads, const int32_t *q_offsets, const int32_t *q_pos, int32_t topk,
+                                  int32_t *sel_idx, int32_t pool_group, int32_t pool_blocks,
+                                  const int32_t *pool_blk, void *workspace, size_t workspace_bytes,
+                                  csa_stream_t stream) {
+    csa_status st = check_index(cache, q_idx, w, n_queries, idx_heads, q_offsets, q_pos, topk, sel_idx);
+    if (st != CSA_OK) return st;
+    if (!pool_blk) return CSA_ERR_NULL;
+    if (pool_shift_of(pool_group) < 0 || pool_blocks < 1) return CSA_ERR_SHAPE;
+    if (!pool_sizes_ok(pool_group, pool_blocks)) return CSA_ERR_UNSUPPORTED;
+    if (!aligned(pool_blk, 4)) return CSA_ERR_ALIGN;
+    const size_t need = csa_index_reindex_workspace(cache, n_queries, pool_group, pool_blocks);
+    if (!workspace || workspace_bytes < need) return CSA_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return CSA_ERR_ALIGN;
+    const int sms = num_sms();
+    if (sms <= 0) return CSA_ERR_CUDA;
+    return from_cuda(csa::launch_index_topk_reindex(*cache, q_idx, w, n_queries, idx_heads, q_offsets, q_pos, topk,
+                                                    sel_idx, pool_shift_of(pool_group), pool_blocks, pool_blk,
+                                                    workspace, sms, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 size_t csa_attend_workspace(const csa_cache *cache, int32_t n_queries, int32_t heads) {

@@ -64,6 +64,9 @@ constexpr int kSegCost = 96;
 constexpr int kSelThreads = 1024;
 constexpr int kPassThreads = 256;
 constexpr int kCandCap = 32768;    // candidate slots per query (members of the threshold bin)
+constexpr int kBmaxThreads = 256;  // pool_bmax_kernel: threads per CTA ...
+constexpr int kBmaxPerThread = 4;  // ... and blocks per thread
+constexpr int kCountThreads = 256; // reindex_count_kernel
 
 // ---------------------------------------------------------------- workspace
 struct IndexWs {
@@ -130,9 +133,11 @@ size_t carve(void *base, int Nq, int cap, IndexWs *w) {
 }
 
 // ---------------------------------------------------------------- schedule
+// n_vis_given (Reindex): per-query key counts computed before (pool positions);
+// otherwise the visible block count from the query position.
 __global__ void schedule_kernel(const int32_t *q_offsets, const int32_t *q_pos, const int32_t *n_blocks,
                                 int batch, int Nq, int m, int cap, int topk, int32_t *req, int32_t *n_vis,
-                                long long *gprefix, int32_t *thresh) {
+                                long long *gprefix, int32_t *thresh, const int32_t *n_vis_given) {
     __shared__ long long red[32];
     __shared__ long long round_total;
     grid_dep_wait();
@@ -143,7 +148,8 @@ __global__ void schedule_kernel(const int32_t *q_offsets, const int32_t *q_pos, 
         long long groups = 0;
         if (i < Nq) {
             const int b = request_of(q_offsets, batch, i);
-            const int n = (b < 0) ? 0 : min(visible_blocks(q_pos[i], m, n_blocks[b]), cap);
+            const int n = n_vis_given ? ((b < 0) ? 0 : n_vis_given[i])
+                                      : ((b < 0) ? 0 : min(visible_blocks(q_pos[i], m, n_blocks[b]), cap));
             req[i] = b;
             n_vis[i] = n;
             groups = (n + 15) / 16;
@@ -258,6 +264,11 @@ struct ScanArgs {
     uint32_t *done;               // [Nq]
     int32_t *thresh;              // [Nq][3]
     int Nq, H_I, cap, topk;
+    int rows;                     // score row stride (cap, or G*P for a pool)
+    // pool mapping (Reindex): local key r of query i is cache block
+    // G * pool[i][r / G] + r % G, G = 1 << pool_shift; null: r itself
+    const int32_t *pool;
+    int pool_shift, pool_p;
 };
 
 // Dimension permutation. The dot product sums over all d_I channels, so the
@@ -375,7 +386,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a) {
         __syncthreads();
 
         const uint8_t *kbase = a.keys + (size_t)b * a.cap * C::KEY_BYTES;
-        float *srow = a.scores + (size_t)i * a.cap;
+        float *srow = a.scores + (size_t)i * a.rows;
+        const int32_t *prow = a.pool ? a.pool + (size_t)i * a.pool_p : nullptr;
 
         for (long long u0 = warp; u0 < nloc; u0 += (long long)kScanWarps * C::U) {
             uint4 raw[C::U][2][C::NV];
@@ -387,7 +399,11 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a) {
                 for (int half = 0; half < 2; ++half) {
                     const long long r = 16 * lg + g + 8 * half;
                     const bool ok = gv && r < n;
-                    const uint4 *src = reinterpret_cast<const uint4 *>(kbase + r * C::KEY_BYTES + t * C::ROW_BYTES_T);
+                    long long row = r;
+                    if (prow && ok)
+                        row = ((long long)__ldg(prow + (r >> a.pool_shift)) << a.pool_shift) +
+                              (r & ((1 << a.pool_shift) - 1));
+                    const uint4 *src = reinterpret_cast<const uint4 *>(kbase + row * C::KEY_BYTES + t * C::ROW_BYTES_T);
 #pragma unroll
                     for (int v = 0; v < C::NV; ++v) raw[uu][half][v] = ok ? ld_stream(src + v, pol_stream) : make_uint4(0, 0, 0, 0);
                 }
@@ -478,7 +494,17 @@ struct SelArgs {
     int32_t *sel_idx;
     int Nq, cap, topk, words, ccap;
     int smem_cands;  // candidates that fit in shared memory after the bitmap
+    // rows are pool positions (Reindex): selected position r is written as
+    // cache block G * pool[i][r / G] + r % G, G = 1 << pool_shift; null: r itself
+    const int32_t *pool;
+    int pool_shift, pool_p;
 };
+
+__device__ __forceinline__ int32_t out_index(const SelArgs &a, int i, int r) {
+    if (!a.pool) return r;
+    return (__ldg(a.pool + (size_t)i * a.pool_p + (r >> a.pool_shift)) << a.pool_shift) +
+           (r & ((1 << a.pool_shift) - 1));
+}
 
 // Keys above the threshold bin -> bitmap; keys in it -> candidate list.
 // Grid: (chunks of 128 x kPassThreads/32 scores, Nq).
@@ -613,7 +639,7 @@ __global__ void __launch_bounds__(kSelThreads) select_final_kernel(SelArgs a) {
     const int K = min(a.topk, n);
     int32_t *out = a.sel_idx + (size_t)i * a.topk;
     if (K == n) {  // select every visible block
-        for (int r = threadIdx.x; r < a.topk; r += blockDim.x) out[r] = r < n ? r : -1;
+        for (int r = threadIdx.x; r < a.topk; r += blockDim.x) out[r] = r < n ? out_index(a, i, r) : -1;
         return;
     }
     const int lane = threadIdx.x & 31;
@@ -758,7 +784,7 @@ __global__ void __launch_bounds__(kSelThreads) select_final_kernel(SelArgs a) {
         while (bits) {
             const int bit = __ffs(bits) - 1;
             bits &= bits - 1;
-            if (pos < (uint32_t)a.topk) out[pos] = w * 32 + bit;
+            if (pos < (uint32_t)a.topk) out[pos] = out_index(a, i, w * 32 + bit);
             ++pos;
         }
     }
@@ -766,24 +792,183 @@ __global__ void __launch_bounds__(kSelThreads) select_final_kernel(SelArgs a) {
     for (int r2 = K + threadIdx.x; r2 < a.topk; r2 += blockDim.x) out[r2] = -1;
 }
 
+// ---------------------------------------------------------------- pool (hierarchical indexer)
+// Block maxima for the pool of the first Full-mode layer: block b of query i
+// holds its visible scores [G b, G b + G) (G = 1 << shift); its score is their
+// maximum. Writes one row of nb = ceil(n_vis / G) block scores per query
+// (stride rows_b) with a 4096-bin histogram of their keys; the CTA that
+// completes a query picks the bin holding the P-th best block (as the scan
+// does for the keys). Grid: (blocks / (threads * per thread), Nq).
+__global__ void __launch_bounds__(kBmaxThreads) pool_bmax_kernel(const float *scores, const int32_t *n_vis, int rows,
+                                                                 int shift, int P, float *bmax, int rows_b,
+                                                                 int32_t *n_vis_b, uint32_t *hist1, uint32_t *done,
+                                                                 int32_t *thresh) {
+    __shared__ uint32_t hist[kBins];
+    __shared__ uint32_t scan_smem[32];
+    __shared__ BinPick pick;
+    __shared__ int last_flag;
+    grid_dep_wait();
+    grid_dep_launch();
+    const int i = blockIdx.y;
+    const int n = n_vis[i];
+    const int G = 1 << shift;
+    const int nb = (n + G - 1) >> shift;
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        n_vis_b[i] = nb;
+        if (P >= nb) {  // every block is kept
+            thresh[3 * i] = -1;
+            thresh[3 * i + 1] = nb;
+            thresh[3 * i + 2] = -1;
+        }
+    }
+    const int b0 = blockIdx.x * kBmaxThreads * kBmaxPerThread;
+    const int b1 = min(nb, b0 + kBmaxThreads * kBmaxPerThread);
+    if (b0 >= b1 || P >= nb) return;
+    for (int k = threadIdx.x; k < kBins; k += kBmaxThreads) hist[k] = 0;
+    __syncthreads();
+    const float *srow = scores + (size_t)i * rows;
+    for (int b = b0 + threadIdx.x; b < b1; b += kBmaxThreads) {
+        const int j0 = b << shift, j1 = min(n, j0 + G);
+        float m = __ldcg(srow + j0);
+        for (int j = j0 + 1; j < j1; ++j) m = fmaxf(m, __ldcg(srow + j));
+        bmax[(size_t)i * rows_b + b] = m;
+        atomicAdd(&hist[ordered_key(m) >> 20], 1u);
+    }
+    __syncthreads();
+    uint32_t *gh = hist1 + (size_t)i * kBins;
+    for (int k = threadIdx.x; k < kBins; k += kBmaxThreads) {
+        const uint32_t cnt = hist[k];
+        if (cnt) atomicAdd(gh + k, cnt);
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const uint32_t mine = (uint32_t)(b1 - b0);
+        last_flag = atomicAdd(done + i, mine) + mine == (uint32_t)nb;
+    }
+    __syncthreads();
+    if (last_flag) {
+        __threadfence();
+        for (int k = threadIdx.x; k < kBins; k += kBmaxThreads) hist[k] = __ldcg(gh + k);
+        __syncthreads();
+        const BinPick p = pick_bin(hist, kBins, (uint32_t)P, scan_smem, &pick);
+        if (threadIdx.x == 0) {
+            const bool all_at = p.above + p.at == (uint32_t)P;
+            thresh[3 * i] = all_at ? p.bin - 1 : p.bin;
+            thresh[3 * i + 1] = (int)p.above;
+            thresh[3 * i + 2] = all_at ? -1 : p.bin;
+        }
+    }
+}
+
+// Reindex: how many positions of query i's pool are visible. The pool lists
+// blocks ascending, -1 padded; positions run block by block, G per block, and
+// the block holding the last visible entry may be partial. A block at or
+// beyond the visible range, or out of ascending order, ends the list there
+// (CSA_DEV_BAD_INDEX). One CTA per query.
+__global__ void __launch_bounds__(kCountThreads) reindex_count_kernel(const int32_t *q_offsets, const int32_t *q_pos,
+                                                                      const int32_t *n_blocks, int batch, int m,
+                                                                      int cap, const int32_t *pool, int P, int shift,
+                                                                      int32_t *n_pos, int32_t *status) {
+    __shared__ int first_bad, first_pad;
+    __shared__ uint32_t total;
+    grid_dep_wait();
+    grid_dep_launch();
+    const int i = blockIdx.x;
+    const int b = request_of(q_offsets, batch, i);
+    const int nv = (b < 0) ? 0 : min(visible_blocks(q_pos[i], m, n_blocks[b]), cap);
+    const int32_t *row = pool + (size_t)i * P;
+    if (threadIdx.x == 0) {
+        first_bad = P;
+        first_pad = P;
+        total = 0;
+    }
+    __syncthreads();
+    for (int r = threadIdx.x; r < P; r += kCountThreads) {
+        const int blk = row[r];
+        if (blk < 0) {
+            atomicMin(&first_pad, r);
+        } else if (((long long)blk << shift) >= nv || (r > 0 && blk <= row[r - 1])) {
+            atomicMin(&first_bad, r);
+        }
+    }
+    __syncthreads();
+    const int end = min(first_bad, first_pad);
+    uint32_t mine = 0;
+    for (int r = threadIdx.x; r < end; r += kCountThreads) mine += (uint32_t)min(1 << shift, nv - (row[r] << shift));
+    mine = __reduce_add_sync(0xffffffffu, mine);
+    if ((threadIdx.x & 31) == 0) atomicAdd(&total, mine);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        n_pos[i] = b < 0 ? 0 : (int)total;
+        if (first_bad < first_pad) flag(status, CSA_DEV_BAD_INDEX);
+    }
+}
+
 template <bool E4M3, int KS>
 cudaError_t launch_scan(const ScanArgs &sa, int grid, cudaStream_t s) {
     return launch_pdl(scan_kernel<E4M3, KS>, dim3(grid), dim3(kScanThreads), 0, s, sa);
+}
+
+// select_pass + select_final over the score rows of ws (row stride `rows`,
+// thresholds from the scan or the block-max kernel), into sel_idx [Nq][topk].
+cudaError_t launch_select(const IndexWs &ws, int Nq, int rows, int topk, int32_t *sel_idx, const int32_t *pool,
+                          int pool_shift, int pool_p, int num_sms, cudaStream_t s) {
+    SelArgs sel;
+    sel.n_vis = ws.n_vis;
+    sel.scores = ws.scores;
+    sel.hist1 = ws.hist1;
+    sel.thresh = ws.thresh;
+    sel.bitmap = ws.bitmap;
+    sel.ncand = ws.ncand;
+    sel.cand_key = ws.cand_key;
+    sel.cand_idx = ws.cand_idx;
+    sel.sel_idx = sel_idx;
+    sel.Nq = Nq;
+    sel.cap = rows;
+    sel.topk = topk;
+    sel.words = ws.words;
+    sel.ccap = ws.ccap;
+    sel.pool = pool;
+    sel.pool_shift = pool_shift;
+    sel.pool_p = pool_p;
+    // enough warps to cover the rows with a few 128-score steps each
+    const int chunks_per_cta = 128 * (kPassThreads / 32);
+    int gx = (rows + chunks_per_cta - 1) / chunks_per_cta;
+    const int want = (16 * num_sms + Nq - 1) / Nq;
+    if (gx > want) gx = want;
+    if (gx < 1) gx = 1;
+    cudaError_t err = launch_pdl(select_pass_kernel, dim3(gx, Nq), dim3(kPassThreads), 0, s, sel);
+    if (err != cudaSuccess) return err;
+    // dynamic shared memory: the bitmap, then as many candidates as fit next to
+    // the ~33 KB of static shared memory (opt in every time: cheap, valid in capture)
+    const int kDynMax = 200 * 1024;
+    sel.smem_cands = (kDynMax - 8 * ws.words) / 8;
+    if (sel.smem_cands < 0) sel.smem_cands = 0;
+    if (sel.smem_cands > ws.ccap) sel.smem_cands = ws.ccap;
+    const int smem = 8 * ws.words + 8 * sel.smem_cands;
+    err = cudaFuncSetAttribute(select_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err != cudaSuccess) return err;
+    return launch_pdl(select_final_kernel, dim3(Nq), dim3(kSelThreads), (size_t)smem, s, sel);
 }
 
 }  // namespace
 
 size_t index_topk_workspace_bytes(int Nq, int cap) { return carve(nullptr, Nq, cap, nullptr); }
 
-cudaError_t launch_index_topk(const csa_cache &c, const void *q_idx, const float *w, int Nq, int H_I,
-                              const int32_t *q_offsets, const int32_t *q_pos, int topk, int32_t *sel_idx,
-                              void *workspace, int num_sms, cudaStream_t s) {
-    IndexWs ws;
-    carve(workspace, Nq, c.capacity, &ws);
+namespace {
+
+// Scores of every key of every query into ws.scores (rows of `rows`), the
+// first-level thresholds, then the selection into sel_idx. n_vis_given and
+// pool describe a Reindex call (keys are pool positions); both null otherwise.
+cudaError_t index_pipeline(const csa_cache &c, const void *q_idx, const float *w, int Nq, int H_I,
+                           const int32_t *q_offsets, const int32_t *q_pos, int topk, int32_t *sel_idx, IndexWs &ws,
+                           int rows, const int32_t *n_vis_given, const int32_t *pool, int pool_shift, int pool_p,
+                           int num_sms, cudaStream_t s) {
     cudaError_t err = cudaMemsetAsync(ws.done, 0, ws.zero_bytes, s);  // counters, histograms, bitmaps
     if (err != cudaSuccess) return err;
     err = launch_pdl(schedule_kernel, dim3(1), dim3(1024), 0, s, q_offsets, q_pos, c.n_blocks, c.batch, Nq, c.block,
-                     c.capacity, topk, ws.req, ws.n_vis, ws.gprefix, ws.thresh);
+                     rows, topk, ws.req, ws.n_vis, ws.gprefix, ws.thresh, n_vis_given);
     if (err != cudaSuccess) return err;
 
     ScanArgs sa;
@@ -801,6 +986,10 @@ cudaError_t launch_index_topk(const csa_cache &c, const void *q_idx, const float
     sa.H_I = H_I;
     sa.cap = c.capacity;
     sa.topk = topk;
+    sa.rows = rows;
+    sa.pool = pool;
+    sa.pool_shift = pool_shift;
+    sa.pool_p = pool_p;
     const int grid = num_sms;
     const bool e4 = c.idx_dtype == CSA_IDX_E4M3;
     switch (c.idx_dim / 16) {
@@ -810,39 +999,67 @@ cudaError_t launch_index_topk(const csa_cache &c, const void *q_idx, const float
         default: return cudaErrorInvalidValue;
     }
     if (err != cudaSuccess) return err;
+    return launch_select(ws, Nq, rows, topk, sel_idx, pool, pool_shift, pool_p, num_sms, s);
+}
 
-    SelArgs sel;
-    sel.n_vis = ws.n_vis;
-    sel.scores = ws.scores;
-    sel.hist1 = ws.hist1;
-    sel.thresh = ws.thresh;
-    sel.bitmap = ws.bitmap;
-    sel.ncand = ws.ncand;
-    sel.cand_key = ws.cand_key;
-    sel.cand_idx = ws.cand_idx;
-    sel.sel_idx = sel_idx;
-    sel.Nq = Nq;
-    sel.cap = c.capacity;
-    sel.topk = topk;
-    sel.words = ws.words;
-    sel.ccap = ws.ccap;
-    // enough warps to cover the rows with a few 128-score steps each
-    const int chunks_per_cta = 128 * (kPassThreads / 32);
-    int gx = (c.capacity + chunks_per_cta - 1) / chunks_per_cta;
-    const int want = (16 * num_sms + Nq - 1) / Nq;
-    if (gx > want) gx = want;
-    if (gx < 1) gx = 1;
-    if ((err = launch_pdl(select_pass_kernel, dim3(gx, Nq), dim3(kPassThreads), 0, s, sel)) != cudaSuccess) return err;
-    // dynamic shared memory: the bitmap, then as many candidates as fit next to
-    // the ~33 KB of static shared memory (opt in every time: cheap, valid in capture)
-    const int kDynMax = 200 * 1024;
-    sel.smem_cands = (kDynMax - 8 * ws.words) / 8;
-    if (sel.smem_cands < 0) sel.smem_cands = 0;
-    if (sel.smem_cands > ws.ccap) sel.smem_cands = ws.ccap;
-    const int smem = 8 * ws.words + 8 * sel.smem_cands;
-    err = cudaFuncSetAttribute(select_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+}  // namespace
+
+cudaError_t launch_index_topk(const csa_cache &c, const void *q_idx, const float *w, int Nq, int H_I,
+                              const int32_t *q_offsets, const int32_t *q_pos, int topk, int32_t *sel_idx,
+                              void *workspace, int num_sms, cudaStream_t s) {
+    IndexWs ws;
+    carve(workspace, Nq, c.capacity, &ws);
+    return index_pipeline(c, q_idx, w, Nq, H_I, q_offsets, q_pos, topk, sel_idx, ws, c.capacity, nullptr, nullptr, 0,
+                          0, num_sms, s);
+}
+
+size_t index_pool_workspace_bytes(int Nq, int cap, int G, int P) {
+    (void)P;
+    const int cap_b = (cap + G - 1) / G;
+    return align256(carve(nullptr, Nq, cap, nullptr)) + carve(nullptr, Nq, cap_b, nullptr);
+}
+
+cudaError_t launch_index_topk_pool(const csa_cache &c, const void *q_idx, const float *w, int Nq, int H_I,
+                                   const int32_t *q_offsets, const int32_t *q_pos, int topk, int32_t *sel_idx,
+                                   int pool_shift, int P, int32_t *pool_blk, void *workspace, int num_sms,
+                                   cudaStream_t s) {
+    const int G = 1 << pool_shift;
+    const int cap_b = (c.capacity + G - 1) / G;
+    IndexWs ws, wb;
+    const size_t main_bytes = align256(carve(workspace, Nq, c.capacity, &ws));
+    carve(static_cast<char *>(workspace) + main_bytes, Nq, cap_b, &wb);
+    // this layer's own top-k; its score rows stay in ws.scores
+    cudaError_t err = index_pipeline(c, q_idx, w, Nq, H_I, q_offsets, q_pos, topk, sel_idx, ws, c.capacity, nullptr,
+                                     nullptr, 0, 0, num_sms, s);
     if (err != cudaSuccess) return err;
-    return launch_pdl(select_final_kernel, dim3(Nq), dim3(kSelThreads), (size_t)smem, s, sel);
+    // block maxima -> the P best blocks, with the same selection kernels
+    if ((err = cudaMemsetAsync(wb.done, 0, wb.zero_bytes, s)) != cudaSuccess) return err;
+    const int per_cta = kBmaxThreads * kBmaxPerThread;
+    const int gx = (cap_b + per_cta - 1) / per_cta;
+    err = launch_pdl(pool_bmax_kernel, dim3(gx, Nq), dim3(kBmaxThreads), 0, s, (const float *)ws.scores,
+                     (const int32_t *)ws.n_vis, c.capacity, pool_shift, P, wb.scores, cap_b, wb.n_vis, wb.hist1,
+                     wb.done, wb.thresh);
+    if (err != cudaSuccess) return err;
+    return launch_select(wb, Nq, cap_b, P, pool_blk, nullptr, 0, 0, num_sms, s);
+}
+
+size_t index_reindex_workspace_bytes(int Nq, int G, int P) { return carve(nullptr, Nq, G * P, nullptr); }
+
+cudaError_t launch_index_topk_reindex(const csa_cache &c, const void *q_idx, const float *w, int Nq, int H_I,
+                                      const int32_t *q_offsets, const int32_t *q_pos, int topk, int32_t *sel_idx,
+                                      int pool_shift, int P, const int32_t *pool_blk, void *workspace, int num_sms,
+                                      cudaStream_t s) {
+    const int rows = P << pool_shift;
+    IndexWs ws;
+    carve(workspace, Nq, rows, &ws);
+    // visible pool positions per query, counted into ws.n_vis (the schedule keeps them)
+    int32_t *n_pos = ws.n_vis;
+    cudaError_t err = launch_pdl(reindex_count_kernel, dim3(Nq), dim3(kCountThreads), 0, s, q_offsets, q_pos,
+                                 c.n_blocks, c.batch, c.block, c.capacity, (const int32_t *)pool_blk, P, pool_shift,
+                                 n_pos, c.status);
+    if (err != cudaSuccess) return err;
+    return index_pipeline(c, q_idx, w, Nq, H_I, q_offsets, q_pos, topk, sel_idx, ws, rows, n_pos, pool_blk,
+                          pool_shift, P, num_sms, s);
 }
 
 }  // namespace csa

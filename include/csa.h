@@ -112,7 +112,8 @@ typedef struct {
 /* Human-readable name of a csa_status value. Never NULL. */
 const char *csa_status_string(int32_t status);
 
-/* Library ABI version (major * 100 + minor). 101 added csa_cache.scale_fmt. */
+/* Library ABI version (major * 100 + minor). 101 added csa_cache.scale_fmt, 102 the pool and
+ * Reindex calls. */
 int32_t csa_version(void);
 
 /*
@@ -194,6 +195,55 @@ csa_status csa_index_topk(const csa_cache *cache, const void *q_idx, const float
 csa_status csa_index_topk_noalloc(const csa_cache *cache, const void *q_idx, const float *w, int32_t n_queries,
                                   int32_t idx_heads, const int32_t *q_offsets, const int32_t *q_pos, int32_t topk,
                                   int32_t *sel_idx, csa_stream_t stream);
+
+/*
+ * Hierarchical indexer and CSA2 Reindex mode.
+ * Source: DeepSeek-V4.1-Flash podcast transcript, cue 12 (three per-layer modes:
+ * Full computes its own indexer scores and top-k; Reindex reuses the main KV and
+ * indexer keys of an earlier Full layer but runs its own indexer query; Reuse
+ * takes an earlier layer's top-k indices, i.e. calls csa_decode_attend with
+ * them) and cue 14 (the first Full layer also keeps the highest-scoring blocks
+ * of about eight positions, scored by their best position, as a candidate pool
+ * of about sixteen thousand positions; Reindex layers search only that pool).
+ *
+ * csa_index_topk_pool: everything csa_index_topk does, plus the pool. The
+ * visible blocks j < n_vis (as for csa_index_topk) are grouped into pool blocks
+ * of pool_group consecutive blocks; pool block p scores max s_j over its
+ * visible j; the min(pool_blocks, ceil(n_vis / pool_group)) pool blocks with
+ * the largest score (ties to the lower p) are written ascending to
+ * pool_blk[i][0 ..], padded with -1.
+ *   pool_group  1, 2, 4, 8, 16 or 32 (8 in the transcript)
+ *   pool_blocks 1 .. 4096 (about 2000 in the transcript); pool_group *
+ *               pool_blocks <= 2^19
+ *   pool_blk    int32 [n_queries][pool_blocks] device, written
+ *   workspace   >= csa_index_pool_workspace(...) bytes, 256-byte aligned
+ * Other arguments as for csa_index_topk.
+ */
+size_t csa_index_pool_workspace(const csa_cache *cache, int32_t n_queries, int32_t topk, int32_t pool_group,
+                                int32_t pool_blocks);
+csa_status csa_index_topk_pool(const csa_cache *cache, const void *q_idx, const float *w, int32_t n_queries,
+                               int32_t idx_heads, const int32_t *q_offsets, const int32_t *q_pos, int32_t topk,
+                               int32_t *sel_idx, int32_t pool_group, int32_t pool_blocks, int32_t *pool_blk,
+                               void *workspace, size_t workspace_bytes, csa_stream_t stream);
+
+/*
+ * csa_index_topk_reindex: a Reindex-mode layer's own indexer query (q_idx, w)
+ * scored only against the blocks of its pool (as written by csa_index_topk_pool
+ * for the same queries and cache): the candidates are the visible blocks
+ * j < n_vis of pool blocks pool_blk[i][0 ..] (ascending, -1 padding at the end);
+ * sel_idx[i] receives the min(topk, #candidates) with the largest s_j (ties to
+ * the lower j), ascending, padded with -1. A pool block at or beyond n_vis, or
+ * out of ascending order, ends the list there and sets CSA_DEV_BAD_INDEX.
+ *   workspace >= csa_index_reindex_workspace(...) bytes, 256-byte aligned
+ * The work per query is bounded by pool_group * pool_blocks, not by the context.
+ */
+size_t csa_index_reindex_workspace(const csa_cache *cache, int32_t n_queries, int32_t pool_group,
+                                   int32_t pool_blocks);
+csa_status csa_index_topk_reindex(const csa_cache *cache, const void *q_idx, const float *w, int32_t n_queries,
+                                  int32_t idx_heads, const int32_t *q_offsets, const int32_t *q_pos, int32_t topk,
+                                  int32_t *sel_idx, int32_t pool_group, int32_t pool_blocks,
+                                  const int32_t *pool_blk, void *workspace, size_t workspace_bytes,
+                                  csa_stream_t stream);
 
 /* Bytes of workspace csa_decode_attend / hca_decode_attend need (0 on bad sizes). */
 size_t csa_attend_workspace(const csa_cache *cache, int32_t n_queries, int32_t heads);

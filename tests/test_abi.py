@@ -32,7 +32,7 @@ def test_every_declared_symbol_is_exported(lib):
     assert set(names) == set(csa.EXPORTED), names
     for n in names:
         assert hasattr(lib, n), n
-    assert lib.csa_version() == 101
+    assert lib.csa_version() == 102
     assert lib.csa_status_string(0) == b"ok"
     assert lib.csa_status_string(99) == b"unknown status"
 
@@ -112,6 +112,37 @@ def test_attend_validation(lib):
     assert call(q=0x90008) == ERR_ALIGN
     assert lib.hca_decode_attend(ctypes.byref(c), 0x90000, 4, 64, 0xB0000, None, None, None, None, 128, 0.1,
                                  0x1000000, None, 0x2000000, 1 << 30, None) != OK
+
+
+def test_pool_and_reindex_validation(lib):
+    c = fake_cache()
+    ws = lib.csa_index_pool_workspace(ctypes.byref(c), 32, 1024, 8, 2000)
+    assert ws > lib.csa_index_topk_workspace(ctypes.byref(c), 32, 1024)
+    assert lib.csa_index_pool_workspace(ctypes.byref(c), 32, 1024, 6, 2000) == 0   # group not a power of two
+    assert lib.csa_index_pool_workspace(ctypes.byref(c), 32, 1024, 64, 2000) == 0  # group above 32
+    wr = lib.csa_index_reindex_workspace(ctypes.byref(c), 32, 8, 2000)
+    assert wr >= 32 * 8 * 2000 * 4  # the score rows over the pool positions
+
+    def pool(cache=c, q=0x90000, k=1024, grp=8, pb=2000, out=0xE0000, wsp=0x1000000, wsb=None):
+        return lib.csa_index_topk_pool(ctypes.byref(cache), q, 0xA0000, 32, 4, 0xB0000, 0xC0000, k, 0xD0000, grp, pb,
+                                       out, wsp, ws if wsb is None else wsb, None)
+
+    def reindex(q=0x90000, grp=8, pb=2000, pl=0xE0000, wsp=0x1000000, wsb=None):
+        return lib.csa_index_topk_reindex(ctypes.byref(c), q, 0xA0000, 32, 4, 0xB0000, 0xC0000, 1024, 0xD0000, grp,
+                                          pb, pl, wsp, wr if wsb is None else wsb, None)
+
+    assert pool(out=0) == ERR_NULL
+    assert pool(q=0) == ERR_NULL
+    assert pool(grp=3) == ERR_SHAPE
+    assert pool(pb=0) == ERR_SHAPE
+    assert pool(pb=5000) == ERR_UNSUPPORTED
+    assert pool(out=0xE0002) == ERR_ALIGN
+    assert pool(wsb=ws - 1) == ERR_WORKSPACE
+    assert pool(cache=fake_cache(idx_key=0)) == ERR_NULL
+    assert reindex(pl=0) == ERR_NULL
+    assert reindex(grp=5) == ERR_SHAPE
+    assert reindex(wsb=wr - 1) == ERR_WORKSPACE
+    assert reindex(wsp=0x1000010) == ERR_ALIGN
 
 
 def test_read_status_needs_status_word(lib):
