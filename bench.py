@@ -36,6 +36,7 @@ sys.path.insert(0, ROOT)
 
 B, D, H, M_CSA, M_HCA, W = 32, 512, 64, 4, 128, 128
 H_I, D_I, TOPK = 4, 128, 1024
+POOL_GROUP, POOL_BLOCKS = 8, 2000  # hierarchical indexer pool: ~2000 blocks of 8 entries
 CTX_MIN, CTX_MAX = 524288, 1048576
 CAP_CSA, CAP_HCA = CTX_MAX // M_CSA, CTX_MAX // M_HCA
 OUR_KERNELS_PER_STEP = 14  # compress 2x(pool, commit); index: schedule, scan, select x2; attend 2x(schedule, main, merge)
@@ -128,6 +129,33 @@ class Workload:
         nws = max(csa.csa_attend_workspace(self.csa, B, H), csa.csa_attend_workspace(self.hca, B, H))
         self.ws_att = torch.empty(nws, dtype=torch.uint8, device=device)
         self.scale = D ** -0.5
+        # CSA2: a Reindex-mode layer's own indexer query over the Full layer's pool
+        self.q_idx_re = torch.randn(B, H_I, D_I, device=device, generator=gen).to(bf)
+        self.w_re = (torch.randn(B, H_I, device=device, generator=gen) / math.sqrt(H_I)).float()
+        self.sel_pool = torch.empty(B, TOPK, dtype=torch.int32, device=device)
+        self.sel_re = torch.empty(B, TOPK, dtype=torch.int32, device=device)
+        self.pool = torch.empty(B, POOL_BLOCKS, dtype=torch.int32, device=device)
+        self.ws_pool = torch.empty(csa.csa_index_pool_workspace(self.csa, B, TOPK, POOL_GROUP, POOL_BLOCKS),
+                                   dtype=torch.uint8, device=device)
+        self.ws_re = torch.empty(csa.csa_index_reindex_workspace(self.csa, B, POOL_GROUP, POOL_BLOCKS),
+                                 dtype=torch.uint8, device=device)
+
+    def stage_index_pool(self):
+        import fp4_kv_cache_csa_b200 as csa
+
+        csa.csa_index_topk_pool(self.csa, self.q_idx, self.w, self.q_offsets, self.q_pos, TOPK, POOL_GROUP,
+                                POOL_BLOCKS, sel_idx=self.sel_pool, pool_blk=self.pool, workspace=self.ws_pool)
+
+    def stage_index_reindex(self):
+        import fp4_kv_cache_csa_b200 as csa
+
+        csa.csa_index_topk_reindex(self.csa, self.q_idx_re, self.w_re, self.q_offsets, self.q_pos, TOPK, self.pool,
+                                   POOL_GROUP, sel_idx=self.sel_re, workspace=self.ws_re)
+
+    def bytes_reindex(self) -> float:
+        """Keys of the pool's entries (about POOL_GROUP * POOL_BLOCKS per request), query, output."""
+        pooled = np.minimum(self.n_csa, POOL_GROUP * POOL_BLOCKS).astype(np.float64)
+        return float(np.sum(pooled)) * D_I + B * (H_I * D_I * 2 + H_I * 4 + TOPK * 4 + POOL_BLOCKS * 4)
 
     def stages(self):
         return (self.stage_compress, self.stage_index, self.stage_attend_csa, self.stage_attend_hca)
@@ -486,6 +514,31 @@ def main():
     step_ms = st_ms.sum(axis=1)
     ms = float(step_ms.mean())
 
+    # ---- CSA2 (not part of the step): a Full layer that also keeps the pool, and
+    # a Reindex layer over that pool, each timed alone with a cold L2
+    csa2_graphs = []
+    with torch.cuda.stream(stream):
+        for fn in (wl.stage_index_pool, wl.stage_index_reindex):
+            fn()
+        stream.synchronize()
+        for fn in (wl.stage_index_pool, wl.stage_index_reindex):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                fn()
+            csa2_graphs.append(g)
+    n2 = max(4, min(args.steps, 50))
+    ev2 = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(2 * n2)]
+    with torch.cuda.stream(stream):
+        for k in range(2 * n2):
+            flush.zero_()
+            ev2[k][0].record(stream)
+            csa2_graphs[k % 2].replay()
+            ev2[k][1].record(stream)
+    stream.synchronize()
+    csa2_ms = [float(np.mean([ev2[k][0].elapsed_time(ev2[k][1]) for k in range(j, 2 * n2, 2)])) for j in range(2)]
+    status |= csa.csa_read_device_status(wl.csa, stream)
+    del csa2_graphs
+
     # ---- end-to-end: pinned host inputs in, results out, every step. Two buffer
     # sets (each with its own graphs): step k+1's inputs are copied in and step
     # k-1's results copied out (own streams) while step k computes.
@@ -600,6 +653,11 @@ def main():
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_n,
                 "overlap": "step k+1 inputs in and step k-1 results out while step k computes",
                 "link_h2d_gbs": h2d / (link_ms[0] * 1e-3) / 1e9, "link_d2h_gbs": d2h / (link_ms[1] * 1e-3) / 1e9},
+        # CSA2 cross-layer modes (not in the step): Full layer + pool, then a Reindex layer over the pool
+        "csa2": {"pool_group": POOL_GROUP, "pool_blocks": POOL_BLOCKS, "full_with_pool_ms": csa2_ms[0],
+                 "reindex_ms": csa2_ms[1], "full_ms": idx_ms,
+                 "reindex_algorithmic_bytes": wl.bytes_reindex(),
+                 "reindex_achieved_gbs": wl.bytes_reindex() / (csa2_ms[1] * 1e-3) / 1e9},
         "gpu_launches": OUR_KERNELS_PER_STEP * args.steps,
         "clocks": clocks.summary(),
         "device_status": status,

@@ -227,6 +227,17 @@ def csa_index_topk(cache: Cache, q_idx, w, q_offsets, q_pos, topk: int, sel_idx=
     return sel_idx
 
 
+def csa_index_pool_workspace(cache: Cache, n_queries: int, topk: int, pool_group: int = 8,
+                             pool_blocks: int = 2000) -> int:
+    return int(load_library().csa_index_pool_workspace(ctypes.byref(cache.c_struct()), n_queries, topk, pool_group,
+                                                       pool_blocks))
+
+
+def csa_index_reindex_workspace(cache: Cache, n_queries: int, pool_group: int = 8, pool_blocks: int = 2000) -> int:
+    return int(load_library().csa_index_reindex_workspace(ctypes.byref(cache.c_struct()), n_queries, pool_group,
+                                                          pool_blocks))
+
+
 def csa_index_topk_pool(cache: Cache, q_idx, w, q_offsets, q_pos, topk: int, pool_group: int = 8,
                         pool_blocks: int = 2000, sel_idx=None, pool_blk=None, workspace=None, stream=None):
     """A Full-mode layer's indexer: its top-k (as csa_index_topk) and the candidate pool of the
@@ -239,8 +250,7 @@ def csa_index_topk_pool(cache: Cache, q_idx, w, q_offsets, q_pos, topk: int, poo
         sel_idx = torch.empty(n_queries, topk, dtype=torch.int32, device=q_idx.device)
     if pool_blk is None:
         pool_blk = torch.empty(n_queries, pool_blocks, dtype=torch.int32, device=q_idx.device)
-    need = int(lib.csa_index_pool_workspace(ctypes.byref(cache.c_struct()), n_queries, topk, pool_group,
-                                            pool_blocks))
+    need = csa_index_pool_workspace(cache, n_queries, topk, pool_group, pool_blocks)
     workspace = _workspace(need, workspace, q_idx.device)
     c = cache.c_struct()
     _check(lib.csa_index_topk_pool(ctypes.byref(c), _ptr(q_idx), _ptr(w), n_queries, idx_heads, _ptr(q_offsets),
@@ -259,7 +269,7 @@ def csa_index_topk_reindex(cache: Cache, q_idx, w, q_offsets, q_pos, topk: int, 
     pool_blocks = int(pool_blk.shape[1])
     if sel_idx is None:
         sel_idx = torch.empty(n_queries, topk, dtype=torch.int32, device=q_idx.device)
-    need = int(lib.csa_index_reindex_workspace(ctypes.byref(cache.c_struct()), n_queries, pool_group, pool_blocks))
+    need = csa_index_reindex_workspace(cache, n_queries, pool_group, pool_blocks)
     workspace = _workspace(need, workspace, q_idx.device)
     c = cache.c_struct()
     _check(lib.csa_index_topk_reindex(ctypes.byref(c), _ptr(q_idx), _ptr(w), n_queries, idx_heads, _ptr(q_offsets),

@@ -287,7 +287,8 @@ struct ScanCfg {
     static constexpr int U = (16 / (2 * NV)) > 0 ? 16 / (2 * NV) : 1;  // groups in flight per warp
 };
 
-template <bool E4M3, int KS>
+// POOL: keys are pool positions (Reindex), mapped to cache blocks through a.pool.
+template <bool E4M3, int KS, bool POOL>
 __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a) {
     using C = ScanCfg<E4M3, KS>;
     grid_dep_wait();    // the schedule kernel's ranges (programmatic launch)
@@ -387,7 +388,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a) {
 
         const uint8_t *kbase = a.keys + (size_t)b * a.cap * C::KEY_BYTES;
         float *srow = a.scores + (size_t)i * a.rows;
-        const int32_t *prow = a.pool ? a.pool + (size_t)i * a.pool_p : nullptr;
+        const int32_t *prow = POOL ? a.pool + (size_t)i * a.pool_p : nullptr;
 
         for (long long u0 = warp; u0 < nloc; u0 += (long long)kScanWarps * C::U) {
             uint4 raw[C::U][2][C::NV];
@@ -400,7 +401,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a) {
                     const long long r = 16 * lg + g + 8 * half;
                     const bool ok = gv && r < n;
                     long long row = r;
-                    if (prow && ok)
+                    if (POOL && ok)
                         row = ((long long)__ldg(prow + (r >> a.pool_shift)) << a.pool_shift) +
                               (r & ((1 << a.pool_shift) - 1));
                     const uint4 *src = reinterpret_cast<const uint4 *>(kbase + row * C::KEY_BYTES + t * C::ROW_BYTES_T);
@@ -907,7 +908,8 @@ __global__ void __launch_bounds__(kCountThreads) reindex_count_kernel(const int3
 
 template <bool E4M3, int KS>
 cudaError_t launch_scan(const ScanArgs &sa, int grid, cudaStream_t s) {
-    return launch_pdl(scan_kernel<E4M3, KS>, dim3(grid), dim3(kScanThreads), 0, s, sa);
+    if (sa.pool) return launch_pdl(scan_kernel<E4M3, KS, true>, dim3(grid), dim3(kScanThreads), 0, s, sa);
+    return launch_pdl(scan_kernel<E4M3, KS, false>, dim3(grid), dim3(kScanThreads), 0, s, sa);
 }
 
 // select_pass + select_final over the score rows of ws (row stride `rows`,
