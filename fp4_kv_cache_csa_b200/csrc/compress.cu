@@ -105,7 +105,16 @@ struct CompressArgs {
     int m, cap, D, dI;
     int idx_e4m3;
     int scale_e4m3;                // 1: one E4M3 scale per 16 elements, 0: one E8M0 scale per 32
+    int batch;
+    int flat;                      // 1: grid over all blocks of all requests (see below)
 };
+
+// Flat grid: the blocks of all requests in one list, request by request; a
+// request whose token count is not a multiple of m has none. Every CTA builds
+// the per-request block prefix in shared memory (s_pref[b] = blocks before
+// request b, batch + 1 entries) and finds the request of its flat block by
+// binary search, so no CTA is launched for a request's missing blocks.
+constexpr int kFlatMaxBatch = 2047;
 
 // E channels per lane (D = 32*E), EI indexer channels per lane (0 = no
 // indexer keys), WPB warps per block: WPB = 1 puts four independent blocks in
@@ -124,14 +133,55 @@ pool_quantize_kernel(CompressArgs a) {
     grid_dep_launch();
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
-    const int b = blockIdx.y;
-    const int jb = WPB == 1 ? blockIdx.x * kWarpsPerCta + warp : blockIdx.x;
     const int wib = WPB == 1 ? 0 : warp;  // warp index inside the block's team
+    int b, jb;
+    bool active;
+    if (a.flat) {
+        extern __shared__ int s_pref[];  // [batch + 1]
+        __shared__ int scan_smem[32];
+        __shared__ int round_total;
+        int carry = 0;
+        for (int r0 = 0; r0 < a.batch; r0 += blockDim.x) {
+            const int r = r0 + (int)threadIdx.x;
+            int nbr = 0;
+            if (r < a.batch) {
+                const int cnt = a.tok_offsets[r + 1] - a.tok_offsets[r];
+                const bool ok = cnt >= 0 && cnt % a.m == 0;
+                nbr = ok ? cnt / a.m : 0;
+                if (!ok && blockIdx.x == 0) flag(a.status, CSA_DEV_TOKEN_COUNT);
+            }
+            const int incl = block_inclusive_scan<int>(nbr, scan_smem);
+            if (r < a.batch) s_pref[r + 1] = carry + incl;
+            if (threadIdx.x == blockDim.x - 1) round_total = incl;
+            __syncthreads();
+            carry += round_total;
+            __syncthreads();
+        }
+        if (threadIdx.x == 0) s_pref[0] = 0;
+        __syncthreads();
+        const int gb = WPB == 1 ? blockIdx.x * kWarpsPerCta + warp : blockIdx.x;
+        active = gb < s_pref[a.batch];  // CTA-uniform when WPB > 1
+        b = 0;
+        jb = 0;
+        if (active) {
+            int lo = 0, hi = a.batch - 1;  // last request with s_pref[b] <= gb
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (s_pref[mid] <= gb) lo = mid; else hi = mid - 1;
+            }
+            b = lo;
+            jb = gb - s_pref[lo];
+        }
+    } else {
+        b = blockIdx.y;
+        jb = WPB == 1 ? blockIdx.x * kWarpsPerCta + warp : blockIdx.x;
+        active = true;  // narrowed below
+    }
     const int t_begin = a.tok_offsets[b];
     const int count = a.tok_offsets[b + 1] - t_begin;
     const bool count_ok = count >= 0 && count % a.m == 0;
     const int nb = count_ok ? count / a.m : 0;
-    const bool active = jb < nb;  // CTA-uniform when WPB > 1
+    active = active && jb < nb;  // CTA-uniform when WPB > 1
     const int base = a.n_blocks[b];  // checked after the token loads are in flight
 
     float wg[E];
@@ -189,8 +239,8 @@ pool_quantize_kernel(CompressArgs a) {
         }
     }
 
-    if (!count_ok) {
-        if (jb == 0 && threadIdx.x == 0) flag(a.status, CSA_DEV_TOKEN_COUNT);
+    if (!count_ok) {  // (flat grid: flagged above; only an idle CTA gets here)
+        if (!a.flat && jb == 0 && threadIdx.x == 0) flag(a.status, CSA_DEV_TOKEN_COUNT);
         return;
     }
     if ((long long)base + nb > a.cap) {
@@ -322,7 +372,8 @@ template <int E, int EI, int WPB>
 cudaError_t launch_one(const CompressArgs &a, dim3 grid, cudaStream_t s) {
     constexpr int W = WPB == 1 ? 1 : team_warps<E, EI>();
     const dim3 block(W == 1 ? kWarpsPerCta * kWarp : W * kWarp);
-    return launch_pdl(pool_quantize_kernel<E, EI, W>, grid, block, 0, s, a);
+    const size_t dyn = a.flat ? sizeof(int) * (size_t)(a.batch + 1) : 0;
+    return launch_pdl(pool_quantize_kernel<E, EI, W>, grid, block, dyn, s, a);
 }
 
 template <int E, int WPB>
@@ -339,8 +390,10 @@ cudaError_t launch_ew(const CompressArgs &a, dim3 grid, cudaStream_t s) {
 // m >= 32: a team of warps per block; otherwise four blocks per CTA, one warp each
 template <int E>
 cudaError_t launch_e(const CompressArgs &a, int max_blocks, int batch, cudaStream_t s) {
-    if (a.m >= 32) return launch_ew<E, 2>(a, dim3(max_blocks, batch), s);
-    return launch_ew<E, 1>(a, dim3((max_blocks + kWarpsPerCta - 1) / kWarpsPerCta, batch), s);
+    // flat grid: max_blocks bounds the blocks of all requests together
+    const int gy = a.flat ? 1 : batch;
+    if (a.m >= 32) return launch_ew<E, 2>(a, dim3(max_blocks, gy), s);
+    return launch_ew<E, 1>(a, dim3((max_blocks + kWarpsPerCta - 1) / kWarpsPerCta, gy), s);
 }
 
 }  // namespace
@@ -364,6 +417,8 @@ cudaError_t launch_compress(const csa_cache &c, const void *kv_tok, const void *
     a.dI = c.idx_key ? c.idx_dim : 0;
     a.idx_e4m3 = c.idx_dtype == CSA_IDX_E4M3;
     a.scale_e4m3 = c.scale_fmt == CSA_SCALE_E4M3_16;
+    a.batch = c.batch;
+    a.flat = c.batch <= kFlatMaxBatch;
     const int max_blocks = (n_tokens + c.block - 1) / c.block;
     if (max_blocks > 0) {
         cudaError_t err;
