@@ -4,6 +4,8 @@ The GPU runs the whole batch; the oracle recomputes sampled queries one by one.
   * csa_b32_1m: 32 requests, 131072..262144 blocks each (512K..1M tokens, m = 4),
     e4m3 indexer keys, k = 1024, D = 512, 64 heads, 128-token window.
   * hca_b64_1m: 64 requests x 8192 blocks (1M tokens, m = 128), dense.
+  * csa2 at csa_b32_1m: the Full layer's pool (2000 blocks of 8 entries) and a
+    Reindex layer over it, on the same kind of cache.
   * csa_b8_64k: 8 requests x 65536 tokens from raw tokens through every kernel
     (per-channel LogNormal(0, 0.5) activations), checked stage by stage, in both
     scale formats (E8M0 per 32, E4M3 per 16).
@@ -65,6 +67,57 @@ def test_csa_b32_1m_sampled():
                                    np.array([0], np.int64), np.array([W], np.int32), D ** -0.5)
         err, _ = parity.attention_row_error(out[b:b + 1], ref)
         assert err <= parity.ATT_TOL, (b, err)
+
+
+def test_csa2_pool_reindex_b32_1m_sampled():
+    # the Full layer's pool (2000 blocks of 8 entries) and a Reindex layer over it,
+    # in the benchmark's configuration; sampled queries recomputed by the oracle
+    import torch
+
+    import fp4_kv_cache_csa_b200 as csa
+    from test_gpu_pool import block_max_rows, check_reindex
+
+    wl = datagen.WORKLOADS["csa_b32_1m"]
+    B, dI, k, G, P = wl.batch, wl.idx_dim, wl.topk, 8, 2000
+    n = (datagen.context_lengths(wl, 530) // wl.block).astype(np.int64)
+    cap = int(n.max())
+    sample = [3, int(np.argmin(n))]
+    key_d = torch.empty(B, cap, dI, dtype=torch.uint8, device="cuda")
+    host_keys = {}
+    for b in range(B):
+        kx = datagen.to_e4m3_bytes(datagen.normal_f32((cap, dI), 531, b, std=0.5))
+        key_d[b].copy_(torch.from_numpy(kx))
+        if b in sample:
+            host_keys[b] = kx
+    D = 128
+    cache = csa.Cache(fp4=torch.zeros(B, cap, D // 2, dtype=torch.uint8, device="cuda"),
+                      scale=torch.zeros(B, cap, D // 32, dtype=torch.uint8, device="cuda"),
+                      n_blocks=dev(n.astype(np.int32)), block=wl.block, idx_key=key_d, idx_dtype=csa.CSA_IDX_E4M3,
+                      status=torch.zeros(1, dtype=torch.int32, device="cuda"))
+    q_full = datagen.normal_bf16((B, wl.idx_heads, dI), 532, 1)
+    w_full = datagen.normal_f32((B, wl.idx_heads), 532, 2, std=0.5)
+    q_re = datagen.normal_bf16((B, wl.idx_heads, dI), 532, 3)
+    w_re = datagen.normal_f32((B, wl.idx_heads), 532, 4, std=0.5)
+    qo = np.arange(B + 1, dtype=np.int32)
+    qp = (n * wl.block - 1).astype(np.int32)
+    sel, pool = csa.csa_index_topk_pool(cache, dev(q_full), dev(w_full), dev(qo), dev(qp), k, pool_group=G,
+                                        pool_blocks=P)
+    sel_re = csa.csa_index_topk_reindex(cache, dev(q_re), dev(w_re), dev(qo), dev(qp), k, pool, pool_group=G)
+    assert csa.csa_read_device_status(cache) == 0
+    sel, pool, sel_re = host(sel), host(pool), host(sel_re)
+    one = np.array([0, 1], np.int32)
+    for b in sample:
+        kx = host_keys[b][None]
+        nb = n[b:b + 1].astype(np.int32)
+        s_full, n_vis = oracle.index_scores(kx, nb, one, qp[b:b + 1], q_full[b:b + 1], w_full[b:b + 1], m=wl.block,
+                                            idx_dtype=1)
+        parity.check_topk(sel[b:b + 1], oracle.topk(s_full, n_vis, k), s_full, n_vis, k)
+        bmax, nbk = block_max_rows(s_full, n_vis, G)
+        parity.check_topk(pool[b:b + 1], oracle.index_pool(s_full, n_vis, G=G, P=P), bmax, nbk, P)
+        s_re, _ = oracle.index_scores(kx, nb, one, qp[b:b + 1], q_re[b:b + 1], w_re[b:b + 1], m=wl.block,
+                                      idx_dtype=1)
+        ref_re = oracle.reindex_topk(s_re, n_vis, pool[b:b + 1], G=G, k=k)
+        check_reindex(sel_re[b:b + 1], ref_re, s_re, n_vis, pool[b:b + 1], G, k)
 
 
 def test_hca_b64_1m_sampled():
