@@ -565,10 +565,14 @@ __device__ __forceinline__ int32_t out_index(const SelArgs &a, int i, int r) {
 
 // Keys above the threshold bin -> bitmap; keys in it -> candidate list.
 // Grid: (chunks of 128 x kPassThreads/32 scores, Nq).
-__global__ void __launch_bounds__(kPassThreads) select_pass_kernel(SelArgs a) {
+// Two independent selections may share a launch: rows blockIdx.y < a0.Nq
+// belong to a0, the rest to a1 (a1.Nq = 0 when there is one).
+__global__ void __launch_bounds__(kPassThreads) select_pass_kernel(SelArgs a0, SelArgs a1) {
     grid_dep_wait();
     grid_dep_launch();
-    const int i = blockIdx.y;
+    const bool second = blockIdx.y >= (unsigned)a0.Nq;
+    const SelArgs a = second ? a1 : a0;
+    const int i = blockIdx.y - (second ? a0.Nq : 0);
     const int n = a.n_vis[i];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int above_bin = a.thresh[3 * i];      // select keys whose bin is > above_bin
@@ -679,9 +683,11 @@ __device__ __forceinline__ int key_digit(int level, uint32_t key) {
     return level == 1 ? (int)((key >> 8) & 0xFFF) : (int)(key & 0xFF);
 }
 
-__global__ void __launch_bounds__(kSelThreads) select_final_kernel(SelArgs a) {
+__global__ void __launch_bounds__(kSelThreads) select_final_kernel(SelArgs a0, SelArgs a1) {
     extern __shared__ uint32_t dyn[];
     grid_dep_wait();
+    const bool second = blockIdx.x >= (unsigned)a0.Nq;
+    const SelArgs a = second ? a1 : a0;
     uint32_t *bm = dyn;                                                // [words] selected blocks
     uint32_t *tie = dyn + a.words;                                     // [words] members tied on the key
     uint32_t *sck = dyn + 2 * a.words;                                 // [smem_cands] candidate keys
@@ -691,7 +697,7 @@ __global__ void __launch_bounds__(kSelThreads) select_final_kernel(SelArgs a) {
     __shared__ BinPick pick;
     __shared__ uint32_t total_s, kmin_s, kmax_s;
     __shared__ int prefix_digit[3];
-    const int i = blockIdx.x;
+    const int i = blockIdx.x - (second ? a0.Nq : 0);
     const int n = a.n_vis[i];
     const int K = min(a.topk, n);
     int32_t *out = a.sel_idx + (size_t)i * a.topk;
@@ -969,46 +975,65 @@ cudaError_t launch_scan(const ScanArgs &sa, int grid, cudaStream_t s) {
     return launch_pdl(scan_kernel<E4M3, KS, false, false>, dim3(grid), dim3(kScanThreads), 0, s, sa);
 }
 
-// select_pass + select_final over the score rows of ws (row stride `rows`,
-// thresholds from the scan or the block-max kernel), into sel_idx [Nq][topk].
-cudaError_t launch_select(const IndexWs &ws, int Nq, int rows, int topk, int32_t *sel_idx, const int32_t *pool,
-                          int pool_shift, int pool_p, int num_sms, cudaStream_t s) {
+// One selection: score rows, thresholds and output of a workspace.
+struct SelJob {
+    const IndexWs *ws;
+    int Nq, rows, topk;
+    int32_t *sel_idx;
+    const int32_t *pool;  // pool positions -> blocks (Reindex) or null
+    int pool_shift, pool_p;
+};
+
+SelArgs sel_args(const SelJob &j, int smem_cands) {
     SelArgs sel;
-    sel.n_vis = ws.n_vis;
-    sel.scores = ws.scores;
-    sel.hist1 = ws.hist1;
-    sel.thresh = ws.thresh;
-    sel.bitmap = ws.bitmap;
-    sel.ncand = ws.ncand;
-    sel.cand_key = ws.cand_key;
-    sel.cand_idx = ws.cand_idx;
-    sel.sel_idx = sel_idx;
-    sel.Nq = Nq;
-    sel.cap = rows;
-    sel.topk = topk;
-    sel.words = ws.words;
-    sel.ccap = ws.ccap;
-    sel.pool = pool;
-    sel.pool_shift = pool_shift;
-    sel.pool_p = pool_p;
-    // enough warps to cover the rows with a few 128-score steps each
-    const int chunks_per_cta = 128 * (kPassThreads / 32);
-    int gx = (rows + chunks_per_cta - 1) / chunks_per_cta;
-    const int want = (16 * num_sms + Nq - 1) / Nq;
-    if (gx > want) gx = want;
-    if (gx < 1) gx = 1;
-    cudaError_t err = launch_pdl(select_pass_kernel, dim3(gx, Nq), dim3(kPassThreads), 0, s, sel);
-    if (err != cudaSuccess) return err;
+    sel.n_vis = j.ws->n_vis;
+    sel.scores = j.ws->scores;
+    sel.hist1 = j.ws->hist1;
+    sel.thresh = j.ws->thresh;
+    sel.bitmap = j.ws->bitmap;
+    sel.ncand = j.ws->ncand;
+    sel.cand_key = j.ws->cand_key;
+    sel.cand_idx = j.ws->cand_idx;
+    sel.sel_idx = j.sel_idx;
+    sel.Nq = j.Nq;
+    sel.cap = j.rows;
+    sel.topk = j.topk;
+    sel.words = j.ws->words;
+    sel.ccap = j.ws->ccap;
+    sel.pool = j.pool;
+    sel.pool_shift = j.pool_shift;
+    sel.pool_p = j.pool_p;
+    sel.smem_cands = smem_cands;
+    return sel;
+}
+
+// select_pass + select_final for one selection, or two independent ones in
+// the same launches (j1 non-null: the keys' top-k and the pool's blocks).
+cudaError_t launch_select(const SelJob &j0, const SelJob *j1, int num_sms, cudaStream_t s) {
     // dynamic shared memory: the bitmap, then as many candidates as fit next to
     // the ~33 KB of static shared memory (opt in every time: cheap, valid in capture)
     const int kDynMax = 200 * 1024;
-    sel.smem_cands = (kDynMax - 8 * ws.words) / 8;
-    if (sel.smem_cands < 0) sel.smem_cands = 0;
-    if (sel.smem_cands > ws.ccap) sel.smem_cands = ws.ccap;
-    const int smem = 8 * ws.words + 8 * sel.smem_cands;
+    const int words = j1 ? max(j0.ws->words, j1->ws->words) : j0.ws->words;
+    int cands = (kDynMax - 8 * words) / 8;
+    if (cands < 0) cands = 0;
+    if (cands > j0.ws->ccap) cands = j0.ws->ccap;
+    const SelArgs a0 = sel_args(j0, cands);
+    SelArgs a1 = j1 ? sel_args(*j1, cands) : a0;
+    if (!j1) a1.Nq = 0;
+    const int nq = a0.Nq + a1.Nq;
+    // enough warps to cover the rows with a few 128-score steps each
+    const int chunks_per_cta = 128 * (kPassThreads / 32);
+    const int rows = j1 ? max(j0.rows, j1->rows) : j0.rows;
+    int gx = (rows + chunks_per_cta - 1) / chunks_per_cta;
+    const int want = (16 * num_sms + nq - 1) / nq;
+    if (gx > want) gx = want;
+    if (gx < 1) gx = 1;
+    cudaError_t err = launch_pdl(select_pass_kernel, dim3(gx, nq), dim3(kPassThreads), 0, s, a0, a1);
+    if (err != cudaSuccess) return err;
+    const int smem = 8 * words + 8 * cands;
     err = cudaFuncSetAttribute(select_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
-    return launch_pdl(select_final_kernel, dim3(Nq), dim3(kSelThreads), (size_t)smem, s, sel);
+    return launch_pdl(select_final_kernel, dim3(nq), dim3(kSelThreads), (size_t)smem, s, a0, a1);
 }
 
 }  // namespace
@@ -1026,7 +1051,7 @@ cudaError_t index_pipeline(const csa_cache &c, const void *q_idx, const float *w
                            const int32_t *q_offsets, const int32_t *q_pos, int topk, int32_t *sel_idx, IndexWs &ws,
                            int rows, const int32_t *n_vis_given, const int32_t *pool, int pool_shift, int pool_p,
                            int num_sms, cudaStream_t s, const IndexWs *wb = nullptr, int pool_keep = 0,
-                           int rows_b = 0) {
+                           int rows_b = 0, bool skip_select = false) {
     cudaError_t err = cudaMemsetAsync(ws.done, 0, ws.zero_bytes, s);  // counters, histograms, bitmaps
     if (err != cudaSuccess) return err;
     err = launch_pdl(schedule_kernel, dim3(1), dim3(1024), 0, s, q_offsets, q_pos, c.n_blocks, c.batch, Nq, c.block,
@@ -1067,7 +1092,9 @@ cudaError_t index_pipeline(const csa_cache &c, const void *q_idx, const float *w
         default: return cudaErrorInvalidValue;
     }
     if (err != cudaSuccess) return err;
-    return launch_select(ws, Nq, rows, topk, sel_idx, pool, pool_shift, pool_p, num_sms, s);
+    if (skip_select) return cudaSuccess;
+    const SelJob job{&ws, Nq, rows, topk, sel_idx, pool, pool_shift, pool_p};
+    return launch_select(job, nullptr, num_sms, s);
 }
 
 }  // namespace
@@ -1103,9 +1130,12 @@ cudaError_t launch_index_topk_pool(const csa_cache &c, const void *q_idx, const 
         // block count of a query without visible blocks stays 0)
         if ((err = cudaMemsetAsync(wb.n_vis, 0, sizeof(int32_t) * (size_t)Nq, s)) != cudaSuccess) return err;
         err = index_pipeline(c, q_idx, w, Nq, H_I, q_offsets, q_pos, topk, sel_idx, ws, c.capacity, nullptr, nullptr,
-                             0, 0, num_sms, s, &wb, P, cap_b);
+                             0, 0, num_sms, s, &wb, P, cap_b, true);
         if (err != cudaSuccess) return err;
-        return launch_select(wb, Nq, cap_b, P, pool_blk, nullptr, 0, 0, num_sms, s);
+        // the keys' top-k and the pool's blocks in the same two launches
+        const SelJob keys{&ws, Nq, c.capacity, topk, sel_idx, nullptr, 0, 0};
+        const SelJob blocks{&wb, Nq, cap_b, P, pool_blk, nullptr, 0, 0};
+        return launch_select(keys, &blocks, num_sms, s);
     }
     // this layer's own top-k; its score rows stay in ws.scores
     err = index_pipeline(c, q_idx, w, Nq, H_I, q_offsets, q_pos, topk, sel_idx, ws, c.capacity, nullptr, nullptr, 0,
@@ -1118,7 +1148,8 @@ cudaError_t launch_index_topk_pool(const csa_cache &c, const void *q_idx, const 
                      (const int32_t *)ws.n_vis, c.capacity, pool_shift, P, wb.scores, cap_b, wb.n_vis, wb.hist1,
                      wb.done, wb.thresh);
     if (err != cudaSuccess) return err;
-    return launch_select(wb, Nq, cap_b, P, pool_blk, nullptr, 0, 0, num_sms, s);
+    const SelJob blocks{&wb, Nq, cap_b, P, pool_blk, nullptr, 0, 0};
+    return launch_select(blocks, nullptr, num_sms, s);
 }
 
 size_t index_reindex_workspace_bytes(int Nq, int G, int P) { return carve(nullptr, Nq, G * P, nullptr); }
