@@ -269,12 +269,6 @@ struct ScanArgs {
     // G * pool[i][r / G] + r % G, G = 1 << pool_shift; null: r itself
     const int32_t *pool;
     int pool_shift, pool_p;
-    // block maxima for the pool (BMAX, groups of 8 keys): one row of maxima per
-    // query (stride rows_b), their histogram, the threshold for keeping pool_keep
-    float *bmax;
-    int rows_b, pool_keep;
-    uint32_t *hist_b;
-    int32_t *thresh_b, *n_vis_b;
 };
 
 // Dimension permutation. The dot product sums over all d_I channels, so the
@@ -294,16 +288,12 @@ struct ScanCfg {
 };
 
 // POOL: keys are pool positions (Reindex), mapped to cache blocks through a.pool.
-// BMAX: also the maximum of every 8 consecutive scores (the hierarchical
-// indexer's pool of the first Full-mode layer): the two halves of a 16-key
-// group are two such blocks.
-template <bool E4M3, int KS, bool POOL, bool BMAX>
+template <bool E4M3, int KS, bool POOL>
 __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a) {
     using C = ScanCfg<E4M3, KS>;
     grid_dep_wait();    // the schedule kernel's ranges (programmatic launch)
     grid_dep_launch();
     __shared__ uint32_t hist[kBins];
-    __shared__ uint32_t hist_b[BMAX ? kBins : 1];
     __shared__ uint32_t scan_smem[32];
     __shared__ BinPick pick;
     __shared__ int last_flag;
@@ -393,10 +383,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a) {
             if (h1 < a.H_I) w_hi = ldexpf(a.w[(size_t)i * a.H_I + h1], -k1);
         }
 
-        for (int k = threadIdx.x; k < kBins; k += kScanThreads) {
-            hist[k] = 0;
-            if (BMAX) hist_b[k] = 0;
-        }
+        for (int k = threadIdx.x; k < kBins; k += kScanThreads) hist[k] = 0;
         __syncthreads();
 
         const uint8_t *kbase = a.keys + (size_t)b * a.cap * C::KEY_BYTES;
@@ -461,22 +448,6 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a) {
                         atomicAdd(&hist[ordered_key(sc) >> 20], 1u);
                     }
                 }
-                if constexpr (BMAX) {
-                    // block 2 lg: rows g of the group, block 2 lg + 1: rows g + 8
-                    const long long r0 = 16 * lg + g;
-                    float m0 = (gv && r0 < n) ? p0 : -INFINITY;
-                    float m1 = (gv && r0 + 8 < n) ? p1 : -INFINITY;
-#pragma unroll
-                    for (int o = 4; o < 32; o <<= 1) {
-                        m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, o));
-                        m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, o));
-                    }
-                    if (gv && lane < 2 && 16 * lg + 8 * lane < n) {  // the block has a visible key
-                        const float mb = lane == 0 ? m0 : m1;
-                        st_keep(a.bmax + (size_t)i * a.rows_b + 2 * lg + lane, mb, pol_keep);
-                        atomicAdd(&hist_b[ordered_key(mb) >> 20], 1u);
-                    }
-                }
             }
         }
         __syncthreads();
@@ -485,10 +456,6 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a) {
         for (int k = threadIdx.x; k < kBins; k += kScanThreads) {
             const uint32_t c = vh[k];
             if (c) atomicAdd(gh + k, c);
-            if (BMAX) {
-                const uint32_t cb = hist_b[k];
-                if (cb) atomicAdd(a.hist_b + (size_t)i * kBins + k, cb);
-            }
         }
         // the CTA that completes a query's scan finds its k-th key bin (no waiting:
         // groups are counted, and only the one that brings the count to the total acts)
@@ -500,29 +467,6 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a) {
             last_flag = atomicAdd(a.done + i, mine) + mine == total;
         }
         __syncthreads();
-        if (BMAX && last_flag) {  // the pool's threshold: the pool_keep best blocks of 8
-            __threadfence();
-            const int nb = (n + 7) >> 3;
-            if (a.pool_keep >= nb) {
-                if (threadIdx.x == 0) {
-                    a.thresh_b[3 * i] = -1;
-                    a.thresh_b[3 * i + 1] = nb;
-                    a.thresh_b[3 * i + 2] = -1;
-                }
-            } else {
-                for (int k = threadIdx.x; k < kBins; k += kScanThreads) hist[k] = __ldcg(a.hist_b + (size_t)i * kBins + k);
-                __syncthreads();
-                const BinPick p = pick_bin(hist, kBins, (uint32_t)a.pool_keep, scan_smem, &pick);
-                if (threadIdx.x == 0) {
-                    const bool all_at = p.above + p.at == (uint32_t)a.pool_keep;
-                    a.thresh_b[3 * i] = all_at ? p.bin - 1 : p.bin;
-                    a.thresh_b[3 * i + 1] = (int)p.above;
-                    a.thresh_b[3 * i + 2] = all_at ? -1 : p.bin;
-                }
-            }
-            if (threadIdx.x == 0) a.n_vis_b[i] = nb;
-            __syncthreads();
-        }
         if (last_flag && a.topk < n) {
             __threadfence();
             for (int k = threadIdx.x; k < kBins; k += kScanThreads) hist[k] = __ldcg(gh + k);
@@ -970,9 +914,8 @@ __global__ void __launch_bounds__(kCountThreads) reindex_count_kernel(const int3
 
 template <bool E4M3, int KS>
 cudaError_t launch_scan(const ScanArgs &sa, int grid, cudaStream_t s) {
-    if (sa.pool) return launch_pdl(scan_kernel<E4M3, KS, true, false>, dim3(grid), dim3(kScanThreads), 0, s, sa);
-    if (sa.bmax) return launch_pdl(scan_kernel<E4M3, KS, false, true>, dim3(grid), dim3(kScanThreads), 0, s, sa);
-    return launch_pdl(scan_kernel<E4M3, KS, false, false>, dim3(grid), dim3(kScanThreads), 0, s, sa);
+    if (sa.pool) return launch_pdl(scan_kernel<E4M3, KS, true>, dim3(grid), dim3(kScanThreads), 0, s, sa);
+    return launch_pdl(scan_kernel<E4M3, KS, false>, dim3(grid), dim3(kScanThreads), 0, s, sa);
 }
 
 // One selection: score rows, thresholds and output of a workspace.
@@ -1045,13 +988,11 @@ namespace {
 // Scores of every key of every query into ws.scores (rows of `rows`), the
 // first-level thresholds, then the selection into sel_idx. n_vis_given and
 // pool describe a Reindex call (keys are pool positions); both null otherwise.
-// wb (groups of 8): the scan also writes the block maxima and the pool's
-// thresholds into wb, whose counters must be zero (wb.zero_bytes) already.
+// skip_select: the caller launches the selection (together with another one).
 cudaError_t index_pipeline(const csa_cache &c, const void *q_idx, const float *w, int Nq, int H_I,
                            const int32_t *q_offsets, const int32_t *q_pos, int topk, int32_t *sel_idx, IndexWs &ws,
                            int rows, const int32_t *n_vis_given, const int32_t *pool, int pool_shift, int pool_p,
-                           int num_sms, cudaStream_t s, const IndexWs *wb = nullptr, int pool_keep = 0,
-                           int rows_b = 0, bool skip_select = false) {
+                           int num_sms, cudaStream_t s, bool skip_select = false) {
     cudaError_t err = cudaMemsetAsync(ws.done, 0, ws.zero_bytes, s);  // counters, histograms, bitmaps
     if (err != cudaSuccess) return err;
     err = launch_pdl(schedule_kernel, dim3(1), dim3(1024), 0, s, q_offsets, q_pos, c.n_blocks, c.batch, Nq, c.block,
@@ -1077,12 +1018,6 @@ cudaError_t index_pipeline(const csa_cache &c, const void *q_idx, const float *w
     sa.pool = pool;
     sa.pool_shift = pool_shift;
     sa.pool_p = pool_p;
-    sa.bmax = wb ? wb->scores : nullptr;
-    sa.rows_b = rows_b;
-    sa.pool_keep = pool_keep;
-    sa.hist_b = wb ? wb->hist1 : nullptr;
-    sa.thresh_b = wb ? wb->thresh : nullptr;
-    sa.n_vis_b = wb ? wb->n_vis : nullptr;
     const int grid = num_sms;
     const bool e4 = c.idx_dtype == CSA_IDX_E4M3;
     switch (c.idx_dim / 16) {
@@ -1123,33 +1058,21 @@ cudaError_t launch_index_topk_pool(const csa_cache &c, const void *q_idx, const 
     IndexWs ws, wb;
     const size_t main_bytes = align256(carve(workspace, Nq, c.capacity, &ws));
     carve(static_cast<char *>(workspace) + main_bytes, Nq, cap_b, &wb);
-    cudaError_t err = cudaMemsetAsync(wb.done, 0, wb.zero_bytes, s);
+    // this layer's scores and its key threshold; its score rows stay in ws.scores
+    cudaError_t err = index_pipeline(c, q_idx, w, Nq, H_I, q_offsets, q_pos, topk, sel_idx, ws, c.capacity, nullptr,
+                                     nullptr, 0, 0, num_sms, s, true);
     if (err != cudaSuccess) return err;
-    if (G == 8) {
-        // the scan writes the block maxima and the pool's thresholds itself (the
-        // block count of a query without visible blocks stays 0)
-        if ((err = cudaMemsetAsync(wb.n_vis, 0, sizeof(int32_t) * (size_t)Nq, s)) != cudaSuccess) return err;
-        err = index_pipeline(c, q_idx, w, Nq, H_I, q_offsets, q_pos, topk, sel_idx, ws, c.capacity, nullptr, nullptr,
-                             0, 0, num_sms, s, &wb, P, cap_b, true);
-        if (err != cudaSuccess) return err;
-        // the keys' top-k and the pool's blocks in the same two launches
-        const SelJob keys{&ws, Nq, c.capacity, topk, sel_idx, nullptr, 0, 0};
-        const SelJob blocks{&wb, Nq, cap_b, P, pool_blk, nullptr, 0, 0};
-        return launch_select(keys, &blocks, num_sms, s);
-    }
-    // this layer's own top-k; its score rows stay in ws.scores
-    err = index_pipeline(c, q_idx, w, Nq, H_I, q_offsets, q_pos, topk, sel_idx, ws, c.capacity, nullptr, nullptr, 0,
-                         0, num_sms, s);
-    if (err != cudaSuccess) return err;
-    // block maxima -> the P best blocks, with the same selection kernels
+    // block maxima and the pool's threshold, then both selections in the same launches
+    if ((err = cudaMemsetAsync(wb.done, 0, wb.zero_bytes, s)) != cudaSuccess) return err;
     const int per_cta = kBmaxThreads * kBmaxPerThread;
     const int gx = (cap_b + per_cta - 1) / per_cta;
     err = launch_pdl(pool_bmax_kernel, dim3(gx, Nq), dim3(kBmaxThreads), 0, s, (const float *)ws.scores,
                      (const int32_t *)ws.n_vis, c.capacity, pool_shift, P, wb.scores, cap_b, wb.n_vis, wb.hist1,
                      wb.done, wb.thresh);
     if (err != cudaSuccess) return err;
+    const SelJob keys{&ws, Nq, c.capacity, topk, sel_idx, nullptr, 0, 0};
     const SelJob blocks{&wb, Nq, cap_b, P, pool_blk, nullptr, 0, 0};
-    return launch_select(blocks, nullptr, num_sms, s);
+    return launch_select(keys, &blocks, num_sms, s);
 }
 
 size_t index_reindex_workspace_bytes(int Nq, int G, int P) { return carve(nullptr, Nq, G * P, nullptr); }
