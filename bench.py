@@ -404,6 +404,26 @@ def index_traffic(key_bytes: float):
     return INDEX_TRAFFIC_CAPTURE["bytes"] * key_bytes / INDEX_TRAFFIC_CAPTURE["key_bytes"] / 1e9  # GB per call
 
 
+# ----------------------------------------------------------------------------- ranks
+def max_over_ranks(values, world: int, device):
+    """Each timing as the maximum over the ranks (the slowest replica sets the pace)."""
+    if world <= 1:
+        return [float(v) for v in values]
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def job_throughput(ms_per_step: float, world: int):
+    """Replicas: every rank decodes its own B requests per step (weak scaling), so the job's
+    tokens per step are B * world and its rate is set by the slowest rank's step time."""
+    tokens = B * world
+    return tokens, tokens / (ms_per_step * 1e-3)
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -615,16 +635,9 @@ def main():
     e2e_ms = t_start.elapsed_time(t_end) / e2e_n
     del graphs2
 
-    if world > 1:
-        t = torch.tensor([ms, e2e_ms, float(st_ms[:, 1].mean()), float((st_ms[:, 1] + st_ms[:, 2]).mean())],
-                         dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, e2e_ms, idx_ms, csa_ms = (float(x) for x in t.tolist())
-    else:
-        idx_ms = float(st_ms[:, 1].mean())
-        csa_ms = float((st_ms[:, 1] + st_ms[:, 2]).mean())
-    tokens = B * world
-    value = tokens / (ms * 1e-3)
+    ms, e2e_ms, idx_ms, csa_ms = max_over_ranks(
+        [ms, e2e_ms, float(st_ms[:, 1].mean()), float((st_ms[:, 1] + st_ms[:, 2]).mean())], world, device)
+    tokens, value = job_throughput(ms, world)
     peak, peak_kind = measured_peaks()
     achieved = wl.bytes_index() / (idx_ms * 1e-3) / 1e9  # GB/s of the indexer stage
     hbm_tbs = wl.bytes_step() / (ms * 1e-3) / 1e12
