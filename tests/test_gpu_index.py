@@ -108,3 +108,13 @@ def test_head_counts(H_I):
     keys = gen_keys(2, 4096, 128, 1, 33)
     qo, qp = decode_layout([4096, 3000])
     run(keys, [4096, 3000], qo, qp, H_I, 128, 200, 1, seed=34)
+
+
+def test_maximum_sizes():
+    # the largest capacity (2^19 blocks, a 2M-token context), the largest top-k (4096),
+    # the most indexer heads (8) and the widest keys (256 bf16 channels)
+    cap = 1 << 19
+    keys = gen_keys(1, cap, 256, 0, 28)
+    qo, qp = decode_layout([cap])
+    sel, _, n_vis = run(keys, [cap], qo, qp, 8, 256, 4096, 0, seed=29)
+    assert n_vis[0] == cap and np.all(sel[0] >= 0) and np.all(np.diff(sel[0]) > 0)
