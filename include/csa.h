@@ -266,6 +266,10 @@ size_t csa_attend_workspace(const csa_cache *cache, int32_t n_queries, int32_t h
  *   workspace  >= csa_attend_workspace(cache, n_queries, heads) bytes, 256-byte aligned;
  *              it holds an fp16 copy of every query (n_queries * 64 * dim * 2 bytes)
  *              and two partial outputs per SM
+ * Kernel choice: with dim 512 and the environment variable CSA_ATTEND_KERNEL=pair
+ * (read once per process) this call and hca_decode_attend run on two-CTA clusters
+ * (half of the latent channels per CTA); results agree with the default kernel
+ * within the same bound, not bit for bit.
  */
 csa_status csa_decode_attend(const csa_cache *cache, const void *q, int32_t n_queries, int32_t heads,
                              const int32_t *q_offsets, const int32_t *sel_idx, int32_t topk,
