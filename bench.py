@@ -376,6 +376,113 @@ def cpu_baseline(n_requests: int = 2):
 
 
 # ----------------------------------------------------------------------------- main
+class Prefill:
+    """prefill_b4_8k: 4 requests with 16384 cached blocks (seeded bytes) receive 8192 new
+    tokens each (2048 blocks); every new token is a query at its own position, causal at
+    block granularity, with the 128 raw tokens ending at it as its window. Timed apart
+    from the decode step, with its own caches."""
+
+    B, T0, NEW, TOPK = 4, 65536, 8192, 512
+
+    def __init__(self, device):
+        import torch
+
+        import fp4_kv_cache_csa_b200 as csa
+
+        B, T0, NEW = self.B, self.T0, self.NEW
+        self.n0, self.cap = T0 // M_CSA, (T0 + NEW) // M_CSA
+        gen = torch.Generator(device=device)
+        gen.manual_seed(SEED + 4)
+        bf = torch.bfloat16
+        self.cache = csa.Cache.allocate(B, self.cap, D, M_CSA, D_I, csa.CSA_IDX_BF16, device, scale_fmt=SCALE_FMT)
+        s_lo, s_hi = (123, 127) if SCALE_FMT == 0 else (0x1C, 0x2D)
+        self.cache.fp4[:, :self.n0].random_(0, 256, generator=gen)
+        self.cache.scale[:, :self.n0].random_(s_lo, s_hi, generator=gen)
+        self.cache.idx_key[:, :self.n0] = (torch.randn(B, self.n0, D_I, device=device, generator=gen) * 0.5).to(bf)
+        self.base = torch.full((B,), self.n0, dtype=torch.int32, device=device)
+        Nq = B * NEW
+        self.Nq = Nq
+        self.kv = torch.randn(Nq, D, device=device, generator=gen).to(bf)
+        self.idx = torch.randn(Nq, D_I, device=device, generator=gen).to(bf)
+        self.gate_w = (torch.randn(D, device=device, generator=gen) * 0.02).float()
+        self.offs = torch.arange(0, Nq + 1, NEW, dtype=torch.int32, device=device)
+        self.q_pos = torch.arange(T0, T0 + NEW, dtype=torch.int32, device=device).repeat(B)
+        self.q_idx = torch.randn(Nq, H_I, D_I, device=device, generator=gen).to(bf)
+        self.w = (torch.randn(Nq, H_I, device=device, generator=gen) / math.sqrt(H_I)).float()
+        self.q = torch.randn(Nq, H, D, device=device, generator=gen).to(bf)
+        rows = NEW + W - 1  # the 127 raw tokens before the new ones, then the new ones
+        self.win = torch.empty(B * rows, D, dtype=bf, device=device)
+        for b in range(B):
+            self.win[b * rows:b * rows + W - 1] = torch.randn(W - 1, D, device=device, generator=gen).to(bf)
+            self.win[b * rows + W - 1:(b + 1) * rows] = self.kv[b * NEW:(b + 1) * NEW]
+        i = torch.arange(Nq, device=device)
+        self.win_start = (i // NEW * rows + i % NEW).to(torch.int64)
+        self.win_len = torch.full((Nq,), W, dtype=torch.int32, device=device)
+        self.sel = torch.empty(Nq, self.TOPK, dtype=torch.int32, device=device)
+        self.out = torch.empty(Nq, H, D, dtype=torch.float32, device=device)
+        self.ws_idx = torch.empty(csa.csa_index_topk_workspace(self.cache, Nq, self.TOPK), dtype=torch.uint8,
+                                  device=device)
+        self.ws_att = torch.empty(csa.csa_attend_workspace(self.cache, Nq, H), dtype=torch.uint8, device=device)
+
+    def stages(self):
+        return (self.stage_compress, self.stage_index, self.stage_attend)
+
+    def stage_compress(self):
+        import fp4_kv_cache_csa_b200 as csa
+
+        self.cache.n_blocks.copy_(self.base)
+        csa.csa_compress_quantize(self.cache, self.kv, self.idx, self.gate_w, self.offs)
+
+    def stage_index(self):
+        import fp4_kv_cache_csa_b200 as csa
+
+        csa.csa_index_topk(self.cache, self.q_idx, self.w, self.offs, self.q_pos, self.TOPK, sel_idx=self.sel,
+                           workspace=self.ws_idx)
+
+    def stage_attend(self):
+        import fp4_kv_cache_csa_b200 as csa
+
+        csa.csa_decode_attend(self.cache, self.q, self.offs, self.sel, self.win, self.win_start, self.win_len,
+                              max_win=W, softmax_scale=D ** -0.5, out=self.out, workspace=self.ws_att)
+
+    def index_flops(self) -> float:
+        """Indexer contraction, causal: sum over queries of n_vis * H_I * d_I * 2."""
+        t = np.arange(self.NEW, dtype=np.float64)
+        n_vis = np.floor((self.T0 + t + 1) / M_CSA)
+        return float(self.B * np.sum(n_vis)) * H_I * D_I * 2
+
+
+def measure_prefill(device, stream, flush, steps: int = 3):
+    """Per-stage CUDA-event times of the prefill workload (cold L2 before each pass)."""
+    import torch
+
+    import fp4_kv_cache_csa_b200 as csa
+
+    pf = Prefill(device)
+    with torch.cuda.stream(stream):
+        for fn in pf.stages():  # warm-up pass
+            fn()
+    stream.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    with torch.cuda.stream(stream):
+        for k in range(steps):
+            flush.zero_()
+            for s_, fn in enumerate(pf.stages()):
+                ev[k][s_].record(stream)
+                fn()
+            ev[k][3].record(stream)
+    stream.synchronize()
+    st = np.array([[ev[k][s_].elapsed_time(ev[k][s_ + 1]) for s_ in range(3)] for k in range(steps)]).mean(axis=0)
+    status = csa.csa_read_device_status(pf.cache, stream)
+    res = {"workload": "prefill_b4_8k", "queries": pf.Nq, "ms": float(st.sum()),
+           "stage_ms": {"compress": float(st[0]), "index_topk": float(st[1]), "attend": float(st[2])},
+           "index_gflop": pf.index_flops() / 1e9,
+           "index_tflops": pf.index_flops() / (st[1] * 1e-3) / 1e12, "device_status": int(status)}
+    del pf
+    torch.cuda.empty_cache()
+    return res
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -383,6 +490,17 @@ def measured_peaks():
             d = json.load(f)
         return float(d.get("hbm_gbs", 6650.0)), "measured"
     return 6650.0, "fallback"
+
+
+def measured_bf16_tflops():
+    """Dense bf16 tensor peak: the burst figure of MEASURED_PEAKS.json, else the fallback."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        if "bf16_tflops" in d:
+            return float(d["bf16_tflops"]), "measured"
+    return 1590.0, "fallback"
 
 
 # DRAM traffic of one indexer call (schedule + scan + both select kernels) from one ncu
@@ -456,6 +574,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill_b4_8k measurement")
     ap.add_argument("--batch", type=int, default=B, help="requests per GPU (default 32; smaller only for profiling)")
     ap.add_argument("--scale-fmt", default="e8m0x32", choices=sorted(SCALE_FMT_NAMES),
                     help="FP4 scale format of both caches (default: E8M0 per 32 elements, MXFP4)")
@@ -558,6 +677,7 @@ def main():
     csa2_ms = [float(np.mean([ev2[k][0].elapsed_time(ev2[k][1]) for k in range(j, 2 * n2, 2)])) for j in range(2)]
     status |= csa.csa_read_device_status(wl.csa, stream)
     del csa2_graphs
+    prefill = measure_prefill(device, stream, flush) if not args.no_prefill else None
 
     # ---- end-to-end: pinned host inputs in, results out, every step. Two buffer
     # sets (each with its own graphs): step k+1's inputs are copied in and step
@@ -671,6 +791,9 @@ def main():
                  "reindex_ms": csa2_ms[1], "full_ms": idx_ms,
                  "reindex_algorithmic_bytes": wl.bytes_reindex(),
                  "reindex_achieved_gbs": wl.bytes_reindex() / (csa2_ms[1] * 1e-3) / 1e9},
+        "prefill": None if prefill is None else dict(
+            prefill, index_tensor_frac=prefill["index_tflops"] / measured_bf16_tflops()[0],
+            index_tensor_peak={"tflops": measured_bf16_tflops()[0], "kind": measured_bf16_tflops()[1] + " bf16 dense"}),
         "gpu_launches": OUR_KERNELS_PER_STEP * args.steps,
         "clocks": clocks.summary(),
         "device_status": status,

@@ -51,6 +51,12 @@
 
 namespace csa {
 
+// prefill.cu: the scores of many queries per request as a tensor-core GEMM.
+bool prefill_scores_supported(int idx_dtype, int idx_dim, int H_I);
+cudaError_t launch_prefill_scores(const void *keys, int cap, int idx_dim, const void *q_idx, const float *w, int Nq,
+                                  int H_I, const int32_t *req, const int32_t *n_vis, float *scores, int rows,
+                                  int32_t *status, int num_sms, cudaStream_t s);
+
 namespace {
 
 constexpr int kBins = 4096;        // histogram bins per level (12 bits)
@@ -67,6 +73,9 @@ constexpr int kCandCap = 32768;    // candidate slots per query (members of the 
 constexpr int kBmaxThreads = 256;  // pool_bmax_kernel: threads per CTA ...
 constexpr int kBmaxPerThread = 4;  // ... and blocks per thread
 constexpr int kCountThreads = 256; // reindex_count_kernel
+// Queries per request (on average over the call) from which the scores are
+// computed as a tensor-core GEMM (prefill.cu) instead of one key stream per query.
+constexpr int kPrefillQueriesPerRequest = 16;
 
 // ---------------------------------------------------------------- workspace
 struct IndexWs {
@@ -481,6 +490,33 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a) {
         }
         __syncthreads();
         gb = seg_end;
+    }
+}
+
+// ---------------------------------------------------------------- prefill threshold
+// After the prefill GEMM has written the score rows: one CTA per query builds
+// the 4096-bin histogram of its scores' top 12 key bits and picks the bin that
+// holds the k-th largest key, as the scan's last CTA does for a streamed query.
+__global__ void __launch_bounds__(1024) prefill_thresh_kernel(const float *scores, int rows, const int32_t *n_vis,
+                                                              int topk, int32_t *thresh) {
+    __shared__ uint32_t hist[kBins];
+    __shared__ uint32_t scan_smem[32];
+    __shared__ BinPick pick;
+    grid_dep_wait();
+    const int i = blockIdx.x;
+    const int n = n_vis[i];
+    if (topk >= n) return;  // every visible block is selected (the schedule kernel wrote that)
+    for (int k = threadIdx.x; k < kBins; k += blockDim.x) hist[k] = 0;
+    __syncthreads();
+    const float *row = scores + (size_t)i * rows;
+    for (int j = threadIdx.x; j < n; j += blockDim.x) atomicAdd(&hist[ordered_key(__ldcg(row + j)) >> 20], 1u);
+    __syncthreads();
+    const BinPick p = pick_bin(hist, kBins, (uint32_t)topk, scan_smem, &pick);
+    if (threadIdx.x == 0) {
+        const bool all_at = p.above + p.at == (uint32_t)topk;  // the whole bin is selected
+        thresh[3 * i] = all_at ? p.bin - 1 : p.bin;
+        thresh[3 * i + 1] = (int)p.above;
+        thresh[3 * i + 2] = all_at ? -1 : p.bin;
     }
 }
 
@@ -1020,11 +1056,21 @@ cudaError_t index_pipeline(const csa_cache &c, const void *q_idx, const float *w
     sa.pool_p = pool_p;
     const int grid = num_sms;
     const bool e4 = c.idx_dtype == CSA_IDX_E4M3;
-    switch (c.idx_dim / 16) {
-        case 4: err = e4 ? launch_scan<true, 4>(sa, grid, s) : launch_scan<false, 4>(sa, grid, s); break;
-        case 8: err = e4 ? launch_scan<true, 8>(sa, grid, s) : launch_scan<false, 8>(sa, grid, s); break;
-        case 16: err = e4 ? launch_scan<true, 16>(sa, grid, s) : launch_scan<false, 16>(sa, grid, s); break;
-        default: return cudaErrorInvalidValue;
+    if (!pool && !n_vis_given && Nq >= kPrefillQueriesPerRequest * c.batch &&
+        prefill_scores_supported(c.idx_dtype, c.idx_dim, H_I)) {
+        // many queries per request: the scores as a tensor-core GEMM, then per-query thresholds
+        err = launch_prefill_scores(c.idx_key, c.capacity, c.idx_dim, q_idx, w, Nq, H_I, ws.req, ws.n_vis, ws.scores,
+                                    rows, c.status, num_sms, s);
+        if (err != cudaSuccess) return err;
+        err = launch_pdl(prefill_thresh_kernel, dim3(Nq), dim3(1024), 0, s, (const float *)ws.scores, rows,
+                         (const int32_t *)ws.n_vis, topk, ws.thresh);
+    } else {
+        switch (c.idx_dim / 16) {
+            case 4: err = e4 ? launch_scan<true, 4>(sa, grid, s) : launch_scan<false, 4>(sa, grid, s); break;
+            case 8: err = e4 ? launch_scan<true, 8>(sa, grid, s) : launch_scan<false, 8>(sa, grid, s); break;
+            case 16: err = e4 ? launch_scan<true, 16>(sa, grid, s) : launch_scan<false, 16>(sa, grid, s); break;
+            default: return cudaErrorInvalidValue;
+        }
     }
     if (err != cudaSuccess) return err;
     if (skip_select) return cudaSuccess;

@@ -52,6 +52,8 @@ WORKLOADS = {
     "csa_b8_64k": Workload("csa_b8_64k", 8, 65536, 65536, 64, 512, 4, 128, 4, 128, 0, 512, 0.5),
     "csa_b32_1m": Workload("csa_b32_1m", 32, 524288, 1048576, 64, 512, 4, 128, 4, 128, 1, 1024),
     "hca_b64_1m": Workload("hca_b64_1m", 64, 1048576, 1048576, 64, 512, 128, 128, 0, 0, 0, 0),
+    # ctx_min = tokens already in the cache, ctx_max = after the 8192 new ones
+    "prefill_b4_8k": Workload("prefill_b4_8k", 4, 65536, 65536 + 8192, 64, 512, 4, 128, 4, 128, 0, 512),
 }
 
 

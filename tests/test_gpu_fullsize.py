@@ -9,6 +9,9 @@ The GPU runs the whole batch; the oracle recomputes sampled queries one by one.
   * csa_b8_64k: 8 requests x 65536 tokens from raw tokens through every kernel
     (per-channel LogNormal(0, 0.5) activations), checked stage by stage, in both
     scale formats (E8M0 per 32, E4M3 per 16).
+  * prefill_b4_8k: 8192 new tokens appended to 65536 cached ones in each of 4
+    requests; every new block checked, then 32768 causal queries indexed and
+    attended with sampled queries recomputed.
 Cache contents for the first two are seeded bytes (the kernels' inputs), not
 outputs of the compression kernel."""
 import numpy as np
@@ -193,3 +196,79 @@ def test_csa_b8_64k_from_tokens(scale_fmt):
     err, _ = parity.attention_row_error(out, want)
     assert err <= parity.ATT_TOL, err
     assert csa.csa_read_device_status(ocache) == 0
+
+
+def test_prefill_b4_8k_sampled():
+    # prefill: 4 requests with 16384 cached blocks each (seeded bytes) receive 8192 new
+    # tokens (2048 blocks); every new token is a query at its own position (causal at
+    # block granularity), with the 128 raw tokens ending at it as its window
+    import torch
+
+    import fp4_kv_cache_csa_b200 as csa
+
+    wl = datagen.WORKLOADS["prefill_b4_8k"]
+    B, D, H, dI, m, k, W = wl.batch, wl.dim, wl.heads, wl.idx_dim, wl.block, wl.topk, wl.window
+    T0, T1 = wl.ctx_min, wl.ctx_max
+    n0, cap, NEW = T0 // m, T1 // m, T1 - T0
+    f0, s0 = datagen.random_cache_bytes(B * n0, D, 540, 0)
+    k0 = datagen.normal_bf16((B * n0, dI), 540, 1, std=0.5)
+    kv = datagen.normal_bf16((B * NEW, D), 541, 1)
+    it = datagen.normal_bf16((B * NEW, dI), 541, 2)
+    wg = datagen.normal_f32((D,), 541, 3, std=0.02)
+    offs = (np.arange(B + 1) * NEW).astype(np.int32)
+    base = np.full(B, n0, np.int32)
+    ref = oracle.compress(kv, it, wg, offs, base, m=m, cap=cap, return_pooled=True)
+    # stage 1: the GPU appends the new blocks behind the cached ones
+    fp4 = np.zeros((B, cap, D // 2), np.uint8)
+    sc = np.zeros((B, cap, D // 32), np.uint8)
+    keys = np.zeros((B, cap, dI), np.uint16)
+    fp4[:, :n0], sc[:, :n0], keys[:, :n0] = (f0.reshape(B, n0, -1), s0.reshape(B, n0, -1),
+                                             k0.reshape(B, n0, dI))
+    cache = make_cache(fp4, sc, base, m, keys, 0)
+    csa.csa_compress_quantize(cache, dev(kv), dev(it), dev(wg), dev(offs))
+    assert csa.csa_read_device_status(cache) == 0
+    assert np.array_equal(host(cache.n_blocks), ref["n_blocks"])
+    new = slice(n0, cap)
+    tol = parity.pooling_tolerance(kv, offs, base, m, cap)[:, new]
+    parity.check_mxfp4(host(cache.fp4)[:, new].reshape(-1, D // 2), host(cache.scale)[:, new].reshape(-1, D // 32),
+                       ref["fp4"][:, new].reshape(-1, D // 2), ref["scale"][:, new].reshape(-1, D // 32),
+                       ref["pooled"][:, new].reshape(-1, D), tol=tol.reshape(-1, D))
+    assert np.array_equal(host(cache.fp4)[:, :n0], fp4[:, :n0])  # cached blocks untouched
+    parity.check_keys(host(cache.idx_key).view(np.uint16)[:, new], ref["idx_key"].view(np.uint16)[:, new],
+                      ref["pooled_idx"][:, new], "bf16",
+                      tol=parity.pooling_tolerance(it, offs, base, m, cap)[:, new])
+    # stages 2 and 3 run on the oracle's new blocks behind the cached ones
+    fp4[:, new], sc[:, new] = ref["fp4"][:, new], ref["scale"][:, new]
+    keys[:, new] = ref["idx_key"].view(np.uint16)[:, new]
+    ocache = make_cache(fp4, sc, ref["n_blocks"], m, keys, 0)
+    Nq = B * NEW
+    qo = (np.arange(B + 1) * NEW).astype(np.int32)
+    qp = np.tile(np.arange(T0, T1, dtype=np.int32), B)
+    q_idx = datagen.normal_bf16((Nq, wl.idx_heads, dI), 542, 1)
+    w = datagen.normal_f32((Nq, wl.idx_heads), 542, 2, std=0.5)
+    sel_d = csa.csa_index_topk(ocache, dev(q_idx), dev(w), dev(qo), dev(qp), k)
+    # windows: the 127 raw tokens before the new ones (seeded) and the new tokens themselves
+    tail = datagen.normal_bf16((B * (W - 1), D), 543, 1)
+    rows = NEW + W - 1
+    win = np.concatenate([np.concatenate([tail[b * (W - 1):(b + 1) * (W - 1)], kv[b * NEW:(b + 1) * NEW]])
+                          for b in range(B)])
+    ws_ = (np.arange(Nq) // NEW * rows + np.arange(Nq) % NEW).astype(np.int64)
+    wl_ = np.full(Nq, W, np.int32)
+    g = torch.Generator(device="cuda").manual_seed(544)
+    q_d = torch.randn(Nq, H, D, generator=g, device="cuda").to(torch.bfloat16)
+    out_d = csa.csa_decode_attend(ocache, q_d, dev(qo), sel_d, dev(win), dev(ws_), dev(wl_))
+    assert csa.csa_read_device_status(ocache) == 0
+    sel = host(sel_d)
+    one = np.array([0, 1], np.int32)
+    for b in range(B):
+        for t in (0, 1, NEW // 2 - 1, NEW - 1):
+            i = b * NEW + t
+            sel_ref, scores, n_vis = oracle.index_topk(keys[b:b + 1].view(np.uint8), ref["n_blocks"][b:b + 1], one,
+                                                       qp[i:i + 1], q_idx[i:i + 1], w[i:i + 1], m=m, k=k)
+            assert n_vis[0] == (T0 + t + 1) // m
+            parity.check_topk(sel[i:i + 1], sel_ref, scores, n_vis, k)  # the GPU's set is a valid top-k
+            qi = host(q_d[i:i + 1])
+            want, _ = oracle.csa_attend(fp4[b:b + 1], sc[b:b + 1], one, qi, sel[i:i + 1], win[b * rows:(b + 1) * rows],
+                                        np.array([t], np.int64), np.array([W], np.int32), D ** -0.5)
+            err, _ = parity.attention_row_error(host(out_d[i:i + 1]), want)
+            assert err <= parity.ATT_TOL, (b, t, err)

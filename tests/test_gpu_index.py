@@ -118,3 +118,19 @@ def test_maximum_sizes():
     qo, qp = decode_layout([cap])
     sel, _, n_vis = run(keys, [cap], qo, qp, 8, 256, 4096, 0, seed=29)
     assert n_vis[0] == cap and np.all(sel[0] >= 0) and np.all(np.diff(sel[0]) > 0)
+
+
+@pytest.mark.parametrize("H_I,dI,cap", [(4, 128, 3000), (1, 64, 3000), (2, 256, 3001), (8, 128, 3001), (4, 64, 3002),
+                                        (4, 256, 3000)])
+def test_many_queries_per_request_gemm_path(H_I, dI, cap):
+    # calls with many queries per request (prefill) score on the tensor cores; ragged
+    # request sizes put two or three requests into one query tile, and capacities that
+    # are not multiples of 4 take the scalar score stores
+    counts = [300, 213, 1]
+    lengths = [3000, 2100, 500]  # filled blocks per request
+    keys = gen_keys(3, cap, dI, 0, 60 + H_I)
+    qo = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    # each request's queries at increasing positions up to its last token (m = 4)
+    qp = np.concatenate([np.linspace(0, 4 * L - 1, c).astype(np.int32) for c, L in zip(counts, lengths)])
+    sel, _, n_vis = run(keys, lengths, qo, qp, H_I, dI, 256, 0, seed=61)
+    assert n_vis.min() < 256 < n_vis.max()
