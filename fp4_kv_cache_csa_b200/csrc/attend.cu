@@ -491,18 +491,39 @@ __global__ void __launch_bounds__(1024) attend_schedule_kernel(
 // CTA covered were written directly by attend_kernel and are skipped.
 constexpr int kMergeHeads = 8;
 
+// by_boundary (calls with more queries than CTAs): blockIdx.x + 1 is a CTA
+// index c; only a query that CTA c - 1 and CTA c both cover can need a merge,
+// and the CTA for the first such boundary of a query merges it, so the grid
+// has G - 1 columns instead of one per query.
 __global__ void __launch_bounds__(256) attend_merge_kernel(const long long *tprefix, int Nq, int H, int D, int G,
                                                            const float *part_o, const float *part_rho,
-                                                           const float *part_l, float *out, float *lse) {
+                                                           const float *part_l, float *out, float *lse,
+                                                           int by_boundary) {
     __shared__ int slots[256];
     __shared__ float wts[256 * kMergeHeads];
     __shared__ float inv_l[kMergeHeads];
     __shared__ int np_s;
     grid_dep_wait();
-    const int i = blockIdx.x;
     const int h0 = blockIdx.y * kMergeHeads;
     if (h0 >= H) return;
-    const long long T = tprefix[Nq], Ti = tprefix[i], Ti1 = tprefix[i + 1];
+    const long long T = tprefix[Nq];
+    int i = blockIdx.x;
+    if (by_boundary) {
+        // the query holding tile rb = first tile of CTA c: largest i with tprefix[i] < rb
+        const int c = blockIdx.x + 1;
+        const long long rb = T * c / G;
+        int lo = 0, hi = Nq - 1;  // tprefix[0] = 0 < rb unless rb = 0 (then no query straddles)
+        if (rb <= 0) return;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (tprefix[mid] < rb) lo = mid; else hi = mid - 1;
+        }
+        i = lo;
+        if (tprefix[i + 1] <= rb) return;  // the boundary is at the end of query i: nothing straddles
+        const long long Ti0 = tprefix[i];
+        if ((int)(((Ti0 + 1) * G - 1) / T) + 1 != c) return;  // not the query's first inner boundary
+    }
+    const long long Ti = tprefix[i], Ti1 = tprefix[i + 1];
     if (Ti1 == Ti) return;  // no entry at all: written by the schedule kernel
     const int c_first = (int)(((Ti + 1) * G - 1) / T);
     const int c_last = (int)((Ti1 * G - 1) / T);
@@ -1697,7 +1718,8 @@ cudaError_t launch_attend(const csa_cache &c, const void *q, int Nq, int H, cons
         return cudaErrorInvalidValue;
     }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(Nq, (H + kMergeHeads - 1) / kMergeHeads, D / 128);
+    const int by_boundary = Nq > G ? 1 : 0;  // many queries: one column per CTA boundary
+    cfg.gridDim = dim3(by_boundary ? max(1, G - 1) : Nq, (H + kMergeHeads - 1) / kMergeHeads, D / 128);
     cfg.blockDim = dim3(256);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = s;
@@ -1707,7 +1729,8 @@ cudaError_t launch_attend(const csa_cache &c, const void *q, int Nq, int H, cons
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, attend_merge_kernel, (const long long *)tprefix, Nq, H, D, G,
-                              (const float *)a.part_o, (const float *)a.part_rho, (const float *)a.part_l, out, lse);
+                              (const float *)a.part_o, (const float *)a.part_rho, (const float *)a.part_l, out, lse,
+                              by_boundary);
 }
 
 }  // namespace csa

@@ -53,7 +53,7 @@ namespace csa {
 
 // prefill.cu: the scores of many queries per request as a tensor-core GEMM.
 bool prefill_scores_supported(int idx_dtype, int idx_dim, int H_I);
-cudaError_t launch_prefill_scores(const void *keys, int cap, int idx_dim, const void *q_idx, const float *w, int Nq,
+cudaError_t launch_prefill_scores(const void *keys, int batch, int cap, int idx_dim, const void *q_idx, const float *w, int Nq,
                                   int H_I, const int32_t *req, const int32_t *n_vis, float *scores, int rows,
                                   int32_t *status, int num_sms, cudaStream_t s);
 
@@ -194,8 +194,21 @@ __device__ BinPick pick_bin(const uint32_t *h, int nbins, uint32_t need, uint32_
     const int top = nbins - 1 - (int)threadIdx.x * per;  // this thread: bins [top-per+1, top]
     const volatile uint32_t *vh = h;
     uint32_t mine = 0;
-    for (int k = 0; k < per; ++k)
-        if (top - k >= 0) mine += vh[top - k];
+    if ((per & 3) == 0 && (nbins & 3) == 0) {  // this thread's bins are whole 16-byte groups
+        for (int k = 0; k < per; k += 4) {
+            const int lo = top - k - 3;
+            if (lo >= 0) {
+                uint32_t x, y, z, w;
+                asm volatile("ld.volatile.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(x), "=r"(y), "=r"(z), "=r"(w)
+                             : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(h + lo))));
+                mine += x + y + z + w;
+            }
+        }
+    } else {
+        for (int k = 0; k < per; ++k)
+            if (top - k >= 0) mine += vh[top - k];
+    }
     const uint32_t incl = block_inclusive_scan<uint32_t>(mine, scan_smem);
     const uint32_t excl = incl - mine;
     if (excl < need && incl >= need) {
@@ -518,6 +531,261 @@ __global__ void __launch_bounds__(1024) prefill_thresh_kernel(const float *score
         thresh[3 * i + 1] = (int)p.above;
         thresh[3 * i + 2] = all_at ? -1 : p.bin;
     }
+}
+
+// ---------------------------------------------------------------- prefill selection
+// Score rows short enough to sit in shared memory (a prefill query sees at
+// most its request's blocks): one CTA per query brings its row in with one
+// bulk copy, turns it into order-preserving keys in place and finds the exact
+// k-th largest key T by three radix levels (key bits 31..20, 19..8, 7..0):
+//   pass 0  every key: level-0 histogram;
+//   pass 1  every key, warp w over a contiguous index range: the keys above the
+//           threshold bin go to a bitmap (one ballot per 32 keys), the bin's
+//           members to a candidate list and a histogram of bits 19..8;
+//   level 2 over the candidates only; the candidates above T, and the
+//           lowest-indexed candidates equal to T, join the bitmap;
+//   output  the bitmap compacted into ascending indices.
+// When the threshold bin holds more members than the list keeps, level 2 and
+// the output scan every key instead. Replaces the threshold, pass and final
+// kernels, which read the row from memory three times.
+constexpr int kRowSelThreads = 512;
+constexpr int kRowSelWarps = kRowSelThreads / 32;
+constexpr int kRowSelMaxRows = 40960;                 // 160 KB of keys per CTA
+constexpr int kRowSelWords = kRowSelMaxRows / 32;     // bitmap words
+constexpr int kRowSelWarpCands = 128;                 // members of the threshold bin listed per warp
+constexpr int kRowSelCands = kRowSelWarps * kRowSelWarpCands;
+
+__device__ __forceinline__ uint4 ordered_key4(uint4 raw) {
+    return make_uint4(ordered_key(__uint_as_float(raw.x)), ordered_key(__uint_as_float(raw.y)),
+                      ordered_key(__uint_as_float(raw.z)), ordered_key(__uint_as_float(raw.w)));
+}
+
+__global__ void __launch_bounds__(kRowSelThreads) row_select_kernel(const float *scores, int rows,
+                                                                    const int32_t *n_vis, int topk,
+                                                                    int32_t *sel_idx, int32_t *status) {
+    extern __shared__ __align__(16) uint32_t rkeys[];  // [rows]: the row's raw bits, then its keys
+    __shared__ uint32_t h[kBins];
+    __shared__ uint32_t bm[kRowSelWords];
+    __shared__ uint32_t ck[kRowSelCands];
+    __shared__ int32_t cj[kRowSelCands];
+    __shared__ uint32_t scan_smem[32];
+    __shared__ BinPick pick;
+    __shared__ uint32_t wdef[kRowSelWarps], wgt[kRowSelWarps], wtie[kRowSelWarps], wcand[kRowSelWarps], over_s;
+    __shared__ __align__(8) uint64_t rbar;
+    grid_dep_wait();
+    const int i = blockIdx.x;
+    const int n = n_vis[i];
+    const int K = min(topk, n);
+    int32_t *out = sel_idx + (size_t)i * topk;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (K == n) {  // every visible block (or none)
+        for (int r = tid; r < topk; r += blockDim.x) out[r] = r < n ? r : -1;
+        return;
+    }
+    const float *row = scores + (size_t)i * rows;
+    const int n4 = (n + 3) >> 2;  // 16-byte groups covering the row (within it: rows % 4 == 0 when bulk)
+    const bool bulk = (rows & 3) == 0;
+    const uint32_t bar = static_cast<uint32_t>(__cvta_generic_to_shared(&rbar));
+    if (bulk && tid == 0) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar) : "memory");
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"((uint32_t)(16 * n4))
+                     : "memory");
+        asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                     ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(rkeys))), "l"(row),
+                     "r"((uint32_t)(16 * n4)), "r"(bar)
+                     : "memory");
+    }
+    for (int k = tid; k < kBins; k += blockDim.x) h[k] = 0u;
+    if (tid == 0) over_s = 0u;
+    if (!bulk)
+        for (int j = tid; j < n; j += blockDim.x) rkeys[j] = __float_as_uint(__ldcs(row + j));
+    __syncthreads();  // the barrier's initialisation is visible before anyone waits on it
+    if (bulk) {
+        // one thread waits (bounded, sleeping between polls) for the copy while the others
+        // wait at the barrier; on a time-out it records it and waits (bounded) once more
+        // before the CTA may leave, so that no copy into this CTA's memory is left running
+        bool done = true;
+        if (tid == 0) {
+            done = false;
+            for (int attempt = 0; attempt < 2 && !done; ++attempt) {
+                const long long t0 = clock64();
+                while (!done) {
+                    uint32_t d;
+                    asm volatile(
+                        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], 0;\n\t"
+                        "selp.u32 %0, 1, 0, p;\n\t}\n"
+                        : "=r"(d)
+                        : "r"(bar)
+                        : "memory");
+                    done = d != 0;
+                    if (done || clock64() - t0 > 2000000000LL) break;
+                    __nanosleep(128);
+                }
+                if (!done && attempt == 0) flag(status, CSA_DEV_TIMEOUT);
+            }
+        }
+        if (__syncthreads_or(!done)) return;
+    }
+    // ---- pass 0: keys in place, level-0 histogram
+    {
+        uint4 *k4 = reinterpret_cast<uint4 *>(rkeys);
+        for (int c = tid; c < n4; c += blockDim.x) {
+            const uint4 kk = ordered_key4(k4[c]);
+            k4[c] = kk;
+            const int j = 4 * c;
+            atomicAdd(&h[kk.x >> 20], 1u);
+            if (j + 1 < n) atomicAdd(&h[kk.y >> 20], 1u);
+            if (j + 2 < n) atomicAdd(&h[kk.z >> 20], 1u);
+            if (j + 3 < n) atomicAdd(&h[kk.w >> 20], 1u);
+        }
+    }
+    __syncthreads();
+    BinPick p = pick_bin(h, kBins, (uint32_t)K, scan_smem, &pick);
+    const uint32_t b0 = (uint32_t)p.bin;
+    uint32_t need = (uint32_t)K - p.above;
+    // ---- pass 1: keys above the bin -> bitmap; the bin's members -> list and histogram of bits 19..8
+    for (int k = tid; k < kBins; k += blockDim.x) h[k] = 0u;
+    __syncthreads();
+    const int seg = (((n + kRowSelWarps - 1) / kRowSelWarps) + 31) & ~31;  // multiple of 32: whole words
+    const int j0 = min(n, warp * seg), j1 = min(n, j0 + seg);
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    {
+        uint32_t def = 0, wc = 0;  // per warp: keys above the bin, members of the bin so far
+        uint32_t *wck = ck + warp * kRowSelWarpCands;
+        int32_t *wcj = cj + warp * kRowSelWarpCands;
+        for (int base = j0; base < j1; base += 32) {
+            const int j = base + lane;
+            const uint32_t kk = j < j1 ? rkeys[j] : 0u;
+            const uint32_t d0 = kk >> 20;
+            const uint32_t am = __ballot_sync(0xffffffffu, j < j1 && d0 > b0);
+            if (lane == 0) bm[base >> 5] = am;
+            def += __popc(am);
+            const bool c = j < j1 && d0 == b0;
+            const uint32_t cm = __ballot_sync(0xffffffffu, c);
+            if (c) {
+                atomicAdd(&h[(kk >> 8) & 0xFFFu], 1u);
+                const uint32_t pos = wc + __popc(cm & lt_mask);
+                if (pos < (uint32_t)kRowSelWarpCands) {
+                    wck[pos] = kk;
+                    wcj[pos] = j;
+                }
+            }
+            wc += __popc(cm);
+        }
+        if (lane == 0) {
+            wdef[warp] = def;
+            wgt[warp] = 0u;
+            wtie[warp] = 0u;
+            wcand[warp] = wc;
+            if (wc > (uint32_t)kRowSelWarpCands) over_s = 1u;
+        }
+    }
+    __syncthreads();
+    p = pick_bin(h, kBins, need, scan_smem, &pick);
+    const uint32_t pre1 = (b0 << 12) | (uint32_t)p.bin;  // key bits 31..8 fixed
+    need -= p.above;
+    // ---- level 2 over the candidates (every key when the list overflowed)
+    const bool in_list = over_s == 0u;  // slot c of warp c / kRowSelWarpCands is valid below wcand
+    for (int k = tid; k < 256; k += blockDim.x) h[k] = 0u;
+    __syncthreads();
+    const uint32_t my_nc = min(wcand[warp], (uint32_t)kRowSelWarpCands);  // this warp's list (in index order)
+    const uint32_t *my_ck = ck + warp * kRowSelWarpCands;
+    const int32_t *my_cj = cj + warp * kRowSelWarpCands;
+    if (in_list) {
+        for (uint32_t c = lane; c < my_nc; c += 32) {
+            const uint32_t kk = my_ck[c];
+            if ((kk >> 8) == pre1) atomicAdd(&h[kk & 0xFFu], 1u);
+        }
+    } else {
+        for (int j = tid; j < n; j += blockDim.x) {
+            const uint32_t kk = rkeys[j];
+            if ((kk >> 8) == pre1) atomicAdd(&h[kk & 0xFFu], 1u);
+        }
+    }
+    __syncthreads();
+    p = pick_bin(h, 256, need, scan_smem, &pick);
+    const uint32_t T = (pre1 << 8) | (uint32_t)p.bin;  // the k-th largest key
+    const uint32_t take_t = need - p.above;           // keys equal to T to take, lowest indices first (>= 1)
+    if (in_list) {
+        // ---- the candidates above T and the first take_t ties (by index) join the bitmap: warp w
+        // ranks the ties of its own list after those of the lists before it (lists follow index order)
+        {
+            uint32_t t = 0;
+            for (uint32_t c = lane; c < my_nc; c += 32) t += my_ck[c] == T ? 1u : 0u;
+            t = __reduce_add_sync(0xffffffffu, t);
+            if (lane == 0) wtie[warp] = t;
+        }
+        __syncthreads();
+        uint32_t tb = 0;
+        for (int w2 = 0; w2 < warp; ++w2) tb += wtie[w2];
+        for (uint32_t base = 0; base < my_nc; base += 32) {
+            const uint32_t c = base + lane;
+            const uint32_t kk = c < my_nc ? my_ck[c] : 0u;
+            const bool eq = c < my_nc && kk == T;
+            const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+            const bool take = (c < my_nc && kk > T) || (eq && tb + __popc(eqm & lt_mask) < take_t);
+            if (take) {
+                const int j = my_cj[c];
+                atomicOr(&bm[j >> 5], 1u << (j & 31));
+            }
+            tb += __popc(eqm);
+        }
+        __syncthreads();
+        // ---- bitmap -> ascending indices: a contiguous word segment per thread
+        const int words = (n + 31) >> 5;
+        const int wpt = (words + kRowSelThreads - 1) / kRowSelThreads;
+        const int w0 = tid * wpt;
+        uint32_t cnt = 0;
+        for (int k = 0; k < wpt; ++k)
+            if (w0 + k < words) cnt += __popc(bm[w0 + k]);
+        uint32_t pos = block_inclusive_scan<uint32_t>(cnt, scan_smem) - cnt;
+        for (int k = 0; k < wpt; ++k) {
+            const int w = w0 + k;
+            if (w >= words) break;
+            uint32_t bits = bm[w];
+            while (bits) {
+                const int bit = __ffs(bits) - 1;
+                bits &= bits - 1;
+                out[pos++] = w * 32 + bit;
+            }
+        }
+    } else {
+        // ---- overflow: per-warp counts and one ordered scan over every key
+        {
+            uint32_t g = 0, t = 0;
+            for (int j = j0 + lane; j < j1; j += 32) {
+                const uint32_t kk = rkeys[j];
+                g += ((kk >> 20) == b0 && kk > T) ? 1u : 0u;
+                t += kk == T ? 1u : 0u;
+            }
+            g = __reduce_add_sync(0xffffffffu, g);
+            t = __reduce_add_sync(0xffffffffu, t);
+            if (lane == 0) {
+                wgt[warp] = g;
+                wtie[warp] = t;
+            }
+        }
+        __syncthreads();
+        uint32_t tb = 0, ob = 0;  // ties and outputs before this warp's range
+        for (int w2 = 0; w2 < warp; ++w2) {
+            const uint32_t t = wtie[w2];
+            ob += wdef[w2] + wgt[w2] + (tb >= take_t ? 0u : min(t, take_t - tb));
+            tb += t;
+        }
+        for (int base = j0; base < j1; base += 32) {
+            const int j = base + lane;
+            const uint32_t kk = j < j1 ? rkeys[j] : 0u;
+            const bool eq = j < j1 && kk == T;
+            const uint32_t eqm = __ballot_sync(0xffffffffu, eq);
+            const bool take = (j < j1 && kk > T) || (eq && tb + __popc(eqm & lt_mask) < take_t);
+            const uint32_t tm = __ballot_sync(0xffffffffu, take);
+            if (take) out[ob + __popc(tm & lt_mask)] = j;
+            ob += __popc(tm);
+            tb += __popc(eqm);
+        }
+    }
+    for (int r = K + tid; r < topk; r += blockDim.x) out[r] = -1;
 }
 
 // ---------------------------------------------------------------- select
@@ -1029,7 +1297,13 @@ cudaError_t index_pipeline(const csa_cache &c, const void *q_idx, const float *w
                            const int32_t *q_offsets, const int32_t *q_pos, int topk, int32_t *sel_idx, IndexWs &ws,
                            int rows, const int32_t *n_vis_given, const int32_t *pool, int pool_shift, int pool_p,
                            int num_sms, cudaStream_t s, bool skip_select = false) {
-    cudaError_t err = cudaMemsetAsync(ws.done, 0, ws.zero_bytes, s);  // counters, histograms, bitmaps
+    // many queries per request (prefill): scores as a tensor-core GEMM, and when the
+    // rows fit in shared memory one selection kernel that needs no zeroed state
+    const bool gemm = !pool && !n_vis_given && Nq >= kPrefillQueriesPerRequest * c.batch &&
+                      prefill_scores_supported(c.idx_dtype, c.idx_dim, H_I);
+    const bool row_sel = gemm && !skip_select && rows <= kRowSelMaxRows;
+    cudaError_t err = cudaSuccess;
+    if (!row_sel) err = cudaMemsetAsync(ws.done, 0, ws.zero_bytes, s);  // counters, histograms, bitmaps
     if (err != cudaSuccess) return err;
     err = launch_pdl(schedule_kernel, dim3(1), dim3(1024), 0, s, q_offsets, q_pos, c.n_blocks, c.batch, Nq, c.block,
                      rows, topk, ws.req, ws.n_vis, ws.gprefix, ws.thresh, n_vis_given);
@@ -1056,12 +1330,18 @@ cudaError_t index_pipeline(const csa_cache &c, const void *q_idx, const float *w
     sa.pool_p = pool_p;
     const int grid = num_sms;
     const bool e4 = c.idx_dtype == CSA_IDX_E4M3;
-    if (!pool && !n_vis_given && Nq >= kPrefillQueriesPerRequest * c.batch &&
-        prefill_scores_supported(c.idx_dtype, c.idx_dim, H_I)) {
-        // many queries per request: the scores as a tensor-core GEMM, then per-query thresholds
-        err = launch_prefill_scores(c.idx_key, c.capacity, c.idx_dim, q_idx, w, Nq, H_I, ws.req, ws.n_vis, ws.scores,
+    if (gemm) {
+        err = launch_prefill_scores(c.idx_key, c.batch, c.capacity, c.idx_dim, q_idx, w, Nq, H_I, ws.req, ws.n_vis, ws.scores,
                                     rows, c.status, num_sms, s);
         if (err != cudaSuccess) return err;
+        if (row_sel) {
+            const int smem = 16 * ((rows + 3) / 4);
+            err = cudaFuncSetAttribute(row_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            if (err != cudaSuccess) return err;
+            return launch_pdl(row_select_kernel, dim3(Nq), dim3(kRowSelThreads), (size_t)smem, s,
+                              (const float *)ws.scores, rows, (const int32_t *)ws.n_vis, topk, sel_idx, c.status);
+        }
+        // per-query thresholds for the shared selection kernels
         err = launch_pdl(prefill_thresh_kernel, dim3(Nq), dim3(1024), 0, s, (const float *)ws.scores, rows,
                          (const int32_t *)ws.n_vis, topk, ws.thresh);
     } else {

@@ -134,3 +134,24 @@ def test_many_queries_per_request_gemm_path(H_I, dI, cap):
     qp = np.concatenate([np.linspace(0, 4 * L - 1, c).astype(np.int32) for c, L in zip(counts, lengths)])
     sel, _, n_vis = run(keys, lengths, qo, qp, H_I, dI, 256, 0, seed=61)
     assert n_vis.min() < 256 < n_vis.max()
+
+
+@pytest.mark.parametrize("case", ["duplicates", "zeros"])
+def test_gemm_path_exact_ties(case):
+    # prefill-sized calls (many queries per request) take the GEMM path and the
+    # one-CTA-per-query selection; equal scores at the threshold go to the lower index:
+    # 3000 identical keys per request, or 5000 all-zero keys (every score exactly 0)
+    cap = 8192
+    keys = gen_keys(2, cap, 128, 0, 70)
+    rng = np.random.default_rng(71)
+    for b in range(2):
+        if case == "duplicates":
+            dup = rng.choice(cap, 3000, replace=False)
+            keys[b, dup] = keys[b, dup[0]]
+        else:
+            keys[b, :5000] = 0
+    counts, lengths = [64, 64], [8192, 6000]
+    qo = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    qp = np.concatenate([np.linspace(2 * L, 4 * L - 1, c).astype(np.int32) for c, L in zip(counts, lengths)])
+    for k in (100, 2999, 3500):
+        run(keys, lengths, qo, qp, 4, 128, k, 0, seed=72)
