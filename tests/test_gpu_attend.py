@@ -247,3 +247,23 @@ def test_pair_kernel_parity():
     env = dict(os.environ, CSA_ATTEND_KERNEL="pair")
     r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=900)
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
+
+
+@pytest.mark.parametrize("D,H", [(128, 16), (512, 64)])
+def test_more_queries_than_ctas(D, H):
+    # prefill-shaped calls: more queries than CTAs, ragged selection lengths (0 to 3 tiles of
+    # 128 entries) and windows, so many queries straddle a CTA boundary and are merged by the
+    # boundary-indexed merge grid; every query is compared with the oracle
+    B, cap, Nq = 2, 2048, 400
+    fp4, sc = cache_bytes(B, cap, D, 60)
+    counts = [230, 170]
+    q_offsets = np.array([0, counts[0], Nq], np.int32)
+    rng = np.random.default_rng(61)
+    k = 384
+    take = rng.integers(0, k + 1, Nq)
+    take[::37] = 0
+    sel = random_sel([cap] * Nq, k, Nq, 62, pad_from=take)
+    wlen = rng.integers(0, 129, Nq)
+    win, ws, wl = window(Nq, 128, D, 63, wlen=wlen)
+    err, st = run_csa(fp4, sc, [cap, cap], q_offsets, sel, H, D, win, ws, wl, seed=64)
+    assert st == 0
