@@ -507,7 +507,7 @@ def measured_bf16_tflops():
 # capture at 8 requests (profiles/dram_traffic_csa_hca_decode_b8.md): read + write bytes
 # and the key bytes of that call; scaled to this run by key bytes. Valid only for the
 # indexer source it was taken on (hash below); otherwise reported as null.
-INDEX_TRAFFIC_CAPTURE = {"bytes": 217487104 + 66048, "key_bytes": 210.427904e6, "source_hash": "ebfa752484c7232e"}
+INDEX_TRAFFIC_CAPTURE = {"bytes": 217488128 + 122112, "key_bytes": 210.427904e6, "source_hash": "1519eeab27c963c7"}
 
 
 def index_traffic(key_bytes: float):
