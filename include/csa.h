@@ -166,6 +166,13 @@ size_t csa_index_topk_workspace(const csa_cache *cache, int32_t n_queries, int32
  *   sel_idx   int32 [n_queries][topk] device, written
  *   idx_heads 1..8; topk 1..4096
  *   workspace >= csa_index_topk_workspace(cache, n_queries, topk) bytes, 256-byte aligned
+ * Calls that bring on average 16 or more queries per request (prefill) with
+ * bf16 keys of 64, 128 or 256 channels and 1, 2, 4 or 8 indexer heads compute
+ * the scores as one tensor-core GEMM per request (TMA tensor maps over the
+ * key plane and q_idx, which must then be 16-byte aligned, as every pointer
+ * here); when the cache holds at most 40960 blocks the top-k then runs one
+ * thread block per query over its score row in shared memory. The results are
+ * the same as on the streaming path: only the speed differs.
  */
 csa_status csa_index_topk(const csa_cache *cache, const void *q_idx, const float *w, int32_t n_queries,
                           int32_t idx_heads, const int32_t *q_offsets, const int32_t *q_pos, int32_t topk,
