@@ -56,7 +56,7 @@ typedef enum {
     CSA_ERR_NULL = 1,        /* a required pointer is NULL                      */
     CSA_ERR_SHAPE = 2,       /* a size is out of range or inconsistent          */
     CSA_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned                */
-    CSA_ERR_UNSUPPORTED = 4, /* valid request this build does not implement     */
+    CSA_ERR_UNSUPPORTED = 4, /* valid request the library does not implement    */
     CSA_ERR_WORKSPACE = 5,   /* workspace NULL or smaller than required         */
     CSA_ERR_CUDA = 6         /* a CUDA runtime call or kernel launch failed     */
 } csa_status;
