@@ -503,10 +503,10 @@ def measured_bf16_tflops():
     return 1590.0, "fallback"
 
 
-# DRAM traffic of one indexer call (schedule + scan + both select kernels) from one ncu
-# capture at 8 requests (profiles/dram_traffic_csa_hca_decode_b8.md): read + write bytes
-# and the key bytes of that call; scaled to this run by key bytes. Valid only for the
-# indexer source it was taken on (hash below); otherwise reported as null.
+# DRAM traffic of one indexer call (schedule + scan + both select kernels): the read +
+# write bytes that one ncu capture of the call at 8 requests of the same workload
+# counted, and the key bytes of that call; scaled to this run by key bytes. Valid only
+# for the indexer source it was taken on (hash below); otherwise reported as null.
 INDEX_TRAFFIC_CAPTURE = {"bytes": 217488128 + 122112, "key_bytes": 210.427904e6, "source_hash": "1519eeab27c963c7"}
 
 

@@ -41,9 +41,6 @@
 // Compressed rows are loaded into registers one tile ahead (their selected
 // indices two tiles ahead); window tiles (bf16) are copied with cp.async into
 // the operand buffer and converted in place.
-#include <cstdlib>
-#include <cstring>
-
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp4.h>
@@ -955,652 +952,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TMEM_COLS) : "memory");
 }
 
-// ---------------------------------------------------------------- CTA-pair kernel (D = 512)
-// Attention on two-CTA clusters. Both CTAs of a pair walk the same tiles; CTA
-// r holds latent channels [256 r, 256 r + 256) of every entry and of the
-// query, so that its entry tile is 64 KB and can be double-buffered:
-//   * 4 conversion warps dequantize tile t + 1 into one E' buffer; once a
-//     tile is converted, their first thread issues S^T(t) = E'(t) Q'^T over
-//     this CTA's channels (a partial sum for all 64 heads), while
-//   * 8 softmax warps own heads [32 r, 32 r + 32) of tile t - 1 or t: they send
-//     the peer the partial logits of the peer's heads, add the peer's partial
-//     of their own heads, take the softmax step (lazy reference rho as in
-//     attend_kernel) and send the peer their half of P' (with the factors of
-//     any rescale), so that both CTAs hold the full P' of the tile; their
-//     first thread then issues O^T += E'(t)^T P'(t) for this CTA's channels.
-// The two exchanges are bulk copies from this CTA's shared memory into the
-// peer's (one thread issues each; the peer's barrier completes on the bytes).
-// The outgoing partial logits are staged in P'[b] (free until P'(t) is
-// written, which happens only after the peer's Y(t) has arrived -- the peer
-// sends it after receiving all of X(t)), the outgoing P' half in X (consumed
-// by then; the peer's X(t+1) arrives only after it has received this Y(t)).
-// X and Y are single-buffered for the same reason.
-namespace pairk {
-constexpr int D = 512;
-constexpr int HC = 256;                          // channels per CTA
-constexpr int E_BYTES = kTile * HC * 2;          // 64 KB per buffer
-constexpr int KREG = kTile * 128;                // 64-channel region of E'
-constexpr int Q_BYTES = kHeads * HC * 2;         // this CTA's half of the Q' image
-constexpr int QREG = kHeads * 128;
-constexpr int P_BYTES = kTile * kHeads * 2;      // 16 KB per buffer
-constexpr int X_BYTES = kTile * 32 * 4;          // partial logits of this CTA's heads from the peer
-constexpr int Y_BYTES = kTile * 32 * 2 + 256;    // the peer's P' half + its rescale factors and flag
-constexpr int MISC = 4096;
-constexpr int SMEM = 1024 + 2 * E_BYTES + Q_BYTES + 2 * P_BYTES + X_BYTES + Y_BYTES + MISC;
-constexpr int SG = 256;                          // softmax threads: warps 0-7, two per entry row
-constexpr int HPT = 16;                          // heads per softmax thread
-constexpr int THREADS = SG + 128;                // + conversion warps 8-11, one thread per entry row
-constexpr int TMEM_COLS = 256;                   // S^T x 2 buffers (128), O^T 2 d-tiles (128)
-constexpr int RJ_EMPTY = -0x40000000;            // R_j of a padding row
-static_assert(SMEM <= 232448, "shared memory of the pair kernel");
-}  // namespace pairk
-
-// Prefetch of this CTA's half of one compressed entry (the conversion thread
-// of row j): 128 code bytes, and the scale bytes it needs -- all 16 E8M0
-// bytes of the row (R_j is taken over the whole row, so that both CTAs scale
-// the row alike), or the 16 E4M3 bytes of its half.
-template <int SF>
-__device__ __forceinline__ void pair_prefetch_row(const AttArgs &a, const TileRef &tr, int blk, uint32_t rank,
-                                                  RowRegs<512> &rr) {
-    rr.valid = 0;
-    if (blk >= 0 && (blk >= tr.nblk || blk >= a.cap)) {
-        flag(a.status, CSA_DEV_BAD_INDEX);
-        blk = -1;
-    }
-    if (blk >= 0) {
-        const size_t row = (size_t)tr.b * a.cap + blk;
-        const uint4 *src = reinterpret_cast<const uint4 *>(a.fp4 + row * 256) + rank * 8;
-#pragma unroll
-        for (int v = 0; v < 8; ++v) rr.code[v] = __ldg(src + v);
-        const uint8_t *sp = SF == kScaleE4M3x16 ? a.scale + row * 32 + rank * 16 : a.scale + row * 16;
-        rr.sc = __ldg(reinterpret_cast<const uint4 *>(sp));
-        rr.valid = 1;
-    }
-}
-
-// Dequantize this CTA's half of the prefetched row into E' (fp16, 32 chunks
-// of 8 channels in the swizzled K-major layout). Returns R_j (E8M0) or 0.
-template <int SF>
-__device__ __forceinline__ int pair_dequant(const RowRegs<512> &rr, uint32_t rank, uint8_t *E) {
-    const int j = threadIdx.x & (kTile - 1);
-    if (!rr.valid) {
-#pragma unroll
-        for (int kc = 0; kc < 32; ++kc) *reinterpret_cast<uint4 *>(E + e_chunk_off<512>(j, kc)) = make_uint4(0, 0, 0, 0);
-        return 0;
-    }
-    int rmax = 0;
-    if constexpr (SF == kScaleE8M0x32) {
-#pragma unroll
-        for (int g = 0; g < 16; ++g) rmax = max(rmax, scale_byte<512>(rr, g));
-    }
-#pragma unroll
-    for (int gl = 0; gl < 8; ++gl) {  // 32-channel group gl of the half: code bytes 16 gl .. 16 gl + 15
-        __half2 s2[2];
-        if constexpr (SF == kScaleE4M3x16) {
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const __half_raw hr =
-                    __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)scale_byte<512>(rr, 2 * gl + h), __NV_E4M3);
-                s2[h] = __halves2half2(__half(hr), __half(hr));
-            }
-        } else {
-            const int k = scale_byte<512>(rr, 8 * (int)rank + gl) - rmax;  // <= 0
-            const uint16_t hb = k >= -14 ? (uint16_t)((k + 15) << 10) : k >= -24 ? (uint16_t)(1u << (k + 24)) : 0;
-            s2[0] = s2[1] = __halves2half2(__ushort_as_half(hb), __ushort_as_half(hb));
-        }
-        const uint32_t *w = reinterpret_cast<const uint32_t *>(&rr.code[gl]);
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-            uint32_t outw[4];
-#pragma unroll
-            for (int bb = 0; bb < 4; ++bb) {
-                __half2_raw hr =
-                    __nv_cvt_fp4x2_to_halfraw2((__nv_fp4x2_storage_t)((w[cc] >> (8 * bb)) & 0xFF), __NV_E2M1);
-                __half2 h = __hmul2(*reinterpret_cast<__half2 *>(&hr), s2[cc >> 1]);
-                outw[bb] = *reinterpret_cast<uint32_t *>(&h);
-            }
-            *reinterpret_cast<uint4 *>(E + e_chunk_off<512>(j, 4 * gl + cc)) =
-                make_uint4(outw[0], outw[1], outw[2], outw[3]);
-        }
-    }
-    return SF == kScaleE8M0x32 ? rmax - 127 : 0;
-}
-
-// Window row j of a window tile: this CTA's half of the bf16 row is copied
-// into E' with cp.async and converted in place to fp16 scaled by 2^-R_j, R_j
-// the exponent of max |x| over the WHOLE row (the thread also reads the other
-// half for the maximum, so that both CTAs of the pair agree on R_j).
-__device__ __forceinline__ int pair_window_row(const AttArgs &a, const TileRef &tr, uint32_t rank, uint8_t *E,
-                                               uint32_t E_s, bool &valid) {
-    const int j = threadIdx.x & (kTile - 1);
-    const int r = (tr.lt - tr.ctiles) * kTile + j;
-    valid = r < tr.wlen;
-    if (!valid) {
-#pragma unroll
-        for (int kc = 0; kc < 32; ++kc) *reinterpret_cast<uint4 *>(E + e_chunk_off<512>(j, kc)) = make_uint4(0, 0, 0, 0);
-        return 0;
-    }
-    const __nv_bfloat16 *row = a.win_kv + ((size_t)a.win_start[tr.i] + r) * 512;
-    const __nv_bfloat16 *own = row + 256 * rank, *other = row + 256 * (rank ^ 1);
-#pragma unroll 8
-    for (int kc = 0; kc < 32; ++kc) cp_async16(E_s + e_chunk_off<512>(j, kc), own + 8 * kc);
-    asm volatile("cp.async.commit_group;" ::: "memory");
-    auto absmax8 = [](uint4 u, float mx) {
-        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const float2 f = __bfloat1622float2(h[k]);
-            mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
-        }
-        return mx;
-    };
-    float mx = 0.f;
-#pragma unroll 8
-    for (int kc = 0; kc < 32; ++kc) mx = absmax8(__ldg(reinterpret_cast<const uint4 *>(other) + kc), mx);
-    asm volatile("cp.async.wait_all;" ::: "memory");
-#pragma unroll 8
-    for (int kc = 0; kc < 32; ++kc) mx = absmax8(*reinterpret_cast<const uint4 *>(E + e_chunk_off<512>(j, kc)), mx);
-    const int R = mx > 0.f ? (int)((__float_as_uint(mx) >> 23) & 0xFF) - 127 : 0;
-    const float inv = ldexpf(1.0f, -R);
-#pragma unroll 8
-    for (int kc = 0; kc < 32; ++kc) {
-        uint4 u = *reinterpret_cast<const uint4 *>(E + e_chunk_off<512>(j, kc));
-        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
-        uint32_t o[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const float2 f = __bfloat1622float2(h[k]);
-            __half2 hh = __floats2half2_rn(f.x * inv, f.y * inv);
-            o[k] = *reinterpret_cast<uint32_t *>(&hh);
-        }
-        *reinterpret_cast<uint4 *>(E + e_chunk_off<512>(j, kc)) = make_uint4(o[0], o[1], o[2], o[3]);
-    }
-    return R;
-}
-
-template <int SF>
-__global__ void __launch_bounds__(pairk::THREADS, 1) attend_pair_kernel(AttArgs a) {
-    using namespace pairk;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *E0 = smem;                  // E'[b] at E0 + b E_BYTES
-    uint8_t *Qh = E0 + 2 * E_BYTES;
-    uint8_t *P0 = Qh + Q_BYTES;          // P'[b] at P0 + b P_BYTES
-    uint8_t *X = P0 + 2 * P_BYTES;
-    uint8_t *Y = X + X_BYTES;
-    uint8_t *misc = Y + Y_BYTES;
-    // barriers: E' full / free, S full / free (two buffers each; "E' free" of
-    // buffer b completes when the PV product of the tile in b does), X and Y
-    // received (arrived on by the peer), Q' loaded, the peer's row sums received.
-    // A wait for the PV of tile m on "E' free" of its buffer is unambiguous: the
-    // waiter has seen E'(m + 1) or E'(m + 2) full, and the conversion warps
-    // wrote those only after the PV of tile m - 1 or m - 2 had completed.
-    enum { B_EFULL = 0, B_EFREE = 2, B_SFULL = 4, B_SFREE = 6, B_X = 8, B_Y = 9, B_Q = 10, B_L = 11 };
-    uint64_t *mb = reinterpret_cast<uint64_t *>(misc);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + 128);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 132);
-    int *resc = reinterpret_cast<int *>(misc + 136);             // this CTA's heads need a rescale (this tile)
-    int *rjv = reinterpret_cast<int *>(misc + 256);              // [2][128] R_j per buffer (RJ_EMPTY: padding)
-    float *rho = reinterpret_cast<float *>(misc + 1280);         // [32] reference of this CTA's heads
-    float *alpha = reinterpret_cast<float *>(misc + 1408);       // [32] rescale factors of this tile
-    float *wred = reinterpret_cast<float *>(misc + 1536);        // [4 lane quarters][32 heads]
-    float *lpeer = reinterpret_cast<float *>(misc + 2048);       // [32] row sums of the peer's heads
-    float *lown = reinterpret_cast<float *>(misc + 2176);        // [32]
-    float *inv_l = reinterpret_cast<float *>(misc + 2304);       // [64]
-    const float *yalpha = reinterpret_cast<const float *>(Y + kTile * 64);     // [32] the peer's factors
-    const volatile int *yresc = reinterpret_cast<const volatile int *>(Y + kTile * 64 + 128);
-
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const uint32_t rank = cluster_ctarank(), peer = rank ^ 1;
-    grid_dep_wait();
-    const long long T = a.tprefix[a.Nq];
-    const int G = gridDim.x >> 1, c = blockIdx.x >> 1;
-    const long long t_begin = T * c / G, t_end = T * (c + 1) / G;
-    if (t_begin >= t_end) return;  // both CTAs of the pair
-
-    auto bar = [&](int k) { return smem_u32(&mb[k]); };
-    const uint32_t E_s = smem_u32(E0), Q_s = smem_u32(Qh), P_s = smem_u32(P0), X_s = smem_u32(X), Y_s = smem_u32(Y);
-    if (tid == 0) {
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(bar(B_EFULL + b), 128);
-            mbar_init(bar(B_EFREE + b), 1);
-            mbar_init(bar(B_SFULL + b), 1);
-            mbar_init(bar(B_SFREE + b), SG);
-        }
-        mbar_init(bar(B_X), 1);  // armed with the expected bytes by this CTA, filled by the peer's copy
-        mbar_init(bar(B_Y), 1);
-        mbar_init(bar(B_Q), 1);
-        mbar_init(bar(B_L), 32);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        *abort_flag = 0;
-        *resc = 0;
-    }
-    if (warp == 0) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                     "r"(TMEM_COLS)
-                     : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-    }
-    tc_fence_before();
-    __syncthreads();
-    cluster_sync_all();  // the peer's barriers are initialised before any remote arrive
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-    const uint32_t X_peer = mapa_shared(X_s, peer), Y_peer = mapa_shared(Y_s, peer);
-    const uint32_t bx_peer = mapa_shared(bar(B_X), peer), by_peer = mapa_shared(bar(B_Y), peer);
-    const uint32_t bl_peer = mapa_shared(bar(B_L), peer), lpeer_peer = mapa_shared(smem_u32(lpeer), peer);
-
-    constexpr uint32_t IDESC_S = idesc_f16(kTile, kHeads, false, false);
-    constexpr uint32_t IDESC_PV = idesc_f16(kTile, kHeads, true, true);
-    const int j = tid & (kTile - 1);  // entry row (softmax and conversion threads)
-    const int hq = (tid >> 7) & 1;    // softmax thread: heads [16 hq, 16 hq + 16) of this CTA's 32
-    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
-
-    // conversion warps: prefetch state (row loads one tile ahead, selected indices two ahead)
-    RowRegs<512> rr;
-    TileRef pcur, pnxt;
-    int pblk_nxt = -1;
-    if (tid >= SG) {
-        pcur = query_ref(a, a.cta_q[c], t_begin);
-        pair_prefetch_row<SF>(a, pcur, row_block_raw(a, pcur), rank, rr);
-        pnxt = pcur;
-        if (t_begin + 1 < t_end) {
-            pnxt = advance(a, pcur, t_begin + 1);
-            pblk_nxt = row_block_raw(a, pnxt);
-        }
-    }
-
-    uint32_t n = 0;      // tiles of this CTA before the current segment
-    uint32_t nseg = 0;   // segments before the current one
-    bool q_pending = false;
-    bool aborted = false;
-    TileRef seg = query_ref(a, a.cta_q[c], t_begin);
-    long long t = t_begin;
-    while (t < t_end) {
-        const int i = seg.i;
-        const long long seg_begin = t;
-        const long long seg_end = min(t_end, seg.t1);
-        const bool whole = (seg_begin == seg.t0) && (seg_end == seg.t1);
-        const uint32_t nt = (uint32_t)(seg_end - seg_begin);
-        bool ok = true;
-        float lsum[HPT];
-#pragma unroll
-        for (int k = 0; k < HPT; ++k) lsum[k] = 0.f;
-
-        if (tid >= SG) {
-            // ================= conversion warps: E'(t) for this CTA's channel half, then S(t)
-            if (tid == SG) {  // this segment's half of the Q' image (the previous segment's S MMAs are complete)
-                mbar_expect_tx(bar(B_Q), Q_BYTES);
-                bulk_g2s(Q_s, a.qimg + (size_t)i * (kHeads * D * 2) + rank * Q_BYTES, Q_BYTES, bar(B_Q));
-                q_pending = true;
-            }
-            for (uint32_t k = 0; k < nt; ++k) {
-                const uint32_t m = n + k, b = m & 1;
-                if (m >= 2) ok = mbar_wait_ab<false>(bar(B_EFREE + b), ((m >> 1) - 1) & 1, abort_flag);
-                if (!ok) break;
-                uint8_t *Eb = E0 + b * E_BYTES;
-                int Rj;
-                bool valid;
-                if (pcur.win) {
-                    Rj = pair_window_row(a, pcur, rank, Eb, E_s + b * E_BYTES, valid);
-                } else {
-                    valid = rr.valid;
-                    Rj = pair_dequant<SF>(rr, rank, Eb);
-                }
-                rjv[b * kTile + j] = valid ? Rj : RJ_EMPTY;
-                fence_async_smem();
-                mbar_arrive(bar(B_EFULL + b));
-                if (warp == SG / 32) {  // S^T(t) over this CTA's channels, once every row of E'(t) is written
-                    if (lane == 0) {
-                        if (q_pending) {
-                            ok = mbar_wait_ab<false>(bar(B_Q), nseg & 1, abort_flag);
-                            if (ok) q_pending = false;
-                        }
-                        ok = ok && mbar_wait_ab<false>(bar(B_EFULL + b), (m >> 1) & 1, abort_flag);
-                        if (ok && m >= 2) ok = mbar_wait_ab<false>(bar(B_SFREE + b), ((m >> 1) - 1) & 1, abort_flag);
-                        if (ok) {
-                            tc_fence_after();
-#pragma unroll
-                            for (int kk = 0; kk < HC / 16; ++kk) {
-                                const uint32_t koff = (uint32_t)((kk & 3) * 32);
-                                const uint64_t da = desc_sw128(E_s + b * E_BYTES + (kk >> 2) * KREG + koff, 16, 1024);
-                                const uint64_t db = desc_sw128(Q_s + (kk >> 2) * QREG + koff, 16, 1024);
-                                mma_f16(tmem + 64 * b, da, db, IDESC_S, kk > 0);
-                            }
-                            mma_commit(bar(B_SFULL + b));
-                        }
-                    }
-                    ok = __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
-                    if (!ok) break;
-                }
-                const long long tt = seg_begin + k;
-                if (tt + 1 < t_end) {
-                    TileRef nxt2 = pnxt;
-                    int blk_nxt2 = -1;
-                    pair_prefetch_row<SF>(a, pnxt, pblk_nxt, rank, rr);
-                    if (tt + 2 < t_end) {
-                        nxt2 = advance(a, pnxt, tt + 2);
-                        blk_nxt2 = row_block_raw(a, nxt2);
-                    }
-                    pcur = pnxt;
-                    pnxt = nxt2;
-                    pblk_nxt = blk_nxt2;
-                }
-            }
-            if (!ok) *abort_flag = 1;
-        } else {
-            // ================= softmax warps: entry row j, heads 32 rank + 16 hq + (0..15)
-            const int sQ = a.sq[i];
-            bool first = true;
-            for (uint32_t k = 0; k < nt; ++k) {
-                const uint32_t m = n + k, b = m & 1;
-                ok = mbar_wait_ab<false>(bar(B_SFULL + b), (m >> 1) & 1, abort_flag) &&
-                     mbar_wait_ab<false>(bar(B_EFULL + b), (m >> 1) & 1, abort_flag);
-                if (bar_or_n<SG>(!ok)) { ok = false; break; }
-                tc_fence_after();
-                if (tid == 0) {  // this tile's exchanges: expected bytes from the peer
-                    mbar_expect_tx(bar(B_X), X_BYTES);
-                    mbar_expect_tx(bar(B_Y), Y_BYTES);
-                }
-                uint8_t *Pb = P0 + b * P_BYTES;
-                float u[HPT];
-                {
-                    float sp[HPT];
-                    tmem_ld16(tmem + lane_off + 64 * b + 32 * rank + HPT * hq, u);
-                    tmem_ld16(tmem + lane_off + 64 * b + 32 * peer + HPT * hq, sp);
-                    tc_fence_before();
-                    mbar_arrive(bar(B_SFREE + b));
-                    // the peer's heads: partial logits, row j with chunks swizzled by j, staged in P'[b]
-#pragma unroll
-                    for (int cc = 0; cc < 4; ++cc)
-                        *reinterpret_cast<float4 *>(Pb + j * 128 + (((4 * hq + cc) ^ (j & 7)) << 4)) =
-                            make_float4(sp[4 * cc], sp[4 * cc + 1], sp[4 * cc + 2], sp[4 * cc + 3]);
-                }
-                fence_async_smem();
-                bar_sync_n<SG>();
-                if (tid == 0) bulk_s2peer(X_peer, P_s + b * P_BYTES, X_BYTES, bx_peer);
-                ok = mbar_wait_ab<true>(bar(B_X), m & 1, abort_flag);
-                if (bar_or_n<SG>(!ok)) { ok = false; break; }
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    const float4 x = *reinterpret_cast<const float4 *>(X + j * 128 + (((4 * hq + cc) ^ (j & 7)) << 4));
-                    u[4 * cc] += x.x;
-                    u[4 * cc + 1] += x.y;
-                    u[4 * cc + 2] += x.z;
-                    u[4 * cc + 3] += x.w;
-                }
-                const int rj_raw = rjv[b * kTile + j];
-                const bool valid = rj_raw != RJ_EMPTY;
-                const int Rj = valid ? rj_raw : 0;
-                const float cj = ldexpf(a.scale_log2, Rj + sQ);
-                const float rjf = (float)Rj;
-                const float *rh = rho + HPT * hq;
-#pragma unroll
-                for (int k2 = 0; k2 < HPT; ++k2) u[k2] = valid ? fmaf(u[k2], cj, rjf) : -INFINITY;
-                float over = -INFINITY;
-#pragma unroll
-                for (int k2 = 0; k2 < HPT; k2 += 4) {
-                    const float4 r4 = *reinterpret_cast<const float4 *>(rh + k2);
-                    over = fmaxf(over, fmaxf(fmaxf(u[k2] - r4.x, u[k2 + 1] - r4.y), fmaxf(u[k2 + 2] - r4.z, u[k2 + 3] - r4.w)));
-                }
-                int resc_own = 0;
-                if (bar_or_n<SG>(first || over > 8.f)) {
-                    {
-                        float mm[HPT];
-#pragma unroll
-                        for (int k2 = 0; k2 < HPT; ++k2) mm[k2] = u[k2];
-                        transpose_reduce<HPT, true>(mm);  // lane L: head 16 hq + L % 16 over this warp's entries
-                        if (lane < HPT) wred[(warp & 3) * 32 + HPT * hq + lane] = mm[0];
-                    }
-                    if (tid == 0) *resc = 0;
-                    bar_sync_n<SG>();
-                    if (tid < 32) {
-                        const float M = fmaxf(fmaxf(wred[tid], wred[32 + tid]), fmaxf(wred[64 + tid], wred[96 + tid]));
-                        float al = 1.f;
-                        if (first) {
-                            rho[tid] = M;
-                        } else if (M > rho[tid] + 8.f) {
-                            al = rho[tid] == -INFINITY ? 0.f : exp2f(rho[tid] - M);
-                            rho[tid] = M;
-                        }
-                        alpha[tid] = al;
-                        if (al != 1.f) *resc = 1;
-                    }
-                    bar_sync_n<SG>();
-                    resc_own = *resc;
-                    if (resc_own) {  // the row sums so far were taken against the old reference
-#pragma unroll
-                        for (int k2 = 0; k2 < HPT; ++k2) lsum[k2] *= alpha[HPT * hq + k2];
-                    }
-                }
-                // ---- P' = 2^(u - rho) of this thread's heads: kept in registers, staged in X for the peer
-                uint32_t pk[HPT / 2];
-                {
-                    const float rj_inv = ldexpf(1.0f, -Rj);
-#pragma unroll
-                    for (int q2 = 0; q2 < HPT / 2; ++q2) {
-                        const int k2 = 2 * q2;
-                        const float2 r2 = *reinterpret_cast<const float2 *>(rh + k2);
-                        const float p0 = valid ? exp2f(u[k2] - r2.x) : 0.f;
-                        const float p1 = valid ? exp2f(u[k2 + 1] - r2.y) : 0.f;
-                        __half2 hh = __floats2half2_rn(p0, p1);
-                        pk[q2] = *reinterpret_cast<uint32_t *>(&hh);
-                        lsum[k2] = fmaf(p0, rj_inv, lsum[k2]);
-                        lsum[k2 + 1] = fmaf(p1, rj_inv, lsum[k2 + 1]);
-                    }
-#pragma unroll
-                    for (int cc = 0; cc < 2; ++cc)
-                        *reinterpret_cast<uint4 *>(X + j * 64 + (((2 * hq + cc) ^ ((j >> 1) & 3)) << 4)) =
-                            make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
-                    float *hdr = reinterpret_cast<float *>(X + kTile * 64);
-                    if (tid < 32) hdr[tid] = resc_own ? alpha[tid] : 1.f;
-                    if (tid == 0) reinterpret_cast<int *>(hdr)[32] = resc_own;
-                }
-                fence_async_smem();
-                bar_sync_n<SG>();
-                if (tid == 0) bulk_s2peer(Y_peer, X_s, Y_BYTES, by_peer);
-                ok = mbar_wait_ab<true>(bar(B_Y), m & 1, abort_flag);
-                if (bar_or_n<SG>(!ok)) { ok = false; break; }
-                {  // P'[b]: this thread's head chunks from registers, the peer's from Y
-#pragma unroll
-                    for (int cc = 0; cc < 2; ++cc) {
-                        const int co = 4 * (int)rank + 2 * hq + cc, cp = 4 * (int)peer + 2 * hq + cc;
-                        *reinterpret_cast<uint4 *>(Pb + (j >> 3) * 1024 + (j & 7) * 128 + ((co ^ (j & 7)) << 4)) =
-                            make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
-                        *reinterpret_cast<uint4 *>(Pb + (j >> 3) * 1024 + (j & 7) * 128 + ((cp ^ (j & 7)) << 4)) =
-                            *reinterpret_cast<const uint4 *>(Y + j * 64 + (((2 * hq + cc) ^ ((j >> 1) & 3)) << 4));
-                    }
-                }
-                const int resc_peer = *yresc;
-                if (resc_own || resc_peer) {
-                    // O^T holds PV(t-1) once it completes; rescale every head whose reference rose.
-                    // Thread (j, hq) takes d-tile hq of its TMEM lane (channel).
-                    ok = mbar_wait_ab<false>(bar(B_EFREE + ((m - 1) & 1)), ((m - 1) >> 1) & 1, abort_flag);
-                    if (bar_or_n<SG>(!ok)) { ok = false; break; }
-                    tc_fence_after();
-#pragma unroll 1
-                    for (int hh = 0; hh < 2; ++hh) {
-                        const bool mine = hh == (int)rank;
-                        if (mine ? !resc_own : !resc_peer) continue;
-#pragma unroll 1
-                        for (int q = 0; q < 2; ++q) {
-                            float o[16];
-                            const uint32_t col = tmem + lane_off + 128 + 64 * hq + 32 * hh + 16 * q;
-                            tmem_ld16(col, o);
-#pragma unroll
-                            for (int k2 = 0; k2 < 16; ++k2) o[k2] *= mine ? alpha[16 * q + k2] : yalpha[16 * q + k2];
-                            tmem_st16(col, o);
-                        }
-                    }
-                }
-                // ---- PV(t): O^T += E'(t)^T P'(t) over this CTA's channels, once all of P'(t) is written
-                fence_async_smem();
-                tc_fence_before();
-                bar_sync_n<SG>();
-                if (tid == 0) {
-                    tc_fence_after();
-#pragma unroll
-                    for (int dt = 0; dt < 2; ++dt) {
-#pragma unroll
-                        for (int kj = 0; kj < kTile / 16; ++kj) {
-                            const uint64_t da = desc_sw128(E_s + b * E_BYTES + (2 * dt) * KREG + kj * 2048, KREG, 1024);
-                            const uint64_t db = desc_sw128(P_s + b * P_BYTES + kj * 2048, 8192, 1024);
-                            mma_f16(tmem + 128 + 64 * dt, da, db, IDESC_PV, (first && kj == 0) ? 0u : 1u);
-                        }
-                    }
-                    mma_commit(bar(B_EFREE + b));
-                }
-                first = false;
-            }
-            if (!ok) *abort_flag = 1;
-        }
-
-        // ---------------- segment epilogue (all warps)
-        if (__syncthreads_or(!ok)) { aborted = true; break; }
-        {  // the segment's last PV (and with it every earlier tensor-core operation) is complete
-            const uint32_t m = n + nt - 1;
-            ok = mbar_wait_ab<false>(bar(B_EFREE + (m & 1)), (m >> 1) & 1, abort_flag);
-        }
-        if (__syncthreads_or(!ok)) { aborted = true; break; }
-        tc_fence_after();
-        if (tid < SG) {
-            transpose_reduce<HPT, false>(lsum);  // lane L: head 16 hq + L % 16 over this warp's entries
-            if (lane < HPT) wred[(warp & 3) * 32 + HPT * hq + lane] = lsum[0];
-            bar_sync_n<SG>();
-            if (tid < 32) {
-                const float l = wred[tid] + wred[32 + tid] + wred[64 + tid] + wred[96 + tid];
-                lown[tid] = l;
-                st_cluster_u32(lpeer_peer + 4 * tid, __float_as_uint(l));
-                mbar_arrive_remote(bl_peer);
-            }
-        }
-        ok = mbar_wait_ab<true>(bar(B_L), nseg & 1, abort_flag);
-        if (__syncthreads_or(!ok)) { aborted = true; break; }
-        if (tid < 64) {
-            const float l = (tid >> 5) == (int)rank ? lown[tid & 31] : lpeer[tid & 31];
-            inv_l[tid] = (whole && l > 0.f) ? 1.0f / l : 1.f;
-        }
-        __syncthreads();
-        const int b_slot = 2 * c + ((seg_begin == T * c / G) ? 0 : 1);
-        if (tid < SG) {  // O^T d-tile warp / 4, TMEM lanes 32 (warp % 4) ..: channel of this lane
-            const int dt = warp >> 2;
-            const int ch = HC * (int)rank + 128 * dt + 32 * (warp & 3) + lane;
-            float *dst = whole ? a.out + (size_t)i * a.H * D : a.part_o + (size_t)b_slot * kHeads * D;
-            const int nh = whole ? a.H : kHeads;
-#pragma unroll 1
-            for (int hh = 0; hh < 2; ++hh) {
-                float o[32];
-                tmem_ld32(tmem + lane_off + 128 + 64 * dt + 32 * hh, o);
-#pragma unroll
-                for (int k2 = 0; k2 < 32; ++k2) {
-                    const int h = 32 * hh + k2;
-                    if (h < nh) dst[(size_t)h * D + ch] = o[k2] * inv_l[h];
-                }
-            }
-        }
-        if (tid < 32) {
-            const int h = 32 * (int)rank + tid;
-            if (whole) {
-                if (a.lse && h < a.H) {
-                    const float l = lown[tid];
-                    a.lse[(size_t)i * a.H + h] = l > 0.f ? (rho[tid] + log2f(l)) * 0.69314718055994531f : -INFINITY;
-                }
-            } else {
-                a.part_rho[(size_t)b_slot * kHeads + h] = rho[tid];
-                a.part_l[(size_t)b_slot * kHeads + h] = lown[tid];
-            }
-        }
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        n += nt;
-        ++nseg;
-        t = seg_end;
-        if (t < t_end) seg = advance(a, seg, t);
-    }
-
-    if (aborted) {
-        if (tid == 0) flag(a.status, CSA_DEV_TIMEOUT);
-        if (tid == SG) {
-            if (q_pending) mbar_wait(bar(B_Q), nseg & 1);  // no copy may land after the CTA exits
-            // let tensor-core work already issued finish before TMEM is released
-            const long long t0 = clock64();
-            while (clock64() - t0 < 2000000) {
-            }
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    cluster_sync_all();  // the peer no longer touches this CTA's shared memory
-    tc_fence_after();
-    if (warp == 0)
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
-}
-
-template <int SF>
-cudaError_t launch_pair(const AttArgs &a, int pairs, cudaStream_t s) {
-    cudaError_t err;
-    if ((err = cudaFuncSetAttribute(attend_pair_kernel<SF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    pairk::SMEM)) != cudaSuccess)
-        return err;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * pairs);
-    cfg.blockDim = dim3(pairk::THREADS);
-    cfg.dynamicSmemBytes = pairk::SMEM;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, attend_pair_kernel<SF>, a);
-}
-
-// Number of CTA pairs that are resident at once (at most num_sms / 2), from the
-// occupancy calculator for the pair kernel's cluster shape; cached per device.
-template <int SF>
-int pair_count(int num_sms) {
-    static int cached[64] = {0};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return num_sms / 2;
-    if (cached[dev] > 0) return cached[dev];
-    int pairs = num_sms / 2;
-    if (cudaFuncSetAttribute(attend_pair_kernel<SF>, cudaFuncAttributeMaxDynamicSharedMemorySize, pairk::SMEM) ==
-        cudaSuccess) {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(2 * pairs);
-        cfg.blockDim = dim3(pairk::THREADS);
-        cfg.dynamicSmemBytes = pairk::SMEM;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = 2;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        int clusters = 0;
-        if (cudaOccupancyMaxActiveClusters(&clusters, attend_pair_kernel<SF>, &cfg) == cudaSuccess && clusters > 0)
-            pairs = min(pairs, clusters);
-    }
-    cudaGetLastError();
-    cached[dev] = pairs;
-    return pairs;
-}
-
-// CSA_ATTEND_KERNEL=pair (read once per process) runs D = 512 on CTA pairs;
-// the one-CTA kernel is the default (the faster of the two as measured).
-bool use_pair_kernel() {
-    static const int mode = [] {
-        const char *e = getenv("CSA_ATTEND_KERNEL");
-        return (e && strcmp(e, "pair") == 0) ? 1 : 0;
-    }();
-    return mode == 1;
-}
-
 template <int D, int SF>
 cudaError_t launch_main(const AttArgs &a, int num_ctas, cudaStream_t s) {
     cudaError_t err;
@@ -1691,16 +1042,8 @@ cudaError_t launch_attend(const csa_cache &c, const void *q, int Nq, int H, cons
     cudaError_t err;
     const int32_t *qp = sel_idx ? nullptr : q_pos;
     const int32_t *wl = win_kv ? win_len : nullptr;
-    int G = num_ctas;  // work ranges: CTAs, or CTA pairs for the pair kernel
-    if (D == 512 && use_pair_kernel()) {
-        const bool e4 = c.scale_fmt == CSA_SCALE_E4M3_16;
-        G = e4 ? pair_count<kScaleE4M3x16>(num_ctas) : pair_count<kScaleE8M0x32>(num_ctas);
-        if ((err = launch_schedule<512>(c, a, q_offsets, qp, wl, topk, max_win, q, G, qinfo, tprefix, cta_q, sq, qimg,
-                                        s)) != cudaSuccess)
-            return err;
-        err = e4 ? launch_pair<kScaleE4M3x16>(a, G, s) : launch_pair<kScaleE8M0x32>(a, G, s);
-        if (err != cudaSuccess) return err;
-    } else if (D == 512) {
+    const int G = num_ctas;  // work ranges, one per CTA
+    if (D == 512) {
         if ((err = launch_schedule<512>(c, a, q_offsets, qp, wl, topk, max_win, q, num_ctas, qinfo, tprefix, cta_q, sq,
                                         qimg, s)) != cudaSuccess)
             return err;

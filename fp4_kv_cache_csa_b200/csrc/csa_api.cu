@@ -65,6 +65,25 @@ csa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? CSA_OK : CSA_ERR
 
 }  // namespace
 
+// Argument checks of every indexer call (csa_index_topk, its pool and Reindex
+// forms, and csa_index_topk_noalloc in noalloc.cu), in the order the status
+// codes are reported; the workspace is checked by each caller afterwards.
+namespace csa {
+csa_status check_index_args(const csa_cache *cache, const void *q_idx, const float *w, int32_t n_queries,
+                            int32_t idx_heads, const int32_t *q_offsets, const int32_t *q_pos, int32_t topk,
+                            const int32_t *sel_idx) {
+    csa_status st = check_cache(cache);
+    if (st != CSA_OK) return st;
+    if (!cache->idx_key || !q_idx || !w || !q_offsets || !q_pos || !sel_idx) return CSA_ERR_NULL;
+    if (n_queries < 1 || idx_heads < 1 || topk < 1) return CSA_ERR_SHAPE;
+    if (idx_heads > 8 || topk > kMaxTopk) return CSA_ERR_UNSUPPORTED;
+    if (!aligned(q_idx, 16) || !aligned(w, 4) || !aligned(q_offsets, 4) || !aligned(q_pos, 4) ||
+        !aligned(sel_idx, 4))
+        return CSA_ERR_ALIGN;
+    return CSA_OK;
+}
+}  // namespace csa
+
 extern "C" {
 
 const char *csa_status_string(int32_t status) {
@@ -104,14 +123,9 @@ size_t csa_index_topk_workspace(const csa_cache *cache, int32_t n_queries, int32
 csa_status csa_index_topk(const csa_cache *cache, const void *q_idx, const float *w, int32_t n_queries,
                           int32_t idx_heads, const int32_t *q_offsets, const int32_t *q_pos, int32_t topk,
                           int32_t *sel_idx, void *workspace, size_t workspace_bytes, csa_stream_t stream) {
-    csa_status st = check_cache(cache);
+    const csa_status st = csa::check_index_args(cache, q_idx, w, n_queries, idx_heads, q_offsets, q_pos, topk,
+                                                 sel_idx);
     if (st != CSA_OK) return st;
-    if (!cache->idx_key || !q_idx || !w || !q_offsets || !q_pos || !sel_idx) return CSA_ERR_NULL;
-    if (n_queries < 1 || idx_heads < 1 || topk < 1) return CSA_ERR_SHAPE;
-    if (idx_heads > 8 || topk > kMaxTopk) return CSA_ERR_UNSUPPORTED;
-    if (!aligned(q_idx, 16) || !aligned(w, 4) || !aligned(q_offsets, 4) || !aligned(q_pos, 4) ||
-        !aligned(sel_idx, 4))
-        return CSA_ERR_ALIGN;
     const size_t need = csa::index_topk_workspace_bytes(n_queries, cache->capacity);
     if (!workspace || workspace_bytes < need) return CSA_ERR_WORKSPACE;
     if (!aligned(workspace, 256)) return CSA_ERR_ALIGN;
@@ -128,20 +142,6 @@ static int pool_shift_of(int32_t g) {
     return -1;
 }
 
-// Checks shared by the pool and Reindex calls.
-static csa_status check_index(const csa_cache *cache, const void *q_idx, const float *w, int32_t n_queries,
-                              int32_t idx_heads, const int32_t *q_offsets, const int32_t *q_pos, int32_t topk,
-                              const int32_t *sel_idx) {
-    csa_status st = check_cache(cache);
-    if (st != CSA_OK) return st;
-    if (!cache->idx_key || !q_idx || !w || !q_offsets || !q_pos || !sel_idx) return CSA_ERR_NULL;
-    if (n_queries < 1 || idx_heads < 1 || topk < 1) return CSA_ERR_SHAPE;
-    if (idx_heads > 8 || topk > kMaxTopk) return CSA_ERR_UNSUPPORTED;
-    if (!aligned(q_idx, 16) || !aligned(w, 4) || !aligned(q_offsets, 4) || !aligned(q_pos, 4) ||
-        !aligned(sel_idx, 4))
-        return CSA_ERR_ALIGN;
-    return CSA_OK;
-}
 
 static bool pool_sizes_ok(int32_t pool_group, int32_t pool_blocks) {
     return pool_shift_of(pool_group) >= 0 && pool_blocks >= 1 && pool_blocks <= kMaxTopk &&
@@ -160,7 +160,7 @@ csa_status csa_index_topk_pool(const csa_cache *cache, const void *q_idx, const 
                                int32_t idx_heads, const int32_t *q_offsets, const int32_t *q_pos, int32_t topk,
                                int32_t *sel_idx, int32_t pool_group, int32_t pool_blocks, int32_t *pool_blk,
                                void *workspace, size_t workspace_bytes, csa_stream_t stream) {
-    csa_status st = check_index(cache, q_idx, w, n_queries, idx_heads, q_offsets, q_pos, topk, sel_idx);
+    csa_status st = csa::check_index_args(cache, q_idx, w, n_queries, idx_heads, q_offsets, q_pos, topk, sel_idx);
     if (st != CSA_OK) return st;
     if (!pool_blk) return CSA_ERR_NULL;
     if (pool_shift_of(pool_group) < 0 || pool_blocks < 1) return CSA_ERR_SHAPE;
@@ -187,7 +187,7 @@ csa_status csa_index_topk_reindex(const csa_cache *cache, const void *q_idx, con
                                   int32_t *sel_idx, int32_t pool_group, int32_t pool_blocks,
                                   const int32_t *pool_blk, void *workspace, size_t workspace_bytes,
                                   csa_stream_t stream) {
-    csa_status st = check_index(cache, q_idx, w, n_queries, idx_heads, q_offsets, q_pos, topk, sel_idx);
+    csa_status st = csa::check_index_args(cache, q_idx, w, n_queries, idx_heads, q_offsets, q_pos, topk, sel_idx);
     if (st != CSA_OK) return st;
     if (!pool_blk) return CSA_ERR_NULL;
     if (pool_shift_of(pool_group) < 0 || pool_blocks < 1) return CSA_ERR_SHAPE;

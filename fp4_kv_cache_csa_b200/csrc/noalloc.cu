@@ -21,6 +21,13 @@
 
 #include "../../include/csa.h"
 
+namespace csa {
+// csa_api.cu: the argument checks every indexer call makes, in the same order.
+csa_status check_index_args(const csa_cache *cache, const void *q_idx, const float *w, int32_t n_queries,
+                            int32_t idx_heads, const int32_t *q_offsets, const int32_t *q_pos, int32_t topk,
+                            const int32_t *sel_idx);
+}  // namespace csa
+
 namespace {
 
 constexpr size_t kScratchBytes = size_t(32) << 20;  // 32 MiB on every device that loads the library
@@ -52,9 +59,12 @@ extern "C" csa_status csa_index_topk_noalloc(const csa_cache *cache, const void 
                                              int32_t n_queries, int32_t idx_heads, const int32_t *q_offsets,
                                              const int32_t *q_pos, int32_t topk, int32_t *sel_idx,
                                              csa_stream_t stream) {
-    const size_t need = csa_index_topk_workspace(cache, n_queries, topk);
-    if (need == 0) return cache ? CSA_ERR_SHAPE : CSA_ERR_NULL;
-    if (need > kScratchBytes) return CSA_ERR_WORKSPACE;  // these sizes do not fit the fixed scratch
+    // the same argument errors as csa_index_topk, reported first; then the size check
+    const csa_status arg = csa::check_index_args(cache, q_idx, w, n_queries, idx_heads, q_offsets, q_pos, topk,
+                                                 sel_idx);
+    if (arg != CSA_OK) return arg;
+    if (csa_index_topk_workspace(cache, n_queries, topk) > kScratchBytes)
+        return CSA_ERR_WORKSPACE;  // these sizes do not fit the fixed scratch
     void *scratch = nullptr;
     const csa_status st = scratch_address(&scratch);
     if (st != CSA_OK) return st;

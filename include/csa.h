@@ -23,9 +23,11 @@
  *
  * Conventions for every call:
  *   - Pointers inside csa_cache and every tensor argument are DEVICE pointers,
- *     owned by the caller. The library allocates no memory and keeps no state;
- *     scratch space is the caller's `workspace` (csa_index_topk_noalloc alone
- *     uses a fixed scratch array the library holds instead).
+ *     owned by the caller. The library allocates no memory. Scratch space is
+ *     the caller's `workspace`, and the calls keep no state between them --
+ *     except csa_index_topk_noalloc, which uses a fixed scratch array that the
+ *     library holds on every device that loads it, and caches that array's
+ *     device address per device after its first call there.
  *   - Every call checks its arguments on the host first. On an argument error
  *     it returns the error code and launches nothing.
  *   - Otherwise it enqueues its kernels on `stream` and returns CSA_OK without
@@ -189,7 +191,8 @@ csa_status csa_index_topk(const csa_cache *cache, const void *q_idx, const float
  *   - The scratch is one fixed 32 MiB array in device memory, held on every
  *     GPU that loads the library until the process exits. Sizes whose
  *     csa_index_topk_workspace() exceeds 32 MiB are rejected with
- *     CSA_ERR_WORKSPACE before anything is launched.
+ *     CSA_ERR_WORKSPACE before anything is launched; the argument checks of
+ *     csa_index_topk come first (same codes, same order).
  *   - The first call on each device looks up that array's device address
  *     (once, with the device current). Make that first call before any
  *     stream capture on the device.
@@ -273,10 +276,6 @@ size_t csa_attend_workspace(const csa_cache *cache, int32_t n_queries, int32_t h
  *   workspace  >= csa_attend_workspace(cache, n_queries, heads) bytes, 256-byte aligned;
  *              it holds an fp16 copy of every query (n_queries * 64 * dim * 2 bytes)
  *              and two partial outputs per SM
- * Kernel choice: with dim 512 and the environment variable CSA_ATTEND_KERNEL=pair
- * (read once per process) this call and hca_decode_attend run on two-CTA clusters
- * (half of the latent channels per CTA); results agree with the default kernel
- * within the same bound, not bit for bit.
  */
 csa_status csa_decode_attend(const csa_cache *cache, const void *q, int32_t n_queries, int32_t heads,
                              const int32_t *q_offsets, const int32_t *sel_idx, int32_t topk,

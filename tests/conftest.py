@@ -27,3 +27,17 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """How many near-tie exceptions each byte comparison used (tests/parity.py)."""
+    try:
+        import parity
+    except Exception:
+        return
+    if not parity.EXCEPTIONS:
+        return
+    tr = terminalreporter
+    tr.section("near-tie exceptions in byte comparisons")
+    for test, kind, count, total in parity.EXCEPTIONS:
+        tr.write_line(f"{count:8d} of {total:11d}  {kind:18s} {test}")

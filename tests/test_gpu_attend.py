@@ -225,30 +225,6 @@ def test_e4m3x16_hca_dense():
             128, win, ws, wl, scale_fmt=E4)
 
 
-PAIR_CASES = ("test_b2_d512_h64_k512", "test_long_selection_is_split_and_merged",
-              "test_padding_partial_window_and_window_only", "test_no_window_and_empty_query",
-              "test_out_of_range_index_is_flagged_and_skipped", "test_scale_spread_rows",
-              "test_hca_dense_8192_entries", "test_csa_with_all_blocks_equals_hca", "test_e4m3x16_csa_d512_h64",
-              "test_e4m3x16_full_scale_range_is_exact_in_fp16", "test_e4m3x16_hca_dense")
-
-
-def test_pair_kernel_parity():
-    # the two-CTA cluster kernel (opt-in through CSA_ATTEND_KERNEL=pair, read once per
-    # process) on every D = 512 case above and the full-size HCA case, in a child process
-    import os
-    import subprocess
-    import sys
-
-    here = os.path.dirname(os.path.abspath(__file__))
-    code = (f"import sys; sys.path[:0] = [{here!r}, {os.path.dirname(here)!r}]\n"
-            "import test_gpu_attend as t, test_gpu_fullsize as f\n"
-            f"for name in {PAIR_CASES!r}: getattr(t, name)()\n"
-            "f.test_hca_b64_1m_sampled()\n")
-    env = dict(os.environ, CSA_ATTEND_KERNEL="pair")
-    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=900)
-    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
-
-
 @pytest.mark.parametrize("D,H", [(128, 16), (512, 64)])
 def test_more_queries_than_ctas(D, H):
     # prefill-shaped calls: more queries than CTAs, ragged selection lengths (0 to 3 tiles of

@@ -30,8 +30,8 @@ def run(D, dI, m, idx_dtype, counts, base, cap, seed, gate_std=0.02, lognormal=0
     status = csa.csa_read_device_status(cache)
     got = dict(fp4=host(cache.fp4), scale=host(cache.scale), n_blocks=host(cache.n_blocks),
                idx_key=None if not dI else host(cache.idx_key))
-    ref["tol"] = parity.pooling_tolerance(kv, offs, base, m, cap)
-    ref["tol_idx"] = parity.pooling_tolerance(idx, offs, base, m, cap) if dI else None
+    ref["tol"] = parity.pooling_tolerance(kv, offs, base, m, cap, kv_bits=kv, w_g=wg)
+    ref["tol_idx"] = parity.pooling_tolerance(idx, offs, base, m, cap, kv_bits=kv, w_g=wg) if dI else None
     return ref, got, status
 
 

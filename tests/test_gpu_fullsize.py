@@ -169,12 +169,12 @@ def test_csa_b8_64k_from_tokens(scale_fmt):
     cache = csa.Cache.allocate(B, cap, D, m, dI, csa.CSA_IDX_BF16, scale_fmt=scale_fmt)
     csa.csa_compress_quantize(cache, dev(kv), dev(it), dev(wg), dev(offs))
     assert csa.csa_read_device_status(cache) == 0
-    tol = parity.pooling_tolerance(kv, offs, np.zeros(B, np.int64), m, cap)
+    tol = parity.pooling_tolerance(kv, offs, np.zeros(B, np.int64), m, cap, kv_bits=kv, w_g=wg)
     parity.check_mxfp4(host(cache.fp4).reshape(B * cap, -1), host(cache.scale).reshape(B * cap, -1),
                        ref["fp4"].reshape(B * cap, -1), ref["scale"].reshape(B * cap, -1),
                        ref["pooled"].reshape(B * cap, D), tol=tol.reshape(B * cap, D), scale_fmt=scale_fmt)
     parity.check_keys(host(cache.idx_key).view(np.uint16), ref["idx_key"].view(np.uint16).reshape(B, cap, dI),
-                      ref["pooled_idx"], "bf16", tol=parity.pooling_tolerance(it, offs, np.zeros(B, np.int64), m, cap))
+                      ref["pooled_idx"], "bf16", tol=parity.pooling_tolerance(it, offs, np.zeros(B, np.int64), m, cap, kv_bits=kv, w_g=wg))
     # stage 2: indexer + top-k on the oracle's cache
     ocache = make_cache(ref["fp4"], ref["scale"], ref["n_blocks"], m, ref["idx_key"].view(np.uint16), 0,
                         scale_fmt=scale_fmt)
@@ -229,14 +229,14 @@ def test_prefill_b4_8k_sampled():
     assert csa.csa_read_device_status(cache) == 0
     assert np.array_equal(host(cache.n_blocks), ref["n_blocks"])
     new = slice(n0, cap)
-    tol = parity.pooling_tolerance(kv, offs, base, m, cap)[:, new]
+    tol = parity.pooling_tolerance(kv, offs, base, m, cap, kv_bits=kv, w_g=wg)[:, new]
     parity.check_mxfp4(host(cache.fp4)[:, new].reshape(-1, D // 2), host(cache.scale)[:, new].reshape(-1, D // 32),
                        ref["fp4"][:, new].reshape(-1, D // 2), ref["scale"][:, new].reshape(-1, D // 32),
                        ref["pooled"][:, new].reshape(-1, D), tol=tol.reshape(-1, D))
     assert np.array_equal(host(cache.fp4)[:, :n0], fp4[:, :n0])  # cached blocks untouched
     parity.check_keys(host(cache.idx_key).view(np.uint16)[:, new], ref["idx_key"].view(np.uint16)[:, new],
                       ref["pooled_idx"][:, new], "bf16",
-                      tol=parity.pooling_tolerance(it, offs, base, m, cap)[:, new])
+                      tol=parity.pooling_tolerance(it, offs, base, m, cap, kv_bits=kv, w_g=wg)[:, new])
     # stages 2 and 3 run on the oracle's new blocks behind the cached ones
     fp4[:, new], sc[:, new] = ref["fp4"][:, new], ref["scale"][:, new]
     keys[:, new] = ref["idx_key"].view(np.uint16)[:, new]

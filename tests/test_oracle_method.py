@@ -109,6 +109,116 @@ def test_pool_one_to_three_gate():
     np.testing.assert_allclose(r["pooled"][0, 0, 0], 0.75, rtol=1e-6)
 
 
+# ---- the pooled indexer key (same gate weights as the main KV) at m > 1
+#
+# The main-KV closed forms above are repeated on the indexer-key plane, whose
+# tokens are chosen independently of the main KV: the gate is a function of
+# the main KV alone, so a key pooled with its own channels as gate input, a
+# plain mean where the gate is not flat, or a key cast to E4M3 before pooling
+# rather than after, each fails one of these.
+
+def _e4m3_byte(x):
+    """E4M3 byte of a float (RNE, saturating at +-448) from PyTorch's own cast."""
+    import torch
+    v = float(np.clip(x, -448.0, 448.0))
+    return int(torch.tensor([v], dtype=torch.float32).to(torch.float8_e4m3fn).view(torch.uint8)[0])
+
+
+def _gated_block(m, logits_over_ln3, dI=32, seed=0):
+    """One block of m tokens whose gate logits are c_t * ln 3 (w_g = ln 3 on main-KV channel 0,
+    kv[t, 0] = c_t); the main KV's other channels are random, the indexer keys are set by the caller."""
+    g = np.random.default_rng(seed)
+    kv = g.standard_normal((m, 32)).astype(np.float32)
+    kv[:, 0] = np.asarray(logits_over_ln3, np.float32)
+    w = np.zeros(32, np.float32)
+    w[0] = np.float32(math.log(3.0))
+    return kv, w
+
+
+@pytest.mark.parametrize("m", [2, 4, 128])
+@pytest.mark.parametrize("idx_dtype", [0, 1])
+def test_pool_key_one_to_three_gate(m, idx_dtype):
+    # logits 0, ln 3, then -128 ln 3 for the rest: weights 1/4, 3/4 and ~1e-61 -> key 0.25 a + 0.75 b
+    c = np.full(m, -128.0, np.float32)
+    c[0], c[1] = 0.0, 1.0
+    kv, w = _gated_block(m, c)
+    idx = np.zeros((m, 32), np.float32)
+    idx[0, :4] = [8.0, -2.0, 0.5, 40.0]
+    idx[1, :4] = [16.0, 6.0, 0.5, 0.0]
+    idx[2:, :4] = 1000.0  # gated away: any weight they kept would show
+    r = _compress(kv, w, m, idx, idx_dtype=idx_dtype)
+    want = np.zeros(32)
+    want[:4] = [14.0, 4.0, 0.5, 10.0]
+    np.testing.assert_allclose(r["pooled_idx"][0, 0], want, rtol=1e-6, atol=1e-30)
+    key = r["idx_key"][0, 0]
+    if idx_dtype == 0:
+        assert np.array_equal(key.view(np.uint16), bf16(want))
+    else:
+        assert [int(b) for b in key[:4]] == [_e4m3_byte(v) for v in want[:4]]
+        assert np.all(key[4:] == 0)
+
+
+@pytest.mark.parametrize("m", [2, 4, 128])
+@pytest.mark.parametrize("idx_dtype", [0, 1])
+def test_pool_key_dominant_gate_selects_the_token(m, idx_dtype):
+    g = np.random.default_rng(20 + m)
+    c = np.full(m, -100.0, np.float32)
+    hot = m // 2
+    c[hot] = 20.0  # logit 20 ln 3 against -100 ln 3: the other weights are below 1e-57
+    kv, w = _gated_block(m, c, seed=m)
+    idx = g.standard_normal((m, 64)).astype(np.float32) * 4.0
+    r = _compress(kv, w, m, idx, idx_dtype=idx_dtype)
+    tok = bf16_val(bf16(idx[hot]))
+    np.testing.assert_array_equal(r["pooled_idx"][0, 0].astype(np.float64), tok)
+    key = r["idx_key"][0, 0]
+    if idx_dtype == 0:
+        assert np.array_equal(key.view(np.uint16), bf16(idx[hot]))
+    else:
+        assert [int(b) for b in key] == [_e4m3_byte(v) for v in tok]
+
+
+@pytest.mark.parametrize("m", [2, 4, 128])
+def test_pool_key_zero_gate_is_the_mean(m):
+    g = np.random.default_rng(30 + m)
+    kv = g.standard_normal((3 * m, 32)).astype(np.float32)
+    idx = g.standard_normal((3 * m, 48)).astype(np.float32)
+    r = _compress(kv, np.zeros(32), m, idx)
+    mean = bf16_val(bf16(idx)).reshape(3, m, 48).mean(axis=1)
+    np.testing.assert_allclose(r["pooled_idx"][0, :3], mean.astype(np.float32), rtol=2 ** -22, atol=1e-30)
+    # the stored bf16 key is the RNE rounding of that float32 mean
+    assert np.array_equal(r["idx_key"][0, :3].view(np.uint16), bf16(r["pooled_idx"][0, :3]))
+
+
+def test_pool_key_e4m3_is_cast_after_pooling():
+    # keys 0 and 1000 under a flat gate: the mean 500 saturates to 448; casting each token first
+    # (0 and 448) would give 224
+    kv = np.zeros((2, 32), np.float32)
+    idx = np.zeros((2, 32), np.float32)
+    idx[1, 0] = 1000.0
+    idx[0, 1], idx[1, 1] = 3.0, 5.0  # mean 4 (E4M3 exact)
+    r = _compress(kv, np.zeros(32), 2, idx, idx_dtype=1)
+    key = r["idx_key"][0, 0]
+    assert int(key[0]) == _e4m3_byte(448.0) == 0x7E
+    assert int(key[1]) == _e4m3_byte(4.0)
+
+
+@pytest.mark.parametrize("m", [2, 4, 128])
+@pytest.mark.parametrize("idx_dtype", [0, 1])
+def test_pool_key_constant_block_gives_the_token(m, idx_dtype):
+    g = np.random.default_rng(40 + m)
+    tok = g.standard_normal((3, 40)).astype(np.float32)
+    idx = np.repeat(tok, m, axis=0)
+    kv = g.standard_normal((3 * m, 32)).astype(np.float32)  # any gate: the weights sum to one
+    r = _compress(kv, g.standard_normal(32), m, idx, idx_dtype=idx_dtype)
+    tv = bf16_val(bf16(tok))
+    np.testing.assert_allclose(r["pooled_idx"][0, :3].astype(np.float64), tv, rtol=2 ** -22, atol=0)
+    key = r["idx_key"][0, :3]
+    if idx_dtype == 0:
+        assert np.array_equal(key.view(np.uint16), bf16(tok))
+    else:
+        assert [int(b) for b in key.reshape(-1)] == [_e4m3_byte(v) for v in tv.reshape(-1)]
+
+
 def test_pool_token_order_within_block_does_not_matter():
     g = np.random.default_rng(13)
     kv = g.standard_normal((4, 256)).astype(np.float32)

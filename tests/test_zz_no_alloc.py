@@ -17,7 +17,10 @@ from fp4_kv_cache_csa_b200 import datagen
 ERR_WORKSPACE = 5
 
 
-def _inputs(seed, lengths, dI, idx_dtype, k):
+def _inputs(seed, lengths, dI, idx_dtype, k, per_req=1):
+    """A cache of random keys; per_req queries per request: one decode query at the end of the
+    context (per_req = 1), or per_req queries at spread positions (a prefill-shaped call, which the
+    library scores with a tensor-core GEMM and selects per row)."""
     import torch
 
     from gpu_util import dev, make_cache
@@ -28,19 +31,29 @@ def _inputs(seed, lengths, dI, idx_dtype, k):
     keys = datagen.to_bf16_bits(x) if idx_dtype == 0 else datagen.to_e4m3_bytes(x)
     cache = make_cache(np.zeros((B, cap, 64), np.uint8), np.zeros((B, cap, 4), np.uint8), lengths, 4, keys,
                        idx_dtype)
-    q_idx = dev(datagen.normal_bf16((B, 4, dI), seed, 2))
-    w = dev(datagen.normal_f32((B, 4), seed, 3, std=0.5))
-    qo = dev(np.arange(B + 1, dtype=np.int32))
-    qp = dev((np.asarray(lengths) * 4 - 1).astype(np.int32))
+    Nq = B * per_req
+    q_idx = dev(datagen.normal_bf16((Nq, 4, dI), seed, 2))
+    w = dev(datagen.normal_f32((Nq, 4), seed, 3, std=0.5))
+    qo = dev((np.arange(B + 1) * per_req).astype(np.int32))
+    if per_req == 1:
+        pos = np.asarray(lengths) * 4 - 1
+    else:
+        rng = datagen.generator(seed, 4)
+        pos = np.concatenate([np.sort(rng.integers(0, 4 * n, per_req)) for n in lengths])
+        pos[::per_req] = 4 * np.asarray(lengths) - 1  # each request's last query sees every block
+    qp = dev(pos.astype(np.int32))
     return cache, q_idx, w, qo, qp, torch
 
 
 @pytest.mark.gpu
 def test_noalloc_matches_the_workspace_call_twice_in_a_row():
-    cases = [(71, [5000, 16384, 700, 12001], 128, 1, 512),   # e4m3 keys, ragged
-             (72, [9000, 300, 16000], 64, 0, 1024)]           # bf16 keys, another shape
-    for seed, lengths, dI, dt, k in cases:  # two consecutive calls on the shared scratch
-        cache, q_idx, w, qo, qp, torch = _inputs(seed, lengths, dI, dt, k)
+    cases = [(71, [5000, 16384, 700, 12001], 128, 1, 512, 1),   # e4m3 keys, ragged decode
+             (72, [9000, 300, 16000], 64, 0, 1024, 1),          # bf16 keys, another shape
+             (73, [8192, 6000], 128, 0, 512, 32),               # prefill-shaped, right after decode
+             (74, [3000, 7000, 200], 64, 1, 256, 1)]            # decode again, after the prefill call
+    for seed, lengths, dI, dt, k, per_req in cases:  # consecutive calls on the shared scratch
+        cache, q_idx, w, qo, qp, torch = _inputs(seed, lengths, dI, dt, k, per_req)
+        assert csa.csa_index_topk_workspace(cache, q_idx.shape[0], k) <= (32 << 20)
         want = csa.csa_index_topk(cache, q_idx, w, qo, qp, k)
         got = torch.full_like(want, -7)
         csa.csa_index_topk_noalloc(cache, q_idx, w, qo, qp, k, got)
@@ -57,3 +70,10 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     assert lib.csa_index_topk_workspace(ctypes.byref(c), 32, 1024) > (32 << 20)
     st = lib.csa_index_topk_noalloc(ctypes.byref(c), 0x90000, 0xA0000, 32, 4, 0xB0000, 0xC0000, 1024, 0xD0000, None)
     assert st == ERR_WORKSPACE
+    # argument errors come first, with csa_index_topk's codes: top-k beyond the supported
+    # maximum, a NULL output, a misaligned query
+    for args, want in (((0x90000, 0xA0000, 32, 4, 0xB0000, 0xC0000, 5000, 0xD0000), 4),
+                       ((0x90000, 0xA0000, 32, 4, 0xB0000, 0xC0000, 1024, None), 1),
+                       ((0x90001, 0xA0000, 32, 4, 0xB0000, 0xC0000, 1024, 0xD0000), 3)):
+        assert lib.csa_index_topk_noalloc(ctypes.byref(c), *args, None) == want
+        assert lib.csa_index_topk(ctypes.byref(c), *args, 0x100000, 1 << 40, None) == want
