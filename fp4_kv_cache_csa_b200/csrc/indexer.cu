@@ -62,6 +62,8 @@ namespace {
 constexpr int kBins = 4096;        // histogram bins per level (12 bits)
 constexpr int kScanThreads = 512;  // 16 warps, one CTA per SM
 constexpr int kScanWarps = kScanThreads / 32;
+constexpr int kMaxScanCtas = 256;
+constexpr int kFusedScheduleQueries = 512;  // up to this many queries the scan computes its own schedule (= its threads)  // scan grid: min(SMs, this); sizes the per-(query, CTA) counts
 // Work units charged for starting a query in a scan range (query fragments,
 // histogram clear and flush, completion count): about as long as scanning this
 // many 16-key groups. The flat split counts them, so ranges that cross a query
@@ -93,6 +95,11 @@ struct IndexWs {
     uint32_t *cand_key;  // [Nq][ccap]
     int32_t *cand_idx;   // [Nq][ccap]
     float *scores;       // [Nq][cap]
+    // streamed decode: each scan CTA's candidates of each query it scanned, at the
+    // segment's own offset in the query's row, and their count per (query, CTA)
+    int32_t *seg_cnt;    // [Nq + kMaxScanCtas]: slot i + c for query i and scan CTA c
+    uint32_t *seg_key;   // [Nq][cap]
+    int32_t *seg_idx;    // [Nq][cap]
     size_t zero_bytes;
     int words, ccap;
 };
@@ -121,6 +128,9 @@ size_t carve(void *base, int Nq, int cap, IndexWs *w) {
     size_t o_ck = take(sizeof(uint32_t) * (size_t)ccap * Nq);
     size_t o_ci = take(sizeof(int32_t) * (size_t)ccap * Nq);
     size_t o_sc = take(sizeof(float) * (size_t)cap * Nq);
+    size_t o_scnt = take(sizeof(int32_t) * ((size_t)Nq + kMaxScanCtas));
+    size_t o_skey = take(sizeof(uint32_t) * (size_t)cap * Nq);
+    size_t o_sidx = take(sizeof(int32_t) * (size_t)cap * Nq);
     if (w) {
         char *b = static_cast<char *>(base);
         w->req = reinterpret_cast<int32_t *>(b + o_req);
@@ -134,6 +144,9 @@ size_t carve(void *base, int Nq, int cap, IndexWs *w) {
         w->cand_key = reinterpret_cast<uint32_t *>(b + o_ck);
         w->cand_idx = reinterpret_cast<int32_t *>(b + o_ci);
         w->scores = reinterpret_cast<float *>(b + o_sc);
+        w->seg_cnt = reinterpret_cast<int32_t *>(b + o_scnt);
+        w->seg_key = reinterpret_cast<uint32_t *>(b + o_skey);
+        w->seg_idx = reinterpret_cast<int32_t *>(b + o_sidx);
         w->zero_bytes = z1 - z0;
         w->words = words;
         w->ccap = ccap;
@@ -178,6 +191,35 @@ __global__ void schedule_kernel(const int32_t *q_offsets, const int32_t *q_pos, 
         carry += round_total;
         __syncthreads();
     }
+}
+
+// Exclusive prefix sum over the threads of a block (blockDim.x a multiple of 32,
+// at most 1024); every thread also gets the block total. Ends with a barrier,
+// so smem may be reused right away.
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *smem /* >= 32 */, uint32_t &total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    uint32_t x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) smem[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        uint32_t t = lane < nw ? smem[lane] : 0u;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, t, o);
+            if (lane >= o) t += y;
+        }
+        if (lane < nw) smem[lane] = t;
+    }
+    __syncthreads();
+    total = smem[nw - 1];
+    const uint32_t excl = x - v + (warp > 0 ? smem[warp - 1] : 0u);
+    __syncthreads();
+    return excl;
 }
 
 // ---------------------------------------------------------------- radix helper
@@ -281,16 +323,24 @@ struct ScanArgs {
     const float *w;               // [Nq][H_I]
     const int32_t *req, *n_vis;
     const long long *gprefix;
-    float *scores;                // [Nq][cap]
-    uint32_t *hist1;              // [Nq][4096]
-    uint32_t *done;               // [Nq]
-    int32_t *thresh;              // [Nq][3]
+    float *scores;                // [Nq][rows]
+    int32_t *seg_cnt;             // [Nq + kMaxScanCtas]
+    uint32_t *seg_key;            // [Nq][rows]
+    int32_t *seg_idx;             // [Nq][rows]
     int Nq, H_I, cap, topk;
     int rows;                     // score row stride (cap, or G*P for a pool)
     // pool mapping (Reindex): local key r of query i is cache block
     // G * pool[i][r / G] + r % G, G = 1 << pool_shift; null: r itself
     const int32_t *pool;
     int pool_shift, pool_p;
+    // fused schedule (calls of at most kFusedScheduleQueries queries): every CTA
+    // computes the per-query counts and the unit prefix itself, and CTA 0 stores
+    // them for the merge; otherwise schedule_kernel has written req, n_vis, gprefix
+    int fused;
+    const int32_t *q_offsets, *q_pos, *n_blocks, *n_vis_given;
+    int32_t *req_out, *n_vis_out;
+    long long *gprefix_out;
+    int batch, m;
 };
 
 // Dimension permutation. The dot product sums over all d_I channels, so the
@@ -310,19 +360,49 @@ struct ScanCfg {
 };
 
 // POOL: keys are pool positions (Reindex), mapped to cache blocks through a.pool.
-template <bool E4M3, int KS, bool POOL>
+// FUSED: the kernel computes the schedule itself (a.fused; at most kFusedScheduleQueries queries).
+template <bool E4M3, int KS, bool POOL, bool FUSED>
 __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a) {
     using C = ScanCfg<E4M3, KS>;
-    grid_dep_wait();    // the schedule kernel's ranges (programmatic launch)
+    grid_dep_wait();    // the schedule kernel's ranges, or the inputs of the fused schedule
     grid_dep_launch();
-    __shared__ uint32_t hist[kBins];
+    __shared__ __align__(16) uint32_t hist[kBins];
     __shared__ uint32_t scan_smem[32];
     __shared__ BinPick pick;
-    __shared__ int last_flag;
+    __shared__ long long s_gp[FUSED ? kFusedScheduleQueries + 1 : 1];
+    __shared__ int32_t s_req[FUSED ? kFusedScheduleQueries : 1], s_nv[FUSED ? kFusedScheduleQueries : 1];
+    __shared__ long long s_red[32];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
     const uint64_t pol_stream = policy_evict_first(), pol_keep = policy_evict_last();
-    const long long NG = a.gprefix[a.Nq];
+    const long long *const gprefix = FUSED ? s_gp : a.gprefix;
+    const int32_t *const req_of = FUSED ? s_req : a.req;
+    const int32_t *const nvis_of = FUSED ? s_nv : a.n_vis;
+    if constexpr (FUSED) {
+        // the schedule kernel's work for at most kFusedScheduleQueries queries, in every CTA
+        const int i = threadIdx.x;
+        long long units = 0;
+        if (i < a.Nq) {
+            const int b = request_of(a.q_offsets, a.batch, i);
+            const int n = a.n_vis_given ? (b < 0 ? 0 : a.n_vis_given[i])
+                                        : (b < 0 ? 0 : min(visible_blocks(a.q_pos[i], a.m, a.n_blocks[b]), a.rows));
+            s_req[i] = b;
+            s_nv[i] = n;
+            units = (n + 15) / 16;
+            if (units > 0) units += kSegCost;
+        }
+        const long long incl = block_inclusive_scan<long long>(units, s_red);
+        if (i < a.Nq) s_gp[i + 1] = incl;
+        if (i == 0) s_gp[0] = 0;
+        __syncthreads();
+        if (blockIdx.x == 0 && i < a.Nq) {  // for the merge kernel
+            a.req_out[i] = s_req[i];
+            a.n_vis_out[i] = s_nv[i];
+            a.gprefix_out[i + 1] = s_gp[i + 1];
+            if (i == 0) a.gprefix_out[0] = 0;
+        }
+    }
+    const long long NG = gprefix[a.Nq];
     long long gb = NG * blockIdx.x / gridDim.x;
     const long long ge = NG * (blockIdx.x + 1) / gridDim.x;
 
@@ -331,17 +411,17 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a) {
         int lo = 0, hi = a.Nq - 1;
         while (lo < hi) {
             int mid = (lo + hi + 1) >> 1;
-            if (a.gprefix[mid] <= gb) lo = mid; else hi = mid - 1;
+            if (gprefix[mid] <= gb) lo = mid; else hi = mid - 1;
         }
         const int i = lo;
-        const long long seg_end = min(ge, a.gprefix[i + 1]);
-        const int b = a.req[i];
-        const int n = a.n_vis[i];
+        const long long seg_end = min(ge, gprefix[i + 1]);
+        const int b = req_of[i];
+        const int n = nvis_of[i];
         // units [gb, seg_end) of query i: the first kSegCost units are its start cost
-        const long long ngroups = (n + 15) / 16;
-        const long long lg0 = max(gb - a.gprefix[i] - kSegCost, 0LL);   // local group index
-        const long long nloc = seg_end - a.gprefix[i] - kSegCost - lg0;  // groups of this query here
-        if (nloc <= 0) {  // the range holds only start-cost units of this query
+        const long long lg0 = max(gb - gprefix[i] - kSegCost, 0LL);   // local group index
+        const long long nloc = seg_end - gprefix[i] - kSegCost - lg0;  // groups of this query here
+        if (nloc <= 0) {  // the range holds only start-cost units of this query: no candidates
+            if (threadIdx.x == 0 && a.topk < n) a.seg_cnt[i + blockIdx.x] = 0;
             gb = seg_end;
             continue;
         }
@@ -423,9 +503,8 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a) {
                     const long long r = 16 * lg + g + 8 * half;
                     const bool ok = gv && r < n;
                     long long row = r;
-                    if (POOL && ok)
-                        row = ((long long)__ldg(prow + (r >> a.pool_shift)) << a.pool_shift) +
-                              (r & ((1 << a.pool_shift) - 1));
+                    if (POOL && ok)  // a plain load behind the bound check (never issued beyond the row)
+                        row = ((long long)prow[r >> a.pool_shift] << a.pool_shift) + (r & ((1 << a.pool_shift) - 1));
                     const uint4 *src = reinterpret_cast<const uint4 *>(kbase + row * C::KEY_BYTES + t * C::ROW_BYTES_T);
 #pragma unroll
                     for (int v = 0; v < C::NV; ++v) raw[uu][half][v] = ok ? ld_stream(src + v, pol_stream) : make_uint4(0, 0, 0, 0);
@@ -472,38 +551,367 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a) {
                 }
             }
         }
-        __syncthreads();
-        uint32_t *gh = a.hist1 + (size_t)i * kBins;
-        const volatile uint32_t *vh = hist;
-        for (int k = threadIdx.x; k < kBins; k += kScanThreads) {
-            const uint32_t c = vh[k];
-            if (c) atomicAdd(gh + k, c);
-        }
-        // the CTA that completes a query's scan finds its k-th key bin (no waiting:
-        // groups are counted, and only the one that brings the count to the total acts)
-        __threadfence();
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            const uint32_t total = (uint32_t)ngroups;
-            const uint32_t mine = (uint32_t)nloc;
-            last_flag = atomicAdd(a.done + i, mine) + mine == total;
-        }
-        __syncthreads();
-        if (last_flag && a.topk < n) {
-            __threadfence();
-            for (int k = threadIdx.x; k < kBins; k += kScanThreads) hist[k] = __ldcg(gh + k);
-            __syncthreads();
-            const BinPick p = pick_bin(hist, kBins, (uint32_t)a.topk, scan_smem, &pick);
-            if (threadIdx.x == 0) {
-                const bool all_at = p.above + p.at == (uint32_t)a.topk;  // the whole bin is selected
-                a.thresh[3 * i] = all_at ? p.bin - 1 : p.bin;            // bins above this are selected
-                a.thresh[3 * i + 1] = (int)p.above;
-                a.thresh[3 * i + 2] = all_at ? -1 : p.bin;                // bin refined by the final kernel
+        __syncthreads();  // the segment's scores and histogram are complete (global writes visible in the CTA)
+        // ---- this segment's candidates: every key of the segment whose top 12 key bits
+        // reach the bin of the segment's own k-th largest key. The query's top-k is a
+        // subset of the union over its segments (a key among the k best of the query is
+        // among the k best of its segment), so select_merge_kernel only looks at these.
+        // They go to the segment's own offset in the query's candidate row, in index
+        // order (one block-wide prefix per chunk of 8 keys per thread).
+        if (a.topk < n) {
+            const long long r0 = 16 * lg0;
+            const long long r1 = min(16 * (lg0 + nloc), (long long)n);
+            const uint32_t ns = (uint32_t)(r1 - r0);
+            const BinPick p = pick_bin(hist, kBins, min((uint32_t)a.topk, ns), scan_smem, &pick);
+            const uint32_t b0 = (uint32_t)p.bin;
+            uint32_t *ck = a.seg_key + (size_t)i * a.rows + r0;
+            int32_t *cj = a.seg_idx + (size_t)i * a.rows + r0;
+            const float *sr = srow + r0;
+            // 8 consecutive scores per thread per chunk (two 16-byte loads when the row is
+            // 16-byte aligned); the loads run three chunks ahead of the prefix and the stores,
+            // since the L2 answers slowly while the other CTAs still stream their keys
+            constexpr int kE = 8;
+            constexpr uint32_t kChunk = kScanThreads * kE;
+            const bool vec = ((reinterpret_cast<uintptr_t>(sr)) & 15) == 0;
+            const uint32_t nch = (ns + kChunk - 1) / kChunk;
+            uint32_t base = 0;
+            float v0[kE], v1[kE], v2[kE];
+            auto load_chunk = [&](float (&v)[kE], uint32_t c) {
+                const uint32_t r = c * kChunk + threadIdx.x * kE;
+                if (c >= nch) return;
+                if (vec && r + kE <= ns) {
+#pragma unroll
+                    for (int q = 0; q < kE / 4; ++q) {
+                        const float4 f = __ldcg(reinterpret_cast<const float4 *>(sr + r) + q);
+                        v[4 * q] = f.x; v[4 * q + 1] = f.y; v[4 * q + 2] = f.z; v[4 * q + 3] = f.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < kE; ++e) v[e] = r + e < ns ? __ldcg(sr + r + e) : 0.f;
+                }
+            };
+            // candidates of chunk c (block-uniform loop), in index order
+            auto take_chunk = [&](const float (&v)[kE], uint32_t c) {
+                if (c >= nch) return;
+                uint32_t key[kE], m = 0;
+#pragma unroll
+                for (int e = 0; e < kE; ++e) {
+                    const uint32_t r = c * kChunk + threadIdx.x * kE + e;
+                    key[e] = ordered_key(v[e]);
+                    if (r < ns && (key[e] >> 20) >= b0) m |= 1u << e;
+                }
+                uint32_t total;
+                uint32_t pos = base + block_excl_scan(__popc(m), scan_smem, total);
+#pragma unroll
+                for (int e = 0; e < kE; ++e) {
+                    if (m & (1u << e)) {
+                        ck[pos] = key[e];
+                        cj[pos] = (int32_t)(r0 + c * kChunk + threadIdx.x * kE + e);
+                        ++pos;
+                    }
+                }
+                base += total;
+            };
+            load_chunk(v0, 0);
+            load_chunk(v1, 1);
+            for (uint32_t c = 0; c < nch; c += 3) {
+                load_chunk(v2, c + 2);
+                take_chunk(v0, c);
+                load_chunk(v0, c + 3);
+                take_chunk(v1, c + 1);
+                load_chunk(v1, c + 4);
+                take_chunk(v2, c + 2);
             }
+            if (threadIdx.x == 0) a.seg_cnt[i + blockIdx.x] = (int32_t)base;  // = p.above + p.at
         }
         __syncthreads();
         gb = seg_end;
     }
+}
+
+// ---------------------------------------------------------------- merge (streamed decode)
+// One CTA per query: the exact top-k among the candidates the scan CTAs left
+// for it (their segments in CTA order, each in index order, so the candidates
+// are in ascending block index), by three radix levels on the key bits
+// (31..20, 19..8, 7..0) until the k-th largest key T is fixed; then the keys
+// above T and the first ties at T (lowest indices: the candidates' order) are
+// written in that order. Up to kMergeStage candidates are staged in shared
+// memory; more (few long queries spread over many CTAs) are read in place.
+constexpr int kMergeThreads = 1024;
+constexpr int kMergeStage = 24576;  // 192 KB of shared memory
+constexpr uint32_t kTakeAll = 0xFFFFFFFFu;
+
+struct MergeArgs {
+    const int32_t *n_vis;
+    const long long *gprefix;
+    const int32_t *seg_cnt;
+    const uint32_t *seg_key;
+    const int32_t *seg_idx;
+    int32_t *sel_idx;
+    int Nq, G, topk, rows;
+    // rows are pool positions (Reindex): position r is written as block
+    // G * pool[i][r / G] + r % G with G = 1 << pool_shift; null: r itself
+    const int32_t *pool;
+    int pool_shift, pool_p;
+};
+
+// Largest bin d of a histogram of nbins (a multiple of 32, at most 4096) bins
+// such that at least `need` elements lie in bins >= d, found by warp 0 alone
+// (lane l sums the nbins/32 bins below the top l*nbins/32), with the count
+// above d and in d. The histogram must be complete (after a barrier); every
+// thread gets the result.
+__device__ BinPick pick_bin_warp(const uint32_t *h, int nbins, uint32_t need, BinPick *out) {
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x, per = nbins >> 5;
+        const int top = nbins - 1 - lane * per;  // this lane: bins top, top - 1, ..., top - per + 1
+        uint32_t sum = 0;
+        for (int k = 0; k < per; ++k) sum += h[top - k];
+        uint32_t incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        const uint32_t excl = incl - sum;
+        if (excl < need && incl >= need) {
+            uint32_t run = excl;
+            for (int k = 0; k < per; ++k) {
+                const uint32_t c = h[top - k];
+                if (run + c >= need) {
+                    out->bin = top - k;
+                    out->above = run;
+                    out->at = c;
+                    break;
+                }
+                run += c;
+            }
+        }
+    }
+    __syncthreads();
+    const BinPick r = *out;
+    __syncthreads();
+    return r;
+}
+
+// Only called with a.pool set: the caller branches on it first (a load through
+// the pool pointer must never be issued, even speculatively, when it is null).
+__device__ __forceinline__ int32_t merge_pool_index(const MergeArgs &a, int i, int r) {
+    return (a.pool[(size_t)i * a.pool_p + (r >> a.pool_shift)] << a.pool_shift) + (r & ((1 << a.pool_shift) - 1));
+}
+
+// Position in the query's candidate row of candidate p (p < the candidates'
+// total): its CTA by binary search over the per-CTA prefix (pre[k] <= p).
+__device__ __forceinline__ uint32_t merge_row_pos(const uint32_t *pre, const uint32_t *off, int nseg, uint32_t p) {
+    int lo = 0, hi = nseg - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (pre[mid] <= p) lo = mid; else hi = mid - 1;
+    }
+    return off[lo] + (p - pre[lo]);
+}
+
+__global__ void __launch_bounds__(kMergeThreads) select_merge_kernel(MergeArgs a) {
+    extern __shared__ uint32_t mdyn[];  // [kMergeStage] keys, then [kMergeStage] indices
+    uint32_t *sk = mdyn;
+    int32_t *sj = reinterpret_cast<int32_t *>(mdyn + kMergeStage);
+    __shared__ __align__(16) uint32_t h[kBins];
+    __shared__ uint32_t scan_smem[32];
+    __shared__ BinPick pick;
+    __shared__ uint32_t s_pre[kMaxScanCtas + 1];  // candidates before each of the query's CTAs
+    __shared__ uint32_t s_off[kMaxScanCtas];      // where that CTA's candidates start in the row
+    grid_dep_wait();
+    const int i = blockIdx.x, tid = threadIdx.x;
+    const int n = a.n_vis[i];
+    const int K = min(a.topk, n);
+    int32_t *out = a.sel_idx + (size_t)i * a.topk;
+    if (K == n) {  // every visible block (or none)
+        if (a.pool) {
+            for (int r = tid; r < a.topk; r += kMergeThreads) out[r] = r < n ? merge_pool_index(a, i, r) : -1;
+        } else {
+            for (int r = tid; r < a.topk; r += kMergeThreads) out[r] = r < n ? r : -1;
+        }
+        return;
+    }
+    // the scan CTAs whose ranges hold this query's units [u0, u1), as the scan split them
+    const long long NG = a.gprefix[a.Nq], u0 = a.gprefix[i], u1 = a.gprefix[i + 1];
+    const int G = a.G;
+    const int c_first = (int)(((u0 + 1) * G - 1) / NG), c_last = (int)((u1 * G - 1) / NG);
+    const int nseg = c_last - c_first + 1;  // <= G <= kMaxScanCtas <= blockDim
+    uint32_t cnt = 0, off = 0;
+    if (tid < nseg) {
+        const int c = c_first + tid;
+        const long long s0 = NG * c / G, s1 = NG * (c + 1) / G;
+        const long long lg0 = max(s0 - u0 - kSegCost, 0LL);
+        const long long lend = min(s1, u1) - u0 - kSegCost;
+        if (s0 < s1 && lend > lg0) {
+            cnt = (uint32_t)a.seg_cnt[i + c];
+            off = (uint32_t)(16 * lg0);
+        }
+    }
+    uint32_t L;
+    const uint32_t pre = block_excl_scan(cnt, scan_smem, L);
+    if (tid < nseg) {
+        s_pre[tid] = pre;
+        s_off[tid] = off;
+    }
+    const uint32_t *gk = a.seg_key + (size_t)i * a.rows;
+    const int32_t *gj = a.seg_idx + (size_t)i * a.rows;
+    const bool staged = L <= (uint32_t)kMergeStage;
+    for (int k = tid; k < kBins; k += kMergeThreads) h[k] = 0u;
+    __syncthreads();
+    // ---- level 0 (and the staging copy: every load of the thread in flight at once)
+    if (staged) {
+        constexpr int kPer = 12;  // loads in flight per thread and round
+        for (uint32_t p0 = 0; p0 < L; p0 += kPer * kMergeThreads) {
+            uint32_t kk[kPer];
+            int32_t jj[kPer];
+#pragma unroll
+            for (int k = 0; k < kPer; ++k) {
+                const uint32_t p = p0 + tid + k * kMergeThreads;
+                if (p < L) {
+                    const uint32_t rp = merge_row_pos(s_pre, s_off, nseg, p);
+                    kk[k] = __ldcg(gk + rp);
+                    jj[k] = __ldcg(gj + rp);
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < kPer; ++k) {
+                const uint32_t p = p0 + tid + k * kMergeThreads;
+                if (p < L) {
+                    sk[p] = kk[k];
+                    sj[p] = jj[k];
+                    atomicAdd(&h[kk[k] >> 20], 1u);
+                }
+            }
+        }
+    } else {
+        for (uint32_t p = tid; p < L; p += kMergeThreads)
+            atomicAdd(&h[__ldcg(gk + merge_row_pos(s_pre, s_off, nseg, p)) >> 20], 1u);
+    }
+    __syncthreads();
+    BinPick pk = pick_bin(h, kBins, (uint32_t)K, scan_smem, &pick);
+    uint32_t T, take;
+    if (pk.above + pk.at == (uint32_t)K) {  // the whole bin
+        T = (uint32_t)pk.bin << 20;
+        take = kTakeAll;
+    } else {
+        const uint32_t b0 = (uint32_t)pk.bin;
+        uint32_t need = (uint32_t)K - pk.above;
+        for (int k = tid; k < kBins; k += kMergeThreads) h[k] = 0u;
+        __syncthreads();
+        for (uint32_t p = tid; p < L; p += kMergeThreads) {
+            uint32_t key;
+            if (staged) key = sk[p]; else key = __ldcg(gk + merge_row_pos(s_pre, s_off, nseg, p));
+            if ((key >> 20) == b0) atomicAdd(&h[(key >> 8) & 0xFFFu], 1u);
+        }
+        __syncthreads();
+        pk = pick_bin(h, kBins, need, scan_smem, &pick);
+        const uint32_t pre1 = (b0 << 12) | (uint32_t)pk.bin;
+        if (pk.above + pk.at == need) {
+            T = pre1 << 8;
+            take = kTakeAll;
+        } else {
+            need -= pk.above;
+            for (int k = tid; k < 256; k += kMergeThreads) h[k] = 0u;
+            __syncthreads();
+            for (uint32_t p = tid; p < L; p += kMergeThreads) {
+                uint32_t key;
+                if (staged) key = sk[p]; else key = __ldcg(gk + merge_row_pos(s_pre, s_off, nseg, p));
+                if ((key >> 8) == pre1) atomicAdd(&h[key & 0xFFu], 1u);
+            }
+            __syncthreads();
+            pk = pick_bin_warp(h, 256, need, &pick);
+            T = (pre1 << 8) | (uint32_t)pk.bin;
+            take = need - pk.above;  // ties at T to keep, lowest indices first (>= 1)
+        }
+    }
+    // ---- output in candidate order: keys above T, and the first `take` keys equal to T
+    if (staged) {
+        // warp w owns a contiguous run of the staged candidates: it counts its keys above T
+        // and at T, every warp learns the counts of the runs before its own, and each warp
+        // writes its selection at its offset (ballots, no block-wide scan per chunk)
+        __shared__ uint32_t w_gt[kMergeThreads / 32], w_eq[kMergeThreads / 32];
+        const int warp = tid >> 5, lane = tid & 31;
+        const uint32_t seg = (((L + 31) >> 5) + 31) & ~31u;
+        const uint32_t w0 = min(L, warp * seg), w1 = min(L, w0 + seg);
+        uint32_t ngt = 0, neq = 0;
+        for (uint32_t base = w0; base < w1; base += 32) {
+            const uint32_t p = base + lane;
+            const uint32_t key = p < w1 ? sk[p] : 0u;
+            ngt += __popc(__ballot_sync(0xffffffffu, p < w1 && key > T));
+            neq += __popc(__ballot_sync(0xffffffffu, p < w1 && key == T));
+        }
+        if (lane == 0) {
+            w_gt[warp] = ngt;
+            w_eq[warp] = neq;
+        }
+        __syncthreads();
+        uint32_t ob = 0, tb = 0;  // outputs and ties before this warp's run
+        for (int v = 0; v < warp; ++v) {
+            const uint32_t e = w_eq[v];
+            ob += w_gt[v] + (take == kTakeAll ? e : (tb >= take ? 0u : min(e, take - tb)));
+            tb += e;
+        }
+        const uint32_t lt = (1u << lane) - 1u;
+        for (uint32_t base = w0; base < w1; base += 32) {
+            const uint32_t p = base + lane;
+            const uint32_t key = p < w1 ? sk[p] : 0u;
+            const bool eq = p < w1 && key == T;
+            const uint32_t em = __ballot_sync(0xffffffffu, eq);
+            const bool pick_it = (p < w1 && key > T) || (eq && (take == kTakeAll || tb + __popc(em & lt) < take));
+            const uint32_t sm = __ballot_sync(0xffffffffu, pick_it);
+            if (pick_it) {
+                const uint32_t pos = ob + __popc(sm & lt);
+                const int32_t r = sj[p];
+                int32_t v = r;
+                if (a.pool) v = merge_pool_index(a, i, r);
+                if (pos < (uint32_t)K) out[pos] = v;
+            }
+            ob += __popc(sm);
+            tb += __popc(em);
+        }
+    } else {
+        constexpr int kE = 4;
+        uint32_t obase = 0, tbase = 0;
+        for (uint32_t c0 = 0; c0 < L; c0 += kMergeThreads * kE) {
+            uint32_t key[kE];
+            uint32_t gt = 0, eq = 0;
+#pragma unroll
+            for (int e = 0; e < kE; ++e) {
+                const uint32_t p = c0 + tid * kE + e;
+                key[e] = 0u;
+                if (p < L) {
+                    key[e] = __ldcg(gk + merge_row_pos(s_pre, s_off, nseg, p));
+                    if (key[e] > T) gt |= 1u << e;
+                    if (key[e] == T) eq |= 1u << e;
+                }
+            }
+            uint32_t ties = 0, trank = tbase;
+            if (take != kTakeAll) trank += block_excl_scan(__popc(eq), scan_smem, ties);
+            uint32_t sel = gt;
+#pragma unroll
+            for (int e = 0; e < kE; ++e)
+                if (eq & (1u << e)) {
+                    if (take == kTakeAll || trank < take) sel |= 1u << e;
+                    ++trank;
+                }
+            uint32_t chosen;
+            uint32_t pos = obase + block_excl_scan(__popc(sel), scan_smem, chosen);
+#pragma unroll
+            for (int e = 0; e < kE; ++e)
+                if (sel & (1u << e)) {
+                    const uint32_t p = c0 + tid * kE + e;
+                    const int32_t r = __ldcg(gj + merge_row_pos(s_pre, s_off, nseg, p));
+                    int32_t v = r;
+                    if (a.pool) v = merge_pool_index(a, i, r);
+                    if (pos < (uint32_t)K) out[pos] = v;
+                    ++pos;
+                }
+            obase += chosen;
+            tbase += ties;
+        }
+    }
+    for (int r = K + tid; r < a.topk; r += kMergeThreads) out[r] = -1;
 }
 
 // ---------------------------------------------------------------- prefill threshold
@@ -512,7 +920,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a) {
 // holds the k-th largest key, as the scan's last CTA does for a streamed query.
 __global__ void __launch_bounds__(1024) prefill_thresh_kernel(const float *scores, int rows, const int32_t *n_vis,
                                                               int topk, int32_t *thresh) {
-    __shared__ uint32_t hist[kBins];
+    __shared__ __align__(16) uint32_t hist[kBins];
     __shared__ uint32_t scan_smem[32];
     __shared__ BinPick pick;
     grid_dep_wait();
@@ -564,7 +972,7 @@ __global__ void __launch_bounds__(kRowSelThreads) row_select_kernel(const float 
                                                                     const int32_t *n_vis, int topk,
                                                                     int32_t *sel_idx, int32_t *status) {
     extern __shared__ __align__(16) uint32_t rkeys[];  // [rows]: the row's raw bits, then its keys
-    __shared__ uint32_t h[kBins];
+    __shared__ __align__(16) uint32_t h[kBins];
     __shared__ uint32_t bm[kRowSelWords];
     __shared__ uint32_t ck[kRowSelCands];
     __shared__ int32_t cj[kRowSelCands];
@@ -704,7 +1112,7 @@ __global__ void __launch_bounds__(kRowSelThreads) row_select_kernel(const float 
         }
     }
     __syncthreads();
-    p = pick_bin(h, 256, need, scan_smem, &pick);
+    p = pick_bin_warp(h, 256, need, &pick);
     const uint32_t T = (pre1 << 8) | (uint32_t)p.bin;  // the k-th largest key
     const uint32_t take_t = need - p.above;           // keys equal to T to take, lowest indices first (>= 1)
     if (in_list) {
@@ -807,8 +1215,8 @@ struct SelArgs {
 
 __device__ __forceinline__ int32_t out_index(const SelArgs &a, int i, int r) {
     if (!a.pool) return r;
-    return (__ldg(a.pool + (size_t)i * a.pool_p + (r >> a.pool_shift)) << a.pool_shift) +
-           (r & ((1 << a.pool_shift) - 1));
+    const int32_t *pp = a.pool;  // a plain load behind the branch, never hoisted above it
+    return (pp[(size_t)i * a.pool_p + (r >> a.pool_shift)] << a.pool_shift) + (r & ((1 << a.pool_shift) - 1));
 }
 
 // Keys above the threshold bin -> bitmap; keys in it -> candidate list.
@@ -940,7 +1348,7 @@ __global__ void __launch_bounds__(kSelThreads) select_final_kernel(SelArgs a0, S
     uint32_t *tie = dyn + a.words;                                     // [words] members tied on the key
     uint32_t *sck = dyn + 2 * a.words;                                 // [smem_cands] candidate keys
     int32_t *scj = reinterpret_cast<int32_t *>(sck + a.smem_cands);   // [smem_cands] candidate indices
-    __shared__ uint32_t h[kBins];
+    __shared__ __align__(16) uint32_t h[kBins];
     __shared__ uint32_t scan_smem[32];
     __shared__ BinPick pick;
     __shared__ uint32_t total_s, kmin_s, kmax_s;
@@ -1037,7 +1445,7 @@ __global__ void __launch_bounds__(kSelThreads) select_final_kernel(SelArgs a0, S
                 atomicAdd(&h[key_digit(level, key)], 1u);
             });
             __syncthreads();
-            const BinPick p = pick_bin(h, level == 1 ? 4096 : 256, need, scan_smem, &pick);
+            const BinPick p = level == 1 ? pick_bin(h, 4096, need, scan_smem, &pick) : pick_bin_warp(h, 256, need, &pick);
             if (threadIdx.x == 0) prefix_digit[level] = p.bin;
             done = (p.above + p.at == need);
             __syncthreads();
@@ -1114,7 +1522,7 @@ __global__ void __launch_bounds__(kBmaxThreads) pool_bmax_kernel(const float *sc
                                                                  int shift, int P, float *bmax, int rows_b,
                                                                  int32_t *n_vis_b, uint32_t *hist1, uint32_t *done,
                                                                  int32_t *thresh) {
-    __shared__ uint32_t hist[kBins];
+    __shared__ __align__(16) uint32_t hist[kBins];
     __shared__ uint32_t scan_smem[32];
     __shared__ BinPick pick;
     __shared__ int last_flag;
@@ -1218,8 +1626,12 @@ __global__ void __launch_bounds__(kCountThreads) reindex_count_kernel(const int3
 
 template <bool E4M3, int KS>
 cudaError_t launch_scan(const ScanArgs &sa, int grid, cudaStream_t s) {
-    if (sa.pool) return launch_pdl(scan_kernel<E4M3, KS, true>, dim3(grid), dim3(kScanThreads), 0, s, sa);
-    return launch_pdl(scan_kernel<E4M3, KS, false>, dim3(grid), dim3(kScanThreads), 0, s, sa);
+    if (sa.pool) {
+        if (sa.fused) return launch_pdl(scan_kernel<E4M3, KS, true, true>, dim3(grid), dim3(kScanThreads), 0, s, sa);
+        return launch_pdl(scan_kernel<E4M3, KS, true, false>, dim3(grid), dim3(kScanThreads), 0, s, sa);
+    }
+    if (sa.fused) return launch_pdl(scan_kernel<E4M3, KS, false, true>, dim3(grid), dim3(kScanThreads), 0, s, sa);
+    return launch_pdl(scan_kernel<E4M3, KS, false, false>, dim3(grid), dim3(kScanThreads), 0, s, sa);
 }
 
 // One selection: score rows, thresholds and output of a workspace.
@@ -1292,22 +1704,26 @@ namespace {
 // Scores of every key of every query into ws.scores (rows of `rows`), the
 // first-level thresholds, then the selection into sel_idx. n_vis_given and
 // pool describe a Reindex call (keys are pool positions); both null otherwise.
-// skip_select: the caller launches the selection (together with another one).
 cudaError_t index_pipeline(const csa_cache &c, const void *q_idx, const float *w, int Nq, int H_I,
                            const int32_t *q_offsets, const int32_t *q_pos, int topk, int32_t *sel_idx, IndexWs &ws,
                            int rows, const int32_t *n_vis_given, const int32_t *pool, int pool_shift, int pool_p,
-                           int num_sms, cudaStream_t s, bool skip_select = false) {
+                           int num_sms, cudaStream_t s) {
     // many queries per request (prefill): scores as a tensor-core GEMM, and when the
     // rows fit in shared memory one selection kernel that needs no zeroed state
     const bool gemm = !pool && !n_vis_given && Nq >= kPrefillQueriesPerRequest * c.batch &&
                       prefill_scores_supported(c.idx_dtype, c.idx_dim, H_I);
-    const bool row_sel = gemm && !skip_select && rows <= kRowSelMaxRows;
+    const bool row_sel = gemm && rows <= kRowSelMaxRows;
     cudaError_t err = cudaSuccess;
-    if (!row_sel) err = cudaMemsetAsync(ws.done, 0, ws.zero_bytes, s);  // counters, histograms, bitmaps
+    // the pass + final selection kernels need zeroed counters, histograms and bitmaps;
+    // the row selection and the streamed path's merge need no zeroed state
+    if (gemm && !row_sel) err = cudaMemsetAsync(ws.done, 0, ws.zero_bytes, s);
     if (err != cudaSuccess) return err;
-    err = launch_pdl(schedule_kernel, dim3(1), dim3(1024), 0, s, q_offsets, q_pos, c.n_blocks, c.batch, Nq, c.block,
-                     rows, topk, ws.req, ws.n_vis, ws.gprefix, ws.thresh, n_vis_given);
-    if (err != cudaSuccess) return err;
+    const bool fused = !gemm && Nq <= kFusedScheduleQueries;
+    if (!fused) {
+        err = launch_pdl(schedule_kernel, dim3(1), dim3(1024), 0, s, q_offsets, q_pos, c.n_blocks, c.batch, Nq,
+                         c.block, rows, topk, ws.req, ws.n_vis, ws.gprefix, ws.thresh, n_vis_given);
+        if (err != cudaSuccess) return err;
+    }
 
     ScanArgs sa;
     sa.keys = static_cast<const uint8_t *>(c.idx_key);
@@ -1317,9 +1733,9 @@ cudaError_t index_pipeline(const csa_cache &c, const void *q_idx, const float *w
     sa.n_vis = ws.n_vis;
     sa.gprefix = ws.gprefix;
     sa.scores = ws.scores;
-    sa.hist1 = ws.hist1;
-    sa.done = ws.done;
-    sa.thresh = ws.thresh;
+    sa.seg_cnt = ws.seg_cnt;
+    sa.seg_key = ws.seg_key;
+    sa.seg_idx = ws.seg_idx;
     sa.Nq = Nq;
     sa.H_I = H_I;
     sa.cap = c.capacity;
@@ -1328,7 +1744,17 @@ cudaError_t index_pipeline(const csa_cache &c, const void *q_idx, const float *w
     sa.pool = pool;
     sa.pool_shift = pool_shift;
     sa.pool_p = pool_p;
-    const int grid = num_sms;
+    sa.fused = fused ? 1 : 0;
+    sa.q_offsets = q_offsets;
+    sa.q_pos = q_pos;
+    sa.n_blocks = c.n_blocks;
+    sa.n_vis_given = n_vis_given;
+    sa.req_out = ws.req;
+    sa.n_vis_out = ws.n_vis;
+    sa.gprefix_out = ws.gprefix;
+    sa.batch = c.batch;
+    sa.m = c.block;
+    const int grid = min(num_sms, kMaxScanCtas);
     const bool e4 = c.idx_dtype == CSA_IDX_E4M3;
     if (gemm) {
         err = launch_prefill_scores(c.idx_key, c.batch, c.capacity, c.idx_dim, q_idx, w, Nq, H_I, ws.req, ws.n_vis, ws.scores,
@@ -1341,21 +1767,39 @@ cudaError_t index_pipeline(const csa_cache &c, const void *q_idx, const float *w
             return launch_pdl(row_select_kernel, dim3(Nq), dim3(kRowSelThreads), (size_t)smem, s,
                               (const float *)ws.scores, rows, (const int32_t *)ws.n_vis, topk, sel_idx, c.status);
         }
-        // per-query thresholds for the shared selection kernels
+        // per-query thresholds, then the pass + final selection kernels
         err = launch_pdl(prefill_thresh_kernel, dim3(Nq), dim3(1024), 0, s, (const float *)ws.scores, rows,
                          (const int32_t *)ws.n_vis, topk, ws.thresh);
-    } else {
-        switch (c.idx_dim / 16) {
-            case 4: err = e4 ? launch_scan<true, 4>(sa, grid, s) : launch_scan<false, 4>(sa, grid, s); break;
-            case 8: err = e4 ? launch_scan<true, 8>(sa, grid, s) : launch_scan<false, 8>(sa, grid, s); break;
-            case 16: err = e4 ? launch_scan<true, 16>(sa, grid, s) : launch_scan<false, 16>(sa, grid, s); break;
-            default: return cudaErrorInvalidValue;
-        }
+        if (err != cudaSuccess) return err;
+        const SelJob job{&ws, Nq, rows, topk, sel_idx, pool, pool_shift, pool_p};
+        return launch_select(job, nullptr, num_sms, s);
+    }
+    switch (c.idx_dim / 16) {
+        case 4: err = e4 ? launch_scan<true, 4>(sa, grid, s) : launch_scan<false, 4>(sa, grid, s); break;
+        case 8: err = e4 ? launch_scan<true, 8>(sa, grid, s) : launch_scan<false, 8>(sa, grid, s); break;
+        case 16: err = e4 ? launch_scan<true, 16>(sa, grid, s) : launch_scan<false, 16>(sa, grid, s); break;
+        default: return cudaErrorInvalidValue;
     }
     if (err != cudaSuccess) return err;
-    if (skip_select) return cudaSuccess;
-    const SelJob job{&ws, Nq, rows, topk, sel_idx, pool, pool_shift, pool_p};
-    return launch_select(job, nullptr, num_sms, s);
+    // the exact top-k of each query among its segments' candidates
+    MergeArgs ma;
+    ma.n_vis = ws.n_vis;
+    ma.gprefix = ws.gprefix;
+    ma.seg_cnt = ws.seg_cnt;
+    ma.seg_key = ws.seg_key;
+    ma.seg_idx = ws.seg_idx;
+    ma.sel_idx = sel_idx;
+    ma.Nq = Nq;
+    ma.G = grid;
+    ma.topk = topk;
+    ma.rows = rows;
+    ma.pool = pool;
+    ma.pool_shift = pool_shift;
+    ma.pool_p = pool_p;
+    const int msmem = 8 * kMergeStage;
+    err = cudaFuncSetAttribute(select_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem);
+    if (err != cudaSuccess) return err;
+    return launch_pdl(select_merge_kernel, dim3(Nq), dim3(kMergeThreads), (size_t)msmem, s, ma);
 }
 
 }  // namespace
@@ -1384,11 +1828,11 @@ cudaError_t launch_index_topk_pool(const csa_cache &c, const void *q_idx, const 
     IndexWs ws, wb;
     const size_t main_bytes = align256(carve(workspace, Nq, c.capacity, &ws));
     carve(static_cast<char *>(workspace) + main_bytes, Nq, cap_b, &wb);
-    // this layer's scores and its key threshold; its score rows stay in ws.scores
+    // this layer's scores and top-k; its score rows stay in ws.scores
     cudaError_t err = index_pipeline(c, q_idx, w, Nq, H_I, q_offsets, q_pos, topk, sel_idx, ws, c.capacity, nullptr,
-                                     nullptr, 0, 0, num_sms, s, true);
+                                     nullptr, 0, 0, num_sms, s);
     if (err != cudaSuccess) return err;
-    // block maxima and the pool's threshold, then both selections in the same launches
+    // block maxima and the pool's threshold, then the pool's selection
     if ((err = cudaMemsetAsync(wb.done, 0, wb.zero_bytes, s)) != cudaSuccess) return err;
     const int per_cta = kBmaxThreads * kBmaxPerThread;
     const int gx = (cap_b + per_cta - 1) / per_cta;
@@ -1396,9 +1840,8 @@ cudaError_t launch_index_topk_pool(const csa_cache &c, const void *q_idx, const 
                      (const int32_t *)ws.n_vis, c.capacity, pool_shift, P, wb.scores, cap_b, wb.n_vis, wb.hist1,
                      wb.done, wb.thresh);
     if (err != cudaSuccess) return err;
-    const SelJob keys{&ws, Nq, c.capacity, topk, sel_idx, nullptr, 0, 0};
     const SelJob blocks{&wb, Nq, cap_b, P, pool_blk, nullptr, 0, 0};
-    return launch_select(keys, &blocks, num_sms, s);
+    return launch_select(blocks, nullptr, num_sms, s);
 }
 
 size_t index_reindex_workspace_bytes(int Nq, int G, int P) { return carve(nullptr, Nq, G * P, nullptr); }
