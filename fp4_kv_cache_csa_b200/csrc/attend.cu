@@ -56,6 +56,14 @@ namespace {
 constexpr int kTile = 128;
 constexpr int kHeads = 64;
 constexpr int kThreads = 256;
+// Relative cost of the work the CTAs share out (measured per-CTA times on B200 at
+// D = 512: a compressed tile ~6.2 us, a window tile ~11.5 us -- bf16 rows 4x the
+// bytes, copied and converted in place -- and each query a CTA starts ~7 us: its
+// Q' copy, the final PV wait, the output or partial write). The flat tile list is
+// cut into equal shares of these units, not of tiles.
+constexpr long long kCTileCost = 100;
+constexpr long long kWTileCost = 185;
+constexpr long long kStartCost = 110;
 
 template <int D>
 struct Cfg {
@@ -93,6 +101,7 @@ struct AttArgs {
     const QInfo *qinfo;              // [Nq]
     const long long *tprefix;        // [Nq+1]
     const int32_t *cta_q;            // [G] first query of each CTA's range
+    const long long *cta_t;          // [G+1] first tile of each CTA's range
     const int32_t *sq;               // [Nq] query scale exponents
     const uint8_t *qimg;             // [Nq][Q_BYTES] Q' images
     float *part_o, *part_rho, *part_l;  // [2G][64][D], [2G][64], [2G][64]
@@ -373,7 +382,8 @@ template <int D>
 __global__ void __launch_bounds__(1024) attend_schedule_kernel(
     const int32_t *q_offsets, const int32_t *q_pos, const int32_t *n_blocks, const int32_t *win_len, int batch,
     int Nq, int m, int cap, int topk, int max_win, const __nv_bfloat16 *q, int H, int G, QInfo *qinfo,
-    long long *tprefix, int32_t *cta_q, int32_t *sq, uint8_t *qimg, float *out, float *lse, int32_t *status) {
+    long long *tprefix, int32_t *cta_q, long long *cta_t, long long *uprefix, int32_t *sq, uint8_t *qimg, float *out,
+    float *lse, int32_t *status) {
     __shared__ long long red[32];
     __shared__ long long round_total;
     __shared__ float fred[32];
@@ -441,14 +451,16 @@ __global__ void __launch_bounds__(1024) attend_schedule_kernel(
     if (qi != Nq) return;
     // ---- CTA Nq (in parallel with the others): per-query records, tile prefix,
     // first query of every CTA range
-    long long carry = 0;
+    long long carry = 0, ucarry = 0;
     for (int base = 0; base < Nq; base += blockDim.x) {
         const int i = base + threadIdx.x;
-        long long tiles = 0;
+        long long tiles = 0, units = 0;
         int b = 0, ne = 0, ct = 0, wl = 0;
         if (i < Nq) {
             query_tiles(q_offsets, q_pos, n_blocks, win_len, batch, m, cap, topk, max_win, i, status, b, ne, ct, wl);
-            tiles = ct + (wl + kTile - 1) / kTile;
+            const int wt = (wl + kTile - 1) / kTile;
+            tiles = ct + wt;
+            units = tiles > 0 ? kStartCost + kCTileCost * ct + kWTileCost * wt : 0;
         }
         const long long incl = block_inclusive_scan<long long>(tiles, red);
         if (i < Nq) {
@@ -465,20 +477,59 @@ __global__ void __launch_bounds__(1024) attend_schedule_kernel(
         __syncthreads();
         carry += round_total;
         __syncthreads();
+        const long long uincl = block_inclusive_scan<long long>(units, red);
+        if (i < Nq) uprefix[i + 1] = ucarry + uincl;
+        if (i == 0) uprefix[0] = 0;
+        if (threadIdx.x == blockDim.x - 1) round_total = uincl;
+        __syncthreads();
+        ucarry += round_total;
+        __syncthreads();
     }
     __threadfence_block();
     __syncthreads();
-    // first query of CTA c: the last i with tprefix[i] <= t_begin(c)
-    const long long T = carry;
-    for (int c = threadIdx.x; c < G; c += blockDim.x) {
-        const long long tb = T * c / G;
-        int lo = 0, hi = Nq - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (tprefix[mid] <= tb) lo = mid; else hi = mid - 1;
+    // CTA c's share starts at unit U c / G: its first tile is the first one of the
+    // query holding that unit whose own units start at or after it; its first query
+    // is the last i with tprefix[i] <= that tile
+    const long long T = carry, U = ucarry;
+    for (int c = threadIdx.x; c <= G; c += blockDim.x) {
+        long long tb = T;
+        if (c < G && U > 0) {
+            const long long ub = U * c / G;
+            int lo = 0, hi = Nq - 1;  // last i with uprefix[i] <= ub
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (uprefix[mid] <= ub) lo = mid; else hi = mid - 1;
+            }
+            const QInfo r = qinfo[lo];
+            const long long ct = r.a.z, nt = r.t.y - r.t.x;
+            const long long x = ub - uprefix[lo] - kStartCost;  // units into the query's tiles
+            long long before = 0;                               // its tiles starting before ub
+            if (x > 0) {
+                if (x <= ct * kCTileCost) before = (x + kCTileCost - 1) / kCTileCost;
+                else before = ct + (x - ct * kCTileCost + kWTileCost - 1) / kWTileCost;
+            }
+            tb = r.t.x + min(before, nt);
         }
-        cta_q[c] = lo;
+        cta_t[c] = tb;
+        if (c < G) {
+            int lo = 0, hi = Nq - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (tprefix[mid] <= tb) lo = mid; else hi = mid - 1;
+            }
+            cta_q[c] = lo;
+        }
     }
+}
+
+// The CTA whose range holds flat tile t: the last c with cta_t[c] <= t.
+__device__ __forceinline__ int cta_of_tile(const long long *cta_t, int G, long long t) {
+    int lo = 0, hi = G - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (cta_t[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    return lo;
 }
 
 // ---------------------------------------------------------------- split merge
@@ -492,7 +543,8 @@ constexpr int kMergeHeads = 8;
 // index c; only a query that CTA c - 1 and CTA c both cover can need a merge,
 // and the CTA for the first such boundary of a query merges it, so the grid
 // has G - 1 columns instead of one per query.
-__global__ void __launch_bounds__(256) attend_merge_kernel(const long long *tprefix, int Nq, int H, int D, int G,
+__global__ void __launch_bounds__(256) attend_merge_kernel(const long long *tprefix, const long long *cta_t, int Nq,
+                                                           int H, int D, int G,
                                                            const float *part_o, const float *part_rho,
                                                            const float *part_l, float *out, float *lse,
                                                            int by_boundary) {
@@ -503,12 +555,11 @@ __global__ void __launch_bounds__(256) attend_merge_kernel(const long long *tpre
     grid_dep_wait();
     const int h0 = blockIdx.y * kMergeHeads;
     if (h0 >= H) return;
-    const long long T = tprefix[Nq];
     int i = blockIdx.x;
     if (by_boundary) {
         // the query holding tile rb = first tile of CTA c: largest i with tprefix[i] < rb
         const int c = blockIdx.x + 1;
-        const long long rb = T * c / G;
+        const long long rb = cta_t[c];
         int lo = 0, hi = Nq - 1;  // tprefix[0] = 0 < rb unless rb = 0 (then no query straddles)
         if (rb <= 0) return;
         while (lo < hi) {
@@ -518,17 +569,17 @@ __global__ void __launch_bounds__(256) attend_merge_kernel(const long long *tpre
         i = lo;
         if (tprefix[i + 1] <= rb) return;  // the boundary is at the end of query i: nothing straddles
         const long long Ti0 = tprefix[i];
-        if ((int)(((Ti0 + 1) * G - 1) / T) + 1 != c) return;  // not the query's first inner boundary
+        if (cta_of_tile(cta_t, G, Ti0) + 1 != c) return;  // not the query's first inner boundary
     }
     const long long Ti = tprefix[i], Ti1 = tprefix[i + 1];
     if (Ti1 == Ti) return;  // no entry at all: written by the schedule kernel
-    const int c_first = (int)(((Ti + 1) * G - 1) / T);
-    const int c_last = (int)((Ti1 * G - 1) / T);
+    const int c_first = cta_of_tile(cta_t, G, Ti);
+    const int c_last = cta_of_tile(cta_t, G, Ti1 - 1);
     if (c_first == c_last) return;  // one CTA covered the query and wrote it
     if (threadIdx.x == 0) {
         int np = 0;
         for (int cc = c_first; cc <= c_last && np < 256; ++cc) {
-            const long long rb = T * cc / G, re = T * (cc + 1) / G;
+            const long long rb = cta_t[cc], re = cta_t[cc + 1];
             if (rb >= re) continue;  // CTA with an empty range
             slots[np++] = 2 * cc + (rb >= Ti ? 0 : 1);
         }
@@ -610,9 +661,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int hf = tid >> 7;               // channel half (dequant) = head half (softmax)
     grid_dep_wait();                       // the schedule kernel's records (programmatic launch)
-    const long long T = a.tprefix[a.Nq];
-    const int G = gridDim.x, c = blockIdx.x;
-    const long long t_begin = T * c / G, t_end = T * (c + 1) / G;
+    const int c = blockIdx.x;
+    const long long t_begin = a.cta_t[c], t_end = a.cta_t[c + 1];
     if (t_begin >= t_end) return;
 
     const uint32_t E_s = smem_u32(E), Q_s = smem_u32(Q), P_s = smem_u32(P);
@@ -903,7 +953,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
             alpha[tid] = l;  // l_h
         }
         __syncthreads();
-        const int b_slot = 2 * c + ((seg_begin == T * c / G) ? 0 : 1);
+        const int b_slot = 2 * c + ((seg_begin == t_begin) ? 0 : 1);
         float *dst = whole ? a.out + (size_t)i * a.H * D : a.part_o + (size_t)b_slot * kHeads * D;
         // O^T (or O / l for a whole query) -> the E' buffer as [head][channel] fp32
         // (64 x D x 4 bytes = the buffer's size), then one bulk copy of the H used rows
@@ -975,10 +1025,11 @@ cudaError_t launch_main(const AttArgs &a, int num_ctas, cudaStream_t s) {
 template <int D>
 cudaError_t launch_schedule(const csa_cache &c, const AttArgs &a, const int32_t *q_offsets, const int32_t *q_pos,
                             const int32_t *win_len, int topk, int max_win, const void *q, int num_ctas, QInfo *qinfo,
-                            long long *tprefix, int32_t *cta_q, int32_t *sq, uint8_t *qimg, cudaStream_t s) {
+                            long long *tprefix, int32_t *cta_q, long long *cta_t, long long *uprefix, int32_t *sq,
+                            uint8_t *qimg, cudaStream_t s) {
     attend_schedule_kernel<D><<<a.Nq + 1, 1024, 0, s>>>(q_offsets, q_pos, c.n_blocks, win_len, c.batch, a.Nq, c.block,
                                                    c.capacity, topk, max_win, static_cast<const __nv_bfloat16 *>(q),
-                                                   a.H, num_ctas, qinfo, tprefix, cta_q, sq, qimg, a.out, a.lse,
+                                                   a.H, num_ctas, qinfo, tprefix, cta_q, cta_t, uprefix, sq, qimg, a.out, a.lse,
                                                    c.status);
     return cudaGetLastError();
 }
@@ -991,6 +1042,8 @@ size_t attend_workspace_bytes(int Nq, int D, int num_ctas) {
     take(sizeof(QInfo) * (size_t)Nq);                 // qinfo
     take(8 * (size_t)(Nq + 1));                       // tprefix
     take(4 * (size_t)num_ctas);                       // cta_q
+    take(8 * (size_t)(num_ctas + 1));                 // cta_t
+    take(8 * (size_t)(Nq + 1));                       // uprefix
     take(4 * (size_t)Nq);                             // sq
     take((size_t)Nq * kHeads * D * 2);                // qimg
     take(4 * (size_t)2 * num_ctas * kHeads * D);      // part_o
@@ -1015,6 +1068,8 @@ cudaError_t launch_attend(const csa_cache &c, const void *q, int Nq, int H, cons
     QInfo *qinfo = reinterpret_cast<QInfo *>(take(sizeof(QInfo) * (size_t)Nq));
     long long *tprefix = reinterpret_cast<long long *>(take(8 * (size_t)(Nq + 1)));
     int32_t *cta_q = reinterpret_cast<int32_t *>(take(4 * (size_t)num_ctas));
+    long long *cta_t = reinterpret_cast<long long *>(take(8 * (size_t)(num_ctas + 1)));
+    long long *uprefix = reinterpret_cast<long long *>(take(8 * (size_t)(Nq + 1)));
     int32_t *sq = reinterpret_cast<int32_t *>(take(4 * (size_t)Nq));
     uint8_t *qimg = reinterpret_cast<uint8_t *>(take((size_t)Nq * kHeads * D * 2));
     a.part_o = reinterpret_cast<float *>(take(4 * (size_t)2 * num_ctas * kHeads * D));
@@ -1031,6 +1086,7 @@ cudaError_t launch_attend(const csa_cache &c, const void *q, int Nq, int H, cons
     a.qinfo = qinfo;
     a.tprefix = tprefix;
     a.cta_q = cta_q;
+    a.cta_t = cta_t;
     a.sq = sq;
     a.qimg = qimg;
     a.Nq = Nq;
@@ -1044,15 +1100,15 @@ cudaError_t launch_attend(const csa_cache &c, const void *q, int Nq, int H, cons
     const int32_t *wl = win_kv ? win_len : nullptr;
     const int G = num_ctas;  // work ranges, one per CTA
     if (D == 512) {
-        if ((err = launch_schedule<512>(c, a, q_offsets, qp, wl, topk, max_win, q, num_ctas, qinfo, tprefix, cta_q, sq,
-                                        qimg, s)) != cudaSuccess)
+        if ((err = launch_schedule<512>(c, a, q_offsets, qp, wl, topk, max_win, q, num_ctas, qinfo, tprefix, cta_q, cta_t,
+                                        uprefix, sq, qimg, s)) != cudaSuccess)
             return err;
         err = c.scale_fmt == CSA_SCALE_E4M3_16 ? launch_main<512, kScaleE4M3x16>(a, num_ctas, s)
                                                 : launch_main<512, kScaleE8M0x32>(a, num_ctas, s);
         if (err != cudaSuccess) return err;
     } else if (D == 128) {
-        if ((err = launch_schedule<128>(c, a, q_offsets, qp, wl, topk, max_win, q, num_ctas, qinfo, tprefix, cta_q, sq,
-                                        qimg, s)) != cudaSuccess)
+        if ((err = launch_schedule<128>(c, a, q_offsets, qp, wl, topk, max_win, q, num_ctas, qinfo, tprefix, cta_q, cta_t,
+                                        uprefix, sq, qimg, s)) != cudaSuccess)
             return err;
         err = c.scale_fmt == CSA_SCALE_E4M3_16 ? launch_main<128, kScaleE4M3x16>(a, num_ctas, s)
                                                 : launch_main<128, kScaleE8M0x32>(a, num_ctas, s);
@@ -1071,7 +1127,7 @@ cudaError_t launch_attend(const csa_cache &c, const void *q, int Nq, int H, cons
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, attend_merge_kernel, (const long long *)tprefix, Nq, H, D, G,
+    return cudaLaunchKernelEx(&cfg, attend_merge_kernel, (const long long *)tprefix, (const long long *)cta_t, Nq, H, D, G,
                               (const float *)a.part_o, (const float *)a.part_rho, (const float *)a.part_l, out, lse,
                               by_boundary);
 }
