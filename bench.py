@@ -39,7 +39,7 @@ H_I, D_I, TOPK = 4, 128, 1024
 POOL_GROUP, POOL_BLOCKS = 8, 2000  # hierarchical indexer pool: ~2000 blocks of 8 entries
 CTX_MIN, CTX_MAX = 524288, 1048576
 CAP_CSA, CAP_HCA = CTX_MAX // M_CSA, CTX_MAX // M_HCA
-OUR_KERNELS_PER_STEP = 14  # compress 2x(pool, commit); index: schedule, scan, select x2; attend 2x(schedule, main, merge)
+OUR_KERNELS_PER_STEP = 12  # compress 2x(pool, commit); index: scan (own schedule), merge; attend 2x(schedule, main, merge)
 SEED = 0x5EED0C5A
 
 
@@ -483,6 +483,136 @@ def measure_prefill(device, stream, flush, steps: int = 3):
     return res
 
 
+class ConfigRun:
+    """One of the other decode workloads, timed apart from the step: its own caches (drawn
+    bytes, as in the step), one CSA layer (indexer + top-k + attention) or one HCA layer."""
+
+    def __init__(self, device, name, B_, T, H_, D_, m, d_i, idx_dtype, k, lognormal=0.0):
+        import torch
+
+        import fp4_kv_cache_csa_b200 as csa
+
+        self.name, self.B, self.T, self.H, self.D, self.m, self.d_i, self.k = name, B_, T, H_, D_, m, d_i, k
+        self.n = T // m
+        gen = torch.Generator(device=device)
+        gen.manual_seed(SEED + 7 + B_)
+        bf = torch.bfloat16
+
+        def act(*shape, std=1.0):
+            x = torch.randn(*shape, device=device, generator=gen) * std
+            if lognormal:
+                x = x * torch.exp(torch.randn(shape[-1], device=device, generator=gen) * lognormal)
+            return x
+
+        self.cache = csa.Cache.allocate(B_, self.n, D_, m, d_i, idx_dtype, device, scale_fmt=SCALE_FMT)
+        s_lo, s_hi = (123, 127) if SCALE_FMT == 0 else (0x1C, 0x2D)
+        self.cache.fp4.random_(0, 256, generator=gen)
+        self.cache.scale.random_(s_lo, s_hi, generator=gen)
+        self.cache.n_blocks.fill_(self.n)
+        if d_i:
+            keys = act(B_, self.n, d_i, std=0.5)
+            self.cache.idx_key.copy_(keys.to(bf) if idx_dtype == csa.CSA_IDX_BF16
+                                     else keys.to(torch.float8_e4m3fn).view(torch.uint8))
+            self.q_idx = act(B_, H_I, d_i).to(bf)
+            self.w = (torch.randn(B_, H_I, device=device, generator=gen) / math.sqrt(H_I)).float()
+            self.sel = torch.empty(B_, k, dtype=torch.int32, device=device)
+            self.ws_idx = torch.empty(csa.csa_index_topk_workspace(self.cache, B_, k), dtype=torch.uint8,
+                                      device=device)
+        self.q = act(B_, H_, D_).to(bf)
+        self.win = act(B_ * W, D_).to(bf)
+        self.win_start = torch.arange(0, B_ * W, W, dtype=torch.int64, device=device)
+        self.win_len = torch.full((B_,), W, dtype=torch.int32, device=device)
+        self.q_offsets = torch.arange(B_ + 1, dtype=torch.int32, device=device)
+        self.q_pos = torch.full((B_,), T - 1, dtype=torch.int32, device=device)
+        self.out = torch.empty(B_, H_, D_, dtype=torch.float32, device=device)
+        self.ws_att = torch.empty(csa.csa_attend_workspace(self.cache, B_, H_), dtype=torch.uint8, device=device)
+
+    def stages(self):
+        import fp4_kv_cache_csa_b200 as csa
+
+        if not self.d_i:  # HCA layer
+            return (lambda: csa.hca_decode_attend(self.cache, self.q, self.q_offsets, self.q_pos, self.win,
+                                                  self.win_start, self.win_len, max_win=W,
+                                                  softmax_scale=self.D ** -0.5, out=self.out,
+                                                  workspace=self.ws_att),)
+        return (lambda: csa.csa_index_topk(self.cache, self.q_idx, self.w, self.q_offsets, self.q_pos, self.k,
+                                           sel_idx=self.sel, workspace=self.ws_idx),
+                lambda: csa.csa_decode_attend(self.cache, self.q, self.q_offsets, self.sel, self.win,
+                                              self.win_start, self.win_len, max_win=W,
+                                              softmax_scale=self.D ** -0.5, out=self.out, workspace=self.ws_att))
+
+    def bytes_flops(self):
+        """Algorithmic HBM bytes and dense-contraction FLOPs of one layer step."""
+        entry = self.D // 2 + self.D // scale_group()
+        per_req = self.B * (W * self.D * 2 + self.H * self.D * 2 + self.H * self.D * 4)
+        if not self.d_i:
+            ents = self.n
+            b = self.B * ents * entry + per_req
+        else:
+            ents = min(self.n, self.k)
+            kb = 2 if self.cache.idx_dtype == 0 else 1
+            b = self.B * (self.n * self.d_i * kb + ents * entry + H_I * self.d_i * 2 + H_I * 4 + self.k * 4) + per_req
+        flops = 4.0 * self.B * self.H * (ents + W) * self.D
+        return float(b), flops
+
+
+def measure_configs(device, stream, flush, steps: int = 20):
+    """Per-layer decode times of the other workloads (CUDA graphs, cold L2 before each replay)."""
+    import torch
+
+    import fp4_kv_cache_csa_b200 as csa
+
+    hbm, hbm_kind = measured_peaks()
+    tflops, tf_kind = measured_bf16_tflops()
+    runs = (("csa_tiny_4k", dict(B_=1, T=4096, H_=16, D_=128, m=4, d_i=64, idx_dtype=csa.CSA_IDX_BF16, k=64)),
+            ("csa_b8_64k", dict(B_=8, T=65536, H_=64, D_=512, m=4, d_i=128, idx_dtype=csa.CSA_IDX_BF16, k=512,
+                                lognormal=0.5)),
+            ("hca_b64_1m", dict(B_=64, T=1048576, H_=64, D_=512, m=128, d_i=0, idx_dtype=csa.CSA_IDX_BF16, k=0)))
+    res = {}
+    for name, kw in runs:
+        cr = ConfigRun(device, name, **kw)
+        fns = cr.stages()
+        with torch.cuda.stream(stream):
+            for fn in fns:
+                fn()
+            stream.synchronize()
+            graphs = []
+            for fn in fns:
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    fn()
+                graphs.append(g)
+            for _ in range(3):
+                flush.zero_()
+                for g in graphs:
+                    g.replay()
+            ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(graphs) + 1)] for _ in range(steps)]
+            for k in range(steps):
+                flush.zero_()
+                for s_, g in enumerate(graphs):
+                    ev[k][s_].record(stream)
+                    g.replay()
+                ev[k][len(graphs)].record(stream)
+        stream.synchronize()
+        st = np.array([[ev[k][j].elapsed_time(ev[k][j + 1]) for j in range(len(graphs))]
+                       for k in range(steps)]).mean(axis=0)
+        ms = float(st.sum())
+        b, fl = cr.bytes_flops()
+        t_hbm, t_tc = b / (hbm * 1e9), fl / (tflops * 1e12)
+        bound = "hbm" if t_hbm >= t_tc else "tensor"
+        res[name] = {"batch": cr.B, "ctx": cr.T, "entries_per_request": cr.n, "ms": ms,
+                     "stage_ms": dict(zip(("hca_attend",) if not cr.d_i else ("index_topk", "csa_attend"),
+                                          (float(x) for x in st))),
+                     "tokens_per_s": cr.B / (ms * 1e-3), "algorithmic_bytes": b, "flops": fl,
+                     "achieved_gbs": b / (ms * 1e-3) / 1e9, "achieved_tflops": fl / (ms * 1e-3) / 1e12,
+                     "bound": bound, "roofline_frac": max(t_hbm, t_tc) / (ms * 1e-3),
+                     "peaks": {"hbm_gbs": hbm, "hbm_kind": hbm_kind, "bf16_tflops": tflops, "bf16_kind": tf_kind},
+                     "device_status": int(csa.csa_read_device_status(cr.cache, stream))}
+        del graphs, cr
+        torch.cuda.empty_cache()
+    return res
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -575,6 +705,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill_b4_8k measurement")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the csa_tiny_4k / csa_b8_64k / hca_b64_1m measurements")
     ap.add_argument("--batch", type=int, default=B, help="requests per GPU (default 32; smaller only for profiling)")
     ap.add_argument("--scale-fmt", default="e8m0x32", choices=sorted(SCALE_FMT_NAMES),
                     help="FP4 scale format of both caches (default: E8M0 per 32 elements, MXFP4)")
@@ -678,6 +810,7 @@ def main():
     status |= csa.csa_read_device_status(wl.csa, stream)
     del csa2_graphs
     prefill = measure_prefill(device, stream, flush) if not args.no_prefill else None
+    configs = measure_configs(device, stream, flush) if not args.no_configs else None
 
     # ---- end-to-end: pinned host inputs in, results out, every step. Two buffer
     # sets (each with its own graphs): step k+1's inputs are copied in and step
@@ -779,7 +912,7 @@ def main():
                       "algorithmic_bytes": wl.bytes_csa_layer(),
                       "achieved_gbs": wl.bytes_csa_layer() / (csa_ms * 1e-3) / 1e9,
                       "frac_of_hbm_peak": wl.bytes_csa_layer() / (csa_ms * 1e-3) / 1e9 / peak},
-        "roofline": {"bound": "hbm", "kernel": "csa_index_topk (scan + select)", "achieved": achieved, "peak": peak,
+        "roofline": {"bound": "hbm", "kernel": "csa_index_topk (scan + merge)", "achieved": achieved, "peak": peak,
                      "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind,
                      "traffic": index_traffic(wl.key_bytes()), "traffic_unit": "GB per call (ncu, scaled by keys)"},
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
@@ -794,6 +927,7 @@ def main():
         "prefill": None if prefill is None else dict(
             prefill, index_tensor_frac=prefill["index_tflops"] / measured_bf16_tflops()[0],
             index_tensor_peak={"tflops": measured_bf16_tflops()[0], "kind": measured_bf16_tflops()[1] + " bf16 dense"}),
+        "configs": configs,
         "gpu_launches": OUR_KERNELS_PER_STEP * args.steps,
         "clocks": clocks.summary(),
         "device_status": status,
