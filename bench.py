@@ -613,6 +613,53 @@ def measure_configs(device, stream, flush, steps: int = 20):
     return res
 
 
+def measure_index_mxfp4(device, stream, flush, wl, steps: int = 20):
+    """The step's indexer call (same requests, queries and k) over a cache whose indexer keys are
+    MXFP4 (E2M1 codes + one E8M0 scale per 32 channels: 68 bytes per key instead of 128)."""
+    import torch
+
+    import fp4_kv_cache_csa_b200 as csa
+
+    gen = torch.Generator(device=device)
+    gen.manual_seed(SEED + 11)
+    cache = csa.Cache(fp4=wl.csa.fp4, scale=wl.csa.scale, n_blocks=wl.csa.n_blocks.clone(), block=M_CSA,
+                      idx_key=torch.empty(B, CAP_CSA, D_I // 2, dtype=torch.uint8, device=device),
+                      idx_dtype=csa.CSA_IDX_MXFP4, status=torch.zeros(1, dtype=torch.int32, device=device),
+                      scale_fmt=SCALE_FMT,
+                      idx_key_scale=torch.empty(B, CAP_CSA, D_I // 32, dtype=torch.uint8, device=device))
+    cache.idx_key.random_(0, 256, generator=gen)
+    cache.idx_key_scale.random_(122, 128, generator=gen)  # pooled N(0, 0.5^2) keys land in 2^-5 .. 2^0
+    cache.n_blocks.copy_(torch.tensor(wl.n_csa, dtype=torch.int32, device=device))
+    sel = torch.empty(B, TOPK, dtype=torch.int32, device=device)
+    ws = torch.empty(csa.csa_index_topk_workspace(cache, B, TOPK), dtype=torch.uint8, device=device)
+    fn = lambda: csa.csa_index_topk(cache, wl.q_idx, wl.w, wl.q_offsets, wl.q_pos, TOPK, sel_idx=sel, workspace=ws)
+    with torch.cuda.stream(stream):
+        fn()
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            fn()
+        for _ in range(3):
+            flush.zero_()
+            g.replay()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+        for k in range(steps):
+            flush.zero_()
+            ev[k][0].record(stream)
+            g.replay()
+            ev[k][1].record(stream)
+    stream.synchronize()
+    ms = float(np.mean([e[0].elapsed_time(e[1]) for e in ev]))
+    key_bytes = float(np.sum(wl.n_csa)) * (D_I // 2 + D_I // 32)
+    b = key_bytes + B * (H_I * D_I * 2 + H_I * 4 + TOPK * 4)
+    hbm, kind = measured_peaks()
+    res = {"ms": ms, "tokens_per_s": B / (ms * 1e-3), "key_bytes_per_block": D_I // 2 + D_I // 32,
+           "algorithmic_bytes": b, "achieved_gbs": b / (ms * 1e-3) / 1e9, "frac_of_hbm_peak": b / (ms * 1e-3) / 1e9 / hbm,
+           "peak_kind": kind, "device_status": int(csa.csa_read_device_status(cache, stream))}
+    del g
+    return res
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -811,6 +858,7 @@ def main():
     del csa2_graphs
     prefill = measure_prefill(device, stream, flush) if not args.no_prefill else None
     configs = measure_configs(device, stream, flush) if not args.no_configs else None
+    index_mxfp4 = measure_index_mxfp4(device, stream, flush, wl) if not args.no_configs else None
 
     # ---- end-to-end: pinned host inputs in, results out, every step. Two buffer
     # sets (each with its own graphs): step k+1's inputs are copied in and step
@@ -928,6 +976,8 @@ def main():
             prefill, index_tensor_frac=prefill["index_tflops"] / measured_bf16_tflops()[0],
             index_tensor_peak={"tflops": measured_bf16_tflops()[0], "kind": measured_bf16_tflops()[1] + " bf16 dense"}),
         "configs": configs,
+        # the same indexer call with MXFP4 indexer keys (not the headline config's e4m3 keys)
+        "index_mxfp4_keys": index_mxfp4,
         "gpu_launches": OUR_KERNELS_PER_STEP * args.steps,
         "clocks": clocks.summary(),
         "device_status": status,

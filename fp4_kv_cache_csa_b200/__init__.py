@@ -22,6 +22,7 @@ LIB_PATH = os.path.join(_HERE, "libcsa.so")
 
 CSA_IDX_BF16 = 0
 CSA_IDX_E4M3 = 1
+CSA_IDX_MXFP4 = 2
 
 CSA_SCALE_E8M0_32 = 0  # one E8M0 scale byte per 32 elements (OCP MXFP4)
 CSA_SCALE_E4M3_16 = 1  # one E4M3 scale byte per 16 elements
@@ -50,6 +51,7 @@ class _CCache(ctypes.Structure):
         ("fp4", ctypes.c_void_p), ("scale", ctypes.c_void_p), ("idx_key", ctypes.c_void_p),
         ("idx_dim", ctypes.c_int32), ("idx_dtype", ctypes.c_int32),
         ("n_blocks", ctypes.c_void_p), ("status", ctypes.c_void_p), ("scale_fmt", ctypes.c_int32),
+        ("idx_key_scale", ctypes.c_void_p),
     ]
 
 
@@ -121,7 +123,8 @@ class Cache:
     """One compressed cache (one layer): device tensors owned by the caller (see include/csa.h).
 
     fp4 [B, cap, D/2] uint8, scale [B, cap, D/32] uint8 (E8M0) or [B, cap, D/16] uint8 (E4M3),
-    idx_key [B, cap, dI] bf16 / uint8 (e4m3) or None, n_blocks [B] int32, status [1] int32 or None.
+    idx_key [B, cap, dI] bf16 / uint8 (e4m3) or [B, cap, dI/2] uint8 (MXFP4 codes, with
+    idx_key_scale [B, cap, dI/32] uint8) or None, n_blocks [B] int32, status [1] int32 or None.
     """
     fp4: object
     scale: object
@@ -131,6 +134,7 @@ class Cache:
     idx_dtype: int = CSA_IDX_BF16
     status: object = None
     scale_fmt: int = CSA_SCALE_E8M0_32
+    idx_key_scale: object = None
 
     @property
     def batch(self) -> int:
@@ -146,12 +150,14 @@ class Cache:
 
     @property
     def idx_dim(self) -> int:
-        return 0 if self.idx_key is None else self.idx_key.shape[2]
+        if self.idx_key is None:
+            return 0
+        return self.idx_key.shape[2] * (2 if self.idx_dtype == CSA_IDX_MXFP4 else 1)
 
     def c_struct(self) -> _CCache:
         return _CCache(self.batch, self.dim, self.block, self.capacity, _ptr(self.fp4), _ptr(self.scale),
                        _ptr(self.idx_key), self.idx_dim, self.idx_dtype, _ptr(self.n_blocks), _ptr(self.status),
-                       self.scale_fmt)
+                       self.scale_fmt, _ptr(self.idx_key_scale))
 
     @staticmethod
     def allocate(batch: int, capacity: int, dim: int, block: int, idx_dim: int = 0, idx_dtype: int = CSA_IDX_BF16,
@@ -159,8 +165,11 @@ class Cache:
         """Zero-filled cache tensors on `device` (torch allocation; the library allocates nothing)."""
         import torch
 
-        idx = None
-        if idx_dim:
+        idx = idx_scale = None
+        if idx_dim and idx_dtype == CSA_IDX_MXFP4:
+            idx = torch.zeros(batch, capacity, idx_dim // 2, dtype=torch.uint8, device=device)
+            idx_scale = torch.zeros(batch, capacity, idx_dim // 32, dtype=torch.uint8, device=device)
+        elif idx_dim:
             dt = torch.bfloat16 if idx_dtype == CSA_IDX_BF16 else torch.uint8
             idx = torch.zeros(batch, capacity, idx_dim, dtype=dt, device=device)
         return Cache(fp4=torch.zeros(batch, capacity, dim // 2, dtype=torch.uint8, device=device),
@@ -168,7 +177,7 @@ class Cache:
                                        dtype=torch.uint8, device=device),
                      n_blocks=torch.zeros(batch, dtype=torch.int32, device=device), block=block,
                      idx_key=idx, idx_dtype=idx_dtype, status=torch.zeros(1, dtype=torch.int32, device=device),
-                     scale_fmt=scale_fmt)
+                     scale_fmt=scale_fmt, idx_key_scale=idx_scale)
 
 
 def csa_version() -> int:

@@ -45,6 +45,27 @@ __device__ __forceinline__ uint32_t ordered_key(float s) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// E2M1 code of a scaled value s (|s| < 8), round to nearest with ties to the
+// even code, saturating at 6; the sign bit is kept even when the magnitude
+// rounds to zero. Thresholds are the midpoints between neighbouring
+// magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6; "<=" sends a tie to the lower (even)
+// code, "<" sends it to the upper (even) code.
+__device__ __forceinline__ uint32_t e2m1_code(float s) {
+    uint32_t sign = (__float_as_uint(s) >> 28) & 8u;
+    float a = fabsf(s);
+    uint32_t c = a <= 0.25f ? 0u : a < 0.75f ? 1u : a <= 1.25f ? 2u : a < 1.75f ? 3u
+               : a <= 2.5f ? 4u : a < 3.5f ? 5u : a <= 5.0f ? 6u : 7u;
+    return sign | c;
+}
+
+// E8M0 byte of a 32-element group with largest magnitude amax (X = floor(log2 amax) - 2,
+// clamped to >= -127: zero and subnormal amax land on the clamp; byte = X + 127), and
+// 2^-X as a float, the factor that maps the group onto E2M1's range.
+__device__ __forceinline__ int e8m0_byte(float amax) {
+    return max((int)((__float_as_uint(amax) >> 23) & 0xFF) - 2, 0);
+}
+__device__ __forceinline__ float e8m0_inverse(int byte) { return __uint_as_float((uint32_t)(254 - byte) << 23); }
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

@@ -41,19 +41,6 @@ __device__ __forceinline__ uint32_t e2m1_code_th(float v, const float (&th)[7]) 
     return sign | c;
 }
 
-// E2M1 code of a scaled value s (|s| < 8), round to nearest with ties to the
-// even code, saturating at 6; the sign bit is kept even when the magnitude
-// rounds to zero. Thresholds are the midpoints between neighbouring
-// magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6; "<=" sends a tie to the lower (even)
-// code, "<" sends it to the upper (even) code.
-__device__ __forceinline__ uint32_t e2m1_code(float s) {
-    uint32_t sign = (__float_as_uint(s) >> 28) & 8u;
-    float a = fabsf(s);
-    uint32_t c = a <= 0.25f ? 0u : a < 0.75f ? 1u : a <= 1.25f ? 2u : a < 1.75f ? 3u
-               : a <= 2.5f ? 4u : a < 3.5f ? 5u : a <= 5.0f ? 6u : 7u;
-    return sign | c;
-}
-
 // N consecutive bf16 values as N/2 raw 32-bit words (widest loads that fit).
 template <int N>
 __device__ __forceinline__ void load_raw(const __nv_bfloat16 *p, uint32_t (&w)[N / 2]) {
@@ -100,10 +87,12 @@ struct CompressArgs {
     const int32_t *n_blocks;       // [B]
     uint8_t *fp4;                  // [B][cap][D/2]
     uint8_t *scale;                // [B][cap][D/32] (E8M0) or [B][cap][D/16] (E4M3)
-    uint8_t *idx_key;              // [B][cap][dI * esize] or null
+    uint8_t *idx_key;              // [B][cap][dI * esize], [B][cap][dI/2] (MXFP4 codes) or null
+    uint8_t *idx_key_scale;        // [B][cap][dI/32] (MXFP4 keys) or null
     int32_t *status;
     int m, cap, D, dI;
     int idx_e4m3;
+    int idx_mxfp4;
     int scale_e4m3;                // 1: one E4M3 scale per 16 elements, 0: one E8M0 scale per 32
     int batch;
     int flat;                      // 1: grid over all blocks of all requests (see below)
@@ -334,9 +323,27 @@ pool_quantize_kernel(CompressArgs a) {
         dst[0] = (uint8_t)packed[0];
     }
 
-    // ---- pooled indexer key -> bf16 or e4m3 ----
+    // ---- pooled indexer key -> bf16, e4m3 or MXFP4 ----
     if constexpr (EI > 0) {
-        if (a.idx_e4m3) {
+        if (a.idx_mxfp4) {
+            // the main KV's E8M0 rule per 32 channels; a group spans 32/EI lanes
+            float kv[EI];
+            float kmax = 0.f;
+#pragma unroll
+            for (int k = 0; k < EI; ++k) {
+                kv[k] = acck[k] / den;
+                kmax = fmaxf(kmax, fabsf(kv[k]));
+            }
+#pragma unroll
+            for (int o = 1; o < 32 / EI; o <<= 1) kmax = fmaxf(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+            const int kbyte = max((int)((__float_as_uint(kmax) >> 23) & 0xFF) - 2, 0);
+            const float kinv = __uint_as_float((uint32_t)(254 - kbyte) << 23);
+            uint8_t *kd = a.idx_key + row * (a.dI / 2) + lane * (EI / 2);
+#pragma unroll
+            for (int k = 0; k < EI; k += 2)
+                kd[k / 2] = (uint8_t)(e2m1_code(kv[k] * kinv) | (e2m1_code(kv[k + 1] * kinv) << 4));
+            if (lane % (32 / EI) == 0) a.idx_key_scale[row * (a.dI / 32) + lane / (32 / EI)] = (uint8_t)kbyte;
+        } else if (a.idx_e4m3) {
             uint8_t *kd = a.idx_key + row * a.dI + lane * EI;
 #pragma unroll
             for (int k = 0; k < EI; ++k)
@@ -416,6 +423,8 @@ cudaError_t launch_compress(const csa_cache &c, const void *kv_tok, const void *
     a.D = c.dim;
     a.dI = c.idx_key ? c.idx_dim : 0;
     a.idx_e4m3 = c.idx_dtype == CSA_IDX_E4M3;
+    a.idx_mxfp4 = c.idx_dtype == CSA_IDX_MXFP4;
+    a.idx_key_scale = c.idx_key_scale;
     a.scale_e4m3 = c.scale_fmt == CSA_SCALE_E4M3_16;
     a.batch = c.batch;
     a.flat = c.batch <= kFlatMaxBatch;

@@ -54,9 +54,14 @@ csa_status check_cache(const csa_cache *c) {
     if (!aligned(c->fp4, 16) || !aligned(c->scale, 16) || !aligned(c->n_blocks, 4)) return CSA_ERR_ALIGN;
     if (c->status && !aligned(c->status, 4)) return CSA_ERR_ALIGN;
     if (c->idx_key) {
-        if (c->idx_dtype != CSA_IDX_BF16 && c->idx_dtype != CSA_IDX_E4M3) return CSA_ERR_SHAPE;
+        if (c->idx_dtype != CSA_IDX_BF16 && c->idx_dtype != CSA_IDX_E4M3 && c->idx_dtype != CSA_IDX_MXFP4)
+            return CSA_ERR_SHAPE;
         if (c->idx_dim != 64 && c->idx_dim != 128 && c->idx_dim != 256) return CSA_ERR_UNSUPPORTED;
         if (!aligned(c->idx_key, 16)) return CSA_ERR_ALIGN;
+        if (c->idx_dtype == CSA_IDX_MXFP4) {
+            if (!c->idx_key_scale) return CSA_ERR_NULL;
+            if (!aligned(c->idx_key_scale, 4)) return CSA_ERR_ALIGN;
+        }
     }
     return CSA_OK;
 }
@@ -77,6 +82,7 @@ csa_status check_index_args(const csa_cache *cache, const void *q_idx, const flo
     if (!cache->idx_key || !q_idx || !w || !q_offsets || !q_pos || !sel_idx) return CSA_ERR_NULL;
     if (n_queries < 1 || idx_heads < 1 || topk < 1) return CSA_ERR_SHAPE;
     if (idx_heads > 8 || topk > kMaxTopk) return CSA_ERR_UNSUPPORTED;
+    if (cache->idx_dtype == CSA_IDX_MXFP4 && idx_heads > 4) return CSA_ERR_UNSUPPORTED;
     if (!aligned(q_idx, 16) || !aligned(w, 4) || !aligned(q_offsets, 4) || !aligned(q_pos, 4) ||
         !aligned(sel_idx, 4))
         return CSA_ERR_ALIGN;
@@ -99,7 +105,7 @@ const char *csa_status_string(int32_t status) {
     }
 }
 
-int32_t csa_version(void) { return 102; }
+int32_t csa_version(void) { return 103; }
 
 csa_status csa_compress_quantize(const csa_cache *cache, const void *kv_tok, const void *idx_tok, const float *gate_w,
                                  const int32_t *tok_offsets, int32_t n_tokens, csa_stream_t stream) {

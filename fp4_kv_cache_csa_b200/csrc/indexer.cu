@@ -45,6 +45,7 @@
 // (-0 folded into +0), so selection is exact for the scores computed here.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp4.h>
 #include <cuda_fp8.h>
 
 #include "common.cuh"
@@ -318,7 +319,8 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_bytes) {
 }
 
 struct ScanArgs {
-    const uint8_t *keys;          // [B][cap][dI*esize]
+    const uint8_t *keys;          // [B][cap][dI*esize] (MXFP4: codes [B][cap][dI/2])
+    const uint8_t *key_scales;    // MXFP4 keys: [B][cap][dI/32] E8M0 bytes, else null
     const __nv_bfloat16 *q_idx;   // [Nq][H_I][dI]
     const float *w;               // [Nq][H_I]
     const int32_t *req, *n_vis;
@@ -350,20 +352,51 @@ struct ScanArgs {
 // t*EPT + 4s + {0,1} as MMA k-columns 2t,2t+1 and t*EPT + 4s + {2,3} as
 // columns 2t+8,2t+9 of k-step s. The query's B fragment uses the identical
 // map, so each thread reads one contiguous stretch of every row.
-template <bool E4M3, int KS>
+// Key storage (template argument KT of the scan).
+constexpr int kKeyBf16 = 0;
+constexpr int kKeyE4M3 = 1;
+constexpr int kKeyMxfp4 = 2;  // E2M1 codes + one E8M0 scale per 32 channels (separate plane)
+
+template <int KT, int KS>
 struct ScanCfg {
     static constexpr int EPT = 4 * KS;                   // channels per thread per row
-    static constexpr int ROW_BYTES_T = EPT * (E4M3 ? 1 : 2);
-    static constexpr int NV = ROW_BYTES_T / 16;          // uint4 loads per thread per row
-    static constexpr int KEY_BYTES = 4 * ROW_BYTES_T;    // bytes per key row
-    static constexpr int U = (16 / (2 * NV)) > 0 ? 16 / (2 * NV) : 1;  // groups in flight per warp
+    static constexpr int ROW_BYTES_T = KT == kKeyBf16 ? EPT * 2 : KT == kKeyE4M3 ? EPT : EPT / 2;
+    static constexpr int NV = (ROW_BYTES_T + 15) / 16;   // 16-byte registers per thread per row
+    static constexpr int KEY_BYTES = 4 * ROW_BYTES_T;    // bytes per key row (MXFP4: codes only)
+    static constexpr int GROUPS = KS / 2;                // 32-channel groups per key (d_I / 32)
+    // 16-key groups in flight per warp
+    static constexpr int U = KT == kKeyMxfp4 ? (KS == 16 ? 2 : 4) : ((16 / (2 * NV)) > 0 ? 16 / (2 * NV) : 1);
+    // MXFP4: MMAs per k-step, each producing (head, group) columns n = 2 head + slot, and the
+    // accumulator sets (the groups a k-step touches change halfway at d_I = 256)
+    static constexpr int NMMA = KT == kKeyMxfp4 && KS > 4 ? 2 : 1;
+    static constexpr int NKH = KT == kKeyMxfp4 && KS == 16 ? 2 : 1;
+    static_assert(NMMA * NKH >= 1, "accumulator sets");
 };
+
+// MXFP4 keys: the 32-channel group of accumulator set (v, kh), column slot j.
+template <int KS>
+__host__ __device__ constexpr int mx_group(int v, int kh, int j) {
+    return KS == 4 ? j : KS == 8 ? 2 * v + j : 2 * (2 * v + j) + kh;
+}
+
+// 2^(byte - 127) as a float (E8M0 value; byte 0 is the subnormal 2^-127).
+__device__ __forceinline__ float e8m0_value(uint32_t byte) {
+    return byte ? __uint_as_float(byte << 23) : __uint_as_float(0x00400000u);
+}
+
+// Two E2M1 codes (low nibble first) -> packed f16x2 (exact: E2M1 is a subset of f16).
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
+    __half2_raw h = __nv_cvt_fp4x2_to_halfraw2((__nv_fp4x2_storage_t)(byte & 0xFFu), __NV_E2M1);
+    return (uint32_t)h.x | ((uint32_t)h.y << 16);
+}
 
 // POOL: keys are pool positions (Reindex), mapped to cache blocks through a.pool.
 // FUSED: the kernel computes the schedule itself (a.fused; at most kFusedScheduleQueries queries).
-template <bool E4M3, int KS, bool POOL, bool FUSED>
+template <int KT, int KS, bool POOL, bool FUSED>
 __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a) {
-    using C = ScanCfg<E4M3, KS>;
+    using C = ScanCfg<KT, KS>;
+    constexpr bool E4M3 = KT == kKeyE4M3;
+    constexpr bool MX = KT == kKeyMxfp4;
     grid_dep_wait();    // the schedule kernel's ranges, or the inputs of the fused schedule
     grid_dep_launch();
     __shared__ __align__(16) uint32_t hist[kBins];
@@ -427,15 +460,18 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a) {
         }
 
         // ---- query fragments: B[k][n=head] with the dimension permutation ----
-        uint32_t bq[KS][2];
-        float w_lo = 0.f, w_hi = 0.f;  // weights of heads 2t and 2t+1 (scaled, see below)
+        // (MXFP4 keys: B[k][n = 2 head + slot] per MMA of a k-step, see below)
+        uint32_t bq[KS][C::NMMA][2];
+        float w_lo = 0.f, w_hi = 0.f;  // weights of heads 2t and 2t+1 (scaled, see below); MXFP4: head t
+        float fq[C::GROUPS];           // MXFP4: 2^X of head t's query groups
         {
             float qv[C::EPT];
-            const bool live = g < a.H_I;
+            const int qh = MX ? (g >> 1) : g;  // the head this thread's B column belongs to
+            const bool live = qh < a.H_I;
 #pragma unroll
             for (int k = 0; k < C::EPT; ++k) qv[k] = 0.f;
             if (live) {
-                const __nv_bfloat16 *qp = a.q_idx + ((size_t)i * a.H_I + g) * (C::EPT * 4) + t * C::EPT;
+                const __nv_bfloat16 *qp = a.q_idx + ((size_t)i * a.H_I + qh) * (C::EPT * 4) + t * C::EPT;
 #pragma unroll
                 for (int v = 0; v < C::EPT / 8; ++v) {
                     uint4 u = __ldg(reinterpret_cast<const uint4 *>(qp) + v);
@@ -449,7 +485,59 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a) {
                 }
             }
             int kexp = 0;  // power-of-two scale of this head's query (fp16 path only)
-            if constexpr (E4M3) {
+            if constexpr (MX) {
+                // the query quantized like the keys: per 32 channels of each head, E8M0 scale
+                // X = floor(log2 amax) - 2, E2M1 codes of q / 2^X (round to nearest even,
+                // saturating). The B operand carries the codes' values (exact in f16); the
+                // scales multiply the per-group products afterwards. This thread's EPT channels
+                // are half a group (d_I = 64, the other half in lane ^ 1), one, or two groups.
+                constexpr int GT = C::EPT >= 32 ? C::EPT / 32 : 1;  // groups held by this thread
+                constexpr int GW = C::EPT >= 32 ? 32 : C::EPT;      // channels of a group held here
+                int xb[GT];
+                uint32_t cw[C::EPT / 8];  // the codes, 8 per word (4 bits each, element 2i low)
+#pragma unroll
+                for (int gg = 0; gg < GT; ++gg) {
+                    float mx = 0.f;
+#pragma unroll
+                    for (int k = 0; k < GW; ++k) mx = fmaxf(mx, fabsf(qv[gg * GW + k]));
+                    if constexpr (C::EPT < 32) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                    xb[gg] = e8m0_byte(mx);
+                    const float inv = e8m0_inverse(xb[gg]);
+#pragma unroll
+                    for (int k = 0; k < GW; k += 8) {
+                        uint32_t wv = 0;
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) wv |= e2m1_code(qv[gg * GW + k + e] * inv) << (4 * e);
+                        cw[(gg * GW + k) / 8] = wv;
+                    }
+                }
+                // B registers: column n = g (head g >> 1, slot g & 1). In k-step s this thread
+                // supplies k-columns 2t, 2t+1, 2t+8, 2t+9 from its channels EPT t + 4s + 0..3,
+                // which lie in one group; the MMA v of the step takes the groups of quad
+                // threads {2v, 2v+1} (d_I = 64: thread pairs {0,1} and {2,3} are groups 0, 1
+                // of the single MMA), so only the slot that matches keeps the query values.
+#pragma unroll
+                for (int s2 = 0; s2 < KS; ++s2) {
+                    const uint32_t byte0 = (cw[s2 / 2] >> (16 * (s2 & 1))) & 0xFFu;      // channels 4s, 4s+1
+                    const uint32_t byte1 = (cw[s2 / 2] >> (16 * (s2 & 1) + 8)) & 0xFFu;  // channels 4s+2, 4s+3
+#pragma unroll
+                    for (int v = 0; v < C::NMMA; ++v) {
+                        const bool mine = KS == 4 ? ((t >> 1) == (g & 1)) : ((t >> 1) == v && (t & 1) == (g & 1));
+                        bq[s2][v][0] = (live && mine) ? e2m1x2_to_f16x2(byte0) : 0u;
+                        bq[s2][v][1] = (live && mine) ? e2m1x2_to_f16x2(byte1) : 0u;
+                    }
+                }
+                // head t's group scales for the epilogue: group G of head h was quantized by
+                // the threads with column g = 2h (or 2h + 1) and quad position owning G
+#pragma unroll
+                for (int G = 0; G < C::GROUPS; ++G) {
+                    const int owner = KS == 4 ? 2 * G : KS == 8 ? G : (G >> 1);
+                    const int src = 4 * (2 * (t & 3)) + owner;
+                    const int mine = GT == 2 ? xb[(KS == 16 && (G & 1)) ? 1 : 0] : xb[0];
+                    fq[G] = e8m0_value((uint32_t)__shfl_sync(0xffffffffu, mine, src));
+                }
+                if (t < a.H_I) w_lo = a.w[(size_t)i * a.H_I + t];
+            } else if constexpr (E4M3) {
                 // fp16 operands: scale head h's query by 2^k_h so its largest
                 // magnitude lands in [2^14, 2^15); every bf16 value within 2^31
                 // of it converts exactly. ReLU(2^k x) = 2^k ReLU(x), so the
@@ -466,23 +554,25 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a) {
                 for (int s = 0; s < KS; ++s) {
                     __half2 h0 = __floats2half2_rn(qv[4 * s] * sc, qv[4 * s + 1] * sc);
                     __half2 h1 = __floats2half2_rn(qv[4 * s + 2] * sc, qv[4 * s + 3] * sc);
-                    bq[s][0] = *reinterpret_cast<uint32_t *>(&h0);
-                    bq[s][1] = *reinterpret_cast<uint32_t *>(&h1);
+                    bq[s][0][0] = *reinterpret_cast<uint32_t *>(&h0);
+                    bq[s][0][1] = *reinterpret_cast<uint32_t *>(&h1);
                 }
             } else {
 #pragma unroll
                 for (int s = 0; s < KS; ++s) {
                     __nv_bfloat162 h0 = __floats2bfloat162_rn(qv[4 * s], qv[4 * s + 1]);
                     __nv_bfloat162 h1 = __floats2bfloat162_rn(qv[4 * s + 2], qv[4 * s + 3]);
-                    bq[s][0] = *reinterpret_cast<uint32_t *>(&h0);
-                    bq[s][1] = *reinterpret_cast<uint32_t *>(&h1);
+                    bq[s][0][0] = *reinterpret_cast<uint32_t *>(&h0);
+                    bq[s][0][1] = *reinterpret_cast<uint32_t *>(&h1);
                 }
             }
-            const int h0 = 2 * t, h1 = 2 * t + 1;
-            const int k0 = __shfl_sync(0xffffffffu, kexp, (4 * h0) & 31);
-            const int k1 = __shfl_sync(0xffffffffu, kexp, (4 * h1) & 31);
-            if (h0 < a.H_I) w_lo = ldexpf(a.w[(size_t)i * a.H_I + h0], -k0);
-            if (h1 < a.H_I) w_hi = ldexpf(a.w[(size_t)i * a.H_I + h1], -k1);
+            if constexpr (!MX) {
+                const int h0 = 2 * t, h1 = 2 * t + 1;
+                const int k0 = __shfl_sync(0xffffffffu, kexp, (4 * h0) & 31);
+                const int k1 = __shfl_sync(0xffffffffu, kexp, (4 * h1) & 31);
+                if (h0 < a.H_I) w_lo = ldexpf(a.w[(size_t)i * a.H_I + h0], -k0);
+                if (h1 < a.H_I) w_hi = ldexpf(a.w[(size_t)i * a.H_I + h1], -k1);
+            }
         }
 
         for (int k = threadIdx.x; k < kBins; k += kScanThreads) hist[k] = 0;
@@ -492,8 +582,10 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a) {
         float *srow = a.scores + (size_t)i * a.rows;
         const int32_t *prow = POOL ? a.pool + (size_t)i * a.pool_p : nullptr;
 
+        const uint8_t *kscale = MX ? a.key_scales + (size_t)b * a.cap * C::GROUPS : nullptr;
         for (long long u0 = warp; u0 < nloc; u0 += (long long)kScanWarps * C::U) {
             uint4 raw[C::U][2][C::NV];
+            uint2 ksr[MX ? C::U : 1][2];  // MXFP4: the scale bytes of the two rows
 #pragma unroll
             for (int uu = 0; uu < C::U; ++uu) {
                 const long long lg = lg0 + u0 + (long long)kScanWarps * uu;
@@ -506,37 +598,97 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a) {
                     if (POOL && ok)  // a plain load behind the bound check (never issued beyond the row)
                         row = ((long long)prow[r >> a.pool_shift] << a.pool_shift) + (r & ((1 << a.pool_shift) - 1));
                     const uint4 *src = reinterpret_cast<const uint4 *>(kbase + row * C::KEY_BYTES + t * C::ROW_BYTES_T);
+                    if constexpr (C::ROW_BYTES_T >= 16) {
 #pragma unroll
-                    for (int v = 0; v < C::NV; ++v) raw[uu][half][v] = ok ? ld_stream(src + v, pol_stream) : make_uint4(0, 0, 0, 0);
+                        for (int v = 0; v < C::NV; ++v)
+                            raw[uu][half][v] = ok ? ld_stream(src + v, pol_stream) : make_uint4(0, 0, 0, 0);
+                    } else {  // 8 bytes per thread (MXFP4 at d_I = 64)
+                        const uint2 w2 = ok ? __ldcs(reinterpret_cast<const uint2 *>(src)) : make_uint2(0, 0);
+                        raw[uu][half][0] = make_uint4(w2.x, w2.y, 0, 0);
+                    }
+                    if constexpr (MX) {
+                        const uint8_t *sp = kscale + row * C::GROUPS;
+                        uint2 sv = make_uint2(0, 0);
+                        if (ok) {
+                            if constexpr (C::GROUPS == 8) sv = __ldcs(reinterpret_cast<const uint2 *>(sp));
+                            else if constexpr (C::GROUPS == 4) sv.x = __ldcs(reinterpret_cast<const unsigned int *>(sp));
+                            else sv.x = __ldcs(reinterpret_cast<const unsigned short *>(sp));
+                        }
+                        ksr[uu][half] = sv;
+                    }
                 }
             }
 #pragma unroll
             for (int uu = 0; uu < C::U; ++uu) {
                 const long long lg = lg0 + u0 + (long long)kScanWarps * uu;
                 const bool gv = (u0 + (long long)kScanWarps * uu) < nloc;
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
                 const uint32_t *w0 = reinterpret_cast<const uint32_t *>(raw[uu][0]);
                 const uint32_t *w1 = reinterpret_cast<const uint32_t *>(raw[uu][1]);
+                float p0, p1;
+                if constexpr (MX) {
+                    // per (MMA v, k-half kh): D[row][n = 2 head + slot] = sum over the channels of
+                    // one group of E2M1 x E2M1 products (exact in fp32); this thread holds head t,
+                    // slots 0 and 1, of rows g and g + 8
+                    float acc[C::NMMA][C::NKH][4];
 #pragma unroll
-                for (int s = 0; s < KS; ++s) {
-                    uint32_t af[4];
-                    if constexpr (E4M3) {
-                        af[0] = e4m3x2_to_f16x2(w0[s]);          // row g,   cols 2t,2t+1
-                        af[1] = e4m3x2_to_f16x2(w1[s]);          // row g+8, cols 2t,2t+1
-                        af[2] = e4m3x2_to_f16x2(w0[s] >> 16);    // row g,   cols 2t+8,2t+9
-                        af[3] = e4m3x2_to_f16x2(w1[s] >> 16);    // row g+8, cols 2t+8,2t+9
-                        mma_f16(acc, af, bq[s][0], bq[s][1]);
-                    } else {
-                        af[0] = w0[2 * s];
-                        af[1] = w1[2 * s];
-                        af[2] = w0[2 * s + 1];
-                        af[3] = w1[2 * s + 1];
-                        mma_bf16(acc, af, bq[s][0], bq[s][1]);
+                    for (int v = 0; v < C::NMMA; ++v)
+#pragma unroll
+                        for (int kh = 0; kh < C::NKH; ++kh)
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) acc[v][kh][e] = 0.f;
+#pragma unroll
+                    for (int s = 0; s < KS; ++s) {
+                        const int kh = C::NKH == 2 ? (s >= KS / 2) : 0;
+                        // channels 4s..4s+3 = code bytes 2s, 2s+1 of this thread's part of the row
+                        const uint32_t c0 = (w0[s / 2] >> (16 * (s & 1))) & 0xFFFFu;  // row g
+                        const uint32_t c1 = (w1[s / 2] >> (16 * (s & 1))) & 0xFFFFu;  // row g + 8
+                        uint32_t af[4];
+                        af[0] = e2m1x2_to_f16x2(c0);       // row g,   cols 2t,2t+1
+                        af[1] = e2m1x2_to_f16x2(c1);       // row g+8, cols 2t,2t+1
+                        af[2] = e2m1x2_to_f16x2(c0 >> 8);  // row g,   cols 2t+8,2t+9
+                        af[3] = e2m1x2_to_f16x2(c1 >> 8);  // row g+8, cols 2t+8,2t+9
+#pragma unroll
+                        for (int v = 0; v < C::NMMA; ++v) mma_f16(acc[v][kh], af, bq[s][v][0], bq[s][v][1]);
                     }
+                    // head t's dot product with each row: the groups' sums times both scales
+                    float d0 = 0.f, d1 = 0.f;
+#pragma unroll
+                    for (int v = 0; v < C::NMMA; ++v)
+#pragma unroll
+                        for (int kh = 0; kh < C::NKH; ++kh)
+#pragma unroll
+                            for (int j = 0; j < 2; ++j) {
+                                const int G = mx_group<KS>(v, kh, j);
+                                const uint32_t b0 = ((G < 4 ? ksr[uu][0].x : ksr[uu][0].y) >> (8 * (G & 3))) & 0xFFu;
+                                const uint32_t b1 = ((G < 4 ? ksr[uu][1].x : ksr[uu][1].y) >> (8 * (G & 3))) & 0xFFu;
+                                d0 = fmaf(acc[v][kh][j] * e8m0_value(b0), fq[G], d0);
+                                d1 = fmaf(acc[v][kh][2 + j] * e8m0_value(b1), fq[G], d1);
+                            }
+                    p0 = w_lo * fmaxf(d0, 0.f);
+                    p1 = w_lo * fmaxf(d1, 0.f);
+                } else {
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int s = 0; s < KS; ++s) {
+                        uint32_t af[4];
+                        if constexpr (E4M3) {
+                            af[0] = e4m3x2_to_f16x2(w0[s]);          // row g,   cols 2t,2t+1
+                            af[1] = e4m3x2_to_f16x2(w1[s]);          // row g+8, cols 2t,2t+1
+                            af[2] = e4m3x2_to_f16x2(w0[s] >> 16);    // row g,   cols 2t+8,2t+9
+                            af[3] = e4m3x2_to_f16x2(w1[s] >> 16);    // row g+8, cols 2t+8,2t+9
+                            mma_f16(acc, af, bq[s][0][0], bq[s][0][1]);
+                        } else {
+                            af[0] = w0[2 * s];
+                            af[1] = w1[2 * s];
+                            af[2] = w0[2 * s + 1];
+                            af[3] = w1[2 * s + 1];
+                            mma_bf16(acc, af, bq[s][0][0], bq[s][0][1]);
+                        }
+                    }
+                    // acc[0..1]: row g, heads 2t,2t+1; acc[2..3]: row g+8
+                    p0 = w_lo * fmaxf(acc[0], 0.f) + w_hi * fmaxf(acc[1], 0.f);
+                    p1 = w_lo * fmaxf(acc[2], 0.f) + w_hi * fmaxf(acc[3], 0.f);
                 }
-                // acc[0..1]: row g, heads 2t,2t+1; acc[2..3]: row g+8
-                float p0 = w_lo * fmaxf(acc[0], 0.f) + w_hi * fmaxf(acc[1], 0.f);
-                float p1 = w_lo * fmaxf(acc[2], 0.f) + w_hi * fmaxf(acc[3], 0.f);
                 p0 += __shfl_xor_sync(0xffffffffu, p0, 1);
                 p1 += __shfl_xor_sync(0xffffffffu, p1, 1);
                 p0 += __shfl_xor_sync(0xffffffffu, p0, 2);
@@ -1624,14 +1776,24 @@ __global__ void __launch_bounds__(kCountThreads) reindex_count_kernel(const int3
     }
 }
 
-template <bool E4M3, int KS>
+template <int KT, int KS>
 cudaError_t launch_scan(const ScanArgs &sa, int grid, cudaStream_t s) {
     if (sa.pool) {
-        if (sa.fused) return launch_pdl(scan_kernel<E4M3, KS, true, true>, dim3(grid), dim3(kScanThreads), 0, s, sa);
-        return launch_pdl(scan_kernel<E4M3, KS, true, false>, dim3(grid), dim3(kScanThreads), 0, s, sa);
+        if (sa.fused) return launch_pdl(scan_kernel<KT, KS, true, true>, dim3(grid), dim3(kScanThreads), 0, s, sa);
+        return launch_pdl(scan_kernel<KT, KS, true, false>, dim3(grid), dim3(kScanThreads), 0, s, sa);
     }
-    if (sa.fused) return launch_pdl(scan_kernel<E4M3, KS, false, true>, dim3(grid), dim3(kScanThreads), 0, s, sa);
-    return launch_pdl(scan_kernel<E4M3, KS, false, false>, dim3(grid), dim3(kScanThreads), 0, s, sa);
+    if (sa.fused) return launch_pdl(scan_kernel<KT, KS, false, true>, dim3(grid), dim3(kScanThreads), 0, s, sa);
+    return launch_pdl(scan_kernel<KT, KS, false, false>, dim3(grid), dim3(kScanThreads), 0, s, sa);
+}
+
+template <int KT>
+cudaError_t launch_scan_kt(const ScanArgs &sa, int idx_dim, int grid, cudaStream_t s) {
+    switch (idx_dim / 16) {
+        case 4: return launch_scan<KT, 4>(sa, grid, s);
+        case 8: return launch_scan<KT, 8>(sa, grid, s);
+        case 16: return launch_scan<KT, 16>(sa, grid, s);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 // One selection: score rows, thresholds and output of a workspace.
@@ -1727,6 +1889,7 @@ cudaError_t index_pipeline(const csa_cache &c, const void *q_idx, const float *w
 
     ScanArgs sa;
     sa.keys = static_cast<const uint8_t *>(c.idx_key);
+    sa.key_scales = c.idx_dtype == CSA_IDX_MXFP4 ? c.idx_key_scale : nullptr;
     sa.q_idx = static_cast<const __nv_bfloat16 *>(q_idx);
     sa.w = w;
     sa.req = ws.req;
@@ -1755,7 +1918,6 @@ cudaError_t index_pipeline(const csa_cache &c, const void *q_idx, const float *w
     sa.batch = c.batch;
     sa.m = c.block;
     const int grid = min(num_sms, kMaxScanCtas);
-    const bool e4 = c.idx_dtype == CSA_IDX_E4M3;
     if (gemm) {
         err = launch_prefill_scores(c.idx_key, c.batch, c.capacity, c.idx_dim, q_idx, w, Nq, H_I, ws.req, ws.n_vis, ws.scores,
                                     rows, c.status, num_sms, s);
@@ -1774,12 +1936,9 @@ cudaError_t index_pipeline(const csa_cache &c, const void *q_idx, const float *w
         const SelJob job{&ws, Nq, rows, topk, sel_idx, pool, pool_shift, pool_p};
         return launch_select(job, nullptr, num_sms, s);
     }
-    switch (c.idx_dim / 16) {
-        case 4: err = e4 ? launch_scan<true, 4>(sa, grid, s) : launch_scan<false, 4>(sa, grid, s); break;
-        case 8: err = e4 ? launch_scan<true, 8>(sa, grid, s) : launch_scan<false, 8>(sa, grid, s); break;
-        case 16: err = e4 ? launch_scan<true, 16>(sa, grid, s) : launch_scan<false, 16>(sa, grid, s); break;
-        default: return cudaErrorInvalidValue;
-    }
+    err = c.idx_dtype == CSA_IDX_MXFP4 ? launch_scan_kt<kKeyMxfp4>(sa, c.idx_dim, grid, s)
+          : c.idx_dtype == CSA_IDX_E4M3 ? launch_scan_kt<kKeyE4M3>(sa, c.idx_dim, grid, s)
+                                         : launch_scan_kt<kKeyBf16>(sa, c.idx_dim, grid, s);
     if (err != cudaSuccess) return err;
     // the exact top-k of each query among its segments' candidates
     MergeArgs ma;

@@ -63,7 +63,15 @@ typedef enum {
     CSA_ERR_CUDA = 6         /* a CUDA runtime call or kernel launch failed     */
 } csa_status;
 
-typedef enum { CSA_IDX_BF16 = 0, CSA_IDX_E4M3 = 1 } csa_idx_dtype;
+/* Storage of the pooled indexer keys:
+ *   CSA_IDX_BF16   bf16;
+ *   CSA_IDX_E4M3   OCP FP8 E4M3, round to nearest even, saturating, unscaled;
+ *   CSA_IDX_MXFP4  MXFP4 like the main KV: E2M1 codes (two per byte, element
+ *                  2i in the low nibble) in idx_key, one E8M0 scale byte per 32
+ *                  channels in idx_key_scale. With these keys the indexer query
+ *                  is quantized the same way (per 32 channels of each head)
+ *                  before the scores, so every product is exact. */
+typedef enum { CSA_IDX_BF16 = 0, CSA_IDX_E4M3 = 1, CSA_IDX_MXFP4 = 2 } csa_idx_dtype;
 
 /* Scale format of the FP4 main KV (E2M1 elements in both):
  *   CSA_SCALE_E8M0_32  one E8M0 byte per 32 elements, value 2^(byte - 127)
@@ -88,13 +96,16 @@ typedef enum { CSA_SCALE_E8M0_32 = 0, CSA_SCALE_E4M3_16 = 1 } csa_scale_fmt;
  *           [batch][capacity][dim/16]  E4M3 bytes                      (CSA_SCALE_E4M3_16)
  *   idx_key [batch][capacity][idx_dim] bf16 or e4m3 pooled indexer keys; NULL for
  *                                      a cache that is only attended densely (HCA)
+ *           [batch][capacity][idx_dim/2]  MXFP4 codes of the keys (CSA_IDX_MXFP4)
+ *   idx_key_scale [batch][capacity][idx_dim/32]  their E8M0 scale bytes
+ *                                      (CSA_IDX_MXFP4 only, else NULL; 4-byte aligned)
  *   n_blocks [batch]                   filled blocks per request; advanced by
  *                                      csa_compress_quantize
  *   status                             one int32 of CSA_DEV_* bits, or NULL
  * An element's value is E2M1(code) * 2^(scale - 127) for E8M0 scales and
  * E2M1(code) * E4M3(scale) for E4M3 scales (the scale byte of its group).
- * scale_fmt was added after status, so the offsets of the other fields are
- * those of ABI version 100.
+ * scale_fmt (ABI 101) and idx_key_scale (ABI 103) were appended, so the
+ * offsets of the other fields are those of ABI version 100.
  */
 typedef struct {
     int32_t batch;     /* requests, >= 1                                  */
@@ -109,6 +120,7 @@ typedef struct {
     int32_t *n_blocks;
     int32_t *status;
     int32_t scale_fmt; /* csa_scale_fmt                                  */
+    uint8_t *idx_key_scale; /* CSA_IDX_MXFP4 key scales, else NULL         */
 } csa_cache;
 
 /* Human-readable name of a csa_status value. Never NULL. */

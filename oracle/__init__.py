@@ -26,6 +26,7 @@ _lib = None
 
 IDX_BF16 = 0
 IDX_E4M3 = 1
+IDX_MXFP4 = 2  # E2M1 codes [.., dI/2] + one E8M0 scale per 32 channels [.., dI/32]
 
 # scale formats of the FP4 cache: E8M0 per 32 elements (OCP MXFP4), E4M3 per 16
 SCALE_E8M0_32 = 0
@@ -72,9 +73,9 @@ def _load():
         lib.orc_mxfp4_quantize_group.restype = None
         lib.orc_e4m3x16_quantize_group.argtypes = [P, P, P]
         lib.orc_e4m3x16_quantize_group.restype = None
-        lib.orc_compress.argtypes = [I, I, I, I, I, I, I, P, P, P, P, P, P, P, P, P, P]
+        lib.orc_compress.argtypes = [I, I, I, I, I, I, I, P, P, P, P, P, P, P, P, P, P, P]
         lib.orc_compress.restype = I
-        lib.orc_index_scores.argtypes = [I, I, I, I, I, I, I, P, P, P, P, P, P, P, P]
+        lib.orc_index_scores.argtypes = [I, I, I, I, I, I, I, P, P, P, P, P, P, P, P, P]
         lib.orc_index_scores.restype = None
         lib.orc_topk.argtypes = [I, I, I, P, P, P]
         lib.orc_topk.restype = None
@@ -194,12 +195,13 @@ def mxfp4_dequantize(fp4_rows, scale_rows):
 # ---- the method ------------------------------------------------------------
 
 def compress(kv_tok, idx_tok, w_g, tok_offsets, n_blocks, *, m, cap, idx_dtype=IDX_BF16,
-             scale_fmt=SCALE_E8M0_32, fp4=None, scale=None, idx_key=None, return_pooled=False):
+             scale_fmt=SCALE_E8M0_32, fp4=None, scale=None, idx_key=None, idx_key_scale=None,
+             return_pooled=False):
     """Gated m-token pooling + FP4 quantization (rows a1, a2), scales per scale_fmt.
 
     kv_tok [T, D] uint16 (bf16 bits), idx_tok [T, dI] uint16 or None, w_g [D] float32,
     tok_offsets [B+1] int32, n_blocks [B] int32 (copied, returned updated).
-    Returns dict(fp4, scale, idx_key, n_blocks[, pooled]).
+    Returns dict(fp4, scale, idx_key, idx_key_scale (MXFP4 keys only), n_blocks[, pooled]).
     """
     kv_tok = _c(kv_tok, np.uint16)
     T, D = kv_tok.shape
@@ -209,34 +211,45 @@ def compress(kv_tok, idx_tok, w_g, tok_offsets, n_blocks, *, m, cap, idx_dtype=I
     dI = 0 if idx_tok is None else idx_tok.shape[1]
     idx_tok = _c(idx_tok, np.uint16)
     w_g = _c(w_g, np.float32)
-    kb = dI * (2 if idx_dtype == IDX_BF16 else 1)
+    kb = {IDX_BF16: 2 * dI, IDX_E4M3: dI, IDX_MXFP4: dI // 2}[idx_dtype]
     fp4 = np.zeros((B, cap, D // 2), np.uint8) if fp4 is None else fp4
     scale = np.zeros((B, cap, D // group_size(scale_fmt)), np.uint8) if scale is None else scale
     assert scale.shape == (B, cap, D // group_size(scale_fmt))
     if idx_tok is not None and idx_key is None:
         idx_key = np.zeros((B, cap, kb), np.uint8)
+    if idx_tok is not None and idx_dtype == IDX_MXFP4 and idx_key_scale is None:
+        idx_key_scale = np.zeros((B, cap, dI // 32), np.uint8)
     pooled = np.zeros((B, cap, D), np.float32) if return_pooled else None
     pooled_idx = np.zeros((B, cap, dI), np.float32) if (return_pooled and idx_tok is not None) else None
     st = _load().orc_compress(B, D, dI, m, idx_dtype, scale_fmt, cap, _ptr(kv_tok), _ptr(idx_tok), _ptr(w_g),
                               _ptr(tok_offsets), _ptr(n_blocks), _ptr(fp4), _ptr(scale),
-                              _ptr(idx_key) if idx_tok is not None else None, _ptr(pooled), _ptr(pooled_idx))
+                              _ptr(idx_key) if idx_tok is not None else None,
+                              _ptr(idx_key_scale) if idx_dtype == IDX_MXFP4 else None, _ptr(pooled),
+                              _ptr(pooled_idx))
     out = dict(fp4=fp4, scale=scale, idx_key=idx_key, n_blocks=n_blocks, status=st)
+    if idx_dtype == IDX_MXFP4:
+        out["idx_key_scale"] = idx_key_scale
     if return_pooled:
         out["pooled"] = pooled
         out["pooled_idx"] = pooled_idx
     return out
 
 
-def index_scores(idx_key, n_blocks, q_offsets, q_pos, q_idx, w, *, m, idx_dtype=IDX_BF16):
-    """Indexer scores (row a3). idx_key [B, cap, key_bytes] uint8, q_idx [Nq, H_I, dI] uint16,
-    w [Nq, H_I] float32. Returns (scores [Nq, cap] float32, n_vis [Nq] int32)."""
+def index_scores(idx_key, n_blocks, q_offsets, q_pos, q_idx, w, *, m, idx_dtype=IDX_BF16, idx_key_scale=None):
+    """Indexer scores (row a3). idx_key [B, cap, key_bytes] uint8 (MXFP4: codes [B, cap, dI/2] and
+    idx_key_scale [B, cap, dI/32]), q_idx [Nq, H_I, dI] uint16, w [Nq, H_I] float32.
+    Returns (scores [Nq, cap] float32, n_vis [Nq] int32)."""
     idx_key = _c(idx_key, np.uint8)
     B, cap, _ = idx_key.shape
     q_idx = _c(q_idx, np.uint16)
     Nq, H_I, dI = q_idx.shape
+    if idx_dtype == IDX_MXFP4:
+        idx_key_scale = _c(idx_key_scale, np.uint8)
+        assert idx_key.shape == (B, cap, dI // 2) and idx_key_scale.shape == (B, cap, dI // 32)
     scores = np.empty((Nq, cap), np.float32)
     n_vis = np.zeros(Nq, np.int32)
-    _load().orc_index_scores(B, Nq, H_I, dI, idx_dtype, m, cap, _ptr(idx_key), _ptr(_c(n_blocks, np.int32)),
+    _load().orc_index_scores(B, Nq, H_I, dI, idx_dtype, m, cap, _ptr(idx_key),
+                             _ptr(idx_key_scale) if idx_dtype == IDX_MXFP4 else None, _ptr(_c(n_blocks, np.int32)),
                              _ptr(_c(q_offsets, np.int32)), _ptr(_c(q_pos, np.int32)), _ptr(q_idx),
                              _ptr(_c(w, np.float32)), _ptr(scores), _ptr(n_vis))
     return scores, n_vis
@@ -271,8 +284,9 @@ def reindex_topk(scores, n_vis, pool, *, G, k):
     return sel
 
 
-def index_topk(idx_key, n_blocks, q_offsets, q_pos, q_idx, w, *, m, k, idx_dtype=IDX_BF16):
-    scores, n_vis = index_scores(idx_key, n_blocks, q_offsets, q_pos, q_idx, w, m=m, idx_dtype=idx_dtype)
+def index_topk(idx_key, n_blocks, q_offsets, q_pos, q_idx, w, *, m, k, idx_dtype=IDX_BF16, idx_key_scale=None):
+    scores, n_vis = index_scores(idx_key, n_blocks, q_offsets, q_pos, q_idx, w, m=m, idx_dtype=idx_dtype,
+                                 idx_key_scale=idx_key_scale)
     return topk(scores, n_vis, k), scores, n_vis
 
 

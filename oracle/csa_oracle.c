@@ -156,16 +156,27 @@ static double fp4_element(const uint8_t *fp4_row, const uint8_t *scale_row, int 
     return orc_e2m1_decode(code) * orc_e4m3_decode(sb);
 }
 
-static double idx_key_element(const uint8_t *key_row, int idx_dtype, int c) {
+/* Element c of one stored indexer key: bf16 (idx_dtype 0), e4m3 (1), or MXFP4
+ * (2: codes two per byte, element 2i in the low nibble, and one E8M0 scale byte
+ * per 32 elements in scale_row). */
+static double idx_key_element(const uint8_t *key_row, const uint8_t *scale_row, int idx_dtype, int c) {
     if (idx_dtype == 0) {
         uint16_t bits;
         memcpy(&bits, key_row + 2 * c, 2);
         return orc_bf16_decode(bits);
     }
+    if (idx_dtype == 2) {
+        uint8_t byte = key_row[c / 2];
+        uint8_t code = (c % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+        return ldexp(orc_e2m1_decode(code), (int)scale_row[c / 32] - 127);
+    }
     return orc_e4m3_decode(key_row[c]);
 }
 
-static size_t idx_key_bytes(int idx_dtype, int dI) { return (size_t)dI * (idx_dtype == 0 ? 2 : 1); }
+/* Bytes of one stored indexer key (codes only for MXFP4; its scales are a plane of their own). */
+static size_t idx_key_bytes(int idx_dtype, int dI) {
+    return idx_dtype == 0 ? (size_t)dI * 2 : idx_dtype == 2 ? (size_t)dI / 2 : (size_t)dI;
+}
 
 /* ======================================================================
  * a1 + a2: gated block pooling, then quantization of the pooled block
@@ -173,7 +184,7 @@ static size_t idx_key_bytes(int idx_dtype, int dI) { return (size_t)dI * (idx_dt
 int orc_compress(int B, int D, int dI, int m, int idx_dtype, int scale_fmt, int cap,
                  const uint16_t *kv_tok, const uint16_t *idx_tok, const float *w_g,
                  const int32_t *tok_offsets, int32_t *n_blocks,
-                 uint8_t *fp4, uint8_t *scale, uint8_t *idx_key, float *pooled_out,
+                 uint8_t *fp4, uint8_t *scale, uint8_t *idx_key, uint8_t *idx_key_scale, float *pooled_out,
                  float *pooled_idx_out) {
     int status = 0;
     for (int b = 0; b < B; ++b) {
@@ -223,21 +234,34 @@ int orc_compress(int B, int D, int dI, int m, int idx_dtype, int scale_fmt, int 
                 for (int i = 0; i < gs / 2; ++i)
                     fp4[row * (D / 2) + (gs / 2) * grp + i] = (uint8_t)(codes[2 * i] | (codes[2 * i + 1] << 4));
             }
-            /* pooled indexer key with the same gate, stored as bf16 or e4m3 */
+            /* pooled indexer key with the same gate, stored as bf16, e4m3, or MXFP4
+             * (one E8M0 scale per 32 channels, the main KV's rule) */
             if (idx_key) {
                 uint8_t *dst = idx_key + row * idx_key_bytes(idx_dtype, dI);
+                float *kfs = malloc(sizeof(float) * dI);
                 for (int c = 0; c < dI; ++c) {
                     double acc = 0.0;
                     for (int t = 0; t < m; ++t) acc += alpha[t] * orc_bf16_decode(idx_tok[(t0 + t) * dI + c]);
                     float kf = (float)acc;
+                    kfs[c] = kf;
                     if (pooled_idx_out) pooled_idx_out[row * dI + c] = kf;
                     if (idx_dtype == 0) {
                         uint16_t bits = orc_bf16_encode(kf);
                         memcpy(dst + 2 * c, &bits, 2);
-                    } else {
+                    } else if (idx_dtype == 1) {
                         dst[c] = orc_e4m3_encode((double)kf);
                     }
                 }
+                if (idx_dtype == 2) {
+                    for (int grp = 0; grp < dI / 32; ++grp) {
+                        uint8_t codes[32], sb;
+                        orc_mxfp4_quantize_group(kfs + 32 * grp, codes, &sb);
+                        idx_key_scale[row * (dI / 32) + grp] = sb;
+                        for (int i2 = 0; i2 < 16; ++i2)
+                            dst[16 * grp + i2] = (uint8_t)(codes[2 * i2] | (codes[2 * i2 + 1] << 4));
+                    }
+                }
+                free(kfs);
             }
             free(g);
             free(alpha);
@@ -264,16 +288,35 @@ static int visible_blocks(int pos, int m, int filled) {
     return (int)v;
 }
 
+/* The indexer query as the scores use it: the bf16 value itself, or, with MXFP4
+ * keys, its MXFP4 quantization per 32 channels of each head (the main KV's rule),
+ * dequantized. qv: [H_I][dI] doubles of query i. */
+static void index_query(int H_I, int dI, int idx_dtype, const uint16_t *q_row, double *qv) {
+    for (int h = 0; h < H_I; ++h) {
+        for (int c = 0; c < dI; ++c) qv[h * dI + c] = orc_bf16_decode(q_row[h * dI + c]);
+        if (idx_dtype != 2) continue;
+        for (int grp = 0; grp < dI / 32; ++grp) {
+            float v[32];
+            uint8_t codes[32], sb;
+            for (int c = 0; c < 32; ++c) v[c] = (float)qv[h * dI + 32 * grp + c];
+            orc_mxfp4_quantize_group(v, codes, &sb);
+            for (int c = 0; c < 32; ++c) qv[h * dI + 32 * grp + c] = ldexp(orc_e2m1_decode(codes[c]), (int)sb - 127);
+        }
+    }
+}
+
 void orc_index_scores(int B, int Nq, int H_I, int dI, int idx_dtype, int m, int cap,
-                      const uint8_t *idx_key, const int32_t *n_blocks,
+                      const uint8_t *idx_key, const uint8_t *idx_key_scale, const int32_t *n_blocks,
                       const int32_t *q_offsets, const int32_t *q_pos,
                       const uint16_t *q_idx, const float *w,
                       float *scores, int32_t *n_vis_out) {
     size_t kb = idx_key_bytes(idx_dtype, dI);
+    double *qv = malloc(sizeof(double) * (size_t)H_I * dI);
     for (int i = 0; i < Nq; ++i) {
         int b = request_of(q_offsets, B, i);
         int n_vis = (b < 0) ? 0 : visible_blocks(q_pos[i], m, n_blocks[b]);
         if (n_vis_out) n_vis_out[i] = n_vis;
+        index_query(H_I, dI, idx_dtype, q_idx + (size_t)i * H_I * dI, qv);
 #pragma omp parallel for schedule(static)
         for (int j = 0; j < cap; ++j) {
             if (j >= n_vis) {
@@ -281,11 +324,12 @@ void orc_index_scores(int B, int Nq, int H_I, int dI, int idx_dtype, int m, int 
                 continue;
             }
             const uint8_t *key = idx_key + ((size_t)b * cap + j) * kb;
+            const uint8_t *ksc = idx_dtype == 2 ? idx_key_scale + ((size_t)b * cap + j) * (dI / 32) : NULL;
             double s = 0.0;
             for (int h = 0; h < H_I; ++h) {
                 double dot = 0.0;
                 for (int c = 0; c < dI; ++c)
-                    dot += orc_bf16_decode(q_idx[((size_t)i * H_I + h) * dI + c]) * idx_key_element(key, idx_dtype, c);
+                    dot += qv[h * dI + c] * idx_key_element(key, ksc, idx_dtype, c);
                 s += (double)w[(size_t)i * H_I + h] * fmax(dot, 0.0);
             }
             float sf = (float)s;
@@ -293,6 +337,7 @@ void orc_index_scores(int B, int Nq, int H_I, int dI, int idx_dtype, int m, int 
             scores[(size_t)i * cap + j] = sf;
         }
     }
+    free(qv);
 }
 
 /* ======================================================================

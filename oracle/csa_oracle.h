@@ -61,7 +61,10 @@ void     orc_e4m3x16_quantize_group(const float *v, uint8_t *codes, uint8_t *sca
  * Output planes (per request stride = cap blocks):
  *   fp4   [B][cap][D/2]  two codes per byte, element 2i in the low nibble
  *   scale [B][cap][D/32] E8M0 bytes, or [B][cap][D/16] E4M3 bytes
- *   idx_key [B][cap][dI] bf16 (idx_dtype 0) or e4m3 (idx_dtype 1)
+ *   idx_key [B][cap][dI] bf16 (idx_dtype 0) or e4m3 (idx_dtype 1), or
+ *           [B][cap][dI/2] MXFP4 codes (idx_dtype 2: the pooled key quantized
+ *           like the main KV, one E8M0 scale per 32 channels, the scales in
+ *           idx_key_scale [B][cap][dI/32]; NULL otherwise)
  * Optional pooled_out [B][cap][D] float and pooled_idx_out [B][cap][dI] float
  * receive the float32 pooled values before quantization (NULL to skip).
  * Returns 0, or -1 when a request's token count is not a multiple of m or
@@ -69,7 +72,7 @@ void     orc_e4m3x16_quantize_group(const float *v, uint8_t *codes, uint8_t *sca
 int orc_compress(int B, int D, int dI, int m, int idx_dtype, int scale_fmt, int cap,
                  const uint16_t *kv_tok, const uint16_t *idx_tok, const float *w_g,
                  const int32_t *tok_offsets, int32_t *n_blocks,
-                 uint8_t *fp4, uint8_t *scale, uint8_t *idx_key, float *pooled_out,
+                 uint8_t *fp4, uint8_t *scale, uint8_t *idx_key, uint8_t *idx_key_scale, float *pooled_out,
                  float *pooled_idx_out);
 
 /* ---- a3: indexer scores ---------------------------------------------- */
@@ -78,9 +81,12 @@ int orc_compress(int B, int D, int dI, int m, int idx_dtype, int scale_fmt, int 
  * j < n_vis is the float32 rounding of
  *     sum_h w[i][h] * max(0, sum_c q_idx[i][h][c] * key_j[c]),
  * with -0 mapped to +0; entries j >= n_vis are set to -INFINITY.
+ * With MXFP4 keys (idx_dtype 2, scales in idx_key_scale) the query is first
+ * quantized the same way, per 32 channels of each head, and dequantized; the
+ * product of two MXFP4 values is then exact and the sums run in double.
  * scores has row stride cap. n_vis_out[i] receives n_vis (may be NULL). */
 void orc_index_scores(int B, int Nq, int H_I, int dI, int idx_dtype, int m, int cap,
-                      const uint8_t *idx_key, const int32_t *n_blocks,
+                      const uint8_t *idx_key, const uint8_t *idx_key_scale, const int32_t *n_blocks,
                       const int32_t *q_offsets, const int32_t *q_pos,
                       const uint16_t *q_idx, const float *w,
                       float *scores, int32_t *n_vis_out);

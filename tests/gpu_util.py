@@ -21,8 +21,9 @@ def host(t):
     return t.cpu().numpy()
 
 
-def make_cache(fp4, scale, n_blocks, block, idx_key=None, idx_dtype=0, scale_fmt=0):
-    """Device cache from numpy planes (idx_key as raw bytes [B, cap, key_bytes])."""
+def make_cache(fp4, scale, n_blocks, block, idx_key=None, idx_dtype=0, scale_fmt=0, idx_key_scale=None):
+    """Device cache from numpy planes (idx_key as raw bytes [B, cap, key_bytes]; MXFP4 keys:
+    codes [B, cap, dI/2] and idx_key_scale [B, cap, dI/32])."""
     import torch
 
     import fp4_kv_cache_csa_b200 as csa
@@ -34,4 +35,4 @@ def make_cache(fp4, scale, n_blocks, block, idx_key=None, idx_dtype=0, scale_fmt
             ik = ik.view(torch.bfloat16)
     return csa.Cache(fp4=dev(fp4), scale=dev(scale), n_blocks=dev(np.asarray(n_blocks, np.int32)), block=block,
                      idx_key=ik, idx_dtype=idx_dtype, status=torch.zeros(1, dtype=torch.int32, device="cuda"),
-                     scale_fmt=scale_fmt)
+                     scale_fmt=scale_fmt, idx_key_scale=None if idx_key_scale is None else dev(idx_key_scale))

@@ -32,7 +32,7 @@ def test_every_declared_symbol_is_exported(lib):
     assert set(names) == set(csa.EXPORTED), names
     for n in names:
         assert hasattr(lib, n), n
-    assert lib.csa_version() == 102
+    assert lib.csa_version() == 103
     assert lib.csa_status_string(0) == b"ok"
     assert lib.csa_status_string(99) == b"unknown status"
 
@@ -43,12 +43,26 @@ def fake_cache(**kw):
              idx_dim=128, idx_dtype=1, n_blocks=0x40000, status=0, scale_fmt=0)
     d.update(kw)
     c = csa._CCache(d["batch"], d["dim"], d["block"], d["capacity"], d["fp4"], d["scale"], d["idx_key"],
-                    d["idx_dim"], d["idx_dtype"], d["n_blocks"], d["status"] or None, d["scale_fmt"])
+                    d["idx_dim"], d["idx_dtype"], d["n_blocks"], d["status"] or None, d["scale_fmt"],
+                    d.get("idx_key_scale") or None)
     return c
 
 
 def compress(lib, c, kv=0x50000, idx=0x60000, gate=0x70000, offs=0x80000, n=16):
     return lib.csa_compress_quantize(ctypes.byref(c) if c is not None else None, kv, idx, gate, offs, n, None)
+
+
+def test_mxfp4_key_validation(lib):
+    # MXFP4 indexer keys need their scale plane (4-byte aligned); the indexer pairs each head with
+    # the key groups in its MMA columns, so at most 4 indexer heads are supported with them
+    assert compress(lib, fake_cache(idx_dtype=2)) == ERR_NULL
+    assert compress(lib, fake_cache(idx_dtype=2, idx_key_scale=0x90002)) == ERR_ALIGN
+    c = fake_cache(idx_dtype=2, idx_key_scale=0x90000)
+    assert compress(lib, fake_cache(idx_dtype=3, idx_key_scale=0x90000)) == ERR_SHAPE
+    args = (0x90000, 0xA0000, 2, 8, 0xB0000, 0xC0000, 64, 0xD0000, 0x100000, 1 << 40, None)
+    assert lib.csa_index_topk(ctypes.byref(c), *args) == ERR_UNSUPPORTED
+    args4 = (0x90000, 0xA0000, 2, 4, 0xB0000, 0xC0000, 64, 0xD0000, 0, 0, None)
+    assert lib.csa_index_topk(ctypes.byref(c), *args4) == ERR_WORKSPACE  # 4 heads pass the checks
 
 
 def test_compress_validation(lib):

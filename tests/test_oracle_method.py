@@ -273,6 +273,105 @@ def test_indexer_worked_example():
         assert list(oracle.topk(scores, n_vis, k)[0]) == want
 
 
+def _read_mxfp4_golden():
+    spec = {"sel": {}}
+    with open(os.path.join(GOLDEN, "indexer_mxfp4_tiny.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            tag, rest = line.split(" ", 1)
+            if tag == "sel":
+                k, idx = rest.split(":")
+                spec["sel"][int(k)] = [int(v) for v in idx.split()]
+            elif tag in ("qbits", "codes", "scales"):
+                base = 16 if tag != "scales" else 10
+                spec[tag] = [[[int(v, base) for v in grp.split()] for grp in item.split("|")]
+                             for item in rest.split(";")]
+            else:
+                spec[tag] = np.array([float(v) for v in rest.split()])
+    return spec
+
+
+def _mxfp4_golden_inputs(s):
+    """Query [1, 2, 64] bf16 bits, codes [1, 3, 32], scales [1, 3, 2] from the golden file
+    (listed channels c0, c1 of group 0 and c32, c33 of group 1; all others zero)."""
+    q = np.zeros((1, 2, 64), np.uint16)
+    for h, (g0, g1) in enumerate(s["qbits"]):
+        q[0, h, 0:2], q[0, h, 32:34] = g0, g1
+    codes = np.zeros((1, 3, 32), np.uint8)
+    for j, (g0, g1) in enumerate(s["codes"]):
+        codes[0, j, 0] = g0[0] | (g0[1] << 4)
+        codes[0, j, 16] = g1[0] | (g1[1] << 4)
+    scales = np.array([[sc[0] for sc in s["scales"]]], np.uint8).reshape(1, 3, 2)
+    return q, codes, scales
+
+
+def test_indexer_mxfp4_worked_example():
+    # MXFP4 keys and the query quantized the same way: hand-derived scores, exact
+    s = _read_mxfp4_golden()
+    q, codes, scales = _mxfp4_golden_inputs(s)
+    w = s["w"].astype(np.float32)[None]
+    args = (np.array([3], np.int32), np.array([0, 1], np.int32), np.array([11], np.int32))
+    scores, n_vis = oracle.index_scores(codes, *args, q, w, m=4, idx_dtype=oracle.IDX_MXFP4, idx_key_scale=scales)
+    assert n_vis[0] == 3
+    assert np.array_equal(scores[0], s["scores"].astype(np.float32))
+    for k, want in s["sel"].items():
+        assert list(oracle.topk(scores, n_vis, k)[0]) == want
+
+
+def _e2m1_value(code):
+    mag = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0][code & 7]
+    return -mag if code & 8 else mag
+
+
+def test_indexer_mxfp4_equals_bf16_on_representable_values():
+    # when the query is already MXFP4-representable (every 32-group holds E2M1 x 2^X with its
+    # largest magnitude in [4, 8) x 2^X) its quantization is the identity, and MXFP4 keys hold
+    # values that bf16 stores exactly: the MXFP4-mode scores must equal the bf16-mode scores of
+    # the same values
+    g = np.random.default_rng(50)
+    B, cap, dI, H_I, Nq = 2, 40, 128, 4, 3
+    codes = g.integers(0, 256, size=(B, cap, dI // 2)).astype(np.uint8)
+    scales = g.integers(120, 131, size=(B, cap, dI // 32)).astype(np.uint8)
+    lo, hi = codes & 0xF, codes >> 4
+    elem = np.stack([lo, hi], axis=-1).reshape(B, cap, dI)
+    vals = np.vectorize(_e2m1_value)(elem) * np.ldexp(1.0, np.repeat(scales.astype(int) - 127, 32, axis=-1))
+    keys_bf16 = bf16(vals.astype(np.float32)).view(np.uint8).reshape(B, cap, 2 * dI)
+    assert np.array_equal(bf16_val(bf16(vals.astype(np.float32))), vals)  # exact in bf16
+    mags = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6])
+    qv = g.choice(mags, size=(Nq, H_I, dI)) * g.choice([-1.0, 1.0], size=(Nq, H_I, dI))
+    qv = qv.reshape(Nq, H_I, dI // 32, 32)
+    qv[..., 0] = 4.0 * np.sign(qv[..., 0] + 0.5)
+    qv = (qv * np.ldexp(1.0, g.integers(-3, 3, size=(Nq, H_I, dI // 32)))[..., None]).reshape(Nq, H_I, dI)
+    w = g.standard_normal((Nq, H_I)).astype(np.float32)
+    args = (np.array([cap, 31], np.int32), np.array([0, 2, 3], np.int32), np.array([10 ** 5, 10 ** 5, 50], np.int32))
+    s_mx, n1 = oracle.index_scores(codes, *args, bf16(qv), w, m=4, idx_dtype=oracle.IDX_MXFP4, idx_key_scale=scales)
+    s_bf, n2 = oracle.index_scores(keys_bf16, *args, bf16(qv), w, m=4)
+    assert np.array_equal(n1, n2) and list(n1) == [cap, cap, 12]
+    assert np.array_equal(s_mx, s_bf)
+
+
+def test_pool_m1_mxfp4_key_store():
+    # m = 1: the stored MXFP4 key decodes to the token's value when the token is representable,
+    # and otherwise to its quantization by the main KV's rule (the same codes and scale bytes
+    # the main-KV plane gets for the same values)
+    g = np.random.default_rng(51)
+    T, dI = 16, 64
+    kv = g.standard_normal((T, 64)).astype(np.float32)
+    idx = g.standard_normal((T, dI)).astype(np.float32) * 3
+    r = _compress(kv, np.zeros(64), 1, idx, idx_dtype=oracle.IDX_MXFP4)
+    ref = _compress(idx, np.zeros(dI), 1)  # the same values through the main-KV plane
+    assert np.array_equal(r["idx_key"][0], ref["fp4"][0])
+    assert np.array_equal(r["idx_key_scale"][0], ref["scale"][0])
+    lossless = lossless_tokens(T, dI, 52)
+    r2 = _compress(kv, np.zeros(64), 1, lossless, idx_dtype=oracle.IDX_MXFP4)
+    codes = r2["idx_key"][0]
+    elem = np.stack([codes & 0xF, codes >> 4], axis=-1).reshape(T, dI)
+    dec = np.vectorize(_e2m1_value)(elem) * np.ldexp(1.0, np.repeat(r2["idx_key_scale"][0].astype(int) - 127, 32, axis=-1))
+    assert np.array_equal(dec, lossless.astype(np.float64))
+
+
 def test_indexer_e4m3_keys_and_homogeneity():
     g = np.random.default_rng(20)
     keys = datagen.to_e4m3_bytes(g.standard_normal((1, 50, 32)) * 0.5)
