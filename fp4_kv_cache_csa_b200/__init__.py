@@ -65,7 +65,12 @@ def load_library(path: str = LIB_PATH):
         return _lib
     if not os.path.exists(path):
         raise CsaError(f"libcsa.so not found at {path}: build it with `python -m fp4_kv_cache_csa_b200.build`")
-    lib = ctypes.CDLL(path)
+    _lib = declare(ctypes.CDLL(path))
+    return _lib
+
+
+def declare(lib):
+    """Declare the C signatures of a loaded libcsa (the library itself or a test variant of it)."""
     P, I, S = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
     CP = ctypes.POINTER(_CCache)
     lib.csa_status_string.argtypes = [I]
@@ -96,7 +101,6 @@ def load_library(path: str = LIB_PATH):
     lib.hca_decode_attend.restype = I
     lib.csa_read_device_status.argtypes = [CP, P, ctypes.POINTER(I)]
     lib.csa_read_device_status.restype = I
-    _lib = lib
     return lib
 
 

@@ -649,7 +649,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
     uint8_t *P = Q + C::Q_BYTES;
     uint8_t *misc = P + C::P_BYTES;
     // [0] S done, [1] PV of the low channel set done, [2] PV all done, [3] Q' loaded,
-    // [4] / [5] low / high channel set of E' written (256 arrivals each)
+    // [4] / [5] low / high channel set of E' written (256 arrivals each), [6] drain on abort
     uint64_t *mbar = reinterpret_cast<uint64_t *>(misc);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + 64);
     int *flags = reinterpret_cast<int *>(misc + 80);                // [0] rescale, [1] abort
@@ -669,6 +669,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
     const uint32_t mbar_s = smem_u32(&mbar[0]), mbar_lo = smem_u32(&mbar[1]), mbar_hi = smem_u32(&mbar[2]);
     const uint32_t mbar_q = smem_u32(&mbar[3]);
     const uint32_t mbar_elo = smem_u32(&mbar[4]), mbar_ehi = smem_u32(&mbar[5]);
+    const uint32_t mbar_drain = smem_u32(&mbar[6]);
     if (tid == 0) {
         mbar_init(mbar_s, 1);
         mbar_init(mbar_lo, 1);
@@ -676,6 +677,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
         mbar_init(mbar_q, 1);
         mbar_init(mbar_elo, kThreads);
         mbar_init(mbar_ehi, kThreads);
+        mbar_init(mbar_drain, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         flags[0] = 0;
         flags[1] = 0;
@@ -705,12 +707,19 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
     RowRegs<D> rr;
     TileRef cur = query_ref(a, a.cta_q[c], t_begin);
     // the first query's Q' image: one bulk copy (the schedule kernel wrote it)
+#ifndef CSA_TEST_UNSENT_Q_COPY
     if (tid == 0) {
         mbar_expect_tx(mbar_q, C::Q_BYTES);
         bulk_g2s(Q_s, a.qimg + (size_t)cur.i * C::Q_BYTES, C::Q_BYTES, mbar_q);
     }
-    uint32_t n_q = 0;           // Q' copies waited for
-    uint32_t n_q_issued = 1;    // ... and issued
+    uint32_t n_q_issued = 1;    // Q' copies issued ...
+#else
+    // a test build of the library announces the copy's bytes but never sends it, so the
+    // wait for it can only run out: the kernel's timeout path is what that test checks
+    if (tid == 0) mbar_expect_tx(mbar_q, C::Q_BYTES);
+    uint32_t n_q_issued = 0;
+#endif
+    uint32_t n_q = 0;           // ... and waited for
     prefetch_row<D, SF>(a, cur, row_block_raw(a, cur), rr);
     // the next tile and this thread's selected index in it (one tile ahead of its row loads)
     TileRef nxt = cur;
@@ -991,8 +1000,14 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(AttArgs a) {
     }
 
     if (aborted) {
+        // nothing this CTA started may still run when it leaves: its Q' copy, and every MMA
+        // thread 0 issued (one commit tracks them all), waited for with the long limit
         if (tid == 0) flag(a.status, CSA_DEV_TIMEOUT);
-        if (n_q_issued > n_q) mbar_wait(mbar_q, n_q & 1);  // no copy may land after the CTA exits
+        if (n_q_issued > n_q) mbar_wait_for(mbar_q, n_q & 1, kDrainCycles);
+        if (tid == 0) {
+            mma_commit(mbar_drain);
+            mbar_wait_for(mbar_drain, 0, kDrainCycles);
+        }
     }
     if (tid == 0) bulk_wait_all();  // output copies complete before the CTA's shared memory goes away
     tc_fence_before();

@@ -13,7 +13,16 @@ namespace csa {
 
 namespace {
 
-constexpr long long kWaitCycles = 2000000000LL;  // bounded mbarrier wait (~1 s)
+// Bounded mbarrier waits: a wait that runs out makes the kernel flag
+// CSA_DEV_TIMEOUT and leave. A test build of the library shortens the limit
+// (-DCSA_WAIT_CYCLES=...) so that the first wait of a call runs out; the waits
+// a kernel makes for its own copies and MMAs before it exits always use the
+// long limit, so that nothing it started is still running when it leaves.
+#ifndef CSA_WAIT_CYCLES
+#define CSA_WAIT_CYCLES 2000000000LL
+#endif
+constexpr long long kWaitCycles = CSA_WAIT_CYCLES;  // ~1 s at the shipped value
+constexpr long long kDrainCycles = 2000000000LL;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -59,6 +68,23 @@ __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.a
 
 __device__ __forceinline__ void mbar_init(uint32_t mbar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(mbar), "r"(count) : "memory");
+}
+
+// Wait for the phase with this parity to complete; gives up after `limit` cycles.
+__device__ __forceinline__ bool mbar_wait_for(uint32_t mbar, uint32_t parity, long long limit) {
+    const long long t0 = clock64();
+    while (true) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}\n"
+            : "=r"(done)
+            : "r"(mbar), "r"(parity)
+            : "memory");
+        if (done) return true;
+        if (clock64() - t0 > limit) return false;
+    }
 }
 
 // Wait for the phase with this parity to complete; gives up after kWaitCycles.
