@@ -37,6 +37,7 @@ sys.path.insert(0, ROOT)
 B, D, H, M_CSA, M_HCA, W = 32, 512, 64, 4, 128, 128
 H_I, D_I, TOPK = 4, 128, 1024
 POOL_GROUP, POOL_BLOCKS = 8, 2000  # hierarchical indexer pool: ~2000 blocks of 8 entries
+REINDEX_LAYERS = 3  # Reindex layers timed together in one call (after the Full layer that keeps the pool)
 CTX_MIN, CTX_MAX = 524288, 1048576
 CAP_CSA, CAP_HCA = CTX_MAX // M_CSA, CTX_MAX // M_HCA
 OUR_KERNELS_PER_STEP = 12  # compress 2x(pool, commit); index: scan (own schedule), merge; attend 2x(schedule, main, merge)
@@ -139,6 +140,12 @@ class Workload:
                                    dtype=torch.uint8, device=device)
         self.ws_re = torch.empty(csa.csa_index_reindex_workspace(self.csa, B, POOL_GROUP, POOL_BLOCKS),
                                  dtype=torch.uint8, device=device)
+        # three Reindex layers over the same pool in one call
+        self.q_idx_re3 = torch.randn(B, REINDEX_LAYERS, H_I, D_I, device=device, generator=gen).to(bf)
+        self.w_re3 = (torch.randn(B, REINDEX_LAYERS, H_I, device=device, generator=gen) / math.sqrt(H_I)).float()
+        self.sel_re3 = torch.empty(B, REINDEX_LAYERS, TOPK, dtype=torch.int32, device=device)
+        self.ws_re3 = torch.empty(csa.csa_index_reindex_layers_workspace(self.csa, B, REINDEX_LAYERS, POOL_GROUP,
+                                                                         POOL_BLOCKS), dtype=torch.uint8, device=device)
 
     def stage_index_pool(self):
         import fp4_kv_cache_csa_b200 as csa
@@ -151,6 +158,12 @@ class Workload:
 
         csa.csa_index_topk_reindex(self.csa, self.q_idx_re, self.w_re, self.q_offsets, self.q_pos, TOPK, self.pool,
                                    POOL_GROUP, sel_idx=self.sel_re, workspace=self.ws_re)
+
+    def stage_index_reindex_layers(self):
+        import fp4_kv_cache_csa_b200 as csa
+
+        csa.csa_index_topk_reindex_layers(self.csa, self.q_idx_re3, self.w_re3, self.q_offsets, self.q_pos, TOPK,
+                                          self.pool, POOL_GROUP, sel_idx=self.sel_re3, workspace=self.ws_re3)
 
     def bytes_reindex(self) -> float:
         """Keys of the pool's entries (about POOL_GROUP * POOL_BLOCKS per request), query, output."""
@@ -835,25 +848,28 @@ def main():
     # ---- CSA2 (not part of the step): a Full layer that also keeps the pool, and
     # a Reindex layer over that pool, each timed alone with a cold L2
     csa2_graphs = []
+    csa2_fns = (wl.stage_index_pool, wl.stage_index_reindex, wl.stage_index_reindex_layers)
     with torch.cuda.stream(stream):
-        for fn in (wl.stage_index_pool, wl.stage_index_reindex):
+        for fn in csa2_fns:
             fn()
         stream.synchronize()
-        for fn in (wl.stage_index_pool, wl.stage_index_reindex):
+        for fn in csa2_fns:
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
                 fn()
             csa2_graphs.append(g)
     n2 = max(4, min(args.steps, 50))
-    ev2 = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(2 * n2)]
+    nf = len(csa2_fns)
+    ev2 = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(nf * n2)]
     with torch.cuda.stream(stream):
-        for k in range(2 * n2):
+        for k in range(nf * n2):
             flush.zero_()
             ev2[k][0].record(stream)
-            csa2_graphs[k % 2].replay()
+            csa2_graphs[k % nf].replay()
             ev2[k][1].record(stream)
     stream.synchronize()
-    csa2_ms = [float(np.mean([ev2[k][0].elapsed_time(ev2[k][1]) for k in range(j, 2 * n2, 2)])) for j in range(2)]
+    csa2_ms = [float(np.mean([ev2[k][0].elapsed_time(ev2[k][1]) for k in range(j, nf * n2, nf)]))
+               for j in range(nf)]
     status |= csa.csa_read_device_status(wl.csa, stream)
     del csa2_graphs
     prefill = measure_prefill(device, stream, flush) if not args.no_prefill else None
@@ -970,6 +986,7 @@ def main():
         # CSA2 cross-layer modes (not in the step): Full layer + pool, then a Reindex layer over the pool
         "csa2": {"pool_group": POOL_GROUP, "pool_blocks": POOL_BLOCKS, "full_with_pool_ms": csa2_ms[0],
                  "reindex_ms": csa2_ms[1], "full_ms": idx_ms,
+                 "reindex_layers": REINDEX_LAYERS, "reindex_layers_one_call_ms": csa2_ms[2],
                  "reindex_algorithmic_bytes": wl.bytes_reindex(),
                  "reindex_achieved_gbs": wl.bytes_reindex() / (csa2_ms[1] * 1e-3) / 1e9},
         "prefill": None if prefill is None else dict(

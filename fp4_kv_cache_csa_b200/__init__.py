@@ -37,7 +37,7 @@ EXPORTED = (
     "csa_status_string", "csa_version", "csa_compress_quantize", "csa_index_topk_workspace", "csa_index_topk",
     "csa_attend_workspace", "csa_decode_attend", "hca_decode_attend", "csa_read_device_status",
     "csa_index_topk_noalloc", "csa_index_pool_workspace", "csa_index_topk_pool", "csa_index_reindex_workspace",
-    "csa_index_topk_reindex",
+    "csa_index_topk_reindex", "csa_index_reindex_layers_workspace", "csa_index_topk_reindex_layers",
 )
 
 
@@ -93,6 +93,10 @@ def declare(lib):
     lib.csa_index_reindex_workspace.restype = S
     lib.csa_index_topk_reindex.argtypes = [CP, P, P, I, I, P, P, I, P, I, I, P, P, S, P]
     lib.csa_index_topk_reindex.restype = I
+    lib.csa_index_reindex_layers_workspace.argtypes = [CP, I, I, I, I]
+    lib.csa_index_reindex_layers_workspace.restype = S
+    lib.csa_index_topk_reindex_layers.argtypes = [CP, P, P, I, I, I, P, P, I, P, I, I, P, P, S, P]
+    lib.csa_index_topk_reindex_layers.restype = I
     lib.csa_attend_workspace.argtypes = [CP, I, I]
     lib.csa_attend_workspace.restype = S
     lib.csa_decode_attend.argtypes = [CP, P, I, I, P, P, I, P, P, P, I, ctypes.c_float, P, P, P, S, P]
@@ -288,6 +292,33 @@ def csa_index_topk_reindex(cache: Cache, q_idx, w, q_offsets, q_pos, topk: int, 
     _check(lib.csa_index_topk_reindex(ctypes.byref(c), _ptr(q_idx), _ptr(w), n_queries, idx_heads, _ptr(q_offsets),
                                       _ptr(q_pos), topk, _ptr(sel_idx), pool_group, pool_blocks, _ptr(pool_blk),
                                       _ptr(workspace), workspace.numel(), _stream(stream)), "csa_index_topk_reindex")
+    return sel_idx
+
+
+def csa_index_reindex_layers_workspace(cache: Cache, n_queries: int, n_layers: int, pool_group: int,
+                                       pool_blocks: int) -> int:
+    return int(load_library().csa_index_reindex_layers_workspace(ctypes.byref(cache.c_struct()), n_queries, n_layers,
+                                                                 pool_group, pool_blocks))
+
+
+def csa_index_topk_reindex_layers(cache: Cache, q_idx, w, q_offsets, q_pos, topk: int, pool_blk, pool_group: int = 8,
+                                  sel_idx=None, workspace=None, stream=None):
+    """Several Reindex-mode layers over one pool in one call. q_idx [Nq, L, H_I, dI] bf16,
+    w [Nq, L, H_I] float32; returns sel_idx [Nq, L, topk]."""
+    import torch
+
+    lib = load_library()
+    n_queries, n_layers, idx_heads = (int(x) for x in q_idx.shape[:3])
+    pool_blocks = int(pool_blk.shape[1])
+    if sel_idx is None:
+        sel_idx = torch.empty(n_queries, n_layers, topk, dtype=torch.int32, device=q_idx.device)
+    need = csa_index_reindex_layers_workspace(cache, n_queries, n_layers, pool_group, pool_blocks)
+    workspace = _workspace(need, workspace, q_idx.device)
+    c = cache.c_struct()
+    _check(lib.csa_index_topk_reindex_layers(ctypes.byref(c), _ptr(q_idx), _ptr(w), n_queries, n_layers, idx_heads,
+                                             _ptr(q_offsets), _ptr(q_pos), topk, _ptr(sel_idx), pool_group,
+                                             pool_blocks, _ptr(pool_blk), _ptr(workspace), workspace.numel(),
+                                             _stream(stream)), "csa_index_topk_reindex_layers")
     return sel_idx
 
 

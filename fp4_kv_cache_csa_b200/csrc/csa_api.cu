@@ -22,7 +22,7 @@ size_t index_reindex_workspace_bytes(int Nq, int G, int P);
 cudaError_t launch_index_topk_reindex(const csa_cache &c, const void *q_idx, const float *w, int Nq, int H_I,
                                       const int32_t *q_offsets, const int32_t *q_pos, int topk, int32_t *sel_idx,
                                       int pool_shift, int P, const int32_t *pool_blk, void *workspace, int num_sms,
-                                      cudaStream_t s);
+                                      cudaStream_t s, int layers);
 size_t attend_workspace_bytes(int Nq, int D, int num_ctas);
 cudaError_t launch_attend(const csa_cache &c, const void *q, int Nq, int H, const int32_t *q_offsets,
                           const int32_t *q_pos, const int32_t *sel_idx, int topk, const void *win_kv,
@@ -34,6 +34,7 @@ namespace {
 
 constexpr int kMaxCapacity = 1 << 19;  // the top-k select keeps two bitmaps of this many bits in shared memory
 constexpr int kMaxTopk = 4096;
+constexpr int kMaxReindexLayers = 16;  // Reindex layers in one csa_index_topk_reindex_layers call
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -182,10 +183,40 @@ csa_status csa_index_topk_pool(const csa_cache *cache, const void *q_idx, const 
                                                  sms, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+size_t csa_index_reindex_layers_workspace(const csa_cache *cache, int32_t n_queries, int32_t n_layers,
+                                          int32_t pool_group, int32_t pool_blocks) {
+    if (!cache || n_queries < 1 || n_layers < 1 || n_layers > kMaxReindexLayers ||
+        !pool_sizes_ok(pool_group, pool_blocks) || (long long)n_queries * n_layers > (1 << 30))
+        return 0;
+    return csa::index_reindex_workspace_bytes(n_queries * n_layers, pool_group, pool_blocks);
+}
+
 size_t csa_index_reindex_workspace(const csa_cache *cache, int32_t n_queries, int32_t pool_group,
                                    int32_t pool_blocks) {
-    if (!cache || n_queries < 1 || !pool_sizes_ok(pool_group, pool_blocks)) return 0;
-    return csa::index_reindex_workspace_bytes(n_queries, pool_group, pool_blocks);
+    return csa_index_reindex_layers_workspace(cache, n_queries, 1, pool_group, pool_blocks);
+}
+
+csa_status csa_index_topk_reindex_layers(const csa_cache *cache, const void *q_idx, const float *w,
+                                         int32_t n_queries, int32_t n_layers, int32_t idx_heads,
+                                         const int32_t *q_offsets, const int32_t *q_pos, int32_t topk,
+                                         int32_t *sel_idx, int32_t pool_group, int32_t pool_blocks,
+                                         const int32_t *pool_blk, void *workspace, size_t workspace_bytes,
+                                         csa_stream_t stream) {
+    csa_status st = csa::check_index_args(cache, q_idx, w, n_queries, idx_heads, q_offsets, q_pos, topk, sel_idx);
+    if (st != CSA_OK) return st;
+    if (!pool_blk) return CSA_ERR_NULL;
+    if (n_layers < 1 || pool_shift_of(pool_group) < 0 || pool_blocks < 1) return CSA_ERR_SHAPE;
+    if (n_layers > kMaxReindexLayers || !pool_sizes_ok(pool_group, pool_blocks)) return CSA_ERR_UNSUPPORTED;
+    if (!aligned(pool_blk, 4)) return CSA_ERR_ALIGN;
+    const size_t need = csa_index_reindex_layers_workspace(cache, n_queries, n_layers, pool_group, pool_blocks);
+    if (!workspace || workspace_bytes < need) return CSA_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return CSA_ERR_ALIGN;
+    const int sms = num_sms();
+    if (sms <= 0) return CSA_ERR_CUDA;
+    return from_cuda(csa::launch_index_topk_reindex(*cache, q_idx, w, n_queries, idx_heads, q_offsets, q_pos, topk,
+                                                    sel_idx, pool_shift_of(pool_group), pool_blocks, pool_blk,
+                                                    workspace, sms, reinterpret_cast<cudaStream_t>(stream),
+                                                    n_layers));
 }
 
 csa_status csa_index_topk_reindex(const csa_cache *cache, const void *q_idx, const float *w, int32_t n_queries,
@@ -193,20 +224,8 @@ csa_status csa_index_topk_reindex(const csa_cache *cache, const void *q_idx, con
                                   int32_t *sel_idx, int32_t pool_group, int32_t pool_blocks,
                                   const int32_t *pool_blk, void *workspace, size_t workspace_bytes,
                                   csa_stream_t stream) {
-    csa_status st = csa::check_index_args(cache, q_idx, w, n_queries, idx_heads, q_offsets, q_pos, topk, sel_idx);
-    if (st != CSA_OK) return st;
-    if (!pool_blk) return CSA_ERR_NULL;
-    if (pool_shift_of(pool_group) < 0 || pool_blocks < 1) return CSA_ERR_SHAPE;
-    if (!pool_sizes_ok(pool_group, pool_blocks)) return CSA_ERR_UNSUPPORTED;
-    if (!aligned(pool_blk, 4)) return CSA_ERR_ALIGN;
-    const size_t need = csa_index_reindex_workspace(cache, n_queries, pool_group, pool_blocks);
-    if (!workspace || workspace_bytes < need) return CSA_ERR_WORKSPACE;
-    if (!aligned(workspace, 256)) return CSA_ERR_ALIGN;
-    const int sms = num_sms();
-    if (sms <= 0) return CSA_ERR_CUDA;
-    return from_cuda(csa::launch_index_topk_reindex(*cache, q_idx, w, n_queries, idx_heads, q_offsets, q_pos, topk,
-                                                    sel_idx, pool_shift_of(pool_group), pool_blocks, pool_blk,
-                                                    workspace, sms, reinterpret_cast<cudaStream_t>(stream)));
+    return csa_index_topk_reindex_layers(cache, q_idx, w, n_queries, 1, idx_heads, q_offsets, q_pos, topk, sel_idx,
+                                         pool_group, pool_blocks, pool_blk, workspace, workspace_bytes, stream);
 }
 
 size_t csa_attend_workspace(const csa_cache *cache, int32_t n_queries, int32_t heads) {

@@ -158,9 +158,11 @@ size_t carve(void *base, int Nq, int cap, IndexWs *w) {
 // ---------------------------------------------------------------- schedule
 // n_vis_given (Reindex): per-query key counts computed before (pool positions);
 // otherwise the visible block count from the query position.
+// layers > 1 (several Reindex layers in one call): query i is layer i % layers of the
+// caller's query i / layers, whose request and position it takes.
 __global__ void schedule_kernel(const int32_t *q_offsets, const int32_t *q_pos, const int32_t *n_blocks,
                                 int batch, int Nq, int m, int cap, int topk, int32_t *req, int32_t *n_vis,
-                                long long *gprefix, int32_t *thresh, const int32_t *n_vis_given) {
+                                long long *gprefix, int32_t *thresh, const int32_t *n_vis_given, int layers) {
     __shared__ long long red[32];
     __shared__ long long round_total;
     grid_dep_wait();
@@ -170,9 +172,9 @@ __global__ void schedule_kernel(const int32_t *q_offsets, const int32_t *q_pos, 
         const int i = base + threadIdx.x;
         long long groups = 0;
         if (i < Nq) {
-            const int b = request_of(q_offsets, batch, i);
+            const int b = request_of(q_offsets, batch, i / layers);
             const int n = n_vis_given ? ((b < 0) ? 0 : n_vis_given[i])
-                                      : ((b < 0) ? 0 : min(visible_blocks(q_pos[i], m, n_blocks[b]), cap));
+                                      : ((b < 0) ? 0 : min(visible_blocks(q_pos[i / layers], m, n_blocks[b]), cap));
             req[i] = b;
             n_vis[i] = n;
             groups = (n + 15) / 16;
@@ -339,6 +341,7 @@ struct ScanArgs {
     // computes the per-query counts and the unit prefix itself, and CTA 0 stores
     // them for the merge; otherwise schedule_kernel has written req, n_vis, gprefix
     int fused;
+    int layers;  // queries per caller query (several Reindex layers in one call), else 1
     const int32_t *q_offsets, *q_pos, *n_blocks, *n_vis_given;
     int32_t *req_out, *n_vis_out;
     long long *gprefix_out;
@@ -416,9 +419,10 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a) {
         const int i = threadIdx.x;
         long long units = 0;
         if (i < a.Nq) {
-            const int b = request_of(a.q_offsets, a.batch, i);
+            const int b = request_of(a.q_offsets, a.batch, i / a.layers);
             const int n = a.n_vis_given ? (b < 0 ? 0 : a.n_vis_given[i])
-                                        : (b < 0 ? 0 : min(visible_blocks(a.q_pos[i], a.m, a.n_blocks[b]), a.rows));
+                                        : (b < 0 ? 0 : min(visible_blocks(a.q_pos[i / a.layers], a.m, a.n_blocks[b]),
+                                                           a.rows));
             s_req[i] = b;
             s_nv[i] = n;
             units = (n + 15) / 16;
@@ -580,7 +584,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a) {
 
         const uint8_t *kbase = a.keys + (size_t)b * a.cap * C::KEY_BYTES;
         float *srow = a.scores + (size_t)i * a.rows;
-        const int32_t *prow = POOL ? a.pool + (size_t)i * a.pool_p : nullptr;
+        const int32_t *prow = POOL ? a.pool + (size_t)(i / a.layers) * a.pool_p : nullptr;
 
         const uint8_t *kscale = MX ? a.key_scales + (size_t)b * a.cap * C::GROUPS : nullptr;
         for (long long u0 = warp; u0 < nloc; u0 += (long long)kScanWarps * C::U) {
@@ -805,6 +809,7 @@ struct MergeArgs {
     // G * pool[i][r / G] + r % G with G = 1 << pool_shift; null: r itself
     const int32_t *pool;
     int pool_shift, pool_p;
+    int layers;  // query i maps to pool row i / layers
 };
 
 // Largest bin d of a histogram of nbins (a multiple of 32, at most 4096) bins
@@ -848,7 +853,8 @@ __device__ BinPick pick_bin_warp(const uint32_t *h, int nbins, uint32_t need, Bi
 // Only called with a.pool set: the caller branches on it first (a load through
 // the pool pointer must never be issued, even speculatively, when it is null).
 __device__ __forceinline__ int32_t merge_pool_index(const MergeArgs &a, int i, int r) {
-    return (a.pool[(size_t)i * a.pool_p + (r >> a.pool_shift)] << a.pool_shift) + (r & ((1 << a.pool_shift) - 1));
+    return (a.pool[(size_t)(i / a.layers) * a.pool_p + (r >> a.pool_shift)] << a.pool_shift) +
+           (r & ((1 << a.pool_shift) - 1));
 }
 
 // Position in the query's candidate row of candidate p (p < the candidates'
@@ -1740,12 +1746,13 @@ __global__ void __launch_bounds__(kBmaxThreads) pool_bmax_kernel(const float *sc
 __global__ void __launch_bounds__(kCountThreads) reindex_count_kernel(const int32_t *q_offsets, const int32_t *q_pos,
                                                                       const int32_t *n_blocks, int batch, int m,
                                                                       int cap, const int32_t *pool, int P, int shift,
-                                                                      int32_t *n_pos, int32_t *status) {
+                                                                      int32_t *n_pos, int32_t *status, int layers) {
     __shared__ int first_bad, first_pad;
     __shared__ uint32_t total;
     grid_dep_wait();
     grid_dep_launch();
-    const int i = blockIdx.x;
+    const int qi = blockIdx.x;      // one per layer of each caller query,
+    const int i = qi / layers;      // all reading that query's pool
     const int b = request_of(q_offsets, batch, i);
     const int nv = (b < 0) ? 0 : min(visible_blocks(q_pos[i], m, n_blocks[b]), cap);
     const int32_t *row = pool + (size_t)i * P;
@@ -1771,8 +1778,8 @@ __global__ void __launch_bounds__(kCountThreads) reindex_count_kernel(const int3
     if ((threadIdx.x & 31) == 0) atomicAdd(&total, mine);
     __syncthreads();
     if (threadIdx.x == 0) {
-        n_pos[i] = b < 0 ? 0 : (int)total;
-        if (first_bad < first_pad) flag(status, CSA_DEV_BAD_INDEX);
+        n_pos[qi] = b < 0 ? 0 : (int)total;
+        if (first_bad < first_pad && qi % layers == 0) flag(status, CSA_DEV_BAD_INDEX);
     }
 }
 
@@ -1869,7 +1876,7 @@ namespace {
 cudaError_t index_pipeline(const csa_cache &c, const void *q_idx, const float *w, int Nq, int H_I,
                            const int32_t *q_offsets, const int32_t *q_pos, int topk, int32_t *sel_idx, IndexWs &ws,
                            int rows, const int32_t *n_vis_given, const int32_t *pool, int pool_shift, int pool_p,
-                           int num_sms, cudaStream_t s) {
+                           int num_sms, cudaStream_t s, int layers = 1) {
     // many queries per request (prefill): scores as a tensor-core GEMM, and when the
     // rows fit in shared memory one selection kernel that needs no zeroed state
     const bool gemm = !pool && !n_vis_given && Nq >= kPrefillQueriesPerRequest * c.batch &&
@@ -1883,7 +1890,7 @@ cudaError_t index_pipeline(const csa_cache &c, const void *q_idx, const float *w
     const bool fused = !gemm && Nq <= kFusedScheduleQueries;
     if (!fused) {
         err = launch_pdl(schedule_kernel, dim3(1), dim3(1024), 0, s, q_offsets, q_pos, c.n_blocks, c.batch, Nq,
-                         c.block, rows, topk, ws.req, ws.n_vis, ws.gprefix, ws.thresh, n_vis_given);
+                         c.block, rows, topk, ws.req, ws.n_vis, ws.gprefix, ws.thresh, n_vis_given, layers);
         if (err != cudaSuccess) return err;
     }
 
@@ -1917,6 +1924,7 @@ cudaError_t index_pipeline(const csa_cache &c, const void *q_idx, const float *w
     sa.gprefix_out = ws.gprefix;
     sa.batch = c.batch;
     sa.m = c.block;
+    sa.layers = layers;
     const int grid = min(num_sms, kMaxScanCtas);
     if (gemm) {
         err = launch_prefill_scores(c.idx_key, c.batch, c.capacity, c.idx_dim, q_idx, w, Nq, H_I, ws.req, ws.n_vis, ws.scores,
@@ -1955,6 +1963,7 @@ cudaError_t index_pipeline(const csa_cache &c, const void *q_idx, const float *w
     ma.pool = pool;
     ma.pool_shift = pool_shift;
     ma.pool_p = pool_p;
+    ma.layers = layers;
     const int msmem = 8 * kMergeStage;
     err = cudaFuncSetAttribute(select_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem);
     if (err != cudaSuccess) return err;
@@ -2005,21 +2014,27 @@ cudaError_t launch_index_topk_pool(const csa_cache &c, const void *q_idx, const 
 
 size_t index_reindex_workspace_bytes(int Nq, int G, int P) { return carve(nullptr, Nq, G * P, nullptr); }
 
+// layers Reindex layers of the same caller queries in one call: query i of the
+// call is layer i % layers of caller query i / layers (its indexer query and
+// weights are laid out that way), and every layer of a caller query reads that
+// query's pool. The layers of a query are adjacent in the flat work list, so the
+// pool's keys they share are read from HBM about once and then from L2.
 cudaError_t launch_index_topk_reindex(const csa_cache &c, const void *q_idx, const float *w, int Nq, int H_I,
                                       const int32_t *q_offsets, const int32_t *q_pos, int topk, int32_t *sel_idx,
                                       int pool_shift, int P, const int32_t *pool_blk, void *workspace, int num_sms,
-                                      cudaStream_t s) {
+                                      cudaStream_t s, int layers) {
     const int rows = P << pool_shift;
+    const int NqL = Nq * layers;
     IndexWs ws;
-    carve(workspace, Nq, rows, &ws);
+    carve(workspace, NqL, rows, &ws);
     // visible pool positions per query, counted into ws.n_vis (the schedule keeps them)
     int32_t *n_pos = ws.n_vis;
-    cudaError_t err = launch_pdl(reindex_count_kernel, dim3(Nq), dim3(kCountThreads), 0, s, q_offsets, q_pos,
+    cudaError_t err = launch_pdl(reindex_count_kernel, dim3(NqL), dim3(kCountThreads), 0, s, q_offsets, q_pos,
                                  c.n_blocks, c.batch, c.block, c.capacity, (const int32_t *)pool_blk, P, pool_shift,
-                                 n_pos, c.status);
+                                 n_pos, c.status, layers);
     if (err != cudaSuccess) return err;
-    return index_pipeline(c, q_idx, w, Nq, H_I, q_offsets, q_pos, topk, sel_idx, ws, rows, n_pos, pool_blk,
-                          pool_shift, P, num_sms, s);
+    return index_pipeline(c, q_idx, w, NqL, H_I, q_offsets, q_pos, topk, sel_idx, ws, rows, n_pos, pool_blk,
+                          pool_shift, P, num_sms, s, layers);
 }
 
 }  // namespace csa

@@ -267,6 +267,30 @@ csa_status csa_index_topk_reindex(const csa_cache *cache, const void *q_idx, con
                                   const int32_t *pool_blk, void *workspace, size_t workspace_bytes,
                                   csa_stream_t stream);
 
+/*
+ * csa_index_topk_reindex_layers: n_layers Reindex-mode layers over the same pool
+ * in one call (cue 12: every Reindex layer runs its own indexer query against
+ * the shared keys of the earlier Full layer). For caller query i and layer l the
+ * result is exactly csa_index_topk_reindex's for that layer's query and weights;
+ * the layers of a query share its pool, its counts and its key reads (adjacent
+ * in one pass, so the pool's keys come from HBM about once), and the call
+ * launches the kernels of one Reindex call, not n_layers of them.
+ *   q_idx    bf16 [n_queries][n_layers][idx_heads][idx_dim]
+ *   w        float32 [n_queries][n_layers][idx_heads]
+ *   sel_idx  int32 [n_queries][n_layers][topk] device, written
+ *   n_layers 1 .. 16 (1 is csa_index_topk_reindex)
+ *   workspace >= csa_index_reindex_layers_workspace(...) bytes, 256-byte aligned
+ * q_offsets, q_pos and pool_blk are per caller query, as for csa_index_topk_reindex.
+ */
+size_t csa_index_reindex_layers_workspace(const csa_cache *cache, int32_t n_queries, int32_t n_layers,
+                                          int32_t pool_group, int32_t pool_blocks);
+csa_status csa_index_topk_reindex_layers(const csa_cache *cache, const void *q_idx, const float *w,
+                                         int32_t n_queries, int32_t n_layers, int32_t idx_heads,
+                                         const int32_t *q_offsets, const int32_t *q_pos, int32_t topk,
+                                         int32_t *sel_idx, int32_t pool_group, int32_t pool_blocks,
+                                         const int32_t *pool_blk, void *workspace, size_t workspace_bytes,
+                                         csa_stream_t stream);
+
 /* Bytes of workspace csa_decode_attend / hca_decode_attend need (0 on bad sizes). */
 size_t csa_attend_workspace(const csa_cache *cache, int32_t n_queries, int32_t heads);
 

@@ -116,3 +116,41 @@ def test_bad_pool_entries_are_flagged_and_end_the_list():
     assert csa.csa_read_device_status(cache) & csa.CSA_DEV_BAD_INDEX
     ref = oracle.reindex_topk(s, n_vis, np.array([[3, 10, -1, -1, -1]], np.int32), G=8, k=8)
     check_reindex(sel, ref, s, n_vis, np.array([[3, 10, -1, -1, -1]]), 8, 8)
+
+
+@pytest.mark.parametrize("idx_dtype,dI,L", [(1, 128, 3), (0, 64, 2), (2, 128, 4)])
+def test_reindex_layers_in_one_call(idx_dtype, dI, L):
+    # L Reindex layers over one Full layer's pool in one call: each layer's selection is
+    # the oracle's Reindex selection for that layer's own query and weights
+    import fp4_kv_cache_csa_b200 as csa
+
+    lengths = [16384, 9000, 700, 12001]
+    B, cap, H_I, k, G, P = 4, 16384, 4, 512, 8, 300
+    qo, qp = decode_layout(lengths)
+    if idx_dtype == 2:
+        from test_gpu_mxfp4_index import mx_keys
+        keys, ksc = mx_keys(B, cap, dI, 90)
+        kw = dict(m=4, idx_dtype=2, idx_key_scale=ksc)
+        cache = make_cache(np.zeros((B, cap, 64), np.uint8), np.zeros((B, cap, 4), np.uint8), lengths, 4, keys, 2,
+                           idx_key_scale=ksc)
+    else:
+        keys = gen_keys(B, cap, dI, idx_dtype, 90)
+        kw = dict(m=4, idx_dtype=idx_dtype)
+        cache = make_cache(np.zeros((B, cap, 64), np.uint8), np.zeros((B, cap, 4), np.uint8), lengths, 4,
+                           keys if idx_dtype == 1 else keys.view(np.uint16), idx_dtype)
+    q_full = datagen.normal_bf16((B, H_I, dI), 91, 30)
+    w_full = datagen.normal_f32((B, H_I), 91, 31, std=0.5)
+    _, pool = csa.csa_index_topk_pool(cache, dev(q_full), dev(w_full), dev(qo), dev(qp), k, pool_group=G,
+                                      pool_blocks=P)
+    pool = host(pool)
+    q_re = datagen.normal_bf16((B, L, H_I, dI), 91, 32)
+    w_re = datagen.normal_f32((B, L, H_I), 91, 33, std=0.5)
+    sel = host(csa.csa_index_topk_reindex_layers(cache, dev(q_re), dev(w_re), dev(qo), dev(qp), k, dev(pool),
+                                                 pool_group=G))
+    assert csa.csa_read_device_status(cache) == 0
+    assert sel.shape == (B, L, k)
+    for l in range(L):
+        s_re, n_vis = oracle.index_scores(keys, lengths, qo, qp, np.ascontiguousarray(q_re[:, l]),
+                                          np.ascontiguousarray(w_re[:, l]), **kw)
+        ref = oracle.reindex_topk(s_re, n_vis, pool, G=G, k=k)
+        check_reindex(sel[:, l], ref, s_re, n_vis, pool, G, k)
