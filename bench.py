@@ -397,7 +397,7 @@ class Prefill:
 
     B, T0, NEW, TOPK = 4, 65536, 8192, 512
 
-    def __init__(self, device):
+    def __init__(self, device, idx_dtype=0):
         import torch
 
         import fp4_kv_cache_csa_b200 as csa
@@ -407,11 +407,15 @@ class Prefill:
         gen = torch.Generator(device=device)
         gen.manual_seed(SEED + 4)
         bf = torch.bfloat16
-        self.cache = csa.Cache.allocate(B, self.cap, D, M_CSA, D_I, csa.CSA_IDX_BF16, device, scale_fmt=SCALE_FMT)
+        self.cache = csa.Cache.allocate(B, self.cap, D, M_CSA, D_I, idx_dtype, device, scale_fmt=SCALE_FMT)
         s_lo, s_hi = (123, 127) if SCALE_FMT == 0 else (0x1C, 0x2D)
         self.cache.fp4[:, :self.n0].random_(0, 256, generator=gen)
         self.cache.scale[:, :self.n0].random_(s_lo, s_hi, generator=gen)
-        self.cache.idx_key[:, :self.n0] = (torch.randn(B, self.n0, D_I, device=device, generator=gen) * 0.5).to(bf)
+        if idx_dtype == csa.CSA_IDX_MXFP4:  # E2M1 codes and E8M0 scales as the pooling writes them
+            self.cache.idx_key[:, :self.n0].random_(0, 256, generator=gen)
+            self.cache.idx_key_scale[:, :self.n0].random_(122, 127, generator=gen)
+        else:
+            self.cache.idx_key[:, :self.n0] = (torch.randn(B, self.n0, D_I, device=device, generator=gen) * 0.5).to(bf)
         self.base = torch.full((B,), self.n0, dtype=torch.int32, device=device)
         Nq = B * NEW
         self.Nq = Nq
@@ -491,6 +495,41 @@ def measure_prefill(device, stream, flush, steps: int = 3):
            "stage_ms": {"compress": float(st[0]), "index_topk": float(st[1]), "attend": float(st[2])},
            "index_gflop": pf.index_flops() / 1e9,
            "index_tflops": pf.index_flops() / (st[1] * 1e-3) / 1e12, "device_status": int(status)}
+    del pf
+    torch.cuda.empty_cache()
+    return res
+
+
+def measure_prefill_index_mxfp4(device, stream, flush, steps: int = 3):
+    """The prefill_b4_8k indexer stage with MXFP4 indexer keys: the block-scaled tensor-core
+    GEMM (kind::mxf4) writes the score rows, then the same selection as with bf16 keys."""
+    import torch
+
+    import fp4_kv_cache_csa_b200 as csa
+
+    pf = Prefill(device, idx_dtype=csa.CSA_IDX_MXFP4)
+    with torch.cuda.stream(stream):
+        pf.stage_compress()
+        pf.stage_index()
+    stream.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    with torch.cuda.stream(stream):
+        for k in range(steps):
+            flush.zero_()
+            ev[k][0].record(stream)
+            pf.stage_index()
+            ev[k][1].record(stream)
+    stream.synchronize()
+    ms = float(np.mean([e[0].elapsed_time(e[1]) for e in ev]))
+    status = csa.csa_read_device_status(pf.cache, stream)
+    bf16_peak, kind = measured_bf16_tflops()
+    fp4_peak = 4.0 * bf16_peak  # dense MXFP4 : bf16 = 9 : 2.25 PFLOP/s nominal
+    flops = pf.index_flops()
+    res = {"workload": "prefill_b4_8k", "idx_dtype": "mxfp4", "queries": pf.Nq, "index_ms": ms,
+           "index_gflop": flops / 1e9, "index_tflops": flops / (ms * 1e-3) / 1e12,
+           "mxfp4_peak_tflops": fp4_peak, "peak_kind": f"{kind} bf16 x 4 (nominal MXFP4 : bf16 ratio)",
+           "frac_of_mxfp4_peak": flops / (ms * 1e-3) / 1e12 / fp4_peak,
+           "score_bytes": 4.0 * pf.index_flops() / (H_I * D_I * 2), "device_status": int(status)}
     del pf
     torch.cuda.empty_cache()
     return res
@@ -873,6 +912,7 @@ def main():
     status |= csa.csa_read_device_status(wl.csa, stream)
     del csa2_graphs
     prefill = measure_prefill(device, stream, flush) if not args.no_prefill else None
+    prefill_mx = measure_prefill_index_mxfp4(device, stream, flush) if not args.no_prefill else None
     configs = measure_configs(device, stream, flush) if not args.no_configs else None
     index_mxfp4 = measure_index_mxfp4(device, stream, flush, wl) if not args.no_configs else None
 
@@ -992,6 +1032,8 @@ def main():
         "prefill": None if prefill is None else dict(
             prefill, index_tensor_frac=prefill["index_tflops"] / measured_bf16_tflops()[0],
             index_tensor_peak={"tflops": measured_bf16_tflops()[0], "kind": measured_bf16_tflops()[1] + " bf16 dense"}),
+        # the prefill indexer stage with MXFP4 indexer keys (block-scaled tensor-core GEMM)
+        "prefill_index_mxfp4": prefill_mx,
         "configs": configs,
         # the same indexer call with MXFP4 indexer keys (not the headline config's e4m3 keys)
         "index_mxfp4_keys": index_mxfp4,

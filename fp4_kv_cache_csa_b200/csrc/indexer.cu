@@ -54,9 +54,10 @@ namespace csa {
 
 // prefill.cu: the scores of many queries per request as a tensor-core GEMM.
 bool prefill_scores_supported(int idx_dtype, int idx_dim, int H_I);
-cudaError_t launch_prefill_scores(const void *keys, int batch, int cap, int idx_dim, const void *q_idx, const float *w, int Nq,
-                                  int H_I, const int32_t *req, const int32_t *n_vis, float *scores, int rows,
-                                  int32_t *status, int num_sms, cudaStream_t s);
+size_t prefill_query_scratch_bytes(int idx_dtype, int idx_dim, int Nq, int H_I);
+cudaError_t launch_prefill_scores(const csa_cache &c, const void *q_idx, const float *w, int Nq, int H_I,
+                                  const int32_t *req, const int32_t *n_vis, float *scores, int rows, void *q_scratch,
+                                  int num_sms, cudaStream_t s);
 
 namespace {
 
@@ -101,6 +102,8 @@ struct IndexWs {
     int32_t *seg_cnt;    // [Nq + kMaxScanCtas]: slot i + c for query i and scan CTA c
     uint32_t *seg_key;   // [Nq][cap]
     int32_t *seg_idx;    // [Nq][cap]
+    void *spare;         // seg_key .. end of seg_idx, free on the GEMM path
+    size_t spare_bytes;
     size_t zero_bytes;
     int words, ccap;
 };
@@ -148,6 +151,10 @@ size_t carve(void *base, int Nq, int cap, IndexWs *w) {
         w->seg_cnt = reinterpret_cast<int32_t *>(b + o_scnt);
         w->seg_key = reinterpret_cast<uint32_t *>(b + o_skey);
         w->seg_idx = reinterpret_cast<int32_t *>(b + o_sidx);
+        // the per-segment candidate lists are the streamed path's; the GEMM path keeps
+        // its quantized query there instead
+        w->spare = b + o_skey;
+        w->spare_bytes = o_sidx + sizeof(int32_t) * (size_t)cap * Nq - o_skey;
         w->zero_bytes = z1 - z0;
         w->words = words;
         w->ccap = ccap;
@@ -1880,7 +1887,8 @@ cudaError_t index_pipeline(const csa_cache &c, const void *q_idx, const float *w
     // many queries per request (prefill): scores as a tensor-core GEMM, and when the
     // rows fit in shared memory one selection kernel that needs no zeroed state
     const bool gemm = !pool && !n_vis_given && Nq >= kPrefillQueriesPerRequest * c.batch &&
-                      prefill_scores_supported(c.idx_dtype, c.idx_dim, H_I);
+                      prefill_scores_supported(c.idx_dtype, c.idx_dim, H_I) &&
+                      prefill_query_scratch_bytes(c.idx_dtype, c.idx_dim, Nq, H_I) <= ws.spare_bytes;
     const bool row_sel = gemm && rows <= kRowSelMaxRows;
     cudaError_t err = cudaSuccess;
     // the pass + final selection kernels need zeroed counters, histograms and bitmaps;
@@ -1927,8 +1935,7 @@ cudaError_t index_pipeline(const csa_cache &c, const void *q_idx, const float *w
     sa.layers = layers;
     const int grid = min(num_sms, kMaxScanCtas);
     if (gemm) {
-        err = launch_prefill_scores(c.idx_key, c.batch, c.capacity, c.idx_dim, q_idx, w, Nq, H_I, ws.req, ws.n_vis, ws.scores,
-                                    rows, c.status, num_sms, s);
+        err = launch_prefill_scores(c, q_idx, w, Nq, H_I, ws.req, ws.n_vis, ws.scores, rows, ws.spare, num_sms, s);
         if (err != cudaSuccess) return err;
         if (row_sel) {
             const int smem = 16 * ((rows + 3) / 4);

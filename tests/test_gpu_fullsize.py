@@ -11,7 +11,8 @@ The GPU runs the whole batch; the oracle recomputes sampled queries one by one.
     scale formats (E8M0 per 32, E4M3 per 16).
   * prefill_b4_8k: 8192 new tokens appended to 65536 cached ones in each of 4
     requests; every new block checked, then 32768 causal queries indexed and
-    attended with sampled queries recomputed.
+    attended with sampled queries recomputed; and the same indexer call over
+    MXFP4 indexer keys (the block-scaled tensor-core GEMM), sampled.
 Cache contents for the first two are seeded bytes (the kernels' inputs), not
 outputs of the compression kernel."""
 import numpy as np
@@ -272,3 +273,37 @@ def test_prefill_b4_8k_sampled():
                                         np.array([t], np.int64), np.array([W], np.int32), D ** -0.5)
             err, _ = parity.attention_row_error(host(out_d[i:i + 1]), want)
             assert err <= parity.ATT_TOL, (b, t, err)
+
+
+def test_prefill_b4_8k_mxfp4_index_sampled():
+    # the prefill_b4_8k indexer call with MXFP4 indexer keys (E2M1 codes, one E8M0 scale
+    # per 32 channels): 32768 causal queries over 16384..18432 blocks per request score on
+    # the block-scaled tensor-core GEMM; sampled queries are recomputed by the oracle
+    import fp4_kv_cache_csa_b200 as csa
+
+    wl = datagen.WORKLOADS["prefill_b4_8k"]
+    B, D, dI, m, k = wl.batch, wl.dim, wl.idx_dim, wl.block, wl.topk
+    T0, T1 = wl.ctx_min, wl.ctx_max
+    cap, NEW = T1 // m, T1 - T0
+    g = datagen.generator(545, 1)
+    codes = g.integers(0, 256, size=(B, cap, dI // 2)).astype(np.uint8)
+    scales = g.integers(122, 127, size=(B, cap, dI // 32)).astype(np.uint8)
+    n_blocks = np.full(B, cap, np.int32)
+    cache = make_cache(np.zeros((B, cap, D // 2), np.uint8), np.zeros((B, cap, D // 32), np.uint8), n_blocks, m,
+                       codes, 2, idx_key_scale=scales)
+    Nq = B * NEW
+    qo = (np.arange(B + 1) * NEW).astype(np.int32)
+    qp = np.tile(np.arange(T0, T1, dtype=np.int32), B)
+    q_idx = datagen.normal_bf16((Nq, wl.idx_heads, dI), 546, 1)
+    w = datagen.normal_f32((Nq, wl.idx_heads), 546, 2, std=0.5)
+    sel = host(csa.csa_index_topk(cache, dev(q_idx), dev(w), dev(qo), dev(qp), k))
+    assert csa.csa_read_device_status(cache) == 0
+    one = np.array([0, 1], np.int32)
+    for b in range(B):
+        for t in (0, 1, NEW // 2 - 1, NEW - 1):
+            i = b * NEW + t
+            sel_ref, scores, n_vis = oracle.index_topk(codes[b:b + 1], n_blocks[b:b + 1], one, qp[i:i + 1],
+                                                       q_idx[i:i + 1], w[i:i + 1], m=m, k=k,
+                                                       idx_dtype=oracle.IDX_MXFP4, idx_key_scale=scales[b:b + 1])
+            assert n_vis[0] == (T0 + t + 1) // m
+            parity.check_topk(sel[i:i + 1], sel_ref, scores, n_vis, k)

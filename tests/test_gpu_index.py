@@ -125,7 +125,7 @@ def test_maximum_sizes():
 def test_many_queries_per_request_gemm_path(H_I, dI, cap):
     # calls with many queries per request (prefill) score on the tensor cores; ragged
     # request sizes put two or three requests into one query tile, and capacities that
-    # are not multiples of 4 take the scalar score stores
+    # are not multiples of 4 give score rows that are not 16-byte aligned
     counts = [300, 213, 1]
     lengths = [3000, 2100, 500]  # filled blocks per request
     keys = gen_keys(3, cap, dI, 0, 60 + H_I)

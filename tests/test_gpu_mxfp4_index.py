@@ -6,7 +6,9 @@ main KV; cue 12: indexer keys come from the main KV) -- and the indexer query
 is quantized by the same rule before the scores, so every product is exact.
 Cases: the key store (m = 1 strict, pooled with the near-tie rule), decode
 scoring at d_I = 64 / 128 / 256 with ragged contexts, many queries per request
-(causal), exact ties, the pool + Reindex calls, and the head limit."""
+(the block-scaled tensor-core GEMM: several requests per query tile, ragged key
+counts, 60 binades of scales, exact ties), exact ties on the streamed path, the
+pool + Reindex calls, and the head limit."""
 import numpy as np
 import pytest
 
@@ -140,7 +142,7 @@ def test_exact_ties_go_to_the_lower_index():
 
 
 def test_many_queries_per_request_causal():
-    # prefill-shaped: 40 queries per request at spread positions (MXFP4 keys take the streamed path)
+    # prefill-shaped: 40 queries per request at spread positions (the block-scaled GEMM path)
     lengths = [3000, 2200]
     codes, scales = mx_keys(2, 3001, 128, 73)
     g = datagen.generator(73, 1)
@@ -148,6 +150,53 @@ def test_many_queries_per_request_causal():
     qo = (np.arange(3) * per).astype(np.int32)
     qp = np.concatenate([np.sort(g.integers(0, 4 * n, per)) for n in lengths]).astype(np.int32)
     run_index(codes, scales, lengths, qo, qp, 4, 256, seed=74)
+
+
+@pytest.mark.parametrize("H_I,cap", [(4, 3000), (2, 3001), (1, 3002)])
+def test_prefill_gemm_path(H_I, cap):
+    # many queries per request score on the block-scaled tensor-core GEMM (kind::mxf4):
+    # ragged request sizes put two or three requests into one 128-column query tile,
+    # key counts end inside a 128-key stage, one request has a single query
+    counts = [300, 213, 1]
+    lengths = [3000, 2100, 500]
+    codes, scales = mx_keys(3, cap, 128, 80 + H_I)
+    qo = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    qp = np.concatenate([np.linspace(0, 4 * L - 1, c).astype(np.int32) for c, L in zip(counts, lengths)])
+    sel, _, n_vis = run_index(codes, scales, lengths, qo, qp, H_I, 256, seed=81)
+    assert n_vis.min() < 256 < n_vis.max()
+
+
+def test_prefill_gemm_path_scale_spread():
+    # key scales over 20 binades on the block-scaled MMA (the streamed path's test above
+    # spans 60): the tensor core anchors a block-scaled sum at the largest block scale
+    # taking part, even where that block's products cancel to zero, so keys whose
+    # 32-channel scales lie dozens of binades apart can lose a small block's part that
+    # fp32 keeps; pooled keys' scales span a few binades
+    counts, lengths = [64, 64], [4000, 3500]
+    codes, scales = mx_keys(2, 4096, 128, 82, scale_lo=117, scale_hi=137)
+    qo = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    qp = np.concatenate([np.linspace(2 * L, 4 * L - 1, c).astype(np.int32) for c, L in zip(counts, lengths)])
+    run_index(codes, scales, lengths, qo, qp, 4, 500, seed=83)
+
+
+@pytest.mark.parametrize("case", ["duplicates", "zeros"])
+def test_prefill_gemm_path_exact_ties(case):
+    # equal scores at the threshold go to the lower index on the GEMM path as well
+    cap = 8192
+    codes, scales = mx_keys(2, cap, 128, 84)
+    rng = np.random.default_rng(85)
+    for b in range(2):
+        if case == "duplicates":
+            dup = rng.choice(cap, 3000, replace=False)
+            codes[b, dup] = codes[b, dup[0]]
+            scales[b, dup] = scales[b, dup[0]]
+        else:
+            codes[b, :5000] = 0
+    counts, lengths = [64, 64], [8192, 6000]
+    qo = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    qp = np.concatenate([np.linspace(2 * L, 4 * L - 1, c).astype(np.int32) for c, L in zip(counts, lengths)])
+    for k in (100, 2999, 3500):
+        run_index(codes, scales, lengths, qo, qp, 4, k, seed=86)
 
 
 def test_pool_and_reindex():
