@@ -67,10 +67,12 @@ constexpr int kScanWarps = kScanThreads / 32;
 constexpr int kMaxScanCtas = 256;
 constexpr int kFusedScheduleQueries = 512;  // up to this many queries the scan computes its own schedule (= its threads)  // scan grid: min(SMs, this); sizes the per-(query, CTA) counts
 // Work units charged for starting a query in a scan range (query fragments,
-// histogram clear and flush, completion count): about as long as scanning this
-// many 16-key groups. The flat split counts them, so ranges that cross a query
-// boundary get fewer keys.
-constexpr int kSegCost = 96;
+// histogram clear, and the segment's candidate extraction at its end): about as
+// long as scanning this many 16-key groups. The flat split counts them, so ranges
+// that cross a query boundary get fewer keys. (Measured on B200 at 32 requests x
+// 512K-1M tokens: with 96 units, CTAs holding two segments ended ~6 us after
+// those holding one with the same units, i.e. a segment costs ~200 groups.)
+constexpr int kSegCost = 200;
 constexpr int kSelThreads = 1024;
 constexpr int kPassThreads = 256;
 constexpr int kCandCap = 32768;    // candidate slots per query (members of the threshold bin)
@@ -886,7 +888,9 @@ __global__ void __launch_bounds__(kMergeThreads) select_merge_kernel(MergeArgs a
     __shared__ uint32_t s_off[kMaxScanCtas];      // where that CTA's candidates start in the row
     grid_dep_wait();
     const int i = blockIdx.x, tid = threadIdx.x;
+    // the query's schedule values, loaded together (one round trip to L2)
     const int n = a.n_vis[i];
+    const long long NG = a.gprefix[a.Nq], u0 = a.gprefix[i], u1 = a.gprefix[i + 1];
     const int K = min(a.topk, n);
     int32_t *out = a.sel_idx + (size_t)i * a.topk;
     if (K == n) {  // every visible block (or none)
@@ -898,7 +902,6 @@ __global__ void __launch_bounds__(kMergeThreads) select_merge_kernel(MergeArgs a
         return;
     }
     // the scan CTAs whose ranges hold this query's units [u0, u1), as the scan split them
-    const long long NG = a.gprefix[a.Nq], u0 = a.gprefix[i], u1 = a.gprefix[i + 1];
     const int G = a.G;
     const int c_first = (int)(((u0 + 1) * G - 1) / NG), c_last = (int)((u1 * G - 1) / NG);
     const int nseg = c_last - c_first + 1;  // <= G <= kMaxScanCtas <= blockDim
@@ -1011,11 +1014,27 @@ __global__ void __launch_bounds__(kMergeThreads) select_merge_kernel(MergeArgs a
             w_eq[warp] = neq;
         }
         __syncthreads();
-        uint32_t ob = 0, tb = 0;  // outputs and ties before this warp's run
-        for (int v = 0; v < warp; ++v) {
-            const uint32_t e = w_eq[v];
-            ob += w_gt[v] + (take == kTakeAll ? e : (tb >= take ? 0u : min(e, take - tb)));
-            tb += e;
+        // outputs and ties before this warp's run: lane v of every warp takes run v's
+        // counts; exclusive warp scans give the ties before run v, then the outputs
+        uint32_t ob, tb;
+        {
+            const uint32_t e = w_eq[lane], gt = w_gt[lane];
+            uint32_t te = e;  // inclusive scan of the ties
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xffffffffu, te, o);
+                if (lane >= o) te += y;
+            }
+            const uint32_t tbl = te - e;  // ties before run `lane`
+            uint32_t outl = gt + (take == kTakeAll ? e : (tbl >= take ? 0u : min(e, take - tbl)));
+            uint32_t to = outl;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xffffffffu, to, o);
+                if (lane >= o) to += y;
+            }
+            ob = __shfl_sync(0xffffffffu, to - outl, warp);
+            tb = __shfl_sync(0xffffffffu, tbl, warp);
         }
         const uint32_t lt = (1u << lane) - 1u;
         for (uint32_t base = w0; base < w1; base += 32) {
