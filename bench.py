@@ -476,6 +476,7 @@ def measure_prefill(device, stream, flush, steps: int = 3):
     import fp4_kv_cache_csa_b200 as csa
 
     pf = Prefill(device)
+    torch.cuda.synchronize()  # the inputs were written on the default stream
     with torch.cuda.stream(stream):
         for fn in pf.stages():  # warm-up pass
             fn()
@@ -508,6 +509,7 @@ def measure_prefill_index_mxfp4(device, stream, flush, steps: int = 3):
     import fp4_kv_cache_csa_b200 as csa
 
     pf = Prefill(device, idx_dtype=csa.CSA_IDX_MXFP4)
+    torch.cuda.synchronize()  # the inputs were written on the default stream
     with torch.cuda.stream(stream):
         pf.stage_compress()
         pf.stage_index()
@@ -623,6 +625,7 @@ def measure_configs(device, stream, flush, steps: int = 20):
     res = {}
     for name, kw in runs:
         cr = ConfigRun(device, name, **kw)
+        torch.cuda.synchronize()  # the caches were written on the default stream
         fns = cr.stages()
         with torch.cuda.stream(stream):
             for fn in fns:
@@ -685,6 +688,7 @@ def measure_index_mxfp4(device, stream, flush, wl, steps: int = 20):
     sel = torch.empty(B, TOPK, dtype=torch.int32, device=device)
     ws = torch.empty(csa.csa_index_topk_workspace(cache, B, TOPK), dtype=torch.uint8, device=device)
     fn = lambda: csa.csa_index_topk(cache, wl.q_idx, wl.w, wl.q_offsets, wl.q_pos, TOPK, sel_idx=sel, workspace=ws)
+    torch.cuda.synchronize()  # the cache was written on the default stream
     with torch.cuda.stream(stream):
         fn()
         stream.synchronize()

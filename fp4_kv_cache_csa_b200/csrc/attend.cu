@@ -355,6 +355,16 @@ __device__ __forceinline__ int load_window_row(const AttArgs &a, const TileRef &
     return R;
 }
 
+// The CTA whose range holds flat tile t: the last c with cta_t[c] <= t.
+__device__ __forceinline__ int cta_of_tile(const long long *cta_t, int G, long long t) {
+    int lo = 0, hi = G - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (cta_t[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
 // ---------------------------------------------------------------- schedule
 // One CTA of 1024 threads per query: its query's scale exponent sq[i] (from
 // max|q|), the Q' image (q * 2^-sq in fp16, in the swizzled K-major layout
@@ -383,7 +393,7 @@ __global__ void __launch_bounds__(1024) attend_schedule_kernel(
     const int32_t *q_offsets, const int32_t *q_pos, const int32_t *n_blocks, const int32_t *win_len, int batch,
     int Nq, int m, int cap, int topk, int max_win, const __nv_bfloat16 *q, int H, int G, QInfo *qinfo,
     long long *tprefix, int32_t *cta_q, long long *cta_t, long long *uprefix, int32_t *sq, uint8_t *qimg, float *out,
-    float *lse, int32_t *status) {
+    float *lse, int32_t *status, int2 *qspan) {
     __shared__ long long red[32];
     __shared__ long long round_total;
     __shared__ float fred[32];
@@ -520,16 +530,12 @@ __global__ void __launch_bounds__(1024) attend_schedule_kernel(
             cta_q[c] = lo;
         }
     }
-}
-
-// The CTA whose range holds flat tile t: the last c with cta_t[c] <= t.
-__device__ __forceinline__ int cta_of_tile(const long long *cta_t, int G, long long t) {
-    int lo = 0, hi = G - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (cta_t[mid] <= t) lo = mid; else hi = mid - 1;
+    __syncthreads();  // cta_t complete (global writes of this CTA, visible to its threads)
+    // the first and last CTA holding each query's tiles, for the merge ((-1, -1): no tiles)
+    for (int i = threadIdx.x; i < Nq; i += blockDim.x) {
+        const long long t0 = tprefix[i], t1 = tprefix[i + 1];
+        qspan[i] = t1 > t0 ? make_int2(cta_of_tile(cta_t, G, t0), cta_of_tile(cta_t, G, t1 - 1)) : make_int2(-1, -1);
     }
-    return lo;
 }
 
 // ---------------------------------------------------------------- split merge
@@ -543,13 +549,14 @@ constexpr int kMergeHeads = 8;
 // index c; only a query that CTA c - 1 and CTA c both cover can need a merge,
 // and the CTA for the first such boundary of a query merges it, so the grid
 // has G - 1 columns instead of one per query.
-__global__ void __launch_bounds__(256) attend_merge_kernel(const long long *tprefix, const long long *cta_t, int Nq,
-                                                           int H, int D, int G,
+__global__ void __launch_bounds__(256) attend_merge_kernel(const long long *tprefix, const long long *cta_t,
+                                                           const int2 *qspan, int Nq, int H, int D, int G,
                                                            const float *part_o, const float *part_rho,
                                                            const float *part_l, float *out, float *lse,
                                                            int by_boundary) {
     __shared__ int slots[256];
     __shared__ float wts[256 * kMergeHeads];
+    __shared__ float s_rho[256 * kMergeHeads], s_l[256 * kMergeHeads];
     __shared__ float inv_l[kMergeHeads];
     __shared__ int np_s;
     grid_dep_wait();
@@ -567,70 +574,77 @@ __global__ void __launch_bounds__(256) attend_merge_kernel(const long long *tpre
             if (tprefix[mid] < rb) lo = mid; else hi = mid - 1;
         }
         i = lo;
-        if (tprefix[i + 1] <= rb) return;  // the boundary is at the end of query i: nothing straddles
-        const long long Ti0 = tprefix[i];
-        if (cta_of_tile(cta_t, G, Ti0) + 1 != c) return;  // not the query's first inner boundary
+        if (tprefix[i + 1] <= rb) return;      // the boundary is at the end of query i: nothing straddles
+        if (qspan[i].x + 1 != c) return;        // not the query's first inner boundary
     }
-    const long long Ti = tprefix[i], Ti1 = tprefix[i + 1];
-    if (Ti1 == Ti) return;  // no entry at all: written by the schedule kernel
-    const int c_first = cta_of_tile(cta_t, G, Ti);
-    const int c_last = cta_of_tile(cta_t, G, Ti1 - 1);
-    if (c_first == c_last) return;  // one CTA covered the query and wrote it
-    if (threadIdx.x == 0) {
+    // the CTAs that hold the query's tiles (the schedule kernel found them)
+    const int2 span = qspan[i];
+    const int c_first = span.x, c_last = span.y;
+    if (c_first < 0 || c_first == c_last) return;  // no entry (written by the schedule kernel) or one CTA wrote it
+    // its partials, in CTA order, CTAs with an empty range skipped: warp 0, 32 CTAs per round
+    if (threadIdx.x < 32) {
         int np = 0;
-        for (int cc = c_first; cc <= c_last && np < 256; ++cc) {
-            const long long rb = cta_t[cc], re = cta_t[cc + 1];
-            if (rb >= re) continue;  // CTA with an empty range
-            slots[np++] = 2 * cc + (rb >= Ti ? 0 : 1);
+        for (int cc0 = c_first; cc0 <= c_last && np < 256; cc0 += 32) {
+            const int cc = cc0 + (int)threadIdx.x;
+            bool has = false;
+            long long rb = 0;
+            if (cc <= c_last) {
+                rb = cta_t[cc];
+                has = rb < cta_t[cc + 1];
+            }
+            const uint32_t m = __ballot_sync(0xffffffffu, has);
+            const int pos = np + __popc(m & ((1u << threadIdx.x) - 1u));
+            if (has && pos < 256) slots[pos] = 2 * cc + (rb >= tprefix[i] ? 0 : 1);
+            np += __popc(m);
         }
-        np_s = np;
+        if (threadIdx.x == 0) np_s = min(np, 256);
     }
     __syncthreads();
     const int np = np_s;
     const int nh = min(kMergeHeads, H - h0);
+    // every partial's (rho, l) of the slice's heads, one load per thread
+    for (int k = threadIdx.x; k < np * kMergeHeads; k += blockDim.x) {
+        const int p = k / kMergeHeads, hh = k % kMergeHeads;
+        const size_t at = (size_t)slots[p] * kHeads + h0 + hh;
+        s_rho[k] = hh < nh ? part_rho[at] : -INFINITY;
+        s_l[k] = hh < nh ? part_l[at] : 0.f;
+    }
+    __syncthreads();
     if (threadIdx.x < nh) {
         const int h = h0 + threadIdx.x;
         float rmax = -INFINITY;
-        for (int p = 0; p < np; ++p) rmax = fmaxf(rmax, part_rho[(size_t)slots[p] * kHeads + h]);
+        for (int p = 0; p < np; ++p) rmax = fmaxf(rmax, s_rho[p * kMergeHeads + threadIdx.x]);
         float l = 0.f;
         for (int p = 0; p < np; ++p) {
             // rho = -inf: no entry of this head in that partial (or in any, if rmax is -inf)
-            const float wgt = rmax == -INFINITY ? 0.f : exp2f(part_rho[(size_t)slots[p] * kHeads + h] - rmax);
+            const float wgt = rmax == -INFINITY ? 0.f : exp2f(s_rho[p * kMergeHeads + threadIdx.x] - rmax);
             wts[p * kMergeHeads + threadIdx.x] = wgt;
-            l += wgt * part_l[(size_t)slots[p] * kHeads + h];
+            l += wgt * s_l[p * kMergeHeads + threadIdx.x];
         }
         inv_l[threadIdx.x] = l > 0.f ? 1.f / l : 0.f;
         if (lse && blockIdx.z == 0) lse[(size_t)i * H + h] = l > 0.f ? (rmax + log2f(l)) * 0.69314718055994531f : -INFINITY;
     }
     __syncthreads();
     // one float4 of one head per thread: this CTA's 8 heads x 128 channels (blockIdx.z);
-    // four partials in flight at a time
+    // eight partials in flight at a time
     const int hh = threadIdx.x >> 5, d4 = blockIdx.z * 32 + (threadIdx.x & 31);
     if (hh < nh && d4 < D / 4) {
         const float4 *src = reinterpret_cast<const float4 *>(part_o + (size_t)(h0 + hh) * D) + d4;
         const size_t slot_stride = (size_t)kHeads * D / 4;  // float4s per partial
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        int p = 0;
-        for (; p + 4 <= np; p += 4) {
-            float4 o[4];
+        for (int p0 = 0; p0 < np; p0 += 8) {
+            float4 o[8];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) o[k] = __ldcg(src + (size_t)slots[p + k] * slot_stride);
+            for (int k = 0; k < 8; ++k)
+                o[k] = p0 + k < np ? __ldcg(src + (size_t)slots[p0 + k] * slot_stride) : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float wgt = wts[(p + k) * kMergeHeads + hh];
+            for (int k = 0; k < 8; ++k) {
+                const float wgt = p0 + k < np ? wts[(p0 + k) * kMergeHeads + hh] : 0.f;
                 acc.x = fmaf(wgt, o[k].x, acc.x);
                 acc.y = fmaf(wgt, o[k].y, acc.y);
                 acc.z = fmaf(wgt, o[k].z, acc.z);
                 acc.w = fmaf(wgt, o[k].w, acc.w);
             }
-        }
-        for (; p < np; ++p) {
-            const float4 o = __ldcg(src + (size_t)slots[p] * slot_stride);
-            const float wgt = wts[p * kMergeHeads + hh];
-            acc.x = fmaf(wgt, o.x, acc.x);
-            acc.y = fmaf(wgt, o.y, acc.y);
-            acc.z = fmaf(wgt, o.z, acc.z);
-            acc.w = fmaf(wgt, o.w, acc.w);
         }
         const float il = inv_l[hh];
         reinterpret_cast<float4 *>(out + ((size_t)i * H + h0 + hh) * D)[d4] =
@@ -1041,11 +1055,11 @@ template <int D>
 cudaError_t launch_schedule(const csa_cache &c, const AttArgs &a, const int32_t *q_offsets, const int32_t *q_pos,
                             const int32_t *win_len, int topk, int max_win, const void *q, int num_ctas, QInfo *qinfo,
                             long long *tprefix, int32_t *cta_q, long long *cta_t, long long *uprefix, int32_t *sq,
-                            uint8_t *qimg, cudaStream_t s) {
+                            uint8_t *qimg, int2 *qspan, cudaStream_t s) {
     attend_schedule_kernel<D><<<a.Nq + 1, 1024, 0, s>>>(q_offsets, q_pos, c.n_blocks, win_len, c.batch, a.Nq, c.block,
                                                    c.capacity, topk, max_win, static_cast<const __nv_bfloat16 *>(q),
                                                    a.H, num_ctas, qinfo, tprefix, cta_q, cta_t, uprefix, sq, qimg, a.out, a.lse,
-                                                   c.status);
+                                                   c.status, qspan);
     return cudaGetLastError();
 }
 
@@ -1064,6 +1078,7 @@ size_t attend_workspace_bytes(int Nq, int D, int num_ctas) {
     take(4 * (size_t)2 * num_ctas * kHeads * D);      // part_o
     take(4 * (size_t)2 * num_ctas * kHeads);          // part_rho
     take(4 * (size_t)2 * num_ctas * kHeads);          // part_l
+    take(8 * (size_t)Nq);                             // qspan
     return off;
 }
 
@@ -1090,6 +1105,7 @@ cudaError_t launch_attend(const csa_cache &c, const void *q, int Nq, int H, cons
     a.part_o = reinterpret_cast<float *>(take(4 * (size_t)2 * num_ctas * kHeads * D));
     a.part_rho = reinterpret_cast<float *>(take(4 * (size_t)2 * num_ctas * kHeads));
     a.part_l = reinterpret_cast<float *>(take(4 * (size_t)2 * num_ctas * kHeads));
+    int2 *qspan = reinterpret_cast<int2 *>(take(8 * (size_t)Nq));
     a.fp4 = c.fp4;
     a.scale = c.scale;
     a.sel_idx = sel_idx;
@@ -1116,14 +1132,14 @@ cudaError_t launch_attend(const csa_cache &c, const void *q, int Nq, int H, cons
     const int G = num_ctas;  // work ranges, one per CTA
     if (D == 512) {
         if ((err = launch_schedule<512>(c, a, q_offsets, qp, wl, topk, max_win, q, num_ctas, qinfo, tprefix, cta_q, cta_t,
-                                        uprefix, sq, qimg, s)) != cudaSuccess)
+                                        uprefix, sq, qimg, qspan, s)) != cudaSuccess)
             return err;
         err = c.scale_fmt == CSA_SCALE_E4M3_16 ? launch_main<512, kScaleE4M3x16>(a, num_ctas, s)
                                                 : launch_main<512, kScaleE8M0x32>(a, num_ctas, s);
         if (err != cudaSuccess) return err;
     } else if (D == 128) {
         if ((err = launch_schedule<128>(c, a, q_offsets, qp, wl, topk, max_win, q, num_ctas, qinfo, tprefix, cta_q, cta_t,
-                                        uprefix, sq, qimg, s)) != cudaSuccess)
+                                        uprefix, sq, qimg, qspan, s)) != cudaSuccess)
             return err;
         err = c.scale_fmt == CSA_SCALE_E4M3_16 ? launch_main<128, kScaleE4M3x16>(a, num_ctas, s)
                                                 : launch_main<128, kScaleE8M0x32>(a, num_ctas, s);
@@ -1142,7 +1158,8 @@ cudaError_t launch_attend(const csa_cache &c, const void *q, int Nq, int H, cons
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, attend_merge_kernel, (const long long *)tprefix, (const long long *)cta_t, Nq, H, D, G,
+    return cudaLaunchKernelEx(&cfg, attend_merge_kernel, (const long long *)tprefix, (const long long *)cta_t,
+                              (const int2 *)qspan, Nq, H, D, G,
                               (const float *)a.part_o, (const float *)a.part_rho, (const float *)a.part_l, out, lse,
                               by_boundary);
 }

@@ -420,24 +420,24 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_score_kernel(const __gr
                     ok = mbar_wait_ab<false>(bar(B_CFULL + u), (g / NACC) & 1, abort_flag);
                     if (__any_sync(0xffffffffu, !ok)) { ok = false; break; }
                     tc_fence_after();
-                    uint32_t r[64];  // the thread's 64 columns, one wait for all four loads
-                    CSA_LD16(tmem + lane_off + u * kPfCols + 64 * ch, r);
-                    CSA_LD16(tmem + lane_off + u * kPfCols + 64 * ch + 16, (r + 16));
-                    CSA_LD16(tmem + lane_off + u * kPfCols + 64 * ch + 32, (r + 32));
-                    CSA_LD16(tmem + lane_off + u * kPfCols + 64 * ch + 48, (r + 48));
-                    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-                    tc_fence_before();
-                    mbar_arrive(bar(B_CFREE + u));  // the accumulator is in registers
                     const int key = kt * kPfKeys + 32 * qw + lane;
 #pragma unroll
-                    for (int jq = 0; jq < QPT; ++jq) {
-                        float sc = 0.f;
+                    for (int c = 0; c < 2; ++c) {
+                        float v[32];
+                        tmem_ld32(tmem + lane_off + u * kPfCols + 64 * ch + 32 * c, v);
 #pragma unroll
-                        for (int h = 0; h < HI; ++h) sc = fmaf(wr[HI * jq + h], fmaxf(__uint_as_float(r[HI * jq + h]), 0.f), sc);
-                        const int lim = NR == QPT ? nr[jq % NR]
-                                                  : (s_req[QPT * ch + jq] == b ? s_nv[QPT * ch + jq] : 0);
-                        if (key < lim) st_score(srow + (size_t)jq * a.rows + key, sc);
+                        for (int j = 0; j < 32 / HI; ++j) {
+                            const int jq = (32 / HI) * c + j;  // query of the thread's QPT
+                            float sc = 0.f;
+#pragma unroll
+                            for (int h = 0; h < HI; ++h) sc = fmaf(wr[HI * jq + h], fmaxf(v[HI * j + h], 0.f), sc);
+                            const int lim = NR == QPT ? nr[jq % NR]
+                                                      : (s_req[QPT * ch + jq] == b ? s_nv[QPT * ch + jq] : 0);
+                            if (key < lim) st_score(srow + (size_t)jq * a.rows + key, sc);
+                        }
                     }
+                    tc_fence_before();
+                    mbar_arrive(bar(B_CFREE + u));
                 }
                 if (!ok) *abort_flag = 1;
             }
