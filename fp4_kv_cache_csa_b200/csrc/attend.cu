@@ -54,6 +54,8 @@ namespace csa {
 namespace {
 
 constexpr int kTile = 128;
+constexpr int kSchedSmemQueries = 1024;  // the schedule searches its prefixes in shared memory up to here
+constexpr int kMaxAttendCtas = 256;      // ... and the CTA ranges up to this many CTAs
 constexpr int kHeads = 64;
 constexpr int kThreads = 256;
 // Relative cost of the work the CTAs share out (measured per-CTA times on B200 at
@@ -460,7 +462,13 @@ __global__ void __launch_bounds__(1024) attend_schedule_kernel(
     }
     if (qi != Nq) return;
     // ---- CTA Nq (in parallel with the others): per-query records, tile prefix,
-    // first query of every CTA range
+    // first query of every CTA range. The prefixes and the CTA ranges are searched
+    // below; up to kSchedSmemQueries queries they are searched in shared memory.
+    __shared__ long long s_tpre[kSchedSmemQueries + 1], s_upre[kSchedSmemQueries + 1], s_ctat[kMaxAttendCtas + 1];
+    const bool in_smem = Nq <= kSchedSmemQueries && G <= kMaxAttendCtas;
+    const long long *tpre = in_smem ? s_tpre : tprefix;
+    const long long *upre = in_smem ? s_upre : uprefix;
+    const long long *ctat = in_smem ? s_ctat : cta_t;
     long long carry = 0, ucarry = 0;
     for (int base = 0; base < Nq; base += blockDim.x) {
         const int i = base + threadIdx.x;
@@ -476,20 +484,30 @@ __global__ void __launch_bounds__(1024) attend_schedule_kernel(
         if (i < Nq) {
             const long long t0 = carry + incl - tiles;
             tprefix[i + 1] = t0 + tiles;
+            if (in_smem) s_tpre[i + 1] = t0 + tiles;
             QInfo r;
             r.a = make_int4(b, ne, ct, wl);
             r.b = make_int4(n_blocks[b], 0, 0, 0);
             r.t = make_longlong2(t0, t0 + tiles);
             qinfo[i] = r;
         }
-        if (i == 0) tprefix[0] = 0;
+        if (i == 0) {
+            tprefix[0] = 0;
+            if (in_smem) s_tpre[0] = 0;
+        }
         if (threadIdx.x == blockDim.x - 1) round_total = incl;
         __syncthreads();
         carry += round_total;
         __syncthreads();
         const long long uincl = block_inclusive_scan<long long>(units, red);
-        if (i < Nq) uprefix[i + 1] = ucarry + uincl;
-        if (i == 0) uprefix[0] = 0;
+        if (i < Nq) {
+            uprefix[i + 1] = ucarry + uincl;
+            if (in_smem) s_upre[i + 1] = ucarry + uincl;
+        }
+        if (i == 0) {
+            uprefix[0] = 0;
+            if (in_smem) s_upre[0] = 0;
+        }
         if (threadIdx.x == blockDim.x - 1) round_total = uincl;
         __syncthreads();
         ucarry += round_total;
@@ -508,11 +526,11 @@ __global__ void __launch_bounds__(1024) attend_schedule_kernel(
             int lo = 0, hi = Nq - 1;  // last i with uprefix[i] <= ub
             while (lo < hi) {
                 const int mid = (lo + hi + 1) >> 1;
-                if (uprefix[mid] <= ub) lo = mid; else hi = mid - 1;
+                if (upre[mid] <= ub) lo = mid; else hi = mid - 1;
             }
             const QInfo r = qinfo[lo];
             const long long ct = r.a.z, nt = r.t.y - r.t.x;
-            const long long x = ub - uprefix[lo] - kStartCost;  // units into the query's tiles
+            const long long x = ub - upre[lo] - kStartCost;  // units into the query's tiles
             long long before = 0;                               // its tiles starting before ub
             if (x > 0) {
                 if (x <= ct * kCTileCost) before = (x + kCTileCost - 1) / kCTileCost;
@@ -521,11 +539,12 @@ __global__ void __launch_bounds__(1024) attend_schedule_kernel(
             tb = r.t.x + min(before, nt);
         }
         cta_t[c] = tb;
+        if (in_smem) s_ctat[c] = tb;
         if (c < G) {
             int lo = 0, hi = Nq - 1;
             while (lo < hi) {
                 const int mid = (lo + hi + 1) >> 1;
-                if (tprefix[mid] <= tb) lo = mid; else hi = mid - 1;
+                if (tpre[mid] <= tb) lo = mid; else hi = mid - 1;
             }
             cta_q[c] = lo;
         }
@@ -533,8 +552,8 @@ __global__ void __launch_bounds__(1024) attend_schedule_kernel(
     __syncthreads();  // cta_t complete (global writes of this CTA, visible to its threads)
     // the first and last CTA holding each query's tiles, for the merge ((-1, -1): no tiles)
     for (int i = threadIdx.x; i < Nq; i += blockDim.x) {
-        const long long t0 = tprefix[i], t1 = tprefix[i + 1];
-        qspan[i] = t1 > t0 ? make_int2(cta_of_tile(cta_t, G, t0), cta_of_tile(cta_t, G, t1 - 1)) : make_int2(-1, -1);
+        const long long t0 = tpre[i], t1 = tpre[i + 1];
+        qspan[i] = t1 > t0 ? make_int2(cta_of_tile(ctat, G, t0), cta_of_tile(ctat, G, t1 - 1)) : make_int2(-1, -1);
     }
 }
 
