@@ -53,6 +53,11 @@ def set_batch(n: int):
     B = int(n)
 
 
+def set_prefill_requests(n: int):
+    """Requests of the prefill workload (4; fewer only for profiling a smaller case)."""
+    Prefill.B = int(n)
+
+
 def set_scale_fmt(name: str):
     global SCALE_FMT
     SCALE_FMT = SCALE_FMT_NAMES[name]
@@ -492,7 +497,7 @@ def measure_prefill(device, stream, flush, steps: int = 3):
     stream.synchronize()
     st = np.array([[ev[k][s_].elapsed_time(ev[k][s_ + 1]) for s_ in range(3)] for k in range(steps)]).mean(axis=0)
     status = csa.csa_read_device_status(pf.cache, stream)
-    res = {"workload": "prefill_b4_8k", "queries": pf.Nq, "ms": float(st.sum()),
+    res = {"workload": f"prefill_b{pf.B}_8k", "queries": pf.Nq, "ms": float(st.sum()),
            "stage_ms": {"compress": float(st[0]), "index_topk": float(st[1]), "attend": float(st[2])},
            "index_gflop": pf.index_flops() / 1e9,
            "index_tflops": pf.index_flops() / (st[1] * 1e-3) / 1e12, "device_status": int(status)}
@@ -527,7 +532,7 @@ def measure_prefill_index_mxfp4(device, stream, flush, steps: int = 3):
     bf16_peak, kind = measured_bf16_tflops()
     fp4_peak = 4.0 * bf16_peak  # dense MXFP4 : bf16 = 9 : 2.25 PFLOP/s nominal
     flops = pf.index_flops()
-    res = {"workload": "prefill_b4_8k", "idx_dtype": "mxfp4", "queries": pf.Nq, "index_ms": ms,
+    res = {"workload": f"prefill_b{pf.B}_8k", "idx_dtype": "mxfp4", "queries": pf.Nq, "index_ms": ms,
            "index_gflop": flops / 1e9, "index_tflops": flops / (ms * 1e-3) / 1e12,
            "mxfp4_peak_tflops": fp4_peak, "peak_kind": f"{kind} bf16 x 4 (nominal MXFP4 : bf16 ratio)",
            "frac_of_mxfp4_peak": flops / (ms * 1e-3) / 1e12 / fp4_peak,
@@ -736,11 +741,11 @@ def measured_bf16_tflops():
     return 1590.0, "fallback"
 
 
-# DRAM traffic of one indexer call (schedule + scan + both select kernels): the read +
-# write bytes that one ncu capture of the call at 8 requests of the same workload
+# DRAM traffic of one indexer call (scan with its own schedule, then the merge): the
+# read + write bytes that one ncu capture of the call at 8 requests of the same workload
 # counted, and the key bytes of that call; scaled to this run by key bytes. Valid only
 # for the indexer source it was taken on (hash below); otherwise reported as null.
-INDEX_TRAFFIC_CAPTURE = {"bytes": 217488128 + 122112, "key_bytes": 210.427904e6, "source_hash": "1519eeab27c963c7"}
+INDEX_TRAFFIC_CAPTURE = {"bytes": 210.501e6 + 0.458e6 + 1.374e6, "key_bytes": 210.427904e6, "source_hash": "7cd6df3edac262c6"}
 
 
 def index_traffic(key_bytes: float):
@@ -811,10 +816,13 @@ def main():
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the csa_tiny_4k / csa_b8_64k / hca_b64_1m measurements")
     ap.add_argument("--batch", type=int, default=B, help="requests per GPU (default 32; smaller only for profiling)")
+    ap.add_argument("--prefill-requests", type=int, default=Prefill.B,
+                    help="requests of the prefill workload (default 4; fewer only for profiling)")
     ap.add_argument("--scale-fmt", default="e8m0x32", choices=sorted(SCALE_FMT_NAMES),
                     help="FP4 scale format of both caches (default: E8M0 per 32 elements, MXFP4)")
     args = ap.parse_args()
     set_batch(args.batch)
+    set_prefill_requests(args.prefill_requests)
     set_scale_fmt(args.scale_fmt)
     if args.impl == "reference":
         return run_reference(args)
