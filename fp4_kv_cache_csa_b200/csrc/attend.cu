@@ -58,14 +58,14 @@ constexpr int kSchedSmemQueries = 1024;  // the schedule searches its prefixes i
 constexpr int kMaxAttendCtas = 256;      // ... and the CTA ranges up to this many CTAs
 constexpr int kHeads = 64;
 constexpr int kThreads = 256;
-// Relative cost of the work the CTAs share out (measured per-CTA times on B200 at
-// D = 512: a compressed tile ~6.2 us, a window tile ~11.5 us -- bf16 rows 4x the
-// bytes, copied and converted in place -- and each query a CTA starts ~7 us: its
-// Q' copy, the final PV wait, the output or partial write). The flat tile list is
-// cut into equal shares of these units, not of tiles.
+// Relative cost of the work the CTAs share out (global-timer traces of every CTA on
+// B200 at D = 512: a compressed tile ~5.2-6.3 us, a window tile ~12.4 us -- bf16 rows
+// 4x the bytes, copied and converted in place -- and each query a CTA starts ~10 us:
+// its Q' copy, the first tile's cold loads, the final PV wait, the output or partial
+// write). The flat tile list is cut into equal shares of these units, not of tiles.
 constexpr long long kCTileCost = 100;
-constexpr long long kWTileCost = 185;
-constexpr long long kStartCost = 110;
+constexpr long long kWTileCost = 220;
+constexpr long long kStartCost = 170;
 
 template <int D>
 struct Cfg {
@@ -532,9 +532,9 @@ __global__ void __launch_bounds__(1024) attend_schedule_kernel(
             const long long ct = r.a.z, nt = r.t.y - r.t.x;
             const long long x = ub - upre[lo] - kStartCost;  // units into the query's tiles
             long long before = 0;                               // its tiles starting before ub
-            if (x > 0) {
-                if (x <= ct * kCTileCost) before = (x + kCTileCost - 1) / kCTileCost;
-                else before = ct + (x - ct * kCTileCost + kWTileCost - 1) / kWTileCost;
+            if (x > 0) {  // the tile boundary nearest to ub (halves the overshoot of a CTA's share)
+                if (x <= ct * kCTileCost) before = (x + kCTileCost / 2) / kCTileCost;
+                else before = ct + (x - ct * kCTileCost + kWTileCost / 2) / kWTileCost;
             }
             tb = r.t.x + min(before, nt);
         }
