@@ -795,15 +795,17 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a) {
 }
 
 // ---------------------------------------------------------------- merge (streamed decode)
-// One CTA per query: the exact top-k among the candidates the scan CTAs left
-// for it (their segments in CTA order, each in index order, so the candidates
-// are in ascending block index), by three radix levels on the key bits
-// (31..20, 19..8, 7..0) until the k-th largest key T is fixed; then the keys
-// above T and the first ties at T (lowest indices: the candidates' order) are
-// written in that order. Up to kMergeStage candidates are staged in shared
-// memory; more (few long queries spread over many CTAs) are read in place.
+// One or two CTAs (a cluster) per query: the exact top-k among the candidates the scan
+// CTAs left for it (their segments in CTA order, each in index order, so the
+// candidates are in ascending block index), by three radix levels on the key bits
+// (31..20, 19..8, 7..0) until the k-th largest key T is fixed; then the keys above
+// T and the first ties at T (lowest indices: the candidates' order) are written in
+// that order. With two CTAs each takes one half of the candidates; up to kMergeStage per CTA
+// are staged in shared memory; more (few long queries spread over many CTAs) are
+// read in place.
 constexpr int kMergeThreads = 1024;
-constexpr int kMergeStage = 24576;  // 192 KB of shared memory
+constexpr int kMergeTwoMinQueries = 16;  // fewest queries for two CTAs (a cluster) per query
+constexpr int kMergeStage = 20480;  // candidates staged per CTA: 160 KB of shared memory
 constexpr uint32_t kTakeAll = 0xFFFFFFFFu;
 
 struct MergeArgs {
@@ -819,6 +821,7 @@ struct MergeArgs {
     const int32_t *pool;
     int pool_shift, pool_p;
     int layers;  // query i maps to pool row i / layers
+    int ctas;    // CTAs per query: 2 (a cluster, each with half the candidates) or 1
 };
 
 // Largest bin d of a histogram of nbins (a multiple of 32, at most 4096) bins
@@ -877,23 +880,62 @@ __device__ __forceinline__ uint32_t merge_row_pos(const uint32_t *pre, const uin
     return off[lo] + (p - pre[lo]);
 }
 
+// With two CTAs (a cluster) per query, CTA r stages and ranks candidates
+// [r L/2, (r+1) L/2) of the query's candidate list; at every radix level the two
+// histograms are summed through distributed shared memory, so both CTAs pick the
+// same digit; CTA 1's outputs follow CTA 0's (candidate order = ascending block).
+__device__ __forceinline__ uint32_t merge_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t ld_peer(const uint32_t *local, uint32_t peer) {
+    uint32_t addr, v;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
+                 : "=r"(addr)
+                 : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(local))), "r"(peer));
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+// Barrier over every thread of both CTAs (release / acquire at cluster scope). Both CTAs
+// of a query take the same path through the kernel, so each reaches every one of these.
+__device__ __forceinline__ void merge_cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// The histogram both CTAs pick from: hs = this CTA's + the peer's (first nb bins); the
+// peer reads h meanwhile, so nothing writes h again before the second barrier. One CTA
+// per query: h itself (complete after the caller's barrier).
+__device__ __forceinline__ const uint32_t *merge_sum_hist(const uint32_t *h, uint32_t *hs, int nb, uint32_t peer,
+                                                          bool two) {
+    if (!two) return h;
+    merge_cluster_sync();
+    for (int k = threadIdx.x; k < nb; k += kMergeThreads) hs[k] = h[k] + ld_peer(h + k, peer);
+    merge_cluster_sync();
+    return hs;
+}
+
 __global__ void __launch_bounds__(kMergeThreads) select_merge_kernel(MergeArgs a) {
     extern __shared__ uint32_t mdyn[];  // [kMergeStage] keys, then [kMergeStage] indices
     uint32_t *sk = mdyn;
     int32_t *sj = reinterpret_cast<int32_t *>(mdyn + kMergeStage);
-    __shared__ __align__(16) uint32_t h[kBins];
+    __shared__ __align__(16) uint32_t h[kBins];   // this CTA's histogram
+    __shared__ __align__(16) uint32_t hs[kBins];  // both CTAs' histograms
     __shared__ uint32_t scan_smem[32];
     __shared__ BinPick pick;
     __shared__ uint32_t s_pre[kMaxScanCtas + 1];  // candidates before each of the query's CTAs
     __shared__ uint32_t s_off[kMaxScanCtas];      // where that CTA's candidates start in the row
+    __shared__ uint32_t s_outs, s_ties;           // outputs written / ties met by this CTA (for CTA 1)
     grid_dep_wait();
-    const int i = blockIdx.x, tid = threadIdx.x;
+    const bool two = a.ctas == 2;
+    const uint32_t rank = two ? merge_rank() : 0u, peer = rank ^ 1u;
+    const int i = blockIdx.x / a.ctas, tid = threadIdx.x;
     // the query's schedule values, loaded together (one round trip to L2)
     const int n = a.n_vis[i];
     const long long NG = a.gprefix[a.Nq], u0 = a.gprefix[i], u1 = a.gprefix[i + 1];
     const int K = min(a.topk, n);
     int32_t *out = a.sel_idx + (size_t)i * a.topk;
-    if (K == n) {  // every visible block (or none)
+    if (K == n) {  // every visible block (or none); the same branch in both CTAs
+        if (rank != 0) return;
         if (a.pool) {
             for (int r = tid; r < a.topk; r += kMergeThreads) out[r] = r < n ? merge_pool_index(a, i, r) : -1;
         } else {
@@ -922,22 +964,25 @@ __global__ void __launch_bounds__(kMergeThreads) select_merge_kernel(MergeArgs a
         s_pre[tid] = pre;
         s_off[tid] = off;
     }
+    const uint32_t half = two ? (L + 1) / 2 : L;
+    const uint32_t pb = rank ? half : 0u, pe = rank ? L : half;  // this CTA's candidates
+    const uint32_t Lr = pe - pb;
     const uint32_t *gk = a.seg_key + (size_t)i * a.rows;
     const int32_t *gj = a.seg_idx + (size_t)i * a.rows;
-    const bool staged = L <= (uint32_t)kMergeStage;
+    const bool staged = half <= (uint32_t)kMergeStage;  // the same in both CTAs
     for (int k = tid; k < kBins; k += kMergeThreads) h[k] = 0u;
     __syncthreads();
     // ---- level 0 (and the staging copy: every load of the thread in flight at once)
     if (staged) {
         constexpr int kPer = 12;  // loads in flight per thread and round
-        for (uint32_t p0 = 0; p0 < L; p0 += kPer * kMergeThreads) {
+        for (uint32_t p0 = 0; p0 < Lr; p0 += kPer * kMergeThreads) {
             uint32_t kk[kPer];
             int32_t jj[kPer];
 #pragma unroll
             for (int k = 0; k < kPer; ++k) {
                 const uint32_t p = p0 + tid + k * kMergeThreads;
-                if (p < L) {
-                    const uint32_t rp = merge_row_pos(s_pre, s_off, nseg, p);
+                if (p < Lr) {
+                    const uint32_t rp = merge_row_pos(s_pre, s_off, nseg, pb + p);
                     kk[k] = __ldcg(gk + rp);
                     jj[k] = __ldcg(gj + rp);
                 }
@@ -945,7 +990,7 @@ __global__ void __launch_bounds__(kMergeThreads) select_merge_kernel(MergeArgs a
 #pragma unroll
             for (int k = 0; k < kPer; ++k) {
                 const uint32_t p = p0 + tid + k * kMergeThreads;
-                if (p < L) {
+                if (p < Lr) {
                     sk[p] = kk[k];
                     sj[p] = jj[k];
                     atomicAdd(&h[kk[k] >> 20], 1u);
@@ -953,11 +998,11 @@ __global__ void __launch_bounds__(kMergeThreads) select_merge_kernel(MergeArgs a
             }
         }
     } else {
-        for (uint32_t p = tid; p < L; p += kMergeThreads)
+        for (uint32_t p = pb + tid; p < pe; p += kMergeThreads)
             atomicAdd(&h[__ldcg(gk + merge_row_pos(s_pre, s_off, nseg, p)) >> 20], 1u);
     }
     __syncthreads();
-    BinPick pk = pick_bin(h, kBins, (uint32_t)K, scan_smem, &pick);
+    BinPick pk = pick_bin(merge_sum_hist(h, hs, kBins, peer, two), kBins, (uint32_t)K, scan_smem, &pick);
     uint32_t T, take;
     if (pk.above + pk.at == (uint32_t)K) {  // the whole bin
         T = (uint32_t)pk.bin << 20;
@@ -967,13 +1012,13 @@ __global__ void __launch_bounds__(kMergeThreads) select_merge_kernel(MergeArgs a
         uint32_t need = (uint32_t)K - pk.above;
         for (int k = tid; k < kBins; k += kMergeThreads) h[k] = 0u;
         __syncthreads();
-        for (uint32_t p = tid; p < L; p += kMergeThreads) {
+        for (uint32_t p = pb + tid; p < pe; p += kMergeThreads) {
             uint32_t key;
-            if (staged) key = sk[p]; else key = __ldcg(gk + merge_row_pos(s_pre, s_off, nseg, p));
+            if (staged) key = sk[p - pb]; else key = __ldcg(gk + merge_row_pos(s_pre, s_off, nseg, p));
             if ((key >> 20) == b0) atomicAdd(&h[(key >> 8) & 0xFFFu], 1u);
         }
         __syncthreads();
-        pk = pick_bin(h, kBins, need, scan_smem, &pick);
+        pk = pick_bin(merge_sum_hist(h, hs, kBins, peer, two), kBins, need, scan_smem, &pick);
         const uint32_t pre1 = (b0 << 12) | (uint32_t)pk.bin;
         if (pk.above + pk.at == need) {
             T = pre1 << 8;
@@ -982,26 +1027,27 @@ __global__ void __launch_bounds__(kMergeThreads) select_merge_kernel(MergeArgs a
             need -= pk.above;
             for (int k = tid; k < 256; k += kMergeThreads) h[k] = 0u;
             __syncthreads();
-            for (uint32_t p = tid; p < L; p += kMergeThreads) {
+            for (uint32_t p = pb + tid; p < pe; p += kMergeThreads) {
                 uint32_t key;
-                if (staged) key = sk[p]; else key = __ldcg(gk + merge_row_pos(s_pre, s_off, nseg, p));
+                if (staged) key = sk[p - pb]; else key = __ldcg(gk + merge_row_pos(s_pre, s_off, nseg, p));
                 if ((key >> 8) == pre1) atomicAdd(&h[key & 0xFFu], 1u);
             }
             __syncthreads();
-            pk = pick_bin_warp(h, 256, need, &pick);
+            pk = pick_bin_warp(merge_sum_hist(h, hs, 256, peer, two), 256, need, &pick);
             T = (pre1 << 8) | (uint32_t)pk.bin;
             take = need - pk.above;  // ties at T to keep, lowest indices first (>= 1)
         }
     }
-    // ---- output in candidate order: keys above T, and the first `take` keys equal to T
+    // ---- output in candidate order: keys above T, and the first `take` keys equal to T;
+    // CTA 1 starts after CTA 0's outputs and counts its ties after CTA 0's
     if (staged) {
         // warp w owns a contiguous run of the staged candidates: it counts its keys above T
         // and at T, every warp learns the counts of the runs before its own, and each warp
         // writes its selection at its offset (ballots, no block-wide scan per chunk)
         __shared__ uint32_t w_gt[kMergeThreads / 32], w_eq[kMergeThreads / 32];
         const int warp = tid >> 5, lane = tid & 31;
-        const uint32_t seg = (((L + 31) >> 5) + 31) & ~31u;
-        const uint32_t w0 = min(L, warp * seg), w1 = min(L, w0 + seg);
+        const uint32_t seg = (((Lr + 31) >> 5) + 31) & ~31u;
+        const uint32_t w0 = min(Lr, warp * seg), w1 = min(Lr, w0 + seg);
         uint32_t ngt = 0, neq = 0;
         for (uint32_t base = w0; base < w1; base += 32) {
             const uint32_t p = base + lane;
@@ -1025,7 +1071,12 @@ __global__ void __launch_bounds__(kMergeThreads) select_merge_kernel(MergeArgs a
                 const uint32_t y = __shfl_up_sync(0xffffffffu, te, o);
                 if (lane >= o) te += y;
             }
-            const uint32_t tbl = te - e;  // ties before run `lane`
+            // this CTA's totals (lane 31 holds them) for CTA 1; CTA 1 adds CTA 0's
+            if (rank == 0 && tid == 31) s_ties = te;
+            uint32_t tb0 = 0, ob0 = 0;
+            if (two) merge_cluster_sync();  // (every thread of both CTAs) s_ties of CTA 0 is written
+            if (rank == 1) tb0 = ld_peer(&s_ties, peer);
+            const uint32_t tbl = tb0 + te - e;  // ties before run `lane`
             uint32_t outl = gt + (take == kTakeAll ? e : (tbl >= take ? 0u : min(e, take - tbl)));
             uint32_t to = outl;
 #pragma unroll
@@ -1033,9 +1084,13 @@ __global__ void __launch_bounds__(kMergeThreads) select_merge_kernel(MergeArgs a
                 const uint32_t y = __shfl_up_sync(0xffffffffu, to, o);
                 if (lane >= o) to += y;
             }
-            ob = __shfl_sync(0xffffffffu, to - outl, warp);
+            if (rank == 0 && tid == 31) s_outs = to;
+            if (two) merge_cluster_sync();  // s_outs of CTA 0 is written; CTA 1 has read s_ties
+            if (rank == 1) ob0 = ld_peer(&s_outs, peer);
+            ob = ob0 + __shfl_sync(0xffffffffu, to - outl, warp);
             tb = __shfl_sync(0xffffffffu, tbl, warp);
         }
+        if (two) merge_cluster_sync();  // CTA 1 has read s_outs before CTA 0 may leave
         const uint32_t lt = (1u << lane) - 1u;
         for (uint32_t base = w0; base < w1; base += 32) {
             const uint32_t p = base + lane;
@@ -1055,16 +1110,23 @@ __global__ void __launch_bounds__(kMergeThreads) select_merge_kernel(MergeArgs a
             tb += __popc(em);
         }
     } else {
-        constexpr int kE = 4;
+        // CTA 0 writes its outputs first; CTA 1 waits for its counts, then writes after them
         uint32_t obase = 0, tbase = 0;
-        for (uint32_t c0 = 0; c0 < L; c0 += kMergeThreads * kE) {
+        if (rank == 1) {  // (only with two CTAs per query)
+            merge_cluster_sync();  // CTA 0 has published its counts
+            obase = ld_peer(&s_outs, peer);
+            tbase = ld_peer(&s_ties, peer);
+            merge_cluster_sync();  // ... and read before CTA 0 may leave
+        }
+        constexpr int kE = 4;
+        for (uint32_t c0 = pb; c0 < pe; c0 += kMergeThreads * kE) {
             uint32_t key[kE];
             uint32_t gt = 0, eq = 0;
 #pragma unroll
             for (int e = 0; e < kE; ++e) {
                 const uint32_t p = c0 + tid * kE + e;
                 key[e] = 0u;
-                if (p < L) {
+                if (p < pe) {
                     key[e] = __ldcg(gk + merge_row_pos(s_pre, s_off, nseg, p));
                     if (key[e] > T) gt |= 1u << e;
                     if (key[e] == T) eq |= 1u << e;
@@ -1092,10 +1154,19 @@ __global__ void __launch_bounds__(kMergeThreads) select_merge_kernel(MergeArgs a
                     ++pos;
                 }
             obase += chosen;
-            tbase += ties;
+            tbase += ties;  // (counted only when ties are ranked: all that CTA 1 needs then)
+        }
+        if (rank == 0 && two) {
+            if (tid == 0) {
+                s_outs = obase;
+                s_ties = tbase;
+            }
+            merge_cluster_sync();  // published
+            merge_cluster_sync();  // CTA 1 has read them
         }
     }
-    for (int r = K + tid; r < a.topk; r += kMergeThreads) out[r] = -1;
+    if (rank == 0)
+        for (int r = K + tid; r < a.topk; r += kMergeThreads) out[r] = -1;
 }
 
 // ---------------------------------------------------------------- prefill threshold
@@ -1990,10 +2061,28 @@ cudaError_t index_pipeline(const csa_cache &c, const void *q_idx, const float *w
     ma.pool_shift = pool_shift;
     ma.pool_p = pool_p;
     ma.layers = layers;
+    // two CTAs per query when they fit in one wave and the call is a plain decode one with
+    // enough queries (measured at 32 requests x 512K-1M: index stage 0.187 -> 0.185 ms; one
+    // query, 8 queries and 96 Reindex queries ran faster on one CTA each)
+    ma.ctas = (!pool && Nq >= kMergeTwoMinQueries && 2 * Nq <= num_sms) ? 2 : 1;
     const int msmem = 8 * kMergeStage;
     err = cudaFuncSetAttribute(select_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem);
     if (err != cudaSuccess) return err;
-    return launch_pdl(select_merge_kernel, dim3(Nq), dim3(kMergeThreads), (size_t)msmem, s, ma);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(ma.ctas * Nq);
+    cfg.blockDim = dim3(kMergeThreads);
+    cfg.dynamicSmemBytes = (size_t)msmem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = ma.ctas;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = ma.ctas == 2 ? attr : attr + 1;  // one CTA per query: no cluster
+    cfg.numAttrs = ma.ctas == 2 ? 2 : 1;
+    return cudaLaunchKernelEx(&cfg, select_merge_kernel, ma);
 }
 
 }  // namespace
