@@ -745,7 +745,7 @@ def measured_bf16_tflops():
 # read + write bytes that one ncu capture of the call at 8 requests of the same workload
 # counted, and the key bytes of that call; scaled to this run by key bytes. Valid only
 # for the indexer source it was taken on (hash below); otherwise reported as null.
-INDEX_TRAFFIC_CAPTURE = {"bytes": 210.501e6 + 0.458e6 + 1.374e6, "key_bytes": 210.427904e6, "source_hash": "7cd6df3edac262c6"}
+INDEX_TRAFFIC_CAPTURE = {"bytes": 210.507e6 + 0.442e6 + 1.329e6, "key_bytes": 210.427904e6, "source_hash": "b4b338c7134dd890"}
 
 
 def index_traffic(key_bytes: float):
