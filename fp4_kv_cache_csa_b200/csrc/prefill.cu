@@ -83,6 +83,8 @@ struct PfCfg {
     static constexpr uint32_t SBO = 8 * REG_ROW;
     static_assert(STAGES >= 2, "key ring needs two stages");
     static_assert(!MX || DI == 128, "MXFP4 GEMM path: d_I = 128");
+    static_assert(!MX || (NACC * kPfCols <= SFA_COL && SFA_COL + 16 * NACC <= SFB_COL && SFB_COL + 4 <= TMEM_COLS),
+                  "accumulator and scale-factor columns overlap");
     static_assert(MX || NACC * kPfCols <= TMEM_COLS, "accumulators exceed tensor memory");
 };
 

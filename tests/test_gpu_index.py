@@ -93,6 +93,23 @@ def test_candidate_overflow_path():
         run(keys, [65536], qo, qp, 4, 64, k, 0, seed=30)
 
 
+@pytest.mark.parametrize("idx_dtype", [0, 1])
+def test_two_ctas_per_query_merge(idx_dtype):
+    # 24 decode queries (one per request) take the merge on two CTAs (a cluster) per
+    # query, each ranking half of the candidates: ragged contexts, one query with fewer
+    # visible blocks than k, and one whose keys are all equal (every score ties, so the
+    # k lowest indices win across the two halves)
+    lengths = [2000 + 613 * b for b in range(24)]
+    lengths[3] = 100
+    cap = max(lengths)
+    keys = gen_keys(24, cap, 128, idx_dtype, 40)
+    keys[7, :] = keys[7, 0]
+    qo, qp = decode_layout(lengths)
+    sel, _, n_vis = run(keys, lengths, qo, qp, 4, 128, 512, idx_dtype, seed=41)
+    assert list(sel[3, :100]) == list(range(100)) and np.all(sel[3, 100:] == -1)
+    assert np.array_equal(sel[7], np.arange(512))
+
+
 def test_prefill_queries_are_causal():
     # 2 requests, several queries each at increasing positions (causal at block granularity)
     lengths = [4000, 2500]
