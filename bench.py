@@ -506,6 +506,32 @@ def measure_prefill(device, stream, flush, steps: int = 3):
     return res
 
 
+def measure_mxf4_peak(device, stream, iters: int = 4000, reps: int = 5):
+    """Dense TFLOP/s of the block-scaled MXFP4 MMA (kind::mxf4, M 128 x N 256 x K 64) issued
+    back to back on every SM from resident tiles (the library's MMA probe), best of `reps`;
+    (None, reason) if the probe reports a timeout."""
+    import torch
+
+    import fp4_kv_cache_csa_b200 as csa
+
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    best = None
+    with torch.cuda.stream(stream):
+        flops = csa.csa_probe_mxf4_mma(iters // 4, status, stream)  # warm-up
+        for _ in range(reps):
+            a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a_.record(stream)
+            flops = csa.csa_probe_mxf4_mma(iters, status, stream)
+            b_.record(stream)
+            b_.synchronize()
+            t = flops / (a_.elapsed_time(b_) * 1e-3) / 1e12
+            best = t if best is None else max(best, t)
+    stream.synchronize()
+    if int(status.item()) != 0:
+        return None, "probe timeout"
+    return best, "measured (block-scaled MMA probe, every SM, resident tiles)"
+
+
 def measure_prefill_index_mxfp4(device, stream, flush, steps: int = 3):
     """The prefill_b4_8k indexer stage with MXFP4 indexer keys: the block-scaled tensor-core
     GEMM (kind::mxf4) writes the score rows, then the same selection as with bf16 keys."""
@@ -529,12 +555,14 @@ def measure_prefill_index_mxfp4(device, stream, flush, steps: int = 3):
     stream.synchronize()
     ms = float(np.mean([e[0].elapsed_time(e[1]) for e in ev]))
     status = csa.csa_read_device_status(pf.cache, stream)
-    bf16_peak, kind = measured_bf16_tflops()
-    fp4_peak = 4.0 * bf16_peak  # dense MXFP4 : bf16 = 9 : 2.25 PFLOP/s nominal
+    fp4_peak, kind = measure_mxf4_peak(device, stream)
+    if fp4_peak is None:  # fall back to the measured bf16 peak x the nominal ratio
+        bf16_peak, bkind = measured_bf16_tflops()
+        fp4_peak, kind = 4.0 * bf16_peak, f"{bkind} bf16 x 4 (nominal MXFP4 : bf16 ratio; {kind})"
     flops = pf.index_flops()
     res = {"workload": f"prefill_b{pf.B}_8k", "idx_dtype": "mxfp4", "queries": pf.Nq, "index_ms": ms,
            "index_gflop": flops / 1e9, "index_tflops": flops / (ms * 1e-3) / 1e12,
-           "mxfp4_peak_tflops": fp4_peak, "peak_kind": f"{kind} bf16 x 4 (nominal MXFP4 : bf16 ratio)",
+           "mxfp4_peak_tflops": fp4_peak, "peak_kind": kind,
            "frac_of_mxfp4_peak": flops / (ms * 1e-3) / 1e12 / fp4_peak,
            "score_bytes": 4.0 * pf.index_flops() / (H_I * D_I * 2), "device_status": int(status)}
     del pf

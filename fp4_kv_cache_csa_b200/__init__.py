@@ -38,6 +38,7 @@ EXPORTED = (
     "csa_attend_workspace", "csa_decode_attend", "hca_decode_attend", "csa_read_device_status",
     "csa_index_topk_noalloc", "csa_index_pool_workspace", "csa_index_topk_pool", "csa_index_reindex_workspace",
     "csa_index_topk_reindex", "csa_index_reindex_layers_workspace", "csa_index_topk_reindex_layers",
+    "csa_probe_mxf4_mma",
 )
 
 
@@ -105,6 +106,8 @@ def declare(lib):
     lib.hca_decode_attend.restype = I
     lib.csa_read_device_status.argtypes = [CP, P, ctypes.POINTER(I)]
     lib.csa_read_device_status.restype = I
+    lib.csa_probe_mxf4_mma.argtypes = [I, P, P, ctypes.POINTER(ctypes.c_int64)]
+    lib.csa_probe_mxf4_mma.restype = I
     return lib
 
 
@@ -364,6 +367,15 @@ def hca_decode_attend(cache: Cache, q, q_offsets, q_pos, win_kv=None, win_start=
                                  _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(), _stream(stream)),
            "hca_decode_attend")
     return out
+
+
+def csa_probe_mxf4_mma(iters: int, status, stream=None) -> int:
+    """Launch the block-scaled MXFP4 MMA probe (one CTA per SM); returns its dense FLOPs.
+    `status` is a device int32 tensor that receives CSA_DEV_TIMEOUT if completion is not seen."""
+    lib = load_library()
+    flops = ctypes.c_int64(0)
+    _check(lib.csa_probe_mxf4_mma(int(iters), _ptr(status), _stream(stream), ctypes.byref(flops)), "csa_probe_mxf4_mma")
+    return int(flops.value)
 
 
 def csa_read_device_status(cache: Cache, stream=None) -> int:

@@ -24,6 +24,7 @@ cudaError_t launch_index_topk_reindex(const csa_cache &c, const void *q_idx, con
                                       int pool_shift, int P, const int32_t *pool_blk, void *workspace, int num_sms,
                                       cudaStream_t s, int layers);
 size_t attend_workspace_bytes(int Nq, int D, int num_ctas);
+cudaError_t launch_mxf4_probe(int iters, int32_t *status, int num_sms, cudaStream_t s);
 cudaError_t launch_attend(const csa_cache &c, const void *q, int Nq, int H, const int32_t *q_offsets,
                           const int32_t *q_pos, const int32_t *sel_idx, int topk, const void *win_kv,
                           const int64_t *win_start, const int32_t *win_len, int max_win, float softmax_scale,
@@ -293,6 +294,16 @@ csa_status csa_read_device_status(const csa_cache *cache, csa_stream_t stream, i
     if (cudaMemcpy(cache->status, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return CSA_ERR_CUDA;
     *out_flags = v;
     return CSA_OK;
+}
+
+csa_status csa_probe_mxf4_mma(int32_t iters, int32_t *status, csa_stream_t stream, int64_t *flops) {
+    if (!status || !flops) return CSA_ERR_NULL;
+    if (iters < 1) return CSA_ERR_SHAPE;
+    if (!aligned(status, 4)) return CSA_ERR_ALIGN;
+    const int sms = num_sms();
+    if (sms <= 0) return CSA_ERR_CUDA;
+    *flops = (int64_t)sms * iters * 2 * 128 * 256 * 128;
+    return from_cuda(csa::launch_mxf4_probe(iters, status, sms, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

@@ -461,6 +461,67 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_score_kernel(const __gr
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TMEM_COLS) : "memory");
 }
 
+// Issue rate of the block-scaled MMA used above: one CTA per SM issues `iters`
+// pairs of kind::mxf4 MMAs (M = 128, N = 256, K = 64 each) from resident shared-memory
+// tiles (non-zero codes of alternating sign, so that every product toggles the
+// datapath; unit scales) into one TMEM accumulator, with the same descriptor and
+// scale-factor layout as the score GEMM. No data moves, so the time measures the
+// tensor pipe alone; FLOPs = 2 * 128 * 256 * 128 * iters per CTA.
+constexpr int kProbeN = 256;
+__global__ void __launch_bounds__(128, 1) mxf4_probe_kernel(int iters, int32_t *status) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *As = smem;                      // 128 rows x 64 B (K = 128 codes), 64-byte swizzle
+    uint8_t *Bs = As + 128 * 64;             // 256 rows x 64 B
+    uint8_t *SFa = Bs + kProbeN * 64;        // one scale-factor block (128 rows)
+    uint8_t *SFb = SFa + 1024;               // two (256 rows)
+    uint64_t *mb = reinterpret_cast<uint64_t *>(SFb + 2048);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mb + 1);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    for (int k = tid; k < (128 + kProbeN) * 64 / 16; k += blockDim.x)  // codes +1.5, -3, +6, -0.5, ...
+        reinterpret_cast<uint4 *>(As)[k] = make_uint4(0xD37A9E15u, 0x6B2C5F91u, 0xA4E3172Du, 0x39C8B6F4u);
+    for (int k = tid; k < 3 * 1024 / 4; k += blockDim.x) reinterpret_cast<uint32_t *>(SFa)[k] = 0x7F7F7F7Fu;
+    if (tid == 0) {
+        mbar_init(smem_u32(mb), 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(512u)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    if (tid == 0) {
+        const uint32_t sfa = tmem + 256, sfb = tmem + 272;  // accumulator in columns 0..255
+        sf_copy(sfa, smem_u32(SFa));
+        sf_copy(sfb, smem_u32(SFb));
+        sf_copy(sfb + 4, smem_u32(SFb + 512));
+        const uint32_t A_s = smem_u32(As), B_s = smem_u32(Bs);
+        for (int it = 0; it < iters; ++it) {
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const uint64_t da = desc_smem(A_s + 32 * k, 16, 512, 4u);
+                const uint64_t db = desc_smem(B_s + 32 * k, 16, 512, 4u);
+                const uint32_t id = (uint32_t)(2 * k);
+                mma_mxf4(tmem, da, db, idesc_mxf4(128, kProbeN, id, id), (it | k) != 0, sfa | (id << 30),
+                         sfb | (id << 30));
+            }
+        }
+        mma_commit(smem_u32(mb));
+        if (!mbar_wait(smem_u32(mb), 0)) flag(status, CSA_DEV_TIMEOUT);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512u) : "memory");
+}
+
 // cuTensorMapEncodeTiled from the driver, looked up once.
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -575,6 +636,15 @@ cudaError_t launch_prefill_scores(const csa_cache &c, const void *q_idx, const f
         case 256: return launch_pf_heads<kPfBf16, 256>(a, H_I, c.idx_key, c.batch, q_idx, num_sms, s);
         default: return cudaErrorInvalidValue;
     }
+}
+
+// The MMA probe on every SM; FLOPs per launch = num_sms * iters * 2 * 128 * 256 * 128.
+cudaError_t launch_mxf4_probe(int iters, int32_t *status, int num_sms, cudaStream_t s) {
+    const int smem = 1024 + 128 * 64 + kProbeN * 64 + 1024 + 2048 + 64;
+    cudaError_t err = cudaFuncSetAttribute(mxf4_probe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err != cudaSuccess) return err;
+    mxf4_probe_kernel<<<num_sms, 128, smem, s>>>(iters, status);
+    return cudaGetLastError();
 }
 
 }  // namespace csa

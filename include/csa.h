@@ -337,6 +337,21 @@ csa_status hca_decode_attend(const csa_cache *cache, const void *q, int32_t n_qu
  */
 csa_status csa_read_device_status(const csa_cache *cache, csa_stream_t stream, int32_t *out_flags);
 
+/*
+ * Measurement helper with no counterpart on the pages: the issue rate of the
+ * block-scaled MXFP4 tensor-core MMA that the prefill indexer GEMM uses
+ * (tcgen05.mma kind::mxf4, M = 128, N = 256, K = 64, E8M0 scales per 32), so
+ * that the GEMM can be reported against a measured MXFP4 peak. One CTA per SM
+ * issues `iters` pairs of MMAs from resident shared-memory tiles into tensor
+ * memory; no global data moves. *flops receives the dense FLOPs of the launch
+ * (SMs x iters x 2 x 128 x 256 x 128); time the call with events on `stream`.
+ * `status`: a device int32 word (4-byte aligned) that receives CSA_DEV_TIMEOUT
+ * if the MMAs' completion is not seen (read it with cudaMemcpy or the caller's
+ * own means). Errors: CSA_ERR_NULL (status or flops NULL), CSA_ERR_SHAPE
+ * (iters < 1), CSA_ERR_ALIGN, CSA_ERR_CUDA (launch failure).
+ */
+csa_status csa_probe_mxf4_mma(int32_t iters, int32_t *status, csa_stream_t stream, int64_t *flops);
+
 #ifdef __cplusplus
 }
 #endif

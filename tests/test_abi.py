@@ -187,3 +187,12 @@ def test_cache_struct_layout_matches_the_header(tmp_path):
     got = [int(x) for x in subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()]
     want = [getattr(csa._CCache, f).offset for f in fields] + [ctypes.sizeof(csa._CCache)]
     assert got == want
+
+
+def test_mxf4_probe_argument_checks(lib):
+    # the MMA probe validates on the host before touching the device
+    flops = ctypes.c_int64(0)
+    assert lib.csa_probe_mxf4_mma(10, None, None, ctypes.byref(flops)) == ERR_NULL
+    assert lib.csa_probe_mxf4_mma(10, ctypes.c_void_p(256), None, None) == ERR_NULL
+    assert lib.csa_probe_mxf4_mma(0, ctypes.c_void_p(256), None, ctypes.byref(flops)) == ERR_SHAPE
+    assert lib.csa_probe_mxf4_mma(10, ctypes.c_void_p(258), None, ctypes.byref(flops)) == ERR_ALIGN

@@ -237,3 +237,17 @@ def test_more_than_four_heads_is_refused():
     w = dev(datagen.normal_f32((1, 8), 77, 2))
     with pytest.raises(csa.CsaError, match="status 4"):
         csa.csa_index_topk(cache, q, w, dev(qo), dev(qp), 16)
+
+
+def test_mxf4_mma_probe_completes():
+    # the measurement helper behind the MXFP4 peak: block-scaled MMAs on every SM finish
+    # within the wait limit and report the FLOPs they issued
+    import torch
+
+    import fp4_kv_cache_csa_b200 as csa
+
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    flops = csa.csa_probe_mxf4_mma(64, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert flops == torch.cuda.get_device_properties(0).multi_processor_count * 64 * 2 * 128 * 256 * 128
