@@ -513,7 +513,10 @@ __global__ void __launch_bounds__(128, 1) mxf4_probe_kernel(int iters, int32_t *
             }
         }
         mma_commit(smem_u32(mb));
-        if (!mbar_wait(smem_u32(mb), 0)) flag(status, CSA_DEV_TIMEOUT);
+        if (!mbar_wait(smem_u32(mb), 0)) {  // flag it, and let the MMAs drain before TMEM is freed
+            flag(status, CSA_DEV_TIMEOUT);
+            mbar_wait_for(smem_u32(mb), 0, kDrainCycles);
+        }
     }
     tc_fence_before();
     __syncthreads();
