@@ -500,7 +500,8 @@ def measure_prefill(device, stream, flush, steps: int = 3):
     res = {"workload": f"prefill_b{pf.B}_8k", "queries": pf.Nq, "ms": float(st.sum()),
            "stage_ms": {"compress": float(st[0]), "index_topk": float(st[1]), "attend": float(st[2])},
            "index_gflop": pf.index_flops() / 1e9,
-           "index_tflops": pf.index_flops() / (st[1] * 1e-3) / 1e12, "device_status": int(status)}
+           "index_tflops": pf.index_flops() / (st[1] * 1e-3) / 1e12,
+           "index_workspace_mb": pf.ws_idx.numel() / 1e6, "device_status": int(status)}
     del pf
     torch.cuda.empty_cache()
     return res
@@ -564,7 +565,8 @@ def measure_prefill_index_mxfp4(device, stream, flush, steps: int = 3):
            "index_gflop": flops / 1e9, "index_tflops": flops / (ms * 1e-3) / 1e12,
            "mxfp4_peak_tflops": fp4_peak, "peak_kind": kind,
            "frac_of_mxfp4_peak": flops / (ms * 1e-3) / 1e12 / fp4_peak,
-           "score_bytes": 4.0 * pf.index_flops() / (H_I * D_I * 2), "device_status": int(status)}
+           "score_bytes": 4.0 * pf.index_flops() / (H_I * D_I * 2), "index_workspace_mb": pf.ws_idx.numel() / 1e6,
+           "device_status": int(status)}
     del pf
     torch.cuda.empty_cache()
     return res
@@ -1058,7 +1060,9 @@ def main():
                       "frac_of_hbm_peak": wl.bytes_csa_layer() / (csa_ms * 1e-3) / 1e9 / peak},
         "roofline": {"bound": "hbm", "kernel": "csa_index_topk (scan + merge)", "achieved": achieved, "peak": peak,
                      "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind,
-                     "traffic": index_traffic(wl.key_bytes()), "traffic_unit": "GB per call (ncu, scaled by keys)"},
+                     "traffic": index_traffic(wl.key_bytes()), "traffic_unit": "GB per call (ncu, scaled by keys)",
+                     "traffic_note": None if index_traffic(wl.key_bytes()) is not None else
+                     "null: the indexer source changed after its last ncu capture; no capture of this source"},
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_n,
                 "overlap": "step k+1 inputs in and step k-1 results out while step k computes",

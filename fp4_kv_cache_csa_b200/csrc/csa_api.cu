@@ -9,10 +9,11 @@
 namespace csa {
 cudaError_t launch_compress(const csa_cache &c, const void *kv_tok, const void *idx_tok, const float *gate_w,
                             const int32_t *tok_offsets, int32_t n_tokens, cudaStream_t s);
-size_t index_topk_workspace_bytes(int Nq, int cap);
+size_t index_topk_workspace_bytes(const csa_cache &c, int Nq);
+size_t index_topk_min_workspace_bytes(const csa_cache &c, int Nq, int H_I);
 cudaError_t launch_index_topk(const csa_cache &c, const void *q_idx, const float *w, int Nq, int H_I,
                               const int32_t *q_offsets, const int32_t *q_pos, int topk, int32_t *sel_idx,
-                              void *workspace, int num_sms, cudaStream_t s);
+                              void *workspace, size_t workspace_bytes, int num_sms, cudaStream_t s);
 size_t index_pool_workspace_bytes(int Nq, int cap, int G, int P);
 cudaError_t launch_index_topk_pool(const csa_cache &c, const void *q_idx, const float *w, int Nq, int H_I,
                                    const int32_t *q_offsets, const int32_t *q_pos, int topk, int32_t *sel_idx,
@@ -125,7 +126,7 @@ csa_status csa_compress_quantize(const csa_cache *cache, const void *kv_tok, con
 
 size_t csa_index_topk_workspace(const csa_cache *cache, int32_t n_queries, int32_t topk) {
     if (!cache || n_queries < 1 || topk < 1 || cache->capacity < 1 || cache->capacity > kMaxCapacity) return 0;
-    return csa::index_topk_workspace_bytes(n_queries, cache->capacity);
+    return csa::index_topk_workspace_bytes(*cache, n_queries);
 }
 
 csa_status csa_index_topk(const csa_cache *cache, const void *q_idx, const float *w, int32_t n_queries,
@@ -134,13 +135,14 @@ csa_status csa_index_topk(const csa_cache *cache, const void *q_idx, const float
     const csa_status st = csa::check_index_args(cache, q_idx, w, n_queries, idx_heads, q_offsets, q_pos, topk,
                                                  sel_idx);
     if (st != CSA_OK) return st;
-    const size_t need = csa::index_topk_workspace_bytes(n_queries, cache->capacity);
+    // one chunk of queries must fit; a larger workspace runs more queries per chunk
+    const size_t need = csa::index_topk_min_workspace_bytes(*cache, n_queries, idx_heads);
     if (!workspace || workspace_bytes < need) return CSA_ERR_WORKSPACE;
     if (!aligned(workspace, 256)) return CSA_ERR_ALIGN;
     const int sms = num_sms();
     if (sms <= 0) return CSA_ERR_CUDA;
     return from_cuda(csa::launch_index_topk(*cache, q_idx, w, n_queries, idx_heads, q_offsets, q_pos, topk, sel_idx,
-                                            workspace, sms, reinterpret_cast<cudaStream_t>(stream)));
+                                            workspace, workspace_bytes, sms, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 // log2 of a pool block size (1, 2, 4, ... 32 entries), or -1

@@ -112,7 +112,10 @@ struct IndexWs {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-size_t carve(void *base, int Nq, int cap, IndexWs *w) {
+// segments: the streamed path's per-segment candidate lists, which also hold the
+// GEMM's quantized query; without them (the GEMM with the pass + final selection)
+// the quantized query gets its own `scratch` bytes at the end.
+size_t carve(void *base, int Nq, int cap, IndexWs *w, bool segments = true, size_t scratch = 0) {
     const int words = (cap + 31) / 32;
     const int ccap = kCandCap;
     size_t off = 0;
@@ -134,9 +137,11 @@ size_t carve(void *base, int Nq, int cap, IndexWs *w) {
     size_t o_ck = take(sizeof(uint32_t) * (size_t)ccap * Nq);
     size_t o_ci = take(sizeof(int32_t) * (size_t)ccap * Nq);
     size_t o_sc = take(sizeof(float) * (size_t)cap * Nq);
-    size_t o_scnt = take(sizeof(int32_t) * ((size_t)Nq + kMaxScanCtas));
-    size_t o_skey = take(sizeof(uint32_t) * (size_t)cap * Nq);
-    size_t o_sidx = take(sizeof(int32_t) * (size_t)cap * Nq);
+    const size_t seg_rows = segments ? (size_t)cap * Nq : 0;
+    size_t o_scnt = take(segments ? sizeof(int32_t) * ((size_t)Nq + kMaxScanCtas) : 0);
+    size_t o_skey = take(sizeof(uint32_t) * seg_rows);
+    size_t o_sidx = take(sizeof(int32_t) * seg_rows);
+    size_t o_q = take(segments ? 0 : scratch);
     if (w) {
         char *b = static_cast<char *>(base);
         w->req = reinterpret_cast<int32_t *>(b + o_req);
@@ -150,16 +155,48 @@ size_t carve(void *base, int Nq, int cap, IndexWs *w) {
         w->cand_key = reinterpret_cast<uint32_t *>(b + o_ck);
         w->cand_idx = reinterpret_cast<int32_t *>(b + o_ci);
         w->scores = reinterpret_cast<float *>(b + o_sc);
-        w->seg_cnt = reinterpret_cast<int32_t *>(b + o_scnt);
-        w->seg_key = reinterpret_cast<uint32_t *>(b + o_skey);
-        w->seg_idx = reinterpret_cast<int32_t *>(b + o_sidx);
+        w->seg_cnt = segments ? reinterpret_cast<int32_t *>(b + o_scnt) : nullptr;
+        w->seg_key = segments ? reinterpret_cast<uint32_t *>(b + o_skey) : nullptr;
+        w->seg_idx = segments ? reinterpret_cast<int32_t *>(b + o_sidx) : nullptr;
         // the per-segment candidate lists are the streamed path's; the GEMM path keeps
-        // its quantized query there instead
-        w->spare = b + o_skey;
-        w->spare_bytes = o_sidx + sizeof(int32_t) * (size_t)cap * Nq - o_skey;
+        // its quantized query there instead, or in its own region
+        w->spare = b + (segments ? o_skey : o_q);
+        w->spare_bytes = segments ? o_sidx + sizeof(int32_t) * seg_rows - o_skey : scratch;
         w->zero_bytes = z1 - z0;
         w->words = words;
         w->ccap = ccap;
+    }
+    return off;
+}
+
+// The GEMM path whose score rows fit the row selection's shared memory needs
+// only the schedule's per-query values, the score rows and the quantized query
+// (`scratch` bytes): no zeroed state, candidate lists or segment buffers.
+size_t carve_rows(void *base, int Nq, int cap, size_t scratch, IndexWs *w) {
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        size_t o = off;
+        off = align256(off + bytes);
+        return o;
+    };
+    size_t o_req = take(sizeof(int32_t) * Nq);
+    size_t o_nvis = take(sizeof(int32_t) * Nq);
+    size_t o_gp = take(sizeof(long long) * (Nq + 1));
+    size_t o_th = take(sizeof(int32_t) * 3 * (size_t)Nq);
+    size_t o_sc = take(sizeof(float) * (size_t)cap * Nq);
+    size_t o_q = take(scratch);
+    if (w) {
+        char *b = static_cast<char *>(base);
+        *w = IndexWs{};
+        w->req = reinterpret_cast<int32_t *>(b + o_req);
+        w->n_vis = reinterpret_cast<int32_t *>(b + o_nvis);
+        w->gprefix = reinterpret_cast<long long *>(b + o_gp);
+        w->thresh = reinterpret_cast<int32_t *>(b + o_th);
+        w->scores = reinterpret_cast<float *>(b + o_sc);
+        w->spare = b + o_q;
+        w->spare_bytes = scratch;
+        w->words = (cap + 31) / 32;
+        w->ccap = kCandCap;
     }
     return off;
 }
@@ -171,7 +208,8 @@ size_t carve(void *base, int Nq, int cap, IndexWs *w) {
 // caller's query i / layers, whose request and position it takes.
 __global__ void schedule_kernel(const int32_t *q_offsets, const int32_t *q_pos, const int32_t *n_blocks,
                                 int batch, int Nq, int m, int cap, int topk, int32_t *req, int32_t *n_vis,
-                                long long *gprefix, int32_t *thresh, const int32_t *n_vis_given, int layers) {
+                                long long *gprefix, int32_t *thresh, const int32_t *n_vis_given, int layers,
+                                int q_base) {
     __shared__ long long red[32];
     __shared__ long long round_total;
     grid_dep_wait();
@@ -181,9 +219,10 @@ __global__ void schedule_kernel(const int32_t *q_offsets, const int32_t *q_pos, 
         const int i = base + threadIdx.x;
         long long groups = 0;
         if (i < Nq) {
-            const int b = request_of(q_offsets, batch, i / layers);
+            const int gi = q_base + i / layers;  // the caller's query index
+            const int b = request_of(q_offsets, batch, gi);
             const int n = n_vis_given ? ((b < 0) ? 0 : n_vis_given[i])
-                                      : ((b < 0) ? 0 : min(visible_blocks(q_pos[i / layers], m, n_blocks[b]), cap));
+                                      : ((b < 0) ? 0 : min(visible_blocks(q_pos[gi], m, n_blocks[b]), cap));
             req[i] = b;
             n_vis[i] = n;
             groups = (n + 15) / 16;
@@ -351,6 +390,7 @@ struct ScanArgs {
     // them for the merge; otherwise schedule_kernel has written req, n_vis, gprefix
     int fused;
     int layers;  // queries per caller query (several Reindex layers in one call), else 1
+    int q_base;  // caller's index of query 0 (a call run in chunks of queries), else 0
     const int32_t *q_offsets, *q_pos, *n_blocks, *n_vis_given;
     int32_t *req_out, *n_vis_out;
     long long *gprefix_out;
@@ -428,10 +468,10 @@ __global__ void __launch_bounds__(kScanThreads, 1) scan_kernel(ScanArgs a) {
         const int i = threadIdx.x;
         long long units = 0;
         if (i < a.Nq) {
-            const int b = request_of(a.q_offsets, a.batch, i / a.layers);
+            const int gi = a.q_base + i / a.layers;
+            const int b = request_of(a.q_offsets, a.batch, gi);
             const int n = a.n_vis_given ? (b < 0 ? 0 : a.n_vis_given[i])
-                                        : (b < 0 ? 0 : min(visible_blocks(a.q_pos[i / a.layers], a.m, a.n_blocks[b]),
-                                                           a.rows));
+                                        : (b < 0 ? 0 : min(visible_blocks(a.q_pos[gi], a.m, a.n_blocks[b]), a.rows));
             s_req[i] = b;
             s_nv[i] = n;
             units = (n + 15) / 16;
@@ -1961,23 +2001,89 @@ cudaError_t launch_select(const SelJob &j0, const SelJob *j1, int num_sms, cudaS
     return launch_pdl(select_final_kernel, dim3(nq), dim3(kSelThreads), (size_t)smem, s, a0, a1);
 }
 
+// ---------------------------------------------------------------- query chunks
+// A call whose workspace for all its queries would exceed what it is given
+// runs its queries in consecutive chunks on the same workspace. Every query is
+// scored and selected on its own, so the results do not depend on the chunks.
+constexpr size_t kIndexWsTarget = size_t(768) << 20;  // what the size query asks for at most (but one chunk)
+constexpr int kChunkQueries = 128;                     // chunks are multiples of this many queries, the last aside
+constexpr int kMaxIdxHeads = 8;
+
+// The call brings many queries per request and its key format has a GEMM kernel.
+bool gemm_call(const csa_cache &c, int Nq, int H_I) {
+    return Nq >= kPrefillQueriesPerRequest * c.batch && prefill_scores_supported(c.idx_dtype, c.idx_dim, H_I);
+}
+
+// A GEMM chunk of the size query holds at least one wave of 32-query tiles (4 heads)
+// on the B200's 148 SMs: fewer tiles leave SMs idle for the whole chunk.
+constexpr int kGemmChunkQueries = 148 * 32;
+
+// Workspace layouts: the full one (streamed path), the GEMM with the pass + final
+// selection (no segment buffers), the GEMM with row selection (score rows only).
+enum Layout { kLayoutFull, kLayoutGemmPass, kLayoutGemmRows };
+
+Layout layout_of(const csa_cache &c, bool gemm) {
+    return !gemm ? kLayoutFull : c.capacity <= kRowSelMaxRows ? kLayoutGemmRows : kLayoutGemmPass;
+}
+
+// Workspace bytes of n queries in a layout (carved at base into w when w is given).
+size_t carve_chunk(void *base, const csa_cache &c, int n, int H_I, Layout lay, IndexWs *w) {
+    const size_t q = lay == kLayoutFull ? 0 : prefill_query_scratch_bytes(c.idx_dtype, c.idx_dim, n, H_I);
+    return lay == kLayoutGemmRows ? carve_rows(base, n, c.capacity, q, w)
+                                  : carve(base, n, c.capacity, w, lay == kLayoutFull, q);
+}
+
+// The most queries whose workspace fits in `bytes`: all Nq, else the largest
+// multiple of kChunkQueries below Nq; 0 when not even that many fit.
+int fit_queries(const csa_cache &c, int Nq, int H_I, Layout lay, size_t bytes) {
+    if (carve_chunk(nullptr, c, Nq, H_I, lay, nullptr) <= bytes) return Nq;
+    int lo = 0, hi = (Nq - 1) / kChunkQueries;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) / 2;
+        if (carve_chunk(nullptr, c, mid * kChunkQueries, H_I, lay, nullptr) <= bytes) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo * kChunkQueries;
+}
+
 }  // namespace
 
-size_t index_topk_workspace_bytes(int Nq, int cap) { return carve(nullptr, Nq, cap, nullptr); }
+// The size query: the layout of all queries if it stays within kIndexWsTarget,
+// else of the most queries that do (at least one chunk; for the GEMM at least
+// kGemmChunkQueries). It does not know the indexer heads: for a GEMM-capable key
+// format it sizes the GEMM layout for the largest head count, and leaves room for
+// one chunk of the full layout, which head counts without a GEMM kernel take.
+size_t index_topk_workspace_bytes(const csa_cache &c, int Nq) {
+    const int first = min(Nq, kChunkQueries);
+    const size_t full_first = carve_chunk(nullptr, c, first, 1, kLayoutFull, nullptr);
+    if (!gemm_call(c, Nq, 1)) {
+        const int n = max(fit_queries(c, Nq, 1, kLayoutFull, kIndexWsTarget), first);
+        return carve_chunk(nullptr, c, n, 1, kLayoutFull, nullptr);
+    }
+    const Layout lay = layout_of(c, true);
+    const int n = max(fit_queries(c, Nq, kMaxIdxHeads, lay, kIndexWsTarget), min(Nq, kGemmChunkQueries));
+    return max(carve_chunk(nullptr, c, n, kMaxIdxHeads, lay, nullptr), full_first);
+}
+
+// The least a call accepts: one chunk in the layout its path uses.
+size_t index_topk_min_workspace_bytes(const csa_cache &c, int Nq, int H_I) {
+    return carve_chunk(nullptr, c, min(Nq, kChunkQueries), H_I, layout_of(c, gemm_call(c, Nq, H_I)), nullptr);
+}
 
 namespace {
 
 // Scores of every key of every query into ws.scores (rows of `rows`), the
 // first-level thresholds, then the selection into sel_idx. n_vis_given and
 // pool describe a Reindex call (keys are pool positions); both null otherwise.
+// gemm_ok: the call may score on the GEMM (gemm_call); q_base: the caller's index of
+// query 0 of this chunk (q_idx, w and sel_idx already point at it).
 cudaError_t index_pipeline(const csa_cache &c, const void *q_idx, const float *w, int Nq, int H_I,
                            const int32_t *q_offsets, const int32_t *q_pos, int topk, int32_t *sel_idx, IndexWs &ws,
                            int rows, const int32_t *n_vis_given, const int32_t *pool, int pool_shift, int pool_p,
-                           int num_sms, cudaStream_t s, int layers = 1) {
+                           int num_sms, cudaStream_t s, int layers, bool gemm_ok, int q_base) {
     // many queries per request (prefill): scores as a tensor-core GEMM, and when the
     // rows fit in shared memory one selection kernel that needs no zeroed state
-    const bool gemm = !pool && !n_vis_given && Nq >= kPrefillQueriesPerRequest * c.batch &&
-                      prefill_scores_supported(c.idx_dtype, c.idx_dim, H_I) &&
+    const bool gemm = gemm_ok && !pool && !n_vis_given &&
                       prefill_query_scratch_bytes(c.idx_dtype, c.idx_dim, Nq, H_I) <= ws.spare_bytes;
     const bool row_sel = gemm && rows <= kRowSelMaxRows;
     cudaError_t err = cudaSuccess;
@@ -1988,7 +2094,7 @@ cudaError_t index_pipeline(const csa_cache &c, const void *q_idx, const float *w
     const bool fused = !gemm && Nq <= kFusedScheduleQueries;
     if (!fused) {
         err = launch_pdl(schedule_kernel, dim3(1), dim3(1024), 0, s, q_offsets, q_pos, c.n_blocks, c.batch, Nq,
-                         c.block, rows, topk, ws.req, ws.n_vis, ws.gprefix, ws.thresh, n_vis_given, layers);
+                         c.block, rows, topk, ws.req, ws.n_vis, ws.gprefix, ws.thresh, n_vis_given, layers, q_base);
         if (err != cudaSuccess) return err;
     }
 
@@ -2023,6 +2129,7 @@ cudaError_t index_pipeline(const csa_cache &c, const void *q_idx, const float *w
     sa.batch = c.batch;
     sa.m = c.block;
     sa.layers = layers;
+    sa.q_base = q_base;
     const int grid = min(num_sms, kMaxScanCtas);
     if (gemm) {
         err = launch_prefill_scores(c, q_idx, w, Nq, H_I, ws.req, ws.n_vis, ws.scores, rows, ws.spare, num_sms, s);
@@ -2089,11 +2196,35 @@ cudaError_t index_pipeline(const csa_cache &c, const void *q_idx, const float *w
 
 cudaError_t launch_index_topk(const csa_cache &c, const void *q_idx, const float *w, int Nq, int H_I,
                               const int32_t *q_offsets, const int32_t *q_pos, int topk, int32_t *sel_idx,
-                              void *workspace, int num_sms, cudaStream_t s) {
-    IndexWs ws;
-    carve(workspace, Nq, c.capacity, &ws);
-    return index_pipeline(c, q_idx, w, Nq, H_I, q_offsets, q_pos, topk, sel_idx, ws, c.capacity, nullptr, nullptr, 0,
-                          0, num_sms, s);
+                              void *workspace, size_t workspace_bytes, int num_sms, cudaStream_t s) {
+    const bool gemm = gemm_call(c, Nq, H_I);
+    const Layout lay = layout_of(c, gemm);
+    int chunk = fit_queries(c, Nq, H_I, lay, workspace_bytes);
+    if (chunk <= 0) return cudaErrorInvalidValue;
+    if (gemm && chunk < Nq) {
+        // whole waves of the GEMM's query tiles where the chunk allows: 128 k queries are
+        // k H_I tiles, a multiple of the SM count when k is one of num_sms / gcd(num_sms, H_I)
+        int g = num_sms, h = H_I;
+        while (h) {
+            const int t = g % h;
+            g = h;
+            h = t;
+        }
+        const int kq = num_sms / g, k = chunk / kChunkQueries;
+        if (k >= kq) chunk = k / kq * kq * kChunkQueries;
+    }
+    const size_t q_bytes = (size_t)H_I * c.idx_dim * sizeof(__nv_bfloat16);  // one query's q_idx
+    for (int q0 = 0; q0 < Nq; q0 += chunk) {
+        const int n = min(chunk, Nq - q0);
+        IndexWs ws;
+        carve_chunk(workspace, c, n, H_I, lay, &ws);
+        const cudaError_t err =
+            index_pipeline(c, static_cast<const char *>(q_idx) + q0 * q_bytes, w + (size_t)q0 * H_I, n, H_I,
+                           q_offsets, q_pos, topk, sel_idx + (size_t)q0 * topk, ws, c.capacity, nullptr, nullptr, 0,
+                           0, num_sms, s, 1, gemm, q0);
+        if (err != cudaSuccess) return err;
+    }
+    return cudaSuccess;
 }
 
 size_t index_pool_workspace_bytes(int Nq, int cap, int G, int P) {
@@ -2113,7 +2244,7 @@ cudaError_t launch_index_topk_pool(const csa_cache &c, const void *q_idx, const 
     carve(static_cast<char *>(workspace) + main_bytes, Nq, cap_b, &wb);
     // this layer's scores and top-k; its score rows stay in ws.scores
     cudaError_t err = index_pipeline(c, q_idx, w, Nq, H_I, q_offsets, q_pos, topk, sel_idx, ws, c.capacity, nullptr,
-                                     nullptr, 0, 0, num_sms, s);
+                                     nullptr, 0, 0, num_sms, s, 1, gemm_call(c, Nq, H_I), 0);
     if (err != cudaSuccess) return err;
     // block maxima and the pool's threshold, then the pool's selection
     if ((err = cudaMemsetAsync(wb.done, 0, wb.zero_bytes, s)) != cudaSuccess) return err;
@@ -2149,7 +2280,7 @@ cudaError_t launch_index_topk_reindex(const csa_cache &c, const void *q_idx, con
                                  n_pos, c.status, layers);
     if (err != cudaSuccess) return err;
     return index_pipeline(c, q_idx, w, NqL, H_I, q_offsets, q_pos, topk, sel_idx, ws, rows, n_pos, pool_blk,
-                          pool_shift, P, num_sms, s, layers);
+                          pool_shift, P, num_sms, s, layers, false, 0);
 }
 
 }  // namespace csa

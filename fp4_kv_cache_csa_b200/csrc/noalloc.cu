@@ -26,6 +26,8 @@ namespace csa {
 csa_status check_index_args(const csa_cache *cache, const void *q_idx, const float *w, int32_t n_queries,
                             int32_t idx_heads, const int32_t *q_offsets, const int32_t *q_pos, int32_t topk,
                             const int32_t *sel_idx);
+// indexer.cu: the least workspace csa_index_topk accepts (one chunk of queries).
+size_t index_topk_min_workspace_bytes(const csa_cache &c, int Nq, int H_I);
 }  // namespace csa
 
 namespace {
@@ -63,8 +65,8 @@ extern "C" csa_status csa_index_topk_noalloc(const csa_cache *cache, const void 
     const csa_status arg = csa::check_index_args(cache, q_idx, w, n_queries, idx_heads, q_offsets, q_pos, topk,
                                                  sel_idx);
     if (arg != CSA_OK) return arg;
-    if (csa_index_topk_workspace(cache, n_queries, topk) > kScratchBytes)
-        return CSA_ERR_WORKSPACE;  // these sizes do not fit the fixed scratch
+    // not even one chunk of queries fits the fixed scratch (larger calls run in chunks)
+    if (csa::index_topk_min_workspace_bytes(*cache, n_queries, idx_heads) > kScratchBytes) return CSA_ERR_WORKSPACE;
     void *scratch = nullptr;
     const csa_status st = scratch_address(&scratch);
     if (st != CSA_OK) return st;

@@ -161,7 +161,15 @@ csa_status csa_compress_quantize(const csa_cache *cache, const void *kv_tok, con
                                  const float *gate_w, const int32_t *tok_offsets, int32_t n_tokens,
                                  csa_stream_t stream);
 
-/* Bytes of workspace csa_index_topk needs for these sizes (0 on bad sizes). */
+/*
+ * Bytes of workspace to give csa_index_topk for these sizes (0 on bad sizes):
+ * the workspace of all n_queries queries when that stays under 768 MiB, else
+ * of the most queries that do, and the call then runs its queries in chunks
+ * of that size. When the key format has a GEMM kernel (bf16 keys of 64, 128
+ * or 256 channels, MXFP4 keys of 128) and the call brings 16 or more queries
+ * per request, a chunk holds at least 4736 queries (one wave of query tiles
+ * on the 148 SMs), above 768 MiB if it must.
+ */
 size_t csa_index_topk_workspace(const csa_cache *cache, int32_t n_queries, int32_t topk);
 
 /*
@@ -179,7 +187,13 @@ size_t csa_index_topk_workspace(const csa_cache *cache, int32_t n_queries, int32
  *   q_offsets int32 [batch+1] device; q_pos int32 [n_queries] device
  *   sel_idx   int32 [n_queries][topk] device, written
  *   idx_heads 1..8; topk 1..4096
- *   workspace >= csa_index_topk_workspace(cache, n_queries, topk) bytes, 256-byte aligned
+ *   workspace 256-byte aligned, workspace_bytes of it usable. Any size from
+ *             what one chunk of min(n_queries, 128) queries needs works
+ *             (smaller: CSA_ERR_WORKSPACE); csa_index_topk_workspace() bytes
+ *             always do. The call runs its queries in consecutive chunks of
+ *             the most queries whose workspace fits (multiples of 128), all
+ *             on the same stream; every query is scored and selected on its
+ *             own, so the results do not depend on the chunks.
  * Calls that bring on average 16 or more queries per request (prefill) with
  * bf16 keys of 64, 128 or 256 channels and 1, 2, 4 or 8 indexer heads compute
  * the scores as one tensor-core GEMM per request (TMA tensor maps over the
@@ -201,10 +215,12 @@ csa_status csa_index_topk(const csa_cache *cache, const void *q_idx, const float
  * passes all inputs and outputs exactly as for csa_index_topk (same meaning,
  * same results); only the scratch space is the library's.
  *   - The scratch is one fixed 32 MiB array in device memory, held on every
- *     GPU that loads the library until the process exits. Sizes whose
- *     csa_index_topk_workspace() exceeds 32 MiB are rejected with
- *     CSA_ERR_WORKSPACE before anything is launched; the argument checks of
- *     csa_index_topk come first (same codes, same order).
+ *     GPU that loads the library until the process exits. A call runs as
+ *     csa_index_topk does with a 32 MiB workspace: in chunks of queries when
+ *     all of them do not fit. Sizes where not even one chunk of 128 queries
+ *     fits are rejected with CSA_ERR_WORKSPACE before anything is launched;
+ *     the argument checks of csa_index_topk come first (same codes, same
+ *     order).
  *   - The first call on each device looks up that array's device address
  *     (once, with the device current). Make that first call before any
  *     stream capture on the device.

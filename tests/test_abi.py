@@ -108,6 +108,29 @@ def test_index_topk_validation(lib):
     assert call(wsp=0x1000010) == ERR_ALIGN
 
 
+def test_index_workspace_is_bounded(lib):
+    # the size query asks for all queries' workspace when it stays under 768 MiB, else for the
+    # most queries that fit (the call runs the rest in further chunks); GEMM calls get at least
+    # one wave of query tiles (4736 queries' score rows)
+    def ws(nq, **kw):
+        return lib.csa_index_topk_workspace(ctypes.byref(fake_cache(**kw)), nq, 512)
+
+    wave = 148 * 32
+    for dt, extra in ((0, {}), (2, {"idx_key_scale": 0x90000})):  # 4 x 8192 prefill tokens over 18432 blocks
+        w = ws(32768, batch=4, capacity=18432, idx_dtype=dt, **extra)
+        assert 4 * 18432 * wave < w <= (768 << 20)
+    w = ws(32, batch=32, capacity=262144, idx_dtype=1)  # decode at 1M: one pass over everything
+    assert w > 32 * 12 * 262144
+    w = ws(8192, batch=1, capacity=262144, idx_dtype=0)  # 8192 prefill tokens over a 1M-token cache
+    assert 4 * 262144 * wave < w < 4 * 262144 * 8192
+    w = ws(8192, batch=1, capacity=262144, idx_dtype=1)  # e4m3 keys: streamed, chunks of 128 queries
+    assert 128 * 12 * 262144 < w < 256 * 12 * 262144
+    # a call accepts less than the size query's answer, down to one chunk of 128 queries
+    c = fake_cache(batch=2, capacity=1024, idx_dtype=0)
+    args = (0x90000, 0xA0000, 1024, 4, 0xB0000, 0xC0000, 256, 0xD0000, 0x1000000)
+    assert lib.csa_index_topk(ctypes.byref(c), *args, 4 * 1024 * 100, None) == ERR_WORKSPACE
+
+
 def test_attend_validation(lib):
     c = fake_cache()
 

@@ -4,7 +4,8 @@ memory budget, or code that cannot afford an allocation's synchronization).
 Its scratch is a fixed 32 MiB array inside the library instead of a caller
 workspace, so its results must equal csa_index_topk's exactly; and since every
 call reuses that array, two calls in a row (with different inputs) must each
-still match. This file is collected last on purpose."""
+still match. A call larger than the scratch runs its queries in chunks
+that fit. This file is collected last on purpose."""
 import ctypes
 
 import numpy as np
@@ -62,8 +63,23 @@ def test_noalloc_matches_the_workspace_call_twice_in_a_row():
         assert csa.csa_read_device_status(cache) == 0
 
 
+@pytest.mark.gpu
+def test_noalloc_runs_a_larger_prefill_in_chunks():
+    # 1400 prefill queries over 8195-block score rows need 46 MB of rows: the fixed scratch
+    # holds 896 queries' rows, so the call runs in two chunks and must still equal one pass
+    cache, q_idx, w, qo, qp, torch = _inputs(75, [8192, 6000], 128, 0, 512, per_req=700)
+    assert q_idx.shape[0] * 4 * 8195 > (32 << 20)
+    want = csa.csa_index_topk(cache, q_idx, w, qo, qp, 512)
+    got = torch.full_like(want, -7)
+    csa.csa_index_topk_noalloc(cache, q_idx, w, qo, qp, 512, got)
+    torch.cuda.synchronize()
+    assert torch.equal(got, want)
+    assert csa.csa_read_device_status(cache) == 0
+
+
 def test_noalloc_rejects_sizes_beyond_its_scratch():
-    # checked on the host before any device work: 32 queries x 262144 blocks needs > 32 MiB
+    # checked on the host before any device work: one chunk of 32 queries x 262144 blocks
+    # (decode: the streamed layout) needs > 32 MiB
     csa_build.build()
     lib = csa.load_library()
     c = csa._CCache(32, 512, 4, 262144, 0x10000, 0x20000, 0x30000, 128, 1, 0x40000, None)
