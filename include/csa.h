@@ -165,7 +165,7 @@ csa_status csa_compress_quantize(const csa_cache *cache, const void *kv_tok, con
  * Bytes of workspace to give csa_index_topk for these sizes (0 on bad sizes):
  * the workspace of all n_queries queries when that stays under 768 MiB, else
  * of the most queries that do, and the call then runs its queries in chunks
- * of that size. When the key format has a GEMM kernel (bf16 keys of 64, 128
+ * that fit. When the key format has a GEMM kernel (bf16 keys of 64, 128
  * or 256 channels, MXFP4 keys of 128) and the call brings 16 or more queries
  * per request, a chunk holds at least 4736 queries (one wave of query tiles
  * on the 148 SMs), above 768 MiB if it must.
