@@ -127,7 +127,7 @@ typedef struct {
 const char *csa_status_string(int32_t status);
 
 /* Library ABI version (major * 100 + minor). 101 added csa_cache.scale_fmt, 102 the pool and
- * Reindex calls. */
+ * Reindex calls, 103 the MXFP4 indexer keys (csa_cache.idx_key_scale). */
 int32_t csa_version(void);
 
 /*
@@ -146,8 +146,9 @@ int32_t csa_version(void);
  *                of e / s saturated to +-6 (zero magnitude when s = 0);
  *                in both the sign is kept (a negative value that rounds to
  *                zero is code 0x8)
- *   indexer key  k[c] = sum_t a_t idx_t[c], stored as bf16 (RNE) or e4m3 (RNE,
- *                saturated to +-448) per cache->idx_dtype
+ *   indexer key  k[c] = sum_t a_t idx_t[c], stored as bf16 (RNE), e4m3 (RNE,
+ *                saturated to +-448) or MXFP4 (the E8M0/32 rule above, codes in
+ *                idx_key, scales in idx_key_scale) per cache->idx_dtype
  * Arguments:
  *   kv_tok      bf16 [n_tokens][dim]
  *   idx_tok     bf16 [n_tokens][idx_dim]; required iff cache->idx_key != NULL
@@ -195,12 +196,17 @@ size_t csa_index_topk_workspace(const csa_cache *cache, int32_t n_queries, int32
  *             on the same stream; every query is scored and selected on its
  *             own, so the results do not depend on the chunks.
  * Calls that bring on average 16 or more queries per request (prefill) with
- * bf16 keys of 64, 128 or 256 channels and 1, 2, 4 or 8 indexer heads compute
- * the scores as one tensor-core GEMM per request (TMA tensor maps over the
- * key plane and q_idx, which must then be 16-byte aligned, as every pointer
- * here); when the cache holds at most 40960 blocks the top-k then runs one
- * thread block per query over its score row in shared memory. The results are
- * the same as on the streaming path: only the speed differs.
+ * bf16 keys of 64, 128 or 256 channels and 1, 2, 4 or 8 indexer heads, or
+ * with MXFP4 keys of 128 channels and 1 to 4 heads, compute the scores as one
+ * tensor-core GEMM per request (TMA tensor maps over the key plane and q_idx,
+ * which must then be 16-byte aligned, as every pointer here; MXFP4 keys on the
+ * block-scaled MXFP4 MMA after the query is quantized); when the cache holds
+ * at most 40960 blocks the top-k then runs one thread block per query over its
+ * score row in shared memory. The results are the same as on the streaming
+ * path; only the speed differs. (With MXFP4 keys this holds while the scale
+ * products of a score's 32-channel blocks -- key scale times query scale --
+ * lie less than 2^38 apart: the block-scaled MMA drops the products of a
+ * block that far below the largest one.)
  */
 csa_status csa_index_topk(const csa_cache *cache, const void *q_idx, const float *w, int32_t n_queries,
                           int32_t idx_heads, const int32_t *q_offsets, const int32_t *q_pos, int32_t topk,
