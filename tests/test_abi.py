@@ -131,6 +131,40 @@ def test_index_workspace_is_bounded(lib):
     assert lib.csa_index_topk(ctypes.byref(c), *args, 4 * 1024 * 100, None) == ERR_WORKSPACE
 
 
+def test_size_query_always_suffices_and_one_chunk_is_the_floor(lib):
+    # Without a GPU a call that passes every host check fails only at its device query
+    # (CSA_ERR_CUDA), so the workspace check's verdict can be read without launching.
+    # On a machine with a GPU it would launch on these fake pointers: skipped there.
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("needs a machine without a GPU (the call would launch)")
+    ERR_CUDA = 6
+
+    def call(c, nq, hi, wsb):
+        return lib.csa_index_topk(ctypes.byref(c), 0x90000, 0xA0000, nq, hi, 0xB0000, 0xC0000, 256, 0xD0000,
+                                  0x1000000, wsb, None)
+
+    # the GEMM + row selection layout of one 128-query chunk: per-query ranges
+    # (4 + 4 + 8 + 12 bytes, each array 256-aligned, gprefix one longer) and score rows
+    def rows_floor(cap):
+        a = lambda x: (x + 255) // 256 * 256
+        return a(4 * 128) + a(4 * 128) + a(8 * 129) + a(12 * 128) + a(4 * cap * 128)
+
+    for cap in (1000, 1024, 18432):
+        c = fake_cache(batch=2, capacity=cap, idx_dtype=0)  # bf16 keys, 2048 queries: prefill-shaped
+        floor = rows_floor(cap)
+        assert call(c, 2048, 4, floor - 1) == ERR_WORKSPACE
+        assert call(c, 2048, 4, floor) == ERR_CUDA
+    for dt, extra in ((0, {}), (1, {}), (2, {"idx_key_scale": 0x90000})):
+        for cap in (64, 3001, 40960, 40961, 262144):
+            for nq in (1, 32, 127, 128, 129, 4000, 40000):
+                c = fake_cache(batch=2, capacity=cap, idx_dtype=dt, **extra)
+                w = lib.csa_index_topk_workspace(ctypes.byref(c), nq, 256)
+                for hi in ((1, 2, 3, 4) if dt == 2 else (1, 2, 3, 4, 5, 8)):
+                    assert call(c, nq, hi, w) == ERR_CUDA, (dt, cap, nq, hi)
+
+
 def test_attend_validation(lib):
     c = fake_cache()
 
